@@ -1,0 +1,259 @@
+"""Seeded synthetic workloads (inputs only).
+
+Both the CUDA path and the CPU oracle are fed from here; the module holds no
+NVFP4 or residual-compensation arithmetic.  Numbers come from the
+counter-based generator in ``synthetic_gen.c`` (definition in its header):
+every value depends only on (seed, stream, index).
+
+Workload recipes follow the shapes and distributions of the five problem
+settings that the QUADS paper's rollout path is exercised on (dense projection,
+MoE prefill expert block, MoE decode step, ratio sweep, trainer fake-quant);
+the pages themselves print no workload, so sizes and distributions are the
+stated benchmark configurations, written out below.
+
+Streams: 1 = activations X, 2 = weights W (gate_up), 3 = calibration batch,
+4 = outlier-channel choice, 5 = per-channel lognormal scales, 6 = router
+logits, 7 = down-projection weights.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+from dataclasses import dataclass, field
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "synthetic_gen.c")
+_LIB = os.path.join(_HERE, "libsynth.so")
+_lib = None
+
+STREAM_X, STREAM_W, STREAM_XCAL, STREAM_OUTLIER, STREAM_CHANSCALE, STREAM_ROUTER, STREAM_WDOWN = 1, 2, 3, 4, 5, 6, 7
+
+
+def build_lib(force: bool = False) -> str:
+    """Compile the generator with gcc (OpenMP) next to its source."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-ffp-contract=off",
+                               _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _get():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build_lib())
+        u64, i64, dbl = ctypes.c_uint64, ctypes.c_int64, ctypes.c_double
+        vp = ctypes.c_void_p
+        lib.synth_uniform_f64.argtypes = [u64, u64, u64, i64, vp]
+        lib.synth_normal_f64.argtypes = [u64, u64, u64, i64, vp]
+        lib.synth_normal_bf16.argtypes = [u64, u64, u64, i64, i64, dbl, vp, vp]
+        lib.synth_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def uniform_f64(seed: int, stream: int, n: int, offset: int = 0) -> np.ndarray:
+    out = np.empty(n, dtype=np.float64)
+    _get().synth_uniform_f64(seed, stream, offset, n, out.ctypes.data)
+    return out
+
+
+def normal_f64(seed: int, stream: int, n: int, offset: int = 0) -> np.ndarray:
+    out = np.empty(n, dtype=np.float64)
+    _get().synth_normal_f64(seed, stream, offset, n, out.ctypes.data)
+    return out
+
+
+def normal_bf16(seed: int, stream: int, rows: int, cols: int, sigma: float = 1.0,
+                colscale: np.ndarray | None = None, offset: int = 0, out: np.ndarray | None = None) -> np.ndarray:
+    """bf16 bit patterns (uint16) of sigma * colscale[c] * N(0,1), shape [rows, cols]."""
+    if out is None:
+        out = np.empty((rows, cols), dtype=np.uint16)
+    assert out.dtype == np.uint16 and out.flags.c_contiguous and out.size == rows * cols
+    cs = None
+    if colscale is not None:
+        colscale = np.ascontiguousarray(colscale, dtype=np.float64)
+        assert colscale.shape == (cols,)
+        cs = colscale.ctypes.data
+    _get().synth_normal_bf16(seed, stream, offset, rows, cols, float(sigma), cs, out.ctypes.data)
+    return out
+
+
+def generator_threads() -> int:
+    return int(_get().synth_num_threads())
+
+
+def bf16_to_f32(a: np.ndarray) -> np.ndarray:
+    """Exact widening of bf16 bit patterns to float32 (storage conversion only)."""
+    return (a.astype(np.uint32) << 16).view(np.float32)
+
+
+# ----------------------------------------------------------------------------------------------
+# structure of the inputs: outlier channels, channel scales, routing
+# ----------------------------------------------------------------------------------------------
+def outlier_channels(seed: int, K: int, count: int = 4) -> np.ndarray:
+    """`count` distinct channels drawn in order from stream 4: k = floor(u*K), repeats skipped."""
+    chosen: list[int] = []
+    i = 0
+    while len(chosen) < count:
+        u = uniform_f64(seed, STREAM_OUTLIER, 64, offset=i)
+        i += 64
+        for v in u:
+            k = int(v * K)
+            if k not in chosen:
+                chosen.append(k)
+                if len(chosen) == count:
+                    break
+    return np.array(chosen, dtype=np.int64)
+
+
+def outlier_colscale(seed: int, K: int, count: int = 4, factor: float = 20.0) -> np.ndarray:
+    cs = np.ones(K, dtype=np.float64)
+    cs[outlier_channels(seed, K, count)] = factor
+    return cs
+
+
+def lognormal_colscale(seed: int, K: int) -> np.ndarray:
+    """c_k = exp(N(0,1)) per channel (stream 5)."""
+    return np.exp(normal_f64(seed, STREAM_CHANSCALE, K))
+
+
+def route_topk(seed: int, T: int, E: int, topk: int) -> np.ndarray:
+    """Top-k experts per token from N(0,1) router logits (stream 6).
+
+    Softmax is monotone, so the top-k of the softmax equals the top-k of the
+    logits; ties go to the lower expert index (stable sort).  Returns [T, topk]
+    int64, best expert first.
+    """
+    logits = normal_f64(seed, STREAM_ROUTER, T * E).reshape(T, E)
+    order = np.argsort(-logits, axis=1, kind="stable")
+    return order[:, :topk].astype(np.int64)
+
+
+def sort_pairs(topk_ids: np.ndarray, E: int):
+    """(token, expert) pairs sorted by (expert, token).
+
+    Returns (pair_token [P], pair_expert [P], counts [E]).
+    """
+    T, k = topk_ids.shape
+    tok = np.repeat(np.arange(T, dtype=np.int64), k)
+    exp = topk_ids.reshape(-1)
+    order = np.lexsort((tok, exp))
+    pair_token = tok[order]
+    pair_expert = exp[order]
+    counts = np.bincount(pair_expert, minlength=E).astype(np.int64)
+    return pair_token, pair_expert, counts
+
+
+def kp_from_ratio(K: int, r: float) -> int:
+    """K' = r*K rounded to the nearest multiple of 64 (ties round up)."""
+    return int(np.floor(r * K / 64.0 + 0.5)) * 64
+
+
+# ----------------------------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------------------------
+@dataclass
+class DenseWorkload:
+    name: str
+    x: np.ndarray          # bf16 bits [M, K]
+    w: np.ndarray          # bf16 bits [N, K]
+    x_cal: np.ndarray      # bf16 bits [T, K]
+    r: float
+    Kp: int
+    out_bf16: bool
+
+    @property
+    def M(self):
+        return self.x.shape[0]
+
+    @property
+    def K(self):
+        return self.x.shape[1]
+
+    @property
+    def N(self):
+        return self.w.shape[0]
+
+
+def dense_tiny(seed: int = 0, r: float = 0.5) -> DenseWorkload:
+    """X 64x256 N(0,1) with 4 channels x20, W 128x256 N(0,0.02), separate 64x256 calibration batch."""
+    M, K, N = 64, 256, 128
+    cs = outlier_colscale(seed, K)
+    x = normal_bf16(seed, STREAM_X, M, K, 1.0, cs)
+    w = normal_bf16(seed, STREAM_W, N, K, 0.02)
+    x_cal = normal_bf16(seed, STREAM_XCAL, M, K, 1.0, cs)
+    return DenseWorkload("dense_tiny_64x128x256", x, w, x_cal, r, kp_from_ratio(K, r), out_bf16=False)
+
+
+def dense_prefill(seed: int = 0, r: float = 0.5, M: int = 8192, K: int = 4096, N: int = 4096,
+                  T_cal: int = 2048) -> DenseWorkload:
+    """X[t,k] = c_k * N(0,1) with c_k = exp(N(0,1)); W N(0,0.02); 2048-token calibration batch."""
+    cs = lognormal_colscale(seed, K)
+    x = normal_bf16(seed, STREAM_X, M, K, 1.0, cs)
+    w = normal_bf16(seed, STREAM_W, N, K, 0.02)
+    x_cal = normal_bf16(seed, STREAM_XCAL, T_cal, K, 1.0, cs)
+    return DenseWorkload(f"dense_prefill_{M}x{N}x{K}", x, w, x_cal, r, kp_from_ratio(K, r), out_bf16=True)
+
+
+@dataclass
+class MoEWorkload:
+    name: str
+    x: np.ndarray            # bf16 bits [T, H]
+    topk_ids: np.ndarray     # [T, topk]
+    pair_token: np.ndarray   # [P] sorted by (expert, token)
+    pair_expert: np.ndarray  # [P]
+    counts: np.ndarray       # [E]
+    E: int
+    H: int                   # hidden size (gate_up K, down N)
+    I: int                   # expert intermediate size (gate_up N = 2I, down K)
+    r: float
+    Kp_gu: int
+    Kp_dn: int
+    seed: int
+    x_cal: np.ndarray | None = None
+    wgu: np.ndarray | None = None   # bf16 bits [E, 2I, H]  (rows [0,I) gate, [I,2I) up)
+    wdn: np.ndarray | None = None   # bf16 bits [E, H, I]
+    extra: dict = field(default_factory=dict)
+
+    def gate_up_expert(self, e: int) -> np.ndarray:
+        """bf16 bits [2I, H] of expert e (generated on demand when not held)."""
+        if self.wgu is not None:
+            return self.wgu[e]
+        return normal_bf16(self.seed, STREAM_W, 2 * self.I, self.H, 0.02, offset=e * 2 * self.I * self.H)
+
+    def down_expert(self, e: int) -> np.ndarray:
+        if self.wdn is not None:
+            return self.wdn[e]
+        return normal_bf16(self.seed, STREAM_WDOWN, self.H, self.I, 0.02, offset=e * self.H * self.I)
+
+
+def moe_block(seed: int = 0, r: float = 0.5, T: int = 4096, H: int = 2048, E: int = 128, topk: int = 8,
+              I: int = 768, T_cal: int = 2048, materialize_weights: bool = True) -> MoEWorkload:
+    """MoE expert block: heavy-tailed X (4 channels x20), softmax top-k routing of N(0,1) logits,
+    gate_up W [E, 2I, H] and down W [E, H, I], all N(0, 0.02)."""
+    cs = outlier_colscale(seed, H)
+    x = normal_bf16(seed, STREAM_X, T, H, 1.0, cs)
+    x_cal = normal_bf16(seed, STREAM_XCAL, T_cal, H, 1.0, cs)
+    topk_ids = route_topk(seed, T, E, topk)
+    pt, pe, counts = sort_pairs(topk_ids, E)
+    wl = MoEWorkload(f"moe_T{T}_H{H}_E{E}_top{topk}_I{I}", x, topk_ids, pt, pe, counts, E, H, I, r,
+                     kp_from_ratio(H, r), kp_from_ratio(I, r), seed, x_cal=x_cal)
+    if materialize_weights:
+        wl.wgu = normal_bf16(seed, STREAM_W, E * 2 * I, H, 0.02).reshape(E, 2 * I, H)
+        wl.wdn = normal_bf16(seed, STREAM_WDOWN, E * H, I, 0.02).reshape(E, H, I)
+    return wl
+
+
+def moe_prefill(seed: int = 0, r: float = 0.5, materialize_weights: bool = True) -> MoEWorkload:
+    """4096 tokens, hidden 2048, 128 experts, top-8, gate_up 128x(1536x2048), down 128x(2048x768)."""
+    return moe_block(seed, r, T=4096, H=2048, E=128, topk=8, I=768, materialize_weights=materialize_weights)
+
+
+def moe_decode(seed: int = 0, r: float = 0.5) -> MoEWorkload:
+    """64 tokens, hidden 7168, 256 experts, top-8, intermediate 2048; weights generated per expert on demand."""
+    return moe_block(seed, r, T=64, H=7168, E=256, topk=8, I=2048, materialize_weights=False)

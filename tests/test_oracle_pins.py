@@ -1,0 +1,422 @@
+"""Pins of the CPU oracle to facts that do not come from the oracle itself.
+
+Each test checks an oracle routine against something independent: the format
+facts stated on the pages (8 E2M1 magnitudes per sign), closed forms of the
+E4M3 / E2M1 encodings, brute-force searches written here in plain Python,
+hand-worked fixtures, exact rational arithmetic, and invariants of the method
+(on-grid round trip, r = 0 reduces to plain W4A4, r = 1 selects every channel,
+compensation lowers the error on the calibration data).
+"""
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+
+from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+E2M1_GRID = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+
+
+# ------------------------------------------------------------------ independent reference encoders
+def brute_e2m1(v: float) -> int:
+    """Nearest grid magnitude by exhaustive exact comparison; ties to even index; saturate."""
+    m = abs(Fraction(v))
+    best = None
+    for i, g in enumerate(E2M1_GRID):
+        d = abs(m - Fraction(g))
+        key = (d, i % 2)  # smaller distance first, then even index
+        if best is None or key < best[0]:
+            best = (key, i)
+    idx = best[1]
+    if m > 6:
+        idx = 7
+    sign = 8 if math.copysign(1.0, v) < 0 else 0
+    return idx | sign
+
+
+def e4m3_value_closed_form(code: int) -> float:
+    e, m = (code >> 3) & 15, code & 7
+    if e == 0:
+        return m * 2.0 ** -9
+    return (1 + m / 8) * 2.0 ** (e - 7)
+
+
+E4M3_POS = [e4m3_value_closed_form(c) for c in range(0x7F)]  # 0x00 .. 0x7E
+
+
+def brute_e4m3(raw: float) -> int:
+    r = Fraction(raw)
+    if r >= 448:
+        return 0x7E
+    best = None
+    for c, val in enumerate(E4M3_POS):
+        d = abs(r - Fraction(val))
+        key = (d, c % 2)
+        if best is None or key < best[0]:
+            best = (key, c)
+    return best[1]
+
+
+def f32(x):
+    return float(np.float32(x))
+
+
+def neighbours(x: float, k: int = 3):
+    """x and its k nearest float32 neighbours on both sides."""
+    out = [np.float32(x)]
+    up = dn = np.float32(x)
+    for _ in range(k):
+        up = np.nextafter(up, np.float32(np.inf), dtype=np.float32)
+        dn = np.nextafter(dn, np.float32(-np.inf), dtype=np.float32)
+        out += [up, dn]
+    return [float(v) for v in out]
+
+
+# ------------------------------------------------------------------ E2M1
+def test_e2m1_has_eight_magnitudes_per_sign(orc):
+    """The failure-mode section: E2M1 gives 8 representable magnitude levels per sign."""
+    pos = [orc.e2m1_decode(c) for c in range(8)]
+    neg = [orc.e2m1_decode(c) for c in range(8, 16)]
+    assert pos == E2M1_GRID
+    assert [-v for v in neg] == E2M1_GRID
+    assert all(math.copysign(1.0, v) < 0 for v in neg)  # -0 included
+    assert len(set(pos)) == 8 and len(set(abs(v) for v in neg)) == 8
+
+
+def test_e2m1_encode_matches_brute_force(orc):
+    pts = []
+    mids = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]
+    for g in E2M1_GRID + mids + [6.5, 7.0, 1e3, 1e30]:
+        for s in (1.0, -1.0):
+            pts += [s * v for v in neighbours(g, 4)]
+    rng = np.random.default_rng(0)
+    pts += list(rng.uniform(-8, 8, 20000).astype(np.float32).astype(float))
+    pts += list((rng.standard_normal(2000) * 1e-30).astype(np.float32).astype(float))
+    pts += [0.0, -0.0, float(np.float32(1.4e-45)), -float(np.float32(1.4e-45))]
+    arr = np.array(pts, dtype=np.float32)
+    got = orc.e2m1_encode_array(arr)
+    exp = np.array([brute_e2m1(float(v)) for v in arr], dtype=np.uint8)
+    bad = np.nonzero(got != exp)[0]
+    assert bad.size == 0, [(float(arr[i]), int(got[i]), int(exp[i])) for i in bad[:10]]
+
+
+def test_e2m1_ties_go_to_even(orc):
+    assert orc.e2m1_encode(0.25) == 0 and orc.e2m1_encode(0.75) == 2
+    assert orc.e2m1_encode(1.25) == 2 and orc.e2m1_encode(1.75) == 4
+    assert orc.e2m1_encode(2.5) == 4 and orc.e2m1_encode(3.5) == 6 and orc.e2m1_encode(5.0) == 6
+    assert orc.e2m1_encode(-0.2) == 8  # sign kept on a zero result
+    assert orc.e2m1_encode(100.0) == 7 and orc.e2m1_encode(-100.0) == 15
+
+
+# ------------------------------------------------------------------ E4M3
+def test_e4m3_decode_closed_form(orc):
+    for c in range(256):
+        v = orc.e4m3_decode(c)
+        if c & 0x7F == 0x7F:
+            assert math.isnan(v)
+            continue
+        ref = e4m3_value_closed_form(c & 0x7F) * (-1 if c & 0x80 else 1)
+        assert v == ref, (c, v, ref)
+    assert orc.e4m3_decode(0x7E) == 448.0
+    assert orc.e4m3_decode(0x01) == 2.0 ** -9
+    assert orc.e4m3_decode(0x08) == 2.0 ** -6
+    assert orc.e4m3_decode(0x38) == 1.0
+    vals = [orc.e4m3_decode(c) for c in range(0x7F)]
+    assert all(a < b for a, b in zip(vals, vals[1:]))
+    # 256 code points: 2 zeros, 2 NaN, 252 finite non-zero values (the 256-level comparison format)
+    assert len({orc.e4m3_decode(c) for c in range(256) if c & 0x7F not in (0, 0x7F)}) == 252
+
+
+def test_e4m3_encode_matches_brute_force(orc):
+    pts = []
+    for a, b in zip(E4M3_POS, E4M3_POS[1:]):
+        pts += neighbours((a + b) / 2, 2) + neighbours(b, 1)
+    pts += neighbours(2.0 ** -10, 3) + neighbours(448.0, 3) + neighbours(464.0, 3) + [1e6, 0.0]
+    rng = np.random.default_rng(1)
+    pts += list(rng.uniform(0, 460, 5000).astype(np.float32).astype(float))
+    pts += list(np.exp(rng.uniform(-12, 6, 5000)).astype(np.float32).astype(float))
+    arr = np.array([p for p in pts if p >= 0], dtype=np.float32)
+    got = orc.e4m3_encode_array(arr)
+    exp = np.array([brute_e4m3(float(v)) for v in arr], dtype=np.uint8)
+    bad = np.nonzero(got != exp)[0]
+    assert bad.size == 0, [(float(arr[i]), int(got[i]), int(exp[i])) for i in bad[:10]]
+
+
+def test_e4m3_saturation_and_underflow(orc):
+    assert orc.e4m3_encode(448.0) == 0x7E and orc.e4m3_encode(1e9) == 0x7E
+    assert orc.e4m3_encode(2.0 ** -10) == 0  # tie between 0 and 2^-9 goes to even code 0
+    assert orc.e4m3_encode(f32(np.nextafter(np.float32(2.0 ** -10), np.float32(1)))) == 1
+
+
+# ------------------------------------------------------------------ bf16 storage
+def test_bf16_rounding_matches_torch(orc):
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(2)
+    v = np.concatenate([rng.standard_normal(3000) * 10.0 ** rng.integers(-30, 30, 3000),
+                        np.array([1.0 + 2 ** -8, 1.0 + 3 * 2 ** -8, -(1.0 + 2 ** -8), 3.3895e38])]).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    got = np.array([orc.f64_to_bf16(float(x)) for x in v], dtype=np.uint16)
+    assert np.array_equal(got, ref)
+
+
+# ------------------------------------------------------------------ scales and blocks
+def test_global_scale_power_of_two(orc):
+    for j in range(-20, 20):
+        assert float(orc.global_scale(2688.0 * 2.0 ** j)) == 2.0 ** j
+    assert float(orc.global_scale(0.0)) == 0.0
+
+
+def test_hand_worked_fixture(orc):
+    g = json.load(open(os.path.join(GOLDEN, "nvfp4_hand_worked_blocks.json")))
+    x = np.array(g["x"], dtype=np.float32)
+    xb = (x.view(np.uint32) >> 16).astype(np.uint16).reshape(1, -1)
+    assert np.array_equal(syn.bf16_to_f32(xb).reshape(-1), x)  # inputs are bf16-exact
+    amax = orc.amax_bf16(xb)
+    s_g = orc.global_scale(amax)
+    assert float(s_g) == g["s_g"]
+    sel = np.array(g["sel"], dtype=np.int32)
+    codes, S, rcodes, rS, resid = orc.act_quant_rac(xb, s_g, sel)
+    assert codes.reshape(-1).tolist() == g["codes"]
+    assert S.reshape(-1).tolist() == g["S"]
+    assert rS.reshape(-1).tolist() == g["rS"]
+    assert rcodes.reshape(-1).tolist() == g["rcodes"]
+    assert resid.reshape(-1).tolist() == g["resid"]
+    _, _, dq = orc.quantize_f32(x.reshape(1, -1), s_g)
+    assert dq.reshape(-1).tolist() == g["dq"]
+
+
+def test_quantize_matches_float32_numpy_steps(orc):
+    """Each block decision re-derived with numpy float32 arithmetic and the brute-force encoders."""
+    rng = np.random.default_rng(3)
+    t = (rng.standard_normal((6, 64)) * np.exp(rng.standard_normal((6, 1)) * 2)).astype(np.float32)
+    t[0, :16] = 0.0
+    amax = np.float32(np.abs(t).max())
+    s_g = np.float32(amax / np.float32(2688.0))
+    codes, S, dq = orc.quantize_f32(t, s_g)
+    t6 = np.float32(np.float32(6.0) * s_g)
+    for r in range(t.shape[0]):
+        for b in range(4):
+            blk = t[r, 16 * b:16 * b + 16]
+            bmax = np.float32(np.abs(blk).max())
+            raw = np.float32(bmax / t6)
+            s_exp = brute_e4m3(float(raw))
+            assert S[r, b] == s_exp
+            if s_exp == 0:
+                assert not codes[r, 16 * b:16 * b + 16].any()
+                continue
+            d = np.float32(np.float32(E4M3_POS[s_exp]) * s_g)
+            inv = np.float32(np.float32(1.0) / d)
+            for i in range(16):
+                v = np.float32(blk[i] * inv)
+                q = brute_e2m1(float(v))
+                assert codes[r, 16 * b + i] == q
+                val = E2M1_GRID[q & 7] * (-1 if q & 8 else 1)
+                assert dq[r, 16 * b + i] == np.float32(np.float32(val) * d)
+
+
+def test_on_grid_values_round_trip_exactly(orc):
+    """Values built from the grid (s_g = 2^j, any E4M3 block scale, a +-6 in every block) are
+    reproduced exactly and leave a zero residual."""
+    rng = np.random.default_rng(4)
+    for j in (-6, 0, 3):
+        rows, K = 8, 128
+        s_g = 2.0 ** j
+        S = rng.integers(1, 0x7F, size=(rows, K // 16))
+        S[0, 0] = 0x7E  # the amax block: 6 * 448 * s_g = 2688 * s_g
+        e_idx = rng.integers(0, 8, size=(rows, K))
+        sign = rng.integers(0, 2, size=(rows, K))
+        e_idx[:, ::16] = 7
+        vals = np.array(E2M1_GRID)[e_idx] * np.where(sign, -1, 1)
+        svals = np.array(E4M3_POS)[S]
+        x = (vals * np.repeat(svals, 16, axis=1) * s_g).astype(np.float32)
+        assert np.array_equal(x.astype(np.float64), vals * np.repeat(svals, 16, axis=1) * s_g)
+        xb = (x.view(np.uint32) >> 16).astype(np.uint16)
+        assert np.array_equal(syn.bf16_to_f32(xb), x)
+        assert float(orc.global_scale(orc.amax_bf16(xb))) == s_g
+        sel = np.arange(0, K, 2, dtype=np.int32)
+        codes, Sq, rcodes, rS, resid = orc.act_quant_rac(xb, s_g, sel)
+        assert np.array_equal(Sq, S)
+        assert np.array_equal(codes & 7, e_idx)
+        _, _, dq = orc.quantize_f32(x, s_g)
+        assert np.array_equal(dq, x)
+        assert not resid.any() and not rS.any()
+
+
+def test_residual_is_input_minus_dequant(orc):
+    wl = syn.dense_tiny()
+    x = wl.x
+    s_g = orc.global_scale(orc.amax_bf16(x))
+    sel = np.arange(0, wl.K, 3, dtype=np.int32)[:64]
+    codes, S, rcodes, rS, resid = orc.act_quant_rac(x, s_g, sel)
+    xf = syn.bf16_to_f32(x)
+    e = np.array(E2M1_GRID, np.float32)[codes & 7] * np.where(codes & 8, np.float32(-1), np.float32(1))
+    d = (np.array(E4M3_POS, np.float32)[S] * np.float32(s_g)).astype(np.float32)
+    dq = (e * np.repeat(d, 16, axis=1)).astype(np.float32)
+    assert np.array_equal(resid, (xf[:, sel] - dq[:, sel]).astype(np.float32))
+    # the residual of a kept channel is what the residual codes approximate
+    rq = orc.dequant(rcodes, rS, s_g)
+    assert np.abs(rq - resid).max() <= np.abs(resid).max() / 6 + 1e-12
+
+
+# ------------------------------------------------------------------ GEMM
+def test_gemm_exact_vs_fraction_brute_force(orc):
+    rng = np.random.default_rng(5)
+    M, N, K, Kp = 3, 4, 32, 16
+    a = rng.integers(0, 16, (M, K), dtype=np.uint8)
+    w = rng.integers(0, 16, (N, K), dtype=np.uint8)
+    r = rng.integers(0, 16, (M, Kp), dtype=np.uint8)
+    ws = rng.integers(0, 16, (N, Kp), dtype=np.uint8)
+    aS = rng.integers(0, 0x7F, (M, K // 16), dtype=np.uint8)
+    wS = rng.integers(0, 0x7F, (N, K // 16), dtype=np.uint8)
+    rS = rng.integers(0, 0x7F, (M, Kp // 16), dtype=np.uint8)
+    wsS = rng.integers(0, 0x7F, (N, Kp // 16), dtype=np.uint8)
+    s_a, s_w = 0.37109375, 1.5 * 2 ** -7
+    y, ad = orc.gemm_rac(a, aS, r, rS, w, wS, ws, wsS, s_a, s_w)
+
+    def val(q, s):
+        e = Fraction(E2M1_GRID[q & 7]) * (-1 if q & 8 else 1)
+        return e * Fraction(E4M3_POS[s])
+
+    for i in range(M):
+        for j in range(N):
+            acc = sum(val(a[i, k], aS[i, k // 16]) * val(w[j, k], wS[j, k // 16]) for k in range(K))
+            acc += sum(val(r[i, k], rS[i, k // 16]) * val(ws[j, k], wsS[j, k // 16]) for k in range(Kp))
+            ref = acc * Fraction(s_a) * Fraction(s_w)
+            assert y[i, j] == float(ref)
+
+
+def test_gemm_matches_dequantized_float_matmul(orc):
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    f = orc.dense_rac_forward(wl.x, wl.w, sel)
+    A = orc.dequant(f["a"], f["aS"], f["s_x"])
+    R = orc.dequant(f["r"], f["rS"], f["s_x"])
+    W = orc.dequant(f["wc"], f["wS"], f["s_w"])
+    WS = orc.dequant(f["wsc"], f["wsS"], f["s_w"])
+    ref = A @ W.T + R @ WS.T
+    assert np.abs(f["y"] - ref).max() <= 1e-12 * f["absdot"].max()
+
+
+def test_r0_reduces_to_plain_w4a4(orc):
+    """The native W4A4 GEMM path stays intact: with no selected channel the result is plain W4A4."""
+    wl = syn.dense_tiny()
+    empty = np.zeros(0, np.int32)
+    f0 = orc.dense_rac_forward(wl.x, wl.w, empty)
+    A = orc.dequant(f0["a"], f0["aS"], f0["s_x"])
+    W = orc.dequant(f0["wc"], f0["wS"], f0["s_w"])
+    assert np.abs(f0["y"] - A @ W.T).max() <= 1e-12 * f0["absdot"].max()
+    # and the main-loop codes do not depend on the selection
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    f1 = orc.dense_rac_forward(wl.x, wl.w, sel)
+    for k in ("a", "aS", "wc", "wS"):
+        assert np.array_equal(f0[k], f1[k])
+
+
+# ------------------------------------------------------------------ calibration / selection
+def test_r1_selects_every_channel(orc):
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.K)
+    assert np.array_equal(sel, np.arange(wl.K))
+
+
+def test_selection_matches_sequential_python(orc):
+    rng = np.random.default_rng(6)
+    T, K, Kp = 12, 64, 32
+    x = syn.normal_bf16(7, 3, T, K, 1.0, np.exp(rng.standard_normal(K)))
+    x[:, 5] = x[:, 6]  # identical channels -> equal errors, tie broken by index
+    sel, err = orc.calibrate(x, Kp)
+    s_g = orc.global_scale(orc.amax_bf16(x))
+    _, _, dq = orc.quantize_f32(syn.bf16_to_f32(x), s_g)
+    r = (syn.bf16_to_f32(x) - dq).astype(np.float32)
+    e = []
+    for k in range(K):
+        acc = 0.0
+        for t in range(T):
+            acc += float(r[t, k]) * float(r[t, k])
+        e.append(acc)
+    assert np.array_equal(np.array(e), err)
+    order = sorted(range(K), key=lambda k: (-e[k], k))
+    assert sel.tolist() == sorted(order[:Kp])
+
+
+def test_outlier_channels_are_selected(orc):
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    for k in syn.outlier_channels(0, wl.K):
+        assert k in sel
+
+
+def test_compensation_never_increases_error_on_calibration_data(orc):
+    """r > 0 lowers mean |Y - Y_bf16| relative to r = 0 on the calibration batch."""
+    wl = syn.dense_tiny()
+    xf = syn.bf16_to_f32(wl.x_cal).astype(np.float64)
+    wf = syn.bf16_to_f32(wl.w).astype(np.float64)
+    y_ref = xf @ wf.T
+    errs = []
+    for r in (0.0, 0.25, 0.5, 1.0):
+        Kp = syn.kp_from_ratio(wl.K, r)
+        sel, _ = orc.calibrate(wl.x_cal, Kp)
+        f = orc.dense_rac_forward(wl.x_cal, wl.w, sel)
+        errs.append(np.abs(f["y"] - y_ref).mean())
+    assert all(e <= errs[0] for e in errs[1:]), errs
+    assert all(b <= a for a, b in zip(errs, errs[1:])), errs  # monotone in r on this batch
+
+
+def test_compensation_shrinks_activation_error(orc):
+    """Against X_bf16 @ DQ(Q(W))^T (weight error removed), the residual pass over all channels
+    removes most of the activation quantisation error."""
+    wl = syn.dense_tiny()
+    xf = syn.bf16_to_f32(wl.x_cal).astype(np.float64)
+    errs = []
+    for r in (0.0, 1.0):
+        Kp = syn.kp_from_ratio(wl.K, r)
+        sel, _ = orc.calibrate(wl.x_cal, Kp)
+        f = orc.dense_rac_forward(wl.x_cal, wl.w, sel)
+        Wq = orc.dequant(f["wc"], f["wS"], f["s_w"])
+        errs.append(np.abs(f["y"] - xf @ Wq.T).mean())
+    assert errs[1] < 0.25 * errs[0], errs
+
+
+# ------------------------------------------------------------------ weights / trainer fake-quant
+def test_shared_weight_path_is_bit_identical(orc):
+    """The packed weights dequantise to exactly the trainer's fake-quantised weights."""
+    w = syn.normal_bf16(0, 2, 64, 256, 0.02)
+    s_w = orc.global_scale(orc.amax_bf16(w))
+    sel = np.arange(64, dtype=np.int32)
+    wc, wS, _, _ = orc.weight_pack(w, s_w, sel)
+    qdq, s2 = orc.weight_qdq(w)
+    assert float(s2) == float(s_w)
+    e = np.array(E2M1_GRID, np.float32)[wc & 7] * np.where(wc & 8, np.float32(-1), np.float32(1))
+    d = (np.array(E4M3_POS, np.float32)[wS] * np.float32(s_w)).astype(np.float32)
+    dq32 = (e * np.repeat(d, 16, axis=1)).astype(np.float32)
+    torch = pytest.importorskip("torch")
+    ref = torch.from_numpy(dq32).to(torch.bfloat16).view(torch.int16).numpy().astype(np.uint16)
+    assert np.array_equal(qdq, ref)
+
+
+def test_weight_sel_is_raw_columns(orc):
+    w = syn.normal_bf16(0, 2, 32, 128, 0.02)
+    s_w = orc.global_scale(orc.amax_bf16(w))
+    sel = np.array(sorted(np.random.default_rng(7).choice(128, 64, replace=False)), np.int32)
+    _, _, sc, sS = orc.weight_pack(w, s_w, sel)
+    c2, S2, _ = orc.quantize_f32(syn.bf16_to_f32(w)[:, sel], s_w)
+    assert np.array_equal(sc, c2) and np.array_equal(sS, S2)
+
+
+# ------------------------------------------------------------------ SwiGLU
+def test_swiglu_closed_form(orc):
+    g = np.array([0.0, 1.0, -1.0, 4.0, -20.0, 0.5], np.float32)
+    u = np.array([3.0, 2.0, 2.0, -0.5, 1.0, 1.0], np.float32)
+    gu = np.concatenate([g, u]).reshape(1, -1)
+    gub = (gu.view(np.uint32) >> 16).astype(np.uint16)
+    h, hx = orc.swiglu(gub)
+    for i in range(6):
+        ref = float(g[i]) / (1 + math.exp(-float(g[i]))) * float(u[i])
+        assert abs(hx[0, i] - ref) <= 1e-15 * max(1.0, abs(ref))
+        assert h[0, i] == orc.f64_to_bf16(ref)
+    assert hx[0, 0] == 0.0
