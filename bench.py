@@ -1,0 +1,414 @@
+"""Benchmark of the NVFP4 W4A4 + RAC MoE prefill expert block on B200.
+
+One step = the rollout hot path over one batch, with weights already packed (packing runs
+once per trainer -> rollout sync, not per step):
+    per-tensor amax of X -> quantise X (+ residual on the calibrated channels) with the
+    gather into expert-sorted, 128-padded rows -> grouped gate_up GEMM (W4A4 + RAC) with the
+    SwiGLU + amax epilogue -> quantise h (+ residual) -> grouped down GEMM (W4A4 + RAC).
+Workload: 4096 tokens, hidden 2048, 128 experts, top-8 of softmax(N(0,1) logits), gate_up
+128 x (1536 x 2048), down 128 x (2048 x 768), r = 0.5; synthetic seeded inputs.
+
+Metric: effective TFLOP/s of the step's GEMMs, 2*rows*N*(K + K') summed over gate_up and down
+(the residual loop counted, as it is part of the method), over the measured step time.
+Also reported: act-quant GB/s and the roofline of the dominant kernel (grouped gate_up).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+Under torchrun every rank runs its own replica (weak scaling, no data-path collective);
+rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP4_OVER_BF16 = 4.0  # nominal dense FP4 / BF16 tensor ratio (9 / 2.25 PFLOP/s)
+METRIC = "W4A4+RAC MoE GEMM effective TFLOPS & % FP4 peak; act-quant GB/s"
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------------------------------ workload
+def build_inputs(seed=0):
+    from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+    wl = syn.moe_prefill(seed=seed)
+    h_cal = syn.moe_down_calibration_batch(wl)
+    return wl, h_cal
+
+
+def flops_of(wl, Kp_gu, Kp_dn):
+    P = int(wl.pair_token.size)
+    gu = 2.0 * P * (2 * wl.I) * (wl.H + Kp_gu)
+    dn = 2.0 * P * wl.H * (wl.I + Kp_dn)
+    return gu, dn
+
+
+def quant_bytes(rows, K, Kp):
+    # bf16 read once + codes and scales of X and R_sel
+    return rows * (2.0 * K + 0.5625 * (K + Kp))
+
+
+class MoEStep:
+    """Device-resident state of one replica and the step itself (C-ABI calls only)."""
+
+    def __init__(self, wl, h_cal, dev):
+        import torch
+
+        from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+
+        self.R, self.torch, self.dev, self.wl = R, torch, dev, wl
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+        self.status = R.new_status(dev)
+        # offline: channel selection on the calibration batches, weight pack
+        self.sel_gu, _ = R.rac_calibrate(to(wl.x_cal), wl.Kp_gu, status=self.status)
+        self.sel_dn, _ = R.rac_calibrate(to(h_cal), wl.Kp_dn, status=self.status)
+        self.pgu, self.pgus = R.pack_weights(to(wl.wgu), self.sel_gu, gate_up_interleave=True, status=self.status)
+        self.pdn, self.pdns = R.pack_weights(to(wl.wdn), self.sel_dn, status=self.status)
+        g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+        self.pair_rows = pair_rows
+        self.rows_padded = int(off[-1])
+        self.gather = torch.from_numpy(g).to(dev)
+        self.offsets = torch.from_numpy(off.astype(np.int32)).to(dev)
+        self.x = to(wl.x)
+        # preallocated outputs (the step allocates nothing)
+        P = R.Packed
+        self.a = P.empty(g.size, wl.H, device=dev)
+        self.ar = P.empty(g.size, wl.Kp_gu, rows_padded=self.a.rows_padded, device=dev)
+        self.h = torch.empty(self.rows_padded, wl.I, dtype=torch.bfloat16, device=dev)
+        self.amax_h = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.hq = P.empty(self.rows_padded, wl.I, device=dev)
+        self.hqr = P.empty(self.rows_padded, wl.Kp_dn, rows_padded=self.hq.rows_padded, device=dev)
+        self.y = torch.empty(self.rows_padded, wl.H, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        R.check_status(self.status)
+
+    def run(self, x=None, events=None):
+        R = self.R
+        x = self.x if x is None else x
+        ev = events or {}
+        if "q0" in ev:
+            ev["q0"].record()
+        R.nvfp4_quantize(x, self.sel_gu, row_gather=self.gather, M_out=self.gather.numel(), out=self.a,
+                         out_res=self.ar, status=self.status)
+        if "g0" in ev:
+            ev["g0"].record()
+        R.grouped_w4a4_rac_moe(self.a, self.ar, self.offsets, self.pgu, self.pgus, swiglu=True, y=self.h,
+                               amax_out=self.amax_h, status=self.status)
+        if "q1" in ev:
+            ev["q1"].record()
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        if "d0" in ev:
+            ev["d0"].record()
+        R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.offsets, self.pdn, self.pdns, y=self.y, status=self.status)
+        if "end" in ev:
+            ev["end"].record()
+        return self.y
+
+    KERNELS_PER_STEP = 5  # amax, quantise X, gate_up GEMM, quantise h, down GEMM
+
+
+# ------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"bench_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------ CPU oracle leg
+def oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=0):
+    """The oracle on a bounded sample of the step: n_pairs (token, expert) rows through quantise,
+    gate_up, SwiGLU, quantise, down.  Returns (seconds, flops of the sample)."""
+    import oracle as orc
+
+    rng = np.random.default_rng(seed)
+    pairs = np.sort(rng.choice(wl.pair_token.size, n_pairs, replace=False))
+    t0 = time.perf_counter()
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    h_rows, exps = [], []
+    for e in np.unique(wl.pair_expert[pairs]):
+        idx = pairs[wl.pair_expert[pairs] == e]
+        xa = wl.x[wl.pair_token[idx]]
+        ac, aS, rc, rS, _ = orc.act_quant_rac(xa, s_x, sel_gu)
+        s_w = orc.global_scale(orc.amax_bf16(wl.wgu[e]))
+        wc, wS, wsc, wsS = orc.weight_pack(wl.wgu[e], s_w, sel_gu)
+        gu, _ = orc.gemm_rac(ac, aS, rc, rS, wc, wS, wsc, wsS, s_x, s_w)
+        gu_b = orc.f64_to_bf16_array(gu)
+        h, _ = orc.swiglu(gu_b)
+        h_rows.append(h)
+        exps.append((e, h.shape[0]))
+    hh = np.concatenate(h_rows)
+    s_h = orc.global_scale(orc.amax_bf16(hh))
+    start = 0
+    for e, n in exps:
+        hc, hS, hrc, hrS, _ = orc.act_quant_rac(hh[start:start + n], s_h, sel_dn)
+        s_w = orc.global_scale(orc.amax_bf16(wl.wdn[e]))
+        dc, dS, dsc, dsS = orc.weight_pack(wl.wdn[e], s_w, sel_dn)
+        orc.gemm_rac(hc, hS, hrc, hrS, dc, dS, dsc, dsS, s_h, s_w)
+        start += n
+    dt = time.perf_counter() - t0
+    gu_f, dn_f = flops_of(wl, len(sel_gu), len(sel_dn))
+    frac = n_pairs / wl.pair_token.size
+    return dt, (gu_f + dn_f) * frac
+
+
+def run_reference(args):
+    """The reference arm: the CPU oracle as it stands, on the same metric and workload."""
+    ws, rank, local = dist_env()
+    if rank != 0:
+        return 0
+    import oracle as orc
+
+    orc.build()
+    wl, h_cal = build_inputs()
+    sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
+    sel_dn, _ = orc.calibrate(h_cal, wl.Kp_dn)
+    n_pairs = args.ref_pairs
+    for _ in range(args.warmup):
+        oracle_sample(wl, sel_gu, sel_dn, max(8, n_pairs // 8))
+    times, flops = [], 0.0
+    for i in range(args.steps):
+        dt, f = oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=i)
+        times.append(dt)
+        flops += f
+    total = sum(times)
+    value = flops / total / 1e12
+    cores = orc.num_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int64-exact GEMM, f32 quant",
+            "data": "synthetic (seeded)",
+            "config": {"workload": wl.name + f"_r{wl.r}", "sample_pairs_per_step": n_pairs},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
+                             "sample": f"{n_pairs} of {wl.pair_token.size} (token, expert) rows per step"},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------ main
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="nvfp4rac", choices=["nvfp4rac", "reference"])
+    ap.add_argument("--ref-pairs", type=int, default=256)
+    ap.add_argument("--cpu-pairs", type=int, default=256)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+
+    ws, rank, local = dist_env()
+    if ws > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+
+    R.load()
+    peaks, peak_kind = load_peaks()
+    wl, h_cal = build_inputs()
+    step = MoEStep(wl, h_cal, dev)
+    gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
+    step_flops = gu_f + dn_f
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+
+    def barrier():
+        if ws > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+
+    # warm-up
+    for _ in range(args.warmup):
+        step.run()
+    torch.cuda.synchronize()
+    R.check_status(step.status)
+
+    # timed region: K steps, L2 flushed between steps (outside the per-step events)
+    names = ["q0", "g0", "q1", "d0", "end"]
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        step.run(events=evs[i])
+    barrier()
+    clk = clocks.stop()
+    R.check_status(step.status)
+    seg = {"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")}
+    per = {k: [] for k in seg}
+    tot = []
+    for e in evs:
+        for k, (a, b) in seg.items():
+            per[k].append(e[a].elapsed_time(e[b]))
+        tot.append(e["q0"].elapsed_time(e["end"]))
+    t_step_ms = float(np.sum(tot)) / args.steps
+    if ws > 1:
+        t = torch.tensor([t_step_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        t_step_ms = float(t.item())
+    value = ws * step_flops / (t_step_ms * 1e-3) / 1e12
+
+    # kernel-level figures (mean over the timed steps)
+    k_ms = {k: float(np.mean(v)) for k, v in per.items()}
+    P = int(wl.pair_token.size)
+    gu_bytes = (wl.E * 2 * wl.I * (wl.H + wl.Kp_gu) * 0.5625 + P * (wl.H + wl.Kp_gu) * 0.5625 + P * wl.I * 2.0)
+    gu_hbm_t = gu_bytes / (peaks["hbm_gbs"] * 1e9)
+    fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
+    gu_tc_t = gu_f / (fp4_peak * 1e12)
+    if gu_hbm_t >= gu_tc_t:
+        achieved = gu_bytes / (k_ms["gate_up"] * 1e-3) / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": achieved / peaks["hbm_gbs"], "traffic": None}
+    else:
+        achieved = gu_f / (k_ms["gate_up"] * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
+                "frac": achieved / fp4_peak, "traffic": None}
+    roof["kernel"] = "grouped gate_up W4A4+RAC GEMM (SwiGLU epilogue)"
+    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
+    qx_bytes = quant_bytes(P, wl.H, wl.Kp_gu)
+    qh_bytes = quant_bytes(P, wl.I, wl.Kp_dn)
+
+    # end-to-end through the public API with host buffers: H2D of X, D2H of Y every step
+    x_host = torch.from_numpy(wl.x.view(np.int16)).pin_memory()
+    y_host = torch.empty(step.y.shape, dtype=torch.bfloat16).pin_memory()
+    x_dev = torch.empty(wl.x.shape, dtype=torch.bfloat16, device=dev)
+    barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e2e_ms = 0.0
+    for i in range(max(3, args.steps // 2)):
+        flush.zero_()
+        e0.record()
+        x_dev.view(torch.int16).copy_(x_host, non_blocking=True)
+        y = step.run(x=x_dev)
+        y_host.copy_(y, non_blocking=True)
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms += e0.elapsed_time(e1)
+    n_e2e = max(3, args.steps // 2)
+    e2e_ms /= n_e2e
+    if ws > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": ws * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(wl.x.nbytes), "d2h_bytes_per_step": int(y_host.numel() * 2)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        import oracle as orc
+
+        orc.build()
+        sel_gu = step.sel_gu.cpu().numpy()
+        sel_dn = step.sel_dn.cpu().numpy()
+        dt, f = oracle_sample(wl, sel_gu, sel_dn, args.cpu_pairs)
+        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+               "sample": f"{args.cpu_pairs} of {P} (token, expert) rows of one step, {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 block scales) -> f32 accumulate",
+            "data": "synthetic (seeded counter-based generator)",
+            "config": {"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P,
+                       "experts": wl.E, "hidden": wl.H, "intermediate": wl.I, "Kp_gate_up": wl.Kp_gu,
+                       "Kp_down": wl.Kp_dn, "rows_padded": step.rows_padded,
+                       "l2": "flushed between timed steps (256 MiB write outside the per-step events)",
+                       "parallelism": f"replicas x{ws}"},
+            "fp4_peak_tflops": fp4_peak,
+            "frac_fp4_peak": value / ws / fp4_peak,
+            "kernel_ms": k_ms,
+            "act_quant_gbs": {"x": qx_bytes / (k_ms["quant_x"] * 1e-3) / 1e9,
+                              "h": qh_bytes / (k_ms["quant_h"] * 1e-3) / 1e9},
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,216 @@
+/*
+ * nvfp4rac.h -- C ABI of the NVFP4 W4A4 + Residual Activation Compensation (RAC) library
+ * (sm_100a, B200).
+ *
+ * The operations follow the rollout-side hot path of QUADS:
+ *   - "QUADS: Stabilizing NVFP4 Reinforcement Learning for MoE via QUantization-error
+ *     Alignment across Dual Sides" (mlsanity.com), Abstract (arXiv): NVFP4 pairs fine-grained
+ *     scaling with native W4A4 FP4 GEMMs; weights are aligned through a shared
+ *     quantization-dequantization path; activations are recomputed (quantised) online.
+ *   - "Why 4-bit RL rollout collapses - and it isn't the weights", section "Two fixes, on two
+ *     different sides": Asymmetric QAT fake-quantizes weights only (trainer side); Residual
+ *     Activation Compensation selects roughly the top 50% of activation channels by
+ *     quantization error and runs a second, residual FP4 pass over just those channels,
+ *     keeping the native W4A4 GEMM intact (rollout side).
+ *   - same post, "The failure mode": E2M1 has 8 magnitude levels per sign.
+ *
+ * NVFP4 storage used by every call (the pages fix no layout; this is the library's):
+ *   element codes  E2M1 (sign bit 3, magnitude index 0..7 = {0,.5,1,1.5,2,3,4,6}); two codes per
+ *                  byte, element 2j in the low nibble, 2j+1 in the high nibble; a matrix of
+ *                  rows x cols is stored row-major as rows_padded x cols/2 bytes.
+ *   block scales   one E4M3 code per 16 consecutive elements of a row, stored in
+ *                  "scale-factor atoms" of 512 bytes, each covering 128 rows x 64 columns:
+ *                  atom(rb, kb) starts at byte (rb * (cols/64) + kb) * 512; inside it the
+ *                  scale of row r (r % 128 = 32*i + j) and 16-column block c (c % 4) is byte
+ *                  j*16 + i*4 + c.  This is the order the tcgen05 block-scaled MMA consumes.
+ *   tensor scale   one FP32 s_g per tensor (per slab for batched weights), s_g = amax / 2688.
+ *   value          x ~= e(code) * S(block) * s_g.
+ * Quantisation (bit-exact contract, binary32 round-to-nearest-even, no FMA contraction):
+ *   b = max|x_i| over the block; S = E4M3_RNE_satfinite(b / (6*s_g)); d = S*s_g;
+ *   S == 0 -> all codes +0; else q_i = E2M1_RNE_satfinite(x_i * (1/d)), sign kept.
+ *   The residual of the selected channels is r_i = x_i - e(q_i)*d, gathered into ascending
+ *   channel order and quantised with the same s_g.  amax == 0 gives s_g = 0 and zero codes.
+ *
+ * Conventions (all calls):
+ *   - Pointers are DEVICE pointers owned by the caller unless stated otherwise.  The library
+ *     never allocates device memory; calls that need scratch take a caller workspace whose
+ *     size the matching *_workspace_size() returns.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t; NULL = legacy default stream).
+ *     Host-detectable errors (null pointers, bad shapes, misalignment) return a status before
+ *     anything is launched.  Errors found on the device (amax out of range, a wait that ran
+ *     out, an invalid channel list) are written, first one wins, to the caller's int32
+ *     *dev_status (device memory, zero on entry); read it after synchronising.
+ *   - No C++ exception crosses this interface.  nvfp4_last_error_string() gives the text of
+ *     the last host-side error of the calling thread.
+ *   - Shapes: K % 64 == 0, 0 <= Kp <= K, Kp % 64 == 0, N % 128 == 0 for GEMM weights.
+ *     16-byte alignment is required for every matrix base pointer and row pitch.
+ *   - bf16 data is passed as uint16_t bit patterns.
+ */
+#ifndef NVFP4RAC_H
+#define NVFP4RAC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,     /* null pointer, bad enum, bad channel list */
+  NVFP4_ERR_UNSUPPORTED_SHAPE = 2,
+  NVFP4_ERR_ALIGNMENT = 3,
+  NVFP4_ERR_RANGE = 4,           /* non-finite input or nonzero amax outside [2^-100, 2^100] */
+  NVFP4_ERR_CUDA = 5,            /* a CUDA runtime/driver call failed */
+  NVFP4_ERR_TIMEOUT = 6          /* a bounded device-side wait ran out */
+} nvfp4_status;
+
+typedef enum { NVFP4_OUT_F32 = 0, NVFP4_OUT_BF16 = 1 } nvfp4_dtype;
+
+typedef enum {
+  NVFP4_EPI_NONE = 0,
+  /* gate_up epilogue of an MoE expert: the packed weight holds gate/up rows interleaved in
+   * 64-row chunks (pack_weights with gate_up_interleave = 1); the output is
+   * h = bf16(silu(bf16(g)) * bf16(u)) with N/2 columns, and max|h| is folded into *amax_out. */
+  NVFP4_EPI_SWIGLU_AMAX = 1
+} nvfp4_epilogue;
+
+/* A packed NVFP4 matrix, or `slabs` equally shaped matrices (MoE experts) back to back.
+ * codes: slabs * rows_padded * cols/2 bytes; sf: slabs * rows_padded * cols/16 bytes (atoms);
+ * s_g: `slabs` floats.  rows_padded % 128 == 0, rows <= rows_padded, cols % 64 == 0. */
+typedef struct {
+  uint8_t* codes;
+  uint8_t* sf;
+  float* s_g;
+  int64_t slabs;
+  int64_t rows;
+  int64_t rows_padded;
+  int64_t cols;
+} nvfp4_tensor;
+
+/* ---------------------------------------------------------------------------------------- */
+/* housekeeping                                                                             */
+/* ---------------------------------------------------------------------------------------- */
+int32_t nvfp4_version(void);
+const char* nvfp4_status_string(nvfp4_status s);
+/* Text of the last host-side error on the calling thread ("" if none). */
+const char* nvfp4_last_error_string(void);
+/* Bytes of codes / scale atoms of one rows_padded x cols NVFP4 matrix. */
+size_t nvfp4_codes_bytes(int64_t rows_padded, int64_t cols);
+size_t nvfp4_sf_bytes(int64_t rows_padded, int64_t cols);
+/* K' = r*K rounded to the nearest multiple of 64 (ties up), clamped to [0, K].
+ * "roughly top-50%" (Two fixes, on two different sides) -> r = 0.5 by default. */
+int32_t nvfp4_kp_from_ratio(int64_t K, double r);
+/* Upper bound of the wait inside every device-side spin loop, in nanoseconds (default 2e9).
+ * A wait that runs out sets NVFP4_ERR_TIMEOUT in *dev_status and the kernel returns. */
+void nvfp4_set_wait_limit_ns(uint64_t ns);
+
+/* ---------------------------------------------------------------------------------------- */
+/* nvfp4_quantize -- online activation quantisation with the RAC residual pass              */
+/* (Abstract: activations are recomputed online; Two fixes: residual FP4 pass over the      */
+/* selected channels).                                                                       */
+/*   x          bf16 [M x K], row pitch ldx elements (ldx >= K, ldx % 8 == 0).               */
+/*   row_gather optional int32 [M_out]: output row o is x row row_gather[o]; -1 (or >= M)   */
+/*              gives a zero row.  NULL: M_out must equal M and row o is x row o.            */
+/*   sel, Kp    ascending channel list [Kp] (Kp % 64 == 0); Kp == 0 disables the residual.   */
+/*   amax_in    optional device float: use it as amax (e.g. from the SwiGLU epilogue); NULL  */
+/*              computes amax over x rows [0, M).                                            */
+/*   q          output: slabs = 1, rows = M_out, rows_padded >= M_out (multiple of 128),     */
+/*              cols = K; rows >= M_out are written as zeros; q->s_g receives s_g.           */
+/*   q_res      output (Kp > 0): cols = Kp, same rows; its s_g receives the same s_g.        */
+/*   workspace  >= nvfp4_quantize_workspace_size() bytes, 16-byte aligned.                   */
+/* ---------------------------------------------------------------------------------------- */
+size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K);
+nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                            const int32_t* row_gather, int64_t M_out, const int32_t* sel, int32_t Kp,
+                            const float* amax_in, const nvfp4_tensor* q, const nvfp4_tensor* q_res,
+                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* rac_calibrate -- pick the Kp channels with the largest quantisation error                */
+/* (Two fixes: "the roughly top-50% of activation channels with the largest quantization    */
+/* error").  The calibration batch is quantised with its own s_g; e_k = sum_t r_{t,k}^2 in   */
+/* binary64 with t ascending; the Kp largest e_k (ties -> lower k) are returned ascending.   */
+/*   x_cal        bf16 [T x K] contiguous.                                                   */
+/*   sel_out      int32 [Kp] (device).  chan_err_out: optional float64 [K] (device).         */
+/* ---------------------------------------------------------------------------------------- */
+size_t rac_calibrate_workspace_size(int64_t T, int64_t K);
+nvfp4_status rac_calibrate(const uint16_t* x_cal, int64_t T, int64_t K, int32_t Kp, int32_t* sel_out,
+                           double* chan_err_out, void* workspace, size_t workspace_bytes,
+                           int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* pack_weights -- rollout side of the shared weight QDQ path (Abstract: weights aligned by  */
+/* a shared quantization-dequantization path), run once per trainer -> rollout sync.         */
+/*   w        bf16 [E x N x K] contiguous (E experts, or E = 1).                             */
+/*   sel, Kp  channel list of the layer input; W_sel = W[:, sel] (raw bf16 columns) is      */
+/*            quantised with the slab's own s_gw.  Kp == 0: w_sel_q may be NULL.             */
+/*   gate_up_interleave  0: packed rows in logical order.  1 (MoE gate_up, N/2 % 64 == 0):   */
+/*            packed row 128q + j holds gate row 64q + j (j < 64) or up row N/2 + 64q + j-64. */
+/*   w_q      output, slabs = E, rows = N, rows_padded = N (N % 128 == 0), cols = K.         */
+/*   w_sel_q  output, slabs = E, rows = N, rows_padded = N, cols = Kp.                       */
+/* ---------------------------------------------------------------------------------------- */
+size_t pack_weights_workspace_size(int64_t E, int64_t N, int64_t K);
+nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel, int32_t Kp,
+                          int32_t gate_up_interleave, const nvfp4_tensor* w_q, const nvfp4_tensor* w_sel_q,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* w4a4_rac_gemm -- Y = s_a*s_w*( Q(X) Q(W)^T + Q(R_sel) Q(W_sel)^T ) in one kernel with     */
+/* one FP32 accumulator (tcgen05 block-scaled FP4 MMA; the residual K' loop follows the main */
+/* K loop into the same tensor-memory accumulator).  "The native W4A4 GEMM path stays        */
+/* intact" (Two fixes): with Kp == 0 this is the plain W4A4 GEMM.                            */
+/*   a, a_res  from nvfp4_quantize (rows >= M, cols K / Kp).                                 */
+/*   w, w_sel  from pack_weights with E = 1 (rows N).                                        */
+/*   y         [M x N] FP32 or bf16, row pitch ldy elements (ldy % 8 == 0).                  */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
+                           const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp,
+                           nvfp4_dtype out, void* y, int64_t ldy, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* grouped_w4a4_rac_moe -- the GEMM above over token-sorted expert segments (MoE rollout).   */
+/*   a, a_res         expert-sorted activations (nvfp4_quantize with row_gather); segment e  */
+/*                    occupies rows [expert_offsets[e], expert_offsets[e+1]).                 */
+/*   expert_offsets   device int32 [E+1], non-decreasing multiples of 128, offsets[0] = 0,   */
+/*                    offsets[E] <= a->rows_padded.  Read on the device only.                */
+/*   w, w_sel         pack_weights output with slabs = E.  alpha_e = a.s_g * w.s_g[e].        */
+/*   ep               NVFP4_EPI_NONE: y [offsets[E] x N]; NVFP4_EPI_SWIGLU_AMAX: y bf16      */
+/*                    [offsets[E] x N/2] and max|y| folded into *amax_out (device float, the  */
+/*                    call zeroes it first).  Rows of padding come out as zeros.             */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
+                                  int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N,
+                                  int64_t K, int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y,
+                                  int64_t ldy, float* amax_out, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* weight_qdq -- trainer-side Asymmetric QAT fake quantisation of weights only (Two fixes):  */
+/* w_out = bf16(DQ(Q(w))) with one s_g per tensor; activations are not touched.  The         */
+/* quantiser is the one pack_weights uses, so DQ(pack_weights(W)) == weight_qdq(W) bitwise.  */
+/*   w, w_out         bf16 [n_tensors x elems_per_tensor] contiguous (elems % 16 == 0).       */
+/*   s_g_out          optional device float [n_tensors].                                     */
+/* ---------------------------------------------------------------------------------------- */
+size_t weight_qdq_workspace_size(int64_t n_tensors, int64_t elems_per_tensor);
+nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_tensor, uint16_t* w_out,
+                        float* s_g_out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                        void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* test helpers (not part of the hot path)                                                   */
+/* ---------------------------------------------------------------------------------------- */
+/* The device E2M1 / E4M3 encoders applied to float32 inputs (v device [n], out device [n],
+ * one code per byte; E4M3 takes non-negative inputs). */
+nvfp4_status nvfp4_encode_e2m1(const float* v, int64_t n, uint8_t* out, void* stream);
+nvfp4_status nvfp4_encode_e4m3(const float* v, int64_t n, uint8_t* out, void* stream);
+/* Runs the bounded mbarrier wait used by every spin loop on a barrier that nothing completes,
+ * with the given limit; expects *dev_status == NVFP4_ERR_TIMEOUT afterwards. */
+nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4RAC_H */

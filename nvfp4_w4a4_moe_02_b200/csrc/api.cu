@@ -1,0 +1,493 @@
+// C-ABI entry points of the NVFP4 W4A4 + RAC library: argument checks, tensor-map encoding
+// and kernel launches.  Nothing here allocates device memory; everything is enqueued on the
+// caller's stream.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "nvfp4rac.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+
+nvfp4_status fail(nvfp4_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+nvfp4_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(NVFP4_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Packed FP4 codes viewed as bytes: [slabs][rows][inner_bytes], 128-byte boxes of box_rows rows,
+// 128-byte swizzle (the layout the tcgen05 descriptors expect).
+nvfp4_status make_code_map(CUtensorMap* m, const void* base, uint64_t inner_bytes, uint64_t rows, uint64_t slabs,
+                           uint32_t box_rows, cuuint32_t rank, const char* what) {
+  auto fn = encode_fn();
+  if (!fn) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  cuuint64_t dims[3] = {inner_bytes, rows, slabs};
+  cuuint64_t strides[2] = {inner_bytes, inner_bytes * rows};
+  cuuint32_t box[3] = {128, box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(NVFP4_ERR_CUDA, "tensor map for %s failed (error %d, inner %llu bytes, rows %llu, slabs %llu)", what,
+                (int)r, (unsigned long long)inner_bytes, (unsigned long long)rows, (unsigned long long)slabs);
+  return NVFP4_OK;
+}
+
+nvfp4_status check_tensor(const nvfp4_tensor* t, const char* name, int64_t cols, int64_t min_rows, int64_t slabs) {
+  if (!t) return fail(NVFP4_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!t->codes || !t->sf || !t->s_g) return fail(NVFP4_ERR_INVALID_ARG, "%s has a NULL buffer", name);
+  if (t->cols != cols) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.cols = %lld, expected %lld", name, (long long)t->cols, (long long)cols);
+  if (t->slabs != slabs) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.slabs = %lld, expected %lld", name, (long long)t->slabs, (long long)slabs);
+  if (t->rows_padded % 128 != 0 || t->rows_padded < min_rows || t->rows < 0 || t->rows > t->rows_padded)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s rows %lld / rows_padded %lld invalid (need >= %lld, multiple of 128)", name,
+                (long long)t->rows, (long long)t->rows_padded, (long long)min_rows);
+  if (!aligned16(t->codes) || !aligned16(t->sf)) return fail(NVFP4_ERR_ALIGNMENT, "%s buffers must be 16-byte aligned", name);
+  return NVFP4_OK;
+}
+
+int act_partials(int64_t M, int64_t K) {
+  int64_t p = (M * K) / 65536;
+  if (p < 1) p = 1;
+  if (p > 256) p = 256;
+  return (int)p;
+}
+int slab_partials(int64_t slabs) {
+  int64_t p = 512 / (slabs > 0 ? slabs : 1);
+  return (int)(p < 1 ? 1 : p);
+}
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+}  // namespace
+
+using namespace nvfp4;
+
+extern "C" {
+
+int32_t nvfp4_version(void) { return 100; }
+
+const char* nvfp4_status_string(nvfp4_status s) {
+  switch (s) {
+    case NVFP4_OK: return "ok";
+    case NVFP4_ERR_INVALID_ARG: return "invalid argument";
+    case NVFP4_ERR_UNSUPPORTED_SHAPE: return "unsupported shape";
+    case NVFP4_ERR_ALIGNMENT: return "misaligned pointer or pitch";
+    case NVFP4_ERR_RANGE: return "value out of range";
+    case NVFP4_ERR_CUDA: return "CUDA error";
+    case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+const char* nvfp4_last_error_string(void) { return g_last_error.c_str(); }
+
+size_t nvfp4_codes_bytes(int64_t rows_padded, int64_t cols) { return (size_t)rows_padded * (size_t)(cols / 2); }
+size_t nvfp4_sf_bytes(int64_t rows_padded, int64_t cols) { return (size_t)rows_padded * (size_t)(cols / 16); }
+
+int32_t nvfp4_kp_from_ratio(int64_t K, double r) {
+  if (!(r > 0.0)) return 0;
+  double q = r * (double)K / 64.0;
+  int64_t kp = (int64_t)(q + 0.5) * 64;
+  if (kp > K) kp = K / 64 * 64;
+  if (kp < 0) kp = 0;
+  return (int32_t)kp;
+}
+
+void nvfp4_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
+
+// ------------------------------------------------------------------------------------------ quantize
+size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K) {
+  (void)M;
+  (void)K;
+  return 256 * sizeof(float);
+}
+
+nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                            int64_t M_out, const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                            const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream) {
+  g_last_error.clear();
+  if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
+  if (M < 0 || M_out < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "negative row count");
+  if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64 <= %lld", (long long)K, (long long)kMaxK);
+  if (ldx < K || ldx % 8 != 0) return fail(NVFP4_ERR_ALIGNMENT, "ldx = %lld must be >= K and a multiple of 8", (long long)ldx);
+  if (x && !aligned16(x)) return fail(NVFP4_ERR_ALIGNMENT, "x must be 16-byte aligned");
+  if (!row_gather && M_out != M) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "without row_gather M_out must equal M");
+  if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp = %d must be a multiple of 64 in [0, K]", Kp);
+  nvfp4_status st = check_tensor(q, "q", K, M_out, 1);
+  if (st != NVFP4_OK) return st;
+  if (Kp > 0) {
+    if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
+    st = check_tensor(q_res, "q_res", Kp, M_out, 1);
+    if (st != NVFP4_OK) return st;
+    if (q_res->rows_padded != q->rows_padded) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res.rows_padded must equal q.rows_padded");
+  }
+  const int P = act_partials(M, K);
+  if (!amax_in) {
+    if (!workspace || workspace_bytes < nvfp4_quantize_workspace_size(M, K))
+      return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* partial = reinterpret_cast<float*>(workspace);
+  if (!amax_in) {
+    cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  }
+  RowArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = kModeAct;
+  a.src = x;
+  a.src_rows = M;
+  a.ld = ldx;
+  a.K = K;
+  a.row_gather = row_gather;
+  a.rows_out = q->rows_padded;
+  a.rows_per_slab = M_out;
+  a.src_slab_stride = 0;
+  a.sel = sel;
+  a.Kp = Kp;
+  a.partial = partial;
+  a.P = P;
+  a.amax_in = amax_in;
+  a.s_g_out = q->s_g;
+  a.s_g_out2 = Kp > 0 ? q_res->s_g : nullptr;
+  a.codes = q->codes;
+  a.sf = q->sf;
+  a.rcodes = Kp > 0 ? q_res->codes : nullptr;
+  a.rsf = Kp > 0 ? q_res->sf : nullptr;
+  a.status = dev_status;
+  if (a.rows_out == 0) return NVFP4_OK;
+  cudaError_t e = launch_rows(a, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return NVFP4_OK;
+}
+
+// ------------------------------------------------------------------------------------------ calibrate
+size_t rac_calibrate_workspace_size(int64_t T, int64_t K) {
+  return round_up(256 * sizeof(float), 256) + round_up((size_t)T * (size_t)K * sizeof(float), 256) +
+         round_up((size_t)K * sizeof(double), 256);
+}
+
+nvfp4_status rac_calibrate(const uint16_t* x_cal, int64_t T, int64_t K, int32_t Kp, int32_t* sel_out,
+                           double* chan_err_out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                           void* stream) {
+  g_last_error.clear();
+  if (!x_cal || (!sel_out && Kp > 0)) return fail(NVFP4_ERR_INVALID_ARG, "x_cal / sel_out is NULL");
+  if (T <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T must be positive");
+  if (K <= 0 || K % 64 != 0 || K > kMaxCalK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64 <= %lld", (long long)K, (long long)kMaxCalK);
+  if (Kp < 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp out of range");
+  if (!aligned16(x_cal)) return fail(NVFP4_ERR_ALIGNMENT, "x_cal must be 16-byte aligned");
+  if (!workspace || workspace_bytes < rac_calibrate_workspace_size(T, K)) return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+  if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  char* ws = reinterpret_cast<char*>(workspace);
+  float* partial = reinterpret_cast<float*>(ws);
+  float* resid = reinterpret_cast<float*>(ws + round_up(256 * sizeof(float), 256));
+  double* err = reinterpret_cast<double*>(ws + round_up(256 * sizeof(float), 256) +
+                                          round_up((size_t)T * (size_t)K * sizeof(float), 256));
+  const int P = act_partials(T, K);
+  cudaError_t e = launch_amax(x_cal, 1, T, K, K, partial, P, dev_status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  RowArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = kModeCal;
+  a.src = x_cal;
+  a.src_rows = T;
+  a.ld = K;
+  a.K = K;
+  a.rows_out = T;
+  a.rows_per_slab = T;
+  a.Kp = 0;
+  a.partial = partial;
+  a.P = P;
+  a.resid_all = resid;
+  a.status = dev_status;
+  e = launch_rows(a, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "calibration residual launch");
+  e = launch_chan_err(resid, T, K, err, s);
+  if (e != cudaSuccess) return cuda_fail(e, "channel error launch");
+  if (Kp > 0 || chan_err_out) {
+    e = launch_select(err, (int32_t)K, Kp, sel_out, chan_err_out, s);
+    if (e != cudaSuccess) return cuda_fail(e, "selection launch");
+  }
+  return NVFP4_OK;
+}
+
+// ------------------------------------------------------------------------------------------ pack
+size_t pack_weights_workspace_size(int64_t E, int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return round_up((size_t)(E > 0 ? E : 1) * (size_t)slab_partials(E) * sizeof(float), 256);
+}
+
+nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel, int32_t Kp,
+                          int32_t gate_up_interleave, const nvfp4_tensor* w_q, const nvfp4_tensor* w_sel_q,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!w) return fail(NVFP4_ERR_INVALID_ARG, "w is NULL");
+  if (E <= 0 || N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E > 0 and N %% 128 == 0 required");
+  if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
+  if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp must be a multiple of 64 in [0, K]");
+  if (gate_up_interleave != 0 && gate_up_interleave != 1) return fail(NVFP4_ERR_INVALID_ARG, "gate_up_interleave must be 0 or 1");
+  if (!aligned16(w)) return fail(NVFP4_ERR_ALIGNMENT, "w must be 16-byte aligned");
+  nvfp4_status st = check_tensor(w_q, "w_q", K, N, E);
+  if (st != NVFP4_OK) return st;
+  if (w_q->rows_padded != N || w_q->rows != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_q rows / rows_padded must equal N");
+  if (Kp > 0) {
+    if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
+    st = check_tensor(w_sel_q, "w_sel_q", Kp, N, E);
+    if (st != NVFP4_OK) return st;
+    if (w_sel_q->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_sel_q rows_padded must equal N");
+  }
+  if (!workspace || workspace_bytes < pack_weights_workspace_size(E, N, K)) return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* partial = reinterpret_cast<float*>(workspace);
+  const int P = slab_partials(E);
+  cudaError_t e = launch_amax(w, E, N, K, K, partial, P, dev_status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  RowArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = kModePack;
+  a.src = w;
+  a.src_rows = N;
+  a.ld = K;
+  a.K = K;
+  a.rows_out = E * N;
+  a.rows_per_slab = N;
+  a.src_slab_stride = N * K;
+  a.interleave = gate_up_interleave;
+  a.N_half = N / 2;
+  a.sel = sel;
+  a.Kp = Kp;
+  a.partial = partial;
+  a.P = P;
+  a.s_g_out = w_q->s_g;
+  a.s_g_out2 = (Kp > 0 && w_sel_q->s_g != w_q->s_g) ? w_sel_q->s_g : nullptr;
+  a.codes = w_q->codes;
+  a.sf = w_q->sf;
+  a.rcodes = Kp > 0 ? w_sel_q->codes : nullptr;
+  a.rsf = Kp > 0 ? w_sel_q->sf : nullptr;
+  a.status = dev_status;
+  e = launch_rows(a, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "pack launch");
+  return NVFP4_OK;
+}
+
+// ------------------------------------------------------------------------------------------ GEMMs
+static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
+                                const nvfp4_tensor* w_sel, int64_t rows_needed, int64_t N, int64_t K, int32_t Kp,
+                                int64_t E, nvfp4_dtype out, void* y, int64_t ldy, int64_t y_cols, int bn,
+                                CUtensorMap* maps, GemmArgs* g) {
+  if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
+  if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp must be a multiple of 64 in [0, K]");
+  if (N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "N must be a positive multiple of 128");
+  if (out != NVFP4_OUT_F32 && out != NVFP4_OUT_BF16) return fail(NVFP4_ERR_INVALID_ARG, "bad output dtype");
+  if (!y) return fail(NVFP4_ERR_INVALID_ARG, "y is NULL");
+  if (!aligned16(y)) return fail(NVFP4_ERR_ALIGNMENT, "y must be 16-byte aligned");
+  if (ldy < y_cols || (out == NVFP4_OUT_BF16 ? ldy % 8 : ldy % 4) != 0)
+    return fail(NVFP4_ERR_ALIGNMENT, "ldy = %lld must be >= %lld and keep rows 16-byte aligned", (long long)ldy, (long long)y_cols);
+  nvfp4_status st = check_tensor(a, "a", K, rows_needed, 1);
+  if (st != NVFP4_OK) return st;
+  st = check_tensor(w, "w", K, N, E);
+  if (st != NVFP4_OK) return st;
+  if (w->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w.rows_padded must equal N");
+  if (Kp > 0) {
+    st = check_tensor(a_res, "a_res", Kp, rows_needed, 1);
+    if (st != NVFP4_OK) return st;
+    if (a_res->rows_padded != a->rows_padded) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "a_res.rows_padded must equal a.rows_padded");
+    st = check_tensor(w_sel, "w_sel", Kp, N, E);
+    if (st != NVFP4_OK) return st;
+    if (w_sel->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_sel.rows_padded must equal N");
+  }
+  memset(maps, 0, 4 * sizeof(CUtensorMap));
+  st = make_code_map(&maps[0], a->codes, (uint64_t)K / 2, (uint64_t)a->rows_padded, 1, 128, 2, "A");
+  if (st != NVFP4_OK) return st;
+  st = make_code_map(&maps[2], w->codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, (uint32_t)bn, 3, "W");
+  if (st != NVFP4_OK) return st;
+  if (Kp > 0) {
+    st = make_code_map(&maps[1], a_res->codes, (uint64_t)Kp / 2, (uint64_t)a_res->rows_padded, 1, 128, 2, "A_res");
+    if (st != NVFP4_OK) return st;
+    st = make_code_map(&maps[3], w_sel->codes, (uint64_t)Kp / 2, (uint64_t)N, (uint64_t)E, (uint32_t)bn, 3, "W_sel");
+    if (st != NVFP4_OK) return st;
+  } else {
+    maps[1] = maps[0];
+    maps[3] = maps[2];
+  }
+  memset(g, 0, sizeof(*g));
+  g->sfa = a->sf;
+  g->sfa_res = Kp > 0 ? a_res->sf : a->sf;
+  g->sfw = w->sf;
+  g->sfw_sel = Kp > 0 ? w_sel->sf : w->sf;
+  g->sfw_slab_bytes = (int64_t)nvfp4_sf_bytes(N, K);
+  g->sfw_sel_slab_bytes = Kp > 0 ? (int64_t)nvfp4_sf_bytes(N, Kp) : 0;
+  g->k64_main = (int32_t)(K / 64);
+  g->k64_res = Kp / 64;
+  g->kt_main = (int32_t)((K + 255) / 256);
+  g->kt_res = (Kp + 255) / 256;
+  g->N = (int32_t)N;
+  g->n_blocks = (int32_t)(N / bn);
+  g->rows_capacity = a->rows_padded;
+  g->s_a = a->s_g;
+  g->s_w = w->s_g;
+  g->y = y;
+  g->ldy = ldy;
+  g->out_bf16 = out == NVFP4_OUT_BF16;
+  g->wait_limit_ns = g_wait_limit_ns.load();
+  return NVFP4_OK;
+}
+
+nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
+                           const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp, nvfp4_dtype out,
+                           void* y, int64_t ldy, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (M < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M must be >= 0");
+  const int bn = (N % 256 == 0) ? 256 : 128;
+  CUtensorMap maps[4];
+  GemmArgs g;
+  nvfp4_status st = gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, bn, maps, &g);
+  if (st != NVFP4_OK) return st;
+  if (M == 0) return NVFP4_OK;
+  g.offsets = nullptr;
+  g.E = 1;
+  g.M = M;
+  g.m_blocks_dense = (int32_t)((M + 127) / 128);
+  g.epi = 0;
+  g.status = dev_status;
+  int64_t tiles = (int64_t)g.m_blocks_dense * g.n_blocks;
+  int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], g, grid, reinterpret_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
+  return NVFP4_OK;
+}
+
+nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
+                                  int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N, int64_t K,
+                                  int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y, int64_t ldy,
+                                  float* amax_out, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!expert_offsets) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets is NULL");
+  if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
+  if (ep != NVFP4_EPI_NONE && ep != NVFP4_EPI_SWIGLU_AMAX) return fail(NVFP4_ERR_INVALID_ARG, "bad epilogue");
+  if (ep == NVFP4_EPI_SWIGLU_AMAX) {
+    if (out != NVFP4_OUT_BF16) return fail(NVFP4_ERR_INVALID_ARG, "the SwiGLU epilogue writes bf16");
+    if (!amax_out) return fail(NVFP4_ERR_INVALID_ARG, "amax_out is NULL with the SwiGLU epilogue");
+  }
+  const int bn = (N % 256 == 0) ? 256 : 128;
+  CUtensorMap maps[4];
+  GemmArgs g;
+  const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
+  nvfp4_status st = gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, bn, maps, &g);
+  if (st != NVFP4_OK) return st;
+  g.offsets = expert_offsets;
+  g.E = E;
+  g.M = a->rows_padded;
+  g.m_blocks_dense = 0;
+  g.epi = ep == NVFP4_EPI_SWIGLU_AMAX ? 1 : 0;
+  g.amax_out = amax_out;
+  g.status = dev_status;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (ep == NVFP4_EPI_SWIGLU_AMAX) {
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax reset");
+  }
+  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], g, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "grouped gemm launch");
+  return NVFP4_OK;
+}
+
+// ------------------------------------------------------------------------------------------ qdq
+size_t weight_qdq_workspace_size(int64_t n_tensors, int64_t elems_per_tensor) {
+  (void)elems_per_tensor;
+  return round_up((size_t)(n_tensors > 0 ? n_tensors : 1) * (size_t)slab_partials(n_tensors) * sizeof(float), 256);
+}
+
+nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_tensor, uint16_t* w_out,
+                        float* s_g_out, void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!w || !w_out) return fail(NVFP4_ERR_INVALID_ARG, "w / w_out is NULL");
+  if (n_tensors <= 0 || elems_per_tensor <= 0 || elems_per_tensor % 16 != 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "n_tensors > 0 and elems_per_tensor %% 16 == 0 required");
+  if (!aligned16(w) || !aligned16(w_out)) return fail(NVFP4_ERR_ALIGNMENT, "w / w_out must be 16-byte aligned");
+  if (!workspace || workspace_bytes < weight_qdq_workspace_size(n_tensors, elems_per_tensor))
+    return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* partial = reinterpret_cast<float*>(workspace);
+  const int P = slab_partials(n_tensors);
+  cudaError_t e = launch_amax(w, n_tensors, 1, elems_per_tensor, elems_per_tensor, partial, P, dev_status, s);
+  if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  e = launch_qdq(w, n_tensors, elems_per_tensor, w_out, partial, P, s_g_out, dev_status, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
+  return NVFP4_OK;
+}
+
+// ------------------------------------------------------------------------------------------ helpers
+nvfp4_status nvfp4_encode_e2m1(const float* v, int64_t n, uint8_t* out, void* stream) {
+  g_last_error.clear();
+  if (n < 0 || (n > 0 && (!v || !out))) return fail(NVFP4_ERR_INVALID_ARG, "bad arguments");
+  if (n == 0) return NVFP4_OK;
+  cudaError_t e = launch_encode_e2m1(v, n, out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "encode launch");
+}
+
+nvfp4_status nvfp4_encode_e4m3(const float* v, int64_t n, uint8_t* out, void* stream) {
+  g_last_error.clear();
+  if (n < 0 || (n > 0 && (!v || !out))) return fail(NVFP4_ERR_INVALID_ARG, "bad arguments");
+  if (n == 0) return NVFP4_OK;
+  cudaError_t e = launch_encode_e4m3(v, n, out, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "encode launch");
+}
+
+nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!dev_status) return fail(NVFP4_ERR_INVALID_ARG, "dev_status is NULL");
+  cudaError_t e = launch_wait_selftest(limit_ns, dev_status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "self-test launch");
+}
+
+}  // extern "C"

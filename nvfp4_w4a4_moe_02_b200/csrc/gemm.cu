@@ -1,0 +1,530 @@
+// W4A4 + RAC GEMM on the 5th-generation tensor cores (sm_100a).
+//
+//   Y = s_a * s_w * ( Q(X) Q(W)^T + Q(R_sel) Q(W_sel)^T )
+//
+// "The native W4A4 GEMM path stays intact; only the highest-error channels get a correction
+// pass layered on top" ("Why 4-bit RL rollout collapses - and it isn't the weights", Two
+// fixes, on two different sides).  Here the correction pass is a second K loop (K' = Kp
+// columns of the residual and of the gathered weight columns) that accumulates into the
+// same tensor-memory accumulator as the main loop, so one epilogue applies the scale.
+//
+// Structure (one CTA per SM, persistent over output tiles of 128 x BN):
+//   warp 0      TMA producer: A/B code tiles (128-byte swizzle) by tensor-map copies, the
+//               scale atoms (512 B each) by bulk copies, into a STAGES-deep shared ring.
+//   warp 1      tensor-memory allocation and the single MMA-issuing thread: scale atoms
+//               shared -> tensor memory (tcgen05.cp 32x128b.warpx4), then
+//               tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 per instruction); commits
+//               free the shared stage and, at the end of a tile, publish the accumulator.
+//   warps 2..5  epilogue: tcgen05.ld of the FP32 accumulator (each warp owns its lane
+//               quadrant), scale by alpha, store bf16/FP32 rows (or SwiGLU + amax).
+// Every mbarrier wait is bounded by a wall-clock limit; on expiry the kernel records
+// NVFP4_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and returns.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+namespace tc {
+
+constexpr int BM = 128;
+constexpr int KT_BYTES = 128;  // bytes of one row per k-tile: 256 FP4 elements
+constexpr int NUM_THREADS = 192;
+
+template <int BN>
+struct Cfg {
+  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int A_BYTES = BM * KT_BYTES;
+  static constexpr int B_BYTES = BN * KT_BYTES;
+  static constexpr int SFA_BYTES = 4 * 512;
+  static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
+  static constexpr int ACC_STAGES = (BN == 256) ? 1 : 2;
+  static constexpr int SF_COLS_A = 16;
+  static constexpr int SF_COLS_B = 16 * (BN / 128);
+  static constexpr int SF_COLS = SF_COLS_A + SF_COLS_B;
+  static constexpr int ACC_COLS = ACC_STAGES * BN;
+  static constexpr int TMEM_COLS = 512;
+  static_assert(ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
+  static constexpr int OFF_A = 0;
+  static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
+  static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_STAGES + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int SMEM = OFF_MISC + 32 + 1024;
+  static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+// ---------------------------------------------------------------------------------------- PTX
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait: false when the limit ran out or another role already aborted.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (abort_flag != nullptr && *abort_flag) return false;
+    if (globaltimer_ns() - t0 > limit_ns) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* map, int32_t x, int32_t y, int32_t z,
+                                            uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+      "[%5];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(bar)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_copy_sf(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+__device__ __forceinline__ void tc_mma_fp4(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                           uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.scale_vec::4X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// 32 lanes x 32 columns of 32-bit accumulator -> 32 registers per thread
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+        "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]),
+        "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// Shared-memory matrix descriptor: K-major operand tile written by a 128-byte-swizzled tensor
+// copy (rows of 128 bytes, 8-row groups 1024 bytes apart).
+__device__ __forceinline__ uint64_t desc_sw128(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)1 << 16;                 // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;       // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;                 // descriptor version
+  d |= (uint64_t)2 << 61;                 // 128-byte swizzle
+  return d;
+}
+// Descriptor of one 512-byte scale atom (32 rows of 16 bytes, no swizzle) for tcgen05.cp.
+__device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
+  uint64_t d = (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)(128 >> 4) << 16;
+  d |= (uint64_t)(128 >> 4) << 32;
+  d |= (uint64_t)1 << 46;
+  return d;
+}
+// Instruction descriptor of kind::mxf4nvf4: E2M1 A and B, UE4M3 scales, K-major, M x N.
+__host__ __device__ constexpr uint32_t idesc_fp4(int M, int N) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ int find_expert(const int32_t* off, int E, int64_t row) {
+  int lo = 0, hi = E - 1;
+  while (lo < hi) {
+    int mid = (lo + hi + 1) >> 1;
+    if ((int64_t)__ldg(off + mid) <= row) lo = mid;
+    else hi = mid - 1;
+  }
+  return lo;
+}
+
+__device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&p);
+}
+
+// ---------------------------------------------------------------------------------------- kernel
+template <int BN>
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_ar,
+                         const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_ws,
+                         const GemmArgs args) {
+  using C = Cfg<BN>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t raw_addr = smem_u32(smem_raw);
+  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
+  unsigned char* smem = smem_raw + (sbase - raw_addr);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  auto bar_full = [&](int s) { return sbase + C::OFF_BAR + 8u * s; };
+  auto bar_empty = [&](int s) { return sbase + C::OFF_BAR + 8u * (C::STAGES + s); };
+  auto bar_accf = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + a); };
+  auto bar_acce = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + C::ACC_STAGES + a); };
+  const uint32_t bar_drain = sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 2 * C::ACC_STAGES);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  volatile int* prod_issued = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
+  volatile int* mma_taken = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 12);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar_full(s), 1);
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int a = 0; a < C::ACC_STAGES; ++a) {
+      mbar_init(bar_accf(a), 1);
+      mbar_init(bar_acce(a), 4);
+    }
+    mbar_init(bar_drain, 1);
+    *abort_flag = 0;
+    *prod_issued = 0;
+    *mma_taken = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  // ---- tile space
+  const bool grouped = args.offsets != nullptr;
+  int64_t m_blocks;
+  int64_t row_limit;
+  if (grouped) {
+    const int64_t rows = __ldg(args.offsets + args.E);
+    m_blocks = rows / BM;
+    row_limit = rows;
+    if (rows % BM != 0 || rows > args.rows_capacity || rows < 0) {
+      if (threadIdx.x == 0) report_status(args.status, kErrInvalid);
+      m_blocks = 0;
+    }
+  } else {
+    m_blocks = args.m_blocks_dense;
+    row_limit = args.M;
+  }
+  const int64_t total_tiles = m_blocks * args.n_blocks;
+  const int kt_total = args.kt_main + args.kt_res;
+  const uint64_t limit = args.wait_limit_ns;
+
+  if (warp == 0) {
+    // ===================================================================== TMA producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int64_t t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+        const int64_t mb = t / args.n_blocks;
+        const int nb = (int)(t - mb * args.n_blocks);
+        const int e = grouped ? find_expert(args.offsets, args.E, mb * BM) : 0;
+        for (int kt = 0; kt < kt_total; ++kt) {
+          if (!mbar_wait(bar_empty(stage), phase ^ 1u, limit, abort_flag)) {
+            report_status(args.status, kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          const bool res = kt >= args.kt_main;
+          const int kk = res ? kt - args.kt_main : kt;
+          const int k64 = res ? args.k64_res : args.k64_main;
+          const int nk64 = min(4, k64 - kk * 4);
+          const uint32_t sf_bytes = (uint32_t)nk64 * 512u;
+          mbar_expect_tx(bar_full(stage), (uint32_t)(C::A_BYTES + C::B_BYTES) + sf_bytes * (1u + BN / 128));
+          tma_load_2d(sbase + C::OFF_A + stage * C::A_BYTES, res ? &tm_ar : &tm_a, kk * KT_BYTES, (int32_t)(mb * BM),
+                      bar_full(stage));
+          tma_load_3d(sbase + C::OFF_B + stage * C::B_BYTES, res ? &tm_ws : &tm_w, kk * KT_BYTES, nb * BN, e,
+                      bar_full(stage));
+          const uint8_t* sfa = (res ? args.sfa_res : args.sfa) + (mb * k64 + kk * 4) * 512;
+          bulk_load(sbase + C::OFF_SFA + stage * C::SFA_BYTES, sfa, sf_bytes, bar_full(stage));
+          const uint8_t* sfw = res ? args.sfw_sel + (int64_t)e * args.sfw_sel_slab_bytes
+                                   : args.sfw + (int64_t)e * args.sfw_slab_bytes;
+#pragma unroll
+          for (int rb = 0; rb < BN / 128; ++rb) {
+            const uint8_t* src = sfw + ((int64_t)(nb * (BN / 128) + rb) * k64 + kk * 4) * 512;
+            bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES + rb * 2048, src, sf_bytes, bar_full(stage));
+          }
+          ++issued;
+          *prod_issued = issued;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ===================================================================== MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_fp4(BM, BN);
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t acc_phase = 0;
+      int taken = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total_tiles && ok && !*abort_flag; t += gridDim.x) {
+        if (!mbar_wait(bar_acce(acc), acc_phase ^ 1u, limit, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        for (int kt = 0; kt < kt_total; ++kt) {
+          if (!mbar_wait(bar_full(stage), phase, limit, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++taken;
+          *mma_taken = taken;
+          tc_fence_after();
+          const bool res = kt >= args.kt_main;
+          const int kk = res ? kt - args.kt_main : kt;
+          const int k64 = res ? args.k64_res : args.k64_main;
+          const int nk64 = min(4, k64 - kk * 4);
+          const uint32_t sfa_t = tmem_base + (uint32_t)(C::ACC_COLS + stage * C::SF_COLS);
+          const uint32_t sfb_t = sfa_t + C::SF_COLS_A;
+          const uint32_t a_s = sbase + C::OFF_A + stage * C::A_BYTES;
+          const uint32_t b_s = sbase + C::OFF_B + stage * C::B_BYTES;
+          const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_BYTES;
+          const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_BYTES;
+          for (int j = 0; j < nk64; ++j) {
+            tc_copy_sf(sfa_t + 4 * j, desc_sf(sfa_s + j * 512));
+#pragma unroll
+            for (int rb = 0; rb < BN / 128; ++rb)
+              tc_copy_sf(sfb_t + j * 4 * (BN / 128) + 4 * rb, desc_sf(sfb_s + rb * 2048 + j * 512));
+          }
+          for (int j = 0; j < nk64; ++j) {
+            tc_mma_fp4(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, sfa_t + 4 * j,
+                       sfb_t + j * 4 * (BN / 128), (kt | j) != 0 ? 1u : 0u);
+          }
+          tc_commit(bar_empty(stage));
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        tc_commit(bar_accf(acc));
+        if (++acc == C::ACC_STAGES) {
+          acc = 0;
+          acc_phase ^= 1u;
+        }
+      }
+      if (!ok) {
+        report_status(args.status, kErrTimeout);
+        *abort_flag = 1;
+      }
+    }
+  } else {
+    // ===================================================================== epilogue
+    const int quad = warp & 3;  // tensor-memory lanes [32*quad, 32*quad + 32)
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    float amax = 0.0f;
+    for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+      const int64_t mb = t / args.n_blocks;
+      const int nb = (int)(t - mb * args.n_blocks);
+      const int e = grouped ? find_expert(args.offsets, args.E, mb * BM) : 0;
+      // every lane polls (acquire), and all lanes agree on the outcome before the
+      // warp-collective tensor-memory loads
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar_accf(acc), acc_phase, limit, abort_flag));
+      if (!got) {
+        if (lane == 0) {
+          report_status(args.status, kErrTimeout);
+          *abort_flag = 1;
+        }
+        break;
+      }
+      tc_fence_after();
+      const int64_t row = mb * BM + quad * 32 + lane;
+      const bool row_ok = row < row_limit && row < args.rows_capacity;
+      const float alpha = __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));
+      const uint32_t t_row = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(quad * 32) << 16);
+      if (args.epi == 0) {
+#pragma unroll 1
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(t_row + c * 32, v);
+          tmem_wait_ld();
+          if (row_ok) {
+            const int64_t col = (int64_t)nb * BN + c * 32;
+            if (args.out_bf16) {
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy + col);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint32_t p[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+                  p[h] = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * q + 2 * h]), alpha),
+                                     __fmul_rn(__uint_as_float(v[8 * q + 2 * h + 1]), alpha));
+                dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
+              }
+            } else {
+              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.y) + row * args.ldy + col);
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                dst[q] = make_float4(__fmul_rn(__uint_as_float(v[4 * q]), alpha),
+                                     __fmul_rn(__uint_as_float(v[4 * q + 1]), alpha),
+                                     __fmul_rn(__uint_as_float(v[4 * q + 2]), alpha),
+                                     __fmul_rn(__uint_as_float(v[4 * q + 3]), alpha));
+            }
+          }
+        }
+      } else {
+        // SwiGLU: within each 128-column half of the tile, columns [0,64) are gate rows and
+        // [64,128) the matching up rows (gate/up interleave of the packed weight).
+#pragma unroll 1
+        for (int hh = 0; hh < BN / 128; ++hh) {
+#pragma unroll 1
+          for (int c = 0; c < 2; ++c) {
+            uint32_t g[32], u[32];
+            tmem_ld32(t_row + hh * 128 + c * 32, g);
+            tmem_ld32(t_row + hh * 128 + 64 + c * 32, u);
+            tmem_wait_ld();
+            if (row_ok) {
+              const int64_t col = (int64_t)nb * (BN / 2) + hh * 64 + c * 32;
+              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy + col);
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint32_t p[4];
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                  float hv[2];
+#pragma unroll
+                  for (int z = 0; z < 2; ++z) {
+                    const int i = 8 * q + 2 * h + z;
+                    const float gv = bf16_round(__fmul_rn(__uint_as_float(g[i]), alpha));
+                    const float uv = bf16_round(__fmul_rn(__uint_as_float(u[i]), alpha));
+                    const float s = gv / (1.0f + expf(-gv));
+                    hv[z] = bf16_round(s * uv);
+                    amax = fmaxf(amax, fabsf(hv[z]));
+                  }
+                  p[h] = pack_bf16x2(hv[0], hv[1]);
+                }
+                dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
+              }
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_acce(acc));
+      if (++acc == C::ACC_STAGES) {
+        acc = 0;
+        acc_phase ^= 1u;
+      }
+    }
+    if (args.epi != 0 && args.amax_out != nullptr) {
+      amax = warp_max(amax);
+      if (lane == 0 && amax > 0.0f) atomicMax(reinterpret_cast<unsigned int*>(args.amax_out), __float_as_uint(amax));
+    }
+  }
+
+  // ---- teardown
+  __syncthreads();
+  if (*abort_flag) {
+    if (warp == 1 && lane == 0) {
+      // all MMAs issued by this thread complete before the commit arrives
+      tc_commit(bar_drain);
+      mbar_wait(bar_drain, 0, limit, nullptr);
+    }
+    if (warp == 0 && lane == 0) {
+      // copies issued but never consumed by the MMA thread
+      for (int i = *mma_taken; i < *prod_issued; ++i)
+        mbar_wait(bar_full(i % C::STAGES), (uint32_t)((i / C::STAGES) & 1), limit, nullptr);
+    }
+    __syncthreads();
+  }
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"((uint32_t)C::TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// A kernel that only runs the bounded wait on a barrier nothing completes (self-test of the
+// timeout path: it must come back with NVFP4_ERR_TIMEOUT in *status).
+__global__ void wait_selftest_kernel(uint64_t limit_ns, int32_t* status) {
+  __shared__ __align__(8) uint64_t bar;
+  const uint32_t b = smem_u32(&bar);
+  if (threadIdx.x == 0) {
+    mbar_init(b, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    if (!mbar_wait(b, 0, limit_ns, nullptr)) report_status(status, kErrTimeout);
+  }
+}
+
+}  // namespace tc
+
+size_t gemm_smem_bytes(int bn) { return bn == 256 ? (size_t)tc::Cfg<256>::SMEM : (size_t)tc::Cfg<128>::SMEM; }
+
+cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
+                        const CUtensorMap& tm_ws, const GemmArgs& args, int grid, cudaStream_t st) {
+  cudaError_t e;
+  if (bn == 256) {
+    e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Cfg<256>::SMEM);
+    if (e != cudaSuccess) return e;
+    tc::w4a4_rac_gemm_kernel<256><<<grid, tc::NUM_THREADS, tc::Cfg<256>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, args);
+  } else if (bn == 128) {
+    e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             tc::Cfg<128>::SMEM);
+    if (e != cudaSuccess) return e;
+    tc::w4a4_rac_gemm_kernel<128><<<grid, tc::NUM_THREADS, tc::Cfg<128>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, args);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t st) {
+  tc::wait_selftest_kernel<<<1, 32, 0, st>>>(limit_ns, status);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

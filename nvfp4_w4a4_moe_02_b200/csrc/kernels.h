@@ -1,0 +1,90 @@
+// Internal launcher declarations shared by the kernel files and the C-ABI layer.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4 {
+
+enum { kModeAct = 0, kModePack = 1, kModeCal = 2 };
+constexpr int64_t kMaxCalK = 16384;
+constexpr int64_t kMaxK = 32768;
+
+// Row quantiser arguments (one warp per output row).
+struct RowArgs {
+  int mode;                      // kModeAct, kModePack, kModeCal
+  const uint16_t* src;           // bf16 rows
+  int64_t src_rows;              // valid source rows (act: M; pack: N per slab; cal: T)
+  int64_t ld;                    // source pitch (elements)
+  int64_t K;                     // channels
+  const int32_t* row_gather;     // act: optional output-row -> source-row map
+  int64_t rows_out;              // output rows to write (act: rows_padded; pack: slabs*rows_padded)
+  int64_t rows_per_slab;         // pack: rows_padded per slab (== N); otherwise rows_out
+  int64_t src_slab_stride;       // pack: N*K elements between slabs
+  int interleave;                // pack: SwiGLU gate/up interleave
+  int64_t N_half;                // pack: N/2
+  const int32_t* sel;            // ascending channel list [Kp]
+  int32_t Kp;
+  // scale source
+  const float* partial;          // amax partials [slabs x P]
+  int P;
+  const float* amax_in;          // act: given amax (overrides partials)
+  float* s_g_out;                // per-slab s_g written by the first warp of each slab
+  float* s_g_out2;               // second copy (residual tensor's s_g), may be null
+  // outputs
+  uint8_t* codes;                // [rows_out x K/2]
+  uint8_t* sf;                   // atoms, K/64 groups per row
+  uint8_t* rcodes;               // [rows_out x Kp/2]
+  uint8_t* rsf;                  // atoms, Kp/64 groups per row
+  float* resid_all;              // cal: [rows_out x K] residual of every channel
+  int32_t* status;
+};
+
+cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64_t cols, int64_t ld, float* partial,
+                        int P, int32_t* status, cudaStream_t st);
+cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st);
+size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps);
+cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, double* err, cudaStream_t st);
+cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t* sel, double* err_out, cudaStream_t st);
+cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint16_t* out, const float* partial, int P,
+                       float* s_g_out, int32_t* status, int num_sms, cudaStream_t st);
+cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
+cudaError_t launch_encode_e4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
+
+// ---- tcgen05 block-scaled GEMM (dense and grouped)
+struct GemmArgs {
+  const uint8_t* sfa;        // A scale atoms, rows_padded/128 x k64_main
+  const uint8_t* sfa_res;    // A residual scale atoms, rows_padded/128 x k64_res
+  const uint8_t* sfw;        // W scale atoms, per slab N/128 x k64_main
+  const uint8_t* sfw_sel;    // W_sel scale atoms, per slab N/128 x k64_res
+  int64_t sfw_slab_bytes;
+  int64_t sfw_sel_slab_bytes;
+  int32_t k64_main, k64_res; // K/64, Kp/64
+  int32_t kt_main, kt_res;   // k-tiles of 256 elements (last may be partial)
+  int32_t N;                 // output columns of the MMA (before the SwiGLU halving)
+  int32_t n_blocks;          // N / BN
+  const int32_t* offsets;    // grouped: device [E+1]; dense: nullptr
+  int32_t E;
+  int64_t M;                 // dense: valid rows (stores masked beyond)
+  int32_t m_blocks_dense;    // dense: ceil(M/128)
+  int64_t rows_capacity;     // rows of the A / Y buffers
+  const float* s_a;          // device scalar
+  const float* s_w;          // device [E]
+  void* y;
+  int64_t ldy;
+  int32_t out_bf16;
+  int32_t epi;               // 0 none, 1 SwiGLU + amax
+  float* amax_out;
+  int32_t* status;
+  uint64_t wait_limit_ns;
+};
+
+// bn: 128 or 256
+cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
+                        const CUtensorMap& tm_ws, const GemmArgs& args, int grid, cudaStream_t st);
+size_t gemm_smem_bytes(int bn);
+
+cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t st);
+
+}  // namespace nvfp4

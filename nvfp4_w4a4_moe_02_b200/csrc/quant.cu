@@ -1,0 +1,532 @@
+// Quantisation kernels: per-tensor amax, the row quantiser (activation + RAC residual,
+// weight pack, calibration residuals), calibration reduction/selection and trainer QDQ.
+//
+// All of them are HBM-streaming kernels: 128-bit loads of 8 bf16, two lanes per 16-element
+// block (one shuffle for the block max), packed e2m1 stores that stay contiguous across the
+// warp, and scales written straight into the 512-byte scale atoms the tcgen05 MMA reads.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+// ----------------------------------------------------------------------------------------
+// K1: segmented amax.  Segment s = rows [s*seg_rows, (s+1)*seg_rows) of a [rows x cols]
+// bf16 matrix with pitch ld.  Grid (P, segments); CTA p writes partial[s*P + p].
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ x, int64_t seg_rows, int64_t cols,
+                                                   int64_t ld, float* __restrict__ partial, int32_t* status) {
+  const int P = gridDim.x;
+  const int64_t seg = blockIdx.y;
+  float m = 0.0f;
+  bool bad = false;
+  const uint16_t* base = x + seg * seg_rows * ld;
+  if (ld == cols) {
+    // contiguous segment: flat vector loop
+    const int64_t nvec = seg_rows * cols / 8;
+    const uint4* v = reinterpret_cast<const uint4*>(base);
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += (int64_t)P * blockDim.x) {
+      uint4 q = __ldg(v + i);
+      uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float a = fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu));
+        float b = fabsf(bf16_bits_to_f32(w[j] >> 16));
+        bad |= !(a <= 3.4e38f) || !(b <= 3.4e38f);
+        m = fmaxf(m, fmaxf(a, b));
+      }
+    }
+  } else {
+    const int64_t vpr = cols / 8;
+    for (int64_t r = blockIdx.x; r < seg_rows; r += P) {
+      const uint4* v = reinterpret_cast<const uint4*>(base + r * ld);
+      for (int64_t i = threadIdx.x; i < vpr; i += blockDim.x) {
+        uint4 q = __ldg(v + i);
+        uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float a = fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu));
+          float b = fabsf(bf16_bits_to_f32(w[j] >> 16));
+          bad |= !(a <= 3.4e38f) || !(b <= 3.4e38f);
+          m = fmaxf(m, fmaxf(a, b));
+        }
+      }
+    }
+  }
+  if (bad) report_status(status, kErrRange);
+  __shared__ float red[8];
+  m = warp_max(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.0f;
+    v = warp_max(v);
+    if (threadIdx.x == 0) partial[seg * P + blockIdx.x] = v;
+  }
+}
+
+// max over P partials of one segment, by one warp (all lanes return the result)
+__device__ __forceinline__ float reduce_partials(const float* partial, int P) {
+  float m = 0.0f;
+  for (int i = threadIdx.x & 31; i < P; i += 32) m = fmaxf(m, partial[i]);
+  return warp_max(m);
+}
+
+// ----------------------------------------------------------------------------------------
+// K2 / K7 / calibration: the row quantiser.  One warp per output row, 512 elements per warp
+// iteration: lane l loads elements [it*512 + 8l, +8) and [it*512 + 256 + 8l, +8), so lanes
+// (2m, 2m+1) hold the two halves of block it*32 + m and of block it*32 + 16 + m.
+// ----------------------------------------------------------------------------------------
+
+
+// Writes the 4-byte scale word of a k64 group: lanes 8g..8g+7 own blocks 4g'..4g'+3 where
+// the pair (2m, 2m+1) owns block m; lane 8g gathers from lanes 8g, 8g+2, 8g+4, 8g+6.
+__device__ __forceinline__ void store_scale_words(uint32_t S, uint8_t* sf, int64_t row, int64_t kb_base, int64_t k64,
+                                                  int lane, bool active) {
+  uint32_t s1 = __shfl_down_sync(0xffffffffu, S, 2);
+  uint32_t s2 = __shfl_down_sync(0xffffffffu, S, 4);
+  uint32_t s3 = __shfl_down_sync(0xffffffffu, S, 6);
+  if (active && (lane & 7) == 0) {
+    uint32_t word = S | (s1 << 8) | (s2 << 16) | (s3 << 24);
+    int64_t kb = kb_base + (lane >> 1);  // first block of this k64 group
+    *reinterpret_cast<uint32_t*>(sf + sf_offset(row, kb, k64)) = word;
+  }
+}
+
+template <int MODE>
+__global__ void __launch_bounds__(256) quant_rows_kernel(const RowArgs a) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  const int64_t K = a.K;
+  const int32_t Kp = a.Kp;
+  constexpr bool kHasSel = (MODE == kModeAct || MODE == kModePack);
+
+  // channel -> compact position map (-1 = not selected), shared by the CTA
+  int16_t* pos = reinterpret_cast<int16_t*>(smem_raw);
+  float* rbuf_all = reinterpret_cast<float*>(smem_raw + ((K * 2 + 15) / 16) * 16);
+  float* rbuf = rbuf_all + (int64_t)warp * (Kp > 0 ? Kp : 1);
+  if (kHasSel && Kp > 0) {
+    for (int64_t c = threadIdx.x; c < K; c += blockDim.x) pos[c] = -1;
+    __syncthreads();
+    for (int32_t j = threadIdx.x; j < Kp; j += blockDim.x) {
+      int32_t c = a.sel[j];
+      bool ok = (c >= 0 && c < K) && (j == 0 || a.sel[j - 1] < c);
+      if (ok) pos[c] = (int16_t)j;
+      else report_status(a.status, kErrInvalid);
+    }
+    __syncthreads();
+  }
+
+  const int64_t k64 = K / 64;
+  const int64_t kp64 = Kp / 64;
+  const int64_t n_it = K / 512;           // full 512-element iterations
+  const int64_t tail = K - n_it * 512;    // 0, 64, ..., 448 (K % 64 == 0)
+  int64_t cached_slab = -1;
+  float s_g = 0.0f, t6 = 0.0f;
+
+  for (int64_t row = (int64_t)blockIdx.x * nwarps + warp; row < a.rows_out; row += (int64_t)gridDim.x * nwarps) {
+    // ---- source row and scale
+    int64_t slab = (MODE == kModePack) ? row / a.rows_per_slab : 0;
+    int64_t r_in_slab = row - slab * a.rows_per_slab;
+    int64_t src_row = r_in_slab;
+    if (MODE == kModeAct && a.row_gather != nullptr) src_row = (r_in_slab < a.rows_per_slab) ? a.row_gather[r_in_slab] : -1;
+    if (MODE == kModeAct && a.row_gather != nullptr && row >= a.rows_per_slab) src_row = -1;
+    if (MODE == kModePack && a.interleave) {
+      int64_t q = r_in_slab >> 7, j = r_in_slab & 127;
+      src_row = (j < 64) ? (q * 64 + j) : (a.N_half + q * 64 + (j - 64));
+    }
+    const bool valid = (src_row >= 0 && src_row < a.src_rows);
+    if (slab != cached_slab) {
+      float amax = (MODE == kModeAct && a.amax_in != nullptr) ? *a.amax_in : reduce_partials(a.partial + slab * a.P, a.P);
+      s_g = scale_from_amax(amax, a.status);
+      t6 = __fmul_rn(6.0f, s_g);
+      cached_slab = slab;
+      if (row == slab * a.rows_per_slab + 0 && lane == 0) {
+        // exactly one warp writes each slab's scale: the one owning the slab's first row
+        if (a.s_g_out) a.s_g_out[slab] = s_g;
+        if (a.s_g_out2) a.s_g_out2[slab] = s_g;
+      }
+    }
+    const uint16_t* srow = a.src + slab * a.src_slab_stride + (valid ? src_row : 0) * a.ld;
+
+    // ---- main pass over the row, 512 (or a 64..448 tail) elements per iteration
+    for (int64_t it = 0; it <= n_it; ++it) {
+      const int64_t base = it * 512;
+      const int64_t span = (it < n_it) ? 512 : tail;
+      if (span == 0) break;
+      // element offsets held by this lane
+      const int64_t e0 = base + 8 * lane;          // first half-block
+      const int64_t e1 = base + 256 + 8 * lane;    // second half-block
+      const bool h0 = e0 < base + span;            // span is a multiple of 64: pair-uniform
+      const bool h1 = e1 < base + span;
+      float x0[8], x1[8];
+      {
+        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
+        if (valid && h0) q0 = __ldg(reinterpret_cast<const uint4*>(srow + e0));
+        if (valid && h1) q1 = __ldg(reinterpret_cast<const uint4*>(srow + e1));
+        uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          x0[2 * j] = bf16_bits_to_f32(w0[j] & 0xFFFFu);
+          x0[2 * j + 1] = bf16_bits_to_f32(w0[j] >> 16);
+          x1[2 * j] = bf16_bits_to_f32(w1[j] & 0xFFFFu);
+          x1[2 * j + 1] = bf16_bits_to_f32(w1[j] >> 16);
+        }
+      }
+      float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        m0 = fmaxf(m0, fabsf(x0[i]));
+        m1 = fmaxf(m1, fabsf(x1[i]));
+      }
+      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+      BlockScale b0 = block_scale(m0, s_g, t6), b1 = block_scale(m1, s_g, t6);
+      float dq0[8], dq1[8];
+      uint32_t c0 = quant8(x0, b0, dq0);
+      uint32_t c1 = quant8(x1, b1, dq1);
+      if (MODE != kModeCal) {
+        uint8_t* crow = a.codes + row * (K / 2);
+        if (h0) *reinterpret_cast<uint32_t*>(crow + e0 / 2) = c0;
+        if (h1) *reinterpret_cast<uint32_t*>(crow + e1 / 2) = c1;
+        // scale words: the first half covers blocks base/16 + [0,16), the second + [16,32)
+        store_scale_words(b0.S, a.sf, row, base / 16, k64, lane, h0);
+        store_scale_words(b1.S, a.sf, row, base / 16 + 16, k64, lane, h1);
+      }
+      if (MODE == kModeCal) {
+        float* rr = a.resid_all + row * K;
+        if (h0) {
+          float4 r0 = make_float4(__fsub_rn(x0[0], dq0[0]), __fsub_rn(x0[1], dq0[1]), __fsub_rn(x0[2], dq0[2]),
+                                  __fsub_rn(x0[3], dq0[3]));
+          float4 r1 = make_float4(__fsub_rn(x0[4], dq0[4]), __fsub_rn(x0[5], dq0[5]), __fsub_rn(x0[6], dq0[6]),
+                                  __fsub_rn(x0[7], dq0[7]));
+          *reinterpret_cast<float4*>(rr + e0) = r0;
+          *reinterpret_cast<float4*>(rr + e0 + 4) = r1;
+        }
+        if (h1) {
+          float4 r0 = make_float4(__fsub_rn(x1[0], dq1[0]), __fsub_rn(x1[1], dq1[1]), __fsub_rn(x1[2], dq1[2]),
+                                  __fsub_rn(x1[3], dq1[3]));
+          float4 r1 = make_float4(__fsub_rn(x1[4], dq1[4]), __fsub_rn(x1[5], dq1[5]), __fsub_rn(x1[6], dq1[6]),
+                                  __fsub_rn(x1[7], dq1[7]));
+          *reinterpret_cast<float4*>(rr + e1) = r0;
+          *reinterpret_cast<float4*>(rr + e1 + 4) = r1;
+        }
+      }
+      if (kHasSel && Kp > 0) {
+        // selected channels: residual (act) or raw value (pack) into the compact row buffer
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          if (h0) {
+            int p = pos[e0 + i];
+            if (p >= 0) rbuf[p] = (MODE == kModeAct) ? __fsub_rn(x0[i], dq0[i]) : x0[i];
+          }
+          if (h1) {
+            int p = pos[e1 + i];
+            if (p >= 0) rbuf[p] = (MODE == kModeAct) ? __fsub_rn(x1[i], dq1[i]) : x1[i];
+          }
+        }
+      }
+    }
+
+    // ---- second pass over the compact selected channels
+    if (kHasSel && Kp > 0) {
+      __syncwarp();
+      const int64_t nr_it = Kp / 512, rtail = Kp - nr_it * 512;
+      for (int64_t it = 0; it <= nr_it; ++it) {
+        const int64_t base = it * 512;
+        const int64_t span = (it < nr_it) ? 512 : rtail;
+        if (span == 0) break;
+        const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
+        const bool h0 = e0 < base + span, h1 = e1 < base + span;
+        float x0[8], x1[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          x0[i] = (valid && h0) ? rbuf[e0 + i] : 0.0f;
+          x1[i] = (valid && h1) ? rbuf[e1 + i] : 0.0f;
+        }
+        float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          m0 = fmaxf(m0, fabsf(x0[i]));
+          m1 = fmaxf(m1, fabsf(x1[i]));
+        }
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+        BlockScale b0 = block_scale(m0, s_g, t6), b1 = block_scale(m1, s_g, t6);
+        uint32_t c0 = quant8_codes(x0, b0);
+        uint32_t c1 = quant8_codes(x1, b1);
+        uint8_t* crow = a.rcodes + row * (Kp / 2);
+        if (h0) *reinterpret_cast<uint32_t*>(crow + e0 / 2) = c0;
+        if (h1) *reinterpret_cast<uint32_t*>(crow + e1 / 2) = c1;
+        store_scale_words(b0.S, a.rsf, row, base / 16, kp64, lane, h0);
+        store_scale_words(b1.S, a.rsf, row, base / 16 + 16, kp64, lane, h1);
+      }
+      __syncwarp();
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// calibration: e_k = sum_t r_{t,k}^2 in binary64, t ascending (one thread per channel), then
+// selection of the Kp largest (ties -> lower k), written ascending.
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) chan_err_kernel(const float* __restrict__ resid, int64_t T, int64_t K,
+                                                       double* __restrict__ err) {
+  int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (k >= K) return;
+  double e = 0.0;
+  for (int64_t t = 0; t < T; ++t) {
+    double v = (double)resid[t * K + k];
+    e = __dadd_rn(e, __dmul_rn(v, v));
+  }
+  err[k] = e;
+}
+
+// One CTA of 1024 threads; K <= kMaxCalK.
+__global__ void __launch_bounds__(1024) select_topk_kernel(const double* __restrict__ err, int32_t K, int32_t Kp,
+                                                           int32_t* __restrict__ sel_out, double* __restrict__ err_out) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  double* e = reinterpret_cast<double*>(smem_raw);
+  int32_t* flag = reinterpret_cast<int32_t*>(e + K);
+  __shared__ int32_t warp_sums[32];
+  for (int32_t k = threadIdx.x; k < K; k += blockDim.x) {
+    e[k] = err[k];
+    if (err_out) err_out[k] = err[k];
+  }
+  __syncthreads();
+  for (int32_t k = threadIdx.x; k < K; k += blockDim.x) {
+    const double ek = e[k];
+    int32_t rank = 0;
+    for (int32_t j = 0; j < K; ++j) {
+      const double ej = e[j];
+      rank += (ej > ek) || (ej == ek && j < k);
+    }
+    flag[k] = rank < Kp;
+  }
+  __syncthreads();
+  // ascending compaction: chunked exclusive scan over K flags
+  int32_t carry = 0;
+  for (int32_t base = 0; base < K; base += blockDim.x) {
+    int32_t k = base + threadIdx.x;
+    int32_t f = (k < K) ? flag[k] : 0;
+    int32_t lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    int32_t incl = f;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int32_t n = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += n;
+    }
+    if (lane == 31) warp_sums[w] = incl;
+    __syncthreads();
+    if (w == 0) {
+      int32_t v = warp_sums[lane];
+      int32_t s = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int32_t n = __shfl_up_sync(0xffffffffu, s, o);
+        if (lane >= o) s += n;
+      }
+      warp_sums[lane] = s - v;  // exclusive prefix of warp totals
+    }
+    __syncthreads();
+    int32_t excl = carry + warp_sums[w] + incl - f;
+    if (f) sel_out[excl] = k;
+    __syncthreads();
+    if (threadIdx.x == blockDim.x - 1) warp_sums[0] = excl + f;  // chunk total (with carry)
+    __syncthreads();
+    carry = warp_sums[0];
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// K8: trainer fake quantisation, bf16(DQ(Q(w))), one scale per tensor.  Same lane layout as
+// the row quantiser over a flat array; each 512-element warp chunk lies inside one tensor
+// when elems_per_tensor % 512 == 0, else the tensor of each 16-block is looked up.
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ w, int64_t n_tensors, int64_t elems,
+                                                  uint16_t* __restrict__ out, const float* __restrict__ partial, int P,
+                                                  float* s_g_out, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t warp_global = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
+  const int64_t total = n_tensors * elems;
+  const int64_t nchunks = (total + 511) / 512;
+  int64_t cached = -1;
+  float s_g = 0.0f, t6 = 0.0f;
+  for (int64_t ch = warp_global; ch < nchunks; ch += nwarps) {
+    const int64_t base = ch * 512;
+    const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
+    const bool h0 = e0 < total, h1 = e1 < total;
+    // tensor of each half-block (uniform over a lane pair: elems % 16 == 0); the scale of a
+    // tensor is reduced from its P partials, cached per lane
+    const int64_t t0 = h0 ? e0 / elems : n_tensors - 1;
+    const int64_t t1 = h1 ? e1 / elems : n_tensors - 1;
+    float sg0, sg1, t60, t61;
+    if (t0 != cached) {
+      float am = 0.0f;
+      for (int i = 0; i < P; ++i) am = fmaxf(am, partial[t0 * P + i]);
+      s_g = scale_from_amax(am, status);
+      t6 = __fmul_rn(6.0f, s_g);
+      cached = t0;
+    }
+    sg0 = s_g;
+    t60 = t6;
+    if (t1 != cached) {
+      float am = 0.0f;
+      for (int i = 0; i < P; ++i) am = fmaxf(am, partial[t1 * P + i]);
+      sg1 = scale_from_amax(am, status);
+      t61 = __fmul_rn(6.0f, sg1);
+    } else {
+      sg1 = s_g;
+      t61 = t6;
+    }
+    if (s_g_out) {
+      if (h0 && e0 % elems == 0) s_g_out[t0] = sg0;
+      if (h1 && e1 % elems == 0) s_g_out[t1] = sg1;
+    }
+    float x0[8], x1[8];
+    uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
+    if (h0) q0 = __ldg(reinterpret_cast<const uint4*>(w + e0));
+    if (h1) q1 = __ldg(reinterpret_cast<const uint4*>(w + e1));
+    uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      x0[2 * j] = bf16_bits_to_f32(w0[j] & 0xFFFFu);
+      x0[2 * j + 1] = bf16_bits_to_f32(w0[j] >> 16);
+      x1[2 * j] = bf16_bits_to_f32(w1[j] & 0xFFFFu);
+      x1[2 * j + 1] = bf16_bits_to_f32(w1[j] >> 16);
+    }
+    float m0 = 0.0f, m1 = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      m0 = fmaxf(m0, fabsf(x0[i]));
+      m1 = fmaxf(m1, fabsf(x1[i]));
+    }
+    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
+    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
+    BlockScale b0 = block_scale(m0, sg0, t60), b1 = block_scale(m1, sg1, t61);
+    float dq0[8], dq1[8];
+    quant8(x0, b0, dq0);
+    quant8(x1, b1, dq1);
+    uint32_t o0[4], o1[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      __nv_bfloat162 p0 = __floats2bfloat162_rn(dq0[2 * j], dq0[2 * j + 1]);
+      __nv_bfloat162 p1 = __floats2bfloat162_rn(dq1[2 * j], dq1[2 * j + 1]);
+      o0[j] = *reinterpret_cast<uint32_t*>(&p0);
+      o1[j] = *reinterpret_cast<uint32_t*>(&p1);
+    }
+    if (h0) *reinterpret_cast<uint4*>(out + e0) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
+    if (h1) *reinterpret_cast<uint4*>(out + e1) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// codec test kernels
+// ----------------------------------------------------------------------------------------
+__global__ void encode_e2m1_kernel(const float* v, int64_t n, uint8_t* out) {
+  int64_t i = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) * 8;
+  if (i >= n) return;
+  float x[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) x[j] = (i + j < n) ? v[i + j] : 0.0f;
+  uint32_t c = e2m1_encode8(x);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if (i + j < n) out[i + j] = (c >> (4 * j)) & 0xF;
+}
+
+__global__ void encode_e4m3_kernel(const float* v, int64_t n, uint8_t* out) {
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) out[i] = (uint8_t)e4m3_encode(v[i]);
+}
+
+// ----------------------------------------------------------------------------------------
+// host launchers
+// ----------------------------------------------------------------------------------------
+cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64_t cols, int64_t ld, float* partial,
+                        int P, int32_t* status, cudaStream_t st) {
+  dim3 grid(P, (unsigned)segs);
+  amax_kernel<<<grid, 256, 0, st>>>(x, seg_rows, cols, ld, partial, status);
+  return cudaGetLastError();
+}
+
+size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps) {
+  return (size_t)((K * 2 + 15) / 16) * 16 + (size_t)warps * (size_t)(Kp > 0 ? Kp : 1) * 4;
+}
+
+cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
+  int warps = 8;
+  size_t smem = rows_smem_bytes(a.K, a.Kp, warps);
+  while (smem > 200 * 1024 && warps > 1) {
+    warps /= 2;
+    smem = rows_smem_bytes(a.K, a.Kp, warps);
+  }
+  if (smem > 200 * 1024) return cudaErrorInvalidValue;
+  int64_t ctas_needed = (a.rows_out + warps - 1) / warps;
+  int per_sm = (int)((220 * 1024) / (smem + 1024));
+  if (per_sm < 1) per_sm = 1;
+  if (per_sm > 8) per_sm = 8;
+  int64_t grid = (int64_t)num_sms * per_sm;
+  if (grid > ctas_needed) grid = ctas_needed;
+  if (grid < 1) grid = 1;
+  cudaError_t e = cudaSuccess;
+  switch (a.mode) {
+    case kModeAct:
+      e = cudaFuncSetAttribute(quant_rows_kernel<kModeAct>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) quant_rows_kernel<kModeAct><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      break;
+    case kModePack:
+      e = cudaFuncSetAttribute(quant_rows_kernel<kModePack>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) quant_rows_kernel<kModePack><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      break;
+    case kModeCal:
+      e = cudaFuncSetAttribute(quant_rows_kernel<kModeCal>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e == cudaSuccess) quant_rows_kernel<kModeCal><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      break;
+    default:
+      return cudaErrorInvalidValue;
+  }
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, double* err, cudaStream_t st) {
+  chan_err_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(resid, T, K, err);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t* sel, double* err_out, cudaStream_t st) {
+  size_t smem = (size_t)K * 8 + (size_t)K * 4;
+  cudaError_t e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  select_topk_kernel<<<1, 1024, smem, st>>>(err, K, Kp, sel, err_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint16_t* out, const float* partial, int P,
+                       float* s_g_out, int32_t* status, int num_sms, cudaStream_t st) {
+  int64_t total = n_tensors * elems;
+  int64_t warps_needed = (total + 511) / 512;
+  int64_t grid = (warps_needed + 7) / 8;
+  int64_t cap = (int64_t)num_sms * 8;
+  if (grid > cap) grid = cap;
+  if (grid < 1) grid = 1;
+  qdq_kernel<<<(unsigned)grid, 256, 0, st>>>(w, n_tensors, elems, out, partial, P, s_g_out, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t st) {
+  int64_t threads = (n + 7) / 8;
+  encode_e2m1_kernel<<<(unsigned)((threads + 255) / 256), 256, 0, st>>>(v, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_encode_e4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t st) {
+  encode_e4m3_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(v, n, out);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,351 @@
+"""Python binding of the C-ABI library ``libnvfp4rac.so`` (ctypes).
+
+Argument marshalling only: every step of the NVFP4 W4A4 + RAC path runs in the CUDA
+kernels behind the C ABI (declared in ``include/nvfp4rac.h``).  PyTorch provides device
+memory and the current stream.  If the compiled library is missing, loading it raises: there
+is no fallback implementation.
+
+Call names match the C ABI: ``nvfp4_quantize``, ``rac_calibrate``, ``pack_weights``,
+``w4a4_rac_gemm``, ``grouped_w4a4_rac_moe``, ``weight_qdq``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libnvfp4rac.so")
+
+OK = 0
+STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED_SHAPE", 3: "ERR_ALIGNMENT", 4: "ERR_RANGE",
+                5: "ERR_CUDA", 6: "ERR_TIMEOUT"}
+OUT_F32, OUT_BF16 = 0, 1
+EPI_NONE, EPI_SWIGLU_AMAX = 0, 1
+
+
+class NVFP4Error(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS_NAMES.get(status, status)}: {msg}")
+        self.status = status
+
+
+class CTensor(ctypes.Structure):
+    _fields_ = [("codes", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("s_g", ctypes.c_void_p),
+                ("slabs", ctypes.c_int64), ("rows", ctypes.c_int64), ("rows_padded", ctypes.c_int64),
+                ("cols", ctypes.c_int64)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load the CUDA library (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m nvfp4_w4a4_moe_02_b200.build_lib`")
+    lib = ctypes.CDLL(LIB_PATH)
+    vp, i64, i32, sz, u64 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t, ctypes.c_uint64
+    tp = ctypes.POINTER(CTensor)
+    sigs = {
+        "nvfp4_version": ([], i32),
+        "nvfp4_status_string": ([ctypes.c_int], ctypes.c_char_p),
+        "nvfp4_last_error_string": ([], ctypes.c_char_p),
+        "nvfp4_codes_bytes": ([i64, i64], sz),
+        "nvfp4_sf_bytes": ([i64, i64], sz),
+        "nvfp4_kp_from_ratio": ([i64, ctypes.c_double], i32),
+        "nvfp4_set_wait_limit_ns": ([u64], None),
+        "nvfp4_quantize_workspace_size": ([i64, i64], sz),
+        "nvfp4_quantize": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "rac_calibrate_workspace_size": ([i64, i64], sz),
+        "rac_calibrate": ([vp, i64, i64, i32, vp, vp, vp, sz, vp, vp], ctypes.c_int),
+        "pack_weights_workspace_size": ([i64, i64, i64], sz),
+        "pack_weights": ([vp, i64, i64, i64, vp, i32, i32, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "w4a4_rac_gemm": ([tp, tp, tp, tp, i64, i64, i64, i32, ctypes.c_int, vp, i64, vp, vp], ctypes.c_int),
+        "grouped_w4a4_rac_moe": ([tp, tp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, i64, vp,
+                                  vp, vp], ctypes.c_int),
+        "weight_qdq_workspace_size": ([i64, i64], sz),
+        "weight_qdq": ([vp, i64, i64, vp, vp, vp, sz, vp, vp], ctypes.c_int),
+        "nvfp4_encode_e2m1": ([vp, i64, vp, vp], ctypes.c_int),
+        "nvfp4_encode_e4m3": ([vp, i64, vp, vp], ctypes.c_int),
+        "nvfp4_selftest_wait_timeout": ([u64, vp, vp], ctypes.c_int),
+    }
+    for name, (args, res) in sigs.items():
+        fn = getattr(lib, name)
+        fn.argtypes = args
+        fn.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != OK:
+        raise NVFP4Error(status, load().nvfp4_last_error_string().decode())
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _u16(x: torch.Tensor) -> torch.Tensor:
+    assert x.is_cuda and x.dtype in (torch.bfloat16, torch.int16, torch.uint16), x.dtype
+    return x
+
+
+def round_up(v: int, a: int) -> int:
+    return (v + a - 1) // a * a
+
+
+@dataclass
+class Packed:
+    """Caller-side owner of one packed NVFP4 tensor (device buffers allocated by torch)."""
+    codes: torch.Tensor   # uint8 [slabs * rows_padded * cols/2]
+    sf: torch.Tensor      # uint8 [slabs * rows_padded * cols/16]
+    s_g: torch.Tensor     # float32 [slabs]
+    slabs: int
+    rows: int
+    rows_padded: int
+    cols: int
+
+    @staticmethod
+    def empty(rows: int, cols: int, slabs: int = 1, rows_padded: int | None = None, device="cuda") -> "Packed":
+        rp = round_up(max(rows, 1), 128) if rows_padded is None else rows_padded
+        codes = torch.empty(slabs * rp * cols // 2, dtype=torch.uint8, device=device)
+        sf = torch.empty(slabs * rp * cols // 16, dtype=torch.uint8, device=device)
+        s_g = torch.empty(slabs, dtype=torch.float32, device=device)
+        return Packed(codes, sf, s_g, slabs, rows, rp, cols)
+
+    def c(self) -> CTensor:
+        return CTensor(self.codes.data_ptr(), self.sf.data_ptr(), self.s_g.data_ptr(), self.slabs, self.rows,
+                       self.rows_padded, self.cols)
+
+
+class Workspace:
+    """Grow-only device scratch buffer handed to calls that need one."""
+
+    def __init__(self, device="cuda"):
+        self.buf = torch.empty(0, dtype=torch.uint8, device=device)
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf.numel() < nbytes:
+            self.buf = torch.empty(round_up(max(nbytes, 1), 1 << 20), dtype=torch.uint8, device=self.buf.device)
+        return self.buf
+
+
+_ws: dict = {}
+
+
+def _workspace(device) -> Workspace:
+    key = str(device)
+    if key not in _ws:
+        _ws[key] = Workspace(device)
+    return _ws[key]
+
+
+def new_status(device="cuda") -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def check_status(status: torch.Tensor):
+    """Raise if a device-side error was recorded (synchronises)."""
+    v = int(status.item())
+    if v != OK:
+        raise NVFP4Error(v, "device-side error")
+
+
+def kp_from_ratio(K: int, r: float) -> int:
+    return int(load().nvfp4_kp_from_ratio(K, r))
+
+
+def set_wait_limit_ns(ns: int):
+    load().nvfp4_set_wait_limit_ns(ns)
+
+
+# ------------------------------------------------------------------------------------- calls
+def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather: torch.Tensor | None = None,
+                   M_out: int | None = None, rows_padded: int | None = None, amax_in: torch.Tensor | None = None,
+                   out: Packed | None = None, out_res: Packed | None = None, status: torch.Tensor | None = None,
+                   stream=None):
+    """Online activation quantisation with the residual pass on ``sel`` -> (Packed, Packed | None)."""
+    lib = load()
+    _u16(x)
+    M, K = x.shape
+    ldx = x.stride(0)
+    assert x.stride(1) == 1
+    Kp = 0 if sel is None else int(sel.numel())
+    if M_out is None:
+        M_out = M if row_gather is None else int(row_gather.numel())
+    if out is None:
+        out = Packed.empty(M_out, K, rows_padded=rows_padded, device=x.device)
+    if Kp > 0 and out_res is None:
+        out_res = Packed.empty(M_out, Kp, rows_padded=out.rows_padded, device=x.device)
+    ws_bytes = lib.nvfp4_quantize_workspace_size(M, K)
+    ws = _workspace(x.device).get(ws_bytes)
+    st = status if status is not None else new_status(x.device)
+    q = out.c()
+    qr = out_res.c() if Kp > 0 else None
+    _check(lib.nvfp4_quantize(x.data_ptr(), M, K, ldx, _ptr(row_gather), M_out, _ptr(sel), Kp, _ptr(amax_in),
+                              ctypes.byref(q), ctypes.byref(qr) if qr is not None else None, ws.data_ptr(),
+                              ws.numel(), st.data_ptr(), _stream(stream)))
+    return out, (out_res if Kp > 0 else None)
+
+
+def rac_calibrate(x_cal: torch.Tensor, Kp: int, want_err: bool = False, status: torch.Tensor | None = None,
+                  stream=None):
+    """Select the Kp highest-error channels of a calibration batch -> (sel int32 [Kp], err float64 [K] | None)."""
+    lib = load()
+    _u16(x_cal)
+    T, K = x_cal.shape
+    assert x_cal.is_contiguous()
+    sel = torch.empty(Kp, dtype=torch.int32, device=x_cal.device)
+    err = torch.empty(K, dtype=torch.float64, device=x_cal.device) if want_err else None
+    ws = _workspace(x_cal.device).get(lib.rac_calibrate_workspace_size(T, K))
+    st = status if status is not None else new_status(x_cal.device)
+    _check(lib.rac_calibrate(x_cal.data_ptr(), T, K, Kp, sel.data_ptr(), _ptr(err), ws.data_ptr(), ws.numel(),
+                             st.data_ptr(), _stream(stream)))
+    return sel, err
+
+
+def pack_weights(w: torch.Tensor, sel: torch.Tensor | None = None, gate_up_interleave: bool = False,
+                 out: Packed | None = None, out_sel: Packed | None = None, status: torch.Tensor | None = None,
+                 stream=None):
+    """Rollout weight pack: Q(W) and Q(W[:, sel]) with one scale per slab -> (Packed, Packed | None)."""
+    lib = load()
+    _u16(w)
+    if w.dim() == 2:
+        w = w.unsqueeze(0)
+    E, N, K = w.shape
+    assert w.is_contiguous()
+    Kp = 0 if sel is None else int(sel.numel())
+    if out is None:
+        out = Packed.empty(N, K, slabs=E, rows_padded=N, device=w.device)
+    if Kp > 0 and out_sel is None:
+        out_sel = Packed.empty(N, Kp, slabs=E, rows_padded=N, device=w.device)
+    ws = _workspace(w.device).get(lib.pack_weights_workspace_size(E, N, K))
+    st = status if status is not None else new_status(w.device)
+    q = out.c()
+    qs = out_sel.c() if Kp > 0 else None
+    _check(lib.pack_weights(w.data_ptr(), E, N, K, _ptr(sel), Kp, int(gate_up_interleave), ctypes.byref(q),
+                            ctypes.byref(qs) if qs is not None else None, ws.data_ptr(), ws.numel(), st.data_ptr(),
+                            _stream(stream)))
+    return out, (out_sel if Kp > 0 else None)
+
+
+def w4a4_rac_gemm(a: Packed, a_res: Packed | None, w: Packed, w_sel: Packed | None, M: int,
+                  out_dtype=torch.bfloat16, y: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                  stream=None) -> torch.Tensor:
+    """Dense Y = s_a s_w (Q(X)Q(W)^T + Q(R_sel)Q(W_sel)^T) -> y [M, N]."""
+    lib = load()
+    N, K = w.rows, w.cols
+    Kp = 0 if a_res is None else a_res.cols
+    if y is None:
+        y = torch.empty(M, N, dtype=out_dtype, device=a.codes.device)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    st = status if status is not None else new_status(a.codes.device)
+    ca, cw = a.c(), w.c()
+    car = a_res.c() if Kp > 0 else None
+    cws = w_sel.c() if Kp > 0 else None
+    _check(lib.w4a4_rac_gemm(ctypes.byref(ca), ctypes.byref(car) if car else None, ctypes.byref(cw),
+                             ctypes.byref(cws) if cws else None, M, N, K, Kp, od, y.data_ptr(), y.stride(0),
+                             st.data_ptr(), _stream(stream)))
+    return y
+
+
+def grouped_w4a4_rac_moe(a: Packed, a_res: Packed | None, expert_offsets: torch.Tensor, w: Packed,
+                         w_sel: Packed | None, swiglu: bool = False, out_dtype=torch.bfloat16,
+                         y: torch.Tensor | None = None, amax_out: torch.Tensor | None = None,
+                         status: torch.Tensor | None = None, stream=None):
+    """Grouped GEMM over expert segments -> y (rows a.rows_padded) [and amax of the SwiGLU output]."""
+    lib = load()
+    E = w.slabs
+    N, K = w.rows, w.cols
+    Kp = 0 if a_res is None else a_res.cols
+    ycols = N // 2 if swiglu else N
+    if y is None:
+        y = torch.empty(a.rows_padded, ycols, dtype=torch.bfloat16 if swiglu else out_dtype, device=a.codes.device)
+    if swiglu and amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=a.codes.device)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    st = status if status is not None else new_status(a.codes.device)
+    ca, cw = a.c(), w.c()
+    car = a_res.c() if Kp > 0 else None
+    cws = w_sel.c() if Kp > 0 else None
+    _check(lib.grouped_w4a4_rac_moe(ctypes.byref(ca), ctypes.byref(car) if car else None, expert_offsets.data_ptr(),
+                                    E, ctypes.byref(cw), ctypes.byref(cws) if cws else None, N, K, Kp,
+                                    EPI_SWIGLU_AMAX if swiglu else EPI_NONE, od, y.data_ptr(), y.stride(0),
+                                    _ptr(amax_out), st.data_ptr(), _stream(stream)))
+    return (y, amax_out) if swiglu else y
+
+
+def weight_qdq(w: torch.Tensor, out: torch.Tensor | None = None, s_g: torch.Tensor | None = None,
+               status: torch.Tensor | None = None, stream=None):
+    """Trainer fake-quant bf16(DQ(Q(w))) per tensor; w is [n_tensors, elems] (or one tensor of any shape)."""
+    lib = load()
+    _u16(w)
+    assert w.is_contiguous()
+    n = w.shape[0] if w.dim() >= 2 else 1
+    elems = w.numel() // n
+    if out is None:
+        out = torch.empty_like(w)
+    if s_g is None:
+        s_g = torch.empty(n, dtype=torch.float32, device=w.device)
+    ws = _workspace(w.device).get(lib.weight_qdq_workspace_size(n, elems))
+    st = status if status is not None else new_status(w.device)
+    _check(lib.weight_qdq(w.data_ptr(), n, elems, out.data_ptr(), s_g.data_ptr(), ws.data_ptr(), ws.numel(),
+                          st.data_ptr(), _stream(stream)))
+    return out, s_g
+
+
+def encode_e2m1(v: torch.Tensor, stream=None) -> torch.Tensor:
+    out = torch.empty(v.numel(), dtype=torch.uint8, device=v.device)
+    _check(load().nvfp4_encode_e2m1(v.data_ptr(), v.numel(), out.data_ptr(), _stream(stream)))
+    return out
+
+
+def encode_e4m3(v: torch.Tensor, stream=None) -> torch.Tensor:
+    out = torch.empty(v.numel(), dtype=torch.uint8, device=v.device)
+    _check(load().nvfp4_encode_e4m3(v.data_ptr(), v.numel(), out.data_ptr(), _stream(stream)))
+    return out
+
+
+def selftest_wait_timeout(limit_ns: int, status: torch.Tensor, stream=None):
+    _check(load().nvfp4_selftest_wait_timeout(limit_ns, status.data_ptr(), _stream(stream)))
+
+
+# ------------------------------------------------------------------------------------- MoE host logic
+def expert_layout(counts, pad: int = 128):
+    """Padded expert segments for a token-sorted pair list.
+
+    counts: pairs per expert.  Returns (offsets_padded [E+1] int64, rows_padded_total, pair_rows [P]) where
+    pair_rows maps the i-th (expert, token)-sorted pair to its row in the padded layout.
+    """
+    import numpy as np
+
+    counts = np.asarray(counts, dtype=np.int64)
+    padded = (counts + pad - 1) // pad * pad
+    off = np.zeros(counts.size + 1, dtype=np.int64)
+    off[1:] = np.cumsum(padded)
+    starts = off[:-1]
+    pair_rows = np.concatenate([starts[e] + np.arange(c) for e, c in enumerate(counts)]) if counts.sum() else \
+        np.zeros(0, np.int64)
+    return off, int(off[-1]), pair_rows
+
+
+def gather_map(pair_token, counts, pad: int = 128):
+    """row_gather [rows_padded] (source token of each padded row, -1 for padding) and offsets."""
+    import numpy as np
+
+    off, total, pair_rows = expert_layout(counts, pad)
+    g = np.full(total, -1, dtype=np.int32)
+    g[pair_rows] = np.asarray(pair_token, dtype=np.int32)
+    return g, off, pair_rows

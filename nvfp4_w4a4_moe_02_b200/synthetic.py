@@ -13,7 +13,7 @@ stated benchmark configurations, written out below.
 
 Streams: 1 = activations X, 2 = weights W (gate_up), 3 = calibration batch,
 4 = outlier-channel choice, 5 = per-channel lognormal scales, 6 = router
-logits, 7 = down-projection weights.
+logits, 7 = down-projection weights, 8 = router logits of the calibration batch.
 """
 from __future__ import annotations
 
@@ -30,6 +30,7 @@ _LIB = os.path.join(_HERE, "libsynth.so")
 _lib = None
 
 STREAM_X, STREAM_W, STREAM_XCAL, STREAM_OUTLIER, STREAM_CHANSCALE, STREAM_ROUTER, STREAM_WDOWN = 1, 2, 3, 4, 5, 6, 7
+STREAM_ROUTER_CAL = 8
 
 
 def build_lib(force: bool = False) -> str:
@@ -122,14 +123,14 @@ def lognormal_colscale(seed: int, K: int) -> np.ndarray:
     return np.exp(normal_f64(seed, STREAM_CHANSCALE, K))
 
 
-def route_topk(seed: int, T: int, E: int, topk: int) -> np.ndarray:
+def route_topk(seed: int, T: int, E: int, topk: int, stream: int = STREAM_ROUTER) -> np.ndarray:
     """Top-k experts per token from N(0,1) router logits (stream 6).
 
     Softmax is monotone, so the top-k of the softmax equals the top-k of the
     logits; ties go to the lower expert index (stable sort).  Returns [T, topk]
     int64, best expert first.
     """
-    logits = normal_f64(seed, STREAM_ROUTER, T * E).reshape(T, E)
+    logits = normal_f64(seed, stream, T * E).reshape(T, E)
     order = np.argsort(-logits, axis=1, kind="stable")
     return order[:, :topk].astype(np.int64)
 
@@ -257,3 +258,36 @@ def moe_prefill(seed: int = 0, r: float = 0.5, materialize_weights: bool = True)
 def moe_decode(seed: int = 0, r: float = 0.5) -> MoEWorkload:
     """64 tokens, hidden 7168, 256 experts, top-8, intermediate 2048; weights generated per expert on demand."""
     return moe_block(seed, r, T=64, H=7168, E=256, topk=8, I=2048, materialize_weights=False)
+
+
+def moe_down_calibration_batch(wl: MoEWorkload, max_pairs: int | None = None) -> np.ndarray:
+    """Input of the down projection on the calibration batch, in full precision.
+
+    The calibration tokens are routed with their own N(0,1) logits (stream 8); for every
+    (token, expert) pair the gate_up product is formed in binary64 from the bf16 weights,
+    followed by silu(g) * u, rounded to bf16.  Rows are pooled over all pairs in
+    (expert, token) order.  Returns bf16 bits [pairs, I].
+    """
+    T = wl.x_cal.shape[0]
+    k = wl.topk_ids.shape[1]
+    topk = route_topk(wl.seed, T, wl.E, k, stream=STREAM_ROUTER_CAL)
+    pt, pe, counts = sort_pairs(topk, wl.E)
+    if max_pairs is not None:
+        pt, pe = pt[:max_pairs], pe[:max_pairs]
+    xf = bf16_to_f32(wl.x_cal).astype(np.float64)
+    out = np.empty((pt.size, wl.I), dtype=np.uint16)
+    for e in np.unique(pe):
+        idx = np.nonzero(pe == e)[0]
+        wgu = bf16_to_f32(wl.gate_up_expert(int(e))).astype(np.float64)
+        gu = xf[pt[idx]] @ wgu.T
+        g, u = gu[:, :wl.I], gu[:, wl.I:]
+        h = (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
+        out[idx] = _f32_to_bf16_bits(h)
+    return out
+
+
+def _f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """float32 -> bf16 bits, round to nearest even (storage conversion)."""
+    u = np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+    lsb = (u >> 16) & 1
+    return ((u + 0x7FFF + lsb) >> 16).astype(np.uint16)

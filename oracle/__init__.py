@@ -61,6 +61,7 @@ def _get():
         "orc_swiglu": ([vp, i64, i64, vp, vp], None),
         "orc_e2m1_encode_array": ([vp, i64, vp], None),
         "orc_e4m3_encode_array": ([vp, i64, vp], None),
+        "orc_f64_to_bf16_array": ([vp, i64, vp], None),
         "orc_num_threads": ([], ctypes.c_int),
     }
     for name, (args, res) in sigs.items():
@@ -116,6 +117,13 @@ def e4m3_encode_array(v: np.ndarray) -> np.ndarray:
 
 def f64_to_bf16(d: float) -> int:
     return int(_get().orc_f64_to_bf16(float(d)))
+
+
+def f64_to_bf16_array(v: np.ndarray) -> np.ndarray:
+    v = _c(v, np.float64)
+    out = np.empty(v.shape, dtype=np.uint16)
+    _get().orc_f64_to_bf16_array(_p(v), v.size, _p(out))
+    return out
 
 
 def bf16_to_f32(b: int) -> float:

@@ -1,0 +1,109 @@
+"""CPU checks of the boundary: the C library loads, exports every declared entry point, and
+rejects bad arguments on the host before touching a device.  Also pins the test-side layout
+decoder against the storage definition written in the header."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "nvfp4rac.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from nvfp4_w4a4_moe_02_b200 import build_lib, nvfp4rac
+
+    build_lib.build()
+    return nvfp4rac.load()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+([A-Za-z_][A-Za-z0-9_]*)\s*\(", text, re.M)
+    return sorted(set(n for n in names if n not in ("if", "return")))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for n in ("nvfp4_quantize", "rac_calibrate", "pack_weights", "w4a4_rac_gemm", "grouped_w4a4_rac_moe",
+              "weight_qdq"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_status_strings_and_sizes(lib):
+    assert lib.nvfp4_version() >= 100
+    assert lib.nvfp4_status_string(0) == b"ok"
+    assert lib.nvfp4_status_string(6) == b"device wait timed out"
+    assert lib.nvfp4_codes_bytes(128, 256) == 128 * 128
+    assert lib.nvfp4_sf_bytes(128, 256) == 128 * 16
+    assert lib.nvfp4_kp_from_ratio(4096, 0.5) == 2048
+    assert lib.nvfp4_kp_from_ratio(768, 0.5) == 384
+    assert lib.nvfp4_kp_from_ratio(768, 0.25) == 192
+    assert lib.nvfp4_kp_from_ratio(256, 0.0) == 0
+    assert lib.nvfp4_kp_from_ratio(256, 1.0) == 256
+
+
+def test_host_side_rejections(lib):
+    from nvfp4_w4a4_moe_02_b200.nvfp4rac import CTensor
+
+    t = CTensor(16, 16, 16, 1, 64, 128, 100)  # fake non-null pointers, never dereferenced
+    # K not a multiple of 64
+    st = lib.nvfp4_quantize(16, 64, 100, 104, None, 64, None, 0, None, ctypes.byref(t), None, 16, 1024, None, None)
+    assert st == 2 and b"K" in lib.nvfp4_last_error_string()
+    # misaligned x
+    t.cols = 128
+    st = lib.nvfp4_quantize(18, 64, 128, 128, None, 64, None, 0, None, ctypes.byref(t), None, 16, 1024, None, None)
+    assert st == 3
+    # Kp not a multiple of 64
+    st = lib.nvfp4_quantize(16, 64, 128, 128, None, 64, 16, 32, None, ctypes.byref(t), ctypes.byref(t), 16, 1024,
+                            None, None)
+    assert st == 2
+    # rows_padded not a multiple of 128
+    t2 = CTensor(16, 16, 16, 1, 64, 100, 128)
+    st = lib.nvfp4_quantize(16, 64, 128, 128, None, 64, None, 0, None, ctypes.byref(t2), None, 16, 1024, None, None)
+    assert st == 2
+    # GEMM: N not a multiple of 128
+    a = CTensor(16, 16, 16, 1, 64, 128, 128)
+    w = CTensor(16, 16, 16, 1, 96, 96, 128)
+    st = lib.w4a4_rac_gemm(ctypes.byref(a), None, ctypes.byref(w), None, 64, 96, 128, 0, 0, 16, 96, None, None)
+    assert st == 2
+    # grouped: SwiGLU needs bf16 output
+    st = lib.grouped_w4a4_rac_moe(ctypes.byref(a), None, 16, 1, ctypes.byref(w), None, 128, 128, 0, 1, 0, 16, 64,
+                                  16, None, None)
+    assert st == 1
+    # weight_qdq: elems not a multiple of 16
+    st = lib.weight_qdq(16, 1, 100, 16, None, 16, 1 << 20, None, None)
+    assert st == 2
+    # calibration: Kp > K
+    st = lib.rac_calibrate(16, 64, 128, 256, 16, None, 16, 1 << 30, None, None)
+    assert st == 2
+    # null status pointer is rejected by the self-test entry
+    assert lib.nvfp4_selftest_wait_timeout(1000, None, None) == 1
+
+
+def test_layout_decoder_matches_storage_definition():
+    from nvfp4_layout import pack_codes, pack_sf, unpack_codes, unpack_sf
+
+    rng = np.random.default_rng(0)
+    rows_p, cols = 256, 192
+    S = rng.integers(0, 0x7F, (rows_p, cols // 16), dtype=np.uint8)
+    flat = pack_sf(S, rows_p)
+    # spot values written straight from the header formula
+    for r, c in [(0, 0), (1, 0), (31, 3), (32, 0), (127, 11), (128, 5), (255, 11), (77, 6)]:
+        atom = (r // 128) * (cols // 64) + c // 4
+        off = atom * 512 + (r % 128 % 32) * 16 + (r % 128 // 32) * 4 + c % 4
+        assert flat[off] == S[r, c]
+    assert np.array_equal(unpack_sf(flat, rows_p, rows_p, cols), S)
+    C = rng.integers(0, 16, (rows_p, cols), dtype=np.uint8)
+    b = pack_codes(C)
+    assert b[0] == C[0, 0] | (C[0, 1] << 4)
+    assert np.array_equal(unpack_codes(b, rows_p, rows_p, cols), C)

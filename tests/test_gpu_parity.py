@@ -1,0 +1,420 @@
+"""Parity of the CUDA path (through the C ABI) with the CPU oracle, on a B200.
+
+Bit-exact: E2M1/E4M3 codes, block scales, per-tensor scales, channel selections,
+fake-quantised weights.  GEMM outputs: |y - y_ref| <= 1e-3 * sum_k |a_k b_k| + 1e-6 per
+element (plus one bf16 ulp of y_ref in bf16-output mode), y_ref being the exact product of
+the identical quantised operands.
+"""
+import numpy as np
+import pytest
+import torch
+
+from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+from nvfp4_layout import unpack_codes, unpack_sf
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def dev():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    R.load()
+    return torch.device("cuda:0")
+
+
+def to_dev(a: np.ndarray, dev) -> torch.Tensor:
+    return torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def bf16_bits(t: torch.Tensor) -> np.ndarray:
+    return t.view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def logical(p: R.Packed, slab: int = 0, rows: int | None = None):
+    rows = p.rows if rows is None else rows
+    cb = p.rows_padded * p.cols // 2
+    sb = p.rows_padded * p.cols // 16
+    codes = p.codes[slab * cb:(slab + 1) * cb].cpu().numpy()
+    sf = p.sf[slab * sb:(slab + 1) * sb].cpu().numpy()
+    return unpack_codes(codes, rows, p.rows_padded, p.cols), unpack_sf(sf, rows, p.rows_padded, p.cols)
+
+
+def f32(v):
+    return np.float32(v)
+
+
+def bf16_ulp(y: np.ndarray) -> np.ndarray:
+    a = np.abs(y).astype(np.float64)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def assert_gemm_close(y_gpu: np.ndarray, y_ref: np.ndarray, absdot: np.ndarray, bf16_out: bool):
+    tol = 1e-3 * absdot + 1e-6
+    if bf16_out:
+        tol = tol + bf16_ulp(y_ref)
+    err = np.abs(y_gpu.astype(np.float64) - y_ref)
+    bad = np.argwhere(err > tol)
+    assert bad.size == 0, (f"{len(bad)} of {err.size} outside tolerance; first {bad[:5].tolist()} "
+                           f"gpu {y_gpu[tuple(bad[0])]} ref {y_ref[tuple(bad[0])]} tol {tol[tuple(bad[0])]}")
+
+
+# ------------------------------------------------------------------------------------------ codecs
+def test_codec_e2m1_matches_oracle(dev, orc):
+    rng = np.random.default_rng(0)
+    pts = [np.float32(0.0), np.float32(-0.0)]
+    for g in [0, .25, .5, .75, 1, 1.25, 1.5, 1.75, 2, 2.5, 3, 3.5, 4, 5, 6, 7, 8, 1e4]:
+        v = np.float32(g)
+        for _ in range(6):
+            pts += [v, -v]
+            v = np.nextafter(v, np.float32(np.inf))
+        v = np.float32(g)
+        for _ in range(6):
+            pts += [v, -v]
+            v = np.nextafter(v, np.float32(-np.inf))
+    arr = np.concatenate([np.array(pts, np.float32), rng.uniform(-9, 9, 1 << 20).astype(np.float32),
+                          (rng.standard_normal(1 << 16) * 1e-20).astype(np.float32)])
+    got = R.encode_e2m1(torch.from_numpy(arr).to(dev)).cpu().numpy()
+    ref = orc.e2m1_encode_array(arr)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(arr[i]), int(got[i]), int(ref[i])) for i in bad[:8]]
+
+
+def test_codec_e4m3_matches_oracle(dev, orc):
+    rng = np.random.default_rng(1)
+    vals = [orc.e4m3_decode(c) for c in range(0x7F)]
+    pts = []
+    for a, b in zip(vals, vals[1:]):
+        m = np.float32((a + b) / 2)
+        for d in (-2, -1, 0, 1, 2):
+            v = m
+            for _ in range(abs(d)):
+                v = np.nextafter(v, np.float32(np.inf if d > 0 else -np.inf))
+            pts.append(v)
+        pts.append(np.float32(b))
+    arr = np.concatenate([np.array(pts, np.float32), rng.uniform(0, 500, 1 << 20).astype(np.float32),
+                          np.exp(rng.uniform(-14, 7, 1 << 18)).astype(np.float32)])
+    got = R.encode_e4m3(torch.from_numpy(arr).to(dev)).cpu().numpy()
+    ref = orc.e4m3_encode_array(arr)
+    bad = np.nonzero(got != ref)[0]
+    assert bad.size == 0, [(float(arr[i]), int(got[i]), int(ref[i])) for i in bad[:8]]
+
+
+# ------------------------------------------------------------------------------------------ quantiser
+def check_act_quant(dev, orc, x: np.ndarray, sel: np.ndarray, rows_padded=None):
+    xd = to_dev(x, dev)
+    seld = torch.from_numpy(sel.astype(np.int32)).to(dev) if sel.size else None
+    st = R.new_status(dev)
+    q, qr = R.nvfp4_quantize(xd, seld, rows_padded=rows_padded, status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    s_ref = orc.global_scale(orc.amax_bf16(x))
+    assert q.s_g.item() == float(s_ref)
+    codes, S, rcodes, rS, _ = orc.act_quant_rac(x, s_ref, sel.astype(np.int32))
+    gc, gS = logical(q)
+    assert np.array_equal(gS, S), np.argwhere(gS != S)[:5]
+    assert np.array_equal(gc, codes), np.argwhere(gc != codes)[:5]
+    # padded rows are zero
+    full_c, full_s = logical(q, rows=q.rows_padded)
+    assert not full_c[x.shape[0]:].any() and not full_s[x.shape[0]:].any()
+    if sel.size:
+        assert qr.s_g.item() == float(s_ref)
+        grc, grS = logical(qr)
+        assert np.array_equal(grS, rS), np.argwhere(grS != rS)[:5]
+        assert np.array_equal(grc, rcodes), np.argwhere(grc != rcodes)[:5]
+    return q, qr
+
+
+def test_quantize_tiny(dev, orc):
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    check_act_quant(dev, orc, wl.x, sel)
+
+
+def test_quantize_ragged_rows_and_tail(dev, orc):
+    rng = np.random.default_rng(2)
+    M, K = 200, 704  # 704 = 512 + 192: a ragged last iteration; 200 rows: a partial row block
+    x = syn.normal_bf16(3, 1, M, K, 1.0, np.exp(rng.standard_normal(K)))
+    x[5] = 0  # an all-zero row
+    sel = np.sort(rng.choice(K, 192, replace=False)).astype(np.int32)
+    check_act_quant(dev, orc, x, sel)
+    check_act_quant(dev, orc, x, np.zeros(0, np.int32), rows_padded=384)
+
+
+def test_quantize_zero_tensor(dev, orc):
+    x = np.zeros((64, 128), np.uint16)
+    q, qr = check_act_quant(dev, orc, x, np.arange(0, 128, 2, dtype=np.int32))
+    assert q.s_g.item() == 0.0
+
+
+def test_quantize_dense_prefill_full(dev, orc):
+    wl = syn.dense_prefill()
+    sel, _ = orc.calibrate(wl.x_cal[:256], wl.Kp)  # any ascending set of the right size
+    check_act_quant(dev, orc, wl.x, sel)
+
+
+def test_quantize_row_gather(dev, orc):
+    wl = syn.moe_block(T=300, H=1024, E=16, topk=4, I=256, T_cal=64, materialize_weights=False)
+    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    xd = to_dev(wl.x, dev)
+    sel = np.arange(1, 1024, 2, dtype=np.int32)
+    gd = torch.from_numpy(g).to(dev)
+    q, qr = R.nvfp4_quantize(xd, torch.from_numpy(sel).to(dev), row_gather=gd, M_out=g.size)
+    torch.cuda.synchronize()
+    s_ref = orc.global_scale(orc.amax_bf16(wl.x))
+    rows_x = np.where(g >= 0, g, 0)
+    xg = wl.x[rows_x].copy()
+    xg[g < 0] = 0
+    codes, S, rcodes, rS, _ = orc.act_quant_rac(xg, s_ref, sel)
+    gc, gS = logical(q)
+    grc, grS = logical(qr)
+    assert np.array_equal(gc, codes) and np.array_equal(gS, S)
+    assert np.array_equal(grc, rcodes) and np.array_equal(grS, rS)
+
+
+# ------------------------------------------------------------------------------------------ calibration
+@pytest.mark.parametrize("shape", [(64, 256, 128), (2048, 4096, 2048), (100, 704, 320)])
+def test_calibrate_matches_oracle(dev, orc, shape):
+    T, K, Kp = shape
+    rng = np.random.default_rng(T)
+    x = syn.normal_bf16(5, 3, T, K, 1.0, np.exp(rng.standard_normal(K)))
+    sel_ref, err_ref = orc.calibrate(x, Kp)
+    sel, err = R.rac_calibrate(to_dev(x, dev), Kp, want_err=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(err.cpu().numpy(), err_ref)
+    assert np.array_equal(sel.cpu().numpy(), sel_ref)
+
+
+def test_calibrate_full_ratio_selects_all(dev):
+    x = syn.normal_bf16(1, 3, 32, 256, 1.0)
+    sel, _ = R.rac_calibrate(to_dev(x, dev), 256)
+    assert np.array_equal(sel.cpu().numpy(), np.arange(256))
+
+
+# ------------------------------------------------------------------------------------------ weights
+@pytest.mark.parametrize("interleave", [False, True])
+def test_pack_weights_matches_oracle(dev, orc, interleave):
+    E, N, K, Kp = 3, 256, 512, 256
+    w = syn.normal_bf16(0, 2, E * N, K, 0.02).reshape(E, N, K)
+    w[1] *= 0  # an all-zero expert: s_g = 0
+    sel = np.sort(np.random.default_rng(9).choice(K, Kp, replace=False)).astype(np.int32)
+    wq, wsq = R.pack_weights(to_dev(w, dev), torch.from_numpy(sel).to(dev), gate_up_interleave=interleave)
+    torch.cuda.synchronize()
+    for e in range(E):
+        s_ref = orc.global_scale(orc.amax_bf16(w[e]))
+        assert wq.s_g[e].item() == float(s_ref) and wsq.s_g[e].item() == float(s_ref)
+        we = w[e]
+        if interleave:
+            p = np.arange(N)
+            q, j = p // 128, p % 128
+            src = np.where(j < 64, q * 64 + j, N // 2 + q * 64 + j - 64)
+            we = we[src]
+        c, S, sc, sS = orc.weight_pack(we, s_ref, sel)
+        gc, gS = logical(wq, e)
+        gsc, gsS = logical(wsq, e)
+        assert np.array_equal(gc, c) and np.array_equal(gS, S)
+        assert np.array_equal(gsc, sc) and np.array_equal(gsS, sS)
+
+
+def test_weight_qdq_matches_oracle(dev, orc):
+    n, elems = 5, 4096 + 16 * 3
+    w = syn.normal_bf16(0, 9, n, elems, 0.02)
+    w[2, :100] *= 64
+    out, s_g = R.weight_qdq(to_dev(w, dev))
+    torch.cuda.synchronize()
+    got = bf16_bits(out).reshape(n, elems)
+    for t in range(n):
+        ref, s_ref = orc.weight_qdq(w[t])
+        assert s_g[t].item() == float(s_ref)
+        assert np.array_equal(got[t], ref), np.argwhere(got[t] != ref)[:5]
+
+
+def test_shared_weight_path_gpu(dev):
+    """DQ(pack_weights(W)) == weight_qdq(W), bitwise, both computed on the GPU."""
+    N, K = 256, 1024
+    w = syn.normal_bf16(4, 2, N, K, 0.02)
+    wd = to_dev(w, dev)
+    wq, _ = R.pack_weights(wd)
+    fq, s_g = R.weight_qdq(wd.reshape(1, -1))
+    torch.cuda.synchronize()
+    c, S = logical(wq)
+    mag = np.array([0, .5, 1, 1.5, 2, 3, 4, 6], np.float32)
+    e = mag[c & 7] * np.where(c & 8, np.float32(-1), np.float32(1))
+    from oracle import e4m3_decode  # decode table only
+
+    table = np.array([e4m3_decode(i) if i != 0x7F else np.nan for i in range(128)], np.float32)
+    d = (table[S] * np.float32(wq.s_g[0].item())).astype(np.float32)
+    dq = (e * np.repeat(d, 16, axis=1)).astype(np.float32)
+    ref = torch.from_numpy(dq).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(bf16_bits(fq).reshape(N, K), ref)
+
+
+# ------------------------------------------------------------------------------------------ GEMM
+def run_dense(dev, orc, x, w, x_cal, Kp, out_dtype, rows=None):
+    sel_np, _ = orc.calibrate(x_cal, Kp)
+    sel_gpu, _ = R.rac_calibrate(to_dev(x_cal, dev), Kp)
+    assert np.array_equal(sel_gpu.cpu().numpy(), sel_np)
+    xd, wd = to_dev(x, dev), to_dev(w, dev)
+    st = R.new_status(dev)
+    q, qr = R.nvfp4_quantize(xd, sel_gpu if Kp else None, status=st)
+    wq, wsq = R.pack_weights(wd, sel_gpu if Kp else None, status=st)
+    y = R.w4a4_rac_gemm(q, qr, wq, wsq, x.shape[0], out_dtype=out_dtype, status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    f = orc.dense_rac_forward(x, w, sel_np if Kp else np.zeros(0, np.int32), rows=rows)
+    yg = y.float().cpu().numpy()
+    if rows is not None:
+        yg = yg[rows]
+    assert_gemm_close(yg, f["y"], f["absdot"], out_dtype == torch.bfloat16)
+    return y, f
+
+
+def test_gemm_tiny_fp32(dev, orc):
+    wl = syn.dense_tiny()
+    run_dense(dev, orc, wl.x, wl.w, wl.x_cal, wl.Kp, torch.float32)
+
+
+def test_gemm_tiny_r0_is_plain_w4a4(dev, orc):
+    wl = syn.dense_tiny()
+    run_dense(dev, orc, wl.x, wl.w, wl.x_cal, 0, torch.float32)
+
+
+@pytest.mark.parametrize("M,N,K,Kp", [(300, 384, 768, 384), (128, 256, 320, 64), (520, 512, 1024, 1024)])
+def test_gemm_ragged_shapes(dev, orc, M, N, K, Kp):
+    rng = np.random.default_rng(M + N)
+    cs = np.exp(rng.standard_normal(K))
+    x = syn.normal_bf16(11, 1, M, K, 1.0, cs)
+    w = syn.normal_bf16(11, 2, N, K, 0.02)
+    x_cal = syn.normal_bf16(11, 3, 128, K, 1.0, cs)
+    run_dense(dev, orc, x, w, x_cal, Kp, torch.float32)
+    run_dense(dev, orc, x, w, x_cal, Kp, torch.bfloat16)
+
+
+def test_gemm_dense_prefill_sampled(dev, orc):
+    wl = syn.dense_prefill()
+    rows = np.array([0, 1, 127, 128, 1000, 4095, 4096, 6000, 8190, 8191])
+    run_dense(dev, orc, wl.x, wl.w, wl.x_cal, wl.Kp, torch.bfloat16, rows=rows)
+
+
+# ------------------------------------------------------------------------------------------ MoE
+def moe_pipeline(dev, wl, sel_gu, sel_dn):
+    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    st = R.new_status(dev)
+    offd = torch.from_numpy(off.astype(np.int32)).to(dev)
+    wgu = to_dev(wl.wgu, dev)
+    wdn = to_dev(wl.wdn, dev)
+    seld_gu = torch.from_numpy(sel_gu).to(dev)
+    seld_dn = torch.from_numpy(sel_dn).to(dev)
+    pgu, pgus = R.pack_weights(wgu, seld_gu, gate_up_interleave=True, status=st)
+    pdn, pdns = R.pack_weights(wdn, seld_dn, status=st)
+    a, ar = R.nvfp4_quantize(to_dev(wl.x, dev), seld_gu, row_gather=torch.from_numpy(g).to(dev), M_out=g.size,
+                             status=st)
+    h, amax_h = R.grouped_w4a4_rac_moe(a, ar, offd, pgu, pgus, swiglu=True, status=st)
+    hq, hqr = R.nvfp4_quantize(h, seld_dn, amax_in=amax_h, status=st)
+    y = R.grouped_w4a4_rac_moe(hq, hqr, offd, pdn, pdns, status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    return dict(g=g, off=off, pair_rows=pair_rows, a=a, ar=ar, h=h, amax_h=amax_h, hq=hq, hqr=hqr, y=y, pgu=pgu,
+                pdn=pdn)
+
+
+def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs):
+    I, H = wl.I, wl.H
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    assert out["a"].s_g.item() == float(s_x)
+    h_gpu = bf16_bits(out["h"])
+    # amax of the SwiGLU output over the real rows equals the device amax; padding rows are 0
+    valid = np.zeros(h_gpu.shape[0], bool)
+    valid[out["pair_rows"]] = True
+    assert not h_gpu[~valid].any()
+    hv = syn.bf16_to_f32(h_gpu[valid])
+    assert np.float32(np.abs(hv).max()) == np.float32(out["amax_h"].item())
+    s_h = orc.global_scale(np.float32(out["amax_h"].item()))
+    assert out["hq"].s_g.item() == float(s_h)
+    gq_c, gq_S = logical(out["hq"], rows=out["hq"].rows_padded)
+    gqr_c, gqr_S = logical(out["hqr"], rows=out["hqr"].rows_padded)
+    for e in sorted(set(int(wl.pair_expert[i]) for i in sample_pairs)):
+        pidx = [i for i in sample_pairs if wl.pair_expert[i] == e]
+        rows = out["pair_rows"][pidx]
+        toks = wl.pair_token[pidx]
+        # gate_up on the oracle: quantise the token rows, exact GEMM against the expert's weights
+        xa = wl.x[toks]
+        a_c, a_S, r_c, r_S, _ = orc.act_quant_rac(xa, s_x, sel_gu)
+        wgu = wl.wgu[e]
+        s_w = orc.global_scale(orc.amax_bf16(wgu))
+        wc, wS, wsc, wsS = orc.weight_pack(wgu, s_w, sel_gu)
+        gu, ad = orc.gemm_rac(a_c, a_S, r_c, r_S, wc, wS, wsc, wsS, s_x, s_w)
+        # bound on h from the GEMM bound on g and u
+        tol_gu = 1e-3 * ad + 1e-6 + bf16_ulp(gu)
+        g, u = gu[:, :I], gu[:, I:]
+        tg, tu = tol_gu[:, :I], tol_gu[:, I:]
+        sig = 1.0 / (1.0 + np.exp(-g))
+        silu = g * sig
+        dsilu = np.abs(sig * (1 + g * (1 - sig))) + 0.1
+        h_ref = silu * u
+        tol_h = 2.0 * (dsilu * tg * (np.abs(u) + tu) + np.abs(silu) * tu) + 2 * bf16_ulp(h_ref) + 1e-30
+        h_g = syn.bf16_to_f32(h_gpu[rows]).astype(np.float64)
+        bad = np.argwhere(np.abs(h_g - h_ref) > tol_h)
+        assert bad.size == 0, (e, bad[:5], h_g[tuple(bad[0])], h_ref[tuple(bad[0])])
+        # down: the GPU's h rows quantised by the oracle must match the GPU codes bit for bit
+        hrows = h_gpu[rows]
+        hc, hS, hrc, hrS, _ = orc.act_quant_rac(hrows, s_h, sel_dn)
+        assert np.array_equal(gq_c[rows], hc) and np.array_equal(gq_S[rows], hS)
+        assert np.array_equal(gqr_c[rows], hrc) and np.array_equal(gqr_S[rows], hrS)
+        wdn = wl.wdn[e]
+        s_wd = orc.global_scale(orc.amax_bf16(wdn))
+        dc, dS, dsc, dsS = orc.weight_pack(wdn, s_wd, sel_dn)
+        y_ref, ad2 = orc.gemm_rac(hc, hS, hrc, hrS, dc, dS, dsc, dsS, s_h, s_wd)
+        y_g = out["y"][torch.from_numpy(rows).to(out["y"].device)].float().cpu().numpy()
+        assert_gemm_close(y_g, y_ref, ad2, True)
+
+
+def test_moe_small_ragged(dev, orc):
+    """Small MoE block with empty, single-row and >128-row experts."""
+    wl = syn.moe_block(T=96, H=512, E=8, topk=2, I=128, T_cal=64)
+    # force a skewed routing: expert 7 gets nothing, expert 0 gets most tokens
+    wl.topk_ids[:, 0] = np.where(np.arange(96) % 3 == 0, 0, wl.topk_ids[:, 0])
+    wl.topk_ids[wl.topk_ids == 7] = 6
+    wl.topk_ids[:, 1] = np.where(wl.topk_ids[:, 1] == wl.topk_ids[:, 0], (wl.topk_ids[:, 0] + 1) % 7,
+                                 wl.topk_ids[:, 1])
+    wl.pair_token, wl.pair_expert, wl.counts = syn.sort_pairs(wl.topk_ids, wl.E)
+    assert wl.counts[7] == 0
+    sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
+    h_cal = syn.moe_down_calibration_batch(wl)
+    sel_dn, _ = orc.calibrate(h_cal, wl.Kp_dn)
+    out = moe_pipeline(dev, wl, sel_gu, sel_dn)
+    check_moe(orc, wl, sel_gu, sel_dn, out, list(range(wl.pair_token.size)))
+
+
+def test_moe_prefill_full_sampled(dev, orc):
+    wl = syn.moe_prefill()
+    sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
+    h_cal = syn.moe_down_calibration_batch(wl)
+    sel_dn, _ = orc.calibrate(h_cal, wl.Kp_dn)
+    out = moe_pipeline(dev, wl, sel_gu, sel_dn)
+    rng = np.random.default_rng(0)
+    P = wl.pair_token.size
+    sample = sorted(set(rng.choice(P, 96, replace=False).tolist() + [0, P - 1]))
+    check_moe(orc, wl, sel_gu, sel_dn, out, sample)
+
+
+# ------------------------------------------------------------------------------------------ failure path
+def test_bounded_wait_reports_timeout(dev):
+    st = R.new_status(dev)
+    R.selftest_wait_timeout(1_000_000, st)  # 1 ms on a barrier nothing completes
+    torch.cuda.synchronize()
+    assert int(st.item()) == 6
+    # the context is still usable
+    x = torch.ones(4, device=dev)
+    assert float(x.sum().item()) == 4.0
+
+
+def test_range_error_reported(dev):
+    x = np.zeros((16, 64), np.uint16)
+    x[3, 5] = 0x7F80  # +inf
+    st = R.new_status(dev)
+    R.nvfp4_quantize(to_dev(x, dev), status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 4
