@@ -199,6 +199,28 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_
                         void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* weight_qdq_noalloc -- weight_qdq for callers that cannot allocate device memory.          */
+/* The paper has no counterpart: this is a library convenience.  Some callers of the         */
+/* trainer-side fake-quant cannot call cudaMalloc: a training framework that owns all device */
+/* memory through its own caching allocator (a raw cudaMalloc outside it fragments the pool  */
+/* and can fail under memory pressure), a latency-bound loop that must not take the implicit  */
+/* device synchronisation cudaMalloc/cudaFree may cause, or a plain C host program that links */
+/* only this library and has no allocator plumbing.  This entry point needs no workspace: its */
+/* amax scratch is a fixed 16 KiB array inside the library, resident on every GPU that loads  */
+/* the library until the process exits.                                                      */
+/*   Arguments, layout and results are those of weight_qdq (bitwise the same output).        */
+/*   Limit: n_tensors * max(1, 512 / n_tensors) <= 4096 scratch floats, i.e. at most 4096     */
+/*   tensors per call; larger calls return NVFP4_ERR_UNSUPPORTED_SHAPE with a message.        */
+/*   The first call on a device looks up the scratch array's device address (once per        */
+/*   device, with that device current); make that first call before any stream capture.      */
+/*   All calls share the one array, so calls that overlap on the GPU (different streams, or  */
+/*   different host threads) race and may corrupt each other's scales: serialise them.        */
+/*   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.            */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status weight_qdq_noalloc(const uint16_t* w, int64_t n_tensors, int64_t elems_per_tensor, uint16_t* w_out,
+                                float* s_g_out, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* test helpers (not part of the hot path)                                                   */
 /* ---------------------------------------------------------------------------------------- */
 /* The device E2M1 / E4M3 encoders applied to float32 inputs (v device [n], out device [n],

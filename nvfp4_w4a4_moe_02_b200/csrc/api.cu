@@ -491,3 +491,10 @@ nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status,
 }
 
 }  // extern "C"
+
+// Helpers for entry points defined in other files of the library.
+namespace nvfp4 {
+nvfp4_status record_host_error(nvfp4_status s, const char* msg) { return fail(s, "%s", msg); }
+int qdq_partial_count(int64_t n_tensors) { return slab_partials(n_tensors); }
+int device_sm_count() { return num_sms(); }
+}  // namespace nvfp4
