@@ -129,6 +129,20 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
                             void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* nvfp4_quantize_scatter -- nvfp4_quantize for an MoE dispatch: each source row is quantised */
+/* once and its codes / scales are written to up to `fanout` output rows.                    */
+/*   row_scatter  int32 [M x fanout]: output rows of source row m (entries < 0 are skipped;  */
+/*                an entry >= q->rows_padded is an error reported in *dev_status).            */
+/*   Output rows that no entry names are left untouched: a caller that pads expert segments  */
+/*   zero-fills q / q_res once, and the padding stays zero across calls.                     */
+/*   Other arguments as nvfp4_quantize; s_g is computed over the M source rows.              */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
+                                    int32_t fanout, const int32_t* sel, int32_t Kp, const float* amax_in,
+                                    const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* rac_calibrate -- pick the Kp channels with the largest quantisation error                */
 /* (Two fixes: "the roughly top-50% of activation channels with the largest quantization    */
 /* error").  The calibration batch is quantised with its own s_g; e_k = sum_t r_{t,k}^2 in   */

@@ -208,6 +208,67 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   return NVFP4_OK;
 }
 
+nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
+                                    int32_t fanout, const int32_t* sel, int32_t Kp, const float* amax_in,
+                                    const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
+  if (!row_scatter && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "row_scatter is NULL");
+  if (M < 0 || fanout <= 0 || fanout > 64) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M >= 0 and 1 <= fanout <= 64 required");
+  if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64 <= %lld", (long long)K, (long long)kMaxK);
+  if (ldx < K || ldx % 8 != 0) return fail(NVFP4_ERR_ALIGNMENT, "ldx = %lld must be >= K and a multiple of 8", (long long)ldx);
+  if (x && !aligned16(x)) return fail(NVFP4_ERR_ALIGNMENT, "x must be 16-byte aligned");
+  if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp = %d must be a multiple of 64 in [0, K]", Kp);
+  nvfp4_status st = check_tensor(q, "q", K, 0, 1);
+  if (st != NVFP4_OK) return st;
+  if (Kp > 0) {
+    if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
+    st = check_tensor(q_res, "q_res", Kp, 0, 1);
+    if (st != NVFP4_OK) return st;
+    if (q_res->rows_padded != q->rows_padded) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res.rows_padded must equal q.rows_padded");
+  }
+  const int P = act_partials(M, K);
+  if (!amax_in) {
+    if (!workspace || workspace_bytes < nvfp4_quantize_workspace_size(M, K))
+      return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  }
+  if (M == 0) return NVFP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* partial = reinterpret_cast<float*>(workspace);
+  if (!amax_in) {
+    cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  }
+  RowArgs a;
+  memset(&a, 0, sizeof(a));
+  a.mode = kModeAct;
+  a.src = x;
+  a.src_rows = M;
+  a.ld = ldx;
+  a.K = K;
+  a.row_scatter = row_scatter;
+  a.fanout = fanout;
+  a.rows_out = q->rows_padded;
+  a.rows_per_slab = M;
+  a.sel = sel;
+  a.Kp = Kp;
+  a.partial = partial;
+  a.P = P;
+  a.amax_in = amax_in;
+  a.s_g_out = q->s_g;
+  a.s_g_out2 = Kp > 0 ? q_res->s_g : nullptr;
+  a.codes = q->codes;
+  a.sf = q->sf;
+  a.rcodes = Kp > 0 ? q_res->codes : nullptr;
+  a.rsf = Kp > 0 ? q_res->sf : nullptr;
+  a.status = dev_status;
+  cudaError_t e = launch_rows(a, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return NVFP4_OK;
+}
+
 // ------------------------------------------------------------------------------------------ calibrate
 size_t rac_calibrate_workspace_size(int64_t T, int64_t K) {
   return round_up(256 * sizeof(float), 256) + round_up((size_t)T * (size_t)K * sizeof(float), 256) +

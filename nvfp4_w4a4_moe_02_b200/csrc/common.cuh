@@ -52,21 +52,25 @@ __device__ __forceinline__ uint32_t e2m1_encode8(const float v[8]) {
   return out;
 }
 
-// E2M1 code -> value, exact, in integer arithmetic: index m = code & 7 is 0 -> 0, 1 -> 0.5,
-// m >= 2 -> (1 + (m & 1)/2) * 2^((m >> 1) - 1); bit 3 is the sign (code 8 is -0).
-// (The f16x2 <- e2m1x2 conversion instruction is not used: it does not produce these values
-// on sm_100.)
-__device__ __forceinline__ float e2m1_value(uint32_t q) {
-  const uint32_t m = q & 7u;
-  uint32_t bits = (m >= 2u) ? ((((m >> 1) + 126u) << 23) | ((m & 1u) << 22)) : (m == 1u ? 0x3F000000u : 0u);
-  bits |= (q & 8u) << 28;
-  return __uint_as_float(bits);
-}
-
-// Eight E2M1 codes (nibble i = element i) -> their values, exact.
+// Eight E2M1 codes (nibble i = element i) -> their values, exact.  The eight magnitudes
+// {0, .5, 1, 1.5, 2, 3, 4, 6} are exact bf16 numbers; their high and low bytes are looked up
+// with byte permutes (index = code & 7), the sign is code bit 3.  (The f16x2 <- e2m1x2
+// conversion instruction is not used: it does not return these values on sm_100.)
 __device__ __forceinline__ void e2m1_decode8(uint32_t codes, float out[8]) {
+  const uint32_t idx = codes & 0x77777777u;
+  const uint32_t hi_a = __byte_perm(0x3F3F3F00u, 0x40404040u, idx & 0xFFFFu);
+  const uint32_t hi_b = __byte_perm(0x3F3F3F00u, 0x40404040u, idx >> 16);
+  const uint32_t lo_a = __byte_perm(0xC0800000u, 0xC0804000u, idx & 0xFFFFu);
+  const uint32_t lo_b = __byte_perm(0xC0800000u, 0xC0804000u, idx >> 16);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) out[i] = e2m1_value(codes >> (4 * i));
+  for (int i = 0; i < 4; ++i) {
+    // bytes 2, 3 of the result = low, high byte of element i's bf16 value
+    const uint32_t sel = ((uint32_t)i << 8) | ((uint32_t)(4 + i) << 12);
+    const uint32_t va = __byte_perm(lo_a, hi_a, sel) & 0xFFFF0000u;
+    const uint32_t vb = __byte_perm(lo_b, hi_b, sel) & 0xFFFF0000u;
+    out[i] = __uint_as_float(va | ((codes << (28 - 4 * i)) & 0x80000000u));
+    out[4 + i] = __uint_as_float(vb | ((codes << (12 - 4 * i)) & 0x80000000u));
+  }
 }
 
 // Non-negative float -> E4M3 code (RNE, saturating at 448).

@@ -15,8 +15,9 @@
 //               shared -> tensor memory (tcgen05.cp 32x128b.warpx4), then
 //               tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 per instruction); commits
 //               free the shared stage and, at the end of a tile, publish the accumulator.
-//   warps 2..5  epilogue: tcgen05.ld of the FP32 accumulator (each warp owns its lane
-//               quadrant), scale by alpha, store bf16/FP32 rows (or SwiGLU + amax).
+//   warps 2..9  epilogue: tcgen05.ld of the FP32 accumulator (two warps per lane quadrant,
+//               one column half each) into registers, release, then scale by alpha and
+//               store bf16/FP32 rows (or SwiGLU + amax) while the next tile's MMAs run.
 // Every mbarrier wait is bounded by a wall-clock limit; on expiry the kernel records
 // NVFP4_ERR_TIMEOUT, drains its own copies and MMAs, frees tensor memory and returns.
 #include "common.cuh"
@@ -27,7 +28,7 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int KT_BYTES = 128;  // bytes of one row per k-tile: 256 FP4 elements
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;  // producer warp, MMA warp, 8 epilogue warps
 
 template <int BN>
 struct Cfg {
@@ -212,7 +213,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int a = 0; a < C::ACC_STAGES; ++a) {
       mbar_init(bar_accf(a), 1);
-      mbar_init(bar_acce(a), 4);
+      mbar_init(bar_acce(a), 8);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -361,7 +362,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else {
     // ===================================================================== epilogue
-    const int quad = warp & 3;  // tensor-memory lanes [32*quad, 32*quad + 32)
+    // Eight warps: two per tensor-memory lane quadrant, each owning half of the tile's
+    // columns.  A warp drains its columns into registers, releases the accumulator, and only
+    // then converts and stores, so the math overlaps the next tile's MMAs.
+    constexpr int NCH = BN / 64;            // 32-column chunks per warp
+    const int quad = warp & 3;              // tensor-memory lanes [32*quad, 32*quad + 32)
+    const int half = (warp - 2) >> 2;       // which half of the tile's columns
     int acc = 0;
     uint32_t acc_phase = 0;
     float amax = 0.0f;
@@ -384,79 +390,84 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const bool row_ok = row < row_limit && row < args.rows_capacity;
       const float alpha = __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));
       const uint32_t t_row = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(quad * 32) << 16);
+      uint32_t v[NCH][32];
       if (args.epi == 0) {
-#pragma unroll 1
-        for (int c = 0; c < BN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(t_row + c * 32, v);
-          tmem_wait_ld();
-          if (row_ok) {
-            const int64_t col = (int64_t)nb * BN + c * 32;
-            if (args.out_bf16) {
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy + col);
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint32_t p[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h)
-                  p[h] = pack_bf16x2(__fmul_rn(__uint_as_float(v[8 * q + 2 * h]), alpha),
-                                     __fmul_rn(__uint_as_float(v[8 * q + 2 * h + 1]), alpha));
-                dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
-              }
-            } else {
-              float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.y) + row * args.ldy + col);
-#pragma unroll
-              for (int q = 0; q < 8; ++q)
-                dst[q] = make_float4(__fmul_rn(__uint_as_float(v[4 * q]), alpha),
-                                     __fmul_rn(__uint_as_float(v[4 * q + 1]), alpha),
-                                     __fmul_rn(__uint_as_float(v[4 * q + 2]), alpha),
-                                     __fmul_rn(__uint_as_float(v[4 * q + 3]), alpha));
-            }
-          }
-        }
+        for (int i = 0; i < NCH; ++i) tmem_ld32(t_row + half * (BN / 2) + 32 * i, v[i]);
       } else {
-        // SwiGLU: within each 128-column half of the tile, columns [0,64) are gate rows and
-        // [64,128) the matching up rows (gate/up interleave of the packed weight).
-#pragma unroll 1
-        for (int hh = 0; hh < BN / 128; ++hh) {
-#pragma unroll 1
-          for (int c = 0; c < 2; ++c) {
-            uint32_t g[32], u[32];
-            tmem_ld32(t_row + hh * 128 + c * 32, g);
-            tmem_ld32(t_row + hh * 128 + 64 + c * 32, u);
-            tmem_wait_ld();
-            if (row_ok) {
-              const int64_t col = (int64_t)nb * (BN / 2) + hh * 64 + c * 32;
-              uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy + col);
+        // SwiGLU: output feature f of the tile reads gate column (f/64)*128 + f%64 and the up
+        // column 64 further (gate/up interleave of the packed weight); this warp owns
+        // features [half*BN/4, (half+1)*BN/4): chunks 0..NCH/2-1 gate, NCH/2.. up.
 #pragma unroll
-              for (int q = 0; q < 4; ++q) {
-                uint32_t p[4];
-#pragma unroll
-                for (int h = 0; h < 4; ++h) {
-                  float hv[2];
-#pragma unroll
-                  for (int z = 0; z < 2; ++z) {
-                    const int i = 8 * q + 2 * h + z;
-                    const float gv = bf16_round(__fmul_rn(__uint_as_float(g[i]), alpha));
-                    const float uv = bf16_round(__fmul_rn(__uint_as_float(u[i]), alpha));
-                    const float s = gv / (1.0f + expf(-gv));
-                    hv[z] = bf16_round(s * uv);
-                    amax = fmaxf(amax, fabsf(hv[z]));
-                  }
-                  p[h] = pack_bf16x2(hv[0], hv[1]);
-                }
-                dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
-              }
-            }
-          }
+        for (int i = 0; i < NCH / 2; ++i) {
+          const int f = half * (BN / 4) + 32 * i;
+          const int gcol = (f / 64) * 128 + (f % 64);
+          tmem_ld32(t_row + gcol, v[i]);
+          tmem_ld32(t_row + gcol + 64, v[NCH / 2 + i]);
         }
       }
+      tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_acce(acc));
       if (++acc == C::ACC_STAGES) {
         acc = 0;
         acc_phase ^= 1u;
+      }
+      if (!row_ok) continue;
+      if (args.epi == 0) {
+        const int64_t col0 = (int64_t)nb * BN + half * (BN / 2);
+        if (args.out_bf16) {
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy + col0);
+#pragma unroll
+          for (int i = 0; i < NCH; ++i)
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              uint32_t p[4];
+#pragma unroll
+              for (int h = 0; h < 4; ++h)
+                p[h] = pack_bf16x2(__fmul_rn(__uint_as_float(v[i][8 * q + 2 * h]), alpha),
+                                   __fmul_rn(__uint_as_float(v[i][8 * q + 2 * h + 1]), alpha));
+              dst[4 * i + q] = make_uint4(p[0], p[1], p[2], p[3]);
+            }
+        } else {
+          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.y) + row * args.ldy + col0);
+#pragma unroll
+          for (int i = 0; i < NCH; ++i)
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              dst[8 * i + q] = make_float4(__fmul_rn(__uint_as_float(v[i][4 * q]), alpha),
+                                           __fmul_rn(__uint_as_float(v[i][4 * q + 1]), alpha),
+                                           __fmul_rn(__uint_as_float(v[i][4 * q + 2]), alpha),
+                                           __fmul_rn(__uint_as_float(v[i][4 * q + 3]), alpha));
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < NCH / 2; ++i) {
+          const int f = half * (BN / 4) + 32 * i;  // first output feature of this chunk
+          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy +
+                                                (int64_t)nb * (BN / 2) + f);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t p[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              float hv[2];
+#pragma unroll
+              for (int z = 0; z < 2; ++z) {
+                const int j = 8 * q + 2 * h + z;
+                const float gv = bf16_round(__fmul_rn(__uint_as_float(v[i][j]), alpha));
+                const float uv = bf16_round(__fmul_rn(__uint_as_float(v[NCH / 2 + i][j]), alpha));
+                // silu(g) = g / (1 + e^-g); e^-g overflowing to inf gives -0 (the limit)
+                const float sg = __fdividef(gv, 1.0f + __expf(-gv));
+                hv[z] = bf16_round(sg * uv);
+                amax = fmaxf(amax, fabsf(hv[z]));
+              }
+              p[h] = pack_bf16x2(hv[0], hv[1]);
+            }
+            dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
+          }
+        }
       }
     }
     if (args.epi != 0 && args.amax_out != nullptr) {

@@ -19,6 +19,8 @@ struct RowArgs {
   int64_t ld;                    // source pitch (elements)
   int64_t K;                     // channels
   const int32_t* row_gather;     // act: optional output-row -> source-row map
+  const int32_t* row_scatter;    // act: optional source-row -> fanout output rows (-1 = none)
+  int fanout;
   int64_t rows_out;              // output rows to write (act: rows_padded; pack: slabs*rows_padded)
   int64_t rows_per_slab;         // pack: rows_padded per slab (== N); otherwise rows_out
   int64_t src_slab_stride;       // pack: N*K elements between slabs

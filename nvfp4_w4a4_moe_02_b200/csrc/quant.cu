@@ -72,24 +72,48 @@ __device__ __forceinline__ float reduce_partials(const float* partial, int P) {
 }
 
 // ----------------------------------------------------------------------------------------
-// K2 / K7 / calibration: the row quantiser.  One warp per output row, 512 elements per warp
+// K2 / K7 / calibration: the row quantiser.  One warp per row, 512 elements per warp
 // iteration: lane l loads elements [it*512 + 8l, +8) and [it*512 + 256 + 8l, +8), so lanes
 // (2m, 2m+1) hold the two halves of block it*32 + m and of block it*32 + 16 + m.
+//
+// The residual pass over the selected channels (activation mode) or the raw selected columns
+// (weight pack) runs after the main pass from a per-warp stash of the row and of each block's
+// (d, 1/d): lane pairs take 16 consecutive compact positions, read their channel numbers and
+// re-derive x, its code and DQ = e*d for exactly those channels.
 // ----------------------------------------------------------------------------------------
 
-
-// Writes the 4-byte scale word of a k64 group: lanes 8g..8g+7 own blocks 4g'..4g'+3 where
-// the pair (2m, 2m+1) owns block m; lane 8g gathers from lanes 8g, 8g+2, 8g+4, 8g+6.
-__device__ __forceinline__ void store_scale_words(uint32_t S, uint8_t* sf, int64_t row, int64_t kb_base, int64_t k64,
-                                                  int lane, bool active) {
+// Scale word of a k64 group: lanes 8g..8g+7 own blocks 4g..4g+3 (the pair (2m, 2m+1) owns
+// block m); lane 8g gathers the codes held by lanes 8g, 8g+2, 8g+4, 8g+6.
+__device__ __forceinline__ uint32_t scale_word(uint32_t S) {
   uint32_t s1 = __shfl_down_sync(0xffffffffu, S, 2);
   uint32_t s2 = __shfl_down_sync(0xffffffffu, S, 4);
   uint32_t s3 = __shfl_down_sync(0xffffffffu, S, 6);
-  if (active && (lane & 7) == 0) {
-    uint32_t word = S | (s1 << 8) | (s2 << 16) | (s3 << 24);
-    int64_t kb = kb_base + (lane >> 1);  // first block of this k64 group
-    *reinterpret_cast<uint32_t*>(sf + sf_offset(row, kb, k64)) = word;
+  return S | (s1 << 8) | (s2 << 16) | (s3 << 24);
+}
+
+// destinations of the current row: the row itself, or up to `fanout` rows in scatter mode
+struct Dests {
+  const int32_t* list;  // null: single destination `row`
+  int n;
+  int64_t row;
+  __device__ __forceinline__ int64_t get(int j) const { return list ? (int64_t)__ldg(list + j) : row; }
+};
+
+__device__ __forceinline__ void load8(const uint16_t* p, bool ok, float x[8], uint4& raw) {
+  raw = ok ? __ldg(reinterpret_cast<const uint4*>(p)) : make_uint4(0, 0, 0, 0);
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+    x[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
   }
+}
+
+__device__ __forceinline__ float pair_max8(const float x[8]) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
+  return fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
 }
 
 template <int MODE>
@@ -101,37 +125,46 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const RowArgs a) {
   const int64_t K = a.K;
   const int32_t Kp = a.Kp;
   constexpr bool kHasSel = (MODE == kModeAct || MODE == kModePack);
+  const bool use_sel = kHasSel && Kp > 0;
 
-  // channel -> compact position map (-1 = not selected), shared by the CTA
-  int16_t* pos = reinterpret_cast<int16_t*>(smem_raw);
-  float* rbuf_all = reinterpret_cast<float*>(smem_raw + ((K * 2 + 15) / 16) * 16);
-  float* rbuf = rbuf_all + (int64_t)warp * (Kp > 0 ? Kp : 1);
-  if (kHasSel && Kp > 0) {
-    for (int64_t c = threadIdx.x; c < K; c += blockDim.x) pos[c] = -1;
-    __syncthreads();
+  // CTA-shared channel list (int16), then per warp: the row's bf16 bits and each block's (d, 1/d)
+  int16_t* sel_s = reinterpret_cast<int16_t*>(smem_raw);
+  const size_t sel_bytes = use_sel ? (((size_t)Kp * 2 + 15) / 16) * 16 : 0;
+  const size_t warp_bytes = use_sel ? (((size_t)K * 2 + 15) / 16) * 16 + (size_t)(K / 16) * 8 : 0;
+  uint16_t* row_s = reinterpret_cast<uint16_t*>(smem_raw + sel_bytes + warp * warp_bytes);
+  float2* dinv_s = reinterpret_cast<float2*>(reinterpret_cast<unsigned char*>(row_s) + ((K * 2 + 15) / 16) * 16);
+  if (use_sel) {
     for (int32_t j = threadIdx.x; j < Kp; j += blockDim.x) {
       int32_t c = a.sel[j];
       bool ok = (c >= 0 && c < K) && (j == 0 || a.sel[j - 1] < c);
-      if (ok) pos[c] = (int16_t)j;
-      else report_status(a.status, kErrInvalid);
+      if (!ok) {
+        report_status(a.status, kErrInvalid);
+        c = 0;
+      }
+      sel_s[j] = (int16_t)c;
     }
     __syncthreads();
   }
 
   const int64_t k64 = K / 64;
   const int64_t kp64 = Kp / 64;
-  const int64_t n_it = K / 512;           // full 512-element iterations
-  const int64_t tail = K - n_it * 512;    // 0, 64, ..., 448 (K % 64 == 0)
+  const bool scatter = (MODE == kModeAct && a.row_scatter != nullptr);
+  const int64_t n_rows = scatter ? a.src_rows : a.rows_out;
   int64_t cached_slab = -1;
   float s_g = 0.0f, t6 = 0.0f;
 
-  for (int64_t row = (int64_t)blockIdx.x * nwarps + warp; row < a.rows_out; row += (int64_t)gridDim.x * nwarps) {
-    // ---- source row and scale
+  for (int64_t row = (int64_t)blockIdx.x * nwarps + warp; row < n_rows; row += (int64_t)gridDim.x * nwarps) {
+    // ---- source row, destinations, scale
     int64_t slab = (MODE == kModePack) ? row / a.rows_per_slab : 0;
     int64_t r_in_slab = row - slab * a.rows_per_slab;
     int64_t src_row = r_in_slab;
-    if (MODE == kModeAct && a.row_gather != nullptr) src_row = (r_in_slab < a.rows_per_slab) ? a.row_gather[r_in_slab] : -1;
-    if (MODE == kModeAct && a.row_gather != nullptr && row >= a.rows_per_slab) src_row = -1;
+    Dests dst{nullptr, 1, row};
+    if (scatter) {
+      dst.list = a.row_scatter + row * a.fanout;
+      dst.n = a.fanout;
+    } else if (MODE == kModeAct && a.row_gather != nullptr) {
+      src_row = (r_in_slab < a.rows_per_slab) ? a.row_gather[r_in_slab] : -1;
+    }
     if (MODE == kModePack && a.interleave) {
       int64_t q = r_in_slab >> 7, j = r_in_slab & 127;
       src_row = (j < 64) ? (q * 64 + j) : (a.N_half + q * 64 + (j - 64));
@@ -142,7 +175,7 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const RowArgs a) {
       s_g = scale_from_amax(amax, a.status);
       t6 = __fmul_rn(6.0f, s_g);
       cached_slab = slab;
-      if (row == slab * a.rows_per_slab + 0 && lane == 0) {
+      if (row == slab * a.rows_per_slab && lane == 0) {
         // exactly one warp writes each slab's scale: the one owning the slab's first row
         if (a.s_g_out) a.s_g_out[slab] = s_g;
         if (a.s_g_out2) a.s_g_out2[slab] = s_g;
@@ -150,117 +183,124 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const RowArgs a) {
     }
     const uint16_t* srow = a.src + slab * a.src_slab_stride + (valid ? src_row : 0) * a.ld;
 
-    // ---- main pass over the row, 512 (or a 64..448 tail) elements per iteration
-    for (int64_t it = 0; it <= n_it; ++it) {
-      const int64_t base = it * 512;
-      const int64_t span = (it < n_it) ? 512 : tail;
-      if (span == 0) break;
-      // element offsets held by this lane
-      const int64_t e0 = base + 8 * lane;          // first half-block
-      const int64_t e1 = base + 256 + 8 * lane;    // second half-block
-      const bool h0 = e0 < base + span;            // span is a multiple of 64: pair-uniform
-      const bool h1 = e1 < base + span;
+    // ---- main pass
+    for (int64_t base = 0; base < K; base += 512) {
+      const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
+      const bool h0 = e0 < K, h1 = e1 < K;  // K % 64 == 0: uniform over lane pairs and 8-lane groups
       float x0[8], x1[8];
-      {
-        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-        if (valid && h0) q0 = __ldg(reinterpret_cast<const uint4*>(srow + e0));
-        if (valid && h1) q1 = __ldg(reinterpret_cast<const uint4*>(srow + e1));
-        uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          x0[2 * j] = bf16_bits_to_f32(w0[j] & 0xFFFFu);
-          x0[2 * j + 1] = bf16_bits_to_f32(w0[j] >> 16);
-          x1[2 * j] = bf16_bits_to_f32(w1[j] & 0xFFFFu);
-          x1[2 * j + 1] = bf16_bits_to_f32(w1[j] >> 16);
-        }
-      }
-      float m0 = 0.0f, m1 = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        m0 = fmaxf(m0, fabsf(x0[i]));
-        m1 = fmaxf(m1, fabsf(x1[i]));
-      }
-      m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-      BlockScale b0 = block_scale(m0, s_g, t6), b1 = block_scale(m1, s_g, t6);
-      float dq0[8], dq1[8];
-      uint32_t c0 = quant8(x0, b0, dq0);
-      uint32_t c1 = quant8(x1, b1, dq1);
-      if (MODE != kModeCal) {
-        uint8_t* crow = a.codes + row * (K / 2);
-        if (h0) *reinterpret_cast<uint32_t*>(crow + e0 / 2) = c0;
-        if (h1) *reinterpret_cast<uint32_t*>(crow + e1 / 2) = c1;
-        // scale words: the first half covers blocks base/16 + [0,16), the second + [16,32)
-        store_scale_words(b0.S, a.sf, row, base / 16, k64, lane, h0);
-        store_scale_words(b1.S, a.sf, row, base / 16 + 16, k64, lane, h1);
-      }
+      uint4 r0, r1;
+      load8(srow + e0, valid && h0, x0, r0);
+      load8(srow + e1, valid && h1, x1, r1);
+      const BlockScale b0 = block_scale(pair_max8(x0), s_g, t6);
+      const BlockScale b1 = block_scale(pair_max8(x1), s_g, t6);
       if (MODE == kModeCal) {
+        float dq0[8], dq1[8];
+        quant8(x0, b0, dq0);
+        quant8(x1, b1, dq1);
         float* rr = a.resid_all + row * K;
         if (h0) {
-          float4 r0 = make_float4(__fsub_rn(x0[0], dq0[0]), __fsub_rn(x0[1], dq0[1]), __fsub_rn(x0[2], dq0[2]),
-                                  __fsub_rn(x0[3], dq0[3]));
-          float4 r1 = make_float4(__fsub_rn(x0[4], dq0[4]), __fsub_rn(x0[5], dq0[5]), __fsub_rn(x0[6], dq0[6]),
-                                  __fsub_rn(x0[7], dq0[7]));
-          *reinterpret_cast<float4*>(rr + e0) = r0;
-          *reinterpret_cast<float4*>(rr + e0 + 4) = r1;
+          *reinterpret_cast<float4*>(rr + e0) = make_float4(__fsub_rn(x0[0], dq0[0]), __fsub_rn(x0[1], dq0[1]),
+                                                            __fsub_rn(x0[2], dq0[2]), __fsub_rn(x0[3], dq0[3]));
+          *reinterpret_cast<float4*>(rr + e0 + 4) = make_float4(__fsub_rn(x0[4], dq0[4]), __fsub_rn(x0[5], dq0[5]),
+                                                                __fsub_rn(x0[6], dq0[6]), __fsub_rn(x0[7], dq0[7]));
         }
         if (h1) {
-          float4 r0 = make_float4(__fsub_rn(x1[0], dq1[0]), __fsub_rn(x1[1], dq1[1]), __fsub_rn(x1[2], dq1[2]),
-                                  __fsub_rn(x1[3], dq1[3]));
-          float4 r1 = make_float4(__fsub_rn(x1[4], dq1[4]), __fsub_rn(x1[5], dq1[5]), __fsub_rn(x1[6], dq1[6]),
-                                  __fsub_rn(x1[7], dq1[7]));
-          *reinterpret_cast<float4*>(rr + e1) = r0;
-          *reinterpret_cast<float4*>(rr + e1 + 4) = r1;
+          *reinterpret_cast<float4*>(rr + e1) = make_float4(__fsub_rn(x1[0], dq1[0]), __fsub_rn(x1[1], dq1[1]),
+                                                            __fsub_rn(x1[2], dq1[2]), __fsub_rn(x1[3], dq1[3]));
+          *reinterpret_cast<float4*>(rr + e1 + 4) = make_float4(__fsub_rn(x1[4], dq1[4]), __fsub_rn(x1[5], dq1[5]),
+                                                                __fsub_rn(x1[6], dq1[6]), __fsub_rn(x1[7], dq1[7]));
+        }
+        continue;
+      }
+      const uint32_t c0 = quant8_codes(x0, b0), c1 = quant8_codes(x1, b1);
+      const uint32_t w0 = scale_word(b0.S), w1 = scale_word(b1.S);
+      if (use_sel) {
+        // stash the row and the block scales for the residual pass
+        if (h0) *reinterpret_cast<uint4*>(row_s + e0) = r0;
+        if (h1) *reinterpret_cast<uint4*>(row_s + e1) = r1;
+        if ((lane & 1) == 0) {
+          if (h0) dinv_s[e0 >> 4] = make_float2(b0.d, b0.inv);
+          if (h1) dinv_s[e1 >> 4] = make_float2(b1.d, b1.inv);
         }
       }
-      if (kHasSel && Kp > 0) {
-        // selected channels: residual (act) or raw value (pack) into the compact row buffer
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          if (h0) {
-            int p = pos[e0 + i];
-            if (p >= 0) rbuf[p] = (MODE == kModeAct) ? __fsub_rn(x0[i], dq0[i]) : x0[i];
-          }
-          if (h1) {
-            int p = pos[e1 + i];
-            if (p >= 0) rbuf[p] = (MODE == kModeAct) ? __fsub_rn(x1[i], dq1[i]) : x1[i];
-          }
+      for (int j = 0; j < dst.n; ++j) {
+        const int64_t drow = dst.get(j);
+        if (drow < 0) continue;
+        if (drow >= a.rows_out) {
+          report_status(a.status, kErrInvalid);
+          continue;
+        }
+        uint8_t* crow = a.codes + drow * (K / 2);
+        if (h0) *reinterpret_cast<uint32_t*>(crow + e0 / 2) = c0;
+        if (h1) *reinterpret_cast<uint32_t*>(crow + e1 / 2) = c1;
+        if ((lane & 7) == 0) {
+          if (h0) *reinterpret_cast<uint32_t*>(a.sf + sf_offset(drow, e0 >> 4, k64)) = w0;
+          if (h1) *reinterpret_cast<uint32_t*>(a.sf + sf_offset(drow, e1 >> 4, k64)) = w1;
         }
       }
     }
 
-    // ---- second pass over the compact selected channels
-    if (kHasSel && Kp > 0) {
+    // ---- residual pass over the compact selected channels
+    if (use_sel) {
       __syncwarp();
-      const int64_t nr_it = Kp / 512, rtail = Kp - nr_it * 512;
-      for (int64_t it = 0; it <= nr_it; ++it) {
-        const int64_t base = it * 512;
-        const int64_t span = (it < nr_it) ? 512 : rtail;
-        if (span == 0) break;
-        const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
-        const bool h0 = e0 < base + span, h1 = e1 < base + span;
-        float x0[8], x1[8];
+      for (int64_t base = 0; base < Kp; base += 512) {
+        const int64_t p0 = base + 8 * lane, p1 = base + 256 + 8 * lane;
+        const bool h0 = p0 < Kp, h1 = p1 < Kp;
+        float v[2][8];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          x0[i] = (valid && h0) ? rbuf[e0 + i] : 0.0f;
-          x1[i] = (valid && h1) ? rbuf[e1 + i] : 0.0f;
-        }
-        float m0 = 0.0f, m1 = 0.0f;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int64_t p = hh ? p1 : p0;
+          const bool ok = hh ? h1 : h0;
+          int32_t ch[8];
+          {
+            const uint4 cv = ok ? *reinterpret_cast<const uint4*>(sel_s + p) : make_uint4(0, 0, 0, 0);
+            const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          m0 = fmaxf(m0, fabsf(x0[i]));
-          m1 = fmaxf(m1, fabsf(x1[i]));
+            for (int j = 0; j < 4; ++j) {
+              ch[2 * j] = (int32_t)(int16_t)(w[j] & 0xFFFFu);
+              ch[2 * j + 1] = (int32_t)(int16_t)(w[j] >> 16);
+            }
+          }
+          float x[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) x[i] = bf16_bits_to_f32(row_s[ch[i]]);
+          if (MODE == kModePack) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[hh][i] = x[i];
+          } else {
+            // re-derive the channel's code under its own block scale, then r = x - e*d
+            float sc[8], d[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 di = dinv_s[ch[i] >> 4];
+              d[i] = di.x;
+              sc[i] = __fmul_rn(x[i], di.y);
+            }
+            float e[8];
+            e2m1_decode8(e2m1_encode8(sc), e);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[hh][i] = __fsub_rn(x[i], d[i] == 0.0f ? 0.0f : __fmul_rn(e[i], d[i]));
+          }
+          if (!ok || !valid) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[hh][i] = 0.0f;
+          }
         }
-        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-        BlockScale b0 = block_scale(m0, s_g, t6), b1 = block_scale(m1, s_g, t6);
-        uint32_t c0 = quant8_codes(x0, b0);
-        uint32_t c1 = quant8_codes(x1, b1);
-        uint8_t* crow = a.rcodes + row * (Kp / 2);
-        if (h0) *reinterpret_cast<uint32_t*>(crow + e0 / 2) = c0;
-        if (h1) *reinterpret_cast<uint32_t*>(crow + e1 / 2) = c1;
-        store_scale_words(b0.S, a.rsf, row, base / 16, kp64, lane, h0);
-        store_scale_words(b1.S, a.rsf, row, base / 16 + 16, kp64, lane, h1);
+        const BlockScale b0 = block_scale(pair_max8(v[0]), s_g, t6);
+        const BlockScale b1 = block_scale(pair_max8(v[1]), s_g, t6);
+        const uint32_t c0 = quant8_codes(v[0], b0), c1 = quant8_codes(v[1], b1);
+        const uint32_t w0 = scale_word(b0.S), w1 = scale_word(b1.S);
+        for (int j = 0; j < dst.n; ++j) {
+          const int64_t drow = dst.get(j);
+          if (drow < 0 || drow >= a.rows_out) continue;
+          uint8_t* crow = a.rcodes + drow * (Kp / 2);
+          if (h0) *reinterpret_cast<uint32_t*>(crow + p0 / 2) = c0;
+          if (h1) *reinterpret_cast<uint32_t*>(crow + p1 / 2) = c1;
+          if ((lane & 7) == 0) {
+            if (h0) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset(drow, p0 >> 4, kp64)) = w0;
+            if (h1) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset(drow, p1 >> 4, kp64)) = w1;
+          }
+        }
       }
       __syncwarp();
     }
@@ -454,7 +494,8 @@ cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64
 }
 
 size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps) {
-  return (size_t)((K * 2 + 15) / 16) * 16 + (size_t)warps * (size_t)(Kp > 0 ? Kp : 1) * 4;
+  if (Kp <= 0) return 16;
+  return (size_t)((Kp * 2 + 15) / 16) * 16 + (size_t)warps * ((size_t)((K * 2 + 15) / 16) * 16 + (size_t)(K / 16) * 8);
 }
 
 cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
@@ -465,7 +506,8 @@ cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
     smem = rows_smem_bytes(a.K, a.Kp, warps);
   }
   if (smem > 200 * 1024) return cudaErrorInvalidValue;
-  int64_t ctas_needed = (a.rows_out + warps - 1) / warps;
+  const int64_t rows = a.row_scatter ? a.src_rows : a.rows_out;
+  int64_t ctas_needed = (rows + warps - 1) / warps;
   int per_sm = (int)((220 * 1024) / (smem + 1024));
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 8) per_sm = 8;

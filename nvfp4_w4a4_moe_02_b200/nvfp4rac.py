@@ -61,6 +61,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_set_wait_limit_ns": ([u64], None),
         "nvfp4_quantize_workspace_size": ([i64, i64], sz),
         "nvfp4_quantize": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "nvfp4_quantize_scatter": ([vp, i64, i64, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
         "rac_calibrate_workspace_size": ([i64, i64], sz),
         "rac_calibrate": ([vp, i64, i64, i32, vp, vp, vp, sz, vp, vp], ctypes.c_int),
         "pack_weights_workspace_size": ([i64, i64, i64], sz),
@@ -118,10 +119,12 @@ class Packed:
     cols: int
 
     @staticmethod
-    def empty(rows: int, cols: int, slabs: int = 1, rows_padded: int | None = None, device="cuda") -> "Packed":
+    def empty(rows: int, cols: int, slabs: int = 1, rows_padded: int | None = None, device="cuda",
+              zero: bool = False) -> "Packed":
         rp = round_up(max(rows, 1), 128) if rows_padded is None else rows_padded
-        codes = torch.empty(slabs * rp * cols // 2, dtype=torch.uint8, device=device)
-        sf = torch.empty(slabs * rp * cols // 16, dtype=torch.uint8, device=device)
+        alloc = torch.zeros if zero else torch.empty
+        codes = alloc(slabs * rp * cols // 2, dtype=torch.uint8, device=device)
+        sf = alloc(slabs * rp * cols // 16, dtype=torch.uint8, device=device)
         s_g = torch.empty(slabs, dtype=torch.float32, device=device)
         return Packed(codes, sf, s_g, slabs, rows, rp, cols)
 
@@ -197,6 +200,34 @@ def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather:
     _check(lib.nvfp4_quantize(x.data_ptr(), M, K, ldx, _ptr(row_gather), M_out, _ptr(sel), Kp, _ptr(amax_in),
                               ctypes.byref(q), ctypes.byref(qr) if qr is not None else None, ws.data_ptr(),
                               ws.numel(), st.data_ptr(), _stream(stream)))
+    return out, (out_res if Kp > 0 else None)
+
+
+def nvfp4_quantize_scatter(x: torch.Tensor, row_scatter: torch.Tensor, rows_padded: int,
+                           sel: torch.Tensor | None = None, amax_in: torch.Tensor | None = None,
+                           out: Packed | None = None, out_res: Packed | None = None,
+                           status: torch.Tensor | None = None, stream=None):
+    """Quantise each row of x once and write it to the rows row_scatter[m, :] of the outputs.
+
+    row_scatter: int32 [M, fanout] (-1 = unused).  Rows no entry names are left untouched, so
+    freshly created outputs are zero-filled.  Returns (Packed, Packed | None)."""
+    lib = load()
+    _u16(x)
+    M, K = x.shape
+    assert x.stride(1) == 1 and row_scatter.dtype == torch.int32 and row_scatter.is_contiguous()
+    fanout = row_scatter.shape[1]
+    Kp = 0 if sel is None else int(sel.numel())
+    if out is None:
+        out = Packed.empty(rows_padded, K, rows_padded=rows_padded, device=x.device, zero=True)
+    if Kp > 0 and out_res is None:
+        out_res = Packed.empty(rows_padded, Kp, rows_padded=rows_padded, device=x.device, zero=True)
+    ws = _workspace(x.device).get(lib.nvfp4_quantize_workspace_size(M, K))
+    st = status if status is not None else new_status(x.device)
+    q = out.c()
+    qr = out_res.c() if Kp > 0 else None
+    _check(lib.nvfp4_quantize_scatter(x.data_ptr(), M, K, x.stride(0), row_scatter.data_ptr(), fanout, _ptr(sel), Kp,
+                                      _ptr(amax_in), ctypes.byref(q), ctypes.byref(qr) if qr is not None else None,
+                                      ws.data_ptr(), ws.numel(), st.data_ptr(), _stream(stream)))
     return out, (out_res if Kp > 0 else None)
 
 
@@ -349,3 +380,15 @@ def gather_map(pair_token, counts, pad: int = 128):
     g = np.full(total, -1, dtype=np.int32)
     g[pair_rows] = np.asarray(pair_token, dtype=np.int32)
     return g, off, pair_rows
+
+
+def scatter_map(pair_token, pair_rows, T: int, fanout: int):
+    """row_scatter [T, fanout]: the padded rows of each token's (token, expert) pairs, -1 padded."""
+    import numpy as np
+
+    m = np.full((T, fanout), -1, dtype=np.int32)
+    fill = np.zeros(T, dtype=np.int64)
+    for t, r in zip(np.asarray(pair_token), np.asarray(pair_rows)):
+        m[t, fill[t]] = r
+        fill[t] += 1
+    return m

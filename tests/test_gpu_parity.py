@@ -174,6 +174,31 @@ def test_quantize_row_gather(dev, orc):
     assert np.array_equal(grc, rcodes) and np.array_equal(grS, rS)
 
 
+def test_quantize_scatter_matches_gather(dev, orc):
+    """Scatter mode (each token quantised once, written to its expert rows) gives the same bytes
+    as the gather mode and as the oracle; unnamed (padding) rows stay zero."""
+    wl = syn.moe_block(T=300, H=1024, E=16, topk=4, I=256, T_cal=64, materialize_weights=False)
+    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    sm = R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], 4)
+    xd = to_dev(wl.x, dev)
+    sel = np.arange(3, 1024, 2, dtype=np.int32)[:448]
+    seld = torch.from_numpy(sel).to(dev)
+    qg, qgr = R.nvfp4_quantize(xd, seld, row_gather=torch.from_numpy(g).to(dev), M_out=g.size)
+    qs, qsr = R.nvfp4_quantize_scatter(xd, torch.from_numpy(sm).to(dev), g.size, seld)
+    torch.cuda.synchronize()
+    assert torch.equal(qg.codes, qs.codes) and torch.equal(qg.sf, qs.sf) and torch.equal(qg.s_g, qs.s_g)
+    assert torch.equal(qgr.codes, qsr.codes) and torch.equal(qgr.sf, qsr.sf)
+    s_ref = orc.global_scale(orc.amax_bf16(wl.x))
+    codes, S, rcodes, rS, _ = orc.act_quant_rac(wl.x, s_ref, sel)
+    gc, gS = logical(qs, rows=qs.rows_padded)
+    assert np.array_equal(gc[pair_rows], codes[wl.pair_token]) and np.array_equal(gS[pair_rows], S[wl.pair_token])
+    grc, grS = logical(qsr, rows=qsr.rows_padded)
+    assert np.array_equal(grc[pair_rows], rcodes[wl.pair_token])
+    pad = np.ones(qs.rows_padded, bool)
+    pad[pair_rows] = False
+    assert not gc[pad].any() and not gS[pad].any() and not grc[pad].any()
+
+
 # ------------------------------------------------------------------------------------------ calibration
 @pytest.mark.parametrize("shape", [(64, 256, 128), (2048, 4096, 2048), (100, 704, 320)])
 def test_calibrate_matches_oracle(dev, orc, shape):
@@ -309,8 +334,8 @@ def moe_pipeline(dev, wl, sel_gu, sel_dn):
     seld_dn = torch.from_numpy(sel_dn).to(dev)
     pgu, pgus = R.pack_weights(wgu, seld_gu, gate_up_interleave=True, status=st)
     pdn, pdns = R.pack_weights(wdn, seld_dn, status=st)
-    a, ar = R.nvfp4_quantize(to_dev(wl.x, dev), seld_gu, row_gather=torch.from_numpy(g).to(dev), M_out=g.size,
-                             status=st)
+    sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
+    a, ar = R.nvfp4_quantize_scatter(to_dev(wl.x, dev), sm, g.size, seld_gu, status=st)
     h, amax_h = R.grouped_w4a4_rac_moe(a, ar, offd, pgu, pgus, swiglu=True, status=st)
     hq, hqr = R.nvfp4_quantize(h, seld_dn, amax_in=amax_h, status=st)
     y = R.grouped_w4a4_rac_moe(hq, hqr, offd, pdn, pdns, status=st)
