@@ -134,9 +134,49 @@ class MoEStep:
     KERNELS_PER_STEP = 5  # amax, quantise X, gate_up GEMM, quantise h, down GEMM
 
 
+class DenseStep:
+    """Dense prefill projection: quantise X (+ residual) and the W4A4 + RAC GEMM, W pre-packed."""
+
+    KERNELS_PER_STEP = 3  # amax, quantise X, GEMM
+
+    def __init__(self, wl, dev):
+        import torch
+
+        from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+
+        self.R, self.torch, self.wl = R, torch, wl
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+        self.status = R.new_status(dev)
+        self.sel, _ = R.rac_calibrate(to(wl.x_cal), wl.Kp, status=self.status)
+        self.w, self.ws = R.pack_weights(to(wl.w), self.sel, status=self.status)
+        self.x = to(wl.x)
+        self.a = R.Packed.empty(wl.M, wl.K, device=dev)
+        self.ar = R.Packed.empty(wl.M, wl.Kp, rows_padded=self.a.rows_padded, device=dev)
+        self.y = torch.empty(wl.M, wl.N, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        R.check_status(self.status)
+        torch.cuda.empty_cache()
+
+    def run(self, x=None, events=None):
+        R = self.R
+        ev = events or {}
+        if "q0" in ev:
+            ev["q0"].record()
+        R.nvfp4_quantize(self.x if x is None else x, self.sel, out=self.a, out_res=self.ar, status=self.status)
+        if "g0" in ev:
+            ev["g0"].record()
+        R.w4a4_rac_gemm(self.a, self.ar, self.w, self.ws, self.wl.M, y=self.y, status=self.status)
+        if "end" in ev:
+            ev["end"].record()
+        return self.y
+
+
 # ------------------------------------------------------------------------------------------ clocks
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi clock / throttle-reason samples every 50 ms; samples are kept for the wall-clock
+    window of the timed region (if the region is shorter than the sampling period, the samples
+    closest to it are used)."""
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -148,36 +188,51 @@ class ClockSampler:
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
-                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
                                          stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
 
-    def stop(self):
+    def wait_first_sample(self, timeout=5.0):
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < timeout:
+            if os.path.exists(self.path) and os.path.getsize(self.path) > 0:
+                return
+            time.sleep(0.05)
+
+    def stop(self, t0=None, t1=None):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.1)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        sm, mx, reasons = [], [], set()
+        import datetime
+
+        rows = []
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for line in open(self.path):
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
             try:
-                sm.append(float(parts[1]))
-                mx.append(float(parts[2]))
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
         os.unlink(self.path)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        if t0 is not None:
+            inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05]
+            if not inside:  # region shorter than the sampling period: the nearest samples
+                inside = sorted(rows, key=lambda r: min(abs(r[0] - t0), abs(r[0] - t1)))[:2]
+            rows = inside
+        reasons = sorted({n for r in rows for n, v in zip(names, r[3]) if v.lower() == "active"})
+        return {"sm_mhz": float(np.median([r[1] for r in rows])), "sm_max_mhz": max(r[2] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
 
 
 # ------------------------------------------------------------------------------------------ CPU oracle leg
@@ -252,14 +307,75 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------------------------------ main
+def spec_moe(dev, args, peaks):
+    wl, h_cal = build_inputs()
+    step = MoEStep(wl, h_cal, dev)
+    gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
+    P = int(wl.pair_token.size)
+    gu_bytes = (wl.E * 2 * wl.I * (wl.H + wl.Kp_gu) * 0.5625 + P * (wl.H + wl.Kp_gu) * 0.5625 + P * wl.I * 2.0)
+
+    def cpu_leg():
+        import oracle as orc
+
+        orc.build()
+        dt, f = oracle_sample(wl, step.sel_gu.cpu().numpy(), step.sel_dn.cpu().numpy(), args.cpu_pairs)
+        return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+                "sample": f"{args.cpu_pairs} of {P} (token, expert) rows of one step, {dt:.1f} s"}
+
+    return dict(
+        step=step, x_np=wl.x, flops=gu_f + dn_f, events=["q0", "g0", "q1", "d0", "end"],
+        segments={"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")},
+        dominant=("gate_up", gu_f, gu_bytes, "grouped gate_up W4A4+RAC GEMM (SwiGLU epilogue)"),
+        quant={"x": ("quant_x", int(wl.x.nbytes) + P * 0.5625 * (wl.H + wl.Kp_gu)),  # X read once, 8 copies out
+               "h": ("quant_h", quant_bytes(P, wl.I, wl.Kp_dn))},
+        config={"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P, "experts": wl.E,
+                "hidden": wl.H, "intermediate": wl.I, "Kp_gate_up": wl.Kp_gu, "Kp_down": wl.Kp_dn,
+                "rows_padded": step.rows_padded},
+        cpu=cpu_leg, kernels_per_step=MoEStep.KERNELS_PER_STEP)
+
+
+def spec_dense(dev, args, peaks):
+    from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+    wl = syn.dense_prefill()
+    step = DenseStep(wl, dev)
+    flops = 2.0 * wl.M * wl.N * (wl.K + wl.Kp)
+    gbytes = 0.5625 * (wl.M + wl.N) * (wl.K + wl.Kp) + 2.0 * wl.M * wl.N
+
+    def cpu_leg():
+        import oracle as orc
+
+        orc.build()
+        rows = np.arange(0, wl.M, wl.M // max(1, args.cpu_rows))[:args.cpu_rows]
+        t0 = time.perf_counter()
+        orc.dense_rac_forward(wl.x, wl.w, step.sel.cpu().numpy(), rows=rows)
+        dt = time.perf_counter() - t0
+        f = 2.0 * rows.size * wl.N * (wl.K + wl.Kp)
+        return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+                "sample": f"{rows.size} of {wl.M} output rows (full quantisation of X and W included), {dt:.1f} s"}
+
+    return dict(
+        step=step, x_np=wl.x, flops=flops, events=["q0", "g0", "end"],
+        segments={"quant_x": ("q0", "g0"), "gemm": ("g0", "end")},
+        dominant=("gemm", flops, gbytes, "dense W4A4+RAC GEMM"),
+        quant={"x": ("quant_x", quant_bytes(wl.M, wl.K, wl.Kp))},
+        config={"workload": wl.name + f"_r{wl.r}", "M": wl.M, "N": wl.N, "K": wl.K, "Kp": wl.Kp},
+        cpu=cpu_leg, kernels_per_step=DenseStep.KERNELS_PER_STEP)
+
+
+SPECS = {"moe_prefill": spec_moe, "dense": spec_dense}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nvfp4rac", choices=["nvfp4rac", "reference"])
+    ap.add_argument("--workload", default="moe_prefill", choices=sorted(SPECS))
     ap.add_argument("--ref-pairs", type=int, default=256)
     ap.add_argument("--cpu-pairs", type=int, default=256)
+    ap.add_argument("--cpu-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
@@ -284,10 +400,8 @@ def main():
 
     R.load()
     peaks, peak_kind = load_peaks()
-    wl, h_cal = build_inputs()
-    step = MoEStep(wl, h_cal, dev)
-    gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
-    step_flops = gu_f + dn_f
+    sp = SPECS[args.workload](dev, args, peaks)
+    step = sp["step"]
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
 
     def barrier():
@@ -295,67 +409,63 @@ def main():
             torch.distributed.barrier()
         torch.cuda.synchronize()
 
-    # warm-up
+    clocks = ClockSampler(local)
+    clocks.start()
+    # warm-up (also gives the clock sampler time to start)
     for _ in range(args.warmup):
+        flush.zero_()
         step.run()
     torch.cuda.synchronize()
+    clocks.wait_first_sample()
     R.check_status(step.status)
 
     # timed region: K steps, L2 flushed between steps (outside the per-step events)
-    names = ["q0", "g0", "q1", "d0", "end"]
-    evs = [{n: torch.cuda.Event(enable_timing=True) for n in names} for _ in range(args.steps)]
-    clocks = ClockSampler(local)
-    clocks.start()
-    time.sleep(0.3)
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in sp["events"]} for _ in range(args.steps)]
     barrier()
+    t_wall0 = time.time()
     for i in range(args.steps):
         flush.zero_()
         step.run(events=evs[i])
     barrier()
-    clk = clocks.stop()
+    t_wall1 = time.time()
+    clk = clocks.stop(t_wall0, t_wall1)
     R.check_status(step.status)
-    seg = {"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")}
-    per = {k: [] for k in seg}
-    tot = []
-    for e in evs:
-        for k, (a, b) in seg.items():
-            per[k].append(e[a].elapsed_time(e[b]))
-        tot.append(e["q0"].elapsed_time(e["end"]))
-    t_step_ms = float(np.sum(tot)) / args.steps
+    first, last = sp["events"][0], sp["events"][-1]
+    per = {k: [e[a].elapsed_time(e[b]) for e in evs] for k, (a, b) in sp["segments"].items()}
+    t_step_ms = float(np.sum([e[first].elapsed_time(e[last]) for e in evs])) / args.steps
     if ws > 1:
         t = torch.tensor([t_step_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         t_step_ms = float(t.item())
-    value = ws * step_flops / (t_step_ms * 1e-3) / 1e12
+    value = ws * sp["flops"] / (t_step_ms * 1e-3) / 1e12
 
-    # kernel-level figures (mean over the timed steps)
+    # roofline of the dominant kernel: algorithmic bytes / flops over its event-timed duration
     k_ms = {k: float(np.mean(v)) for k, v in per.items()}
-    P = int(wl.pair_token.size)
-    gu_bytes = (wl.E * 2 * wl.I * (wl.H + wl.Kp_gu) * 0.5625 + P * (wl.H + wl.Kp_gu) * 0.5625 + P * wl.I * 2.0)
-    gu_hbm_t = gu_bytes / (peaks["hbm_gbs"] * 1e9)
+    seg, d_flops, d_bytes, d_label = sp["dominant"]
     fp4_peak = peaks["bf16_tflops"] * FP4_OVER_BF16
-    gu_tc_t = gu_f / (fp4_peak * 1e12)
-    if gu_hbm_t >= gu_tc_t:
-        achieved = gu_bytes / (k_ms["gate_up"] * 1e-3) / 1e9
+    if d_bytes / (peaks["hbm_gbs"] * 1e9) >= d_flops / (fp4_peak * 1e12):
+        achieved = d_bytes / (k_ms[seg] * 1e-3) / 1e9
         roof = {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": achieved / peaks["hbm_gbs"], "traffic": None}
     else:
-        achieved = gu_f / (k_ms["gate_up"] * 1e-3) / 1e12
+        achieved = d_flops / (k_ms[seg] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak, "traffic": None}
-    roof["kernel"] = "grouped gate_up W4A4+RAC GEMM (SwiGLU epilogue)"
-    roof["peak_source"] = f"{peak_kind} ({'MEASURED_PEAKS.json' if peak_kind == 'measured' else 'recipe fallback'})"
-    qx_bytes = int(wl.x.nbytes) + P * 0.5625 * (wl.H + wl.Kp_gu)  # X read once, 8 expert copies written
-    qh_bytes = quant_bytes(P, wl.I, wl.Kp_dn)
+    roof["kernel"] = d_label
+    roof["algorithmic"] = {"bytes": d_bytes, "flops": d_flops}
+    roof["peak_source"] = (f"{peak_kind}: HBM = copy bandwidth, FP4 = bf16 burst x {FP4_OVER_BF16:g} (nominal ratio)"
+                           if peak_kind == "measured" else "recipe fallback")
 
     # end-to-end through the public API with host buffers: H2D of X, D2H of Y every step
-    x_host = torch.from_numpy(wl.x.view(np.int16)).pin_memory()
+    x_np = sp["x_np"]
+    x_host = torch.from_numpy(x_np.view(np.int16)).pin_memory()
     y_host = torch.empty(step.y.shape, dtype=torch.bfloat16).pin_memory()
-    x_dev = torch.empty(wl.x.shape, dtype=torch.bfloat16, device=dev)
+    x_dev = torch.empty(x_np.shape, dtype=torch.bfloat16, device=dev)
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    n_e2e = max(3, args.steps // 4)
     e2e_ms = 0.0
-    for i in range(max(3, args.steps // 2)):
+    for _ in range(n_e2e):
         flush.zero_()
         e0.record()
         x_dev.view(torch.int16).copy_(x_host, non_blocking=True)
@@ -364,46 +474,34 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         e2e_ms += e0.elapsed_time(e1)
-    n_e2e = max(3, args.steps // 2)
     e2e_ms /= n_e2e
     if ws > 1:
         t = torch.tensor([e2e_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    e2e = {"value": ws * step_flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
-           "h2d_bytes_per_step": int(wl.x.nbytes), "d2h_bytes_per_step": int(y_host.numel() * 2)}
+    e2e = {"value": ws * sp["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+           "h2d_bytes_per_step": int(x_np.nbytes), "d2h_bytes_per_step": int(y_host.numel() * 2)}
 
-    cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        import oracle as orc
-
-        orc.build()
-        sel_gu = step.sel_gu.cpu().numpy()
-        sel_dn = step.sel_dn.cpu().numpy()
-        dt, f = oracle_sample(wl, sel_gu, sel_dn, args.cpu_pairs)
-        cpu = {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
-               "sample": f"{args.cpu_pairs} of {P} (token, expert) rows of one step, {dt:.1f} s"}
+    cpu = sp["cpu"]() if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
 
     if rank == 0:
+        config = dict(sp["config"])
+        config["l2"] = "flushed between timed steps (256 MiB write outside the per-step events)"
+        config["parallelism"] = f"replicas x{ws}"
         line = {
             "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step_ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 block scales) -> f32 accumulate",
             "data": "synthetic (seeded counter-based generator)",
-            "config": {"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P,
-                       "experts": wl.E, "hidden": wl.H, "intermediate": wl.I, "Kp_gate_up": wl.Kp_gu,
-                       "Kp_down": wl.Kp_dn, "rows_padded": step.rows_padded,
-                       "l2": "flushed between timed steps (256 MiB write outside the per-step events)",
-                       "parallelism": f"replicas x{ws}"},
+            "config": config,
             "fp4_peak_tflops": fp4_peak,
             "frac_fp4_peak": value / ws / fp4_peak,
             "kernel_ms": k_ms,
-            "act_quant_gbs": {"x": qx_bytes / (k_ms["quant_x"] * 1e-3) / 1e9,
-                              "h": qh_bytes / (k_ms["quant_h"] * 1e-3) / 1e9},
+            "act_quant_gbs": {k: b / (k_ms[s] * 1e-3) / 1e9 for k, (s, b) in sp["quant"].items()},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps,
+            "gpu_launches": sp["kernels_per_step"] * args.steps,
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)

@@ -105,6 +105,8 @@ int32_t nvfp4_kp_from_ratio(int64_t K, double r);
 /* Upper bound of the wait inside every device-side spin loop, in nanoseconds (default 2e9).
  * A wait that runs out sets NVFP4_ERR_TIMEOUT in *dev_status and the kernel returns. */
 void nvfp4_set_wait_limit_ns(uint64_t ns);
+/* Tuning: N-tile of the GEMM kernels, 128 or 256 (0 = automatic choice per shape). */
+void nvfp4_set_gemm_tile_n(int32_t n);
 
 /* ---------------------------------------------------------------------------------------- */
 /* nvfp4_quantize -- online activation quantisation with the RAC residual pass              */

@@ -18,6 +18,7 @@ namespace {
 
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
+std::atomic<int> g_tile_n{0};  // 0: automatic
 
 nvfp4_status fail(nvfp4_status s, const char* fmt, ...) {
   char buf[512];
@@ -79,6 +80,25 @@ nvfp4_status make_code_map(CUtensorMap* m, const void* base, uint64_t inner_byte
   return NVFP4_OK;
 }
 
+// Output matrix [rows x cols] (bf16 or fp32, row pitch ld elements) stored by the GEMM epilogue
+// in boxes of 32 rows x 128 bytes, 128-byte swizzle.  Rows beyond `rows` are clipped.
+nvfp4_status make_out_map(CUtensorMap* m, void* base, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld) {
+  auto fn = encode_fn();
+  if (!fn) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
+  const uint64_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * esz};
+  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return fail(NVFP4_ERR_CUDA, "tensor map for the output failed (error %d, cols %llu, rows %llu)", (int)r,
+                (unsigned long long)cols, (unsigned long long)rows);
+  return NVFP4_OK;
+}
+
 nvfp4_status check_tensor(const nvfp4_tensor* t, const char* name, int64_t cols, int64_t min_rows, int64_t slabs) {
   if (!t) return fail(NVFP4_ERR_INVALID_ARG, "%s is NULL", name);
   if (!t->codes || !t->sf || !t->s_g) return fail(NVFP4_ERR_INVALID_ARG, "%s has a NULL buffer", name);
@@ -92,9 +112,9 @@ nvfp4_status check_tensor(const nvfp4_tensor* t, const char* name, int64_t cols,
 }
 
 int act_partials(int64_t M, int64_t K) {
-  int64_t p = (M * K) / 65536;
+  int64_t p = (M * K) / 16384;
   if (p < 1) p = 1;
-  if (p > 256) p = 256;
+  if (p > 1024) p = 1024;
   return (int)p;
 }
 int slab_partials(int64_t slabs) {
@@ -102,6 +122,17 @@ int slab_partials(int64_t slabs) {
   return (int)(p < 1 ? 1 : p);
 }
 size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// N-tile of the GEMM: 256 (one accumulator, best MMA / scale-copy ratio) unless forced or N
+// is not a multiple of 256.
+int choose_tile_n(int64_t N, int64_t K, int64_t Kp) {
+  (void)K;
+  (void)Kp;
+  const int forced = g_tile_n.load();
+  if (forced == 128) return 128;
+  if (forced == 256 && N % 256 == 0) return 256;
+  return (N % 256 == 0) ? 256 : 128;
+}
 
 }  // namespace
 
@@ -140,11 +171,13 @@ int32_t nvfp4_kp_from_ratio(int64_t K, double r) {
 
 void nvfp4_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 
+void nvfp4_set_gemm_tile_n(int32_t n) { g_tile_n.store((n == 128 || n == 256) ? n : 0); }
+
 // ------------------------------------------------------------------------------------------ quantize
 size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K) {
   (void)M;
   (void)K;
-  return 256 * sizeof(float);
+  return 1024 * sizeof(float);
 }
 
 nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
@@ -271,7 +304,7 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
 
 // ------------------------------------------------------------------------------------------ calibrate
 size_t rac_calibrate_workspace_size(int64_t T, int64_t K) {
-  return round_up(256 * sizeof(float), 256) + round_up((size_t)T * (size_t)K * sizeof(float), 256) +
+  return round_up(1024 * sizeof(float), 256) + round_up((size_t)T * (size_t)K * sizeof(float), 256) +
          round_up((size_t)K * sizeof(double), 256);
 }
 
@@ -289,8 +322,8 @@ nvfp4_status rac_calibrate(const uint16_t* x_cal, int64_t T, int64_t K, int32_t 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* ws = reinterpret_cast<char*>(workspace);
   float* partial = reinterpret_cast<float*>(ws);
-  float* resid = reinterpret_cast<float*>(ws + round_up(256 * sizeof(float), 256));
-  double* err = reinterpret_cast<double*>(ws + round_up(256 * sizeof(float), 256) +
+  float* resid = reinterpret_cast<float*>(ws + round_up(1024 * sizeof(float), 256));
+  double* err = reinterpret_cast<double*>(ws + round_up(1024 * sizeof(float), 256) +
                                           round_up((size_t)T * (size_t)K * sizeof(float), 256));
   const int P = act_partials(T, K);
   cudaError_t e = launch_amax(x_cal, 1, T, K, K, partial, P, dev_status, s);
@@ -383,8 +416,8 @@ nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, co
 // ------------------------------------------------------------------------------------------ GEMMs
 static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
                                 const nvfp4_tensor* w_sel, int64_t rows_needed, int64_t N, int64_t K, int32_t Kp,
-                                int64_t E, nvfp4_dtype out, void* y, int64_t ldy, int64_t y_cols, int bn,
-                                CUtensorMap* maps, GemmArgs* g) {
+                                int64_t E, nvfp4_dtype out, void* y, int64_t ldy, int64_t y_cols, int64_t y_rows,
+                                int bn, CUtensorMap* maps, GemmArgs* g) {
   if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
   if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp must be a multiple of 64 in [0, K]");
   if (N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "N must be a positive multiple of 128");
@@ -406,7 +439,11 @@ static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res
     if (st != NVFP4_OK) return st;
     if (w_sel->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_sel.rows_padded must equal N");
   }
-  memset(maps, 0, 4 * sizeof(CUtensorMap));
+  memset(maps, 0, 5 * sizeof(CUtensorMap));
+  if (y_rows > 0) {
+    st = make_out_map(&maps[4], y, out == NVFP4_OUT_BF16, (uint64_t)y_cols, (uint64_t)y_rows, (uint64_t)ldy);
+    if (st != NVFP4_OK) return st;
+  }
   st = make_code_map(&maps[0], a->codes, (uint64_t)K / 2, (uint64_t)a->rows_padded, 1, 128, 2, "A");
   if (st != NVFP4_OK) return st;
   st = make_code_map(&maps[2], w->codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, (uint32_t)bn, 3, "W");
@@ -448,10 +485,10 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, con
                            void* y, int64_t ldy, int32_t* dev_status, void* stream) {
   g_last_error.clear();
   if (M < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M must be >= 0");
-  const int bn = (N % 256 == 0) ? 256 : 128;
-  CUtensorMap maps[4];
+  const int bn = choose_tile_n(N, K, Kp);
+  CUtensorMap maps[5];
   GemmArgs g;
-  nvfp4_status st = gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, bn, maps, &g);
+  nvfp4_status st = gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, M, bn, maps, &g);
   if (st != NVFP4_OK) return st;
   if (M == 0) return NVFP4_OK;
   g.offsets = nullptr;
@@ -462,7 +499,8 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, con
   g.status = dev_status;
   int64_t tiles = (int64_t)g.m_blocks_dense * g.n_blocks;
   int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], g, grid, reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, grid,
+                              reinterpret_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return NVFP4_OK;
 }
@@ -479,11 +517,14 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
     if (out != NVFP4_OUT_BF16) return fail(NVFP4_ERR_INVALID_ARG, "the SwiGLU epilogue writes bf16");
     if (!amax_out) return fail(NVFP4_ERR_INVALID_ARG, "amax_out is NULL with the SwiGLU epilogue");
   }
-  const int bn = (N % 256 == 0) ? 256 : 128;
-  CUtensorMap maps[4];
+  if (ep == NVFP4_EPI_SWIGLU_AMAX && N % 256 != 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the SwiGLU epilogue needs N %% 256 == 0");
+  const int bn = ep == NVFP4_EPI_SWIGLU_AMAX ? 256 : choose_tile_n(N, K, Kp);
+  CUtensorMap maps[5];
   GemmArgs g;
   const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
-  nvfp4_status st = gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, bn, maps, &g);
+  nvfp4_status st =
+      gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, a ? a->rows_padded : 0, bn, maps, &g);
   if (st != NVFP4_OK) return st;
   g.offsets = expert_offsets;
   g.E = E;
@@ -497,7 +538,7 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
     cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
     if (e != cudaSuccess) return cuda_fail(e, "amax reset");
   }
-  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], g, num_sms(), s);
+  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "grouped gemm launch");
   return NVFP4_OK;
 }

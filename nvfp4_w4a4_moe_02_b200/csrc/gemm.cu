@@ -32,26 +32,38 @@ constexpr int NUM_THREADS = 320;  // producer warp, MMA warp, 8 epilogue warps
 
 template <int BN>
 struct Cfg {
-  static constexpr int STAGES = (BN == 256) ? 4 : 6;
+  static constexpr int STAGES = (BN == 256) ? 3 : 5;
+  // epilogue staging: per epilogue warp, STG boxes of 32 rows x 128 bytes for TMA stores
+  static constexpr int STG = (BN == 256) ? 2 : 1;
+  static constexpr int BOX_BYTES = 32 * 128;
   static constexpr int A_BYTES = BM * KT_BYTES;
   static constexpr int B_BYTES = BN * KT_BYTES;
   static constexpr int SFA_BYTES = 4 * 512;
   static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
-  static constexpr int ACC_STAGES = (BN == 256) ? 1 : 2;
-  static constexpr int SF_COLS_A = 16;
-  static constexpr int SF_COLS_B = 16 * (BN / 128);
-  static constexpr int SF_COLS = SF_COLS_A + SF_COLS_B;
-  static constexpr int ACC_COLS = ACC_STAGES * BN;
+  // Tensor memory: two accumulator buffers and two per-MMA scale slots (A: 4 columns, B: 4
+  // per 128 columns of N).  The tensor pipe executes copies and MMAs of one thread in order,
+  // so a scale slot can be rewritten for the next-but-one MMA.  With BN = 256 the buffers
+  // overlap: buffer 1 starts ACC_OVERLAP columns before buffer 0 ends, and the epilogue drains
+  // that strip first and releases it early.
+  static constexpr int SF_SLOT = 4 + 4 * (BN / 128);
+  static constexpr int SF_COLS = 2 * SF_SLOT;
   static constexpr int TMEM_COLS = 512;
-  static_assert(ACC_COLS + STAGES * SF_COLS <= TMEM_COLS, "tensor memory budget");
+  static constexpr int ACC_OVERLAP = (2 * BN + SF_COLS > TMEM_COLS) ? (2 * BN + SF_COLS - TMEM_COLS) : 0;
+  static constexpr int ACC1_BASE = BN - ACC_OVERLAP;
+  static constexpr int SF_BASE = ACC1_BASE + BN;
+  static_assert(SF_BASE + SF_COLS <= TMEM_COLS, "tensor memory budget");
+  static_assert(ACC_OVERLAP <= 32, "the shared strip must lie in one 32-column chunk");
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_BAR = OFF_SFB + STAGES * SFB_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_STAGES + 1;
+  static constexpr int OFF_STG = OFF_SFB + STAGES * SFB_BYTES;  // 1024-aligned
+  static constexpr int OFF_BAR = OFF_STG + 8 * STG * BOX_BYTES;
+  // full[S], empty[S], accf[2], acce[2], ovf[2], drain
+  static constexpr int NUM_BARS = 2 * STAGES + 7;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
-  static constexpr int SMEM = OFF_MISC + 32 + 1024;
+  // the dynamic shared window starts 1024-byte aligned (checked in the kernel)
+  static constexpr int SMEM = OFF_MISC + 32;
   static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -67,23 +79,28 @@ __device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+// try_wait with a suspend-time hint: the waiting thread sleeps in hardware until the phase
+// completes or the hint (ns) expires, instead of spinning and taking issue slots from the
+// MMA-issuing and copy-issuing threads.
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity, uint32_t hint_ns) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
-// Bounded wait: false when the limit ran out or another role already aborted.
+// Bounded wait: false when the limit ran out or another role already aborted.  The clock is
+// read only after a try that came back unfinished.
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns, volatile int* abort_flag) {
-  if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = limit_ns < 1000000ull ? (uint32_t)limit_ns : 1000000u;
+  if (mbar_try_wait(bar, parity, hint)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait(bar, parity, hint)) return true;
     if (abort_flag != nullptr && *abort_flag) return false;
     if (globaltimer_ns() - t0 > limit_ns) return false;
   }
@@ -108,6 +125,23 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(src), "r"(bytes), "r"(bar)
                : "memory");
+}
+
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_group_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_group_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
@@ -187,20 +221,24 @@ template <int BN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_ar,
                          const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_ws,
-                         const GemmArgs args) {
+                         const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
   using C = Cfg<BN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  const uint32_t raw_addr = smem_u32(smem_raw);
-  const uint32_t sbase = (raw_addr + 1023u) & ~1023u;
-  unsigned char* smem = smem_raw + (sbase - raw_addr);
+  const uint32_t sbase = smem_u32(smem_raw);
+  unsigned char* smem = smem_raw;
+  if ((sbase & 1023u) != 0) {  // the swizzled tiles need a 1024-byte aligned window
+    if (threadIdx.x == 0) report_status(args.status, kErrAlign);
+    return;
+  }
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   auto bar_full = [&](int s) { return sbase + C::OFF_BAR + 8u * s; };
   auto bar_empty = [&](int s) { return sbase + C::OFF_BAR + 8u * (C::STAGES + s); };
-  auto bar_accf = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + a); };
-  auto bar_acce = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + C::ACC_STAGES + a); };
-  const uint32_t bar_drain = sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 2 * C::ACC_STAGES);
+  auto bar_accf = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + a); };      // accumulator ready
+  auto bar_acce = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 2 + a); };  // fully drained
+  auto bar_ovf = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 4 + a); };   // shared strip drained
+  const uint32_t bar_drain = sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 6);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* prod_issued = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
@@ -211,9 +249,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), 1);
     }
-    for (int a = 0; a < C::ACC_STAGES; ++a) {
+    for (int a = 0; a < 2; ++a) {
       mbar_init(bar_accf(a), 1);
       mbar_init(bar_acce(a), 8);
+      mbar_init(bar_ovf(a), 4);
     }
     mbar_init(bar_drain, 1);
     *abort_flag = 0;
@@ -303,17 +342,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr uint32_t idesc = idesc_fp4(BM, BN);
       int stage = 0;
       uint32_t phase = 0;
-      int acc = 0;
-      uint32_t acc_phase = 0;
       int taken = 0;
+      uint32_t mma_count = 0;
       bool ok = true;
-      for (int64_t t = blockIdx.x; t < total_tiles && ok && !*abort_flag; t += gridDim.x) {
-        if (!mbar_wait(bar_acce(acc), acc_phase ^ 1u, limit, abort_flag)) {
+      int64_t tile_idx = 0;
+      for (int64_t t = blockIdx.x; t < total_tiles && ok && !*abort_flag; t += gridDim.x, ++tile_idx) {
+        const int acc = (int)(tile_idx & 1);
+        const int64_t use = tile_idx >> 1;  // how many times buffer `acc` was used before
+        // buffer `acc` fully drained by the epilogue of its previous tile
+        if (use >= 1 && !mbar_wait(bar_acce(acc), (uint32_t)((use - 1) & 1), limit, abort_flag)) {
+          ok = false;
+          break;
+        }
+        // the strip shared with the other buffer drained by the epilogue of the previous tile
+        if (C::ACC_OVERLAP > 0 && tile_idx >= 1 &&
+            !mbar_wait(bar_ovf(acc ^ 1), (uint32_t)(((tile_idx - 1) >> 1) & 1), limit, abort_flag)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc ? C::ACC1_BASE : 0);
         for (int kt = 0; kt < kt_total; ++kt) {
           if (!mbar_wait(bar_full(stage), phase, limit, abort_flag)) {
             ok = false;
@@ -326,21 +374,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int kk = res ? kt - args.kt_main : kt;
           const int k64 = res ? args.k64_res : args.k64_main;
           const int nk64 = min(4, k64 - kk * 4);
-          const uint32_t sfa_t = tmem_base + (uint32_t)(C::ACC_COLS + stage * C::SF_COLS);
-          const uint32_t sfb_t = sfa_t + C::SF_COLS_A;
           const uint32_t a_s = sbase + C::OFF_A + stage * C::A_BYTES;
           const uint32_t b_s = sbase + C::OFF_B + stage * C::B_BYTES;
           const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_BYTES;
           const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_BYTES;
-          for (int j = 0; j < nk64; ++j) {
-            tc_copy_sf(sfa_t + 4 * j, desc_sf(sfa_s + j * 512));
+          // each MMA's scale atoms are copied right before it (into alternating slots): the
+          // tensor pipe overlaps the copies with the preceding MMA
+          for (int j = 0; j < nk64; ++j, ++mma_count) {
+            const uint32_t sfa_t = tmem_base + (uint32_t)(C::SF_BASE + (mma_count & 1) * C::SF_SLOT);
+            const uint32_t sfb_t = sfa_t + 4;
+            tc_copy_sf(sfa_t, desc_sf(sfa_s + j * 512));
 #pragma unroll
-            for (int rb = 0; rb < BN / 128; ++rb)
-              tc_copy_sf(sfb_t + j * 4 * (BN / 128) + 4 * rb, desc_sf(sfb_s + rb * 2048 + j * 512));
-          }
-          for (int j = 0; j < nk64; ++j) {
-            tc_mma_fp4(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, sfa_t + 4 * j,
-                       sfb_t + j * 4 * (BN / 128), (kt | j) != 0 ? 1u : 0u);
+            for (int rb = 0; rb < BN / 128; ++rb) tc_copy_sf(sfb_t + 4 * rb, desc_sf(sfb_s + rb * 2048 + j * 512));
+            tc_mma_fp4(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, sfa_t, sfb_t,
+                       (kt | j) != 0 ? 1u : 0u);
           }
           tc_commit(bar_empty(stage));
           if (++stage == C::STAGES) {
@@ -350,10 +397,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         }
         if (!ok) break;
         tc_commit(bar_accf(acc));
-        if (++acc == C::ACC_STAGES) {
-          acc = 0;
-          acc_phase ^= 1u;
-        }
       }
       if (!ok) {
         report_status(args.status, kErrTimeout);
@@ -368,10 +411,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     constexpr int NCH = BN / 64;            // 32-column chunks per warp
     const int quad = warp & 3;              // tensor-memory lanes [32*quad, 32*quad + 32)
     const int half = (warp - 2) >> 2;       // which half of the tile's columns
-    int acc = 0;
-    uint32_t acc_phase = 0;
     float amax = 0.0f;
-    for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x) {
+    int64_t tile_idx = 0;
+    for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tile_idx) {
+      const int acc = (int)(tile_idx & 1);
+      const uint32_t acc_phase = (uint32_t)((tile_idx >> 1) & 1);
       const int64_t mb = t / args.n_blocks;
       const int nb = (int)(t - mb * args.n_blocks);
       const int e = grouped ? find_expert(args.offsets, args.E, mb * BM) : 0;
@@ -389,87 +433,104 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int64_t row = mb * BM + quad * 32 + lane;
       const bool row_ok = row < row_limit && row < args.rows_capacity;
       const float alpha = __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));
-      const uint32_t t_row = tmem_base + (uint32_t)(acc * BN) + ((uint32_t)(quad * 32) << 16);
-      uint32_t v[NCH][32];
-      if (args.epi == 0) {
-#pragma unroll
-        for (int i = 0; i < NCH; ++i) tmem_ld32(t_row + half * (BN / 2) + 32 * i, v[i]);
-      } else {
-        // SwiGLU: output feature f of the tile reads gate column (f/64)*128 + f%64 and the up
-        // column 64 further (gate/up interleave of the packed weight); this warp owns
-        // features [half*BN/4, (half+1)*BN/4): chunks 0..NCH/2-1 gate, NCH/2.. up.
-#pragma unroll
-        for (int i = 0; i < NCH / 2; ++i) {
-          const int f = half * (BN / 4) + 32 * i;
-          const int gcol = (f / 64) * 128 + (f % 64);
-          tmem_ld32(t_row + gcol, v[i]);
-          tmem_ld32(t_row + gcol + 64, v[NCH / 2 + i]);
-        }
+      const uint32_t t_row = tmem_base + (uint32_t)(acc ? C::ACC1_BASE : 0) + ((uint32_t)(quad * 32) << 16);
+      // chunk i of this warp: plain -> columns half*BN/2 + 32i; SwiGLU -> output features
+      // [half*BN/4, ...): chunks 0..NCH/2-1 gate (column (f/64)*128 + f%64), NCH/2.. the up
+      // columns 64 further (gate/up interleave of the packed weight)
+      auto chunk_col = [&](int i) -> int {
+        if (args.epi == 0) return half * (BN / 2) + 32 * i;
+        const int ii = i % (NCH / 2);
+        const int f = half * (BN / 4) + 32 * ii;
+        return (f / 64) * 128 + (f % 64) + (i >= NCH / 2 ? 64 : 0);
+      };
+      // the chunk holding the strip shared with the other buffer is drained and released first
+      int ovl_i = -1;
+      if (C::ACC_OVERLAP > 0) {
+        if (acc == 0 && half == 1) ovl_i = NCH - 1;  // buffer 0: its last columns
+        if (acc == 1 && half == 0) ovl_i = 0;        // buffer 1: its first columns
       }
+      uint32_t v[NCH][32];
+      if (ovl_i >= 0) {
+#pragma unroll
+        for (int i = 0; i < NCH; ++i)
+          if (i == ovl_i) tmem_ld32(t_row + chunk_col(i), v[i]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_ovf(acc));
+      }
+#pragma unroll
+      for (int i = 0; i < NCH; ++i)
+        if (i != ovl_i) tmem_ld32(t_row + chunk_col(i), v[i]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_acce(acc));
-      if (++acc == C::ACC_STAGES) {
-        acc = 0;
-        acc_phase ^= 1u;
-      }
-      if (!row_ok) continue;
-      if (args.epi == 0) {
-        const int64_t col0 = (int64_t)nb * BN + half * (BN / 2);
-        if (args.out_bf16) {
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy + col0);
+      // ---- output through shared memory: each box is 32 rows x 128 bytes in the 128-byte
+      // swizzled layout (16-byte chunk c of row r at chunk c ^ (r % 8)), stored by one TMA copy
+      const uint32_t stg = sbase + C::OFF_STG + (uint32_t)((warp - 2) * C::STG * C::BOX_BYTES);
+      const int32_t y0 = (int32_t)(mb * BM + quad * 32);
+      auto put_box = [&](int slot, const uint32_t (&w)[32], int32_t x) {
+        // at most STG - 1 earlier stores of this warp may still be reading the staging boxes
+        if (lane == 0) bulk_wait_group_read<C::STG - 1>();
+        __syncwarp();
+        const uint32_t rowp = stg + (uint32_t)(slot * C::BOX_BYTES + lane * 128);
 #pragma unroll
-          for (int i = 0; i < NCH; ++i)
+        for (int c = 0; c < 8; ++c)
+          st_shared_v4(rowp + (uint32_t)(((c ^ (lane & 7)) * 16)), w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, stg + (uint32_t)(slot * C::BOX_BYTES), x, y0);
+          bulk_commit_group();
+        }
+      };
+      if (args.epi == 0 && args.out_bf16) {
+        // 64 columns per box
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              uint32_t p[4];
+        for (int b = 0; b < NCH / 2; ++b) {
+          uint32_t w[32];
 #pragma unroll
-              for (int h = 0; h < 4; ++h)
-                p[h] = pack_bf16x2(__fmul_rn(__uint_as_float(v[i][8 * q + 2 * h]), alpha),
-                                   __fmul_rn(__uint_as_float(v[i][8 * q + 2 * h + 1]), alpha));
-              dst[4 * i + q] = make_uint4(p[0], p[1], p[2], p[3]);
-            }
-        } else {
-          float4* dst = reinterpret_cast<float4*>(reinterpret_cast<float*>(args.y) + row * args.ldy + col0);
+          for (int h = 0; h < 2; ++h)
 #pragma unroll
-          for (int i = 0; i < NCH; ++i)
+            for (int k = 0; k < 16; ++k)
+              w[16 * h + k] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * b + h][2 * k]), alpha),
+                                          __fmul_rn(__uint_as_float(v[2 * b + h][2 * k + 1]), alpha));
+          put_box(b % C::STG, w, (int32_t)(nb * BN + half * (BN / 2) + 64 * b));
+        }
+      } else if (args.epi == 0) {
+        // fp32: 32 columns per box
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              dst[8 * i + q] = make_float4(__fmul_rn(__uint_as_float(v[i][4 * q]), alpha),
-                                           __fmul_rn(__uint_as_float(v[i][4 * q + 1]), alpha),
-                                           __fmul_rn(__uint_as_float(v[i][4 * q + 2]), alpha),
-                                           __fmul_rn(__uint_as_float(v[i][4 * q + 3]), alpha));
+        for (int b = 0; b < NCH; ++b) {
+          uint32_t w[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__fmul_rn(__uint_as_float(v[b][k]), alpha));
+          put_box(b % C::STG, w, (int32_t)(nb * BN + half * (BN / 2) + 32 * b));
         }
       } else {
+        // SwiGLU (BN = 256): this warp's 64 output features form one box
+        uint32_t w[32];
 #pragma unroll
-        for (int i = 0; i < NCH / 2; ++i) {
-          const int f = half * (BN / 4) + 32 * i;  // first output feature of this chunk
-          uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<uint16_t*>(args.y) + row * args.ldy +
-                                                (int64_t)nb * (BN / 2) + f);
+        for (int i = 0; i < NCH / 2; ++i)
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t p[4];
+          for (int k = 0; k < 16; ++k) {
+            float hv[2];
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              float hv[2];
-#pragma unroll
-              for (int z = 0; z < 2; ++z) {
-                const int j = 8 * q + 2 * h + z;
-                const float gv = bf16_round(__fmul_rn(__uint_as_float(v[i][j]), alpha));
-                const float uv = bf16_round(__fmul_rn(__uint_as_float(v[NCH / 2 + i][j]), alpha));
-                // silu(g) = g / (1 + e^-g); e^-g overflowing to inf gives -0 (the limit)
-                const float sg = __fdividef(gv, 1.0f + __expf(-gv));
-                hv[z] = bf16_round(sg * uv);
-                amax = fmaxf(amax, fabsf(hv[z]));
-              }
-              p[h] = pack_bf16x2(hv[0], hv[1]);
+            for (int z = 0; z < 2; ++z) {
+              const int j = 2 * k + z;
+              const float gv = bf16_round(__fmul_rn(__uint_as_float(v[i][j]), alpha));
+              const float uv = bf16_round(__fmul_rn(__uint_as_float(v[NCH / 2 + i][j]), alpha));
+              // silu(g) = g / (1 + e^-g); e^-g overflowing to inf gives -0 (the limit)
+              const float sg = __fdividef(gv, 1.0f + __expf(-gv));
+              hv[z] = bf16_round(sg * uv);
+              if (row_ok) amax = fmaxf(amax, fabsf(hv[z]));
             }
-            dst[q] = make_uint4(p[0], p[1], p[2], p[3]);
+            w[16 * i + k] = pack_bf16x2(hv[0], hv[1]);
           }
-        }
+        put_box(0, w, (int32_t)(nb * (BN / 2) + half * (BN / 4)));
       }
     }
+    if (lane == 0) bulk_wait_group_all();  // this warp's stores complete before exit
     if (args.epi != 0 && args.amax_out != nullptr) {
       amax = warp_max(amax);
       if (lane == 0 && amax > 0.0f) atomicMax(reinterpret_cast<unsigned int*>(args.amax_out), __float_as_uint(amax));
@@ -515,18 +576,19 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, int32_t* status) {
 size_t gemm_smem_bytes(int bn) { return bn == 256 ? (size_t)tc::Cfg<256>::SMEM : (size_t)tc::Cfg<128>::SMEM; }
 
 cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
-                        const CUtensorMap& tm_ws, const GemmArgs& args, int grid, cudaStream_t st) {
+                        const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
+                        cudaStream_t st) {
   cudaError_t e;
   if (bn == 256) {
     e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tc::Cfg<256>::SMEM);
     if (e != cudaSuccess) return e;
-    tc::w4a4_rac_gemm_kernel<256><<<grid, tc::NUM_THREADS, tc::Cfg<256>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, args);
+    tc::w4a4_rac_gemm_kernel<256><<<grid, tc::NUM_THREADS, tc::Cfg<256>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args);
   } else if (bn == 128) {
     e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              tc::Cfg<128>::SMEM);
     if (e != cudaSuccess) return e;
-    tc::w4a4_rac_gemm_kernel<128><<<grid, tc::NUM_THREADS, tc::Cfg<128>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, args);
+    tc::w4a4_rac_gemm_kernel<128><<<grid, tc::NUM_THREADS, tc::Cfg<128>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args);
   } else {
     return cudaErrorInvalidValue;
   }

@@ -84,7 +84,8 @@ struct GemmArgs {
 
 // bn: 128 or 256
 cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
-                        const CUtensorMap& tm_ws, const GemmArgs& args, int grid, cudaStream_t st);
+                        const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
+                        cudaStream_t st);
 size_t gemm_smem_bytes(int bn);
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t st);

@@ -21,18 +21,24 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
   bool bad = false;
   const uint16_t* base = x + seg * seg_rows * ld;
   if (ld == cols) {
-    // contiguous segment: flat vector loop
+    // contiguous segment: flat vector loop, four independent 16-byte loads in flight per thread
     const int64_t nvec = seg_rows * cols / 8;
     const uint4* v = reinterpret_cast<const uint4*>(base);
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nvec; i += (int64_t)P * blockDim.x) {
-      uint4 q = __ldg(v + i);
-      uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    const int64_t stride = (int64_t)P * blockDim.x;
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < nvec; i0 += 4 * stride) {
+      uint4 q[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float a = fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu));
-        float b = fabsf(bf16_bits_to_f32(w[j] >> 16));
-        bad |= !(a <= 3.4e38f) || !(b <= 3.4e38f);
-        m = fmaxf(m, fmaxf(a, b));
+      for (int u = 0; u < 4; ++u) q[u] = (i0 + u * stride < nvec) ? __ldg(v + i0 + u * stride) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float a = fabsf(bf16_bits_to_f32(w[j] & 0xFFFFu));
+          float b = fabsf(bf16_bits_to_f32(w[j] >> 16));
+          bad |= !(a <= 3.4e38f) || !(b <= 3.4e38f);
+          m = fmaxf(m, fmaxf(a, b));
+        }
       }
     }
   } else {
@@ -109,6 +115,15 @@ __device__ __forceinline__ void load8(const uint16_t* p, bool ok, float x[8], ui
   }
 }
 
+__device__ __forceinline__ void unpack8(const uint4 raw, float x[8]) {
+  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    x[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
+    x[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
+  }
+}
+
 __device__ __forceinline__ float pair_max8(const float x[8]) {
   float m = 0.0f;
 #pragma unroll
@@ -117,7 +132,7 @@ __device__ __forceinline__ float pair_max8(const float x[8]) {
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(256) quant_rows_kernel(const RowArgs a) {
+__global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -183,14 +198,21 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(const RowArgs a) {
     }
     const uint16_t* srow = a.src + slab * a.src_slab_stride + (valid ? src_row : 0) * a.ld;
 
-    // ---- main pass
+    // ---- main pass (the loads of the next 512 elements are issued before this block's math)
+    uint4 n0 = (valid && 8 * lane < K) ? __ldg(reinterpret_cast<const uint4*>(srow + 8 * lane)) : make_uint4(0, 0, 0, 0);
+    uint4 n1 = (valid && 256 + 8 * lane < K) ? __ldg(reinterpret_cast<const uint4*>(srow + 256 + 8 * lane))
+                                             : make_uint4(0, 0, 0, 0);
     for (int64_t base = 0; base < K; base += 512) {
       const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
       const bool h0 = e0 < K, h1 = e1 < K;  // K % 64 == 0: uniform over lane pairs and 8-lane groups
+      const uint4 r0 = n0, r1 = n1;
+      if (base + 512 < K) {
+        n0 = (valid && e0 + 512 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + e0 + 512)) : make_uint4(0, 0, 0, 0);
+        n1 = (valid && e1 + 512 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + e1 + 512)) : make_uint4(0, 0, 0, 0);
+      }
       float x0[8], x1[8];
-      uint4 r0, r1;
-      load8(srow + e0, valid && h0, x0, r0);
-      load8(srow + e1, valid && h1, x1, r1);
+      unpack8(r0, x0);
+      unpack8(r1, x1);
       const BlockScale b0 = block_scale(pair_max8(x0), s_g, t6);
       const BlockScale b1 = block_scale(pair_max8(x1), s_g, t6);
       if (MODE == kModeCal) {

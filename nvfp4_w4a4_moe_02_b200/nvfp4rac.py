@@ -59,6 +59,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_sf_bytes": ([i64, i64], sz),
         "nvfp4_kp_from_ratio": ([i64, ctypes.c_double], i32),
         "nvfp4_set_wait_limit_ns": ([u64], None),
+        "nvfp4_set_gemm_tile_n": ([i32], None),
         "nvfp4_quantize_workspace_size": ([i64, i64], sz),
         "nvfp4_quantize": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
         "nvfp4_quantize_scatter": ([vp, i64, i64, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
@@ -172,6 +173,11 @@ def kp_from_ratio(K: int, r: float) -> int:
 
 def set_wait_limit_ns(ns: int):
     load().nvfp4_set_wait_limit_ns(ns)
+
+
+def set_gemm_tile_n(n: int):
+    """Force the GEMM N-tile (128 or 256); 0 restores the automatic choice."""
+    load().nvfp4_set_gemm_tile_n(n)
 
 
 # ------------------------------------------------------------------------------------- calls
