@@ -171,6 +171,83 @@ class DenseStep:
         return self.y
 
 
+class DecodeStep:
+    """MoE decode step: 64 tokens routed top-8 over 256 experts; each expert's tokens gathered into
+    16-token slabs; swap-AB decode GEMMs stream the touched experts' packed weights."""
+
+    KERNELS_PER_STEP = 5  # amax, quantise X, decode gate_up, quantise h, decode down
+
+    def __init__(self, wl, dev):
+        import torch
+
+        from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+        from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+        self.R, self.torch, self.wl = R, torch, wl
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+        self.status = R.new_status(dev)
+        # offline: channel selection, then the pack of every expert (weights made on the device)
+        self.sel_gu, _ = R.rac_calibrate(to(wl.x_cal), wl.Kp_gu, status=self.status)
+        h_cal = syn.moe_down_calibration_batch_torch(wl, dev)
+        self.sel_dn, _ = R.rac_calibrate(to(h_cal), wl.Kp_dn, status=self.status)
+        N_gu = 2 * wl.I
+        P = R.Packed
+        self.pgu = P.empty(N_gu, wl.H, slabs=wl.E, rows_padded=N_gu, device=dev)
+        self.pgus = P.empty(N_gu, wl.Kp_gu, slabs=wl.E, rows_padded=N_gu, device=dev)
+        self.pdn = P.empty(wl.H, wl.I, slabs=wl.E, rows_padded=wl.H, device=dev)
+        self.pdns = P.empty(wl.H, wl.Kp_dn, slabs=wl.E, rows_padded=wl.H, device=dev)
+        wbuf = torch.empty(N_gu, wl.H, dtype=torch.bfloat16, device=dev)
+        dbuf = torch.empty(wl.H, wl.I, dtype=torch.bfloat16, device=dev)
+        for e in range(wl.E):
+            R.pack_weights(wl.gate_up_expert_torch(e, dev, out=wbuf), self.sel_gu, gate_up_interleave=True,
+                           out=self.pgu.slab(e), out_sel=self.pgus.slab(e), status=self.status)
+            R.pack_weights(wl.down_expert_torch(e, dev, out=dbuf), self.sel_dn, out=self.pdn.slab(e),
+                           out_sel=self.pdns.slab(e), status=self.status)
+        del wbuf, dbuf
+        se, sc, pair_rows = R.decode_slots(wl.counts)
+        self.n_slots = int(se.size)
+        self.rows = 16 * self.n_slots
+        self.slot_expert = torch.from_numpy(se).to(dev)
+        self.slot_count = torch.from_numpy(sc).to(dev)
+        self.scatter = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0],
+                                                      wl.topk_ids.shape[1])).to(dev)
+        self.x = to(wl.x)
+        S16 = R.SF_SLAB16
+        # rows of a slab past its count are never named by the scatter map: zero them once
+        self.a = P.empty(self.rows, wl.H, rows_padded=self.rows, device=dev, zero=True, sf_layout=S16)
+        self.ar = P.empty(self.rows, wl.Kp_gu, rows_padded=self.rows, device=dev, zero=True, sf_layout=S16)
+        self.h = torch.empty(self.rows, wl.I, dtype=torch.bfloat16, device=dev)
+        self.amax_h = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.hq = P.empty(self.rows, wl.I, rows_padded=self.rows, device=dev, sf_layout=S16)
+        self.hqr = P.empty(self.rows, wl.Kp_dn, rows_padded=self.rows, device=dev, sf_layout=S16)
+        self.y = torch.empty(self.rows, wl.H, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        R.check_status(self.status)
+        torch.cuda.empty_cache()
+
+    def run(self, x=None, events=None):
+        R = self.R
+        ev = events or {}
+        if "q0" in ev:
+            ev["q0"].record()
+        R.nvfp4_quantize_scatter(self.x if x is None else x, self.scatter, self.rows, self.sel_gu, out=self.a,
+                                 out_res=self.ar, status=self.status)
+        if "g0" in ev:
+            ev["g0"].record()
+        R.grouped_w4a4_rac_moe_decode(self.a, self.ar, self.slot_expert, self.slot_count, self.pgu, self.pgus,
+                                      swiglu=True, y=self.h, amax_out=self.amax_h, status=self.status)
+        if "q1" in ev:
+            ev["q1"].record()
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        if "d0" in ev:
+            ev["d0"].record()
+        R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.slot_expert, self.slot_count, self.pdn, self.pdns,
+                                      y=self.y, status=self.status)
+        if "end" in ev:
+            ev["end"].record()
+        return self.y
+
+
 # ------------------------------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples every 50 ms; samples are kept for the wall-clock
@@ -250,8 +327,9 @@ def oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=0):
         idx = pairs[wl.pair_expert[pairs] == e]
         xa = wl.x[wl.pair_token[idx]]
         ac, aS, rc, rS, _ = orc.act_quant_rac(xa, s_x, sel_gu)
-        s_w = orc.global_scale(orc.amax_bf16(wl.wgu[e]))
-        wc, wS, wsc, wsS = orc.weight_pack(wl.wgu[e], s_w, sel_gu)
+        wgu = wl.gate_up_expert(int(e))
+        s_w = orc.global_scale(orc.amax_bf16(wgu))
+        wc, wS, wsc, wsS = orc.weight_pack(wgu, s_w, sel_gu)
         gu, _ = orc.gemm_rac(ac, aS, rc, rS, wc, wS, wsc, wsS, s_x, s_w)
         gu_b = orc.f64_to_bf16_array(gu)
         h, _ = orc.swiglu(gu_b)
@@ -262,8 +340,9 @@ def oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=0):
     start = 0
     for e, n in exps:
         hc, hS, hrc, hrS, _ = orc.act_quant_rac(hh[start:start + n], s_h, sel_dn)
-        s_w = orc.global_scale(orc.amax_bf16(wl.wdn[e]))
-        dc, dS, dsc, dsS = orc.weight_pack(wl.wdn[e], s_w, sel_dn)
+        wdn = wl.down_expert(int(e))
+        s_w = orc.global_scale(orc.amax_bf16(wdn))
+        dc, dS, dsc, dsS = orc.weight_pack(wdn, s_w, sel_dn)
         orc.gemm_rac(hc, hS, hrc, hrS, dc, dS, dsc, dsS, s_h, s_w)
         start += n
     dt = time.perf_counter() - t0
@@ -363,7 +442,46 @@ def spec_dense(dev, args, peaks):
         cpu=cpu_leg, kernels_per_step=DenseStep.KERNELS_PER_STEP)
 
 
-SPECS = {"moe_prefill": spec_moe, "dense": spec_dense}
+def spec_decode(dev, args, peaks):
+    from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+    wl = syn.moe_decode()
+    step = DecodeStep(wl, dev)
+    gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
+    P = int(wl.pair_token.size)
+    touched = int((wl.counts > 0).sum())
+    # algorithmic bytes: each touched expert's packed W + W_sel once, the slab activations once,
+    # the output once
+    gu_w = touched * 2 * wl.I * (wl.H + wl.Kp_gu) * 0.5625
+    dn_w = touched * wl.H * (wl.I + wl.Kp_dn) * 0.5625
+    gu_bytes = gu_w + step.rows * (wl.H + wl.Kp_gu) * 0.5625 + step.rows * wl.I * 2.0
+    dn_bytes = dn_w + step.rows * (wl.I + wl.Kp_dn) * 0.5625 + step.rows * wl.H * 2.0
+    n_cpu = max(2, args.cpu_pairs // 32)
+
+    def cpu_leg():
+        import oracle as orc
+
+        orc.build()
+        dt, f = oracle_sample(wl, step.sel_gu.cpu().numpy(), step.sel_dn.cpu().numpy(), n_cpu)
+        return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+                "sample": f"{n_cpu} of {P} (token, expert) rows of one step (their experts' weights packed by the "
+                          f"oracle), {dt:.1f} s"}
+
+    return dict(
+        step=step, x_np=wl.x, flops=gu_f + dn_f, events=["q0", "g0", "q1", "d0", "end"],
+        segments={"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")},
+        dominant=("gate_up", gu_f, gu_bytes, "decode gate_up W4A4+RAC GEMM (swap-AB, SwiGLU epilogue)"),
+        quant={"x": ("quant_x", int(wl.x.nbytes) + P * 0.5625 * (wl.H + wl.Kp_gu)),
+               "h": ("quant_h", quant_bytes(step.rows, wl.I, wl.Kp_dn))},
+        extra_gbs={"gate_up": ("gate_up", gu_bytes), "down": ("down", dn_bytes),
+                   "weights_step": (None, gu_w + dn_w)},
+        config={"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P, "experts": wl.E,
+                "touched_experts": touched, "slabs": step.n_slots, "hidden": wl.H, "intermediate": wl.I,
+                "Kp_gate_up": wl.Kp_gu, "Kp_down": wl.Kp_dn, "weight_bytes_touched": gu_w + dn_w},
+        cpu=cpu_leg, kernels_per_step=DecodeStep.KERNELS_PER_STEP)
+
+
+SPECS = {"moe_prefill": spec_moe, "dense": spec_dense, "moe_decode": spec_decode}
 
 
 def main():
@@ -498,6 +616,8 @@ def main():
             "frac_fp4_peak": value / ws / fp4_peak,
             "kernel_ms": k_ms,
             "act_quant_gbs": {k: b / (k_ms[s] * 1e-3) / 1e9 for k, (s, b) in sp["quant"].items()},
+            "kernel_gbs": {k: b / ((k_ms[s] if s else t_step_ms) * 1e-3) / 1e9
+                           for k, (s, b) in sp.get("extra_gbs", {}).items()},
             "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": e2e,

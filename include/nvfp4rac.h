@@ -76,9 +76,21 @@ typedef enum {
   NVFP4_EPI_SWIGLU_AMAX = 1
 } nvfp4_epilogue;
 
+/* Order of the block scales of a packed matrix.
+ *   NVFP4_SF_ATOM128  the atom order above: rows in groups of 128 (rows_padded % 128 == 0);
+ *                     sf holds rows_padded * cols/16 bytes.
+ *   NVFP4_SF_SLAB16   decode activations: rows in slabs of 16 (rows_padded % 16 == 0); slab
+ *                     s = row / 16 owns one whole atom per 64 columns, atom(s, kb) at byte
+ *                     (s * (cols/64) + kb) * 512, and row r of the slab uses atom row r % 16 with
+ *                     i = 0 (scale of block c at byte (r % 16)*16 + c % 4); the other bytes of the
+ *                     atom are never read.  sf holds rows_padded/16 * cols/64 * 512 bytes.  The
+ *                     decode GEMM reads one atom per slab as the scales of its 16-token operand. */
+typedef enum { NVFP4_SF_ATOM128 = 0, NVFP4_SF_SLAB16 = 1 } nvfp4_sf_layout;
+
 /* A packed NVFP4 matrix, or `slabs` equally shaped matrices (MoE experts) back to back.
- * codes: slabs * rows_padded * cols/2 bytes; sf: slabs * rows_padded * cols/16 bytes (atoms);
- * s_g: `slabs` floats.  rows_padded % 128 == 0, rows <= rows_padded, cols % 64 == 0. */
+ * codes: slabs * rows_padded * cols/2 bytes; sf: slabs * nvfp4_sf_bytes(...) bytes (atoms);
+ * s_g: `slabs` floats.  rows <= rows_padded, cols % 64 == 0; rows_padded % 128 == 0 for
+ * NVFP4_SF_ATOM128 (the default of a zero-initialised struct), % 16 == 0 for NVFP4_SF_SLAB16. */
 typedef struct {
   uint8_t* codes;
   uint8_t* sf;
@@ -87,6 +99,7 @@ typedef struct {
   int64_t rows;
   int64_t rows_padded;
   int64_t cols;
+  int32_t sf_layout; /* nvfp4_sf_layout */
 } nvfp4_tensor;
 
 /* ---------------------------------------------------------------------------------------- */
@@ -99,6 +112,8 @@ const char* nvfp4_last_error_string(void);
 /* Bytes of codes / scale atoms of one rows_padded x cols NVFP4 matrix. */
 size_t nvfp4_codes_bytes(int64_t rows_padded, int64_t cols);
 size_t nvfp4_sf_bytes(int64_t rows_padded, int64_t cols);
+/* Bytes of scale atoms of one rows_padded x cols matrix in the given nvfp4_sf_layout. */
+size_t nvfp4_sf_bytes_layout(int64_t rows_padded, int64_t cols, int32_t sf_layout);
 /* K' = r*K rounded to the nearest multiple of 64 (ties up), clamped to [0, K].
  * "roughly top-50%" (Two fixes, on two different sides) -> r = 0.5 by default. */
 int32_t nvfp4_kp_from_ratio(int64_t K, double r);
@@ -118,9 +133,10 @@ void nvfp4_set_gemm_tile_n(int32_t n);
 /*   sel, Kp    ascending channel list [Kp] (Kp % 64 == 0); Kp == 0 disables the residual.   */
 /*   amax_in    optional device float: use it as amax (e.g. from the SwiGLU epilogue); NULL  */
 /*              computes amax over x rows [0, M).                                            */
-/*   q          output: slabs = 1, rows = M_out, rows_padded >= M_out (multiple of 128),     */
-/*              cols = K; rows >= M_out are written as zeros; q->s_g receives s_g.           */
-/*   q_res      output (Kp > 0): cols = Kp, same rows; its s_g receives the same s_g.        */
+/*   q          output: slabs = 1, rows = M_out, rows_padded >= M_out, cols = K; either      */
+/*              scale layout; rows >= M_out are written as zeros; q->s_g receives s_g.       */
+/*   q_res      output (Kp > 0): cols = Kp, same rows and scale layout; its s_g receives the */
+/*              same s_g.                                                                     */
 /*   workspace  >= nvfp4_quantize_workspace_size() bytes, 16-byte aligned.                   */
 /* ---------------------------------------------------------------------------------------- */
 size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K);
@@ -201,6 +217,29 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
                                   int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N,
                                   int64_t K, int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y,
                                   int64_t ldy, float* amax_out, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* grouped_w4a4_rac_moe_decode -- the grouped GEMM above for decode, where each expert sees   */
+/* only a few tokens.  The expert's weight rows are streamed as the MMA's 128-row operand and  */
+/* the expert's tokens, gathered into 16-row slabs, are the 16-column operand, so one pass     */
+/* reads each touched expert's W and W_sel once per slab.  Same arithmetic as                 */
+/* grouped_w4a4_rac_moe: y = alpha_e * (Q(X) Q(W_e)^T + Q(R_sel) Q(W_sel,e)^T), one FP32       */
+/* accumulator, residual K' loop after the main K loop (Two fixes, on two different sides).    */
+/*   a, a_res        activations in the NVFP4_SF_SLAB16 layout (nvfp4_quantize_scatter with    */
+/*                   row_scatter naming rows 16*slot + j); rows_padded >= 16 * n_slots.        */
+/*   slot_expert     device int32 [n_slots]: expert of each slab (0 <= e < E, else            */
+/*                   NVFP4_ERR_INVALID_ARG in *dev_status and the call stops).                 */
+/*   slot_count      device int32 [n_slots]: tokens in the slab (rows 16*slot + [0, count)    */
+/*                   are results; the others are written as zeros).                           */
+/*   w, w_sel, N, K, Kp, ep, amax_out  as grouped_w4a4_rac_moe (ep == SWIGLU_AMAX needs the   */
+/*                   gate/up interleaved pack; amax covers the counted rows only).             */
+/*   y               [16 * n_slots x N] (or N/2 with SwiGLU), FP32 or bf16, pitch ldy.         */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status grouped_w4a4_rac_moe_decode(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
+                                         const int32_t* slot_expert, const int32_t* slot_count, int32_t n_slots,
+                                         int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N,
+                                         int64_t K, int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y,
+                                         int64_t ldy, float* amax_out, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* weight_qdq -- trainer-side Asymmetric QAT fake quantisation of weights only (Two fixes):  */

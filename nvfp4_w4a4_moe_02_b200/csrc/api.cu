@@ -99,14 +99,25 @@ nvfp4_status make_out_map(CUtensorMap* m, void* base, bool bf16, uint64_t cols, 
   return NVFP4_OK;
 }
 
-nvfp4_status check_tensor(const nvfp4_tensor* t, const char* name, int64_t cols, int64_t min_rows, int64_t slabs) {
+// layouts: bit mask of the accepted nvfp4_sf_layout values (1 << layout)
+constexpr int kAtom128Only = 1 << NVFP4_SF_ATOM128;
+constexpr int kSlab16Only = 1 << NVFP4_SF_SLAB16;
+constexpr int kAnyLayout = kAtom128Only | kSlab16Only;
+
+nvfp4_status check_tensor(const nvfp4_tensor* t, const char* name, int64_t cols, int64_t min_rows, int64_t slabs,
+                          int layouts = kAtom128Only) {
   if (!t) return fail(NVFP4_ERR_INVALID_ARG, "%s is NULL", name);
   if (!t->codes || !t->sf || !t->s_g) return fail(NVFP4_ERR_INVALID_ARG, "%s has a NULL buffer", name);
   if (t->cols != cols) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.cols = %lld, expected %lld", name, (long long)t->cols, (long long)cols);
   if (t->slabs != slabs) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.slabs = %lld, expected %lld", name, (long long)t->slabs, (long long)slabs);
-  if (t->rows_padded % 128 != 0 || t->rows_padded < min_rows || t->rows < 0 || t->rows > t->rows_padded)
-    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s rows %lld / rows_padded %lld invalid (need >= %lld, multiple of 128)", name,
-                (long long)t->rows, (long long)t->rows_padded, (long long)min_rows);
+  if (t->sf_layout != NVFP4_SF_ATOM128 && t->sf_layout != NVFP4_SF_SLAB16)
+    return fail(NVFP4_ERR_INVALID_ARG, "%s.sf_layout = %d is not a scale layout", name, (int)t->sf_layout);
+  if (((1 << t->sf_layout) & layouts) == 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.sf_layout = %d is not accepted by this call", name, (int)t->sf_layout);
+  const int64_t group = t->sf_layout == NVFP4_SF_SLAB16 ? 16 : 128;
+  if (t->rows_padded % group != 0 || t->rows_padded < min_rows || t->rows < 0 || t->rows > t->rows_padded)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s rows %lld / rows_padded %lld invalid (need >= %lld, multiple of %lld)", name,
+                (long long)t->rows, (long long)t->rows_padded, (long long)min_rows, (long long)group);
   if (!aligned16(t->codes) || !aligned16(t->sf)) return fail(NVFP4_ERR_ALIGNMENT, "%s buffers must be 16-byte aligned", name);
   return NVFP4_OK;
 }
@@ -159,6 +170,10 @@ const char* nvfp4_last_error_string(void) { return g_last_error.c_str(); }
 
 size_t nvfp4_codes_bytes(int64_t rows_padded, int64_t cols) { return (size_t)rows_padded * (size_t)(cols / 2); }
 size_t nvfp4_sf_bytes(int64_t rows_padded, int64_t cols) { return (size_t)rows_padded * (size_t)(cols / 16); }
+size_t nvfp4_sf_bytes_layout(int64_t rows_padded, int64_t cols, int32_t sf_layout) {
+  if (sf_layout == NVFP4_SF_SLAB16) return (size_t)(rows_padded / 16) * (size_t)(cols / 64) * 512;
+  return nvfp4_sf_bytes(rows_padded, cols);
+}
 
 int32_t nvfp4_kp_from_ratio(int64_t K, double r) {
   if (!(r > 0.0)) return 0;
@@ -192,13 +207,14 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   if (x && !aligned16(x)) return fail(NVFP4_ERR_ALIGNMENT, "x must be 16-byte aligned");
   if (!row_gather && M_out != M) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "without row_gather M_out must equal M");
   if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp = %d must be a multiple of 64 in [0, K]", Kp);
-  nvfp4_status st = check_tensor(q, "q", K, M_out, 1);
+  nvfp4_status st = check_tensor(q, "q", K, M_out, 1, kAnyLayout);
   if (st != NVFP4_OK) return st;
   if (Kp > 0) {
     if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
-    st = check_tensor(q_res, "q_res", Kp, M_out, 1);
+    st = check_tensor(q_res, "q_res", Kp, M_out, 1, kAnyLayout);
     if (st != NVFP4_OK) return st;
-    if (q_res->rows_padded != q->rows_padded) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res.rows_padded must equal q.rows_padded");
+    if (q_res->rows_padded != q->rows_padded || q_res->sf_layout != q->sf_layout)
+      return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res must have q's rows_padded and sf_layout");
   }
   const int P = act_partials(M, K);
   if (!amax_in) {
@@ -232,6 +248,7 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   a.s_g_out2 = Kp > 0 ? q_res->s_g : nullptr;
   a.codes = q->codes;
   a.sf = q->sf;
+  a.sf_slab16 = q->sf_layout == NVFP4_SF_SLAB16;
   a.rcodes = Kp > 0 ? q_res->codes : nullptr;
   a.rsf = Kp > 0 ? q_res->sf : nullptr;
   a.status = dev_status;
@@ -253,13 +270,14 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
   if (ldx < K || ldx % 8 != 0) return fail(NVFP4_ERR_ALIGNMENT, "ldx = %lld must be >= K and a multiple of 8", (long long)ldx);
   if (x && !aligned16(x)) return fail(NVFP4_ERR_ALIGNMENT, "x must be 16-byte aligned");
   if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp = %d must be a multiple of 64 in [0, K]", Kp);
-  nvfp4_status st = check_tensor(q, "q", K, 0, 1);
+  nvfp4_status st = check_tensor(q, "q", K, 0, 1, kAnyLayout);
   if (st != NVFP4_OK) return st;
   if (Kp > 0) {
     if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
-    st = check_tensor(q_res, "q_res", Kp, 0, 1);
+    st = check_tensor(q_res, "q_res", Kp, 0, 1, kAnyLayout);
     if (st != NVFP4_OK) return st;
-    if (q_res->rows_padded != q->rows_padded) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res.rows_padded must equal q.rows_padded");
+    if (q_res->rows_padded != q->rows_padded || q_res->sf_layout != q->sf_layout)
+      return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res must have q's rows_padded and sf_layout");
   }
   const int P = act_partials(M, K);
   if (!amax_in) {
@@ -294,6 +312,7 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
   a.s_g_out2 = Kp > 0 ? q_res->s_g : nullptr;
   a.codes = q->codes;
   a.sf = q->sf;
+  a.sf_slab16 = q->sf_layout == NVFP4_SF_SLAB16;
   a.rcodes = Kp > 0 ? q_res->codes : nullptr;
   a.rsf = Kp > 0 ? q_res->sf : nullptr;
   a.status = dev_status;
@@ -540,6 +559,91 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
   }
   cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "grouped gemm launch");
+  return NVFP4_OK;
+}
+
+nvfp4_status grouped_w4a4_rac_moe_decode(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
+                                         const int32_t* slot_expert, const int32_t* slot_count, int32_t n_slots,
+                                         int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N,
+                                         int64_t K, int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y,
+                                         int64_t ldy, float* amax_out, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (n_slots < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "n_slots must be >= 0");
+  if (n_slots > 0 && (!slot_expert || !slot_count)) return fail(NVFP4_ERR_INVALID_ARG, "slot_expert / slot_count is NULL");
+  if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
+  if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
+  if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp must be a multiple of 64 in [0, K]");
+  if (N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "N must be a positive multiple of 128");
+  if (ep != NVFP4_EPI_NONE && ep != NVFP4_EPI_SWIGLU_AMAX) return fail(NVFP4_ERR_INVALID_ARG, "bad epilogue");
+  if (ep == NVFP4_EPI_SWIGLU_AMAX && !amax_out) return fail(NVFP4_ERR_INVALID_ARG, "amax_out is NULL with the SwiGLU epilogue");
+  if (out != NVFP4_OUT_F32 && out != NVFP4_OUT_BF16) return fail(NVFP4_ERR_INVALID_ARG, "bad output dtype");
+  const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
+  if (!y && n_slots > 0) return fail(NVFP4_ERR_INVALID_ARG, "y is NULL");
+  if (ldy < y_cols) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "ldy = %lld must be >= %lld", (long long)ldy, (long long)y_cols);
+  const int64_t rows = 16 * (int64_t)n_slots;
+  nvfp4_status st = check_tensor(a, "a", K, rows, 1, kSlab16Only);
+  if (st != NVFP4_OK) return st;
+  st = check_tensor(w, "w", K, N, E);
+  if (st != NVFP4_OK) return st;
+  if (w->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w.rows_padded must equal N");
+  if (Kp > 0) {
+    st = check_tensor(a_res, "a_res", Kp, rows, 1, kSlab16Only);
+    if (st != NVFP4_OK) return st;
+    st = check_tensor(w_sel, "w_sel", Kp, N, E);
+    if (st != NVFP4_OK) return st;
+    if (w_sel->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_sel.rows_padded must equal N");
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (ep == NVFP4_EPI_SWIGLU_AMAX) {
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax reset");
+  }
+  if (n_slots == 0) return NVFP4_OK;
+  CUtensorMap maps[4];
+  memset(maps, 0, sizeof(maps));
+  st = make_code_map(&maps[0], w->codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, 128, 3, "W");
+  if (st != NVFP4_OK) return st;
+  st = make_code_map(&maps[2], a->codes, (uint64_t)K / 2, (uint64_t)a->rows_padded, 1, 16, 2, "X");
+  if (st != NVFP4_OK) return st;
+  if (Kp > 0) {
+    st = make_code_map(&maps[1], w_sel->codes, (uint64_t)Kp / 2, (uint64_t)N, (uint64_t)E, 128, 3, "W_sel");
+    if (st != NVFP4_OK) return st;
+    st = make_code_map(&maps[3], a_res->codes, (uint64_t)Kp / 2, (uint64_t)a_res->rows_padded, 1, 16, 2, "X_res");
+    if (st != NVFP4_OK) return st;
+  } else {
+    maps[1] = maps[0];
+    maps[3] = maps[2];
+  }
+  DecodeArgs d;
+  memset(&d, 0, sizeof(d));
+  d.sfx = a->sf;
+  d.sfx_res = Kp > 0 ? a_res->sf : a->sf;
+  d.sfw = w->sf;
+  d.sfw_sel = Kp > 0 ? w_sel->sf : w->sf;
+  d.sfw_slab_bytes = (int64_t)nvfp4_sf_bytes(N, K);
+  d.sfw_sel_slab_bytes = Kp > 0 ? (int64_t)nvfp4_sf_bytes(N, Kp) : 0;
+  d.k64_main = (int32_t)(K / 64);
+  d.k64_res = Kp / 64;
+  d.kt_main = (int32_t)((K + 255) / 256);
+  d.kt_res = (Kp + 255) / 256;
+  d.m_tiles = (int32_t)(N / 128);
+  d.slot_expert = slot_expert;
+  d.slot_count = slot_count;
+  d.n_slots = n_slots;
+  d.E = E;
+  d.s_x = a->s_g;
+  d.s_w = w->s_g;
+  d.y = y;
+  d.ldy = ldy;
+  d.out_bf16 = out == NVFP4_OUT_BF16;
+  d.epi = ep == NVFP4_EPI_SWIGLU_AMAX ? 1 : 0;
+  d.amax_out = amax_out;
+  d.status = dev_status;
+  d.wait_limit_ns = g_wait_limit_ns.load();
+  const int64_t units = (int64_t)n_slots * d.m_tiles;
+  const int grid = (int)(units < num_sms() ? units : num_sms());
+  cudaError_t e = launch_decode(maps[0], maps[1], maps[2], maps[3], d, grid, s);
+  if (e != cudaSuccess) return cuda_fail(e, "decode gemm launch");
   return NVFP4_OK;
 }
 

@@ -146,6 +146,14 @@ __device__ __forceinline__ float scale_from_amax(float amax, int32_t* status) {
 __device__ __forceinline__ int64_t sf_offset(int64_t row, int64_t kb, int64_t k64) {
   return ((row >> 7) * k64 + (kb >> 2)) * 512 + (row & 31) * 16 + ((row >> 5) & 3) * 4 + (kb & 3);
 }
+// The same for the 16-row slab layout of decode activations: slab row / 16 owns one atom per 64
+// columns and uses its first 16 atom rows (row % 16 at i = 0).
+__device__ __forceinline__ int64_t sf_offset_slab16(int64_t row, int64_t kb, int64_t k64) {
+  return ((row >> 4) * k64 + (kb >> 2)) * 512 + (row & 15) * 16 + (kb & 3);
+}
+__device__ __forceinline__ int64_t sf_offset_any(int64_t row, int64_t kb, int64_t k64, bool slab16) {
+  return slab16 ? sf_offset_slab16(row, kb, k64) : sf_offset(row, kb, k64);
+}
 
 // ----------------------------------------------------------------------------------------
 // warp reductions

@@ -37,6 +37,7 @@ struct RowArgs {
   // outputs
   uint8_t* codes;                // [rows_out x K/2]
   uint8_t* sf;                   // atoms, K/64 groups per row
+  int sf_slab16;                 // act: scales of codes/rcodes in the 16-row slab layout
   uint8_t* rcodes;               // [rows_out x Kp/2]
   uint8_t* rsf;                  // atoms, Kp/64 groups per row
   float* resid_all;              // cal: [rows_out x K] residual of every channel
@@ -87,6 +88,35 @@ cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_a
                         const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
                         cudaStream_t st);
 size_t gemm_smem_bytes(int bn);
+
+// ---- swap-AB decode GEMM (weights = MMA A, 16-token slabs = MMA B)
+struct DecodeArgs {
+  const uint8_t* sfx;        // activation scale atoms, slab layout, n_slots x k64_main
+  const uint8_t* sfx_res;    // residual activation scale atoms, slab layout, n_slots x k64_res
+  const uint8_t* sfw;        // W scale atoms, per slab N/128 x k64_main
+  const uint8_t* sfw_sel;    // W_sel scale atoms, per slab N/128 x k64_res
+  int64_t sfw_slab_bytes;
+  int64_t sfw_sel_slab_bytes;
+  int32_t k64_main, k64_res;
+  int32_t kt_main, kt_res;
+  int32_t m_tiles;           // N / 128
+  const int32_t* slot_expert;  // device [n_slots]
+  const int32_t* slot_count;   // device [n_slots], tokens of the slab (<= 16)
+  int32_t n_slots;
+  int32_t E;
+  const float* s_x;          // device scalar
+  const float* s_w;          // device [E]
+  void* y;
+  int64_t ldy;
+  int32_t out_bf16;
+  int32_t epi;               // 0 none, 1 SwiGLU + amax
+  float* amax_out;
+  int32_t* status;
+  uint64_t wait_limit_ns;
+};
+cudaError_t launch_decode(const CUtensorMap& tm_w, const CUtensorMap& tm_ws, const CUtensorMap& tm_x,
+                          const CUtensorMap& tm_xr, const DecodeArgs& args, int grid, cudaStream_t st);
+size_t decode_smem_bytes();
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t st);
 

@@ -256,8 +256,8 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
         if (h0) *reinterpret_cast<uint32_t*>(crow + e0 / 2) = c0;
         if (h1) *reinterpret_cast<uint32_t*>(crow + e1 / 2) = c1;
         if ((lane & 7) == 0) {
-          if (h0) *reinterpret_cast<uint32_t*>(a.sf + sf_offset(drow, e0 >> 4, k64)) = w0;
-          if (h1) *reinterpret_cast<uint32_t*>(a.sf + sf_offset(drow, e1 >> 4, k64)) = w1;
+          if (h0) *reinterpret_cast<uint32_t*>(a.sf + sf_offset_any(drow, e0 >> 4, k64, a.sf_slab16)) = w0;
+          if (h1) *reinterpret_cast<uint32_t*>(a.sf + sf_offset_any(drow, e1 >> 4, k64, a.sf_slab16)) = w1;
         }
       }
     }
@@ -319,8 +319,8 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
           if (h0) *reinterpret_cast<uint32_t*>(crow + p0 / 2) = c0;
           if (h1) *reinterpret_cast<uint32_t*>(crow + p1 / 2) = c1;
           if ((lane & 7) == 0) {
-            if (h0) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset(drow, p0 >> 4, kp64)) = w0;
-            if (h1) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset(drow, p1 >> 4, kp64)) = w1;
+            if (h0) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset_any(drow, p0 >> 4, kp64, a.sf_slab16)) = w0;
+            if (h1) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset_any(drow, p1 >> 4, kp64, a.sf_slab16)) = w1;
           }
         }
       }

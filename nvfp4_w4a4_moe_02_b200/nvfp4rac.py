@@ -35,7 +35,7 @@ class NVFP4Error(RuntimeError):
 class CTensor(ctypes.Structure):
     _fields_ = [("codes", ctypes.c_void_p), ("sf", ctypes.c_void_p), ("s_g", ctypes.c_void_p),
                 ("slabs", ctypes.c_int64), ("rows", ctypes.c_int64), ("rows_padded", ctypes.c_int64),
-                ("cols", ctypes.c_int64)]
+                ("cols", ctypes.c_int64), ("sf_layout", ctypes.c_int32)]
 
 
 _lib = None
@@ -57,6 +57,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_last_error_string": ([], ctypes.c_char_p),
         "nvfp4_codes_bytes": ([i64, i64], sz),
         "nvfp4_sf_bytes": ([i64, i64], sz),
+        "nvfp4_sf_bytes_layout": ([i64, i64, i32], sz),
         "nvfp4_kp_from_ratio": ([i64, ctypes.c_double], i32),
         "nvfp4_set_wait_limit_ns": ([u64], None),
         "nvfp4_set_gemm_tile_n": ([i32], None),
@@ -70,6 +71,8 @@ def load() -> ctypes.CDLL:
         "w4a4_rac_gemm": ([tp, tp, tp, tp, i64, i64, i64, i32, ctypes.c_int, vp, i64, vp, vp], ctypes.c_int),
         "grouped_w4a4_rac_moe": ([tp, tp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, i64, vp,
                                   vp, vp], ctypes.c_int),
+        "grouped_w4a4_rac_moe_decode": ([tp, tp, vp, vp, i32, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int,
+                                         vp, i64, vp, vp, vp], ctypes.c_int),
         "weight_qdq_workspace_size": ([i64, i64], sz),
         "weight_qdq": ([vp, i64, i64, vp, vp, vp, sz, vp, vp], ctypes.c_int),
         "nvfp4_encode_e2m1": ([vp, i64, vp, vp], ctypes.c_int),
@@ -108,30 +111,49 @@ def round_up(v: int, a: int) -> int:
     return (v + a - 1) // a * a
 
 
+SF_ATOM128, SF_SLAB16 = 0, 1
+
+
+def sf_bytes(rows_padded: int, cols: int, sf_layout: int = SF_ATOM128) -> int:
+    """Scale-atom bytes of one rows_padded x cols matrix (same rule as nvfp4_sf_bytes_layout)."""
+    if sf_layout == SF_SLAB16:
+        return rows_padded // 16 * (cols // 64) * 512
+    return rows_padded * cols // 16
+
+
 @dataclass
 class Packed:
     """Caller-side owner of one packed NVFP4 tensor (device buffers allocated by torch)."""
     codes: torch.Tensor   # uint8 [slabs * rows_padded * cols/2]
-    sf: torch.Tensor      # uint8 [slabs * rows_padded * cols/16]
+    sf: torch.Tensor      # uint8 [slabs * sf_bytes(rows_padded, cols, sf_layout)]
     s_g: torch.Tensor     # float32 [slabs]
     slabs: int
     rows: int
     rows_padded: int
     cols: int
+    sf_layout: int = SF_ATOM128
 
     @staticmethod
     def empty(rows: int, cols: int, slabs: int = 1, rows_padded: int | None = None, device="cuda",
-              zero: bool = False) -> "Packed":
-        rp = round_up(max(rows, 1), 128) if rows_padded is None else rows_padded
+              zero: bool = False, sf_layout: int = SF_ATOM128) -> "Packed":
+        group = 16 if sf_layout == SF_SLAB16 else 128
+        rp = round_up(max(rows, 1), group) if rows_padded is None else rows_padded
         alloc = torch.zeros if zero else torch.empty
         codes = alloc(slabs * rp * cols // 2, dtype=torch.uint8, device=device)
-        sf = alloc(slabs * rp * cols // 16, dtype=torch.uint8, device=device)
+        sf = alloc(slabs * sf_bytes(rp, cols, sf_layout), dtype=torch.uint8, device=device)
         s_g = torch.empty(slabs, dtype=torch.float32, device=device)
-        return Packed(codes, sf, s_g, slabs, rows, rp, cols)
+        return Packed(codes, sf, s_g, slabs, rows, rp, cols, sf_layout)
 
     def c(self) -> CTensor:
         return CTensor(self.codes.data_ptr(), self.sf.data_ptr(), self.s_g.data_ptr(), self.slabs, self.rows,
-                       self.rows_padded, self.cols)
+                       self.rows_padded, self.cols, self.sf_layout)
+
+    def slab(self, e: int) -> "Packed":
+        """View of slab e alone (slabs = 1), sharing storage (e.g. to pack one expert at a time)."""
+        cb = self.rows_padded * self.cols // 2
+        sb = sf_bytes(self.rows_padded, self.cols, self.sf_layout)
+        return Packed(self.codes[e * cb:(e + 1) * cb], self.sf[e * sb:(e + 1) * sb], self.s_g[e:e + 1], 1,
+                      self.rows, self.rows_padded, self.cols, self.sf_layout)
 
 
 class Workspace:
@@ -212,11 +234,12 @@ def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather:
 def nvfp4_quantize_scatter(x: torch.Tensor, row_scatter: torch.Tensor, rows_padded: int,
                            sel: torch.Tensor | None = None, amax_in: torch.Tensor | None = None,
                            out: Packed | None = None, out_res: Packed | None = None,
-                           status: torch.Tensor | None = None, stream=None):
+                           status: torch.Tensor | None = None, stream=None, sf_layout: int = SF_ATOM128):
     """Quantise each row of x once and write it to the rows row_scatter[m, :] of the outputs.
 
     row_scatter: int32 [M, fanout] (-1 = unused).  Rows no entry names are left untouched, so
-    freshly created outputs are zero-filled.  Returns (Packed, Packed | None)."""
+    freshly created outputs are zero-filled.  sf_layout picks the scale order of outputs created
+    here (SF_SLAB16 for the decode GEMM).  Returns (Packed, Packed | None)."""
     lib = load()
     _u16(x)
     M, K = x.shape
@@ -224,9 +247,10 @@ def nvfp4_quantize_scatter(x: torch.Tensor, row_scatter: torch.Tensor, rows_padd
     fanout = row_scatter.shape[1]
     Kp = 0 if sel is None else int(sel.numel())
     if out is None:
-        out = Packed.empty(rows_padded, K, rows_padded=rows_padded, device=x.device, zero=True)
+        out = Packed.empty(rows_padded, K, rows_padded=rows_padded, device=x.device, zero=True, sf_layout=sf_layout)
     if Kp > 0 and out_res is None:
-        out_res = Packed.empty(rows_padded, Kp, rows_padded=rows_padded, device=x.device, zero=True)
+        out_res = Packed.empty(rows_padded, Kp, rows_padded=rows_padded, device=x.device, zero=True,
+                               sf_layout=sf_layout)
     ws = _workspace(x.device).get(lib.nvfp4_quantize_workspace_size(M, K))
     st = status if status is not None else new_status(x.device)
     q = out.c()
@@ -324,6 +348,38 @@ def grouped_w4a4_rac_moe(a: Packed, a_res: Packed | None, expert_offsets: torch.
     return (y, amax_out) if swiglu else y
 
 
+def grouped_w4a4_rac_moe_decode(a: Packed, a_res: Packed | None, slot_expert: torch.Tensor,
+                                slot_count: torch.Tensor, w: Packed, w_sel: Packed | None, swiglu: bool = False,
+                                out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
+                                amax_out: torch.Tensor | None = None, status: torch.Tensor | None = None,
+                                stream=None):
+    """Swap-AB decode GEMM over 16-token expert slabs -> y [16 * n_slots, N (or N/2)] [and amax of h].
+
+    a / a_res are in the SF_SLAB16 layout; slot_expert / slot_count are device int32 [n_slots]."""
+    lib = load()
+    E = w.slabs
+    N, K = w.rows, w.cols
+    Kp = 0 if a_res is None else a_res.cols
+    n_slots = int(slot_expert.numel())
+    assert slot_expert.dtype == torch.int32 and slot_count.dtype == torch.int32
+    ycols = N // 2 if swiglu else N
+    if y is None:
+        y = torch.empty(16 * n_slots, ycols, dtype=out_dtype, device=a.codes.device)
+    if swiglu and amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=a.codes.device)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    st = status if status is not None else new_status(a.codes.device)
+    ca, cw = a.c(), w.c()
+    car = a_res.c() if Kp > 0 else None
+    cws = w_sel.c() if Kp > 0 else None
+    _check(lib.grouped_w4a4_rac_moe_decode(ctypes.byref(ca), ctypes.byref(car) if car else None,
+                                           slot_expert.data_ptr(), slot_count.data_ptr(), n_slots, E,
+                                           ctypes.byref(cw), ctypes.byref(cws) if cws else None, N, K, Kp,
+                                           EPI_SWIGLU_AMAX if swiglu else EPI_NONE, od, y.data_ptr(), y.stride(0),
+                                           _ptr(amax_out), st.data_ptr(), _stream(stream)))
+    return (y, amax_out) if swiglu else y
+
+
 def weight_qdq(w: torch.Tensor, out: torch.Tensor | None = None, s_g: torch.Tensor | None = None,
                status: torch.Tensor | None = None, stream=None):
     """Trainer fake-quant bf16(DQ(Q(w))) per tensor; w is [n_tensors, elems] (or one tensor of any shape)."""
@@ -398,3 +454,25 @@ def scatter_map(pair_token, pair_rows, T: int, fanout: int):
         m[t, fill[t]] = r
         fill[t] += 1
     return m
+
+
+def decode_slots(counts, slab: int = 16):
+    """16-token slabs for a decode step's (expert, token)-sorted pair list.
+
+    counts: pairs per expert.  Returns (slot_expert [S] int32, slot_count [S] int32, pair_rows [P] int64)
+    where expert e's pairs fill ceil(counts[e] / 16) consecutive slabs and pair i lands in row
+    16 * slot + j of the slab layout.
+    """
+    import numpy as np
+
+    counts = np.asarray(counts, dtype=np.int64)
+    slot_expert, slot_count, pair_rows = [], [], []
+    for e, c in enumerate(counts):
+        for k in range(0, int(c), slab):
+            n = min(slab, int(c) - k)
+            base = len(slot_expert) * slab
+            slot_expert.append(e)
+            slot_count.append(n)
+            pair_rows.extend(range(base, base + n))
+    return (np.asarray(slot_expert, dtype=np.int32), np.asarray(slot_count, dtype=np.int32),
+            np.asarray(pair_rows, dtype=np.int64))

@@ -84,6 +84,81 @@ def normal_bf16(seed: int, stream: int, rows: int, cols: int, sigma: float = 1.0
     return out
 
 
+# ----------------------------------------------------------------------------------------------
+# the same generator evaluated by torch on a device (for weights too large to make on the host)
+# ----------------------------------------------------------------------------------------------
+_MASK64 = (1 << 64) - 1
+
+
+def _s64(v: int) -> int:
+    """uint64 constant as the int64 with the same bits."""
+    v &= _MASK64
+    return v - (1 << 64) if v >= (1 << 63) else v
+
+
+def _mix64_int(z: int) -> int:
+    z &= _MASK64
+    z ^= z >> 30
+    z = (z * 0xBF58476D1CE4E5B9) & _MASK64
+    z ^= z >> 27
+    z = (z * 0x94D049BB133111EB) & _MASK64
+    z ^= z >> 31
+    return z
+
+
+def synth_key_int(seed: int, stream: int) -> int:
+    return _mix64_int((seed & _MASK64) ^ _mix64_int(stream + 0x632BE59BD9B4E019))
+
+
+def _mix64_torch(z):
+    # int64 tensors hold the uint64 bit patterns: products wrap modulo 2^64, right shifts are
+    # made logical by masking the sign-extended bits
+    z = z ^ ((z >> 30) & ((1 << 34) - 1))
+    z = z * _s64(0xBF58476D1CE4E5B9)
+    z = z ^ ((z >> 27) & ((1 << 37) - 1))
+    z = z * _s64(0x94D049BB133111EB)
+    z = z ^ ((z >> 31) & ((1 << 33) - 1))
+    return z
+
+
+def _uniform_torch(key: int, idx):
+    import torch
+
+    b = _mix64_torch((idx + 1) * _s64(0x9E3779B97F4A7C15) + _s64(key))
+    return (((b >> 11) & ((1 << 53) - 1)).to(torch.float64) + 0.5) * (1.0 / 9007199254740992.0)
+
+
+def normal_bf16_torch(seed: int, stream: int, rows: int, cols: int, sigma: float = 1.0, offset: int = 0,
+                      device="cpu", out=None, chunk: int = 1 << 23):
+    """normal_bf16 evaluated with torch ops on `device`: torch.bfloat16 [rows, cols].
+
+    Same definition as the C generator (counter of element (r, c) = offset + r*cols + c, Box-Muller
+    in binary64, float RN, bf16 RNE).  The transcendental functions are the device's, so a value
+    may differ from the host's by one binary64 ulp before rounding to bf16; consumers that need
+    the exact bytes read them back from the device.
+    """
+    import torch
+
+    key = synth_key_int(seed, stream)
+    n = rows * cols
+    if out is None:
+        out = torch.empty(rows, cols, dtype=torch.bfloat16, device=device)
+    flat = out.view(-1)
+    for s0 in range(0, n, chunk):
+        s1 = min(n, s0 + chunk)
+        i0, i1 = offset + s0, offset + s1            # element counters [i0, i1)
+        p0, p1 = i0 >> 1, (i1 - 1) >> 1              # Box-Muller pairs touched
+        p = torch.arange(p0, p1 + 1, dtype=torch.int64, device=device)
+        u1 = _uniform_torch(key, 2 * p)
+        u2 = _uniform_torch(key, 2 * p + 1)
+        rad = torch.sqrt(-2.0 * torch.log(u1))
+        th = 6.283185307179586476925286766559 * u2
+        pair = torch.stack([rad * torch.cos(th), rad * torch.sin(th)], dim=1).view(-1)  # counters 2*p0 ..
+        v = sigma * pair[i0 - 2 * p0:i1 - 2 * p0]
+        flat[s0:s1] = v.to(torch.float32).to(torch.bfloat16)
+    return out
+
+
 def generator_threads() -> int:
     return int(_get().synth_num_threads())
 
@@ -232,6 +307,16 @@ class MoEWorkload:
             return self.wdn[e]
         return normal_bf16(self.seed, STREAM_WDOWN, self.H, self.I, 0.02, offset=e * self.H * self.I)
 
+    def gate_up_expert_torch(self, e: int, device, out=None):
+        """Expert e's gate_up weight made on `device` (torch.bfloat16 [2I, H])."""
+        return normal_bf16_torch(self.seed, STREAM_W, 2 * self.I, self.H, 0.02, offset=e * 2 * self.I * self.H,
+                                 device=device, out=out)
+
+    def down_expert_torch(self, e: int, device, out=None):
+        """Expert e's down weight made on `device` (torch.bfloat16 [H, I])."""
+        return normal_bf16_torch(self.seed, STREAM_WDOWN, self.H, self.I, 0.02, offset=e * self.H * self.I,
+                                 device=device, out=out)
+
 
 def moe_block(seed: int = 0, r: float = 0.5, T: int = 4096, H: int = 2048, E: int = 128, topk: int = 8,
               I: int = 768, T_cal: int = 2048, materialize_weights: bool = True) -> MoEWorkload:
@@ -284,6 +369,31 @@ def moe_down_calibration_batch(wl: MoEWorkload, max_pairs: int | None = None) ->
         h = (g / (1.0 + np.exp(-g)) * u).astype(np.float32)
         out[idx] = _f32_to_bf16_bits(h)
     return out
+
+
+def moe_down_calibration_batch_torch(wl: MoEWorkload, device, max_pairs: int | None = None) -> np.ndarray:
+    """moe_down_calibration_batch with the binary64 products formed by torch on `device` and the
+    weights made there (for experts too large to make on the host).  Same routing, pooling and
+    rounding; sums run in the device library's order, so a row may differ from the host version
+    where a binary64 rounding difference reaches the bf16 rounding.  Returns bf16 bits [pairs, I]."""
+    import torch
+
+    T = wl.x_cal.shape[0]
+    k = wl.topk_ids.shape[1]
+    topk = route_topk(wl.seed, T, wl.E, k, stream=STREAM_ROUTER_CAL)
+    pt, pe, counts = sort_pairs(topk, wl.E)
+    if max_pairs is not None:
+        pt, pe = pt[:max_pairs], pe[:max_pairs]
+    xf = torch.from_numpy(bf16_to_f32(wl.x_cal).astype(np.float64)).to(device)
+    out = torch.empty(pt.size, wl.I, dtype=torch.float32, device=device)
+    w = torch.empty(2 * wl.I, wl.H, dtype=torch.bfloat16, device=device)
+    for e in np.unique(pe):
+        idx = np.nonzero(pe == e)[0]
+        wl.gate_up_expert_torch(int(e), device, out=w)
+        gu = xf[torch.from_numpy(pt[idx]).to(device)] @ w.to(torch.float64).T
+        g, u = gu[:, :wl.I], gu[:, wl.I:]
+        out[torch.from_numpy(idx).to(device)] = (g / (1.0 + torch.exp(-g)) * u).to(torch.float32)
+    return _f32_to_bf16_bits(out.cpu().numpy())
 
 
 def _f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:

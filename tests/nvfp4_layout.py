@@ -3,7 +3,8 @@
 Follows the storage definition in include/nvfp4rac.h: two E2M1 codes per byte (element 2j in
 the low nibble), scales in 512-byte atoms covering 128 rows x 64 columns, where the scale of
 row r (r % 128 = 32 i + j) and 16-column block c sits at byte j*16 + i*4 + (c % 4) of atom
-(r // 128, c // 4), atoms ordered row-block major.
+(r // 128, c // 4), atoms ordered row-block major.  In the 16-row slab layout of decode
+activations, slab s = r // 16 owns atoms (s, c // 4) and row r uses byte (r % 16)*16 + (c % 4).
 """
 import numpy as np
 
@@ -24,9 +25,18 @@ def sf_index(rows_padded: int, cols: int) -> np.ndarray:
     return atom * 512 + (r % 32) * 16 + ((r // 32) % 4) * 4 + (c % 4)
 
 
-def unpack_sf(sf: np.ndarray, rows: int, rows_padded: int, cols: int) -> np.ndarray:
+def sf_index_slab16(rows_padded: int, cols: int) -> np.ndarray:
+    """sf_index for the 16-row slab layout."""
+    r = np.arange(rows_padded)[:, None]
+    c = np.arange(cols // 16)[None, :]
+    atom = (r // 16) * (cols // 64) + c // 4
+    return atom * 512 + (r % 16) * 16 + (c % 4)
+
+
+def unpack_sf(sf: np.ndarray, rows: int, rows_padded: int, cols: int, slab16: bool = False) -> np.ndarray:
     flat = np.asarray(sf, dtype=np.uint8).reshape(-1)
-    return flat[sf_index(rows_padded, cols)][:rows]
+    idx = sf_index_slab16(rows_padded, cols) if slab16 else sf_index(rows_padded, cols)
+    return flat[idx][:rows]
 
 
 def pack_sf(S: np.ndarray, rows_padded: int) -> np.ndarray:

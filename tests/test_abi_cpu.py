@@ -90,6 +90,61 @@ def test_host_side_rejections(lib):
     assert lib.nvfp4_selftest_wait_timeout(1000, None, None) == 1
 
 
+def test_decode_and_layout_rejections(lib):
+    from nvfp4_w4a4_moe_02_b200.nvfp4rac import SF_SLAB16, CTensor
+
+    assert lib.nvfp4_sf_bytes_layout(128, 256, 0) == 128 * 16
+    assert lib.nvfp4_sf_bytes_layout(48, 256, SF_SLAB16) == 3 * 4 * 512
+    w = CTensor(16, 16, 16, 4, 256, 256, 128)
+    a16 = CTensor(16, 16, 16, 1, 32, 32, 128, SF_SLAB16)
+    a128 = CTensor(16, 16, 16, 1, 128, 128, 128)
+    args = lambda a, n_slots=2, N=256, ep=0: (ctypes.byref(a), None, 16, 16, n_slots, 4, ctypes.byref(w), None, N, 128,
+                                              0, ep, 0, 16, N, None, None, None)
+    # the decode GEMM takes slab-layout activations only
+    assert lib.grouped_w4a4_rac_moe_decode(*args(a128)) == 2
+    assert b"sf_layout" in lib.nvfp4_last_error_string()
+    # more slots than rows
+    assert lib.grouped_w4a4_rac_moe_decode(*args(a16, n_slots=3)) == 2
+    # N not a multiple of 128
+    assert lib.grouped_w4a4_rac_moe_decode(*args(a16, N=192)) == 2
+    # SwiGLU without amax_out
+    assert lib.grouped_w4a4_rac_moe_decode(*args(a16, ep=1)) == 1
+    # missing slot tables
+    st = lib.grouped_w4a4_rac_moe_decode(ctypes.byref(a16), None, None, 16, 2, 4, ctypes.byref(w), None, 256, 128, 0,
+                                         0, 0, 16, 256, None, None, None)
+    assert st == 1
+    # an unknown layout value, and prefill GEMMs refuse slab-layout operands
+    bad = CTensor(16, 16, 16, 1, 32, 32, 128, 7)
+    st = lib.nvfp4_quantize(16, 32, 128, 128, None, 32, None, 0, None, ctypes.byref(bad), None, 16, 1024, None, None)
+    assert st == 1
+    w1 = CTensor(16, 16, 16, 1, 256, 256, 128)
+    st = lib.w4a4_rac_gemm(ctypes.byref(a16), None, ctypes.byref(w1), None, 32, 256, 128, 0, 0, 16, 256, None, None)
+    assert st == 2
+    # q and q_res must share the layout
+    r128 = CTensor(16, 16, 16, 1, 32, 128, 64)
+    st = lib.nvfp4_quantize(16, 32, 128, 128, None, 32, 16, 64, None, ctypes.byref(a16), ctypes.byref(r128), 16, 1024,
+                            None, None)
+    assert st == 2
+
+
+def test_decode_slots_host_logic():
+    from nvfp4_w4a4_moe_02_b200.nvfp4rac import decode_slots
+
+    counts = [0, 3, 16, 17, 0, 1, 40]
+    se, sc, rows = decode_slots(counts)
+    assert se.tolist() == [1, 2, 3, 3, 5, 6, 6, 6]
+    assert sc.tolist() == [3, 16, 16, 1, 1, 16, 16, 8]
+    assert rows.size == sum(counts) and len(set(rows.tolist())) == rows.size
+    # pairs of expert e land in its own slabs, in order
+    start = 0
+    for e, c in enumerate(counts):
+        r = rows[start:start + c]
+        assert all(se[x // 16] == e for x in r)
+        assert all(x % 16 < sc[x // 16] for x in r)
+        start += c
+    assert decode_slots([0, 0])[0].size == 0
+
+
 def test_layout_decoder_matches_storage_definition():
     from nvfp4_layout import pack_codes, pack_sf, unpack_codes, unpack_sf
 
@@ -103,6 +158,15 @@ def test_layout_decoder_matches_storage_definition():
         off = atom * 512 + (r % 128 % 32) * 16 + (r % 128 // 32) * 4 + c % 4
         assert flat[off] == S[r, c]
     assert np.array_equal(unpack_sf(flat, rows_p, rows_p, cols), S)
+    # 16-row slab layout: slab r // 16 owns atom (r // 16, c // 4); row r at byte (r % 16)*16 + c % 4
+    from nvfp4_layout import sf_index_slab16
+
+    idx = sf_index_slab16(48, cols)
+    for r, c in [(0, 0), (15, 3), (16, 0), (17, 5), (47, 11)]:
+        assert idx[r, c] == ((r // 16) * (cols // 64) + c // 4) * 512 + (r % 16) * 16 + c % 4
+    assert len(set(idx.reshape(-1).tolist())) == idx.size
+    assert np.array_equal(unpack_sf(np.arange(3 * 3 * 512) % 251, 48, 48, cols, slab16=True),
+                          (np.arange(3 * 3 * 512) % 251)[idx])
     C = rng.integers(0, 16, (rows_p, cols), dtype=np.uint8)
     b = pack_codes(C)
     assert b[0] == C[0, 0] | (C[0, 1] << 4)

@@ -35,10 +35,11 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
 def logical(p: R.Packed, slab: int = 0, rows: int | None = None):
     rows = p.rows if rows is None else rows
     cb = p.rows_padded * p.cols // 2
-    sb = p.rows_padded * p.cols // 16
+    sb = R.sf_bytes(p.rows_padded, p.cols, p.sf_layout)
     codes = p.codes[slab * cb:(slab + 1) * cb].cpu().numpy()
     sf = p.sf[slab * sb:(slab + 1) * sb].cpu().numpy()
-    return unpack_codes(codes, rows, p.rows_padded, p.cols), unpack_sf(sf, rows, p.rows_padded, p.cols)
+    return (unpack_codes(codes, rows, p.rows_padded, p.cols),
+            unpack_sf(sf, rows, p.rows_padded, p.cols, slab16=p.sf_layout == R.SF_SLAB16))
 
 
 def f32(v):
@@ -345,7 +346,11 @@ def moe_pipeline(dev, wl, sel_gu, sel_dn):
                 pdn=pdn)
 
 
-def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs):
+def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs, wgu_of=None, wdn_of=None):
+    """Sampled (token, expert) rows of an MoE pipeline against the oracle.  wgu_of / wdn_of give
+    an expert's bf16 weight bits (default: the workload's host copies)."""
+    wgu_of = wgu_of or wl.gate_up_expert
+    wdn_of = wdn_of or wl.down_expert
     I, H = wl.I, wl.H
     s_x = orc.global_scale(orc.amax_bf16(wl.x))
     assert out["a"].s_g.item() == float(s_x)
@@ -367,7 +372,7 @@ def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs):
         # gate_up on the oracle: quantise the token rows, exact GEMM against the expert's weights
         xa = wl.x[toks]
         a_c, a_S, r_c, r_S, _ = orc.act_quant_rac(xa, s_x, sel_gu)
-        wgu = wl.wgu[e]
+        wgu = wgu_of(e)
         s_w = orc.global_scale(orc.amax_bf16(wgu))
         wc, wS, wsc, wsS = orc.weight_pack(wgu, s_w, sel_gu)
         gu, ad = orc.gemm_rac(a_c, a_S, r_c, r_S, wc, wS, wsc, wsS, s_x, s_w)
@@ -388,7 +393,7 @@ def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs):
         hc, hS, hrc, hrS, _ = orc.act_quant_rac(hrows, s_h, sel_dn)
         assert np.array_equal(gq_c[rows], hc) and np.array_equal(gq_S[rows], hS)
         assert np.array_equal(gqr_c[rows], hrc) and np.array_equal(gqr_S[rows], hrS)
-        wdn = wl.wdn[e]
+        wdn = wdn_of(e)
         s_wd = orc.global_scale(orc.amax_bf16(wdn))
         dc, dS, dsc, dsS = orc.weight_pack(wdn, s_wd, sel_dn)
         y_ref, ad2 = orc.gemm_rac(hc, hS, hrc, hrS, dc, dS, dsc, dsS, s_h, s_wd)
@@ -423,6 +428,157 @@ def test_moe_prefill_full_sampled(dev, orc):
     P = wl.pair_token.size
     sample = sorted(set(rng.choice(P, 96, replace=False).tolist() + [0, P - 1]))
     check_moe(orc, wl, sel_gu, sel_dn, out, sample)
+
+
+# ------------------------------------------------------------------------------------------ MoE decode
+def decode_pipeline(dev, wl, sel_gu, sel_dn, packed, counts=None):
+    """quantise (scatter into 16-token expert slabs) -> decode gate_up + SwiGLU -> quantise h ->
+    decode down, all through the C ABI."""
+    st = R.new_status(dev)
+    pgu, pgus, pdn, pdns = packed
+    counts = wl.counts if counts is None else counts
+    se, sc, pair_rows = R.decode_slots(counts)
+    rows = 16 * se.size
+    sed = torch.from_numpy(se).to(dev)
+    scd = torch.from_numpy(sc).to(dev)
+    seld_gu = torch.from_numpy(sel_gu).to(dev) if sel_gu.size else None
+    seld_dn = torch.from_numpy(sel_dn).to(dev) if sel_dn.size else None
+    sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
+    a, ar = R.nvfp4_quantize_scatter(to_dev(wl.x, dev), sm, rows, seld_gu, status=st, sf_layout=R.SF_SLAB16)
+    h, amax_h = R.grouped_w4a4_rac_moe_decode(a, ar, sed, scd, pgu, pgus, swiglu=True, status=st)
+    hq = R.Packed.empty(rows, wl.I, rows_padded=rows, device=dev, sf_layout=R.SF_SLAB16)
+    hqr = R.Packed.empty(rows, sel_dn.size, rows_padded=rows, device=dev, sf_layout=R.SF_SLAB16) if sel_dn.size \
+        else None
+    R.nvfp4_quantize(h, seld_dn, amax_in=amax_h, out=hq, out_res=hqr, status=st)
+    y = R.grouped_w4a4_rac_moe_decode(hq, hqr, sed, scd, pdn, pdns, status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    return dict(pair_rows=pair_rows, slot_expert=se, slot_count=sc, a=a, ar=ar, h=h, amax_h=amax_h, hq=hq, hqr=hqr,
+                y=y)
+
+
+def pack_host_weights(dev, wl, sel_gu, sel_dn):
+    st = R.new_status(dev)
+    seld_gu = torch.from_numpy(sel_gu).to(dev) if sel_gu.size else None
+    seld_dn = torch.from_numpy(sel_dn).to(dev) if sel_dn.size else None
+    pgu, pgus = R.pack_weights(to_dev(wl.wgu, dev), seld_gu, gate_up_interleave=True, status=st)
+    pdn, pdns = R.pack_weights(to_dev(wl.wdn, dev), seld_dn, status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    return pgu, pgus, pdn, pdns
+
+
+def skewed_decode_workload():
+    """Decode-sized routing with every slab shape: experts with 1, 4, 7, 16, 17 and 33 tokens
+    and experts with none."""
+    wl = syn.moe_block(T=40, H=1024, E=12, topk=2, I=256, T_cal=64)
+    ids = np.zeros((40, 2), np.int64)
+    ids[:, 0] = np.repeat([0, 1, 2], [17, 16, 7])          # 17, 16 tokens
+    ids[:33, 1] = 3                                       # 33 tokens
+    ids[33:, 1] = np.array([4, 4, 4, 4, 5, 6, 11])        # 4 tokens, singles; 7..10 empty
+    ids[33:40, 0] = np.where(ids[33:40, 1] == 4, 2, ids[33:40, 0])
+    wl.topk_ids = ids
+    wl.pair_token, wl.pair_expert, wl.counts = syn.sort_pairs(ids, wl.E)
+    return wl
+
+
+def test_decode_small_every_slab_shape(dev, orc):
+    wl = skewed_decode_workload()
+    assert {1, 16, 17, 33}.issubset(set(wl.counts.tolist())) and (wl.counts == 0).any()
+    sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
+    sel_dn, _ = orc.calibrate(syn.moe_down_calibration_batch(wl), wl.Kp_dn)
+    out = decode_pipeline(dev, wl, sel_gu, sel_dn, pack_host_weights(dev, wl, sel_gu, sel_dn))
+    check_moe(orc, wl, sel_gu, sel_dn, out, list(range(wl.pair_token.size)))
+    # rows of a slab past its count come out as zeros in both projections
+    y = bf16_bits(out["y"])
+    valid = np.zeros(y.shape[0], bool)
+    valid[out["pair_rows"]] = True
+    assert not y[~valid].any()
+
+
+@pytest.mark.parametrize("r", [0.0, 0.5])
+def test_decode_plain_epilogue_fp32(dev, orc, r):
+    """No-SwiGLU epilogue with FP32 output (the tolerance without the bf16 ulp), r = 0 included."""
+    wl = skewed_decode_workload()
+    Kp = syn.kp_from_ratio(wl.H, r)
+    sel = orc.calibrate(wl.x_cal, Kp)[0] if Kp else np.zeros(0, np.int32)
+    st = R.new_status(dev)
+    seld = torch.from_numpy(sel).to(dev) if Kp else None
+    w, ws = R.pack_weights(to_dev(wl.wgu, dev), seld, status=st)
+    se, sc, pair_rows = R.decode_slots(wl.counts)
+    sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], 2)).to(dev)
+    a, ar = R.nvfp4_quantize_scatter(to_dev(wl.x, dev), sm, 16 * se.size, seld, status=st, sf_layout=R.SF_SLAB16)
+    y = R.grouped_w4a4_rac_moe_decode(a, ar, torch.from_numpy(se).to(dev), torch.from_numpy(sc).to(dev), w, ws,
+                                      out_dtype=torch.float32, status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    yg = y.cpu().numpy()
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    for e in np.nonzero(wl.counts)[0]:
+        idx = np.nonzero(wl.pair_expert == e)[0]
+        ac, aS, rc, rS, _ = orc.act_quant_rac(wl.x[wl.pair_token[idx]], s_x, sel)
+        s_w = orc.global_scale(orc.amax_bf16(wl.wgu[e]))
+        wc, wS, wsc, wsS = orc.weight_pack(wl.wgu[e], s_w, sel)
+        y_ref, ad = orc.gemm_rac(ac, aS, rc, rS, wc, wS, wsc, wsS, s_x, s_w)
+        assert_gemm_close(yg[pair_rows[idx]], y_ref, ad, False)
+
+
+def test_decode_no_slots_and_bad_expert(dev):
+    wl = skewed_decode_workload()
+    st = R.new_status(dev)
+    w, _ = R.pack_weights(to_dev(wl.wgu[:2], dev), status=st)
+    a = R.Packed.empty(32, wl.H, rows_padded=32, device=dev, zero=True, sf_layout=R.SF_SLAB16)
+    a.s_g.fill_(1.0)
+    empty = torch.zeros(0, dtype=torch.int32, device=dev)
+    y = R.grouped_w4a4_rac_moe_decode(a, None, empty, empty, w, None, status=st)
+    assert y.shape[0] == 0
+    torch.cuda.synchronize()
+    R.check_status(st)
+    # an expert index outside [0, E) stops the call with an error status; the context stays usable
+    bad = torch.tensor([1, 2], dtype=torch.int32, device=dev)
+    cnt = torch.tensor([16, 16], dtype=torch.int32, device=dev)
+    R.grouped_w4a4_rac_moe_decode(a, None, bad, cnt, w, None, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1
+    assert float(torch.ones(8, device=dev).sum().item()) == 8.0
+
+
+def test_moe_decode_full_sampled(dev, orc):
+    """The decode configuration at full size (64 tokens, hidden 7168, 256 experts, top-8,
+    intermediate 2048, r = 0.5), weights made on the device; sampled rows vs the oracle on
+    the exact weight bytes the device used."""
+    wl = syn.moe_decode()
+    touched = np.nonzero(wl.counts)[0]
+    st = R.new_status(dev)
+    sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
+    h_cal = syn.moe_down_calibration_batch_torch(wl, dev, max_pairs=2048)
+    sel_dn, _ = orc.calibrate(h_cal, wl.Kp_dn)
+    seld_gu, seld_dn = torch.from_numpy(sel_gu).to(dev), torch.from_numpy(sel_dn).to(dev)
+    N_gu = 2 * wl.I
+    pgu = R.Packed.empty(N_gu, wl.H, slabs=wl.E, rows_padded=N_gu, device=dev)
+    pgus = R.Packed.empty(N_gu, wl.Kp_gu, slabs=wl.E, rows_padded=N_gu, device=dev)
+    pdn = R.Packed.empty(wl.H, wl.I, slabs=wl.E, rows_padded=wl.H, device=dev)
+    pdns = R.Packed.empty(wl.H, wl.Kp_dn, slabs=wl.E, rows_padded=wl.H, device=dev)
+    wbuf = torch.empty(N_gu, wl.H, dtype=torch.bfloat16, device=dev)
+    dbuf = torch.empty(wl.H, wl.I, dtype=torch.bfloat16, device=dev)
+    for e in touched:
+        R.pack_weights(wl.gate_up_expert_torch(int(e), dev, out=wbuf), seld_gu, gate_up_interleave=True,
+                       out=pgu.slab(int(e)), out_sel=pgus.slab(int(e)), status=st)
+        R.pack_weights(wl.down_expert_torch(int(e), dev, out=dbuf), seld_dn, out=pdn.slab(int(e)),
+                       out_sel=pdns.slab(int(e)), status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    out = decode_pipeline(dev, wl, sel_gu, sel_dn, (pgu, pgus, pdn, pdns))
+    rng = np.random.default_rng(1)
+    P = wl.pair_token.size
+    # the busiest expert, and a spread of others
+    busiest = int(np.argmax(wl.counts))
+    sample = set(np.nonzero(wl.pair_expert == busiest)[0].tolist())
+    sample |= set(rng.choice(P, 10, replace=False).tolist()) | {0, P - 1}
+    dev_bits = lambda t: bf16_bits(t.contiguous())
+    check_moe(orc, wl, sel_gu, sel_dn, out, sorted(sample),
+              wgu_of=lambda e: dev_bits(wl.gate_up_expert_torch(int(e), dev)),
+              wdn_of=lambda e: dev_bits(wl.down_expert_torch(int(e), dev)))
 
 
 # ------------------------------------------------------------------------------------------ failure path
