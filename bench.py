@@ -52,10 +52,11 @@ def dist_env():
 
 
 # ------------------------------------------------------------------------------------------ workload
-def build_inputs(seed=0):
+def build_inputs(seed=0, experts=None):
     from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 
-    wl = syn.moe_prefill(seed=seed)
+    wl = syn.moe_prefill(seed=seed) if experts is None else \
+        syn.moe_block(seed, 0.5, T=4096, H=2048, E=experts, topk=8, I=768)
     h_cal = syn.moe_down_calibration_batch(wl)
     return wl, h_cal
 
@@ -387,7 +388,7 @@ def run_reference(args):
 
 # ------------------------------------------------------------------------------------------ main
 def spec_moe(dev, args, peaks):
-    wl, h_cal = build_inputs()
+    wl, h_cal = build_inputs(experts=args.experts)
     step = MoEStep(wl, h_cal, dev)
     gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
     P = int(wl.pair_token.size)
@@ -445,7 +446,8 @@ def spec_dense(dev, args, peaks):
 def spec_decode(dev, args, peaks):
     from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 
-    wl = syn.moe_decode()
+    wl = syn.moe_decode() if args.experts is None else \
+        syn.moe_block(0, 0.5, T=64, H=7168, E=args.experts, topk=8, I=2048, materialize_weights=False)
     step = DecodeStep(wl, dev)
     gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
     P = int(wl.pair_token.size)
@@ -495,6 +497,8 @@ def main():
     ap.add_argument("--cpu-pairs", type=int, default=256)
     ap.add_argument("--cpu-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--experts", type=int, default=None,
+                    help="MoE workloads: expert count override (smaller device footprint for profiler captures)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
