@@ -249,6 +249,33 @@ class DecodeStep:
         return self.y
 
 
+class QdqStep:
+    """Trainer-side fake quantisation of a set of weight tensors: one weight_qdq call."""
+
+    KERNELS_PER_STEP = 2  # amax, qdq
+
+    def __init__(self, w_np, dev):
+        import torch
+
+        from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+
+        self.R, self.torch = R, torch
+        self.status = R.new_status(dev)
+        self.n_tensors, self.elems = w_np.shape
+        self.x = torch.from_numpy(w_np.view(np.int16)).to(dev).view(torch.bfloat16)
+        self.y = torch.empty_like(self.x)
+        self.s_g = torch.empty(self.n_tensors, dtype=torch.float32, device=dev)
+
+    def run(self, x=None, events=None):
+        ev = events or {}
+        if "q0" in ev:
+            ev["q0"].record()
+        self.R.weight_qdq(self.x if x is None else x, out=self.y, s_g=self.s_g, status=self.status)
+        if "end" in ev:
+            ev["end"].record()
+        return self.y
+
+
 # ------------------------------------------------------------------------------------------ clocks
 class ClockSampler:
     """nvidia-smi clock / throttle-reason samples every 50 ms; samples are kept for the wall-clock
@@ -483,7 +510,119 @@ def spec_decode(dev, args, peaks):
         cpu=cpu_leg, kernels_per_step=DecodeStep.KERNELS_PER_STEP)
 
 
-SPECS = {"moe_prefill": spec_moe, "dense": spec_dense, "moe_decode": spec_decode}
+def _spec_qdq(dev, args, n_tensors):
+    from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+    w = syn.trainer_weights(n_tensors=n_tensors)
+    step = QdqStep(w, dev)
+    n = w.size
+    label = f"weight_qdq_{n_tensors}x{w.shape[1]}"
+
+    def cpu_leg():
+        import oracle as orc
+
+        orc.build()
+        k = max(1, min(n_tensors, 64))
+        rows = w.reshape(n_tensors, -1)[:k] if n_tensors > 1 else w.reshape(-1)[:k << 21].reshape(1, -1)
+        t0 = time.perf_counter()
+        for r in rows:
+            orc.weight_qdq(r)  # amax of the tensor, then the fake-quant
+        dt = time.perf_counter() - t0
+        return {"value": 4.0 * rows.size / dt / 1e9, "unit": "GB/s", "cores": orc.num_threads(), "kind": "oracle",
+                "sample": f"{rows.shape[0]} tensors of {rows.shape[1]} elements (amax + QDQ), {dt:.1f} s"}
+
+    return dict(
+        step=step, x_np=w, flops=0.0, work=4.0 * n, unit="GB/s", dtype="bf16 -> nvfp4 -> bf16 (f32 arithmetic)",
+        events=["q0", "end"], segments={"qdq": ("q0", "end")},
+        dominant=("qdq", 0.0, 4.0 * n, "weight_qdq (amax + fake-quant, 4 B/element algorithmic)"), quant={},
+        config={"workload": label, "tensors": n_tensors, "elements": int(n), "distribution": "N(0, 0.02)"},
+        cpu=cpu_leg, kernels_per_step=QdqStep.KERNELS_PER_STEP)
+
+
+def spec_qdq(dev, args, peaks):
+    return _spec_qdq(dev, args, 1024)
+
+
+def spec_qdq_single(dev, args, peaks):
+    return _spec_qdq(dev, args, 1)
+
+
+SPECS = {"moe_prefill": spec_moe, "dense": spec_dense, "moe_decode": spec_decode, "qdq": spec_qdq,
+         "qdq_single": spec_qdq_single}
+
+
+def run_sweep(args):
+    """RAC ratio sweep on the MoE prefill shapes: r in {0, 0.25, 0.5, 1}; per r the step's
+    TFLOP/s and the error of h (SwiGLU output) and y (down output) against the binary64 product
+    of the bf16 inputs on sampled (token, expert) rows."""
+    import dataclasses
+
+    import torch
+
+    from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+    from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    R.load()
+    base, h_cal = build_inputs(experts=args.experts)
+    rng = np.random.default_rng(0)
+    P = int(base.pair_token.size)
+    sample = np.sort(rng.choice(P, 256, replace=False))
+    I = base.I
+    # binary64 reference of the sampled rows from the bf16 inputs
+    f64 = lambda a: syn.bf16_to_f32(a).astype(np.float64)
+    h_ref, y_ref = [], []
+    for i in sample:
+        e, t = int(base.pair_expert[i]), int(base.pair_token[i])
+        gu = f64(base.x[t]) @ f64(base.wgu[e]).T
+        h = gu[:I] / (1.0 + np.exp(-gu[:I])) * gu[I:]
+        h_ref.append(h)
+        y_ref.append(h @ f64(base.wdn[e]).T)
+    h_ref, y_ref = np.array(h_ref), np.array(y_ref)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    rows = []
+    for r in (0.0, 0.25, 0.5, 1.0):
+        wl = dataclasses.replace(base, r=r, Kp_gu=syn.kp_from_ratio(base.H, r), Kp_dn=syn.kp_from_ratio(base.I, r))
+        step = MoEStep(wl, h_cal, dev)
+        for _ in range(max(3, args.warmup)):
+            flush.zero_()
+            step.run()
+        evs = [{n: torch.cuda.Event(enable_timing=True) for n in ("q0", "end")} for _ in range(args.steps)]
+        for i in range(args.steps):
+            flush.zero_()
+            step.run(events=evs[i])
+        torch.cuda.synchronize()
+        R.check_status(step.status)
+        ms = float(np.mean([e["q0"].elapsed_time(e["end"]) for e in evs]))
+        gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
+        plain_f = sum(flops_of(wl, 0, 0))
+        prow = torch.from_numpy(step.pair_rows[sample]).to(dev)
+        h_g = step.h[prow].double().cpu().numpy()
+        y_g = step.y[prow].double().cpu().numpy()
+        err = lambda a, b: (float(np.linalg.norm(a - b) / np.linalg.norm(b)), float(np.mean(np.abs(a - b))))
+        (hf, hm), (yf, ym) = err(h_g, h_ref), err(y_g, y_ref)
+        rows.append({"r": r, "Kp_gate_up": wl.Kp_gu, "Kp_down": wl.Kp_dn, "ms_per_step": ms,
+                     "tflops": (gu_f + dn_f) / (ms * 1e-3) / 1e12,
+                     "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12,
+                     "h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym})
+        del step
+        torch.cuda.empty_cache()
+    mono = all(rows[i + 1]["y_mean_abs"] <= rows[i]["y_mean_abs"] for i in range(len(rows) - 1))
+    at = {x["r"]: x for x in rows}
+    line = {"metric": METRIC, "value": at[0.5]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": max(3, args.warmup), "ms_per_step": at[0.5]["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None,
+            "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 block scales) -> f32 accumulate",
+            "data": "synthetic (seeded counter-based generator)",
+            "config": {"workload": base.name + "_r_sweep", "r": [x["r"] for x in rows],
+                       "error_reference": "binary64 product of the bf16 inputs (gate_up, silu(g)*u, down) on 256 "
+                                          "sampled (token, expert) rows",
+                       "l2": "flushed between timed steps (256 MiB write outside the per-step events)"},
+            "sweep": rows, "y_error_non_increasing_in_r": mono, "e2e": None,
+            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * len(rows)}
+    print(json.dumps(line), flush=True)
+    return 0
 
 
 def main():
@@ -492,7 +631,7 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="nvfp4rac", choices=["nvfp4rac", "reference"])
-    ap.add_argument("--workload", default="moe_prefill", choices=sorted(SPECS))
+    ap.add_argument("--workload", default="moe_prefill", choices=sorted(SPECS) + ["sweep"])
     ap.add_argument("--ref-pairs", type=int, default=256)
     ap.add_argument("--cpu-pairs", type=int, default=256)
     ap.add_argument("--cpu-rows", type=int, default=16)
@@ -504,6 +643,8 @@ def main():
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "sweep":
+        return run_sweep(args)
 
     import torch
 
@@ -559,7 +700,10 @@ def main():
         t = torch.tensor([t_step_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         t_step_ms = float(t.item())
-    value = ws * sp["flops"] / (t_step_ms * 1e-3) / 1e12
+    unit = sp.get("unit", "TFLOP/s")
+    work = sp.get("work", sp["flops"])
+    scale = 1e12 if unit == "TFLOP/s" else 1e9
+    value = ws * work / (t_step_ms * 1e-3) / scale
 
     # roofline of the dominant kernel: algorithmic bytes / flops over its event-timed duration
     k_ms = {k: float(np.mean(v)) for k, v in per.items()}
@@ -601,7 +745,7 @@ def main():
         t = torch.tensor([e2e_ms], device=dev)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
-    e2e = {"value": ws * sp["flops"] / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+    e2e = {"value": ws * work / (e2e_ms * 1e-3) / scale, "unit": unit,
            "h2d_bytes_per_step": int(x_np.nbytes), "d2h_bytes_per_step": int(y_host.numel() * 2)}
 
     cpu = sp["cpu"]() if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
@@ -611,13 +755,14 @@ def main():
         config["l2"] = "flushed between timed steps (256 MiB write outside the per-step events)"
         config["parallelism"] = f"replicas x{ws}"
         line = {
-            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": args.steps,
+            "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step_ms, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 block scales) -> f32 accumulate",
+            "vs_baseline": None,
+            "dtype": sp.get("dtype", "nvfp4 (e2m1 x e2m1, ue4m3 block scales) -> f32 accumulate"),
             "data": "synthetic (seeded counter-based generator)",
             "config": config,
             "fp4_peak_tflops": fp4_peak,
-            "frac_fp4_peak": value / ws / fp4_peak,
+            "frac_fp4_peak": value / ws / fp4_peak if unit == "TFLOP/s" else None,
             "kernel_ms": k_ms,
             "act_quant_gbs": {k: b / (k_ms[s] * 1e-3) / 1e9 for k, (s, b) in sp["quant"].items()},
             "kernel_gbs": {k: b / ((k_ms[s] if s else t_step_ms) * 1e-3) / 1e9

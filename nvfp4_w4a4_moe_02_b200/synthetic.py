@@ -345,6 +345,13 @@ def moe_decode(seed: int = 0, r: float = 0.5) -> MoEWorkload:
     return moe_block(seed, r, T=64, H=7168, E=256, topk=8, I=2048, materialize_weights=False)
 
 
+def trainer_weights(seed: int = 0, n_tensors: int = 1024, elems: int = 1 << 31) -> np.ndarray:
+    """Trainer fake-quant input: `elems` bf16 N(0, 0.02) weights (stream 2) viewed as n_tensors
+    tensors of elems / n_tensors elements each (1024 x (1024 x 2048) by default)."""
+    assert elems % n_tensors == 0
+    return normal_bf16(seed, STREAM_W, n_tensors, elems // n_tensors, 0.02)
+
+
 def moe_down_calibration_batch(wl: MoEWorkload, max_pairs: int | None = None) -> np.ndarray:
     """Input of the down projection on the calibration batch, in full precision.
 

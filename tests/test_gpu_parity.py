@@ -257,6 +257,36 @@ def test_weight_qdq_matches_oracle(dev, orc):
         assert np.array_equal(got[t], ref), np.argwhere(got[t] != ref)[:5]
 
 
+def test_weight_qdq_trainer_full_sampled(dev, orc):
+    """The trainer fake-quant configuration at full size: 2^31 bf16 N(0, 0.02) weights as 1024
+    tensors of 1024 x 2048 (one scale each), then as a single tensor (one scale); sampled tensors
+    and chunks against the oracle, every per-tensor scale exact."""
+    w = syn.trainer_weights()
+    n, elems = w.shape
+    wd = to_dev(w, dev)
+    out, s_g = R.weight_qdq(wd)
+    torch.cuda.synchronize()
+    s_all = s_g.cpu().numpy()
+    for t in range(n):
+        assert s_all[t] == orc.global_scale(orc.amax_bf16(w[t:t + 1]))
+    for t in (0, 1, 511, n - 1):
+        ref, s_ref = orc.weight_qdq(w[t])
+        assert s_all[t] == s_ref
+        got = bf16_bits(out[t])
+        assert np.array_equal(got, ref), (t, np.argwhere(got != ref)[:5])
+    # one tensor of 2^31 elements: a single scale over everything (int64 indexing throughout)
+    out1, s1 = R.weight_qdq(wd.view(1, -1), out=out.view(1, -1))
+    torch.cuda.synchronize()
+    s_ref = orc.global_scale(orc.amax_bf16(w))
+    assert s1.item() == float(s_ref)
+    flat = out1.view(-1)
+    for start in (0, (1 << 30) + 48, (1 << 31) - (1 << 20)):
+        chunk = w.reshape(-1)[start:start + (1 << 20)]
+        ref, _ = orc.weight_qdq(chunk, s_ref)
+        got = bf16_bits(flat[start:start + (1 << 20)])
+        assert np.array_equal(got, ref), (start, np.argwhere(got != ref)[:5])
+
+
 def test_shared_weight_path_gpu(dev):
     """DQ(pack_weights(W)) == weight_qdq(W), bitwise, both computed on the GPU."""
     N, K = 256, 1024
