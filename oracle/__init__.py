@@ -63,6 +63,9 @@ def _get():
         "orc_e4m3_encode_array": ([vp, i64, vp], None),
         "orc_f64_to_bf16_array": ([vp, i64, vp], None),
         "orc_num_threads": ([], ctypes.c_int),
+        "orc_route_topk": ([vp, i64, i32, i32, vp, vp], None),
+        "orc_dispatch_plan": ([vp, i64, i32, i32, i32, vp, vp], None),
+        "orc_combine": ([vp, i64, vp, vp, i64, i32, i64, vp], None),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -223,6 +226,38 @@ def calibrate(x_cal: np.ndarray, Kp: int):
     err = np.empty(K, np.float64)
     _get().orc_calibrate(_p(x), T, K, int(Kp), _p(sel), _p(err))
     return sel, err
+
+
+def route_topk(logits: np.ndarray, k: int):
+    """Router: float32 logits [T, E] -> (expert ids int32 [T, k], best first; weights float32 [T, k])."""
+    lg = _c(logits, np.float32)
+    T, E = lg.shape
+    ids = np.empty((T, k), np.int32)
+    w = np.empty((T, k), np.float32)
+    _get().orc_route_topk(_p(lg), T, E, int(k), _p(ids), _p(w))
+    return ids, w
+
+
+def dispatch_plan(ids: np.ndarray, E: int, pad: int):
+    """Expert-grouped layout of the (token, expert) pairs -> (offsets int64 [E+1], row int64 [T, k])."""
+    ids = _c(ids, np.int32)
+    T, k = ids.shape
+    off = np.empty(E + 1, np.int64)
+    row = np.empty((T, k), np.int64)
+    _get().orc_dispatch_plan(_p(ids), T, int(k), int(E), int(pad), _p(off), _p(row))
+    return off, row
+
+
+def combine(y: np.ndarray, row: np.ndarray, w: np.ndarray):
+    """out[t] = sum_j w[t, j] * y[row[t, j]] in binary64; y bf16 bits [R, H] -> float64 [T, H]."""
+    y = _c(y, np.uint16)
+    row = _c(row, np.int64)
+    w = _c(w, np.float32)
+    T, k = row.shape
+    H = y.shape[1]
+    out = np.empty((T, H), np.float64)
+    _get().orc_combine(_p(y), H, _p(row), _p(w), T, int(k), H, _p(out))
+    return out
 
 
 def swiglu(gu: np.ndarray):

@@ -425,3 +425,69 @@ void orc_f64_to_bf16_array(const double* v, int64_t n, uint16_t* out) {
 #pragma omp parallel for schedule(static)
   for (int64_t i = 0; i < n; ++i) out[i] = orc_f64_to_bf16(v[i]);
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* The MoE block around the expert GEMMs: routing, dispatch layout, combine.                  */
+/* The pages fix none of this; the readings are:                                              */
+/*  - routing: the top-k of softmax(logits) are the top-k logits (softmax is monotone), ties   */
+/*    to the lower expert index; the combine weight of a chosen expert is its probability     */
+/*    renormalised over the k chosen, w_j = exp(l_j - l_max) / sum_i exp(l_i - l_max),        */
+/*    evaluated in binary64 and stored as binary32;                                            */
+/*  - dispatch: (token, expert) pairs grouped by expert, tokens ascending inside an expert;    */
+/*    expert e's segment starts at offsets[e] and is padded to a multiple of `pad` rows;       */
+/*  - combine: out[t] = sum_j w_tj * y[row(t, j)] in binary64 over the expert outputs.         */
+/* ------------------------------------------------------------------------------------------ */
+void orc_route_topk(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* ids, float* w) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t) {
+    const float* l = logits + t * E;
+    unsigned char* taken = (unsigned char*)calloc((size_t)E, 1);
+    double* p = (double*)malloc(sizeof(double) * (size_t)k);
+    for (int32_t j = 0; j < k; ++j) {
+      int32_t best = -1;
+      for (int32_t e = 0; e < E; ++e) /* strictly greater: the lower index keeps a tie */
+        if (!taken[e] && (best < 0 || l[e] > l[best])) best = e;
+      taken[best] = 1;
+      ids[t * k + j] = best;
+    }
+    const double lmax = (double)l[ids[t * k]];
+    double s = 0.0;
+    for (int32_t j = 0; j < k; ++j) {
+      p[j] = exp((double)l[ids[t * k + j]] - lmax);
+      s += p[j];
+    }
+    for (int32_t j = 0; j < k; ++j) w[t * k + j] = (float)(p[j] / s);
+    free(p);
+    free(taken);
+  }
+}
+
+/* offsets [E+1] (padded segment starts), row_of [T*k] (row of pair (t, j)) */
+void orc_dispatch_plan(const int32_t* ids, int64_t T, int32_t k, int32_t E, int32_t pad, int64_t* offsets,
+                       int64_t* row_of) {
+  int64_t* count = (int64_t*)calloc((size_t)E, sizeof(int64_t));
+  for (int64_t i = 0; i < T * k; ++i) count[ids[i]] += 1;
+  offsets[0] = 0;
+  for (int32_t e = 0; e < E; ++e) offsets[e + 1] = offsets[e] + (count[e] + pad - 1) / pad * pad;
+  memset(count, 0, sizeof(int64_t) * (size_t)E);
+  for (int64_t t = 0; t < T; ++t) /* tokens in increasing order fill each segment */
+    for (int32_t j = 0; j < k; ++j) {
+      const int32_t e = ids[t * k + j];
+      row_of[t * k + j] = offsets[e] + count[e];
+      count[e] += 1;
+    }
+  free(count);
+}
+
+/* y: bf16 [.. x ldy]; out: binary64 [T x H] */
+void orc_combine(const uint16_t* y, int64_t ldy, const int64_t* row_of, const float* w, int64_t T, int32_t k,
+                 int64_t H, double* out) {
+#pragma omp parallel for schedule(static)
+  for (int64_t t = 0; t < T; ++t)
+    for (int64_t h = 0; h < H; ++h) {
+      double s = 0.0;
+      for (int32_t j = 0; j < k; ++j)
+        s += (double)w[t * k + j] * (double)orc_bf16_to_f32(y[row_of[t * k + j] * ldy + h]);
+      out[t * H + h] = s;
+    }
+}

@@ -420,3 +420,73 @@ def test_swiglu_closed_form(orc):
         assert abs(hx[0, i] - ref) <= 1e-15 * max(1.0, abs(ref))
         assert h[0, i] == orc.f64_to_bf16(ref)
     assert hx[0, 0] == 0.0
+
+
+# ------------------------------------------------------------------------------------------ MoE block
+def test_route_topk_matches_stable_sort(orc):
+    """Top-k of the logits, ties to the lower expert: a stable sort of the negated logits."""
+    rng = np.random.default_rng(3)
+    logits = rng.integers(-3, 4, (128, 32)).astype(np.float32)  # many exact ties
+    for k in (1, 2, 8):
+        ids, _ = orc.route_topk(logits, k)
+        ref = np.argsort(-logits, axis=1, kind="stable")[:, :k]
+        assert np.array_equal(ids, ref)
+
+
+def test_route_weights_closed_forms(orc):
+    rng = np.random.default_rng(4)
+    logits = rng.standard_normal((64, 40)).astype(np.float32)
+    ids, w = orc.route_topk(logits, 1)
+    assert np.all(w == 1.0)
+    ids, w = orc.route_topk(logits, 8)
+    assert np.allclose(w.sum(axis=1), 1.0, atol=1e-6)
+    assert np.all(np.diff(w, axis=1) <= 0)  # best first
+    chosen = np.take_along_axis(logits.astype(np.float64), ids.astype(np.int64), axis=1)
+    ratio = w[:, 1:].astype(np.float64) / w[:, :1]
+    assert np.allclose(ratio, np.exp(chosen[:, 1:] - chosen[:, :1]), rtol=1e-6)
+    # two equal best logits share the weight exactly
+    two = np.array([[0.0, 1.5, 1.5, -2.0]], np.float32)
+    ids, w = orc.route_topk(two, 2)
+    assert ids.tolist() == [[1, 2]] and w.tolist() == [[0.5, 0.5]]
+
+
+def test_dispatch_plan_brute_force(orc):
+    rng = np.random.default_rng(5)
+    T, E, k = 50, 9, 3
+    ids = np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    ids[:, 0] = np.where(np.arange(T) % 4 == 0, 2, ids[:, 0])  # a busy expert
+    ids[ids == 7] = 8                                           # an empty one (may duplicate: fix below)
+    for t in range(T):
+        if len(set(ids[t].tolist())) < k:
+            ids[t] = np.array([e for e in [0, 1, 3, 4, 5, 6] if e not in ids[t]][:k], np.int32)
+    for pad in (1, 16, 128):
+        off, row = orc.dispatch_plan(ids, E, pad)
+        pairs = sorted((int(ids[t, j]), t, j) for t in range(T) for j in range(k))
+        counts = [sum(1 for p in pairs if p[0] == e) for e in range(E)]
+        start = [0]
+        for c in counts:
+            start.append(start[-1] + -(-c // pad) * pad)
+        assert off.tolist() == start
+        seen = {}
+        for e, t, j in pairs:
+            r = start[e] + seen.get(e, 0)
+            seen[e] = seen.get(e, 0) + 1
+            assert row[t, j] == r
+        assert counts[7] == 0 and off[8] == off[7]
+
+
+def test_combine_reduces_to_gather_and_is_linear(orc):
+    rng = np.random.default_rng(6)
+    R, H, T, k = 40, 48, 10, 3
+    y = syn._f32_to_bf16_bits(rng.standard_normal((R, H)).astype(np.float32))
+    row = np.stack([rng.permutation(R)[:k] for _ in range(T)]).astype(np.int64)
+    onehot = np.zeros((T, k), np.float32)
+    onehot[:, 1] = 1.0
+    out = orc.combine(y, row, onehot)
+    assert np.array_equal(out, syn.bf16_to_f32(y[row[:, 1]]).astype(np.float64))
+    # dyadic weights: w1 + w2 is exact in binary32, so linearity holds to binary64 rounding
+    w1 = (rng.integers(0, 256, (T, k)) / 256.0).astype(np.float32)
+    w2 = (rng.integers(0, 256, (T, k)) / 256.0).astype(np.float32)
+    a, b, c = orc.combine(y, row, w1), orc.combine(y, row, w2), orc.combine(y, row, w1 + w2)
+    ref = np.einsum("tj,tjh->th", (w1 + w2).astype(np.float64), syn.bf16_to_f32(y[row]).astype(np.float64))
+    assert np.allclose(c, a + b, rtol=1e-12, atol=1e-12) and np.allclose(c, ref, rtol=1e-12, atol=1e-12)
