@@ -227,8 +227,9 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
 /* accumulator, residual K' loop after the main K loop (Two fixes, on two different sides).    */
 /*   a, a_res        activations in the NVFP4_SF_SLAB16 layout (nvfp4_quantize_scatter with    */
 /*                   row_scatter naming rows 16*slot + j); rows_padded >= 16 * n_slots.        */
-/*   slot_expert     device int32 [n_slots]: expert of each slab (0 <= e < E, else            */
-/*                   NVFP4_ERR_INVALID_ARG in *dev_status and the call stops).                 */
+/*   slot_expert     device int32 [n_slots]: expert of each slab; e < 0 marks an unused slab  */
+/*                   (skipped, its rows of y untouched); e >= E is NVFP4_ERR_INVALID_ARG in    */
+/*                   *dev_status and the call stops.                                          */
 /*   slot_count      device int32 [n_slots]: tokens in the slab (rows 16*slot + [0, count)    */
 /*                   are results; the others are written as zeros).                           */
 /*   w, w_sel, N, K, Kp, ep, amax_out  as grouped_w4a4_rac_moe (ep == SWIGLU_AMAX needs the   */
@@ -240,6 +241,44 @@ nvfp4_status grouped_w4a4_rac_moe_decode(const nvfp4_tensor* a, const nvfp4_tens
                                          int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N,
                                          int64_t K, int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y,
                                          int64_t ldy, float* amax_out, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* The MoE block around the expert GEMMs, on the device, so that a step needs no host work.   */
+/* The pages describe none of it (the method only names MoE rollout, Abstract); the readings: */
+/* the top-k of softmax(logits) are the k largest logits, ties to the lower expert; a chosen  */
+/* expert's weight is its probability renormalised over the k chosen,                          */
+/* w_j = exp(l_j - l_max) / sum_i exp(l_i - l_max); pairs are grouped by expert with tokens   */
+/* ascending; out[t] = sum_j w_tj * y[row(t, j)].                                             */
+/* ---------------------------------------------------------------------------------------- */
+/* moe_route_topk -- logits float32 [T x E] (finite, else NVFP4_ERR_RANGE in *dev_status),    */
+/*   E <= 1024, k <= min(32, E).  topk_ids int32 [T x k] (best first), topk_w float32 [T x k]. */
+nvfp4_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_ids, float* topk_w,
+                            int32_t* dev_status, void* stream);
+/* Rows a dispatch plan can need at most (every routed expert wasting pad - 1 rows), rounded
+ * up to a multiple of 128: size activation buffers with it (decode: rows / 16 slots). */
+int64_t moe_rows_capacity(int64_t T, int32_t k, int32_t E, int32_t pad);
+size_t moe_dispatch_workspace_size(int32_t E);
+/* moe_dispatch_plan -- expert-grouped layout of the (token, expert) pairs of topk_ids [T x k]  */
+/* (a token's experts must be distinct).                                                      */
+/*   pad            segment granularity, a multiple of 16: 128 for grouped_w4a4_rac_moe, 16 for */
+/*                  the decode slabs.                                                          */
+/*   expert_offsets int32 [E+1]: padded segment starts; offsets[E] = rows used, or -1 if they   */
+/*                  would exceed rows_capacity (or the slot table), with NVFP4_ERR_INVALID_ARG */
+/*                  in *dev_status; the GEMMs then do nothing.                                 */
+/*   row_scatter    int32 [T x k]: row of pair (t, j), the row_scatter of                      */
+/*                  nvfp4_quantize_scatter (fanout k) and of moe_combine; -1 if unrouted.     */
+/*   slot_expert, slot_count  optional int32 [n_slots] (pad == 16): the decode slot tables;    */
+/*                  slots past the used ones get expert -1, which the decode GEMM skips.      */
+nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E, int32_t pad,
+                               int64_t rows_capacity, int32_t* expert_offsets, int32_t* row_scatter,
+                               int32_t* slot_expert, int32_t* slot_count, int32_t n_slots, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, void* stream);
+/* moe_combine -- out[t, :] = sum_j topk_w[t, j] * y[row_scatter[t, j], :] (binary32 sums in   */
+/* j order, bf16 out); y bf16 with y_rows rows, pitch ldy; out bf16 [T x H], pitch ldo;       */
+/* H % 8 == 0.  A row < 0 contributes nothing; a row >= y_rows is NVFP4_ERR_INVALID_ARG.      */
+nvfp4_status moe_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* row_scatter,
+                         const float* topk_w, int64_t T, int32_t k, int64_t H, uint16_t* out, int64_t ldo,
+                         int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* weight_qdq -- trainer-side Asymmetric QAT fake quantisation of weights only (Two fixes):  */

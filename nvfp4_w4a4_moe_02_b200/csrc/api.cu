@@ -647,6 +647,64 @@ nvfp4_status grouped_w4a4_rac_moe_decode(const nvfp4_tensor* a, const nvfp4_tens
   return NVFP4_OK;
 }
 
+// ------------------------------------------------------------------------------------------ MoE block
+nvfp4_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k, int32_t* topk_ids, float* topk_w,
+                            int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (T < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T must be >= 0");
+  if (E <= 0 || E > kMaxRouteExperts) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E = %d must be in [1, %d]", E, kMaxRouteExperts);
+  if (k <= 0 || k > 32 || k > E) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "k = %d must be in [1, min(32, E)]", k);
+  if (T > 0 && (!logits || !topk_ids || !topk_w)) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if (T == 0) return NVFP4_OK;
+  cudaError_t e = launch_route_topk(logits, T, E, k, topk_ids, topk_w, dev_status, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "router launch");
+}
+
+int64_t moe_rows_capacity(int64_t T, int32_t k, int32_t E, int32_t pad) {
+  if (T < 0 || k <= 0 || E <= 0 || pad <= 0) return 0;
+  // at most min(E, T*k) experts are routed to, and each wastes at most pad - 1 rows of padding
+  const int64_t pairs = T * k;
+  const int64_t used = pairs < (int64_t)E ? pairs : (int64_t)E;
+  const int64_t worst = pairs + used * (pad - 1);
+  return (worst + 127) / 128 * 128;
+}
+
+size_t moe_dispatch_workspace_size(int32_t E) { return round_up((size_t)(E > 0 ? E : 1) * sizeof(int32_t), 256); }
+
+nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E, int32_t pad,
+                               int64_t rows_capacity, int32_t* expert_offsets, int32_t* row_scatter,
+                               int32_t* slot_expert, int32_t* slot_count, int32_t n_slots, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (T < 0 || k <= 0 || E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T >= 0, k > 0 and E > 0 required");
+  if (pad <= 0 || pad % 16 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "pad = %d must be a positive multiple of 16", pad);
+  if (rows_capacity < 0 || rows_capacity > INT32_MAX) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rows_capacity out of range");
+  if (!expert_offsets || (T > 0 && (!topk_ids || !row_scatter))) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if ((slot_expert == nullptr) != (slot_count == nullptr))
+    return fail(NVFP4_ERR_INVALID_ARG, "slot_expert and slot_count go together");
+  if (slot_expert && (pad != 16 || n_slots < 0)) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "slot tables need pad == 16");
+  if (!workspace || workspace_bytes < moe_dispatch_workspace_size(E)) return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_dispatch_plan(topk_ids, T, k, E, pad, rows_capacity, reinterpret_cast<int32_t*>(workspace),
+                                       expert_offsets, row_scatter, slot_expert, slot_count, n_slots, num_sms(),
+                                       dev_status, s);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "dispatch plan launch");
+}
+
+nvfp4_status moe_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* row_scatter,
+                         const float* topk_w, int64_t T, int32_t k, int64_t H, uint16_t* out, int64_t ldo,
+                         int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (T < 0 || k <= 0 || H <= 0 || H % 8 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T >= 0, k > 0, H %% 8 == 0 required");
+  if (T == 0) return NVFP4_OK;
+  if (!y || !row_scatter || !topk_w || !out) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if (ldy < H || ldo < H || ldy % 8 != 0 || ldo % 8 != 0 || !aligned16(y) || !aligned16(out))
+    return fail(NVFP4_ERR_ALIGNMENT, "y / out must be 16-byte aligned with pitches >= H, multiples of 8");
+  cudaError_t e = launch_combine(y, ldy, y_rows, row_scatter, topk_w, T, k, H, out, ldo, num_sms(), dev_status,
+                                 reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "combine launch");
+}
+
 // ------------------------------------------------------------------------------------------ qdq
 size_t weight_qdq_workspace_size(int64_t n_tensors, int64_t elems_per_tensor) {
   (void)elems_per_tensor;

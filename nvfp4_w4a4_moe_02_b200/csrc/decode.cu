@@ -130,11 +130,12 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
   const int64_t total_units = (int64_t)args.n_slots * args.m_tiles;
   const int kt_total = args.kt_main + args.kt_res;
   const uint64_t limit = args.wait_limit_ns;
-  // every role reads the same slot table; an expert index out of range stops all of them at
-  // the same unit (the producer loads nothing for it)
+  // every role reads the same slot table: a negative expert marks an unused slot that all of
+  // them skip; an expert index >= E stops all of them at the same unit (nothing is loaded for it)
+  constexpr int kSkip = -1, kBad = -2;
   auto unit_expert = [&](int slot) -> int {
     const int e = __ldg(args.slot_expert + slot);
-    return (e >= 0 && e < args.E) ? e : -1;
+    return e < 0 ? kSkip : (e < args.E ? e : kBad);
   };
 
   if (warp == 0) {
@@ -147,7 +148,8 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
         const int slot = (int)(u / args.m_tiles);
         const int mt = (int)(u - (int64_t)slot * args.m_tiles);
         const int e = unit_expert(slot);
-        if (e < 0) {
+        if (e == kSkip) continue;
+        if (e == kBad) {
           report_status(args.status, kErrInvalid);
           *abort_flag = 1;
           break;
@@ -199,10 +201,12 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
       int taken = 0;
       uint32_t mma_count = 0;
       bool ok = true;
-      int64_t uidx = 0;
-      for (int64_t u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x, ++uidx) {
+      int64_t uidx = 0;  // units processed by this CTA (skipped slots not counted)
+      for (int64_t u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
         const int slot = (int)(u / args.m_tiles);
-        if (unit_expert(slot) < 0) break;  // reported by the producer
+        const int eu = unit_expert(slot);
+        if (eu == kSkip) continue;
+        if (eu == kBad) break;  // reported by the producer
         const int buf = (int)(uidx % ACC_BUFS);
         const int64_t use = uidx / ACC_BUFS;
         if (use >= 1 && !mbar_wait(bar_acce(buf), (uint32_t)((use - 1) & 1), limit, abort_flag)) {
@@ -245,6 +249,7 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
         }
         if (!ok) break;
         tc_commit(bar_accf(buf));
+        ++uidx;
       }
       if (!ok) {
         report_status(args.status, kErrTimeout);
@@ -258,12 +263,13 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
     const bool bf16 = args.out_bf16 != 0;
     float* xch = reinterpret_cast<float*>(smem + OFF_XCH);
     float amax = 0.0f;
-    int64_t uidx = 0;
-    for (int64_t u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x, ++uidx) {
+    int64_t uidx = 0;  // units processed by this CTA, as counted by the MMA issuer
+    for (int64_t u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
       const int slot = (int)(u / args.m_tiles);
       const int mt = (int)(u - (int64_t)slot * args.m_tiles);
       const int e = unit_expert(slot);
-      if (e < 0) break;
+      if (e == kSkip) continue;
+      if (e == kBad) break;
       const int cnt = min(BT, max(0, (int)__ldg(args.slot_count + slot)));
       const int buf = (int)(uidx % ACC_BUFS);
       const uint32_t parity = (uint32_t)((uidx / ACC_BUFS) & 1);
@@ -334,6 +340,7 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
         }
         break;
       }
+      ++uidx;
     }
     if (swiglu && args.amax_out != nullptr) {
       amax = warp_max(amax);

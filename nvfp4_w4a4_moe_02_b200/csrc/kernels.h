@@ -118,6 +118,17 @@ cudaError_t launch_decode(const CUtensorMap& tm_w, const CUtensorMap& tm_ws, con
                           const CUtensorMap& tm_xr, const DecodeArgs& args, int grid, cudaStream_t st);
 size_t decode_smem_bytes();
 
+// ---- MoE block around the GEMMs (csrc/moe.cu)
+constexpr int kMaxRouteExperts = 1024;
+cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* status,
+                              cudaStream_t st);
+cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, int pad, int64_t rows_capacity,
+                                 int32_t* counts, int32_t* offsets, int32_t* row_scatter, int32_t* slot_expert,
+                                 int32_t* slot_count, int n_slots, int num_sms, int32_t* status, cudaStream_t st);
+cudaError_t launch_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* rows, const float* w,
+                           int64_t T, int k, int64_t H, uint16_t* out, int64_t ldo, int num_sms, int32_t* status,
+                           cudaStream_t st);
+
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t st);
 
 }  // namespace nvfp4

@@ -1,0 +1,251 @@
+// The MoE block around the expert GEMMs, on the device: router top-k, the expert-grouped
+// dispatch layout of the (token, expert) pairs, and the weighted combine of expert outputs.
+//
+// Readings (the pages fix none of this): the top-k of softmax(logits) are the k largest logits,
+// ties to the lower expert; a chosen expert's weight is its probability renormalised over the
+// k chosen, exp(l_j - l_max) / sum_i exp(l_i - l_max); pairs are grouped by expert with tokens
+// ascending, each expert segment padded to a multiple of `pad` rows; out[t] = sum_j w_tj y_row(t,j).
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+// ----------------------------------------------------------------------------------------
+// router: one warp per token; lane l holds logits l, l + 32, ...; k rounds of a warp arg-max
+// ordered by (value descending, expert ascending)
+// ----------------------------------------------------------------------------------------
+
+__global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
+                                                         int32_t* __restrict__ ids, float* __restrict__ w,
+                                                         int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  constexpr int V = kMaxRouteExperts / 32;
+  float v[V];
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < V; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = e < E ? __ldg(logits + t * E + e) : -INFINITY;
+    if (e < E && !(fabsf(v[i]) <= 3.4e38f)) bad = true;
+  }
+  if (__any_sync(0xffffffffu, bad)) {
+    if (lane == 0) report_status(status, kErrRange);
+    return;
+  }
+  float lmax = 0.0f, sum = 0.0f;
+  float chosen_v = 0.0f;  // lane j keeps the value of the j-th choice
+  int chosen_e = 0;
+  for (int j = 0; j < k; ++j) {
+    // local best: the first maximum over this lane's experts (ascending); experts already
+    // chosen hold -inf and lose to every finite logit
+    float bv = -INFINITY;
+    int be = 0x7FFFFFFF;
+#pragma unroll
+    for (int i = 0; i < V; ++i) {
+      const int e = lane + 32 * i;
+      if (e < E && (be == 0x7FFFFFFF || v[i] > bv)) {
+        bv = v[i];
+        be = e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
+      const int oe = __shfl_xor_sync(0xffffffffu, be, o);
+      if (ov > bv || (ov == bv && oe < be)) {
+        bv = ov;
+        be = oe;
+      }
+    }
+    // every lane now holds the winner; its owner takes it out of the running
+    if ((be & 31) == lane) {
+#pragma unroll
+      for (int i = 0; i < V; ++i)
+        if (lane + 32 * i == be) v[i] = -INFINITY;
+    }
+    if (j == 0) lmax = bv;
+    const float p = expf(__fsub_rn(bv, lmax));
+    sum = __fadd_rn(sum, p);
+    if (lane == j) {
+      chosen_v = p;
+      chosen_e = be;
+    }
+  }
+  if (lane < k) {
+    ids[t * k + lane] = chosen_e;
+    w[t * k + lane] = __fdiv_rn(chosen_v, sum);
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// dispatch plan
+// ----------------------------------------------------------------------------------------
+__global__ void count_kernel(const int32_t* __restrict__ ids, int64_t n, int E, int32_t* __restrict__ counts,
+                             int32_t* status) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int e = __ldg(ids + i);
+    if (e < 0 || e >= E) {
+      report_status(status, kErrInvalid);
+      continue;
+    }
+    atomicAdd(counts + e, 1);
+  }
+}
+
+// one CTA: padded segment starts (exclusive scan), then the decode slot tables
+__global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ counts, int E, int pad,
+                                                       int64_t rows_capacity, int32_t* __restrict__ offsets,
+                                                       int32_t* slot_expert, int32_t* slot_count, int n_slots,
+                                                       int32_t* status) {
+  __shared__ int64_t part[1024];
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = threadIdx.x * per;
+  int64_t mine = 0;
+  for (int e = e0; e < min(E, e0 + per); ++e) mine += (int64_t)(counts[e] + pad - 1) / pad * pad;
+  part[threadIdx.x] = mine;
+  __syncthreads();
+  // inclusive scan over the threads' sums (Hillis-Steele)
+  for (int o = 1; o < (int)blockDim.x; o <<= 1) {
+    const int64_t add = threadIdx.x >= (unsigned)o ? part[threadIdx.x - o] : 0;
+    __syncthreads();
+    part[threadIdx.x] += add;
+    __syncthreads();
+  }
+  int64_t run = part[threadIdx.x] - mine;
+  const int64_t total = part[blockDim.x - 1];
+  const bool fits = total <= rows_capacity && (slot_expert == nullptr || total / 16 <= n_slots);
+  if (!fits && threadIdx.x == 0) report_status(status, kErrInvalid);
+  for (int e = e0; e < min(E, e0 + per); ++e) {
+    offsets[e] = fits ? (int32_t)run : 0;
+    const int c = counts[e];
+    if (slot_expert != nullptr && fits) {
+      const int s0 = (int)(run / 16);
+      for (int s = 0; 16 * s < c; ++s) {
+        slot_expert[s0 + s] = e;
+        slot_count[s0 + s] = min(16, c - 16 * s);
+      }
+    }
+    run += (int64_t)(c + pad - 1) / pad * pad;
+  }
+  // an unusable plan is marked by offsets[E] = -1: no pair gets a row, the GEMMs do nothing
+  if (threadIdx.x == 0) offsets[E] = fits ? (int32_t)total : -1;
+  if (slot_expert != nullptr) {
+    const int used = fits ? (int)(total / 16) : 0;
+    for (int s = used + threadIdx.x; s < n_slots; s += blockDim.x) {
+      slot_expert[s] = -1;  // unused slot: the decode GEMM skips it
+      slot_count[s] = 0;
+    }
+  }
+}
+
+// one CTA per expert: the rank of each of its tokens (ascending) -> row of the pair
+__global__ void __launch_bounds__(256) rank_kernel(const int32_t* __restrict__ ids, int64_t T, int k,
+                                                   const int32_t* __restrict__ offsets, int E,
+                                                   int32_t* __restrict__ row_scatter) {
+  __shared__ int warp_sum[8];
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (offsets[E] < 0) return;  // unusable plan (reported): every pair stays unrouted (-1)
+  int64_t run = offsets[e];
+  for (int64_t base = 0; base < T; base += blockDim.x) {
+    const int64_t t = base + threadIdx.x;
+    int hit = -1;
+    if (t < T)
+      for (int j = 0; j < k; ++j)
+        if (__ldg(ids + t * k + j) == e) hit = j;
+    const unsigned m = __ballot_sync(0xffffffffu, hit >= 0);
+    if (lane == 0) warp_sum[warp] = __popc(m);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
+      before += i < warp ? warp_sum[i] : 0;
+      total += warp_sum[i];
+    }
+    if (hit >= 0) row_scatter[t * k + hit] = (int32_t)(run + before + __popc(m & ((1u << lane) - 1u)));
+    run += total;
+    __syncthreads();
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// combine: thread = 8 consecutive features of one token; binary32 accumulation in j order
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ y, int64_t ldy, int64_t y_rows,
+                                                      const int32_t* __restrict__ rows, const float* __restrict__ w,
+                                                      int64_t T, int k, int64_t H, uint16_t* __restrict__ out,
+                                                      int64_t ldo, int32_t* status) {
+  const int64_t per_tok = H / 8;
+  const int64_t n = T * per_tok;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / per_tok;
+    const int64_t h = (i - t * per_tok) * 8;
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    for (int j = 0; j < k; ++j) {
+      const int32_t r = __ldg(rows + t * k + j);
+      if (r < 0) continue;  // an unrouted pair contributes nothing
+      if (r >= y_rows) {
+        report_status(status, kErrInvalid);
+        continue;
+      }
+      const float wj = __ldg(w + t * k + j);
+      const uint4 q = __ldg(reinterpret_cast<const uint4*>(y + r * ldy + h));
+      const uint32_t u[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        acc[2 * c] = fmaf(wj, bf16_bits_to_f32(u[c] & 0xFFFFu), acc[2 * c]);
+        acc[2 * c + 1] = fmaf(wj, bf16_bits_to_f32(u[c] >> 16), acc[2 * c + 1]);
+      }
+    }
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(acc[2 * c], acc[2 * c + 1]);
+      ow[c] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    *reinterpret_cast<uint4*>(out + t * ldo + h) = o;
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// launchers
+// ----------------------------------------------------------------------------------------
+cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* status,
+                              cudaStream_t st) {
+  const int64_t blocks = (T + 7) / 8;
+  route_topk_kernel<<<(unsigned)blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, int pad, int64_t rows_capacity,
+                                 int32_t* counts, int32_t* offsets, int32_t* row_scatter, int32_t* slot_expert,
+                                 int32_t* slot_count, int n_slots, int num_sms, int32_t* status, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)E, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(row_scatter, 0xFF, sizeof(int32_t) * (size_t)(T * k), st);  // -1: unrouted
+  if (e != cudaSuccess) return e;
+  const int64_t n = T * k;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+  if (blocks < 1) blocks = 1;
+  count_kernel<<<(unsigned)blocks, 256, 0, st>>>(ids, n, E, counts, status);
+  offsets_kernel<<<1, 1024, 0, st>>>(counts, E, pad, rows_capacity, offsets, slot_expert, slot_count, n_slots,
+                                     status);
+  rank_kernel<<<(unsigned)E, 256, 0, st>>>(ids, T, k, offsets, E, row_scatter);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* rows, const float* w,
+                           int64_t T, int k, int64_t H, uint16_t* out, int64_t ldo, int num_sms, int32_t* status,
+                           cudaStream_t st) {
+  const int64_t n = T * (H / 8);
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > (int64_t)num_sms * 16) blocks = (int64_t)num_sms * 16;
+  if (blocks < 1) blocks = 1;
+  combine_kernel<<<(unsigned)blocks, 256, 0, st>>>(y, ldy, y_rows, rows, w, T, k, H, out, ldo, status);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

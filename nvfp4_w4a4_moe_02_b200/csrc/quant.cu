@@ -86,6 +86,10 @@ __device__ __forceinline__ float reduce_partials(const float* partial, int P) {
 // (weight pack) runs after the main pass from a per-warp stash of the row and of each block's
 // (d, 1/d): lane pairs take 16 consecutive compact positions, read their channel numbers and
 // re-derive x, its code and DQ = e*d for exactly those channels.
+//
+// SPLIT (activations with few rows, e.g. the tokens of one decode step): a whole CTA works on
+// one row; warp w takes the 512-element chunks w, w + nwarps, ... of both passes and the stash
+// is shared by the CTA, so a 64-token batch still occupies every warp of 64 CTAs.
 // ----------------------------------------------------------------------------------------
 
 // Scale word of a k64 group: lanes 8g..8g+7 own blocks 4g..4g+3 (the pair (2m, 2m+1) owns
@@ -105,16 +109,6 @@ struct Dests {
   __device__ __forceinline__ int64_t get(int j) const { return list ? (int64_t)__ldg(list + j) : row; }
 };
 
-__device__ __forceinline__ void load8(const uint16_t* p, bool ok, float x[8], uint4& raw) {
-  raw = ok ? __ldg(reinterpret_cast<const uint4*>(p)) : make_uint4(0, 0, 0, 0);
-  const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    x[2 * j] = bf16_bits_to_f32(w[j] & 0xFFFFu);
-    x[2 * j + 1] = bf16_bits_to_f32(w[j] >> 16);
-  }
-}
-
 __device__ __forceinline__ void unpack8(const uint4 raw, float x[8]) {
   const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
 #pragma unroll
@@ -131,7 +125,7 @@ __device__ __forceinline__ float pair_max8(const float x[8]) {
   return fmaxf(m, __shfl_xor_sync(0xffffffffu, m, 1));
 }
 
-template <int MODE>
+template <int MODE, bool SPLIT>
 __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int lane = threadIdx.x & 31;
@@ -142,11 +136,12 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   constexpr bool kHasSel = (MODE == kModeAct || MODE == kModePack);
   const bool use_sel = kHasSel && Kp > 0;
 
-  // CTA-shared channel list (int16), then per warp: the row's bf16 bits and each block's (d, 1/d)
+  // CTA-shared channel list (int16), then per warp (per CTA when SPLIT): the row's bf16 bits
+  // and each block's (d, 1/d)
   int16_t* sel_s = reinterpret_cast<int16_t*>(smem_raw);
   const size_t sel_bytes = use_sel ? (((size_t)Kp * 2 + 15) / 16) * 16 : 0;
   const size_t warp_bytes = use_sel ? (((size_t)K * 2 + 15) / 16) * 16 + (size_t)(K / 16) * 8 : 0;
-  uint16_t* row_s = reinterpret_cast<uint16_t*>(smem_raw + sel_bytes + warp * warp_bytes);
+  uint16_t* row_s = reinterpret_cast<uint16_t*>(smem_raw + sel_bytes + (SPLIT ? 0 : warp) * warp_bytes);
   float2* dinv_s = reinterpret_cast<float2*>(reinterpret_cast<unsigned char*>(row_s) + ((K * 2 + 15) / 16) * 16);
   if (use_sel) {
     for (int32_t j = threadIdx.x; j < Kp; j += blockDim.x) {
@@ -168,7 +163,11 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   int64_t cached_slab = -1;
   float s_g = 0.0f, t6 = 0.0f;
 
-  for (int64_t row = (int64_t)blockIdx.x * nwarps + warp; row < n_rows; row += (int64_t)gridDim.x * nwarps) {
+  const int64_t row_first = SPLIT ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * nwarps + warp;
+  const int64_t row_step = SPLIT ? (int64_t)gridDim.x : (int64_t)gridDim.x * nwarps;
+  const int64_t chunk0 = SPLIT ? 512 * warp : 0;          // this warp's first chunk of a row
+  const int64_t chunk_step = SPLIT ? 512 * nwarps : 512;  // distance to its next chunk
+  for (int64_t row = row_first; row < n_rows; row += row_step) {
     // ---- source row, destinations, scale
     int64_t slab = (MODE == kModePack) ? row / a.rows_per_slab : 0;
     int64_t r_in_slab = row - slab * a.rows_per_slab;
@@ -190,7 +189,7 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
       s_g = scale_from_amax(amax, a.status);
       t6 = __fmul_rn(6.0f, s_g);
       cached_slab = slab;
-      if (row == slab * a.rows_per_slab && lane == 0) {
+      if (row == slab * a.rows_per_slab && lane == 0 && (!SPLIT || warp == 0)) {
         // exactly one warp writes each slab's scale: the one owning the slab's first row
         if (a.s_g_out) a.s_g_out[slab] = s_g;
         if (a.s_g_out2) a.s_g_out2[slab] = s_g;
@@ -199,16 +198,19 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
     const uint16_t* srow = a.src + slab * a.src_slab_stride + (valid ? src_row : 0) * a.ld;
 
     // ---- main pass (the loads of the next 512 elements are issued before this block's math)
-    uint4 n0 = (valid && 8 * lane < K) ? __ldg(reinterpret_cast<const uint4*>(srow + 8 * lane)) : make_uint4(0, 0, 0, 0);
-    uint4 n1 = (valid && 256 + 8 * lane < K) ? __ldg(reinterpret_cast<const uint4*>(srow + 256 + 8 * lane))
-                                             : make_uint4(0, 0, 0, 0);
-    for (int64_t base = 0; base < K; base += 512) {
+    uint4 n0 = (valid && chunk0 + 8 * lane < K) ? __ldg(reinterpret_cast<const uint4*>(srow + chunk0 + 8 * lane))
+                                                : make_uint4(0, 0, 0, 0);
+    uint4 n1 = (valid && chunk0 + 256 + 8 * lane < K)
+                   ? __ldg(reinterpret_cast<const uint4*>(srow + chunk0 + 256 + 8 * lane))
+                   : make_uint4(0, 0, 0, 0);
+    for (int64_t base = chunk0; base < K; base += chunk_step) {
       const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
       const bool h0 = e0 < K, h1 = e1 < K;  // K % 64 == 0: uniform over lane pairs and 8-lane groups
       const uint4 r0 = n0, r1 = n1;
-      if (base + 512 < K) {
-        n0 = (valid && e0 + 512 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + e0 + 512)) : make_uint4(0, 0, 0, 0);
-        n1 = (valid && e1 + 512 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + e1 + 512)) : make_uint4(0, 0, 0, 0);
+      if (base + chunk_step < K) {
+        const int64_t f0 = e0 + chunk_step, f1 = e1 + chunk_step;
+        n0 = (valid && f0 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + f0)) : make_uint4(0, 0, 0, 0);
+        n1 = (valid && f1 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + f1)) : make_uint4(0, 0, 0, 0);
       }
       float x0[8], x1[8];
       unpack8(r0, x0);
@@ -264,8 +266,8 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
 
     // ---- residual pass over the compact selected channels
     if (use_sel) {
-      __syncwarp();
-      for (int64_t base = 0; base < Kp; base += 512) {
+      if (SPLIT) __syncthreads(); else __syncwarp();  // the whole row is stashed
+      for (int64_t base = chunk0; base < Kp; base += chunk_step) {
         const int64_t p0 = base + 8 * lane, p1 = base + 256 + 8 * lane;
         const bool h0 = p0 < Kp, h1 = p1 < Kp;
         float v[2][8];
@@ -324,7 +326,7 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
           }
         }
       }
-      __syncwarp();
+      if (SPLIT) __syncthreads(); else __syncwarp();  // stash reads done before the next row
     }
   }
 }
@@ -522,14 +524,17 @@ size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps) {
 
 cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
   int warps = 8;
-  size_t smem = rows_smem_bytes(a.K, a.Kp, warps);
-  while (smem > 200 * 1024 && warps > 1) {
+  const int64_t rows = a.row_scatter ? a.src_rows : a.rows_out;
+  // few activation rows: one CTA of 8 warps per row (SPLIT), so that every warp of the grid
+  // has work; otherwise one warp per row with as many warps per CTA as the stashes allow
+  const bool split = a.mode == kModeAct && rows * 2 < (int64_t)num_sms * warps;
+  size_t smem = rows_smem_bytes(a.K, a.Kp, split ? 1 : warps);
+  while (!split && smem > 200 * 1024 && warps > 1) {
     warps /= 2;
     smem = rows_smem_bytes(a.K, a.Kp, warps);
   }
   if (smem > 200 * 1024) return cudaErrorInvalidValue;
-  const int64_t rows = a.row_scatter ? a.src_rows : a.rows_out;
-  int64_t ctas_needed = (rows + warps - 1) / warps;
+  int64_t ctas_needed = split ? rows : (rows + warps - 1) / warps;
   int per_sm = (int)((220 * 1024) / (smem + 1024));
   if (per_sm < 1) per_sm = 1;
   if (per_sm > 8) per_sm = 8;
@@ -539,16 +544,25 @@ cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
   cudaError_t e = cudaSuccess;
   switch (a.mode) {
     case kModeAct:
-      e = cudaFuncSetAttribute(quant_rows_kernel<kModeAct>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) quant_rows_kernel<kModeAct><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      if (split) {
+        e = cudaFuncSetAttribute(quant_rows_kernel<kModeAct, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e == cudaSuccess) quant_rows_kernel<kModeAct, true><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      } else {
+        e = cudaFuncSetAttribute(quant_rows_kernel<kModeAct, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem);
+        if (e == cudaSuccess) quant_rows_kernel<kModeAct, false><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      }
       break;
     case kModePack:
-      e = cudaFuncSetAttribute(quant_rows_kernel<kModePack>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) quant_rows_kernel<kModePack><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      e = cudaFuncSetAttribute(quant_rows_kernel<kModePack, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e == cudaSuccess) quant_rows_kernel<kModePack, false><<<(unsigned)grid, warps * 32, smem, st>>>(a);
       break;
     case kModeCal:
-      e = cudaFuncSetAttribute(quant_rows_kernel<kModeCal>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-      if (e == cudaSuccess) quant_rows_kernel<kModeCal><<<(unsigned)grid, warps * 32, smem, st>>>(a);
+      e = cudaFuncSetAttribute(quant_rows_kernel<kModeCal, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)smem);
+      if (e == cudaSuccess) quant_rows_kernel<kModeCal, false><<<(unsigned)grid, warps * 32, smem, st>>>(a);
       break;
     default:
       return cudaErrorInvalidValue;

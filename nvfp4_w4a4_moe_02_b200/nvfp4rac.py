@@ -73,6 +73,11 @@ def load() -> ctypes.CDLL:
                                   vp, vp], ctypes.c_int),
         "grouped_w4a4_rac_moe_decode": ([tp, tp, vp, vp, i32, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int,
                                          vp, i64, vp, vp, vp], ctypes.c_int),
+        "moe_route_topk": ([vp, i64, i32, i32, vp, vp, vp, vp], ctypes.c_int),
+        "moe_rows_capacity": ([i64, i32, i32, i32], i64),
+        "moe_dispatch_workspace_size": ([i32], sz),
+        "moe_dispatch_plan": ([vp, i64, i32, i32, i32, i64, vp, vp, vp, vp, i32, vp, sz, vp, vp], ctypes.c_int),
+        "moe_combine": ([vp, i64, i64, vp, vp, i64, i32, i64, vp, i64, vp, vp], ctypes.c_int),
         "weight_qdq_workspace_size": ([i64, i64], sz),
         "weight_qdq": ([vp, i64, i64, vp, vp, vp, sz, vp, vp], ctypes.c_int),
         "nvfp4_encode_e2m1": ([vp, i64, vp, vp], ctypes.c_int),
@@ -378,6 +383,62 @@ def grouped_w4a4_rac_moe_decode(a: Packed, a_res: Packed | None, slot_expert: to
                                            EPI_SWIGLU_AMAX if swiglu else EPI_NONE, od, y.data_ptr(), y.stride(0),
                                            _ptr(amax_out), st.data_ptr(), _stream(stream)))
     return (y, amax_out) if swiglu else y
+
+
+def moe_route_topk(logits: torch.Tensor, k: int, ids: torch.Tensor | None = None, w: torch.Tensor | None = None,
+                   status: torch.Tensor | None = None, stream=None):
+    """Router top-k: float32 logits [T, E] -> (ids int32 [T, k], weights float32 [T, k])."""
+    lib = load()
+    assert logits.is_cuda and logits.dtype == torch.float32 and logits.is_contiguous()
+    T, E = logits.shape
+    ids = torch.empty(T, k, dtype=torch.int32, device=logits.device) if ids is None else ids
+    w = torch.empty(T, k, dtype=torch.float32, device=logits.device) if w is None else w
+    st = status if status is not None else new_status(logits.device)
+    _check(lib.moe_route_topk(logits.data_ptr(), T, E, k, ids.data_ptr(), w.data_ptr(), st.data_ptr(),
+                              _stream(stream)))
+    return ids, w
+
+
+def moe_rows_capacity(T: int, k: int, E: int, pad: int) -> int:
+    return int(load().moe_rows_capacity(T, k, E, pad))
+
+
+def moe_dispatch_plan(ids: torch.Tensor, E: int, pad: int, rows_capacity: int | None = None,
+                      n_slots: int | None = None, offsets: torch.Tensor | None = None,
+                      row_scatter: torch.Tensor | None = None, slot_expert: torch.Tensor | None = None,
+                      slot_count: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None):
+    """Expert-grouped layout of the pairs of ids [T, k] -> (offsets [E+1], row_scatter [T, k], slot_expert,
+    slot_count); the slot tables (pad 16) only when n_slots is given."""
+    lib = load()
+    assert ids.dtype == torch.int32 and ids.is_contiguous()
+    T, k = ids.shape
+    dev = ids.device
+    cap = moe_rows_capacity(T, k, E, pad) if rows_capacity is None else rows_capacity
+    offsets = torch.empty(E + 1, dtype=torch.int32, device=dev) if offsets is None else offsets
+    row_scatter = torch.empty(T, k, dtype=torch.int32, device=dev) if row_scatter is None else row_scatter
+    if n_slots is not None:
+        slot_expert = torch.empty(n_slots, dtype=torch.int32, device=dev) if slot_expert is None else slot_expert
+        slot_count = torch.empty(n_slots, dtype=torch.int32, device=dev) if slot_count is None else slot_count
+    ws = _workspace(dev).get(lib.moe_dispatch_workspace_size(E))
+    st = status if status is not None else new_status(dev)
+    _check(lib.moe_dispatch_plan(ids.data_ptr(), T, k, E, pad, cap, offsets.data_ptr(), row_scatter.data_ptr(),
+                                 _ptr(slot_expert), _ptr(slot_count), 0 if n_slots is None else n_slots,
+                                 ws.data_ptr(), ws.numel(), st.data_ptr(), _stream(stream)))
+    return offsets, row_scatter, slot_expert, slot_count
+
+
+def moe_combine(y: torch.Tensor, row_scatter: torch.Tensor, w: torch.Tensor, out: torch.Tensor | None = None,
+                status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """out[t] = sum_j w[t, j] * y[row_scatter[t, j]] -> bf16 [T, H]."""
+    lib = load()
+    _u16(y)
+    T, k = row_scatter.shape
+    H = y.shape[1]
+    out = torch.empty(T, H, dtype=torch.bfloat16, device=y.device) if out is None else out
+    st = status if status is not None else new_status(y.device)
+    _check(lib.moe_combine(y.data_ptr(), y.stride(0), y.shape[0], row_scatter.data_ptr(), w.data_ptr(), T, k, H,
+                           out.data_ptr(), out.stride(0), st.data_ptr(), _stream(stream)))
+    return out
 
 
 def weight_qdq(w: torch.Tensor, out: torch.Tensor | None = None, s_g: torch.Tensor | None = None,
