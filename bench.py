@@ -249,6 +249,90 @@ class DecodeStep:
         return self.y
 
 
+class MoEBlockStep:
+    """A whole MoE layer on the device, nothing on the host per step: router top-k of the logits,
+    dispatch plan, quantise-scatter of X, gate_up (SwiGLU + amax), quantise h, down, weighted
+    combine into [T, H].  Prefill uses 128-row expert segments and the grouped GEMM; decode uses
+    16-token slabs (worst-case slot count, unused slots skipped) and the swap-AB GEMM."""
+
+    KERNELS_PER_STEP = 10  # router, count, offsets, rank, amax, quantise X, gate_up, quantise h, down, combine
+
+    def __init__(self, wl, packed, sel_gu, sel_dn, decode, dev):
+        import torch
+
+        from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+        from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+        self.R, self.torch, self.wl, self.decode = R, torch, wl, decode
+        self.status = R.new_status(dev)
+        self.sel_gu, self.sel_dn = sel_gu, sel_dn
+        self.pgu, self.pgus, self.pdn, self.pdns = packed
+        T, k = wl.topk_ids.shape
+        self.T, self.k = T, k
+        self.pad = 16 if decode else 128
+        self.cap = R.moe_rows_capacity(T, k, wl.E, self.pad)
+        self.n_slots = self.cap // 16 if decode else None
+        self.logits_np = syn.normal_f64(wl.seed, syn.STREAM_ROUTER, T * wl.E).reshape(T, wl.E).astype(np.float32)
+        self.logits = torch.from_numpy(self.logits_np).to(dev)
+        self.x = torch.from_numpy(np.ascontiguousarray(wl.x).view(np.int16)).to(dev).view(torch.bfloat16)
+        P = R.Packed
+        lay = R.SF_SLAB16 if decode else R.SF_ATOM128
+        self.ids = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.w = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.off = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
+        self.rows = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.se = torch.empty(self.n_slots, dtype=torch.int32, device=dev) if decode else None
+        self.sc = torch.empty(self.n_slots, dtype=torch.int32, device=dev) if decode else None
+        self.a = P.empty(self.cap, wl.H, rows_padded=self.cap, device=dev, zero=True, sf_layout=lay)
+        self.ar = P.empty(self.cap, wl.Kp_gu, rows_padded=self.cap, device=dev, zero=True, sf_layout=lay)
+        self.h = torch.zeros(self.cap, wl.I, dtype=torch.bfloat16, device=dev)
+        self.amax_h = torch.zeros(1, dtype=torch.float32, device=dev)
+        self.hq = P.empty(self.cap, wl.I, rows_padded=self.cap, device=dev, sf_layout=lay)
+        self.hqr = P.empty(self.cap, wl.Kp_dn, rows_padded=self.cap, device=dev, sf_layout=lay)
+        self.ye = torch.zeros(self.cap, wl.H, dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+
+    def run(self, x=None, logits=None, events=None):
+        R = self.R
+        ev = events or {}
+        if "r0" in ev:
+            ev["r0"].record()
+        R.moe_route_topk(self.logits if logits is None else logits, self.k, ids=self.ids, w=self.w,
+                         status=self.status)
+        R.moe_dispatch_plan(self.ids, self.wl.E, self.pad, rows_capacity=self.cap, n_slots=self.n_slots,
+                            offsets=self.off, row_scatter=self.rows, slot_expert=self.se, slot_count=self.sc,
+                            status=self.status)
+        if "q0" in ev:
+            ev["q0"].record()
+        R.nvfp4_quantize_scatter(self.x if x is None else x, self.rows, self.cap, self.sel_gu, out=self.a,
+                                 out_res=self.ar, status=self.status)
+        if "g0" in ev:
+            ev["g0"].record()
+        if self.decode:
+            R.grouped_w4a4_rac_moe_decode(self.a, self.ar, self.se, self.sc, self.pgu, self.pgus, swiglu=True,
+                                          y=self.h, amax_out=self.amax_h, status=self.status)
+        else:
+            R.grouped_w4a4_rac_moe(self.a, self.ar, self.off, self.pgu, self.pgus, swiglu=True, y=self.h,
+                                   amax_out=self.amax_h, status=self.status)
+        if "q1" in ev:
+            ev["q1"].record()
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        if "d0" in ev:
+            ev["d0"].record()
+        if self.decode:
+            R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.se, self.sc, self.pdn, self.pdns, y=self.ye,
+                                          status=self.status)
+        else:
+            R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.off, self.pdn, self.pdns, y=self.ye, status=self.status)
+        if "c0" in ev:
+            ev["c0"].record()
+        R.moe_combine(self.ye, self.rows, self.w, out=self.y, status=self.status)
+        if "end" in ev:
+            ev["end"].record()
+        return self.y
+
+
 class QdqStep:
     """Trainer-side fake quantisation of a set of weight tensors: one weight_qdq call."""
 
@@ -510,6 +594,50 @@ def spec_decode(dev, args, peaks):
         cpu=cpu_leg, kernels_per_step=DecodeStep.KERNELS_PER_STEP)
 
 
+def _spec_block(dev, args, decode):
+    if decode:
+        from nvfp4_w4a4_moe_02_b200 import synthetic as syn
+
+        wl = syn.moe_decode() if args.experts is None else \
+            syn.moe_block(0, 0.5, T=64, H=7168, E=args.experts, topk=8, I=2048, materialize_weights=False)
+        inner = DecodeStep(wl, dev)
+    else:
+        wl, h_cal = build_inputs(experts=args.experts)
+        inner = MoEStep(wl, h_cal, dev)
+    step = MoEBlockStep(wl, (inner.pgu, inner.pgus, inner.pdn, inner.pdns), inner.sel_gu, inner.sel_dn, decode, dev)
+    # the device router must reproduce the workload's routing (same logits, same reading)
+    step.run()
+    import torch
+
+    torch.cuda.synchronize()
+    step.R.check_status(step.status)
+    gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
+    T = wl.x.shape[0]
+    P = int(wl.pair_token.size)
+    n_w = int((wl.counts > 0).sum()) if decode else wl.E  # experts whose weights the step reads
+    rows = step.cap if decode else P
+    gu_bytes = n_w * 2 * wl.I * (wl.H + wl.Kp_gu) * 0.5625 + rows * (wl.H + wl.Kp_gu) * 0.5625 + rows * wl.I * 2.0
+    name = wl.name + f"_r{wl.r}_layer"
+    return dict(
+        step=step, x_np=wl.x, extra_h2d={"logits": step.logits_np}, flops=gu_f + dn_f,
+        events=["r0", "q0", "g0", "q1", "d0", "c0", "end"],
+        segments={"route_plan": ("r0", "q0"), "quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"),
+                  "quant_h": ("q1", "d0"), "down": ("d0", "c0"), "combine": ("c0", "end")},
+        dominant=("gate_up", gu_f, gu_bytes, "gate_up W4A4+RAC GEMM of the layer (SwiGLU epilogue)"),
+        quant={}, config={"workload": name, "tokens": T, "experts": wl.E, "hidden": wl.H, "intermediate": wl.I,
+                          "plan": "device (router top-k, dispatch plan); combine into [T, H]",
+                          "rows_capacity": step.cap},
+        cpu=lambda: None, kernels_per_step=MoEBlockStep.KERNELS_PER_STEP)
+
+
+def spec_block_prefill(dev, args, peaks):
+    return _spec_block(dev, args, False)
+
+
+def spec_block_decode(dev, args, peaks):
+    return _spec_block(dev, args, True)
+
+
 def _spec_qdq(dev, args, n_tensors):
     from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 
@@ -548,7 +676,8 @@ def spec_qdq_single(dev, args, peaks):
 
 
 SPECS = {"moe_prefill": spec_moe, "dense": spec_dense, "moe_decode": spec_decode, "qdq": spec_qdq,
-         "qdq_single": spec_qdq_single}
+         "qdq_single": spec_qdq_single, "moe_prefill_layer": spec_block_prefill,
+         "moe_decode_layer": spec_block_decode}
 
 
 def run_sweep(args):
@@ -727,6 +856,8 @@ def main():
     x_host = torch.from_numpy(x_np.view(np.int16)).pin_memory()
     y_host = torch.empty(step.y.shape, dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty(x_np.shape, dtype=torch.bfloat16, device=dev)
+    extra_host = {k: torch.from_numpy(v).pin_memory() for k, v in sp.get("extra_h2d", {}).items()}
+    extra_dev = {k: torch.empty_like(v, device=dev) for k, v in extra_host.items()}
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = max(3, args.steps // 4)
@@ -735,7 +866,9 @@ def main():
         flush.zero_()
         e0.record()
         x_dev.view(torch.int16).copy_(x_host, non_blocking=True)
-        y = step.run(x=x_dev)
+        for k, v in extra_host.items():
+            extra_dev[k].copy_(v, non_blocking=True)
+        y = step.run(x=x_dev, **extra_dev)
         y_host.copy_(y, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
@@ -746,7 +879,8 @@ def main():
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
         e2e_ms = float(t.item())
     e2e = {"value": ws * work / (e2e_ms * 1e-3) / scale, "unit": unit,
-           "h2d_bytes_per_step": int(x_np.nbytes), "d2h_bytes_per_step": int(y_host.numel() * 2)}
+           "h2d_bytes_per_step": int(x_np.nbytes) + sum(int(v.nbytes) for v in sp.get("extra_h2d", {}).values()),
+           "d2h_bytes_per_step": int(y_host.numel() * 2)}
 
     cpu = sp["cpu"]() if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
 
