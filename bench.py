@@ -517,6 +517,8 @@ def spec_moe(dev, args, peaks):
         step=step, x_np=wl.x, flops=gu_f + dn_f, events=["q0", "g0", "q1", "d0", "end"],
         segments={"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")},
         dominant=("gate_up", gu_f, gu_bytes, "grouped gate_up W4A4+RAC GEMM (SwiGLU epilogue)"),
+        # dram__bytes_read.sum + dram__bytes_write.sum of one launch, grouped_gemm_gate_up_moe_prefill.md
+        traffic=(410.365440e6 + 51.551488e6) if args.experts is None else None,
         quant={"x": ("quant_x", int(wl.x.nbytes) + P * 0.5625 * (wl.H + wl.Kp_gu)),  # X read once, 8 copies out
                "h": ("quant_h", quant_bytes(P, wl.I, wl.Kp_dn))},
         config={"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P, "experts": wl.E,
@@ -846,6 +848,9 @@ def main():
         achieved = d_flops / (k_ms[seg] * 1e-3) / 1e12
         roof = {"bound": "tensor", "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s",
                 "frac": achieved / fp4_peak, "traffic": None}
+    # DRAM traffic of the dominant kernel from the committed ncu capture of this workload (None
+    # when no capture of the current kernel exists)
+    roof["traffic"] = sp.get("traffic")
     roof["kernel"] = d_label
     roof["algorithmic"] = {"bytes": d_bytes, "flops": d_flops}
     roof["peak_source"] = (f"{peak_kind}: HBM = copy bandwidth, FP4 = bf16 burst x {FP4_OVER_BF16:g} (nominal ratio)"
