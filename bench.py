@@ -44,6 +44,23 @@ def load_peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
+def max_over_ranks(value: float, ws: int, device) -> float:
+    """The largest per-rank value (a step time): every rank takes part, every rank gets it."""
+    if ws <= 1:
+        return value
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(work_per_rank: float, ws: int, t_ms_max: float, scale: float) -> float:
+    """Weak scaling: every rank does work_per_rank in t_ms_max (the slowest rank's time)."""
+    return ws * work_per_rank / (t_ms_max * 1e-3) / scale
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -827,14 +844,11 @@ def main():
     first, last = sp["events"][0], sp["events"][-1]
     per = {k: [e[a].elapsed_time(e[b]) for e in evs] for k, (a, b) in sp["segments"].items()}
     t_step_ms = float(np.sum([e[first].elapsed_time(e[last]) for e in evs])) / args.steps
-    if ws > 1:
-        t = torch.tensor([t_step_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        t_step_ms = float(t.item())
+    t_step_ms = max_over_ranks(t_step_ms, ws, dev)
     unit = sp.get("unit", "TFLOP/s")
     work = sp.get("work", sp["flops"])
     scale = 1e12 if unit == "TFLOP/s" else 1e9
-    value = ws * work / (t_step_ms * 1e-3) / scale
+    value = whole_job_rate(work, ws, t_step_ms, scale)
 
     # roofline of the dominant kernel: algorithmic bytes / flops over its event-timed duration
     k_ms = {k: float(np.mean(v)) for k, v in per.items()}
@@ -878,12 +892,8 @@ def main():
         e1.record()
         torch.cuda.synchronize()
         e2e_ms += e0.elapsed_time(e1)
-    e2e_ms /= n_e2e
-    if ws > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": ws * work / (e2e_ms * 1e-3) / scale, "unit": unit,
+    e2e_ms = max_over_ranks(e2e_ms / n_e2e, ws, dev)
+    e2e = {"value": whole_job_rate(work, ws, e2e_ms, scale), "unit": unit,
            "h2d_bytes_per_step": int(x_np.nbytes) + sum(int(v.nbytes) for v in sp.get("extra_h2d", {}).values()),
            "d2h_bytes_per_step": int(y_host.numel() * 2)}
 
