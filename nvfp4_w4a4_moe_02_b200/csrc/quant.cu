@@ -406,9 +406,42 @@ __global__ void __launch_bounds__(1024) select_topk_kernel(const double* __restr
 
 // ----------------------------------------------------------------------------------------
 // K8: trainer fake quantisation, bf16(DQ(Q(w))), one scale per tensor.  Same lane layout as
-// the row quantiser over a flat array; each 512-element warp chunk lies inside one tensor
-// when elems_per_tensor % 512 == 0, else the tensor of each 16-block is looked up.
+// the row quantiser over the flat array of all tensors (lane pairs hold the two halves of a
+// 16-block).  Each warp takes a contiguous run of 512-element chunks, so it streams sequential
+// memory, changes tensor (and recomputes the tensor's scale) rarely, and finds the tensor of a
+// chunk by counting instead of dividing; the next chunk's loads are issued before this
+// chunk's arithmetic.
 // ----------------------------------------------------------------------------------------
+struct QdqScale {
+  int64_t t;  // tensor whose scale is cached (-1: none)
+  float s_g, t6;
+};
+
+__device__ __forceinline__ void qdq_scale_for(QdqScale& c, int64_t t, const float* __restrict__ partial, int P,
+                                              int32_t* status) {
+  if (t == c.t) return;
+  float am = 0.0f;
+  for (int i = 0; i < P; ++i) am = fmaxf(am, __ldg(partial + t * P + i));
+  c.s_g = scale_from_amax(am, status);
+  c.t6 = __fmul_rn(6.0f, c.s_g);
+  c.t = t;
+}
+
+__device__ __forceinline__ void qdq_half(const uint4 q, float s_g, float t6, uint4& o) {
+  float x[8];
+  unpack8(q, x);
+  const BlockScale b = block_scale(pair_max8(x), s_g, t6);
+  float dq[8];
+  quant8(x, b, dq);
+  uint32_t r[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(dq[2 * j], dq[2 * j + 1]);
+    r[j] = *reinterpret_cast<uint32_t*>(&p);
+  }
+  o = make_uint4(r[0], r[1], r[2], r[3]);
+}
+
 __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ w, int64_t n_tensors, int64_t elems,
                                                   uint16_t* __restrict__ out, const float* __restrict__ partial, int P,
                                                   float* s_g_out, int32_t* status) {
@@ -417,73 +450,37 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ w
   const int64_t nwarps = ((int64_t)gridDim.x * blockDim.x) >> 5;
   const int64_t total = n_tensors * elems;
   const int64_t nchunks = (total + 511) / 512;
-  int64_t cached = -1;
-  float s_g = 0.0f, t6 = 0.0f;
-  for (int64_t ch = warp_global; ch < nchunks; ch += nwarps) {
-    const int64_t base = ch * 512;
-    const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
+  const int64_t c_begin = nchunks * warp_global / nwarps, c_end = nchunks * (warp_global + 1) / nwarps;
+  if (c_begin >= c_end) return;
+  // tensor of each lane's two half-blocks (lane pairs agree: elems % 16 == 0), kept by counting
+  int64_t e0 = c_begin * 512 + 8 * lane, e1 = e0 + 256;
+  int64_t t0 = min(e0 / elems, n_tensors - 1), t1 = min(e1 / elems, n_tensors - 1);  // once per warp
+  int64_t b0 = t0 * elems, b1 = t1 * elems;        // first element of each lane's current tensor
+  QdqScale sc0{-1, 0.f, 0.f}, sc1{-1, 0.f, 0.f};
+  uint4 n0 = e0 < total ? __ldg(reinterpret_cast<const uint4*>(w + e0)) : make_uint4(0, 0, 0, 0);
+  uint4 n1 = e1 < total ? __ldg(reinterpret_cast<const uint4*>(w + e1)) : make_uint4(0, 0, 0, 0);
+  for (int64_t ch = c_begin; ch < c_end; ++ch) {
+    const uint4 q0 = n0, q1 = n1;
     const bool h0 = e0 < total, h1 = e1 < total;
-    // tensor of each half-block (uniform over a lane pair: elems % 16 == 0); the scale of a
-    // tensor is reduced from its P partials, cached per lane
-    const int64_t t0 = h0 ? e0 / elems : n_tensors - 1;
-    const int64_t t1 = h1 ? e1 / elems : n_tensors - 1;
-    float sg0, sg1, t60, t61;
-    if (t0 != cached) {
-      float am = 0.0f;
-      for (int i = 0; i < P; ++i) am = fmaxf(am, partial[t0 * P + i]);
-      s_g = scale_from_amax(am, status);
-      t6 = __fmul_rn(6.0f, s_g);
-      cached = t0;
+    if (ch + 1 < c_end) {
+      n0 = e0 + 512 < total ? __ldg(reinterpret_cast<const uint4*>(w + e0 + 512)) : make_uint4(0, 0, 0, 0);
+      n1 = e1 + 512 < total ? __ldg(reinterpret_cast<const uint4*>(w + e1 + 512)) : make_uint4(0, 0, 0, 0);
     }
-    sg0 = s_g;
-    t60 = t6;
-    if (t1 != cached) {
-      float am = 0.0f;
-      for (int i = 0; i < P; ++i) am = fmaxf(am, partial[t1 * P + i]);
-      sg1 = scale_from_amax(am, status);
-      t61 = __fmul_rn(6.0f, sg1);
-    } else {
-      sg1 = s_g;
-      t61 = t6;
-    }
+    while (t0 + 1 < n_tensors && e0 >= b0 + elems) { ++t0; b0 += elems; }
+    while (t1 + 1 < n_tensors && e1 >= b1 + elems) { ++t1; b1 += elems; }
+    qdq_scale_for(sc0, t0, partial, P, status);
+    qdq_scale_for(sc1, t1, partial, P, status);
     if (s_g_out) {
-      if (h0 && e0 % elems == 0) s_g_out[t0] = sg0;
-      if (h1 && e1 % elems == 0) s_g_out[t1] = sg1;
+      if (h0 && e0 == b0) s_g_out[t0] = sc0.s_g;
+      if (h1 && e1 == b1) s_g_out[t1] = sc1.s_g;
     }
-    float x0[8], x1[8];
-    uint4 q0 = make_uint4(0, 0, 0, 0), q1 = make_uint4(0, 0, 0, 0);
-    if (h0) q0 = __ldg(reinterpret_cast<const uint4*>(w + e0));
-    if (h1) q1 = __ldg(reinterpret_cast<const uint4*>(w + e1));
-    uint32_t w0[4] = {q0.x, q0.y, q0.z, q0.w}, w1[4] = {q1.x, q1.y, q1.z, q1.w};
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      x0[2 * j] = bf16_bits_to_f32(w0[j] & 0xFFFFu);
-      x0[2 * j + 1] = bf16_bits_to_f32(w0[j] >> 16);
-      x1[2 * j] = bf16_bits_to_f32(w1[j] & 0xFFFFu);
-      x1[2 * j + 1] = bf16_bits_to_f32(w1[j] >> 16);
-    }
-    float m0 = 0.0f, m1 = 0.0f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      m0 = fmaxf(m0, fabsf(x0[i]));
-      m1 = fmaxf(m1, fabsf(x1[i]));
-    }
-    m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, 1));
-    m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, 1));
-    BlockScale b0 = block_scale(m0, sg0, t60), b1 = block_scale(m1, sg1, t61);
-    float dq0[8], dq1[8];
-    quant8(x0, b0, dq0);
-    quant8(x1, b1, dq1);
-    uint32_t o0[4], o1[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      __nv_bfloat162 p0 = __floats2bfloat162_rn(dq0[2 * j], dq0[2 * j + 1]);
-      __nv_bfloat162 p1 = __floats2bfloat162_rn(dq1[2 * j], dq1[2 * j + 1]);
-      o0[j] = *reinterpret_cast<uint32_t*>(&p0);
-      o1[j] = *reinterpret_cast<uint32_t*>(&p1);
-    }
-    if (h0) *reinterpret_cast<uint4*>(out + e0) = make_uint4(o0[0], o0[1], o0[2], o0[3]);
-    if (h1) *reinterpret_cast<uint4*>(out + e1) = make_uint4(o1[0], o1[1], o1[2], o1[3]);
+    uint4 o0, o1;
+    qdq_half(q0, sc0.s_g, sc0.t6, o0);
+    qdq_half(q1, sc1.s_g, sc1.t6, o1);
+    if (h0) *reinterpret_cast<uint4*>(out + e0) = o0;
+    if (h1) *reinterpret_cast<uint4*>(out + e1) = o1;
+    e0 += 512;
+    e1 += 512;
   }
 }
 

@@ -257,6 +257,21 @@ def test_weight_qdq_matches_oracle(dev, orc):
         assert np.array_equal(got[t], ref), np.argwhere(got[t] != ref)[:5]
 
 
+@pytest.mark.parametrize("n,elems", [(3, 16), (300, 512 * 7 + 16), (7, 512 * 5), (2, 2 << 20)])
+def test_weight_qdq_shapes_match_oracle(dev, orc, n, elems):
+    """Tensor boundaries inside and at the edges of 512-element chunks, tiny and 4 MB tensors."""
+    w = syn.normal_bf16(1, 9, n, elems, 0.02)
+    h = min(32, elems)
+    w[0, :h] = syn.normal_bf16(1, 10, 1, h, 1.28)[0]  # a heavier head in one tensor
+    out, s_g = R.weight_qdq(to_dev(w, dev))
+    torch.cuda.synchronize()
+    got = bf16_bits(out).reshape(n, elems)
+    for t in sorted({0, 1 % n, n // 2, n - 1}):
+        ref, s_ref = orc.weight_qdq(w[t])
+        assert s_g[t].item() == float(s_ref)
+        assert np.array_equal(got[t], ref), (t, np.argwhere(got[t] != ref)[:5])
+
+
 def test_weight_qdq_trainer_full_sampled(dev, orc):
     """The trainer fake-quant configuration at full size: 2^31 bf16 N(0, 0.02) weights as 1024
     tensors of 1024 x 2048 (one scale each), then as a single tensor (one scale); sampled tensors
