@@ -1,18 +1,23 @@
-"""Benchmark of the NVFP4 W4A4 + RAC MoE prefill expert block on B200.
+"""Benchmark of the NVFP4 W4A4 + RAC hot path on B200.
 
-One step = the rollout hot path over one batch, with weights already packed (packing runs
-once per trainer -> rollout sync, not per step):
-    per-tensor amax of X -> quantise X (+ residual on the calibrated channels) with the
-    gather into expert-sorted, 128-padded rows -> grouped gate_up GEMM (W4A4 + RAC) with the
-    SwiGLU + amax epilogue -> quantise h (+ residual) -> grouped down GEMM (W4A4 + RAC).
-Workload: 4096 tokens, hidden 2048, 128 experts, top-8 of softmax(N(0,1) logits), gate_up
-128 x (1536 x 2048), down 128 x (2048 x 768), r = 0.5; synthetic seeded inputs.
+Default workload (moe_prefill), the MoE prefill expert block, one step = the rollout hot path
+over one batch with weights already packed (packing runs once per trainer -> rollout sync):
+    per-tensor amax of X -> quantise X (+ residual on the calibrated channels) scattered into
+    expert-sorted, 128-padded rows -> grouped gate_up GEMM (W4A4 + RAC) with the SwiGLU + amax
+    epilogue -> quantise h (+ residual) -> grouped down GEMM (W4A4 + RAC).
+    4096 tokens, hidden 2048, 128 experts, top-8 of softmax(N(0,1) logits), gate_up
+    128 x (1536 x 2048), down 128 x (2048 x 768), r = 0.5; synthetic seeded inputs.
+Other workloads (--workload): dense (8192 x 4096 x 4096 projection), moe_decode (64 tokens,
+hidden 7168, 256 experts, swap-AB decode GEMMs), moe_prefill_layer / moe_decode_layer (the
+same with the device router, dispatch plan and combine: no host work per step), qdq /
+qdq_single (trainer fake-quant of 2^31 weights), sweep (r in {0, 0.25, 0.5, 1}).
 
-Metric: effective TFLOP/s of the step's GEMMs, 2*rows*N*(K + K') summed over gate_up and down
-(the residual loop counted, as it is part of the method), over the measured step time.
-Also reported: act-quant GB/s and the roofline of the dominant kernel (grouped gate_up).
+Metric: effective TFLOP/s of the step's GEMMs, 2*rows*N*(K + K') summed over the GEMMs (the
+residual loop counted, as it is part of the method), over the measured step time; GB/s for
+the fake-quant workloads.  Also reported: act-quant GB/s, per-kernel times and the roofline of
+the dominant kernel.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload W] [--impl reference]
 Under torchrun every rank runs its own replica (weak scaling, no data-path collective);
 rank 0 prints one JSON line.
 """

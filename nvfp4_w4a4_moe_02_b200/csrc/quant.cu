@@ -79,34 +79,43 @@ __device__ __forceinline__ float reduce_partials(const float* partial, int P) {
 
 // ----------------------------------------------------------------------------------------
 // K2 / K7 / calibration: the row quantiser.  One warp per row, 512 elements per warp
-// iteration: lane l loads elements [it*512 + 8l, +8) and [it*512 + 256 + 8l, +8), so lanes
-// (2m, 2m+1) hold the two halves of block it*32 + m and of block it*32 + 16 + m.
+// iteration: lane l owns the 16-element block [it*512 + 16l, +16), so a block's scale is
+// computed once, by one lane, with no shuffles; its 8 bytes of codes and its scale byte are
+// stored by that lane.
 //
 // The residual pass over the selected channels (activation mode) or the raw selected columns
-// (weight pack) runs after the main pass from a per-warp stash of the row and of each block's
-// (d, 1/d): lane pairs take 16 consecutive compact positions, read their channel numbers and
-// re-derive x, its code and DQ = e*d for exactly those channels.
+// (weight pack) runs after the main pass: each lane takes 16 consecutive compact positions, reads
+// their channel numbers, gathers x from the row again (it was just read: the loads hit L1) and
+// re-derives its code and DQ = e*d from a per-warp stash of each block's (d, 1/d).  Keeping only
+// the block scales in shared memory, not the row, leaves room for more warps per SM.
 //
 // SPLIT (activations with few rows, e.g. the tokens of one decode step): a whole CTA works on
 // one row; warp w takes the 512-element chunks w, w + nwarps, ... of both passes and the stash
 // is shared by the CTA, so a 64-token batch still occupies every warp of 64 CTAs.
 // ----------------------------------------------------------------------------------------
 
-// Scale word of a k64 group: lanes 8g..8g+7 own blocks 4g..4g+3 (the pair (2m, 2m+1) owns
-// block m); lane 8g gathers the codes held by lanes 8g, 8g+2, 8g+4, 8g+6.
-__device__ __forceinline__ uint32_t scale_word(uint32_t S) {
-  uint32_t s1 = __shfl_down_sync(0xffffffffu, S, 2);
-  uint32_t s2 = __shfl_down_sync(0xffffffffu, S, 4);
-  uint32_t s3 = __shfl_down_sync(0xffffffffu, S, 6);
-  return S | (s1 << 8) | (s2 << 16) | (s3 << 24);
-}
-
-// destinations of the current row: the row itself, or up to `fanout` rows in scatter mode
+// destinations of the current row: the row itself, or up to `fanout` (<= 64) rows in scatter
+// mode, read once per row into the warp's registers (lane l holds entries l and l + 32) so that
+// the per-chunk store loops pick them with a shuffle instead of a dependent global load
 struct Dests {
-  const int32_t* list;  // null: single destination `row`
+  bool scatter;
   int n;
   int64_t row;
-  __device__ __forceinline__ int64_t get(int j) const { return list ? (int64_t)__ldg(list + j) : row; }
+  int32_t mine0, mine1;
+  __device__ __forceinline__ void load(const int32_t* list, int fanout) {
+    const int lane = threadIdx.x & 31;
+    scatter = true;
+    n = fanout;
+    mine0 = lane < fanout ? __ldg(list + lane) : -1;
+    mine1 = lane + 32 < fanout ? __ldg(list + 32 + lane) : -1;
+  }
+  // all lanes call get(j) with the same j
+  __device__ __forceinline__ int64_t get(int j) const {
+    if (!scatter) return row;
+    const int32_t v0 = __shfl_sync(0xffffffffu, mine0, j & 31);
+    const int32_t v1 = __shfl_sync(0xffffffffu, mine1, j & 31);
+    return (int64_t)(j < 32 ? v0 : v1);
+  }
 };
 
 __device__ __forceinline__ void unpack8(const uint4 raw, float x[8]) {
@@ -131,18 +140,16 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   const int nwarps = blockDim.x >> 5;
-  const int64_t K = a.K;
+  const int32_t K = (int32_t)a.K;  // <= 32768: offsets inside a row fit in 32 bits
   const int32_t Kp = a.Kp;
   constexpr bool kHasSel = (MODE == kModeAct || MODE == kModePack);
   const bool use_sel = kHasSel && Kp > 0;
 
-  // CTA-shared channel list (int16), then per warp (per CTA when SPLIT): the row's bf16 bits
-  // and each block's (d, 1/d)
+  // CTA-shared channel list (int16), then per warp (per CTA when SPLIT) each block's (d, 1/d)
   int16_t* sel_s = reinterpret_cast<int16_t*>(smem_raw);
   const size_t sel_bytes = use_sel ? (((size_t)Kp * 2 + 15) / 16) * 16 : 0;
-  const size_t warp_bytes = use_sel ? (((size_t)K * 2 + 15) / 16) * 16 + (size_t)(K / 16) * 8 : 0;
-  uint16_t* row_s = reinterpret_cast<uint16_t*>(smem_raw + sel_bytes + (SPLIT ? 0 : warp) * warp_bytes);
-  float2* dinv_s = reinterpret_cast<float2*>(reinterpret_cast<unsigned char*>(row_s) + ((K * 2 + 15) / 16) * 16);
+  const size_t warp_bytes = use_sel ? (size_t)(K / 16) * 8 : 0;
+  float2* dinv_s = reinterpret_cast<float2*>(smem_raw + sel_bytes + (SPLIT ? 0 : warp) * warp_bytes);
   if (use_sel) {
     for (int32_t j = threadIdx.x; j < Kp; j += blockDim.x) {
       int32_t c = a.sel[j];
@@ -160,22 +167,29 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   const int64_t kp64 = Kp / 64;
   const bool scatter = (MODE == kModeAct && a.row_scatter != nullptr);
   const int64_t n_rows = scatter ? a.src_rows : a.rows_out;
+  const bool slab16 = a.sf_slab16 != 0;
   int64_t cached_slab = -1;
   float s_g = 0.0f, t6 = 0.0f;
 
+  // byte offset of a row's part of a scale-atom array, and of a block's part (see sf_offset)
+  auto sf_row = [&](int64_t r, int64_t groups) -> int64_t {
+    return slab16 ? (r >> 4) * groups * 512 + (r & 15) * 16
+                  : (r >> 7) * groups * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4;
+  };
+  auto sf_blk = [](int32_t kb) -> int32_t { return (kb >> 2) * 512 + (kb & 3); };
+
   const int64_t row_first = SPLIT ? (int64_t)blockIdx.x : (int64_t)blockIdx.x * nwarps + warp;
   const int64_t row_step = SPLIT ? (int64_t)gridDim.x : (int64_t)gridDim.x * nwarps;
-  const int64_t chunk0 = SPLIT ? 512 * warp : 0;          // this warp's first chunk of a row
-  const int64_t chunk_step = SPLIT ? 512 * nwarps : 512;  // distance to its next chunk
+  const int32_t chunk0 = SPLIT ? 512 * warp : 0;          // this warp's first chunk of a row
+  const int32_t chunk_step = SPLIT ? 512 * nwarps : 512;  // distance to its next chunk
   for (int64_t row = row_first; row < n_rows; row += row_step) {
     // ---- source row, destinations, scale
     int64_t slab = (MODE == kModePack) ? row / a.rows_per_slab : 0;
     int64_t r_in_slab = row - slab * a.rows_per_slab;
     int64_t src_row = r_in_slab;
-    Dests dst{nullptr, 1, row};
+    Dests dst{false, 1, row, -1, -1};
     if (scatter) {
-      dst.list = a.row_scatter + row * a.fanout;
-      dst.n = a.fanout;
+      dst.load(a.row_scatter + row * a.fanout, a.fanout);
     } else if (MODE == kModeAct && a.row_gather != nullptr) {
       src_row = (r_in_slab < a.rows_per_slab) ? a.row_gather[r_in_slab] : -1;
     }
@@ -197,133 +211,105 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
     }
     const uint16_t* srow = a.src + slab * a.src_slab_stride + (valid ? src_row : 0) * a.ld;
 
-    // ---- main pass (the loads of the next 512 elements are issued before this block's math)
-    uint4 n0 = (valid && chunk0 + 8 * lane < K) ? __ldg(reinterpret_cast<const uint4*>(srow + chunk0 + 8 * lane))
-                                                : make_uint4(0, 0, 0, 0);
-    uint4 n1 = (valid && chunk0 + 256 + 8 * lane < K)
-                   ? __ldg(reinterpret_cast<const uint4*>(srow + chunk0 + 256 + 8 * lane))
-                   : make_uint4(0, 0, 0, 0);
-    for (int64_t base = chunk0; base < K; base += chunk_step) {
-      const int64_t e0 = base + 8 * lane, e1 = base + 256 + 8 * lane;
-      const bool h0 = e0 < K, h1 = e1 < K;  // K % 64 == 0: uniform over lane pairs and 8-lane groups
+    // ---- main pass: lane l owns the 16-element block starting at chunk + 16 l (the next
+    // chunk's loads are issued before this block's arithmetic)
+    auto load16 = [&](int32_t e, uint4& u0, uint4& u1) {
+      const bool ok = valid && e < K;
+      u0 = ok ? __ldg(reinterpret_cast<const uint4*>(srow + e)) : make_uint4(0, 0, 0, 0);
+      u1 = ok ? __ldg(reinterpret_cast<const uint4*>(srow + e + 8)) : make_uint4(0, 0, 0, 0);
+    };
+    uint4 n0, n1;
+    load16(chunk0 + 16 * lane, n0, n1);
+    for (int32_t base = chunk0; base < K; base += chunk_step) {
+      const int32_t e = base + 16 * lane;
+      const bool h = e < K;  // K % 16 == 0: a block is wholly inside or outside
       const uint4 r0 = n0, r1 = n1;
-      if (base + chunk_step < K) {
-        const int64_t f0 = e0 + chunk_step, f1 = e1 + chunk_step;
-        n0 = (valid && f0 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + f0)) : make_uint4(0, 0, 0, 0);
-        n1 = (valid && f1 < K) ? __ldg(reinterpret_cast<const uint4*>(srow + f1)) : make_uint4(0, 0, 0, 0);
-      }
-      float x0[8], x1[8];
-      unpack8(r0, x0);
-      unpack8(r1, x1);
-      const BlockScale b0 = block_scale(pair_max8(x0), s_g, t6);
-      const BlockScale b1 = block_scale(pair_max8(x1), s_g, t6);
+      if (base + chunk_step < K) load16(e + chunk_step, n0, n1);
+      float x[16];
+      unpack8(r0, x);
+      unpack8(r1, x + 8);
+      float b = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(x[i]));
+      const BlockScale bs = block_scale(b, s_g, t6);
       if (MODE == kModeCal) {
-        float dq0[8], dq1[8];
-        quant8(x0, b0, dq0);
-        quant8(x1, b1, dq1);
-        float* rr = a.resid_all + row * K;
-        if (h0) {
-          *reinterpret_cast<float4*>(rr + e0) = make_float4(__fsub_rn(x0[0], dq0[0]), __fsub_rn(x0[1], dq0[1]),
-                                                            __fsub_rn(x0[2], dq0[2]), __fsub_rn(x0[3], dq0[3]));
-          *reinterpret_cast<float4*>(rr + e0 + 4) = make_float4(__fsub_rn(x0[4], dq0[4]), __fsub_rn(x0[5], dq0[5]),
-                                                                __fsub_rn(x0[6], dq0[6]), __fsub_rn(x0[7], dq0[7]));
-        }
-        if (h1) {
-          *reinterpret_cast<float4*>(rr + e1) = make_float4(__fsub_rn(x1[0], dq1[0]), __fsub_rn(x1[1], dq1[1]),
-                                                            __fsub_rn(x1[2], dq1[2]), __fsub_rn(x1[3], dq1[3]));
-          *reinterpret_cast<float4*>(rr + e1 + 4) = make_float4(__fsub_rn(x1[4], dq1[4]), __fsub_rn(x1[5], dq1[5]),
-                                                                __fsub_rn(x1[6], dq1[6]), __fsub_rn(x1[7], dq1[7]));
+        float dq[16];
+        quant8(x, bs, dq);
+        quant8(x + 8, bs, dq + 8);
+        if (h) {
+          float* rr = a.resid_all + row * K + e;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<float4*>(rr + 4 * q) =
+                make_float4(__fsub_rn(x[4 * q], dq[4 * q]), __fsub_rn(x[4 * q + 1], dq[4 * q + 1]),
+                            __fsub_rn(x[4 * q + 2], dq[4 * q + 2]), __fsub_rn(x[4 * q + 3], dq[4 * q + 3]));
         }
         continue;
       }
-      const uint32_t c0 = quant8_codes(x0, b0), c1 = quant8_codes(x1, b1);
-      const uint32_t w0 = scale_word(b0.S), w1 = scale_word(b1.S);
-      if (use_sel) {
-        // stash the row and the block scales for the residual pass
-        if (h0) *reinterpret_cast<uint4*>(row_s + e0) = r0;
-        if (h1) *reinterpret_cast<uint4*>(row_s + e1) = r1;
-        if ((lane & 1) == 0) {
-          if (h0) dinv_s[e0 >> 4] = make_float2(b0.d, b0.inv);
-          if (h1) dinv_s[e1 >> 4] = make_float2(b1.d, b1.inv);
-        }
-      }
+      const uint2 c = make_uint2(quant8_codes(x, bs), quant8_codes(x + 8, bs));
+      const int32_t kb = e >> 4;
+      if (use_sel && h) dinv_s[kb] = make_float2(bs.d, bs.inv);  // block scales for the residual pass
+      const int32_t blk = sf_blk(kb);
       for (int j = 0; j < dst.n; ++j) {
         const int64_t drow = dst.get(j);
-        if (drow < 0) continue;
+        if (drow < 0 || !h) continue;
         if (drow >= a.rows_out) {
           report_status(a.status, kErrInvalid);
           continue;
         }
-        uint8_t* crow = a.codes + drow * (K / 2);
-        if (h0) *reinterpret_cast<uint32_t*>(crow + e0 / 2) = c0;
-        if (h1) *reinterpret_cast<uint32_t*>(crow + e1 / 2) = c1;
-        if ((lane & 7) == 0) {
-          if (h0) *reinterpret_cast<uint32_t*>(a.sf + sf_offset_any(drow, e0 >> 4, k64, a.sf_slab16)) = w0;
-          if (h1) *reinterpret_cast<uint32_t*>(a.sf + sf_offset_any(drow, e1 >> 4, k64, a.sf_slab16)) = w1;
-        }
+        *reinterpret_cast<uint2*>(a.codes + drow * (K / 2) + e / 2) = c;
+        a.sf[sf_row(drow, k64) + blk] = (uint8_t)bs.S;
       }
     }
 
-    // ---- residual pass over the compact selected channels
+    // ---- residual pass: lane l owns the compact 16 positions starting at chunk + 16 l
     if (use_sel) {
-      if (SPLIT) __syncthreads(); else __syncwarp();  // the whole row is stashed
-      for (int64_t base = chunk0; base < Kp; base += chunk_step) {
-        const int64_t p0 = base + 8 * lane, p1 = base + 256 + 8 * lane;
-        const bool h0 = p0 < Kp, h1 = p1 < Kp;
-        float v[2][8];
+      if (SPLIT) __syncthreads(); else __syncwarp();  // every block's scale is stashed
+      for (int32_t base = chunk0; base < Kp; base += chunk_step) {
+        const int32_t p = base + 16 * lane;
+        const bool h = p < Kp;
+        int32_t ch[16];
+        {
+          const uint4 c0 = h ? *reinterpret_cast<const uint4*>(sel_s + p) : make_uint4(0, 0, 0, 0);
+          const uint4 c1 = h ? *reinterpret_cast<const uint4*>(sel_s + p + 8) : make_uint4(0, 0, 0, 0);
+          const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          const int64_t p = hh ? p1 : p0;
-          const bool ok = hh ? h1 : h0;
-          int32_t ch[8];
-          {
-            const uint4 cv = ok ? *reinterpret_cast<const uint4*>(sel_s + p) : make_uint4(0, 0, 0, 0);
-            const uint32_t w[4] = {cv.x, cv.y, cv.z, cv.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              ch[2 * j] = (int32_t)(int16_t)(w[j] & 0xFFFFu);
-              ch[2 * j + 1] = (int32_t)(int16_t)(w[j] >> 16);
-            }
-          }
-          float x[8];
-#pragma unroll
-          for (int i = 0; i < 8; ++i) x[i] = bf16_bits_to_f32(row_s[ch[i]]);
-          if (MODE == kModePack) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[hh][i] = x[i];
-          } else {
-            // re-derive the channel's code under its own block scale, then r = x - e*d
-            float sc[8], d[8];
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float2 di = dinv_s[ch[i] >> 4];
-              d[i] = di.x;
-              sc[i] = __fmul_rn(x[i], di.y);
-            }
-            float e[8];
-            e2m1_decode8(e2m1_encode8(sc), e);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[hh][i] = __fsub_rn(x[i], d[i] == 0.0f ? 0.0f : __fmul_rn(e[i], d[i]));
-          }
-          if (!ok || !valid) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) v[hh][i] = 0.0f;
+          for (int q = 0; q < 8; ++q) {
+            ch[2 * q] = (int32_t)(int16_t)(w[q] & 0xFFFFu);
+            ch[2 * q + 1] = (int32_t)(int16_t)(w[q] >> 16);
           }
         }
-        const BlockScale b0 = block_scale(pair_max8(v[0]), s_g, t6);
-        const BlockScale b1 = block_scale(pair_max8(v[1]), s_g, t6);
-        const uint32_t c0 = quant8_codes(v[0], b0), c1 = quant8_codes(v[1], b1);
-        const uint32_t w0 = scale_word(b0.S), w1 = scale_word(b1.S);
+        float v[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) v[i] = (h && valid) ? bf16_bits_to_f32(__ldg(srow + ch[i])) : 0.0f;
+        if (MODE != kModePack) {
+          // re-derive each channel's code under its own block scale, then r = x - e*d
+#pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
+            float sc[8], d[8], ev[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const float2 di = dinv_s[ch[8 * hh + i] >> 4];
+              d[i] = di.x;
+              sc[i] = __fmul_rn(v[8 * hh + i], di.y);
+            }
+            e2m1_decode8(e2m1_encode8(sc), ev);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              v[8 * hh + i] = __fsub_rn(v[8 * hh + i], d[i] == 0.0f ? 0.0f : __fmul_rn(ev[i], d[i]));
+          }
+        }
+        float b = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(v[i]));
+        const BlockScale bs = block_scale(b, s_g, t6);
+        const uint2 c = make_uint2(quant8_codes(v, bs), quant8_codes(v + 8, bs));
+        const int32_t blk = sf_blk(p >> 4);
         for (int j = 0; j < dst.n; ++j) {
           const int64_t drow = dst.get(j);
-          if (drow < 0 || drow >= a.rows_out) continue;
-          uint8_t* crow = a.rcodes + drow * (Kp / 2);
-          if (h0) *reinterpret_cast<uint32_t*>(crow + p0 / 2) = c0;
-          if (h1) *reinterpret_cast<uint32_t*>(crow + p1 / 2) = c1;
-          if ((lane & 7) == 0) {
-            if (h0) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset_any(drow, p0 >> 4, kp64, a.sf_slab16)) = w0;
-            if (h1) *reinterpret_cast<uint32_t*>(a.rsf + sf_offset_any(drow, p1 >> 4, kp64, a.sf_slab16)) = w1;
-          }
+          if (drow < 0 || drow >= a.rows_out || !h) continue;
+          *reinterpret_cast<uint2*>(a.rcodes + drow * (Kp / 2) + p / 2) = c;
+          a.rsf[sf_row(drow, kp64) + blk] = (uint8_t)bs.S;
         }
       }
       if (SPLIT) __syncthreads(); else __syncwarp();  // stash reads done before the next row
@@ -516,7 +502,7 @@ cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64
 
 size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps) {
   if (Kp <= 0) return 16;
-  return (size_t)((Kp * 2 + 15) / 16) * 16 + (size_t)warps * ((size_t)((K * 2 + 15) / 16) * 16 + (size_t)(K / 16) * 8);
+  return (size_t)((Kp * 2 + 15) / 16) * 16 + (size_t)warps * (size_t)(K / 16) * 8;
 }
 
 cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
