@@ -117,6 +117,7 @@ class MoEStep:
         self.scatter = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0],
                                                       wl.topk_ids.shape[1])).to(dev)
         self.offsets = torch.from_numpy(off.astype(np.int32)).to(dev)
+        self.expert_rows = torch.from_numpy(np.asarray(wl.counts, dtype=np.int32)).to(dev)
         self.x = to(wl.x)
         # preallocated outputs (the step allocates nothing)
         P = R.Packed
@@ -143,13 +144,14 @@ class MoEStep:
         if "g0" in ev:
             ev["g0"].record()
         R.grouped_w4a4_rac_moe(self.a, self.ar, self.offsets, self.pgu, self.pgus, swiglu=True, y=self.h,
-                               amax_out=self.amax_h, status=self.status)
+                               amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
         if "q1" in ev:
             ev["q1"].record()
         R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
         if "d0" in ev:
             ev["d0"].record()
-        R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.offsets, self.pdn, self.pdns, y=self.y, status=self.status)
+        R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.offsets, self.pdn, self.pdns, y=self.y, status=self.status,
+                               expert_rows=self.expert_rows)
         if "end" in ev:
             ev["end"].record()
         return self.y
@@ -303,6 +305,7 @@ class MoEBlockStep:
         self.w = torch.empty(T, k, dtype=torch.float32, device=dev)
         self.off = torch.empty(wl.E + 1, dtype=torch.int32, device=dev)
         self.rows = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.expert_rows = torch.empty(wl.E, dtype=torch.int32, device=dev)
         self.se = torch.empty(self.n_slots, dtype=torch.int32, device=dev) if decode else None
         self.sc = torch.empty(self.n_slots, dtype=torch.int32, device=dev) if decode else None
         self.a = P.empty(self.cap, wl.H, rows_padded=self.cap, device=dev, zero=True, sf_layout=lay)
@@ -324,7 +327,7 @@ class MoEBlockStep:
                          status=self.status)
         R.moe_dispatch_plan(self.ids, self.wl.E, self.pad, rows_capacity=self.cap, n_slots=self.n_slots,
                             offsets=self.off, row_scatter=self.rows, slot_expert=self.se, slot_count=self.sc,
-                            status=self.status)
+                            status=self.status, expert_rows=self.expert_rows)
         if "q0" in ev:
             ev["q0"].record()
         R.nvfp4_quantize_scatter(self.x if x is None else x, self.rows, self.cap, self.sel_gu, out=self.a,
@@ -336,7 +339,7 @@ class MoEBlockStep:
                                           y=self.h, amax_out=self.amax_h, status=self.status)
         else:
             R.grouped_w4a4_rac_moe(self.a, self.ar, self.off, self.pgu, self.pgus, swiglu=True, y=self.h,
-                                   amax_out=self.amax_h, status=self.status)
+                                   amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
         if "q1" in ev:
             ev["q1"].record()
         R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
@@ -346,7 +349,8 @@ class MoEBlockStep:
             R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.se, self.sc, self.pdn, self.pdns, y=self.ye,
                                           status=self.status)
         else:
-            R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.off, self.pdn, self.pdns, y=self.ye, status=self.status)
+            R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.off, self.pdn, self.pdns, y=self.ye, status=self.status,
+                                   expert_rows=self.expert_rows)
         if "c0" in ev:
             ev["c0"].record()
         R.moe_combine(self.ye, self.rows, self.w, out=self.y, status=self.status)

@@ -208,15 +208,20 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, con
 /*                    occupies rows [expert_offsets[e], expert_offsets[e+1]).                 */
 /*   expert_offsets   device int32 [E+1], non-decreasing multiples of 128, offsets[0] = 0,   */
 /*                    offsets[E] <= a->rows_padded.  Read on the device only.                */
+/*   expert_rows      optional device int32 [E]: rows of segment e that hold tokens (the     */
+/*                    rest is padding).  Output boxes of 32 rows that hold padding only are  */
+/*                    not written (their contents stay as they were) and the SwiGLU amax     */
+/*                    covers the counted rows.  NULL: every row is written (padding as 0).  */
 /*   w, w_sel         pack_weights output with slabs = E.  alpha_e = a.s_g * w.s_g[e].        */
 /*   ep               NVFP4_EPI_NONE: y [offsets[E] x N]; NVFP4_EPI_SWIGLU_AMAX: y bf16      */
 /*                    [offsets[E] x N/2] and max|y| folded into *amax_out (device float, the  */
 /*                    call zeroes it first).  Rows of padding come out as zeros.             */
 /* ---------------------------------------------------------------------------------------- */
 nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
-                                  int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N,
-                                  int64_t K, int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y,
-                                  int64_t ldy, float* amax_out, int32_t* dev_status, void* stream);
+                                  const int32_t* expert_rows, int32_t E, const nvfp4_tensor* w,
+                                  const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp, nvfp4_epilogue ep,
+                                  nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
+                                  void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* grouped_w4a4_rac_moe_decode -- the grouped GEMM above for decode, where each expert sees   */
@@ -267,12 +272,14 @@ size_t moe_dispatch_workspace_size(int32_t E);
 /*                  in *dev_status; the GEMMs then do nothing.                                 */
 /*   row_scatter    int32 [T x k]: row of pair (t, j), the row_scatter of                      */
 /*                  nvfp4_quantize_scatter (fanout k) and of moe_combine; -1 if unrouted.     */
+/*   expert_rows    optional int32 [E]: tokens routed to each expert (the expert_rows of       */
+/*                  grouped_w4a4_rac_moe).                                                    */
 /*   slot_expert, slot_count  optional int32 [n_slots] (pad == 16): the decode slot tables;    */
 /*                  slots past the used ones get expert -1, which the decode GEMM skips.      */
 nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E, int32_t pad,
                                int64_t rows_capacity, int32_t* expert_offsets, int32_t* row_scatter,
-                               int32_t* slot_expert, int32_t* slot_count, int32_t n_slots, void* workspace,
-                               size_t workspace_bytes, int32_t* dev_status, void* stream);
+                               int32_t* expert_rows, int32_t* slot_expert, int32_t* slot_count, int32_t n_slots,
+                               void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 /* moe_combine -- out[t, :] = sum_j topk_w[t, j] * y[row_scatter[t, j], :] (binary32 sums in   */
 /* j order, bf16 out); y bf16 with y_rows rows, pitch ldy; out bf16 [T x H], pitch ldo;       */
 /* H % 8 == 0.  A row < 0 contributes nothing; a row >= y_rows is NVFP4_ERR_INVALID_ARG.      */

@@ -525,7 +525,8 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, con
 }
 
 nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
-                                  int32_t E, const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N, int64_t K,
+                                  const int32_t* expert_rows, int32_t E, const nvfp4_tensor* w,
+                                  const nvfp4_tensor* w_sel, int64_t N, int64_t K,
                                   int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y, int64_t ldy,
                                   float* amax_out, int32_t* dev_status, void* stream) {
   g_last_error.clear();
@@ -546,6 +547,7 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
       gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, a ? a->rows_padded : 0, bn, maps, &g);
   if (st != NVFP4_OK) return st;
   g.offsets = expert_offsets;
+  g.expert_rows = expert_rows;
   g.E = E;
   g.M = a->rows_padded;
   g.m_blocks_dense = 0;
@@ -673,7 +675,8 @@ size_t moe_dispatch_workspace_size(int32_t E) { return round_up((size_t)(E > 0 ?
 
 nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E, int32_t pad,
                                int64_t rows_capacity, int32_t* expert_offsets, int32_t* row_scatter,
-                               int32_t* slot_expert, int32_t* slot_count, int32_t n_slots, void* workspace,
+                               int32_t* expert_rows, int32_t* slot_expert, int32_t* slot_count, int32_t n_slots,
+                               void* workspace,
                                size_t workspace_bytes, int32_t* dev_status, void* stream) {
   g_last_error.clear();
   if (T < 0 || k <= 0 || E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T >= 0, k > 0 and E > 0 required");
@@ -686,8 +689,8 @@ nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, in
   if (!workspace || workspace_bytes < moe_dispatch_workspace_size(E)) return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = launch_dispatch_plan(topk_ids, T, k, E, pad, rows_capacity, reinterpret_cast<int32_t*>(workspace),
-                                       expert_offsets, row_scatter, slot_expert, slot_count, n_slots, num_sms(),
-                                       dev_status, s);
+                                       expert_offsets, row_scatter, expert_rows, slot_expert, slot_count, n_slots,
+                                       num_sms(), dev_status, s);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "dispatch plan launch");
 }
 

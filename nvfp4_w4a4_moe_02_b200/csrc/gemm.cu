@@ -283,7 +283,12 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
       tc_fence_after();
       const int64_t row = mb * BM + quad * 32 + lane;
-      const bool row_ok = row < row_limit && row < args.rows_capacity;
+      // with per-expert row counts, rows past the expert's tokens are padding: a 32-row output
+      // box that holds no token row is not stored
+      const int64_t rows_e = (grouped && args.expert_rows != nullptr)
+                                 ? (int64_t)__ldg(args.offsets + e) + __ldg(args.expert_rows + e)
+                                 : row_limit;
+      const bool row_ok = row < row_limit && row < args.rows_capacity && row < rows_e;
       const float alpha = __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));
       const uint32_t t_row = tmem_base + (uint32_t)(acc ? C::ACC1_BASE : 0) + ((uint32_t)(quad * 32) << 16);
       // chunk i of this warp: plain -> columns half*BN/2 + 32i; SwiGLU -> output features
@@ -322,6 +327,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // swizzled layout (16-byte chunk c of row r at chunk c ^ (r % 8)), stored by one TMA copy
       const uint32_t stg = sbase + C::OFF_STG + (uint32_t)((warp - 2) * C::STG * C::BOX_BYTES);
       const int32_t y0 = (int32_t)(mb * BM + quad * 32);
+      const bool box_live = (int64_t)y0 < rows_e;
       auto put_box = [&](int slot, const uint32_t (&w)[32], int32_t x) {
         // at most STG - 1 earlier stores of this warp may still be reading the staging boxes
         if (lane == 0) bulk_wait_group_read<C::STG - 1>();
@@ -337,7 +343,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           bulk_commit_group();
         }
       };
-      if (args.epi == 0 && args.out_bf16) {
+      if (!box_live) {
+        // padding only: nothing to store
+      } else if (args.epi == 0 && args.out_bf16) {
         // 64 columns per box
 #pragma unroll
         for (int b = 0; b < NCH / 2; ++b) {

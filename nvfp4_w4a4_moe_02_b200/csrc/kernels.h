@@ -68,6 +68,7 @@ struct GemmArgs {
   int32_t N;                 // output columns of the MMA (before the SwiGLU halving)
   int32_t n_blocks;          // N / BN
   const int32_t* offsets;    // grouped: device [E+1]; dense: nullptr
+  const int32_t* expert_rows;  // grouped, optional device [E]: rows holding tokens per segment
   int32_t E;
   int64_t M;                 // dense: valid rows (stores masked beyond)
   int32_t m_blocks_dense;    // dense: ceil(M/128)
@@ -123,8 +124,9 @@ constexpr int kMaxRouteExperts = 1024;
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* status,
                               cudaStream_t st);
 cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, int pad, int64_t rows_capacity,
-                                 int32_t* counts, int32_t* offsets, int32_t* row_scatter, int32_t* slot_expert,
-                                 int32_t* slot_count, int n_slots, int num_sms, int32_t* status, cudaStream_t st);
+                                 int32_t* counts, int32_t* offsets, int32_t* row_scatter, int32_t* expert_rows,
+                                 int32_t* slot_expert, int32_t* slot_count, int n_slots, int num_sms,
+                                 int32_t* status, cudaStream_t st);
 cudaError_t launch_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* rows, const float* w,
                            int64_t T, int k, int64_t H, uint16_t* out, int64_t ldo, int num_sms, int32_t* status,
                            cudaStream_t st);

@@ -97,8 +97,8 @@ __global__ void count_kernel(const int32_t* __restrict__ ids, int64_t n, int E, 
 // one CTA: padded segment starts (exclusive scan), then the decode slot tables
 __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ counts, int E, int pad,
                                                        int64_t rows_capacity, int32_t* __restrict__ offsets,
-                                                       int32_t* slot_expert, int32_t* slot_count, int n_slots,
-                                                       int32_t* status) {
+                                                       int32_t* expert_rows, int32_t* slot_expert,
+                                                       int32_t* slot_count, int n_slots, int32_t* status) {
   __shared__ int64_t part[1024];
   const int per = (E + blockDim.x - 1) / blockDim.x;
   const int e0 = threadIdx.x * per;
@@ -120,6 +120,7 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
   for (int e = e0; e < min(E, e0 + per); ++e) {
     offsets[e] = fits ? (int32_t)run : 0;
     const int c = counts[e];
+    if (expert_rows != nullptr) expert_rows[e] = fits ? c : 0;
     if (slot_expert != nullptr && fits) {
       const int s0 = (int)(run / 16);
       for (int s = 0; 16 * s < c; ++s) {
@@ -220,8 +221,9 @@ cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int3
 }
 
 cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, int pad, int64_t rows_capacity,
-                                 int32_t* counts, int32_t* offsets, int32_t* row_scatter, int32_t* slot_expert,
-                                 int32_t* slot_count, int n_slots, int num_sms, int32_t* status, cudaStream_t st) {
+                                 int32_t* counts, int32_t* offsets, int32_t* row_scatter, int32_t* expert_rows,
+                                 int32_t* slot_expert, int32_t* slot_count, int n_slots, int num_sms,
+                                 int32_t* status, cudaStream_t st) {
   cudaError_t e = cudaMemsetAsync(counts, 0, sizeof(int32_t) * (size_t)E, st);
   if (e != cudaSuccess) return e;
   e = cudaMemsetAsync(row_scatter, 0xFF, sizeof(int32_t) * (size_t)(T * k), st);  // -1: unrouted
@@ -231,8 +233,8 @@ cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, in
   if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
   if (blocks < 1) blocks = 1;
   count_kernel<<<(unsigned)blocks, 256, 0, st>>>(ids, n, E, counts, status);
-  offsets_kernel<<<1, 1024, 0, st>>>(counts, E, pad, rows_capacity, offsets, slot_expert, slot_count, n_slots,
-                                     status);
+  offsets_kernel<<<1, 1024, 0, st>>>(counts, E, pad, rows_capacity, offsets, expert_rows, slot_expert, slot_count,
+                                     n_slots, status);
   rank_kernel<<<(unsigned)E, 256, 0, st>>>(ids, T, k, offsets, E, row_scatter);
   return cudaGetLastError();
 }

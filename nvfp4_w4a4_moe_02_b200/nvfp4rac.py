@@ -69,14 +69,14 @@ def load() -> ctypes.CDLL:
         "pack_weights_workspace_size": ([i64, i64, i64], sz),
         "pack_weights": ([vp, i64, i64, i64, vp, i32, i32, tp, tp, vp, sz, vp, vp], ctypes.c_int),
         "w4a4_rac_gemm": ([tp, tp, tp, tp, i64, i64, i64, i32, ctypes.c_int, vp, i64, vp, vp], ctypes.c_int),
-        "grouped_w4a4_rac_moe": ([tp, tp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, i64, vp,
-                                  vp, vp], ctypes.c_int),
+        "grouped_w4a4_rac_moe": ([tp, tp, vp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, i64,
+                                  vp, vp, vp], ctypes.c_int),
         "grouped_w4a4_rac_moe_decode": ([tp, tp, vp, vp, i32, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int,
                                          vp, i64, vp, vp, vp], ctypes.c_int),
         "moe_route_topk": ([vp, i64, i32, i32, vp, vp, vp, vp], ctypes.c_int),
         "moe_rows_capacity": ([i64, i32, i32, i32], i64),
         "moe_dispatch_workspace_size": ([i32], sz),
-        "moe_dispatch_plan": ([vp, i64, i32, i32, i32, i64, vp, vp, vp, vp, i32, vp, sz, vp, vp], ctypes.c_int),
+        "moe_dispatch_plan": ([vp, i64, i32, i32, i32, i64, vp, vp, vp, vp, vp, i32, vp, sz, vp, vp], ctypes.c_int),
         "moe_combine": ([vp, i64, i64, vp, vp, i64, i32, i64, vp, i64, vp, vp], ctypes.c_int),
         "weight_qdq_workspace_size": ([i64, i64], sz),
         "weight_qdq": ([vp, i64, i64, vp, vp, vp, sz, vp, vp], ctypes.c_int),
@@ -330,8 +330,11 @@ def w4a4_rac_gemm(a: Packed, a_res: Packed | None, w: Packed, w_sel: Packed | No
 def grouped_w4a4_rac_moe(a: Packed, a_res: Packed | None, expert_offsets: torch.Tensor, w: Packed,
                          w_sel: Packed | None, swiglu: bool = False, out_dtype=torch.bfloat16,
                          y: torch.Tensor | None = None, amax_out: torch.Tensor | None = None,
-                         status: torch.Tensor | None = None, stream=None):
-    """Grouped GEMM over expert segments -> y (rows a.rows_padded) [and amax of the SwiGLU output]."""
+                         status: torch.Tensor | None = None, stream=None, expert_rows: torch.Tensor | None = None):
+    """Grouped GEMM over expert segments -> y (rows a.rows_padded) [and amax of the SwiGLU output].
+
+    expert_rows (optional device int32 [E]): token rows per segment; 32-row output boxes of padding
+    only are then left unwritten."""
     lib = load()
     E = w.slabs
     N, K = w.rows, w.cols
@@ -347,7 +350,7 @@ def grouped_w4a4_rac_moe(a: Packed, a_res: Packed | None, expert_offsets: torch.
     car = a_res.c() if Kp > 0 else None
     cws = w_sel.c() if Kp > 0 else None
     _check(lib.grouped_w4a4_rac_moe(ctypes.byref(ca), ctypes.byref(car) if car else None, expert_offsets.data_ptr(),
-                                    E, ctypes.byref(cw), ctypes.byref(cws) if cws else None, N, K, Kp,
+                                    _ptr(expert_rows), E, ctypes.byref(cw), ctypes.byref(cws) if cws else None, N, K, Kp,
                                     EPI_SWIGLU_AMAX if swiglu else EPI_NONE, od, y.data_ptr(), y.stride(0),
                                     _ptr(amax_out), st.data_ptr(), _stream(stream)))
     return (y, amax_out) if swiglu else y
@@ -406,7 +409,8 @@ def moe_rows_capacity(T: int, k: int, E: int, pad: int) -> int:
 def moe_dispatch_plan(ids: torch.Tensor, E: int, pad: int, rows_capacity: int | None = None,
                       n_slots: int | None = None, offsets: torch.Tensor | None = None,
                       row_scatter: torch.Tensor | None = None, slot_expert: torch.Tensor | None = None,
-                      slot_count: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None):
+                      slot_count: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None,
+                      expert_rows: torch.Tensor | None = None):
     """Expert-grouped layout of the pairs of ids [T, k] -> (offsets [E+1], row_scatter [T, k], slot_expert,
     slot_count); the slot tables (pad 16) only when n_slots is given."""
     lib = load()
@@ -422,7 +426,7 @@ def moe_dispatch_plan(ids: torch.Tensor, E: int, pad: int, rows_capacity: int | 
     ws = _workspace(dev).get(lib.moe_dispatch_workspace_size(E))
     st = status if status is not None else new_status(dev)
     _check(lib.moe_dispatch_plan(ids.data_ptr(), T, k, E, pad, cap, offsets.data_ptr(), row_scatter.data_ptr(),
-                                 _ptr(slot_expert), _ptr(slot_count), 0 if n_slots is None else n_slots,
+                                 _ptr(expert_rows), _ptr(slot_expert), _ptr(slot_count), 0 if n_slots is None else n_slots,
                                  ws.data_ptr(), ws.numel(), st.data_ptr(), _stream(stream)))
     return offsets, row_scatter, slot_expert, slot_count
 

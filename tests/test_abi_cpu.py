@@ -77,8 +77,8 @@ def test_host_side_rejections(lib):
     st = lib.w4a4_rac_gemm(ctypes.byref(a), None, ctypes.byref(w), None, 64, 96, 128, 0, 0, 16, 96, None, None)
     assert st == 2
     # grouped: SwiGLU needs bf16 output
-    st = lib.grouped_w4a4_rac_moe(ctypes.byref(a), None, 16, 1, ctypes.byref(w), None, 128, 128, 0, 1, 0, 16, 64,
-                                  16, None, None)
+    st = lib.grouped_w4a4_rac_moe(ctypes.byref(a), None, 16, None, 1, ctypes.byref(w), None, 128, 128, 0, 1, 0, 16,
+                                  64, 16, None, None)
     assert st == 1
     # weight_qdq: elems not a multiple of 16
     st = lib.weight_qdq(16, 1, 100, 16, None, 16, 1 << 20, None, None)

@@ -463,6 +463,38 @@ def test_moe_small_ragged(dev, orc):
     check_moe(orc, wl, sel_gu, sel_dn, out, list(range(wl.pair_token.size)))
 
 
+def test_grouped_expert_rows_skips_padding_boxes(dev, orc):
+    """With per-expert token counts, output boxes of padding only keep their old contents, every
+    token row is bit-identical to the call without counts, and the SwiGLU amax is unchanged."""
+    wl = syn.moe_block(T=300, H=512, E=6, topk=2, I=128, T_cal=64)
+    sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
+    st = R.new_status(dev)
+    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    seld = torch.from_numpy(sel_gu).to(dev)
+    a, ar = R.nvfp4_quantize(to_dev(wl.x, dev), seld, row_gather=torch.from_numpy(g).to(dev), M_out=g.size, status=st)
+    w, ws = R.pack_weights(to_dev(wl.wgu, dev), seld, gate_up_interleave=True, status=st)
+    offd = torch.from_numpy(off.astype(np.int32)).to(dev)
+    rows = torch.from_numpy(np.asarray(wl.counts, dtype=np.int32)).to(dev)
+    for swiglu in (False, True):
+        ycols = wl.I if swiglu else 2 * wl.I
+        y_ref = torch.full((a.rows_padded, ycols), 7.0, dtype=torch.bfloat16, device=dev)
+        y_new = y_ref.clone()
+        out_ref = R.grouped_w4a4_rac_moe(a, ar, offd, w, ws, swiglu=swiglu, y=y_ref, status=st)
+        out_new = R.grouped_w4a4_rac_moe(a, ar, offd, w, ws, swiglu=swiglu, y=y_new, status=st, expert_rows=rows)
+        torch.cuda.synchronize()
+        R.check_status(st)
+        tok = torch.from_numpy(pair_rows).to(dev)
+        assert torch.equal(y_new[tok].view(torch.int16), y_ref[tok].view(torch.int16))
+        if swiglu:
+            assert out_new[1].item() == out_ref[1].item()
+        yn = y_new.float().cpu().numpy()
+        for e in range(wl.E):
+            lo, n = int(off[e]), int(wl.counts[e])
+            live_end = lo + (n + 31) // 32 * 32 if n else lo  # boxes that hold a token row
+            assert np.all(yn[live_end:int(off[e + 1])] == 7.0), e      # padding boxes untouched
+            assert np.all(yn[lo + n:live_end] == 0.0), e               # padding rows of live boxes
+
+
 def test_moe_prefill_full_sampled(dev, orc):
     wl = syn.moe_prefill()
     sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
