@@ -63,6 +63,7 @@ def _get():
         "orc_e4m3_encode_array": ([vp, i64, vp], None),
         "orc_f64_to_bf16_array": ([vp, i64, vp], None),
         "orc_num_threads": ([], ctypes.c_int),
+        "orc_act_quant_masked": ([vp, i64, i64, i64, f32, vp, i32, vp, vp, vp, vp], None),
         "orc_route_topk": ([vp, i64, i32, i32, vp, vp], None),
         "orc_dispatch_plan": ([vp, i64, i32, i32, i32, vp, vp], None),
         "orc_combine": ([vp, i64, vp, vp, i64, i32, i64, vp], None),
@@ -170,6 +171,30 @@ def act_quant_rac(x: np.ndarray, s_g: float, sel: np.ndarray):
     _get().orc_act_quant_rac(_p(x), rows, K, K, np.float32(s_g), _p(sel), Kp, _p(codes), _p(S), _p(rcodes),
                              _p(rS), _p(resid))
     return codes, S, rcodes, rS, resid
+
+
+def act_quant_masked(x: np.ndarray, s_g: float, sel: np.ndarray):
+    """RAC variant with the residual kept at its channels (zero off sel) and quantised along K:
+    bf16 x [rows, K] -> (codes [rows,K], S [rows,K/16], mcodes [rows,K], mS [rows,K/16])."""
+    x = _c(x, np.uint16)
+    rows, K = x.shape
+    sel = _c(sel, np.int32)
+    codes = np.empty((rows, K), np.uint8)
+    S = np.empty((rows, K // 16), np.uint8)
+    mcodes = np.empty((rows, K), np.uint8)
+    mS = np.empty((rows, K // 16), np.uint8)
+    _get().orc_act_quant_masked(_p(x), rows, K, K, np.float32(s_g), _p(sel), sel.size, _p(codes), _p(S),
+                                _p(mcodes), _p(mS))
+    return codes, S, mcodes, mS
+
+
+def masked_rac_forward(x: np.ndarray, w: np.ndarray, sel: np.ndarray):
+    """Y = s_x s_w (Q(X) Q(W)^T + Q(M) Q(W)^T) for the masked full-K variant -> (y float64, absdot)."""
+    s_x = global_scale(amax_bf16(x))
+    s_w = global_scale(amax_bf16(w))
+    codes, S, mcodes, mS = act_quant_masked(x, s_x, sel)
+    wc, wS, _, _ = weight_pack(w, s_w, np.zeros(0, np.int32))
+    return gemm_rac(codes, S, mcodes, mS, wc, wS, wc, wS, s_x, s_w)
 
 
 def weight_pack(w: np.ndarray, s_gw: float, sel: np.ndarray):

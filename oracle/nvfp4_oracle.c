@@ -238,6 +238,37 @@ void orc_act_quant_rac(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, 
 }
 
 /* ------------------------------------------------------------------------------------------ */
+/* RAC variant "masked full-K residual" (the selection is the same as above; only the layout   */
+/* of the residual pass differs, so it is a flag of its own, not the method's default):         */
+/*   m = RN(x - DQ(Q(X))) on the channels in sel and 0 on the others, kept at its channel (no   */
+/*   compaction) and quantised with the same s_g in blocks of 16 along K.  The residual pass of  */
+/*   the GEMM then multiplies Q(M) by the main packed weight Q(W): no W_sel is stored.           */
+/* x: bf16 [rows x K] (leading dimension ldx); mcodes [rows x K], mS [rows x K/16].             */
+/* ------------------------------------------------------------------------------------------ */
+void orc_act_quant_masked(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, float s_g, const int32_t* sel,
+                          int32_t Kp, uint8_t* codes, uint8_t* S, uint8_t* mcodes, uint8_t* mS) {
+#pragma omp parallel
+  {
+    float* t = (float*)malloc(sizeof(float) * (size_t)K);
+    float* dq = (float*)malloc(sizeof(float) * (size_t)K);
+    float* m = (float*)malloc(sizeof(float) * (size_t)K);
+#pragma omp for schedule(static)
+    for (int64_t r = 0; r < rows; ++r) {
+      for (int64_t k = 0; k < K; ++k) t[k] = orc_bf16_to_f32(x[r * ldx + k]);
+      for (int64_t b = 0; b < K / 16; ++b)
+        quant_block16(t + b * 16, s_g, codes + r * K + b * 16, S + r * (K / 16) + b, dq + b * 16);
+      for (int64_t k = 0; k < K; ++k) m[k] = 0.0f;
+      for (int32_t j = 0; j < Kp; ++j) m[sel[j]] = t[sel[j]] - dq[sel[j]];
+      for (int64_t b = 0; b < K / 16; ++b)
+        quant_block16(m + b * 16, s_g, mcodes + r * K + b * 16, mS + r * (K / 16) + b, NULL);
+    }
+    free(t);
+    free(dq);
+    free(m);
+  }
+}
+
+/* ------------------------------------------------------------------------------------------ */
 /* weight side of the shared QDQ path [ABS]: Q(W) with its own s_gw, and W_sel = W[:, sel]    */
 /* (raw bf16 columns, ascending) quantised with the same s_gw.                                */
 /* ------------------------------------------------------------------------------------------ */

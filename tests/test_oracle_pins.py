@@ -490,3 +490,63 @@ def test_combine_reduces_to_gather_and_is_linear(orc):
     a, b, c = orc.combine(y, row, w1), orc.combine(y, row, w2), orc.combine(y, row, w1 + w2)
     ref = np.einsum("tj,tjh->th", (w1 + w2).astype(np.float64), syn.bf16_to_f32(y[row]).astype(np.float64))
     assert np.allclose(c, a + b, rtol=1e-12, atol=1e-12) and np.allclose(c, ref, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------------------------------ RAC variant
+def test_masked_residual_empty_selection_is_plain_w4a4(orc):
+    """Masked full-K variant: no selected channel -> zero residual codes and the plain W4A4 GEMM."""
+    wl = syn.dense_tiny()
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    c, S, mc, mS = orc.act_quant_masked(wl.x, s_x, np.zeros(0, np.int32))
+    assert not mc.any() and not mS.any()
+    y, _ = orc.masked_rac_forward(wl.x, wl.w, np.zeros(0, np.int32))
+    y0 = orc.dense_rac_forward(wl.x, wl.w, np.zeros(0, np.int32))["y"]
+    assert np.array_equal(y, y0)
+
+
+def test_masked_residual_matches_compact_on_aligned_and_full_selections(orc):
+    """When the selection is whole aligned 16-blocks, every masked residual block is the compact
+    residual block of the same channels (same 16 values, same order); when it is every channel
+    the two layouts coincide.  Off the selection the masked residual is exactly zero."""
+    wl = syn.dense_tiny()
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    K = wl.x.shape[1]
+    sel = np.concatenate([np.arange(32, 64), np.arange(160, 176)]).astype(np.int32)
+    c, S, mc, mS = orc.act_quant_masked(wl.x, s_x, sel)
+    c2, S2, rc, rS, _ = orc.act_quant_rac(wl.x, s_x, sel)
+    assert np.array_equal(c, c2) and np.array_equal(S, S2)  # the main pass is unchanged
+    assert np.array_equal(mc[:, 32:64], rc[:, 0:32]) and np.array_equal(mS[:, 2:4], rS[:, 0:2])
+    assert np.array_equal(mc[:, 160:176], rc[:, 32:48]) and np.array_equal(mS[:, 10], rS[:, 2])
+    off = np.ones(K, bool)
+    off[sel] = False
+    assert not mc[:, off].any()
+    full = np.arange(K, dtype=np.int32)
+    _, _, mcf, mSf = orc.act_quant_masked(wl.x, s_x, full)
+    _, _, rcf, rSf, _ = orc.act_quant_rac(wl.x, s_x, full)
+    assert np.array_equal(mcf, rcf) and np.array_equal(mSf, rSf)
+
+
+def test_masked_gemm_matches_dequantized_float_matmul(orc):
+    """Y = DQ(Q(X)) DQ(Q(W))^T + DQ(Q(M)) DQ(Q(W))^T with the masked residual (float64 reference)."""
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    s_w = orc.global_scale(orc.amax_bf16(wl.w))
+    c, S, mc, mS = orc.act_quant_masked(wl.x, s_x, sel)
+    wc, wS, _, _ = orc.weight_pack(wl.w, s_w, np.zeros(0, np.int32))
+    ref = (orc.dequant(c, S, s_x) + orc.dequant(mc, mS, s_x)) @ orc.dequant(wc, wS, s_w).T
+    y, ad = orc.masked_rac_forward(wl.x, wl.w, sel)
+    assert np.abs(y - ref).max() <= 1e-12 * ad.max()
+
+
+def test_masked_residual_reduces_error_on_calibration_data(orc):
+    """Like the compact residual, the masked residual lowers the mean error against the exact
+    bf16 product on the calibration batch."""
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    xf = syn.bf16_to_f32(wl.x_cal).astype(np.float64)
+    wf = syn.bf16_to_f32(wl.w).astype(np.float64)
+    exact = xf @ wf.T
+    y_plain = orc.dense_rac_forward(wl.x_cal, wl.w, np.zeros(0, np.int32))["y"]
+    y_mask, _ = orc.masked_rac_forward(wl.x_cal, wl.w, sel)
+    assert np.mean(np.abs(y_mask - exact)) < np.mean(np.abs(y_plain - exact))
