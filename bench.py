@@ -98,19 +98,26 @@ def quant_bytes(rows, K, Kp):
 class MoEStep:
     """Device-resident state of one replica and the step itself (C-ABI calls only)."""
 
-    def __init__(self, wl, h_cal, dev):
+    def __init__(self, wl, h_cal, dev, masked=False):
         import torch
 
         from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
 
-        self.R, self.torch, self.dev, self.wl = R, torch, dev, wl
+        self.R, self.torch, self.dev, self.wl, self.masked = R, torch, dev, wl, masked
         to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
         self.status = R.new_status(dev)
         # offline: channel selection on the calibration batches, weight pack
         self.sel_gu, _ = R.rac_calibrate(to(wl.x_cal), wl.Kp_gu, status=self.status)
         self.sel_dn, _ = R.rac_calibrate(to(h_cal), wl.Kp_dn, status=self.status)
-        self.pgu, self.pgus = R.pack_weights(to(wl.wgu), self.sel_gu, gate_up_interleave=True, status=self.status)
-        self.pdn, self.pdns = R.pack_weights(to(wl.wdn), self.sel_dn, status=self.status)
+        if masked:
+            # masked full-K residual variant: the residual pass reuses the main packed weights
+            self.pgu, _ = R.pack_weights(to(wl.wgu), None, gate_up_interleave=True, status=self.status)
+            self.pdn, _ = R.pack_weights(to(wl.wdn), None, status=self.status)
+            self.pgus, self.pdns = self.pgu, self.pdn
+        else:
+            self.pgu, self.pgus = R.pack_weights(to(wl.wgu), self.sel_gu, gate_up_interleave=True,
+                                                 status=self.status)
+            self.pdn, self.pdns = R.pack_weights(to(wl.wdn), self.sel_dn, status=self.status)
         g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
         self.pair_rows = pair_rows
         self.rows_padded = int(off[-1])
@@ -123,11 +130,12 @@ class MoEStep:
         P = R.Packed
         # padding rows of the expert-sorted activations are never written: zero them once
         self.a = P.empty(self.rows_padded, wl.H, rows_padded=self.rows_padded, device=dev, zero=True)
-        self.ar = P.empty(self.rows_padded, wl.Kp_gu, rows_padded=self.rows_padded, device=dev, zero=True)
+        self.ar = P.empty(self.rows_padded, wl.H if masked else wl.Kp_gu, rows_padded=self.rows_padded, device=dev,
+                          zero=True)
         self.h = torch.empty(self.rows_padded, wl.I, dtype=torch.bfloat16, device=dev)
         self.amax_h = torch.zeros(1, dtype=torch.float32, device=dev)
         self.hq = P.empty(self.rows_padded, wl.I, device=dev)
-        self.hqr = P.empty(self.rows_padded, wl.Kp_dn, rows_padded=self.hq.rows_padded, device=dev)
+        self.hqr = P.empty(self.rows_padded, wl.I if masked else wl.Kp_dn, rows_padded=self.hq.rows_padded, device=dev)
         self.y = torch.empty(self.rows_padded, wl.H, dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize()
         R.check_status(self.status)
@@ -765,6 +773,32 @@ def run_sweep(args):
                      "h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym})
         del step
         torch.cuda.empty_cache()
+    # the masked full-K residual variant at r = 0.5 (residual over all K, main weights reused)
+    wl = dataclasses.replace(base, r=0.5, Kp_gu=syn.kp_from_ratio(base.H, 0.5), Kp_dn=syn.kp_from_ratio(base.I, 0.5))
+    step = MoEStep(wl, h_cal, dev, masked=True)
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step.run()
+    evs = [{n: torch.cuda.Event(enable_timing=True) for n in ("q0", "end")} for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        step.run(events=evs[i])
+    torch.cuda.synchronize()
+    R.check_status(step.status)
+    ms = float(np.mean([e["q0"].elapsed_time(e["end"]) for e in evs]))
+    f_full = sum(flops_of(wl, wl.H, wl.I))  # both residual loops run over all K
+    prow = torch.from_numpy(step.pair_rows[sample]).to(dev)
+    h_g = step.h[prow].double().cpu().numpy()
+    y_g = step.y[prow].double().cpu().numpy()
+    err = lambda a, b: (float(np.linalg.norm(a - b) / np.linalg.norm(b)), float(np.mean(np.abs(a - b))))
+    (hf, hm), (yf, ym) = err(h_g, h_ref), err(y_g, y_ref)
+    masked_row = {"variant": "masked_full_k_residual", "r": 0.5, "ms_per_step": ms,
+                  "tflops": f_full / (ms * 1e-3) / 1e12,
+                  "tflops_plain_w4a4_equivalent": sum(flops_of(wl, 0, 0)) / (ms * 1e-3) / 1e12,
+                  "h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym,
+                  "weight_bytes_per_elem": 0.5625}
+    del step
+    torch.cuda.empty_cache()
     mono = all(rows[i + 1]["y_mean_abs"] <= rows[i]["y_mean_abs"] for i in range(len(rows) - 1))
     at = {x["r"]: x for x in rows}
     line = {"metric": METRIC, "value": at[0.5]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
@@ -776,7 +810,7 @@ def run_sweep(args):
                        "error_reference": "binary64 product of the bf16 inputs (gate_up, silu(g)*u, down) on 256 "
                                           "sampled (token, expert) rows",
                        "l2": "flushed between timed steps (256 MiB write outside the per-step events)"},
-            "sweep": rows, "y_error_non_increasing_in_r": mono, "e2e": None,
+            "sweep": rows, "masked_variant": masked_row, "y_error_non_increasing_in_r": mono, "e2e": None,
             "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * len(rows)}
     print(json.dumps(line), flush=True)
     return 0

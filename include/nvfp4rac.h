@@ -135,8 +135,11 @@ void nvfp4_set_gemm_tile_n(int32_t n);
 /*              computes amax over x rows [0, M).                                            */
 /*   q          output: slabs = 1, rows = M_out, rows_padded >= M_out, cols = K; either      */
 /*              scale layout; rows >= M_out are written as zeros; q->s_g receives s_g.       */
-/*   q_res      output (Kp > 0): cols = Kp, same rows and scale layout; its s_g receives the */
-/*              same s_g.                                                                     */
+/*   q_res      output (Kp > 0), same rows and scale layout; its s_g receives the same s_g.  */
+/*              cols = Kp: the method's residual, gathered into ascending channel order.     */
+/*              cols = K (a variant of the method, "masked full-K residual"): the residual   */
+/*              stays at its channel, zero off sel, in 16-blocks along K; the GEMM then      */
+/*              takes the main packed weight as w_sel with Kp = K (no W_sel is stored).      */
 /*   workspace  >= nvfp4_quantize_workspace_size() bytes, 16-byte aligned.                   */
 /* ---------------------------------------------------------------------------------------- */
 size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K);

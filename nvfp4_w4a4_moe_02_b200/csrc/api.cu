@@ -211,7 +211,8 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   if (st != NVFP4_OK) return st;
   if (Kp > 0) {
     if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
-    st = check_tensor(q_res, "q_res", Kp, M_out, 1, kAnyLayout);
+    const int64_t res_cols = (q_res && q_res->cols == K && Kp < K) ? K : Kp;  // K: masked residual
+    st = check_tensor(q_res, "q_res", res_cols, M_out, 1, kAnyLayout);
     if (st != NVFP4_OK) return st;
     if (q_res->rows_padded != q->rows_padded || q_res->sf_layout != q->sf_layout)
       return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res must have q's rows_padded and sf_layout");
@@ -249,6 +250,7 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   a.codes = q->codes;
   a.sf = q->sf;
   a.sf_slab16 = q->sf_layout == NVFP4_SF_SLAB16;
+  a.masked_res = (Kp > 0 && Kp < K && q_res->cols == K) ? 1 : 0;
   a.rcodes = Kp > 0 ? q_res->codes : nullptr;
   a.rsf = Kp > 0 ? q_res->sf : nullptr;
   a.status = dev_status;
@@ -274,7 +276,8 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
   if (st != NVFP4_OK) return st;
   if (Kp > 0) {
     if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
-    st = check_tensor(q_res, "q_res", Kp, 0, 1, kAnyLayout);
+    const int64_t res_cols = (q_res && q_res->cols == K && Kp < K) ? K : Kp;  // K: masked residual
+    st = check_tensor(q_res, "q_res", res_cols, 0, 1, kAnyLayout);
     if (st != NVFP4_OK) return st;
     if (q_res->rows_padded != q->rows_padded || q_res->sf_layout != q->sf_layout)
       return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res must have q's rows_padded and sf_layout");
@@ -313,6 +316,7 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
   a.codes = q->codes;
   a.sf = q->sf;
   a.sf_slab16 = q->sf_layout == NVFP4_SF_SLAB16;
+  a.masked_res = (Kp > 0 && Kp < K && q_res->cols == K) ? 1 : 0;
   a.rcodes = Kp > 0 ? q_res->codes : nullptr;
   a.rsf = Kp > 0 ? q_res->sf : nullptr;
   a.status = dev_status;

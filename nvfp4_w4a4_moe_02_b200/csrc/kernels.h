@@ -38,6 +38,7 @@ struct RowArgs {
   uint8_t* codes;                // [rows_out x K/2]
   uint8_t* sf;                   // atoms, K/64 groups per row
   int sf_slab16;                 // act: scales of codes/rcodes in the 16-row slab layout
+  int masked_res;                // act: residual kept at its channel (zero off sel), K wide
   uint8_t* rcodes;               // [rows_out x Kp/2]
   uint8_t* rsf;                  // atoms, Kp/64 groups per row
   float* resid_all;              // cal: [rows_out x K] residual of every channel
@@ -47,7 +48,7 @@ struct RowArgs {
 cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64_t cols, int64_t ld, float* partial,
                         int P, int32_t* status, cudaStream_t st);
 cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st);
-size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps);
+size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps, bool masked = false);
 cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, double* err, cudaStream_t st);
 cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t* sel, double* err_out, cudaStream_t st);
 cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint16_t* out, const float* partial, int P,

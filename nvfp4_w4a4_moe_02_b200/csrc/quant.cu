@@ -89,6 +89,11 @@ __device__ __forceinline__ float reduce_partials(const float* partial, int P) {
 // re-derives its code and DQ = e*d from a per-warp stash of each block's (d, 1/d).  Keeping only
 // the block scales in shared memory, not the row, leaves room for more warps per SM.
 //
+// Masked residual (activation mode, a variant of the method): the residual stays at its channel,
+// zero off the selection, and is quantised in 16-blocks along K in the main pass itself (each
+// lane knows which of its 16 channels are selected from a CTA-shared bitmap); there is no
+// residual pass, and the GEMM reuses the main packed weights for it.
+//
 // SPLIT (activations with few rows, e.g. the tokens of one decode step): a whole CTA works on
 // one row; warp w takes the 512-element chunks w, w + nwarps, ... of both passes and the stash
 // is shared by the CTA, so a 64-token batch still occupies every warp of 64 CTAs.
@@ -143,14 +148,21 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   const int32_t K = (int32_t)a.K;  // <= 32768: offsets inside a row fit in 32 bits
   const int32_t Kp = a.Kp;
   constexpr bool kHasSel = (MODE == kModeAct || MODE == kModePack);
-  const bool use_sel = kHasSel && Kp > 0;
+  const bool masked = MODE == kModeAct && a.masked_res != 0 && Kp > 0;
+  const bool use_sel = kHasSel && Kp > 0 && !masked;  // compact residual pass
 
-  // CTA-shared channel list (int16), then per warp (per CTA when SPLIT) each block's (d, 1/d)
+  // CTA-shared channel list (int16), then per warp (per CTA when SPLIT) each block's (d, 1/d);
+  // the masked variant keeps a bitmap of the selected channels instead
   int16_t* sel_s = reinterpret_cast<int16_t*>(smem_raw);
+  uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem_raw);
   const size_t sel_bytes = use_sel ? (((size_t)Kp * 2 + 15) / 16) * 16 : 0;
   const size_t warp_bytes = use_sel ? (size_t)(K / 16) * 8 : 0;
   float2* dinv_s = reinterpret_cast<float2*>(smem_raw + sel_bytes + (SPLIT ? 0 : warp) * warp_bytes);
-  if (use_sel) {
+  if (use_sel || masked) {
+    if (masked) {
+      for (int32_t w = threadIdx.x; w < (K + 31) / 32; w += blockDim.x) mask_s[w] = 0u;
+      __syncthreads();
+    }
     for (int32_t j = threadIdx.x; j < Kp; j += blockDim.x) {
       int32_t c = a.sel[j];
       bool ok = (c >= 0 && c < K) && (j == 0 || a.sel[j - 1] < c);
@@ -158,7 +170,8 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
         report_status(a.status, kErrInvalid);
         c = 0;
       }
-      sel_s[j] = (int16_t)c;
+      if (masked) atomicOr(mask_s + (c >> 5), 1u << (c & 31));
+      else sel_s[j] = (int16_t)c;
     }
     __syncthreads();
   }
@@ -246,8 +259,26 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
         }
         continue;
       }
-      const uint2 c = make_uint2(quant8_codes(x, bs), quant8_codes(x + 8, bs));
       const int32_t kb = e >> 4;
+      uint2 c, mc = make_uint2(0u, 0u);
+      uint32_t mS = 0;
+      if (masked) {
+        // residual of the selected channels of this block, zero elsewhere, quantised in place
+        float dq[16], m[16];
+        c = make_uint2(quant8(x, bs, dq), quant8(x + 8, bs, dq + 8));
+        const uint32_t bits = h ? (mask_s[e >> 5] >> (e & 31)) & 0xFFFFu : 0u;
+        float bm = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          m[i] = ((bits >> i) & 1u) ? __fsub_rn(x[i], dq[i]) : 0.0f;
+          bm = fmaxf(bm, fabsf(m[i]));
+        }
+        const BlockScale ms = block_scale(bm, s_g, t6);
+        mc = make_uint2(quant8_codes(m, ms), quant8_codes(m + 8, ms));
+        mS = ms.S;
+      } else {
+        c = make_uint2(quant8_codes(x, bs), quant8_codes(x + 8, bs));
+      }
       if (use_sel && h) dinv_s[kb] = make_float2(bs.d, bs.inv);  // block scales for the residual pass
       const int32_t blk = sf_blk(kb);
       for (int j = 0; j < dst.n; ++j) {
@@ -259,6 +290,10 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
         }
         *reinterpret_cast<uint2*>(a.codes + drow * (K / 2) + e / 2) = c;
         a.sf[sf_row(drow, k64) + blk] = (uint8_t)bs.S;
+        if (masked) {
+          *reinterpret_cast<uint2*>(a.rcodes + drow * (K / 2) + e / 2) = mc;
+          a.rsf[sf_row(drow, k64) + blk] = (uint8_t)mS;
+        }
       }
     }
 
@@ -500,8 +535,9 @@ cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64
   return cudaGetLastError();
 }
 
-size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps) {
+size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps, bool masked) {
   if (Kp <= 0) return 16;
+  if (masked) return (size_t)((K + 31) / 32) * 4;
   return (size_t)((Kp * 2 + 15) / 16) * 16 + (size_t)warps * (size_t)(K / 16) * 8;
 }
 
@@ -511,10 +547,11 @@ cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
   // few activation rows: one CTA of 8 warps per row (SPLIT), so that every warp of the grid
   // has work; otherwise one warp per row with as many warps per CTA as the stashes allow
   const bool split = a.mode == kModeAct && rows * 2 < (int64_t)num_sms * warps;
-  size_t smem = rows_smem_bytes(a.K, a.Kp, split ? 1 : warps);
+  const bool masked = a.mode == kModeAct && a.masked_res != 0;
+  size_t smem = rows_smem_bytes(a.K, a.Kp, split ? 1 : warps, masked);
   while (!split && smem > 200 * 1024 && warps > 1) {
     warps /= 2;
-    smem = rows_smem_bytes(a.K, a.Kp, warps);
+    smem = rows_smem_bytes(a.K, a.Kp, warps, masked);
   }
   if (smem > 200 * 1024) return cudaErrorInvalidValue;
   int64_t ctas_needed = split ? rows : (rows + warps - 1) / warps;

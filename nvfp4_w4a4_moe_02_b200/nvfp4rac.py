@@ -211,8 +211,11 @@ def set_gemm_tile_n(n: int):
 def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather: torch.Tensor | None = None,
                    M_out: int | None = None, rows_padded: int | None = None, amax_in: torch.Tensor | None = None,
                    out: Packed | None = None, out_res: Packed | None = None, status: torch.Tensor | None = None,
-                   stream=None):
-    """Online activation quantisation with the residual pass on ``sel`` -> (Packed, Packed | None)."""
+                   stream=None, masked: bool = False):
+    """Online activation quantisation with the residual pass on ``sel`` -> (Packed, Packed | None).
+
+    masked=True selects the masked full-K residual variant (residual at its channel, zero off
+    ``sel``, K wide): pair it with the main packed weight as w_sel in w4a4_rac_gemm."""
     lib = load()
     _u16(x)
     M, K = x.shape
@@ -224,7 +227,7 @@ def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather:
     if out is None:
         out = Packed.empty(M_out, K, rows_padded=rows_padded, device=x.device)
     if Kp > 0 and out_res is None:
-        out_res = Packed.empty(M_out, Kp, rows_padded=out.rows_padded, device=x.device)
+        out_res = Packed.empty(M_out, K if masked else Kp, rows_padded=out.rows_padded, device=x.device)
     ws_bytes = lib.nvfp4_quantize_workspace_size(M, K)
     ws = _workspace(x.device).get(ws_bytes)
     st = status if status is not None else new_status(x.device)

@@ -463,6 +463,35 @@ def test_moe_small_ragged(dev, orc):
     check_moe(orc, wl, sel_gu, sel_dn, out, list(range(wl.pair_token.size)))
 
 
+@pytest.mark.parametrize("which", ["tiny", "ragged", "aligned_full"])
+def test_masked_residual_variant_matches_oracle(dev, orc, which):
+    """The masked full-K residual variant: codes and scales bit-exact, and the GEMM with the main
+    packed weight as the residual weight within the GEMM tolerance."""
+    if which == "tiny":
+        wl = syn.dense_tiny()
+        x, w = wl.x, wl.w
+        sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    else:
+        x = syn.normal_bf16(2, 1, 300, 1024, 1.0, syn.outlier_colscale(2, 1024))
+        w = syn.normal_bf16(2, 2, 384, 1024, 0.02)
+        sel = np.arange(5, 1024, 3, dtype=np.int32)[:320] if which == "ragged" else np.arange(1024, dtype=np.int32)
+    s_x = orc.global_scale(orc.amax_bf16(x))
+    st = R.new_status(dev)
+    seld = torch.from_numpy(sel).to(dev)
+    q, qm = R.nvfp4_quantize(to_dev(x, dev), seld, masked=True, status=st)
+    wq, _ = R.pack_weights(to_dev(w, dev), status=st)
+    y = R.w4a4_rac_gemm(q, qm, wq, wq, x.shape[0], out_dtype=torch.float32, status=st)
+    torch.cuda.synchronize()
+    R.check_status(st)
+    c, S, mc, mS = orc.act_quant_masked(x, s_x, sel)
+    gc, gS = logical(q)
+    gmc, gmS = logical(qm)
+    assert np.array_equal(gc, c) and np.array_equal(gS, S)
+    assert np.array_equal(gmc, mc) and np.array_equal(gmS, mS), np.argwhere(gmc != mc)[:5]
+    y_ref, ad = orc.masked_rac_forward(x, w, sel)
+    assert_gemm_close(y.cpu().numpy(), y_ref, ad, False)
+
+
 def test_grouped_expert_rows_skips_padding_boxes(dev, orc):
     """With per-expert token counts, output boxes of padding only keep their old contents, every
     token row is bit-identical to the call without counts, and the SwiGLU amax is unchanged."""
