@@ -552,7 +552,7 @@ def spec_moe(dev, args, peaks):
         segments={"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")},
         dominant=("gate_up", gu_f, gu_bytes, "grouped gate_up W4A4+RAC GEMM (SwiGLU epilogue)"),
         # dram__bytes_read.sum + dram__bytes_write.sum of one launch, grouped_gemm_gate_up_moe_prefill.md
-        traffic=(410.365440e6 + 51.551488e6) if args.experts is None else None,
+        traffic=(410.415104e6 + 43.660032e6) if args.experts is None else None,
         quant={"x": ("quant_x", int(wl.x.nbytes) + P * 0.5625 * (wl.H + wl.Kp_gu)),  # X read once, 8 copies out
                "h": ("quant_h", quant_bytes(P, wl.I, wl.Kp_dn))},
         config={"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P, "experts": wl.E,
