@@ -58,6 +58,7 @@ def _get():
         "orc_weight_qdq": ([vp, i64, f32, vp], None),
         "orc_gemm_rac": ([vp, vp, vp, vp, i64, i32, vp, vp, vp, vp, i64, f64, f64, vp, i64, vp, vp], None),
         "orc_calibrate": ([vp, i64, i64, i32, vp, vp], None),
+        "orc_calibrate_grouped": ([vp, i64, i64, vp, i32, i32, vp, vp], None),
         "orc_swiglu": ([vp, i64, i64, vp, vp], None),
         "orc_e2m1_encode_array": ([vp, i64, vp], None),
         "orc_e4m3_encode_array": ([vp, i64, vp], None),
@@ -251,6 +252,49 @@ def calibrate(x_cal: np.ndarray, Kp: int):
     err = np.empty(K, np.float64)
     _get().orc_calibrate(_p(x), T, K, int(Kp), _p(sel), _p(err))
     return sel, err
+
+
+def calibrate_grouped(x_cal: np.ndarray, offsets: np.ndarray, Kp: int):
+    """Per-expert RAC selection: rows [offsets[g], offsets[g+1]) of the calibration batch form
+    group g; the batch is quantised once with its own s_g and each group keeps the Kp channels with
+    the largest error over its own rows -> (sel int32 [G, Kp] ascending per row, err float64 [G, K])."""
+    x = _c(x_cal, np.uint16)
+    T, K = x.shape
+    off = _c(offsets, np.int64)
+    G = off.size - 1
+    assert G >= 1 and off[0] == 0 and off[-1] == T and np.all(np.diff(off) >= 0)
+    sel = np.empty((G, Kp), np.int32)
+    err = np.empty((G, K), np.float64)
+    _get().orc_calibrate_grouped(_p(x), T, K, _p(off), G, int(Kp), _p(sel), _p(err))
+    return sel, err
+
+
+def act_quant_rac_grouped(x: np.ndarray, s_g: float, sel: np.ndarray, row_group: np.ndarray):
+    """act_quant_rac with one channel list per group: row t uses sel[row_group[t]] (all rows share
+    s_g); a row with row_group < 0 gets an all-zero residual (codes 0, scales 0)."""
+    x = _c(x, np.uint16)
+    sel = _c(sel, np.int32)
+    rows, K = x.shape
+    G, Kp = sel.shape
+    rg = np.asarray(row_group, np.int64)
+    codes, S, _, _, _ = act_quant_rac(x, s_g, np.zeros(0, np.int32))
+    rcodes = np.zeros((rows, Kp), np.uint8)
+    rS = np.zeros((rows, Kp // 16), np.uint8)
+    resid = np.zeros((rows, Kp), np.float32)
+    for g in range(G):
+        idx = np.nonzero(rg == g)[0]
+        if idx.size == 0:
+            continue
+        _, _, rc, rs, rr = act_quant_rac(x[idx], s_g, sel[g])
+        rcodes[idx], rS[idx], resid[idx] = rc, rs, rr
+    return codes, S, rcodes, rS, resid
+
+
+def weight_pack_grouped(w: np.ndarray, s_gw: np.ndarray, sel: np.ndarray):
+    """weight_pack of E expert matrices w [E, N, K], expert e with its own s_gw[e] and channel
+    list sel[e] -> (codes [E,N,K], S, sel codes [E,N,Kp], sel S)."""
+    outs = [weight_pack(w[e], float(s_gw[e]), sel[e]) for e in range(w.shape[0])]
+    return tuple(np.stack([o[i] for o in outs]) for i in range(4))
 
 
 def route_topk(logits: np.ndarray, k: int):

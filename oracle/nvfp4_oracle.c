@@ -373,7 +373,8 @@ static int cmp_int_asc(const void* a, const void* b) {
   return (i < j) ? -1 : (i > j) ? 1 : 0;
 }
 
-void orc_calibrate(const uint16_t* x, int64_t T, int64_t K, int32_t Kp, int32_t* sel, double* err_out) {
+/* residuals r = x - DQ(Q(x)) of the calibration batch, quantised with its own s_g (FP32) */
+static float* calib_residuals(const uint16_t* x, int64_t T, int64_t K) {
   float amax = orc_amax_bf16(x, T, K, K);
   float s_g = orc_global_scale(amax);
   float* resid = (float*)malloc(sizeof(float) * (size_t)(T * K));
@@ -394,24 +395,57 @@ void orc_calibrate(const uint16_t* x, int64_t T, int64_t K, int32_t Kp, int32_t*
     free(c);
     free(S);
   }
-  double* err = (double*)malloc(sizeof(double) * (size_t)K);
+  return resid;
+}
+
+/* e_k = sum over rows [r0, r1) of r_{t,k}^2, t ascending, binary64 */
+static void calib_errors(const float* resid, int64_t r0, int64_t r1, int64_t K, double* err) {
 #pragma omp parallel for schedule(static)
   for (int64_t k = 0; k < K; ++k) {
     double e = 0.0;
-    for (int64_t r = 0; r < T; ++r) {
+    for (int64_t r = r0; r < r1; ++r) {
       double v = (double)resid[r * K + k];
       e += v * v;
     }
     err[k] = e;
   }
+}
+
+/* the Kp channels with the largest e_k (ties -> lower k), ascending */
+static void calib_select(const double* err, int64_t K, int32_t Kp, int32_t* sel) {
   int32_t* idx = (int32_t*)malloc(sizeof(int32_t) * (size_t)K);
   for (int32_t k = 0; k < K; ++k) idx[k] = k;
   g_sort_err = err;
   qsort(idx, (size_t)K, sizeof(int32_t), cmp_err_desc);
   for (int32_t j = 0; j < Kp; ++j) sel[j] = idx[j];
   qsort(sel, (size_t)Kp, sizeof(int32_t), cmp_int_asc);
-  if (err_out) memcpy(err_out, err, sizeof(double) * (size_t)K);
   free(idx);
+}
+
+void orc_calibrate(const uint16_t* x, int64_t T, int64_t K, int32_t Kp, int32_t* sel, double* err_out) {
+  float* resid = calib_residuals(x, T, K);
+  double* err = (double*)malloc(sizeof(double) * (size_t)K);
+  calib_errors(resid, 0, T, K, err);
+  calib_select(err, K, Kp, sel);
+  if (err_out) memcpy(err_out, err, sizeof(double) * (size_t)K);
+  free(err);
+  free(resid);
+}
+
+/* Per-expert selection (a variant the pages leave open: one channel list per expert of the    */
+/* down projection).  Reading: the pooled calibration batch (rows grouped by expert, group g =  */
+/* rows [off[g], off[g+1])) is quantised once with its own s_g, as for the shared list; e_k of  */
+/* group g sums only that group's rows, t ascending; each group keeps its own Kp channels.      */
+/* sel: [G x Kp]; err_out (nullable): [G x K].                                                  */
+void orc_calibrate_grouped(const uint16_t* x, int64_t T, int64_t K, const int64_t* off, int32_t G, int32_t Kp,
+                           int32_t* sel, double* err_out) {
+  float* resid = calib_residuals(x, T, K);
+  double* err = (double*)malloc(sizeof(double) * (size_t)K);
+  for (int32_t g = 0; g < G; ++g) {
+    calib_errors(resid, off[g], off[g + 1], K, err);
+    calib_select(err, K, Kp, sel + (int64_t)g * Kp);
+    if (err_out) memcpy(err_out + (int64_t)g * K, err, sizeof(double) * (size_t)K);
+  }
   free(err);
   free(resid);
 }

@@ -550,3 +550,125 @@ def test_masked_residual_reduces_error_on_calibration_data(orc):
     y_plain = orc.dense_rac_forward(wl.x_cal, wl.w, np.zeros(0, np.int32))["y"]
     y_mask, _ = orc.masked_rac_forward(wl.x_cal, wl.w, sel)
     assert np.mean(np.abs(y_mask - exact)) < np.mean(np.abs(y_plain - exact))
+
+
+# ---- per-expert channel lists (a RAC variant the pages leave open: one list per expert) ----
+
+def _grouped_batch(seed=11, T=30, K=128, offsets=(0, 7, 7, 19, 30)):
+    rng = np.random.default_rng(seed)
+    x = syn.normal_bf16(seed, 3, T, K, 1.0, np.exp(rng.standard_normal(K)))
+    return x, np.array(offsets, np.int64)
+
+
+def test_grouped_selection_single_group_equals_shared(orc):
+    x, _ = _grouped_batch()
+    sel, err = orc.calibrate(x, 64)
+    sg, eg = orc.calibrate_grouped(x, np.array([0, x.shape[0]]), 64)
+    assert np.array_equal(sg[0], sel) and np.array_equal(eg[0], err)
+
+
+def test_grouped_selection_matches_sequential_python(orc):
+    """e_k of group g sums only rows [off[g], off[g+1]) of the residual of the pooled batch
+    (quantised once with the batch's own s_g), t ascending; ties go to the lower channel."""
+    x, off = _grouped_batch()
+    x[:, 9] = x[:, 10]  # equal errors in every group: the tie goes to channel 9
+    Kp = 32
+    sel, err = orc.calibrate_grouped(x, off, Kp)
+    s_g = orc.global_scale(orc.amax_bf16(x))
+    _, _, dq = orc.quantize_f32(syn.bf16_to_f32(x), s_g)
+    r = (syn.bf16_to_f32(x) - dq).astype(np.float32)
+    K = x.shape[1]
+    for g in range(off.size - 1):
+        e = []
+        for k in range(K):
+            acc = 0.0
+            for t in range(int(off[g]), int(off[g + 1])):
+                acc += float(r[t, k]) * float(r[t, k])
+            e.append(acc)
+        assert np.array_equal(np.array(e), err[g]), g
+        order = sorted(range(K), key=lambda k: (-e[k], k))
+        assert sel[g].tolist() == sorted(order[:Kp]), g
+
+
+def test_grouped_selection_empty_group_takes_lowest_channels(orc):
+    x, off = _grouped_batch()  # group 1 is empty
+    sel, err = orc.calibrate_grouped(x, off, 32)
+    assert np.all(err[1] == 0.0) and sel[1].tolist() == list(range(32))
+
+
+def test_grouped_selection_follows_each_groups_outliers(orc):
+    """Channels scaled x20 in one group's rows only: a x20 channel sets its 16-block's scale, so
+    the largest residuals sit in that block (its other channels are flushed towards zero).  Each
+    group's list lies inside its own hot blocks and avoids the other group's."""
+    T, K = 40, 128
+    x = syn.normal_bf16(5, 3, T, K, 1.0)
+    xf = syn.bf16_to_f32(x).astype(np.float64)
+    hot = {0: [3, 70], 1: [40, 101]}
+    off = np.array([0, 20, 40])
+    for g, chans in hot.items():
+        for c in chans:
+            xf[off[g]:off[g + 1], c] *= 20.0
+    x = orc.f64_to_bf16_array(xf)
+    sel, _ = orc.calibrate_grouped(x, off, 16)
+    for g, chans in hot.items():
+        own = {c // 16 for c in chans}
+        other = {c // 16 for c in hot[1 - g]}
+        blocks = {int(c) // 16 for c in sel[g]}
+        assert blocks <= own and not (blocks & other), (g, sel[g])
+
+
+def test_grouped_selection_drops_no_more_residual_energy_than_shared(orc):
+    """For every group, the residual energy left outside its own list is at most what the shared
+    list leaves outside (the group's list takes the group's Kp largest e_k)."""
+    wl = syn.dense_tiny()
+    x = wl.x_cal
+    off = np.array([0, 16, 40, x.shape[0]])
+    Kp = wl.Kp
+    sel_g, err_g = orc.calibrate_grouped(x, off, Kp)
+    sel_s, _ = orc.calibrate(x, Kp)
+    for g in range(off.size - 1):
+        mask_g = np.ones(x.shape[1], bool)
+        mask_g[sel_g[g]] = False
+        mask_s = np.ones(x.shape[1], bool)
+        mask_s[sel_s] = False
+        assert err_g[g][mask_g].sum() <= err_g[g][mask_s].sum()
+
+
+def test_grouped_residual_rows_follow_their_group(orc):
+    x, _ = _grouped_batch(T=12, K=128)
+    s_g = orc.global_scale(orc.amax_bf16(x))
+    rng = np.random.default_rng(3)
+    sel = np.stack([np.sort(rng.choice(128, 64, replace=False)) for _ in range(3)]).astype(np.int32)
+    rg = np.array([2, 0, -1, 1, 1, 0, 2, -1, 0, 0, 1, 2])
+    codes, S, rc, rS, rr = orc.act_quant_rac_grouped(x, s_g, sel, rg)
+    c0, S0, _, _, _ = orc.act_quant_rac(x, s_g, sel[0])
+    assert np.array_equal(codes, c0) and np.array_equal(S, S0)  # the main pass ignores the lists
+    xf = syn.bf16_to_f32(x)
+    _, _, dq = orc.quantize_f32(xf, s_g)
+    for t in range(x.shape[0]):
+        if rg[t] < 0:
+            assert not rc[t].any() and not rS[t].any() and not rr[t].any()
+            continue
+        r = (xf[t] - dq[t]).astype(np.float32)[sel[rg[t]]]
+        assert np.array_equal(rr[t], r), t
+        c2, S2, _ = orc.quantize_f32(r[None, :], s_g)
+        assert np.array_equal(rc[t], c2[0]) and np.array_equal(rS[t], S2[0]), t
+    # one list for every group reduces to the shared residual
+    same = np.stack([sel[1]] * 3)
+    _, _, rc1, rS1, _ = orc.act_quant_rac_grouped(x, s_g, same, np.abs(rg))
+    _, _, rc2, rS2, _ = orc.act_quant_rac(x, s_g, sel[1])
+    assert np.array_equal(rc1, rc2) and np.array_equal(rS1, rS2)
+
+
+def test_grouped_weight_sel_is_each_experts_raw_columns(orc):
+    E, N, K = 3, 32, 128
+    w = np.stack([syn.normal_bf16(e, 2, N, K, 0.02) for e in range(E)])
+    s_w = np.array([orc.global_scale(orc.amax_bf16(w[e])) for e in range(E)], np.float32)
+    rng = np.random.default_rng(8)
+    sel = np.stack([np.sort(rng.choice(K, 64, replace=False)) for _ in range(E)]).astype(np.int32)
+    codes, S, sc, sS = orc.weight_pack_grouped(w, s_w, sel)
+    for e in range(E):
+        c2, S2, _ = orc.quantize_f32(syn.bf16_to_f32(w[e])[:, sel[e]], s_w[e])
+        assert np.array_equal(sc[e], c2) and np.array_equal(sS[e], S2)
+        c3, S3, _ = orc.quantize_f32(syn.bf16_to_f32(w[e]), s_w[e])
+        assert np.array_equal(codes[e], c3) and np.array_equal(S[e], S3)
