@@ -98,7 +98,9 @@ def quant_bytes(rows, K, Kp):
 class MoEStep:
     """Device-resident state of one replica and the step itself (C-ABI calls only)."""
 
-    def __init__(self, wl, h_cal, dev, masked=False):
+    def __init__(self, wl, h_cal, dev, masked=False, h_cal_offsets=None):
+        """h_cal_offsets (int64 [E + 1], rows of h_cal per expert) selects the per-expert variant:
+        one down-projection channel list per expert, calibrated on that expert's rows."""
         import torch
 
         from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
@@ -108,7 +110,11 @@ class MoEStep:
         self.status = R.new_status(dev)
         # offline: channel selection on the calibration batches, weight pack
         self.sel_gu, _ = R.rac_calibrate(to(wl.x_cal), wl.Kp_gu, status=self.status)
-        self.sel_dn, _ = R.rac_calibrate(to(h_cal), wl.Kp_dn, status=self.status)
+        if h_cal_offsets is None:
+            self.sel_dn, _ = R.rac_calibrate(to(h_cal), wl.Kp_dn, status=self.status)
+        else:
+            offd = torch.from_numpy(np.asarray(h_cal_offsets, np.int32)).to(dev)
+            self.sel_dn, _ = R.rac_calibrate_grouped(to(h_cal), offd, wl.Kp_dn, status=self.status)
         if masked:
             # masked full-K residual variant: the residual pass reuses the main packed weights
             self.pgu, _ = R.pack_weights(to(wl.wgu), None, gate_up_interleave=True, status=self.status)
@@ -125,6 +131,9 @@ class MoEStep:
                                                       wl.topk_ids.shape[1])).to(dev)
         self.offsets = torch.from_numpy(off.astype(np.int32)).to(dev)
         self.expert_rows = torch.from_numpy(np.asarray(wl.counts, dtype=np.int32)).to(dev)
+        # per-expert lists: each expert-sorted row of h takes its expert's list (routing is fixed
+        # for the step, like the offsets)
+        self.row_group = R.moe_row_groups(self.offsets, wl.E, self.rows_padded) if h_cal_offsets is not None else None
         self.x = to(wl.x)
         # preallocated outputs (the step allocates nothing)
         P = R.Packed
@@ -155,7 +164,8 @@ class MoEStep:
                                amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status,
+                         row_group=self.row_group)
         if "d0" in ev:
             ev["d0"].record()
         R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.offsets, self.pdn, self.pdns, y=self.y, status=self.status,
@@ -271,7 +281,8 @@ class DecodeStep:
                                       swiglu=True, y=self.h, amax_out=self.amax_h, status=self.status)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status,
+                         row_group=self.row_group)
         if "d0" in ev:
             ev["d0"].record()
         R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.slot_expert, self.slot_count, self.pdn, self.pdns,
@@ -350,7 +361,8 @@ class MoEBlockStep:
                                    amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status,
+                         row_group=self.row_group)
         if "d0" in ev:
             ev["d0"].record()
         if self.decode:
@@ -746,10 +758,10 @@ def run_sweep(args):
         y_ref.append(h @ f64(base.wdn[e]).T)
     h_ref, y_ref = np.array(h_ref), np.array(y_ref)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    rows = []
-    for r in (0.0, 0.25, 0.5, 1.0):
-        wl = dataclasses.replace(base, r=r, Kp_gu=syn.kp_from_ratio(base.H, r), Kp_dn=syn.kp_from_ratio(base.I, r))
-        step = MoEStep(wl, h_cal, dev)
+    err = lambda a, b: (float(np.linalg.norm(a - b) / np.linalg.norm(b)), float(np.mean(np.abs(a - b))))
+
+    def measure(step):
+        """mean step time (ms) and the errors of h and y on the sampled rows"""
         for _ in range(max(3, args.warmup)):
             flush.zero_()
             step.run()
@@ -760,43 +772,41 @@ def run_sweep(args):
         torch.cuda.synchronize()
         R.check_status(step.status)
         ms = float(np.mean([e["q0"].elapsed_time(e["end"]) for e in evs]))
+        prow = torch.from_numpy(step.pair_rows[sample]).to(dev)
+        (hf, hm), (yf, ym) = err(step.h[prow].double().cpu().numpy(), h_ref), err(step.y[prow].double().cpu().numpy(),
+                                                                                  y_ref)
+        return ms, {"h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym}
+
+    rows = []
+    for r in (0.0, 0.25, 0.5, 1.0):
+        wl = dataclasses.replace(base, r=r, Kp_gu=syn.kp_from_ratio(base.H, r), Kp_dn=syn.kp_from_ratio(base.I, r))
+        step = MoEStep(wl, h_cal, dev)
+        ms, e = measure(step)
         gu_f, dn_f = flops_of(wl, wl.Kp_gu, wl.Kp_dn)
         plain_f = sum(flops_of(wl, 0, 0))
-        prow = torch.from_numpy(step.pair_rows[sample]).to(dev)
-        h_g = step.h[prow].double().cpu().numpy()
-        y_g = step.y[prow].double().cpu().numpy()
-        err = lambda a, b: (float(np.linalg.norm(a - b) / np.linalg.norm(b)), float(np.mean(np.abs(a - b))))
-        (hf, hm), (yf, ym) = err(h_g, h_ref), err(y_g, y_ref)
         rows.append({"r": r, "Kp_gate_up": wl.Kp_gu, "Kp_down": wl.Kp_dn, "ms_per_step": ms,
                      "tflops": (gu_f + dn_f) / (ms * 1e-3) / 1e12,
-                     "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12,
-                     "h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym})
+                     "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12, **e})
         del step
         torch.cuda.empty_cache()
-    # the masked full-K residual variant at r = 0.5 (residual over all K, main weights reused)
     wl = dataclasses.replace(base, r=0.5, Kp_gu=syn.kp_from_ratio(base.H, 0.5), Kp_dn=syn.kp_from_ratio(base.I, 0.5))
+    plain_f = sum(flops_of(wl, 0, 0))
+    # the masked full-K residual variant at r = 0.5 (residual over all K, main weights reused)
     step = MoEStep(wl, h_cal, dev, masked=True)
-    for _ in range(max(3, args.warmup)):
-        flush.zero_()
-        step.run()
-    evs = [{n: torch.cuda.Event(enable_timing=True) for n in ("q0", "end")} for _ in range(args.steps)]
-    for i in range(args.steps):
-        flush.zero_()
-        step.run(events=evs[i])
-    torch.cuda.synchronize()
-    R.check_status(step.status)
-    ms = float(np.mean([e["q0"].elapsed_time(e["end"]) for e in evs]))
+    ms, e = measure(step)
     f_full = sum(flops_of(wl, wl.H, wl.I))  # both residual loops run over all K
-    prow = torch.from_numpy(step.pair_rows[sample]).to(dev)
-    h_g = step.h[prow].double().cpu().numpy()
-    y_g = step.y[prow].double().cpu().numpy()
-    err = lambda a, b: (float(np.linalg.norm(a - b) / np.linalg.norm(b)), float(np.mean(np.abs(a - b))))
-    (hf, hm), (yf, ym) = err(h_g, h_ref), err(y_g, y_ref)
     masked_row = {"variant": "masked_full_k_residual", "r": 0.5, "ms_per_step": ms,
-                  "tflops": f_full / (ms * 1e-3) / 1e12,
-                  "tflops_plain_w4a4_equivalent": sum(flops_of(wl, 0, 0)) / (ms * 1e-3) / 1e12,
-                  "h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym,
-                  "weight_bytes_per_elem": 0.5625}
+                  "tflops": f_full / (ms * 1e-3) / 1e12, "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12,
+                  **e, "weight_bytes_per_elem": 0.5625}
+    del step
+    torch.cuda.empty_cache()
+    # per-expert channel lists for the down projection at r = 0.5 (gate_up keeps the shared list:
+    # each token's X residual is quantised once for all its experts)
+    step = MoEStep(wl, h_cal, dev, h_cal_offsets=syn.moe_down_calibration_offsets(base))
+    ms, e = measure(step)
+    per_expert_row = {"variant": "per_expert_down_lists", "r": 0.5, "ms_per_step": ms,
+                      "tflops": sum(flops_of(wl, wl.Kp_gu, wl.Kp_dn)) / (ms * 1e-3) / 1e12,
+                      "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12, **e}
     del step
     torch.cuda.empty_cache()
     mono = all(rows[i + 1]["y_mean_abs"] <= rows[i]["y_mean_abs"] for i in range(len(rows) - 1))
@@ -810,8 +820,9 @@ def run_sweep(args):
                        "error_reference": "binary64 product of the bf16 inputs (gate_up, silu(g)*u, down) on 256 "
                                           "sampled (token, expert) rows",
                        "l2": "flushed between timed steps (256 MiB write outside the per-step events)"},
-            "sweep": rows, "masked_variant": masked_row, "y_error_non_increasing_in_r": mono, "e2e": None,
-            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * len(rows)}
+            "sweep": rows, "masked_variant": masked_row, "per_expert_variant": per_expert_row,
+            "y_error_non_increasing_in_r": mono, "e2e": None,
+            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * (len(rows) + 2)}
     print(json.dumps(line), flush=True)
     return 0
 

@@ -164,6 +164,26 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
                                     size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* nvfp4_quantize_grouped_sel -- nvfp4_quantize with one channel list per group of output    */
+/* rows: the per-expert RAC variant for the down projection (the pages pick "the channels     */
+/* with the largest quantization error" (Two fixes) without saying whether one list serves    */
+/* every expert; this call takes one list per expert).                                        */
+/*   row_group  int32 [q->rows_padded] (device): output row o uses list row_group[o]; a value */
+/*              < 0 writes an all-zero residual row (padding); >= groups is an error reported */
+/*              in *dev_status (the row's residual is then zero).  moe_row_groups makes it    */
+/*              from expert offsets.                                                          */
+/*   groups, sel  sel int32 [groups x Kp] (device, 16-byte aligned), each row ascending in    */
+/*              [0, K) (checked on the device: NVFP4_ERR_INVALID_ARG in *dev_status).         */
+/*   q_res      the compact residual only (cols == Kp > 0).  Other arguments as               */
+/*              nvfp4_quantize; the main codes and s_g do not depend on the lists.             */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status nvfp4_quantize_grouped_sel(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                        const int32_t* row_gather, int64_t M_out, const int32_t* row_group,
+                                        int32_t groups, const int32_t* sel, int32_t Kp, const float* amax_in,
+                                        const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                                        size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* rac_calibrate -- pick the Kp channels with the largest quantisation error                */
 /* (Two fixes: "the roughly top-50% of activation channels with the largest quantization    */
 /* error").  The calibration batch is quantised with its own s_g; e_k = sum_t r_{t,k}^2 in   */
@@ -175,6 +195,21 @@ size_t rac_calibrate_workspace_size(int64_t T, int64_t K);
 nvfp4_status rac_calibrate(const uint16_t* x_cal, int64_t T, int64_t K, int32_t Kp, int32_t* sel_out,
                            double* chan_err_out, void* workspace, size_t workspace_bytes,
                            int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* rac_calibrate_grouped -- one channel list per group of calibration rows (per-expert        */
+/* variant).  x_cal rows are grouped: group g = rows [group_offsets[g], group_offsets[g+1])   */
+/* (int32 [groups + 1], device, non-decreasing inside [0, T], else NVFP4_ERR_INVALID_ARG in   */
+/* *dev_status).  The whole batch is quantised once with its own s_g (as rac_calibrate); e_k  */
+/* of group g sums only its rows in binary64, t ascending; each group keeps its Kp largest    */
+/* (ties -> lower k), ascending.  An empty group gets channels 0 .. Kp-1.                     */
+/*   sel_out      int32 [groups x Kp]; chan_err_out optional float64 [groups x K] (device).    */
+/*   workspace    >= rac_calibrate_grouped_workspace_size(T, K, groups) bytes.                */
+/* ---------------------------------------------------------------------------------------- */
+size_t rac_calibrate_grouped_workspace_size(int64_t T, int64_t K, int32_t groups);
+nvfp4_status rac_calibrate_grouped(const uint16_t* x_cal, int64_t T, int64_t K, const int32_t* group_offsets,
+                                   int32_t groups, int32_t Kp, int32_t* sel_out, double* chan_err_out,
+                                   void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* pack_weights -- rollout side of the shared weight QDQ path (Abstract: weights aligned by  */
@@ -191,6 +226,14 @@ size_t pack_weights_workspace_size(int64_t E, int64_t N, int64_t K);
 nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel, int32_t Kp,
                           int32_t gate_up_interleave, const nvfp4_tensor* w_q, const nvfp4_tensor* w_sel_q,
                           void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* pack_weights_grouped_sel -- pack_weights with one channel list per expert: sel int32        */
+/* [E x Kp] (device, 16-byte aligned; each row ascending in [0, K), checked on the device);    */
+/* W_sel of expert e = W_e[:, sel[e]] with e's own s_gw.  Other arguments as pack_weights.     */
+nvfp4_status pack_weights_grouped_sel(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel,
+                                      int32_t Kp, int32_t gate_up_interleave, const nvfp4_tensor* w_q,
+                                      const nvfp4_tensor* w_sel_q, void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* w4a4_rac_gemm -- Y = s_a*s_w*( Q(X) Q(W)^T + Q(R_sel) Q(W_sel)^T ) in one kernel with     */
@@ -283,6 +326,13 @@ nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, in
                                int64_t rows_capacity, int32_t* expert_offsets, int32_t* row_scatter,
                                int32_t* expert_rows, int32_t* slot_expert, int32_t* slot_count, int32_t n_slots,
                                void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream);
+/* moe_row_groups -- row_group[r] = e for rows r in [expert_offsets[e], expert_offsets[e+1])  */
+/* of an expert-grouped layout (moe_dispatch_plan's offsets, any padding), -1 for rows at or  */
+/* past expert_offsets[E] and for every row when expert_offsets[E] < 0 (a plan that did not   */
+/* fit).  row_group: int32 [rows] (device).  Feeds nvfp4_quantize_grouped_sel.                */
+nvfp4_status moe_row_groups(const int32_t* expert_offsets, int32_t E, int64_t rows, int32_t* row_group,
+                            void* stream);
+
 /* moe_combine -- out[t, :] = sum_j topk_w[t, j] * y[row_scatter[t, j], :] (binary32 sums in   */
 /* j order, bf16 out); y bf16 with y_rows rows, pitch ldy; out bf16 [T x H], pitch ldo;       */
 /* H % 8 == 0.  A row < 0 contributes nothing; a row >= y_rows is NVFP4_ERR_INVALID_ARG.      */

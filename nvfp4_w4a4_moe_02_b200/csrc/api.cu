@@ -195,11 +195,15 @@ size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K) {
   return 1024 * sizeof(float);
 }
 
-nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
-                            int64_t M_out, const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
-                            const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                            void* stream) {
-  g_last_error.clear();
+}  // extern "C"
+
+namespace {
+// nvfp4_quantize and its per-group form: groups == 0 -> one shared list sel [Kp]; groups > 0 ->
+// sel [groups x Kp] and output row o takes the list of group row_group[o].
+nvfp4_status quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                           int64_t M_out, const int32_t* row_group, int32_t groups, const int32_t* sel, int32_t Kp,
+                           const float* amax_in, const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
   if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
   if (M < 0 || M_out < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "negative row count");
   if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64 <= %lld", (long long)K, (long long)kMaxK);
@@ -216,6 +220,12 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
     if (st != NVFP4_OK) return st;
     if (q_res->rows_padded != q->rows_padded || q_res->sf_layout != q->sf_layout)
       return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res must have q's rows_padded and sf_layout");
+  }
+  if (groups > 0) {
+    if (Kp == 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "per-group channel lists need Kp > 0");
+    if (q_res->cols != Kp) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "per-group lists take the compact residual (q_res cols == Kp)");
+    if (!row_group && q->rows_padded > 0) return fail(NVFP4_ERR_INVALID_ARG, "row_group is NULL");
+    if (!aligned16(sel)) return fail(NVFP4_ERR_ALIGNMENT, "sel must be 16-byte aligned");
   }
   const int P = act_partials(M, K);
   if (!amax_in) {
@@ -242,6 +252,8 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   a.src_slab_stride = 0;
   a.sel = sel;
   a.Kp = Kp;
+  a.sel_groups = groups;
+  a.row_group = row_group;
   a.partial = partial;
   a.P = P;
   a.amax_in = amax_in;
@@ -258,6 +270,30 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
   cudaError_t e = launch_rows(a, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return NVFP4_OK;
+}
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                            int64_t M_out, const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                            const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                            void* stream) {
+  g_last_error.clear();
+  return quantize_rows(x, M, K, ldx, row_gather, M_out, nullptr, 0, sel, Kp, amax_in, q, q_res, workspace,
+                       workspace_bytes, dev_status, stream);
+}
+
+nvfp4_status nvfp4_quantize_grouped_sel(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                        const int32_t* row_gather, int64_t M_out, const int32_t* row_group,
+                                        int32_t groups, const int32_t* sel, int32_t Kp, const float* amax_in,
+                                        const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (groups <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "groups must be positive");
+  if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL");
+  return quantize_rows(x, M, K, ldx, row_gather, M_out, row_group, groups, sel, Kp, amax_in, q, q_res, workspace,
+                       workspace_bytes, dev_status, stream);
 }
 
 nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
@@ -326,21 +362,29 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
 }
 
 // ------------------------------------------------------------------------------------------ calibrate
-size_t rac_calibrate_workspace_size(int64_t T, int64_t K) {
+size_t rac_calibrate_workspace_size(int64_t T, int64_t K) { return rac_calibrate_grouped_workspace_size(T, K, 1); }
+
+size_t rac_calibrate_grouped_workspace_size(int64_t T, int64_t K, int32_t groups) {
+  const size_t G = (size_t)(groups > 0 ? groups : 1);
   return round_up(1024 * sizeof(float), 256) + round_up((size_t)T * (size_t)K * sizeof(float), 256) +
-         round_up((size_t)K * sizeof(double), 256);
+         round_up(G * (size_t)K * sizeof(double), 256);
 }
 
-nvfp4_status rac_calibrate(const uint16_t* x_cal, int64_t T, int64_t K, int32_t Kp, int32_t* sel_out,
-                           double* chan_err_out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
-                           void* stream) {
-  g_last_error.clear();
+}  // extern "C"
+
+namespace {
+// rac_calibrate and its per-group form (offsets == nullptr: one group of all T rows)
+nvfp4_status calibrate_rows(const uint16_t* x_cal, int64_t T, int64_t K, const int32_t* offsets, int32_t groups,
+                            int32_t Kp, int32_t* sel_out, double* chan_err_out, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, void* stream) {
   if (!x_cal || (!sel_out && Kp > 0)) return fail(NVFP4_ERR_INVALID_ARG, "x_cal / sel_out is NULL");
   if (T <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T must be positive");
   if (K <= 0 || K % 64 != 0 || K > kMaxCalK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64 <= %lld", (long long)K, (long long)kMaxCalK);
   if (Kp < 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp out of range");
+  if (groups < 1 || groups > 65535) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "groups must be in [1, 65535]");
   if (!aligned16(x_cal)) return fail(NVFP4_ERR_ALIGNMENT, "x_cal must be 16-byte aligned");
-  if (!workspace || workspace_bytes < rac_calibrate_workspace_size(T, K)) return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+  if (!workspace || workspace_bytes < rac_calibrate_grouped_workspace_size(T, K, groups))
+    return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
   if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   char* ws = reinterpret_cast<char*>(workspace);
@@ -367,26 +411,20 @@ nvfp4_status rac_calibrate(const uint16_t* x_cal, int64_t T, int64_t K, int32_t 
   a.status = dev_status;
   e = launch_rows(a, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "calibration residual launch");
-  e = launch_chan_err(resid, T, K, err, s);
+  e = launch_chan_err(resid, T, K, offsets, groups, err, dev_status, s);
   if (e != cudaSuccess) return cuda_fail(e, "channel error launch");
   if (Kp > 0 || chan_err_out) {
-    e = launch_select(err, (int32_t)K, Kp, sel_out, chan_err_out, s);
+    e = launch_select(err, (int32_t)K, Kp, groups, sel_out, chan_err_out, s);
     if (e != cudaSuccess) return cuda_fail(e, "selection launch");
   }
   return NVFP4_OK;
 }
 
-// ------------------------------------------------------------------------------------------ pack
-size_t pack_weights_workspace_size(int64_t E, int64_t N, int64_t K) {
-  (void)N;
-  (void)K;
-  return round_up((size_t)(E > 0 ? E : 1) * (size_t)slab_partials(E) * sizeof(float), 256);
-}
-
-nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel, int32_t Kp,
-                          int32_t gate_up_interleave, const nvfp4_tensor* w_q, const nvfp4_tensor* w_sel_q,
-                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
-  g_last_error.clear();
+// pack_weights and its per-expert form (sel [E x Kp] when per_expert)
+nvfp4_status pack_rows(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel, int32_t Kp,
+                       bool per_expert, int32_t gate_up_interleave, const nvfp4_tensor* w_q,
+                       const nvfp4_tensor* w_sel_q, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                       void* stream) {
   if (!w) return fail(NVFP4_ERR_INVALID_ARG, "w is NULL");
   if (E <= 0 || N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E > 0 and N %% 128 == 0 required");
   if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
@@ -398,6 +436,7 @@ nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, co
   if (w_q->rows_padded != N || w_q->rows != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_q rows / rows_padded must equal N");
   if (Kp > 0) {
     if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
+    if (per_expert && !aligned16(sel)) return fail(NVFP4_ERR_ALIGNMENT, "sel must be 16-byte aligned");
     st = check_tensor(w_sel_q, "w_sel_q", Kp, N, E);
     if (st != NVFP4_OK) return st;
     if (w_sel_q->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_sel_q rows_padded must equal N");
@@ -422,6 +461,7 @@ nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, co
   a.N_half = N / 2;
   a.sel = sel;
   a.Kp = Kp;
+  a.sel_groups = (per_expert && Kp > 0) ? (int32_t)E : 0;
   a.partial = partial;
   a.P = P;
   a.s_g_out = w_q->s_g;
@@ -434,6 +474,50 @@ nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, co
   e = launch_rows(a, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "pack launch");
   return NVFP4_OK;
+}
+}  // namespace
+
+extern "C" {
+
+nvfp4_status rac_calibrate(const uint16_t* x_cal, int64_t T, int64_t K, int32_t Kp, int32_t* sel_out,
+                           double* chan_err_out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                           void* stream) {
+  g_last_error.clear();
+  return calibrate_rows(x_cal, T, K, nullptr, 1, Kp, sel_out, chan_err_out, workspace, workspace_bytes, dev_status,
+                        stream);
+}
+
+nvfp4_status rac_calibrate_grouped(const uint16_t* x_cal, int64_t T, int64_t K, const int32_t* group_offsets,
+                                   int32_t groups, int32_t Kp, int32_t* sel_out, double* chan_err_out,
+                                   void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!group_offsets) return fail(NVFP4_ERR_INVALID_ARG, "group_offsets is NULL");
+  return calibrate_rows(x_cal, T, K, group_offsets, groups, Kp, sel_out, chan_err_out, workspace, workspace_bytes,
+                        dev_status, stream);
+}
+
+// ------------------------------------------------------------------------------------------ pack
+size_t pack_weights_workspace_size(int64_t E, int64_t N, int64_t K) {
+  (void)N;
+  (void)K;
+  return round_up((size_t)(E > 0 ? E : 1) * (size_t)slab_partials(E) * sizeof(float), 256);
+}
+
+nvfp4_status pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel, int32_t Kp,
+                          int32_t gate_up_interleave, const nvfp4_tensor* w_q, const nvfp4_tensor* w_sel_q,
+                          void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  return pack_rows(w, E, N, K, sel, Kp, false, gate_up_interleave, w_q, w_sel_q, workspace, workspace_bytes,
+                   dev_status, stream);
+}
+
+nvfp4_status pack_weights_grouped_sel(const uint16_t* w, int64_t E, int64_t N, int64_t K, const int32_t* sel,
+                                      int32_t Kp, int32_t gate_up_interleave, const nvfp4_tensor* w_q,
+                                      const nvfp4_tensor* w_sel_q, void* workspace, size_t workspace_bytes,
+                                      int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  return pack_rows(w, E, N, K, sel, Kp, true, gate_up_interleave, w_q, w_sel_q, workspace, workspace_bytes,
+                   dev_status, stream);
 }
 
 // ------------------------------------------------------------------------------------------ GEMMs
@@ -696,6 +780,16 @@ nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, in
                                        expert_offsets, row_scatter, expert_rows, slot_expert, slot_count, n_slots,
                                        num_sms(), dev_status, s);
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "dispatch plan launch");
+}
+
+nvfp4_status moe_row_groups(const int32_t* expert_offsets, int32_t E, int64_t rows, int32_t* row_group,
+                            void* stream) {
+  g_last_error.clear();
+  if (E <= 0 || rows < 0 || rows > INT32_MAX) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E > 0 and 0 <= rows <= INT32_MAX required");
+  if (rows == 0) return NVFP4_OK;
+  if (!expert_offsets || !row_group) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  cudaError_t e = launch_row_groups(expert_offsets, E, rows, row_group, num_sms(), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "row groups launch");
 }
 
 nvfp4_status moe_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* row_scatter,

@@ -26,8 +26,10 @@ struct RowArgs {
   int64_t src_slab_stride;       // pack: N*K elements between slabs
   int interleave;                // pack: SwiGLU gate/up interleave
   int64_t N_half;                // pack: N/2
-  const int32_t* sel;            // ascending channel list [Kp]
+  const int32_t* sel;            // ascending channel list [Kp], or [sel_groups x Kp]
   int32_t Kp;
+  int32_t sel_groups;            // 0: one shared list; G > 0: one list per group (per-expert variant)
+  const int32_t* row_group;      // act with sel_groups: output row -> group (< 0: zero residual)
   // scale source
   const float* partial;          // amax partials [slabs x P]
   int P;
@@ -49,8 +51,10 @@ cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64
                         int P, int32_t* status, cudaStream_t st);
 cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st);
 size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps, bool masked = false);
-cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, double* err, cudaStream_t st);
-cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t* sel, double* err_out, cudaStream_t st);
+cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, const int32_t* off, int32_t groups,
+                            double* err, int32_t* status, cudaStream_t st);
+cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t groups, int32_t* sel, double* err_out,
+                          cudaStream_t st);
 cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint16_t* out, const float* partial, int P,
                        float* s_g_out, int32_t* status, int num_sms, cudaStream_t st);
 cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
@@ -128,6 +132,7 @@ cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, in
                                  int32_t* counts, int32_t* offsets, int32_t* row_scatter, int32_t* expert_rows,
                                  int32_t* slot_expert, int32_t* slot_count, int n_slots, int num_sms,
                                  int32_t* status, cudaStream_t st);
+cudaError_t launch_row_groups(const int32_t* off, int E, int64_t rows, int32_t* group, int num_sms, cudaStream_t st);
 cudaError_t launch_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* rows, const float* w,
                            int64_t T, int k, int64_t H, uint16_t* out, int64_t ldo, int num_sms, int32_t* status,
                            cudaStream_t st);

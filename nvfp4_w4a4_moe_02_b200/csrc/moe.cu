@@ -211,8 +211,40 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 }
 
 // ----------------------------------------------------------------------------------------
+// row -> expert of an expert-grouped layout: row r of segment [off[e], off[e+1]) gets e, rows at or
+// past off[E] get -1 (padding capacity); off[E] < 0 (a plan that did not fit) gives -1 everywhere.
+// Used to pick each row's channel list when the down projection has one list per expert.
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) row_groups_kernel(const int32_t* __restrict__ off, int E, int64_t rows,
+                                                         int32_t* __restrict__ group) {
+  const int32_t end = __ldg(off + E);
+  for (int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; r < rows; r += (int64_t)gridDim.x * blockDim.x) {
+    int32_t g = -1;
+    if (end >= 0 && r < end && r >= __ldg(off)) {
+      // largest e with off[e] <= r (segments are non-decreasing); empty segments are skipped over
+      int lo = 0, hi = E - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((int64_t)__ldg(off + mid) <= r) lo = mid;
+        else hi = mid - 1;
+      }
+      g = lo;
+    }
+    group[r] = g;
+  }
+}
+
+// ----------------------------------------------------------------------------------------
 // launchers
 // ----------------------------------------------------------------------------------------
+cudaError_t launch_row_groups(const int32_t* off, int E, int64_t rows, int32_t* group, int num_sms, cudaStream_t st) {
+  int64_t blocks = (rows + 255) / 256;
+  if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+  if (blocks < 1) blocks = 1;
+  row_groups_kernel<<<(unsigned)blocks, 256, 0, st>>>(off, E, rows, group);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* status,
                               cudaStream_t st) {
   const int64_t blocks = (T + 7) / 8;

@@ -150,15 +150,18 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
   constexpr bool kHasSel = (MODE == kModeAct || MODE == kModePack);
   const bool masked = MODE == kModeAct && a.masked_res != 0 && Kp > 0;
   const bool use_sel = kHasSel && Kp > 0 && !masked;  // compact residual pass
+  // per-group channel lists (pack: group = slab; act: group = row_group[row]) are read from
+  // global memory (L1-resident) in the residual pass instead of the CTA-shared copy
+  const bool grouped = use_sel && a.sel_groups > 0;
 
   // CTA-shared channel list (int16), then per warp (per CTA when SPLIT) each block's (d, 1/d);
   // the masked variant keeps a bitmap of the selected channels instead
   int16_t* sel_s = reinterpret_cast<int16_t*>(smem_raw);
   uint32_t* mask_s = reinterpret_cast<uint32_t*>(smem_raw);
-  const size_t sel_bytes = use_sel ? (((size_t)Kp * 2 + 15) / 16) * 16 : 0;
+  const size_t sel_bytes = (use_sel && !grouped) ? (((size_t)Kp * 2 + 15) / 16) * 16 : 0;
   const size_t warp_bytes = use_sel ? (size_t)(K / 16) * 8 : 0;
   float2* dinv_s = reinterpret_cast<float2*>(smem_raw + sel_bytes + (SPLIT ? 0 : warp) * warp_bytes);
-  if (use_sel || masked) {
+  if ((use_sel && !grouped) || masked) {
     if (masked) {
       for (int32_t w = threadIdx.x; w < (K + 31) / 32; w += blockDim.x) mask_s[w] = 0u;
       __syncthreads();
@@ -211,6 +214,16 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
       src_row = (j < 64) ? (q * 64 + j) : (a.N_half + q * 64 + (j - 64));
     }
     const bool valid = (src_row >= 0 && src_row < a.src_rows);
+    // this row's channel list when the lists are per group (nullptr: the residual row is zero)
+    const int32_t* gsel = nullptr;
+    if (grouped) {
+      const int64_t g = (MODE == kModePack) ? slab : (int64_t)a.row_group[row];
+      if (g >= a.sel_groups) {
+        if (lane == 0) report_status(a.status, kErrInvalid);
+      } else if (g >= 0) {
+        gsel = a.sel + g * Kp;
+      }
+    }
     if (slab != cached_slab) {
       float amax = (MODE == kModeAct && a.amax_in != nullptr) ? *a.amax_in : reduce_partials(a.partial + slab * a.P, a.P);
       s_g = scale_from_amax(amax, a.status);
@@ -304,7 +317,8 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
         const int32_t p = base + 16 * lane;
         const bool h = p < Kp;
         int32_t ch[16];
-        {
+        bool rvalid = valid;
+        if (!grouped) {
           const uint4 c0 = h ? *reinterpret_cast<const uint4*>(sel_s + p) : make_uint4(0, 0, 0, 0);
           const uint4 c1 = h ? *reinterpret_cast<const uint4*>(sel_s + p + 8) : make_uint4(0, 0, 0, 0);
           const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
@@ -313,10 +327,33 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
             ch[2 * q] = (int32_t)(int16_t)(w[q] & 0xFFFFu);
             ch[2 * q + 1] = (int32_t)(int16_t)(w[q] >> 16);
           }
+        } else {
+          rvalid = valid && gsel != nullptr;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int4 c = (h && gsel) ? __ldg(reinterpret_cast<const int4*>(gsel + p) + q) : make_int4(0, 0, 0, 0);
+            ch[4 * q] = c.x;
+            ch[4 * q + 1] = c.y;
+            ch[4 * q + 2] = c.z;
+            ch[4 * q + 3] = c.w;
+          }
+          // the list must be ascending and inside [0, K): checked where it is used
+          bool bad = false;
+          int32_t prev = (h && gsel && p > 0) ? __ldg(gsel + p - 1) : -1;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            bad |= (ch[i] <= prev) || (ch[i] >= K);
+            prev = ch[i];
+          }
+          if (h && gsel && bad) {
+            report_status(a.status, kErrInvalid);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) ch[i] = 0;
+          }
         }
         float v[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = (h && valid) ? bf16_bits_to_f32(__ldg(srow + ch[i])) : 0.0f;
+        for (int i = 0; i < 16; ++i) v[i] = (h && rvalid) ? bf16_bits_to_f32(__ldg(srow + ch[i])) : 0.0f;
         if (MODE != kModePack) {
           // re-derive each channel's code under its own block scale, then r = x - e*d
 #pragma unroll
@@ -356,22 +393,35 @@ __global__ void __launch_bounds__(256, 4) quant_rows_kernel(const RowArgs a) {
 // calibration: e_k = sum_t r_{t,k}^2 in binary64, t ascending (one thread per channel), then
 // selection of the Kp largest (ties -> lower k), written ascending.
 // ----------------------------------------------------------------------------------------
+// Grouped form (one channel list per expert): blockIdx.y = group g sums rows [off[g], off[g+1])
+// into err[g * K + k]; off == nullptr is the single group [0, T).
 __global__ void __launch_bounds__(256) chan_err_kernel(const float* __restrict__ resid, int64_t T, int64_t K,
-                                                       double* __restrict__ err) {
+                                                       const int32_t* __restrict__ off, double* __restrict__ err,
+                                                       int32_t* status) {
   int64_t k = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (k >= K) return;
+  const int64_t g = blockIdx.y;
+  int64_t t0 = off ? (int64_t)off[g] : 0, t1 = off ? (int64_t)off[g + 1] : T;
+  if (t0 < 0 || t1 < t0 || t1 > T) {  // offsets must be non-decreasing inside [0, T]
+    if (k == 0) report_status(status, kErrInvalid);
+    t0 = t1 = 0;
+  }
   double e = 0.0;
-  for (int64_t t = 0; t < T; ++t) {
+  for (int64_t t = t0; t < t1; ++t) {
     double v = (double)resid[t * K + k];
     e = __dadd_rn(e, __dmul_rn(v, v));
   }
-  err[k] = e;
+  err[g * K + k] = e;
 }
 
-// One CTA of 1024 threads; K <= kMaxCalK.
+// One CTA of 1024 threads per group (blockIdx.x = g selects from err + g K into sel_out + g Kp);
+// K <= kMaxCalK.
 __global__ void __launch_bounds__(1024) select_topk_kernel(const double* __restrict__ err, int32_t K, int32_t Kp,
                                                            int32_t* __restrict__ sel_out, double* __restrict__ err_out) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
+  err += (int64_t)blockIdx.x * K;
+  sel_out += (int64_t)blockIdx.x * Kp;
+  if (err_out) err_out += (int64_t)blockIdx.x * K;
   double* e = reinterpret_cast<double*>(smem_raw);
   int32_t* flag = reinterpret_cast<int32_t*>(e + K);
   __shared__ int32_t warp_sums[32];
@@ -591,16 +641,19 @@ cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, double* err, cudaStream_t st) {
-  chan_err_kernel<<<(unsigned)((K + 255) / 256), 256, 0, st>>>(resid, T, K, err);
+cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, const int32_t* off, int32_t groups,
+                            double* err, int32_t* status, cudaStream_t st) {
+  const dim3 grid((unsigned)((K + 255) / 256), (unsigned)(off ? groups : 1));
+  chan_err_kernel<<<grid, 256, 0, st>>>(resid, T, K, off, err, status);
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t* sel, double* err_out, cudaStream_t st) {
+cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t groups, int32_t* sel, double* err_out,
+                          cudaStream_t st) {
   size_t smem = (size_t)K * 8 + (size_t)K * 4;
   cudaError_t e = cudaFuncSetAttribute(select_topk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  select_topk_kernel<<<1, 1024, smem, st>>>(err, K, Kp, sel, err_out);
+  select_topk_kernel<<<(unsigned)groups, 1024, smem, st>>>(err, K, Kp, sel, err_out);
   return cudaGetLastError();
 }
 

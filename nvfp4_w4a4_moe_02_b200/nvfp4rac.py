@@ -64,10 +64,16 @@ def load() -> ctypes.CDLL:
         "nvfp4_quantize_workspace_size": ([i64, i64], sz),
         "nvfp4_quantize": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
         "nvfp4_quantize_scatter": ([vp, i64, i64, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "nvfp4_quantize_grouped_sel": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp],
+                                       ctypes.c_int),
         "rac_calibrate_workspace_size": ([i64, i64], sz),
         "rac_calibrate": ([vp, i64, i64, i32, vp, vp, vp, sz, vp, vp], ctypes.c_int),
+        "rac_calibrate_grouped_workspace_size": ([i64, i64, i32], sz),
+        "rac_calibrate_grouped": ([vp, i64, i64, vp, i32, i32, vp, vp, vp, sz, vp, vp], ctypes.c_int),
         "pack_weights_workspace_size": ([i64, i64, i64], sz),
         "pack_weights": ([vp, i64, i64, i64, vp, i32, i32, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "pack_weights_grouped_sel": ([vp, i64, i64, i64, vp, i32, i32, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "moe_row_groups": ([vp, i32, i64, vp, vp], ctypes.c_int),
         "w4a4_rac_gemm": ([tp, tp, tp, tp, i64, i64, i64, i32, ctypes.c_int, vp, i64, vp, vp], ctypes.c_int),
         "grouped_w4a4_rac_moe": ([tp, tp, vp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, i64,
                                   vp, vp, vp], ctypes.c_int),
@@ -211,17 +217,20 @@ def set_gemm_tile_n(n: int):
 def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather: torch.Tensor | None = None,
                    M_out: int | None = None, rows_padded: int | None = None, amax_in: torch.Tensor | None = None,
                    out: Packed | None = None, out_res: Packed | None = None, status: torch.Tensor | None = None,
-                   stream=None, masked: bool = False):
+                   stream=None, masked: bool = False, row_group: torch.Tensor | None = None):
     """Online activation quantisation with the residual pass on ``sel`` -> (Packed, Packed | None).
 
     masked=True selects the masked full-K residual variant (residual at its channel, zero off
-    ``sel``, K wide): pair it with the main packed weight as w_sel in w4a4_rac_gemm."""
+    ``sel``, K wide): pair it with the main packed weight as w_sel in w4a4_rac_gemm.
+    A 2-D ``sel`` [G, Kp] is one channel list per group (the per-expert variant): output row o
+    uses list ``row_group[o]`` (int32 [rows_padded]; < 0 gives a zero residual row)."""
     lib = load()
     _u16(x)
     M, K = x.shape
     ldx = x.stride(0)
     assert x.stride(1) == 1
-    Kp = 0 if sel is None else int(sel.numel())
+    grouped = sel is not None and sel.dim() == 2
+    Kp = 0 if sel is None else int(sel.shape[-1])
     if M_out is None:
         M_out = M if row_gather is None else int(row_gather.numel())
     if out is None:
@@ -233,6 +242,14 @@ def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather:
     st = status if status is not None else new_status(x.device)
     q = out.c()
     qr = out_res.c() if Kp > 0 else None
+    if grouped:
+        assert not masked and row_group is not None and row_group.dtype == torch.int32
+        assert sel.dtype == torch.int32 and sel.is_contiguous() and row_group.numel() >= out.rows_padded
+        _check(lib.nvfp4_quantize_grouped_sel(x.data_ptr(), M, K, ldx, _ptr(row_gather), M_out, row_group.data_ptr(),
+                                              int(sel.shape[0]), sel.data_ptr(), Kp, _ptr(amax_in), ctypes.byref(q),
+                                              ctypes.byref(qr), ws.data_ptr(), ws.numel(), st.data_ptr(),
+                                              _stream(stream)))
+        return out, out_res
     _check(lib.nvfp4_quantize(x.data_ptr(), M, K, ldx, _ptr(row_gather), M_out, _ptr(sel), Kp, _ptr(amax_in),
                               ctypes.byref(q), ctypes.byref(qr) if qr is not None else None, ws.data_ptr(),
                               ws.numel(), st.data_ptr(), _stream(stream)))
@@ -285,17 +302,49 @@ def rac_calibrate(x_cal: torch.Tensor, Kp: int, want_err: bool = False, status: 
     return sel, err
 
 
+def rac_calibrate_grouped(x_cal: torch.Tensor, offsets: torch.Tensor, Kp: int, want_err: bool = False,
+                          status: torch.Tensor | None = None, stream=None):
+    """One channel list per group of calibration rows (group g = rows [offsets[g], offsets[g+1]),
+    int32 device tensor [G + 1]) -> (sel int32 [G, Kp], err float64 [G, K] | None)."""
+    lib = load()
+    _u16(x_cal)
+    T, K = x_cal.shape
+    assert x_cal.is_contiguous() and offsets.dtype == torch.int32 and offsets.is_cuda
+    G = int(offsets.numel()) - 1
+    sel = torch.empty(G, Kp, dtype=torch.int32, device=x_cal.device)
+    err = torch.empty(G, K, dtype=torch.float64, device=x_cal.device) if want_err else None
+    ws = _workspace(x_cal.device).get(lib.rac_calibrate_grouped_workspace_size(T, K, G))
+    st = status if status is not None else new_status(x_cal.device)
+    _check(lib.rac_calibrate_grouped(x_cal.data_ptr(), T, K, offsets.data_ptr(), G, Kp, sel.data_ptr(), _ptr(err),
+                                     ws.data_ptr(), ws.numel(), st.data_ptr(), _stream(stream)))
+    return sel, err
+
+
+def moe_row_groups(expert_offsets: torch.Tensor, E: int, rows: int, out: torch.Tensor | None = None, stream=None):
+    """Expert of every row of an expert-grouped layout (-1 past the last segment) -> int32 [rows]."""
+    lib = load()
+    if out is None:
+        out = torch.empty(max(rows, 1), dtype=torch.int32, device=expert_offsets.device)
+    _check(lib.moe_row_groups(expert_offsets.data_ptr(), E, rows, out.data_ptr(), _stream(stream)))
+    return out
+
+
 def pack_weights(w: torch.Tensor, sel: torch.Tensor | None = None, gate_up_interleave: bool = False,
                  out: Packed | None = None, out_sel: Packed | None = None, status: torch.Tensor | None = None,
                  stream=None):
-    """Rollout weight pack: Q(W) and Q(W[:, sel]) with one scale per slab -> (Packed, Packed | None)."""
+    """Rollout weight pack: Q(W) and Q(W[:, sel]) with one scale per slab -> (Packed, Packed | None).
+
+    A 2-D ``sel`` [E, Kp] is one channel list per expert (W_sel of expert e = W_e[:, sel[e]])."""
     lib = load()
     _u16(w)
     if w.dim() == 2:
         w = w.unsqueeze(0)
     E, N, K = w.shape
     assert w.is_contiguous()
-    Kp = 0 if sel is None else int(sel.numel())
+    grouped = sel is not None and sel.dim() == 2
+    if grouped:
+        assert sel.shape[0] == E and sel.dtype == torch.int32 and sel.is_contiguous()
+    Kp = 0 if sel is None else int(sel.shape[-1])
     if out is None:
         out = Packed.empty(N, K, slabs=E, rows_padded=N, device=w.device)
     if Kp > 0 and out_sel is None:
@@ -304,9 +353,9 @@ def pack_weights(w: torch.Tensor, sel: torch.Tensor | None = None, gate_up_inter
     st = status if status is not None else new_status(w.device)
     q = out.c()
     qs = out_sel.c() if Kp > 0 else None
-    _check(lib.pack_weights(w.data_ptr(), E, N, K, _ptr(sel), Kp, int(gate_up_interleave), ctypes.byref(q),
-                            ctypes.byref(qs) if qs is not None else None, ws.data_ptr(), ws.numel(), st.data_ptr(),
-                            _stream(stream)))
+    fn = lib.pack_weights_grouped_sel if grouped else lib.pack_weights
+    _check(fn(w.data_ptr(), E, N, K, _ptr(sel), Kp, int(gate_up_interleave), ctypes.byref(q),
+              ctypes.byref(qs) if qs is not None else None, ws.data_ptr(), ws.numel(), st.data_ptr(), _stream(stream)))
     return out, (out_sel if Kp > 0 else None)
 
 

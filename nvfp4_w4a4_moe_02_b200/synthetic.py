@@ -378,6 +378,18 @@ def moe_down_calibration_batch(wl: MoEWorkload, max_pairs: int | None = None) ->
     return out
 
 
+def moe_down_calibration_offsets(wl: MoEWorkload, max_pairs: int | None = None) -> np.ndarray:
+    """Expert segments of moe_down_calibration_batch's rows (same routing, (expert, token) order):
+    rows [off[e], off[e+1]) belong to expert e.  Returns int64 [E + 1]."""
+    T = wl.x_cal.shape[0]
+    k = wl.topk_ids.shape[1]
+    topk = route_topk(wl.seed, T, wl.E, k, stream=STREAM_ROUTER_CAL)
+    _, pe, _ = sort_pairs(topk, wl.E)
+    if max_pairs is not None:
+        pe = pe[:max_pairs]
+    return np.searchsorted(pe, np.arange(wl.E + 1), side="left").astype(np.int64)
+
+
 def moe_down_calibration_batch_torch(wl: MoEWorkload, device, max_pairs: int | None = None) -> np.ndarray:
     """moe_down_calibration_batch with the binary64 products formed by torch on `device` and the
     weights made there (for experts too large to make on the host).  Same routing, pooling and

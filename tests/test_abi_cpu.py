@@ -127,6 +127,39 @@ def test_decode_and_layout_rejections(lib):
     assert st == 2
 
 
+def test_grouped_sel_rejections(lib):
+    """Per-expert channel lists: argument checks on the host, before any device work."""
+    from nvfp4_w4a4_moe_02_b200.nvfp4rac import CTensor
+
+    q = CTensor(16, 16, 16, 1, 64, 128, 128)
+    qr = CTensor(16, 16, 16, 1, 64, 128, 64)
+    qm = CTensor(16, 16, 16, 1, 64, 128, 128)  # K wide: the masked variant's residual
+
+    def quant(row_group=16, groups=2, sel=16, res=qr):
+        return lib.nvfp4_quantize_grouped_sel(16, 64, 128, 128, None, 64, row_group, groups, sel, 64, None,
+                                              ctypes.byref(q), ctypes.byref(res), 16, 1024, None, None)
+
+    assert quant(groups=0) == 2
+    assert quant(sel=None) == 1
+    assert quant(res=qm) == 2 and b"compact" in lib.nvfp4_last_error_string()
+    assert quant(row_group=None) == 1
+    assert quant(sel=24) == 3
+    # calibration: offsets required, group count in range
+    assert lib.rac_calibrate_grouped(16, 64, 128, None, 2, 64, 16, None, 16, 1 << 30, None, None) == 1
+    assert lib.rac_calibrate_grouped(16, 64, 128, 16, 0, 64, 16, None, 16, 1 << 30, None, None) == 2
+    assert lib.rac_calibrate_grouped_workspace_size(64, 128, 3) > lib.rac_calibrate_workspace_size(64, 128)
+    # pack: per-expert lists must be 16-byte aligned
+    w_q = CTensor(16, 16, 16, 2, 128, 128, 128)
+    w_s = CTensor(16, 16, 16, 2, 128, 128, 64)
+    st = lib.pack_weights_grouped_sel(16, 2, 128, 128, 24, 64, 0, ctypes.byref(w_q), ctypes.byref(w_s), 16, 1 << 20,
+                                      None, None)
+    assert st == 3
+    # row groups: nothing to do for zero rows; E must be positive; buffers must be given
+    assert lib.moe_row_groups(None, 4, 0, None, None) == 0
+    assert lib.moe_row_groups(16, 0, 8, 16, None) == 2
+    assert lib.moe_row_groups(None, 4, 8, 16, None) == 1
+
+
 def test_decode_slots_host_logic():
     from nvfp4_w4a4_moe_02_b200.nvfp4rac import decode_slots
 

@@ -377,13 +377,14 @@ def moe_pipeline(dev, wl, sel_gu, sel_dn):
     wgu = to_dev(wl.wgu, dev)
     wdn = to_dev(wl.wdn, dev)
     seld_gu = torch.from_numpy(sel_gu).to(dev)
-    seld_dn = torch.from_numpy(sel_dn).to(dev)
+    seld_dn = torch.from_numpy(np.ascontiguousarray(sel_dn)).to(dev)  # 2-D: one list per expert
     pgu, pgus = R.pack_weights(wgu, seld_gu, gate_up_interleave=True, status=st)
     pdn, pdns = R.pack_weights(wdn, seld_dn, status=st)
     sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
     a, ar = R.nvfp4_quantize_scatter(to_dev(wl.x, dev), sm, g.size, seld_gu, status=st)
     h, amax_h = R.grouped_w4a4_rac_moe(a, ar, offd, pgu, pgus, swiglu=True, status=st)
-    hq, hqr = R.nvfp4_quantize(h, seld_dn, amax_in=amax_h, status=st)
+    row_group = R.moe_row_groups(offd, wl.E, g.size) if seld_dn.dim() == 2 else None
+    hq, hqr = R.nvfp4_quantize(h, seld_dn, amax_in=amax_h, status=st, row_group=row_group)
     y = R.grouped_w4a4_rac_moe(hq, hqr, offd, pdn, pdns, status=st)
     torch.cuda.synchronize()
     R.check_status(st)
@@ -434,13 +435,14 @@ def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs, wgu_of=None, wdn_of=No
         bad = np.argwhere(np.abs(h_g - h_ref) > tol_h)
         assert bad.size == 0, (e, bad[:5], h_g[tuple(bad[0])], h_ref[tuple(bad[0])])
         # down: the GPU's h rows quantised by the oracle must match the GPU codes bit for bit
+        sel_e = sel_dn[e] if sel_dn.ndim == 2 else sel_dn  # per-expert lists: the expert's own
         hrows = h_gpu[rows]
-        hc, hS, hrc, hrS, _ = orc.act_quant_rac(hrows, s_h, sel_dn)
+        hc, hS, hrc, hrS, _ = orc.act_quant_rac(hrows, s_h, sel_e)
         assert np.array_equal(gq_c[rows], hc) and np.array_equal(gq_S[rows], hS)
         assert np.array_equal(gqr_c[rows], hrc) and np.array_equal(gqr_S[rows], hrS)
         wdn = wdn_of(e)
         s_wd = orc.global_scale(orc.amax_bf16(wdn))
-        dc, dS, dsc, dsS = orc.weight_pack(wdn, s_wd, sel_dn)
+        dc, dS, dsc, dsS = orc.weight_pack(wdn, s_wd, sel_e)
         y_ref, ad2 = orc.gemm_rac(hc, hS, hrc, hrS, dc, dS, dsc, dsS, s_h, s_wd)
         y_g = out["y"][torch.from_numpy(rows).to(out["y"].device)].float().cpu().numpy()
         assert_gemm_close(y_g, y_ref, ad2, True)
@@ -461,6 +463,29 @@ def test_moe_small_ragged(dev, orc):
     sel_dn, _ = orc.calibrate(h_cal, wl.Kp_dn)
     out = moe_pipeline(dev, wl, sel_gu, sel_dn)
     check_moe(orc, wl, sel_gu, sel_dn, out, list(range(wl.pair_token.size)))
+
+
+def test_moe_per_expert_down_lists(dev, orc):
+    """The per-expert variant: the down projection's channel lists come from each expert's own
+    calibration rows (GPU calibration bit-exact against the oracle), the weights are packed with
+    them, h is quantised with its row's list, and the outputs match the oracle per expert."""
+    wl = syn.moe_block(T=96, H=512, E=8, topk=2, I=128, T_cal=64)
+    sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
+    h_cal = syn.moe_down_calibration_batch(wl)
+    off_cal = syn.moe_down_calibration_offsets(wl)
+    sel_dn, err_dn = orc.calibrate_grouped(h_cal, off_cal, wl.Kp_dn)
+    gsel, gerr = R.rac_calibrate_grouped(to_dev(h_cal, dev), torch.from_numpy(off_cal.astype(np.int32)).to(dev),
+                                         wl.Kp_dn, want_err=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(gerr.cpu().numpy(), err_dn) and np.array_equal(gsel.cpu().numpy(), sel_dn)
+    assert len({tuple(r) for r in sel_dn}) > 1  # the lists really differ between experts
+    out = moe_pipeline(dev, wl, sel_gu, sel_dn)
+    check_moe(orc, wl, sel_gu, sel_dn, out, list(range(wl.pair_token.size)))
+    # padding rows (row group -1) carry an all-zero residual
+    gqr_c, gqr_S = logical(out["hqr"], rows=out["hqr"].rows_padded)
+    pad = np.ones(gqr_c.shape[0], bool)
+    pad[out["pair_rows"]] = False
+    assert not gqr_c[pad].any() and not gqr_S[pad].any()
 
 
 @pytest.mark.parametrize("which", ["tiny", "ragged", "aligned_full"])
