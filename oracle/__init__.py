@@ -68,6 +68,11 @@ def _get():
         "orc_route_topk": ([vp, i64, i32, i32, vp, vp], None),
         "orc_dispatch_plan": ([vp, i64, i32, i32, i32, vp, vp], None),
         "orc_combine": ([vp, i64, vp, vp, i64, i32, i64, vp], None),
+        "orc_mx8_exponent": ([f32], ctypes.c_int),
+        "orc_e4m3_encode_signed": ([f32], ctypes.c_int),
+        "orc_e4m3_decode_signed": ([ctypes.c_int], f64),
+        "orc_mx8_quantize": ([vp, i64, i64, i64, vp, vp], None),
+        "orc_mx8_gemm": ([vp, vp, vp, vp, i64, i64, i64, vp, vp], None),
     }
     for name, (args, res) in sigs.items():
         fn = getattr(lib, name)
@@ -360,3 +365,46 @@ def dense_rac_forward(x: np.ndarray, w: np.ndarray, sel: np.ndarray, rows=None):
     y, ad = gemm_rac(a, aS, r, rS, wc, wS, wsc, wsS, s_x, s_w, rows=rows)
     return dict(s_x=s_x, a=a, aS=aS, r=r, rS=rS, resid=resid, s_w=s_w, wc=wc, wS=wS, wsc=wsc, wsS=wsS, y=y,
                 absdot=ad)
+
+
+# ---- FP8 comparison format: E4M3 elements, one power-of-two scale per 32 elements along K ----
+def mx8_exponent(b: float) -> int:
+    """Smallest X in [-127, 127] with 448 * 2^X >= b."""
+    return int(_get().orc_mx8_exponent(np.float32(b)))
+
+
+def e4m3_encode_signed(v: float) -> int:
+    return int(_get().orc_e4m3_encode_signed(np.float32(v)))
+
+
+def e4m3_decode_signed(code: int) -> float:
+    return float(_get().orc_e4m3_decode_signed(int(code)))
+
+
+def mx8_quantize(x: np.ndarray):
+    """bf16 x [rows, K] (K % 32 == 0) -> (codes uint8 [rows, K], E8M0 scale codes uint8 [rows, K/32])."""
+    x = _c(x, np.uint16)
+    rows, K = x.shape
+    codes = np.empty((rows, K), np.uint8)
+    S = np.empty((rows, K // 32), np.uint8)
+    _get().orc_mx8_quantize(_p(x), rows, K, K, _p(codes), _p(S))
+    return codes, S
+
+
+def mx8_dequant(codes: np.ndarray, S: np.ndarray) -> np.ndarray:
+    """Values of MXFP8 codes as float64 [rows, K]."""
+    table = np.array([e4m3_decode_signed(c) for c in range(256)])
+    rows, K = codes.shape
+    scale = np.ldexp(1.0, S.astype(np.int64) - 127)
+    return table[codes] * np.repeat(scale, 32, axis=1).reshape(rows, K)
+
+
+def mx8_gemm(ac, aS, wc, wS):
+    """y = A W^T over MXFP8 operands (block sums exact, added in binary64) -> (y, absdot)."""
+    ac, aS, wc, wS = (_c(v, np.uint8) for v in (ac, aS, wc, wS))
+    rows, K = ac.shape
+    N = wc.shape[0]
+    y = np.empty((rows, N), np.float64)
+    ad = np.empty((rows, N), np.float64)
+    _get().orc_mx8_gemm(_p(ac), _p(aS), _p(wc), _p(wS), rows, N, K, _p(y), _p(ad))
+    return y, ad

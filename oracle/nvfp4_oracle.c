@@ -556,3 +556,76 @@ void orc_combine(const uint16_t* y, int64_t ldy, const int64_t* row_of, const fl
       out[t * H + h] = s;
     }
 }
+
+/* ------------------------------------------------------------------------------------------ */
+/* FP8 comparison format (the pages set their FP4 path against FP8 without fixing an FP8       */
+/* recipe; reading): E4M3 elements with one power-of-two scale 2^X per 32 consecutive elements */
+/* along K (stored as the E8M0 code X + 127), no tensor scale.  X is the smallest integer with */
+/* 448 * 2^X >= b, b = max|x| of the block, clamped to [-127, 127] (b = 0 gives X = -127), so  */
+/* no element saturates.  q = E4M3_RNE_satfinite(RN(x * 2^-X)) with the sign kept; the value  */
+/* of a code pair is val(q) * 2^X.                                                             */
+/* ------------------------------------------------------------------------------------------ */
+int orc_mx8_exponent(float b) {
+  int X = -127;
+  while (X < 127 && ldexp(448.0, X) < (double)b) ++X;
+  return X;
+}
+
+/* signed E4M3: sign bit 0x80 from the sign of v (so -0 gives 0x80), magnitude by orc_e4m3_encode */
+int orc_e4m3_encode_signed(float v) {
+  int c = orc_e4m3_encode(fabsf(v));
+  return signbit(v) ? (c | 0x80) : c;
+}
+
+double orc_e4m3_decode_signed(int code) {
+  double m = orc_e4m3_decode(code & 0x7F);
+  return (code & 0x80) ? -m : m;
+}
+
+/* x: bf16 [rows x K] (pitch ldx), K % 32 == 0 -> codes u8 [rows x K], S (E8M0) u8 [rows x K/32] */
+void orc_mx8_quantize(const uint16_t* x, int64_t rows, int64_t K, int64_t ldx, uint8_t* codes, uint8_t* S) {
+#pragma omp parallel for schedule(static)
+  for (int64_t r = 0; r < rows; ++r)
+    for (int64_t b = 0; b < K / 32; ++b) {
+      float t[32], m = 0.0f;
+      for (int i = 0; i < 32; ++i) {
+        t[i] = orc_bf16_to_f32(x[r * ldx + b * 32 + i]);
+        if (fabsf(t[i]) > m) m = fabsf(t[i]);
+      }
+      const int X = orc_mx8_exponent(m);
+      const float inv = (float)ldexp(1.0, -X); /* exact: 2^-X is a normal binary32 number */
+      S[r * (K / 32) + b] = (uint8_t)(X + 127);
+      for (int i = 0; i < 32; ++i) codes[r * K + b * 32 + i] = (uint8_t)orc_e4m3_encode_signed(t[i] * inv);
+    }
+}
+
+/* y[m, n] = sum over 32-blocks of (sum_i qa_i qw_i) 2^(Xa + Xw): each block's sum is exact in    */
+/* int64 (values times 2^9 are integers below 2^18), scaled by a power of two and added in     */
+/* binary64 in block order.  absdot = sum |a_k w_k| (for the tolerance).  [rows x K] x [N x K]. */
+void orc_mx8_gemm(const uint8_t* ac, const uint8_t* aS, const uint8_t* wc, const uint8_t* wS, int64_t rows,
+                  int64_t N, int64_t K, double* y, double* absdot) {
+  int64_t* qa = (int64_t*)malloc(sizeof(int64_t) * (size_t)(rows * K));
+  int64_t* qw = (int64_t*)malloc(sizeof(int64_t) * (size_t)(N * K));
+  for (int64_t i = 0; i < rows * K; ++i) qa[i] = (int64_t)ldexp(orc_e4m3_decode_signed(ac[i]), 9);
+  for (int64_t i = 0; i < N * K; ++i) qw[i] = (int64_t)ldexp(orc_e4m3_decode_signed(wc[i]), 9);
+#pragma omp parallel for schedule(static)
+  for (int64_t m = 0; m < rows; ++m)
+    for (int64_t n = 0; n < N; ++n) {
+      double s = 0.0, sa = 0.0;
+      for (int64_t b = 0; b < K / 32; ++b) {
+        int64_t acc = 0, aacc = 0;
+        for (int64_t i = b * 32; i < b * 32 + 32; ++i) {
+          const int64_t p = qa[m * K + i] * qw[n * K + i];
+          acc += p;
+          aacc += p < 0 ? -p : p;
+        }
+        const int e = (int)aS[m * (K / 32) + b] + (int)wS[n * (K / 32) + b] - 254 - 18;
+        s += ldexp((double)acc, e);
+        sa += ldexp((double)aacc, e);
+      }
+      y[m * N + n] = s;
+      absdot[m * N + n] = sa;
+    }
+  free(qa);
+  free(qw);
+}
