@@ -10,7 +10,8 @@ over one batch with weights already packed (packing runs once per trainer -> rol
 Other workloads (--workload): dense (8192 x 4096 x 4096 projection), moe_decode (64 tokens,
 hidden 7168, 256 experts, swap-AB decode GEMMs), moe_prefill_layer / moe_decode_layer (the
 same with the device router, dispatch plan and combine: no host work per step), qdq /
-qdq_single (trainer fake-quant of 2^31 weights), sweep (r in {0, 0.25, 0.5, 1}).
+qdq_single (trainer fake-quant of 2^31 weights), sweep (r in {0, 0.25, 0.5, 1}, the masked and per-expert
+variants, and the same block on the FP8 comparison format).
 
 Metric: effective TFLOP/s of the step's GEMMs, 2*rows*N*(K + K') summed over the GEMMs (the
 residual loop counted, as it is part of the method), over the measured step time; GB/s for
@@ -175,6 +176,56 @@ class MoEStep:
         return self.y
 
     KERNELS_PER_STEP = 5  # amax, quantise X, gate_up GEMM, quantise h, down GEMM
+
+
+class Mx8MoEStep:
+    """The same MoE expert block on the FP8 comparison format (E4M3, one power-of-two scale per
+    32 elements; C-ABI calls only): quantise-scatter X, grouped gate_up with SwiGLU, quantise h,
+    grouped down.  No calibration, no residual, no tensor scales."""
+
+    KERNELS_PER_STEP = 4  # quantise X, gate_up GEMM, quantise h, down GEMM
+
+    def __init__(self, wl, dev):
+        import torch
+
+        from nvfp4_w4a4_moe_02_b200 import mxfp8 as F
+        from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+
+        self.F, self.R, self.wl = F, R, wl
+        to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
+        self.status = R.new_status(dev)
+        self.wgu = F.pack_weights(to(wl.wgu), gate_up_interleave=True, status=self.status)
+        self.wdn = F.pack_weights(to(wl.wdn), status=self.status)
+        _, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+        self.pair_rows = pair_rows
+        self.rows_padded = int(off[-1])
+        self.scatter = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0],
+                                                      wl.topk_ids.shape[1])).to(dev)
+        self.offsets = torch.from_numpy(off.astype(np.int32)).to(dev)
+        self.expert_rows = torch.from_numpy(np.asarray(wl.counts, dtype=np.int32)).to(dev)
+        self.x = to(wl.x)
+        # padding rows are never written: the activations and h start zeroed and stay so
+        self.a = F.Mx8Packed.empty(self.rows_padded, wl.H, rows_padded=self.rows_padded, device=dev, zero=True)
+        self.h = torch.zeros(self.rows_padded, wl.I, dtype=torch.bfloat16, device=dev)
+        self.hq = F.Mx8Packed.empty(self.rows_padded, wl.I, device=dev)
+        self.y = torch.empty(self.rows_padded, wl.H, dtype=torch.bfloat16, device=dev)
+        torch.cuda.synchronize()
+        R.check_status(self.status)
+        torch.cuda.empty_cache()
+
+    def run(self, x=None, events=None):
+        F = self.F
+        ev = events or {}
+        if "q0" in ev:
+            ev["q0"].record()
+        F.quantize_scatter(self.x if x is None else x, self.scatter, self.rows_padded, out=self.a, status=self.status)
+        F.grouped_moe(self.a, self.offsets, self.wgu, swiglu=True, y=self.h, status=self.status,
+                      expert_rows=self.expert_rows)
+        F.quantize(self.h, out=self.hq, status=self.status)
+        F.grouped_moe(self.hq, self.offsets, self.wdn, y=self.y, status=self.status, expert_rows=self.expert_rows)
+        if "end" in ev:
+            ev["end"].record()
+        return self.y
 
 
 class DenseStep:
@@ -728,6 +779,10 @@ SPECS = {"moe_prefill": spec_moe, "dense": spec_dense, "moe_decode": spec_decode
          "moe_decode_layer": spec_block_decode}
 
 
+def at_r(rows, r):
+    return next(x for x in rows if x["r"] == r)
+
+
 def run_sweep(args):
     """RAC ratio sweep on the MoE prefill shapes: r in {0, 0.25, 0.5, 1}; per r the step's
     TFLOP/s and the error of h (SwiGLU output) and y (down output) against the binary64 product
@@ -809,6 +864,14 @@ def run_sweep(args):
                       "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12, **e}
     del step
     torch.cuda.empty_cache()
+    # the FP8 comparison format on the same block (E4M3, power-of-two scale per 32 elements)
+    step = Mx8MoEStep(base, dev)
+    ms, e = measure(step)
+    fp8_row = {"variant": "fp8_e4m3_pow2_scale_per_32", "ms_per_step": ms,
+               "tflops": plain_f / (ms * 1e-3) / 1e12, **e, "weight_bytes_per_elem": 1.0 + 1.0 / 32,
+               "nvfp4_rac_r0.5_speedup": ms / at_r(rows, 0.5)["ms_per_step"]}
+    del step
+    torch.cuda.empty_cache()
     mono = all(rows[i + 1]["y_mean_abs"] <= rows[i]["y_mean_abs"] for i in range(len(rows) - 1))
     at = {x["r"]: x for x in rows}
     line = {"metric": METRIC, "value": at[0.5]["tflops"], "unit": "TFLOP/s", "n_gpus": 1, "steps": args.steps,
@@ -821,8 +884,9 @@ def run_sweep(args):
                                           "sampled (token, expert) rows",
                        "l2": "flushed between timed steps (256 MiB write outside the per-step events)"},
             "sweep": rows, "masked_variant": masked_row, "per_expert_variant": per_expert_row,
-            "y_error_non_increasing_in_r": mono, "e2e": None,
-            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * (len(rows) + 2)}
+            "fp8_comparison": fp8_row, "y_error_non_increasing_in_r": mono, "e2e": None,
+            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * (len(rows) + 2) +
+            Mx8MoEStep.KERNELS_PER_STEP * args.steps}
     print(json.dumps(line), flush=True)
     return 0
 

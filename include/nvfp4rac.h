@@ -374,6 +374,54 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_
 nvfp4_status weight_qdq_noalloc(const uint16_t* w, int64_t n_tensors, int64_t elems_per_tensor, uint16_t* w_out,
                                 float* s_g_out, int32_t* dev_status, void* stream);
 
+/* ======================================================================================== */
+/* FP8 comparison path.  The QUADS abstract reports the 4-bit rollouts about 16 % faster than */
+/* FP8 rollouts but fixes no FP8 recipe; this is the block-scaled FP8 the tensor cores take   */
+/* natively, run on the same shapes through the same GEMM kernel, so that the two formats     */
+/* can be timed side by side.                                                                 */
+/*   Format: E4M3 element codes (one byte each, row-major, sign kept), one power-of-two scale */
+/*   2^X per 32 consecutive elements along K stored as the E8M0 code X + 127 in 512-byte     */
+/*   atoms (128 rows x 4 blocks, the FP4 atom order with 32-element blocks); X is the         */
+/*   smallest integer with 448 * 2^X >= max|x| of the block, clamped to [-127, 127], so no    */
+/*   element saturates; q = E4M3_RNE_satfinite(RN(x * 2^-X)).  No tensor scale.              */
+/*   Shape rules: K % 128 == 0, N % 128 == 0, rows_padded % 128 == 0.  A block holding an inf */
+/*   or NaN is written as zero and NVFP4_ERR_RANGE goes to *dev_status.                       */
+/* ======================================================================================== */
+typedef struct mxfp8_tensor {
+  uint8_t* codes;       /* device, slabs * rows_padded * cols bytes, 16-byte aligned */
+  uint8_t* sf;          /* device, slabs * mxfp8_sf_bytes(rows_padded, cols) bytes, 16-byte aligned */
+  int64_t slabs;        /* experts (weights) or 1 */
+  int64_t rows;         /* logical rows per slab */
+  int64_t rows_padded;  /* multiple of 128 */
+  int64_t cols;         /* K */
+} mxfp8_tensor;
+
+size_t mxfp8_codes_bytes(int64_t rows_padded, int64_t cols);
+size_t mxfp8_sf_bytes(int64_t rows_padded, int64_t cols);
+
+/* mxfp8_quantize -- x bf16 [M x K] (pitch ldx, ldx % 8 == 0) -> q (rows >= M_out; rows past   */
+/* M_out are written as zeros).  row_gather as in nvfp4_quantize.                              */
+nvfp4_status mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                            int64_t M_out, const mxfp8_tensor* q, int32_t* dev_status, void* stream);
+/* mxfp8_quantize_scatter -- each x row quantised once and written to its row_scatter[m, :]    */
+/* output rows (fanout <= 32; entries < 0 skipped; rows no entry names are left untouched).    */
+nvfp4_status mxfp8_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
+                                    int32_t fanout, const mxfp8_tensor* q, int32_t* dev_status, void* stream);
+/* mxfp8_pack_weights -- w bf16 [E x N x K] -> w_q (slabs = E, rows = rows_padded = N);        */
+/* gate_up_interleave as pack_weights.                                                         */
+nvfp4_status mxfp8_pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, int32_t gate_up_interleave,
+                                const mxfp8_tensor* w_q, int32_t* dev_status, void* stream);
+/* mxfp8_gemm -- y [M x N] = A W^T over FP8 operands (one tensor-memory accumulator, K = 32    */
+/* per block-scaled MMA); output and pitch rules as w4a4_rac_gemm.                             */
+nvfp4_status mxfp8_gemm(const mxfp8_tensor* a, const mxfp8_tensor* w, int64_t M, int64_t N, int64_t K,
+                        nvfp4_dtype out, void* y, int64_t ldy, int32_t* dev_status, void* stream);
+/* grouped_mxfp8_moe -- grouped_w4a4_rac_moe over FP8 operands (no residual, alpha = 1);       */
+/* amax_out is optional here (the FP8 format needs no tensor scale for h).                     */
+nvfp4_status grouped_mxfp8_moe(const mxfp8_tensor* a, const int32_t* expert_offsets, const int32_t* expert_rows,
+                               int32_t E, const mxfp8_tensor* w, int64_t N, int64_t K, nvfp4_epilogue ep,
+                               nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
+                               void* stream);
+
 /* ---------------------------------------------------------------------------------------- */
 /* test helpers (not part of the hot path)                                                   */
 /* ---------------------------------------------------------------------------------------- */

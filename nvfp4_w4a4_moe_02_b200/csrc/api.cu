@@ -855,6 +855,212 @@ nvfp4_status nvfp4_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status,
   return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "self-test launch");
 }
 
+// ------------------------------------------------------------------------------------------ FP8 comparison path
+size_t mxfp8_codes_bytes(int64_t rows_padded, int64_t cols) { return (size_t)rows_padded * (size_t)cols; }
+size_t mxfp8_sf_bytes(int64_t rows_padded, int64_t cols) { return (size_t)rows_padded * (size_t)(cols / 32); }
+
+}  // extern "C"
+
+namespace {
+nvfp4_status check_mx8(const mxfp8_tensor* t, const char* name, int64_t cols, int64_t min_rows, int64_t slabs) {
+  if (!t) return fail(NVFP4_ERR_INVALID_ARG, "%s is NULL", name);
+  if (!t->codes || !t->sf) return fail(NVFP4_ERR_INVALID_ARG, "%s has a NULL buffer", name);
+  if (t->cols != cols) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.cols = %lld, expected %lld", name, (long long)t->cols, (long long)cols);
+  if (t->slabs != slabs) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s.slabs = %lld, expected %lld", name, (long long)t->slabs, (long long)slabs);
+  if (t->rows_padded % 128 != 0 || t->rows_padded < min_rows || t->rows < 0 || t->rows > t->rows_padded)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "%s rows %lld / rows_padded %lld invalid (need >= %lld, multiple of 128)", name,
+                (long long)t->rows, (long long)t->rows_padded, (long long)min_rows);
+  if (!aligned16(t->codes) || !aligned16(t->sf)) return fail(NVFP4_ERR_ALIGNMENT, "%s buffers must be 16-byte aligned", name);
+  return NVFP4_OK;
+}
+
+nvfp4_status mx8_check_k(int64_t K) {
+  if (K <= 0 || K % 128 != 0 || K > kMaxK)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 128 <= %lld", (long long)K, (long long)kMaxK);
+  return NVFP4_OK;
+}
+
+nvfp4_status mx8_gemm_setup(const mxfp8_tensor* a, const mxfp8_tensor* w, int64_t rows_needed, int64_t N, int64_t K,
+                            int64_t E, nvfp4_dtype out, void* y, int64_t ldy, int64_t y_cols, int64_t y_rows, int bn,
+                            CUtensorMap* maps, GemmArgs* g) {
+  nvfp4_status st = mx8_check_k(K);
+  if (st != NVFP4_OK) return st;
+  if (N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "N must be a positive multiple of 128");
+  if (out != NVFP4_OUT_F32 && out != NVFP4_OUT_BF16) return fail(NVFP4_ERR_INVALID_ARG, "bad output dtype");
+  if (!y) return fail(NVFP4_ERR_INVALID_ARG, "y is NULL");
+  if (!aligned16(y)) return fail(NVFP4_ERR_ALIGNMENT, "y must be 16-byte aligned");
+  if (ldy < y_cols || (out == NVFP4_OUT_BF16 ? ldy % 8 : ldy % 4) != 0)
+    return fail(NVFP4_ERR_ALIGNMENT, "ldy = %lld must be >= %lld and keep rows 16-byte aligned", (long long)ldy, (long long)y_cols);
+  st = check_mx8(a, "a", K, rows_needed, 1);
+  if (st != NVFP4_OK) return st;
+  st = check_mx8(w, "w", K, N, E);
+  if (st != NVFP4_OK) return st;
+  if (w->rows_padded != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w.rows_padded must equal N");
+  memset(maps, 0, 5 * sizeof(CUtensorMap));
+  if (y_rows > 0) {
+    st = make_out_map(&maps[4], y, out == NVFP4_OUT_BF16, (uint64_t)y_cols, (uint64_t)y_rows, (uint64_t)ldy);
+    if (st != NVFP4_OK) return st;
+  }
+  st = make_code_map(&maps[0], a->codes, (uint64_t)K, (uint64_t)a->rows_padded, 1, 128, 2, "A");
+  if (st != NVFP4_OK) return st;
+  st = make_code_map(&maps[2], w->codes, (uint64_t)K, (uint64_t)N, (uint64_t)E, (uint32_t)bn, 3, "W");
+  if (st != NVFP4_OK) return st;
+  maps[1] = maps[0];
+  maps[3] = maps[2];
+  memset(g, 0, sizeof(*g));
+  g->fp8 = 1;
+  g->sfa = a->sf;
+  g->sfa_res = a->sf;
+  g->sfw = w->sf;
+  g->sfw_sel = w->sf;
+  g->sfw_slab_bytes = (int64_t)mxfp8_sf_bytes(N, K);
+  g->k64_main = (int32_t)(K / 64);
+  g->kt_main = (int32_t)(K / 128);
+  g->kt_res = 0;
+  g->N = (int32_t)N;
+  g->n_blocks = (int32_t)(N / bn);
+  g->rows_capacity = a->rows_padded;
+  g->y = y;
+  g->ldy = ldy;
+  g->out_bf16 = out == NVFP4_OUT_BF16;
+  g->wait_limit_ns = g_wait_limit_ns.load();
+  return NVFP4_OK;
+}
+
+nvfp4_status mx8_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                      const int32_t* row_scatter, int32_t fanout, int64_t M_out, const mxfp8_tensor* q,
+                      int32_t* dev_status, void* stream) {
+  if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
+  if (M < 0 || M_out < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "negative row count");
+  nvfp4_status st = mx8_check_k(K);
+  if (st != NVFP4_OK) return st;
+  if (ldx < K || ldx % 8 != 0) return fail(NVFP4_ERR_ALIGNMENT, "ldx = %lld must be >= K and a multiple of 8", (long long)ldx);
+  if (x && !aligned16(x)) return fail(NVFP4_ERR_ALIGNMENT, "x must be 16-byte aligned");
+  st = check_mx8(q, "q", K, row_scatter ? 0 : M_out, 1);
+  if (st != NVFP4_OK) return st;
+  Mx8RowArgs a;
+  memset(&a, 0, sizeof(a));
+  a.src = x;
+  a.src_rows = M;
+  a.ld = ldx;
+  a.K = K;
+  a.row_gather = row_gather;
+  a.row_scatter = row_scatter;
+  a.fanout = fanout;
+  a.rows_out = q->rows_padded;
+  a.rows_per_slab = row_scatter ? M : M_out;
+  a.codes = q->codes;
+  a.sf = q->sf;
+  a.status = dev_status;
+  if ((row_scatter ? M : a.rows_out) == 0) return NVFP4_OK;
+  cudaError_t e = launch_mx8_rows(a, num_sms(), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "fp8 quantize launch");
+}
+}  // namespace
+
+extern "C" {
+
+nvfp4_status mxfp8_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                            int64_t M_out, const mxfp8_tensor* q, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!row_gather && M_out != M) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "without row_gather M_out must equal M");
+  return mx8_rows(x, M, K, ldx, row_gather, nullptr, 1, M_out, q, dev_status, stream);
+}
+
+nvfp4_status mxfp8_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
+                                    int32_t fanout, const mxfp8_tensor* q, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!row_scatter && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "row_scatter is NULL");
+  if (fanout <= 0 || fanout > 32) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "1 <= fanout <= 32 required");
+  return mx8_rows(x, M, K, ldx, nullptr, row_scatter, fanout, 0, q, dev_status, stream);
+}
+
+nvfp4_status mxfp8_pack_weights(const uint16_t* w, int64_t E, int64_t N, int64_t K, int32_t gate_up_interleave,
+                                const mxfp8_tensor* w_q, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!w) return fail(NVFP4_ERR_INVALID_ARG, "w is NULL");
+  if (E <= 0 || N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E > 0 and N %% 128 == 0 required");
+  nvfp4_status st = mx8_check_k(K);
+  if (st != NVFP4_OK) return st;
+  if (gate_up_interleave != 0 && gate_up_interleave != 1) return fail(NVFP4_ERR_INVALID_ARG, "gate_up_interleave must be 0 or 1");
+  if (!aligned16(w)) return fail(NVFP4_ERR_ALIGNMENT, "w must be 16-byte aligned");
+  st = check_mx8(w_q, "w_q", K, N, E);
+  if (st != NVFP4_OK) return st;
+  if (w_q->rows_padded != N || w_q->rows != N) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "w_q rows / rows_padded must equal N");
+  Mx8RowArgs a;
+  memset(&a, 0, sizeof(a));
+  a.src = w;
+  a.src_rows = N;
+  a.ld = K;
+  a.K = K;
+  a.rows_out = E * N;
+  a.rows_per_slab = N;
+  a.src_slab_stride = N * K;
+  a.pack = 1;
+  a.interleave = gate_up_interleave;
+  a.N_half = N / 2;
+  a.codes = w_q->codes;
+  a.sf = w_q->sf;
+  a.status = dev_status;
+  cudaError_t e = launch_mx8_rows(a, num_sms(), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "fp8 pack launch");
+}
+
+nvfp4_status mxfp8_gemm(const mxfp8_tensor* a, const mxfp8_tensor* w, int64_t M, int64_t N, int64_t K,
+                        nvfp4_dtype out, void* y, int64_t ldy, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (M < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M must be >= 0");
+  const int bn = choose_tile_n(N, K, 0);
+  CUtensorMap maps[5];
+  GemmArgs g;
+  nvfp4_status st = mx8_gemm_setup(a, w, M, N, K, 1, out, y, ldy, N, M, bn, maps, &g);
+  if (st != NVFP4_OK) return st;
+  if (M == 0) return NVFP4_OK;
+  g.E = 1;
+  g.M = M;
+  g.m_blocks_dense = (int32_t)((M + 127) / 128);
+  g.status = dev_status;
+  const int64_t tiles = (int64_t)g.m_blocks_dense * g.n_blocks;
+  const int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, grid,
+                              reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "fp8 gemm launch");
+}
+
+nvfp4_status grouped_mxfp8_moe(const mxfp8_tensor* a, const int32_t* expert_offsets, const int32_t* expert_rows,
+                               int32_t E, const mxfp8_tensor* w, int64_t N, int64_t K, nvfp4_epilogue ep,
+                               nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
+                               void* stream) {
+  g_last_error.clear();
+  if (!expert_offsets) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets is NULL");
+  if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
+  if (ep != NVFP4_EPI_NONE && ep != NVFP4_EPI_SWIGLU_AMAX) return fail(NVFP4_ERR_INVALID_ARG, "bad epilogue");
+  if (ep == NVFP4_EPI_SWIGLU_AMAX) {
+    if (out != NVFP4_OUT_BF16) return fail(NVFP4_ERR_INVALID_ARG, "the SwiGLU epilogue writes bf16");
+    if (N % 256 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the SwiGLU epilogue needs N %% 256 == 0");
+  }
+  const int bn = ep == NVFP4_EPI_SWIGLU_AMAX ? 256 : choose_tile_n(N, K, 0);
+  CUtensorMap maps[5];
+  GemmArgs g;
+  const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
+  nvfp4_status st = mx8_gemm_setup(a, w, 0, N, K, E, out, y, ldy, y_cols, a ? a->rows_padded : 0, bn, maps, &g);
+  if (st != NVFP4_OK) return st;
+  g.offsets = expert_offsets;
+  g.expert_rows = expert_rows;
+  g.E = E;
+  g.M = a->rows_padded;
+  g.epi = ep == NVFP4_EPI_SWIGLU_AMAX ? 1 : 0;
+  g.amax_out = amax_out;
+  g.status = dev_status;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (ep == NVFP4_EPI_SWIGLU_AMAX && amax_out) {
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax reset");
+  }
+  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms(), s);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "grouped fp8 gemm launch");
+}
+
 }  // extern "C"
 
 // Helpers for entry points defined in other files of the library.

@@ -69,7 +69,10 @@ struct Cfg {
 };
 
 // ---------------------------------------------------------------------------------------- kernel
-template <int BN>
+// FP8: the comparison operands (E4M3 codes, one E8M0 scale per 32 elements): a 128-byte k-tile
+// holds 128 elements and one scale atom per 128 rows, copied once per k-tile; its four K = 32
+// MMAs pick their scale byte by id.  No residual loop, no tensor scales (alpha = 1).
+template <int BN, bool FP8>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_ar,
                          const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_ws,
@@ -162,21 +165,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           const bool res = kt >= args.kt_main;
           const int kk = res ? kt - args.kt_main : kt;
+          // scale atoms of this k-tile: FP4 one per 64 elements (fewer in a partial last tile),
+          // FP8 one per 128 elements; at_row = atoms per 128-row block of the operand
           const int k64 = res ? args.k64_res : args.k64_main;
-          const int nk64 = min(4, k64 - kk * 4);
-          const uint32_t sf_bytes = (uint32_t)nk64 * 512u;
+          const int n_at = FP8 ? 1 : min(4, k64 - kk * 4);
+          const int64_t at_row = FP8 ? (int64_t)args.kt_main : (int64_t)k64;
+          const int64_t at0 = FP8 ? (int64_t)kk : (int64_t)kk * 4;
+          const uint32_t sf_bytes = (uint32_t)n_at * 512u;
           mbar_expect_tx(bar_full(stage), (uint32_t)(C::A_BYTES + C::B_BYTES) + sf_bytes * (1u + BN / 128));
           tma_load_2d(sbase + C::OFF_A + stage * C::A_BYTES, res ? &tm_ar : &tm_a, kk * KT_BYTES, (int32_t)(mb * BM),
                       bar_full(stage));
           tma_load_3d(sbase + C::OFF_B + stage * C::B_BYTES, res ? &tm_ws : &tm_w, kk * KT_BYTES, nb * BN, e,
                       bar_full(stage));
-          const uint8_t* sfa = (res ? args.sfa_res : args.sfa) + (mb * k64 + kk * 4) * 512;
+          const uint8_t* sfa = (res ? args.sfa_res : args.sfa) + (mb * at_row + at0) * 512;
           bulk_load(sbase + C::OFF_SFA + stage * C::SFA_BYTES, sfa, sf_bytes, bar_full(stage));
           const uint8_t* sfw = res ? args.sfw_sel + (int64_t)e * args.sfw_sel_slab_bytes
                                    : args.sfw + (int64_t)e * args.sfw_slab_bytes;
 #pragma unroll
           for (int rb = 0; rb < BN / 128; ++rb) {
-            const uint8_t* src = sfw + ((int64_t)(nb * (BN / 128) + rb) * k64 + kk * 4) * 512;
+            const uint8_t* src = sfw + ((int64_t)(nb * (BN / 128) + rb) * at_row + at0) * 512;
             bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES + rb * 2048, src, sf_bytes, bar_full(stage));
           }
           ++issued;
@@ -191,7 +198,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // ===================================================================== MMA issuer
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_fp4(BM, BN);
+      constexpr uint32_t idesc = FP8 ? idesc_fp8(BM, BN) : idesc_fp4(BM, BN);
       int stage = 0;
       uint32_t phase = 0;
       int taken = 0;
@@ -230,9 +237,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b_s = sbase + C::OFF_B + stage * C::B_BYTES;
           const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_BYTES;
           const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_BYTES;
-          // each MMA's scale atoms are copied right before it (into alternating slots): the
+          if constexpr (FP8) {
+            // one scale atom per operand block covers the whole k-tile: copy once, then the
+            // four K = 32 MMAs take scale byte j of each row
+            const uint32_t sfa_t = tmem_base + (uint32_t)(C::SF_BASE + (mma_count & 1) * C::SF_SLOT);
+            const uint32_t sfb_t = sfa_t + 4;
+            ++mma_count;
+            tc_copy_sf(sfa_t, desc_sf(sfa_s));
+#pragma unroll
+            for (int rb = 0; rb < BN / 128; ++rb) tc_copy_sf(sfb_t + 4 * rb, desc_sf(sfb_s + rb * 2048));
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tc_mma_fp8(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j),
+                         idesc | idesc_sf_ids((uint32_t)j, (uint32_t)j), sfa_t, sfb_t, (kt | j) != 0 ? 1u : 0u);
+          }
+          // FP4: each MMA's scale atoms are copied right before it (into alternating slots): the
           // tensor pipe overlaps the copies with the preceding MMA
-          for (int j = 0; j < nk64; ++j, ++mma_count) {
+          for (int j = 0; j < (FP8 ? 0 : nk64); ++j, ++mma_count) {
             const uint32_t sfa_t = tmem_base + (uint32_t)(C::SF_BASE + (mma_count & 1) * C::SF_SLOT);
             const uint32_t sfb_t = sfa_t + 4;
             tc_copy_sf(sfa_t, desc_sf(sfa_s + j * 512));
@@ -289,7 +310,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                  ? (int64_t)__ldg(args.offsets + e) + __ldg(args.expert_rows + e)
                                  : row_limit;
       const bool row_ok = row < row_limit && row < args.rows_capacity && row < rows_e;
-      const float alpha = __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));
+      const float alpha = FP8 ? 1.0f : __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));
       const uint32_t t_row = tmem_base + (uint32_t)(acc ? C::ACC1_BASE : 0) + ((uint32_t)(quad * 32) << 16);
       // chunk i of this warp: plain -> columns half*BN/2 + 32i; SwiGLU -> output features
       // [half*BN/4, ...): chunks 0..NCH/2-1 gate (column (f/64)*128 + f%64), NCH/2.. the up
@@ -435,24 +456,28 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, int32_t* status) {
 
 size_t gemm_smem_bytes(int bn) { return bn == 256 ? (size_t)tc::Cfg<256>::SMEM : (size_t)tc::Cfg<128>::SMEM; }
 
+template <int BN, bool FP8>
+static cudaError_t launch_gemm_t(const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
+                                 const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
+                                 cudaStream_t st) {
+  cudaError_t e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<BN, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       tc::Cfg<BN>::SMEM);
+  if (e != cudaSuccess) return e;
+  tc::w4a4_rac_gemm_kernel<BN, FP8><<<grid, tc::NUM_THREADS, tc::Cfg<BN>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y,
+                                                                                     args);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
                         const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
                         cudaStream_t st) {
-  cudaError_t e;
-  if (bn == 256) {
-    e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::Cfg<256>::SMEM);
-    if (e != cudaSuccess) return e;
-    tc::w4a4_rac_gemm_kernel<256><<<grid, tc::NUM_THREADS, tc::Cfg<256>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args);
-  } else if (bn == 128) {
-    e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             tc::Cfg<128>::SMEM);
-    if (e != cudaSuccess) return e;
-    tc::w4a4_rac_gemm_kernel<128><<<grid, tc::NUM_THREADS, tc::Cfg<128>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args);
-  } else {
-    return cudaErrorInvalidValue;
-  }
-  return cudaGetLastError();
+  if (bn == 256)
+    return args.fp8 ? launch_gemm_t<256, true>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args, grid, st)
+                    : launch_gemm_t<256, false>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args, grid, st);
+  if (bn == 128)
+    return args.fp8 ? launch_gemm_t<128, true>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args, grid, st)
+                    : launch_gemm_t<128, false>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args, grid, st);
+  return cudaErrorInvalidValue;
 }
 
 cudaError_t launch_wait_selftest(uint64_t limit_ns, int32_t* status, cudaStream_t st) {

@@ -60,6 +60,27 @@ cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint
 cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
 cudaError_t launch_encode_e4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
 
+// ---- FP8 comparison format: E4M3 codes, one E8M0 scale per 32 elements (atoms of 128 x 128)
+struct Mx8RowArgs {
+  const uint16_t* src;           // bf16 rows
+  int64_t src_rows;              // valid source rows (act: M; pack: N per slab)
+  int64_t ld;                    // source pitch (elements)
+  int64_t K;                     // channels, K % 128 == 0
+  const int32_t* row_gather;     // act: optional output-row -> source-row map
+  const int32_t* row_scatter;    // act: optional source-row -> fanout output rows (-1 = none)
+  int fanout;                    // <= 32
+  int64_t rows_out;              // output rows (act: rows_padded; pack: slabs * N)
+  int64_t rows_per_slab;         // pack: N; act: M_out
+  int64_t src_slab_stride;       // pack: N*K elements between slabs
+  int pack;                      // weight pack (slabs, optional gate/up interleave)
+  int interleave;
+  int64_t N_half;
+  uint8_t* codes;                // [rows_out x K]
+  uint8_t* sf;                   // atoms, K/128 per 128-row block
+  int32_t* status;
+};
+cudaError_t launch_mx8_rows(const Mx8RowArgs& a, int num_sms, cudaStream_t st);
+
 // ---- tcgen05 block-scaled GEMM (dense and grouped)
 struct GemmArgs {
   const uint8_t* sfa;        // A scale atoms, rows_padded/128 x k64_main
@@ -87,6 +108,7 @@ struct GemmArgs {
   float* amax_out;
   int32_t* status;
   uint64_t wait_limit_ns;
+  int32_t fp8;               // 1: the FP8 comparison operands (E4M3, E8M0 per 32; kt_main = K/128, no residual)
 };
 
 // bn: 128 or 256

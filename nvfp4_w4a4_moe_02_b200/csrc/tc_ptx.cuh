@@ -102,6 +102,19 @@ __device__ __forceinline__ void tc_mma_fp4(uint32_t d, uint64_t adesc, uint64_t 
       : "memory");
 }
 
+// FP8 comparison operands: kind::mxf8f6f4 with one E8M0 scale per 32 elements (K = 32 per
+// instruction); the scale byte of each row is picked from its 32-bit tensor-memory word by the
+// scale-factor ids of the instruction descriptor.
+__device__ __forceinline__ void tc_mma_fp8(uint32_t d, uint64_t adesc, uint64_t bdesc, uint32_t idesc, uint32_t sfa,
+                                           uint32_t sfb, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale.scale_vec::1X [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
 // 32 lanes x 32 columns of 32-bit accumulator -> 32 registers per thread
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -138,6 +151,12 @@ __device__ __forceinline__ uint64_t desc_sf(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t idesc_fp4(int M, int N) {
   return (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Instruction descriptor of kind::mxf8f6f4: E4M3 A and B (format 0), E8M0 scales (bit 23),
+// K-major, M x N; the scale byte ids of A (bits 29-30) and B (bits 4-5) are or-ed in per MMA.
+__host__ __device__ constexpr uint32_t idesc_fp8(int M, int N) {
+  return (1u << 23) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_sf_ids(uint32_t a_id, uint32_t b_id) { return (a_id << 29) | (b_id << 4); }
 
 __device__ __forceinline__ int find_expert(const int32_t* off, int E, int64_t row) {
   int lo = 0, hi = E - 1;

@@ -160,6 +160,29 @@ def test_grouped_sel_rejections(lib):
     assert lib.moe_row_groups(None, 4, 8, 16, None) == 1
 
 
+def test_fp8_path_rejections(lib):
+    """The FP8 comparison entry points check shapes on the host, before any device work."""
+    from nvfp4_w4a4_moe_02_b200.mxfp8 import CMx8Tensor, load
+
+    load()
+    assert lib.mxfp8_codes_bytes(128, 256) == 128 * 256 and lib.mxfp8_sf_bytes(128, 256) == 128 * 8
+    q = CMx8Tensor(16, 16, 1, 64, 128, 192)
+    # K must be a multiple of 128
+    assert lib.mxfp8_quantize(16, 64, 192, 192, None, 64, ctypes.byref(q), None, None) == 2
+    q.cols = 256
+    assert lib.mxfp8_quantize(16, 64, 256, 256, None, 32, ctypes.byref(q), None, None) == 2  # M_out != M
+    assert lib.mxfp8_quantize_scatter(16, 64, 256, 256, 16, 33, ctypes.byref(q), None, None) == 2  # fanout > 32
+    assert lib.mxfp8_quantize(24, 64, 256, 256, None, 64, ctypes.byref(q), None, None) == 3  # misaligned x
+    w = CMx8Tensor(16, 16, 2, 96, 96, 256)
+    assert lib.mxfp8_pack_weights(16, 2, 96, 256, 0, ctypes.byref(w), None, None) == 2  # N % 128
+    a = CMx8Tensor(16, 16, 1, 128, 128, 256)
+    w1 = CMx8Tensor(16, 16, 1, 128, 128, 256)
+    # SwiGLU writes bf16 only; N % 128
+    assert lib.grouped_mxfp8_moe(ctypes.byref(a), 16, None, 1, ctypes.byref(w1), 128, 256, 1, 0, 16, 64, None, None,
+                                 None) == 1
+    assert lib.mxfp8_gemm(ctypes.byref(a), ctypes.byref(w1), 128, 96, 256, 0, 16, 96, None, None) == 2
+
+
 def test_decode_slots_host_logic():
     from nvfp4_w4a4_moe_02_b200.nvfp4rac import decode_slots
 
