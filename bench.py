@@ -219,9 +219,15 @@ class Mx8MoEStep:
         if "q0" in ev:
             ev["q0"].record()
         F.quantize_scatter(self.x if x is None else x, self.scatter, self.rows_padded, out=self.a, status=self.status)
+        if "g0" in ev:
+            ev["g0"].record()
         F.grouped_moe(self.a, self.offsets, self.wgu, swiglu=True, y=self.h, status=self.status,
                       expert_rows=self.expert_rows)
+        if "q1" in ev:
+            ev["q1"].record()
         F.quantize(self.h, out=self.hq, status=self.status)
+        if "d0" in ev:
+            ev["d0"].record()
         F.grouped_moe(self.hq, self.offsets, self.wdn, y=self.y, status=self.status, expert_rows=self.expert_rows)
         if "end" in ev:
             ev["end"].record()
@@ -820,17 +826,20 @@ def run_sweep(args):
         for _ in range(max(3, args.warmup)):
             flush.zero_()
             step.run()
-        evs = [{n: torch.cuda.Event(enable_timing=True) for n in ("q0", "end")} for _ in range(args.steps)]
+        evs = [{n: torch.cuda.Event(enable_timing=True) for n in ("q0", "g0", "q1", "d0", "end")}
+               for _ in range(args.steps)]
         for i in range(args.steps):
             flush.zero_()
             step.run(events=evs[i])
         torch.cuda.synchronize()
         R.check_status(step.status)
         ms = float(np.mean([e["q0"].elapsed_time(e["end"]) for e in evs]))
+        seg = {"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")}
+        kernel_ms = {k: float(np.mean([e[a].elapsed_time(e[b]) for e in evs])) for k, (a, b) in seg.items()}
         prow = torch.from_numpy(step.pair_rows[sample]).to(dev)
         (hf, hm), (yf, ym) = err(step.h[prow].double().cpu().numpy(), h_ref), err(step.y[prow].double().cpu().numpy(),
                                                                                   y_ref)
-        return ms, {"h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym}
+        return ms, {"h_rel_fro": hf, "h_mean_abs": hm, "y_rel_fro": yf, "y_mean_abs": ym, "kernel_ms": kernel_ms}
 
     rows = []
     for r in (0.0, 0.25, 0.5, 1.0):
