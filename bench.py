@@ -630,6 +630,56 @@ def spec_moe(dev, args, peaks):
         cpu=cpu_leg, kernels_per_step=MoEStep.KERNELS_PER_STEP)
 
 
+def oracle_sample_fp8(wl, n_pairs, seed=0):
+    """The oracle on a bounded sample of the FP8 comparison step: n_pairs (token, expert) rows
+    through FP8 quantise, gate_up, SwiGLU, FP8 quantise, down.  Returns (seconds, flops)."""
+    import oracle as orc
+
+    rng = np.random.default_rng(seed)
+    pairs = np.sort(rng.choice(wl.pair_token.size, n_pairs, replace=False))
+    t0 = time.perf_counter()
+    for e in np.unique(wl.pair_expert[pairs]):
+        idx = pairs[wl.pair_expert[pairs] == e]
+        ac, aS = orc.mx8_quantize(wl.x[wl.pair_token[idx]])
+        wc, wS = orc.mx8_quantize(wl.gate_up_expert(int(e)))
+        gu, _ = orc.mx8_gemm(ac, aS, wc, wS)
+        h, _ = orc.swiglu(orc.f64_to_bf16_array(gu))
+        hc, hS = orc.mx8_quantize(h)
+        dc, dS = orc.mx8_quantize(wl.down_expert(int(e)))
+        orc.mx8_gemm(hc, hS, dc, dS)
+    dt = time.perf_counter() - t0
+    return dt, sum(flops_of(wl, 0, 0)) * n_pairs / wl.pair_token.size
+
+
+def spec_fp8_moe(dev, args, peaks):
+    """The MoE prefill block on the FP8 comparison format (E4M3, power-of-two scale per 32)."""
+    wl, _ = build_inputs(experts=args.experts)
+    step = Mx8MoEStep(wl, dev)
+    gu_f, dn_f = flops_of(wl, 0, 0)
+    P = int(wl.pair_token.size)
+    b8 = 1.0 + 1.0 / 32  # bytes per FP8 element with its scale
+    gu_bytes = wl.E * 2 * wl.I * wl.H * b8 + P * wl.H * b8 + P * wl.I * 2.0
+
+    def cpu_leg():
+        import oracle as orc
+
+        orc.build()
+        dt, f = oracle_sample_fp8(wl, args.cpu_pairs)
+        return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
+                "sample": f"{args.cpu_pairs} of {P} (token, expert) rows of one step, {dt:.1f} s"}
+
+    return dict(
+        step=step, x_np=wl.x, flops=gu_f + dn_f, events=["q0", "g0", "q1", "d0", "end"],
+        segments={"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")},
+        dominant=("gate_up", gu_f, gu_bytes, "grouped gate_up FP8 GEMM (SwiGLU epilogue)"),
+        traffic=None,
+        quant={"x": ("quant_x", int(wl.x.nbytes) + P * b8 * wl.H), "h": ("quant_h", P * (2.0 + b8) * wl.I)},
+        config={"workload": wl.name.replace(f"_r{wl.r}", "") + "_fp8_e4m3_pow2_per32", "tokens": int(wl.x.shape[0]),
+                "pairs": P, "experts": wl.E, "hidden": wl.H, "intermediate": wl.I, "rows_padded": step.rows_padded},
+        cpu=cpu_leg, kernels_per_step=Mx8MoEStep.KERNELS_PER_STEP,
+        dtype="fp8 (e4m3 x e4m3, e8m0 power-of-two scale per 32) -> f32 accumulate")
+
+
 def spec_dense(dev, args, peaks):
     from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 
@@ -780,7 +830,8 @@ def spec_qdq_single(dev, args, peaks):
     return _spec_qdq(dev, args, 1)
 
 
-SPECS = {"moe_prefill": spec_moe, "dense": spec_dense, "moe_decode": spec_decode, "qdq": spec_qdq,
+SPECS = {"moe_prefill": spec_moe, "fp8_moe_prefill": spec_fp8_moe, "dense": spec_dense, "moe_decode": spec_decode,
+         "qdq": spec_qdq,
          "qdq_single": spec_qdq_single, "moe_prefill_layer": spec_block_prefill,
          "moe_decode_layer": spec_block_decode}
 
