@@ -338,8 +338,7 @@ class DecodeStep:
                                       swiglu=True, y=self.h, amax_out=self.amax_h, status=self.status)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status,
-                         row_group=self.row_group)
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
         if "d0" in ev:
             ev["d0"].record()
         R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.slot_expert, self.slot_count, self.pdn, self.pdns,
@@ -418,8 +417,7 @@ class MoEBlockStep:
                                    amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status,
-                         row_group=self.row_group)
+        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
         if "d0" in ev:
             ev["d0"].record()
         if self.decode:
