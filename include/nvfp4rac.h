@@ -367,6 +367,9 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_
 /*   tensors per call; larger calls return NVFP4_ERR_UNSUPPORTED_SHAPE with a message.        */
 /*   The first call on a device looks up the scratch array's device address (once per        */
 /*   device, with that device current); make that first call before any stream capture.      */
+/*   The looked-up address is kept for the life of the process and is not refreshed: after   */
+/*   cudaDeviceReset (or any other teardown of the device's primary context) it is stale, so  */
+/*   do not call this entry point on that device again in the same process.                   */
 /*   All calls share the one array, so calls that overlap on the GPU (different streams, or  */
 /*   different host threads) race and may corrupt each other's scales: serialise them.        */
 /*   Allocates nothing: no cudaMalloc, no cudaFree, no allocating library routine.            */

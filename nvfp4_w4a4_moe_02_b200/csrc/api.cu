@@ -1066,6 +1066,7 @@ nvfp4_status grouped_mxfp8_moe(const mxfp8_tensor* a, const int32_t* expert_offs
 // Helpers for entry points defined in other files of the library.
 namespace nvfp4 {
 nvfp4_status record_host_error(nvfp4_status s, const char* msg) { return fail(s, "%s", msg); }
+void clear_host_error() { g_last_error.clear(); }
 int qdq_partial_count(int64_t n_tensors) { return slab_partials(n_tensors); }
 int device_sm_count() { return num_sms(); }
 }  // namespace nvfp4

@@ -13,6 +13,7 @@
 
 namespace nvfp4 {
 nvfp4_status record_host_error(nvfp4_status s, const char* msg);
+void clear_host_error();
 int qdq_partial_count(int64_t n_tensors);
 int device_sm_count();
 }  // namespace nvfp4
@@ -30,6 +31,8 @@ float* g_scratch_addr[kMaxDevices] = {nullptr};
 
 // Device address of the scratch array on the current device, looked up once per device.  In
 // host code the array's name only stands in for the symbol; the kernels need this address.
+// The cached address belongs to the device's primary context: after cudaDeviceReset (or any
+// teardown of that context) it is stale, and a later call would launch on a dangling pointer.
 nvfp4_status scratch_on_current_device(float** out) {
   int dev = -1;
   cudaError_t e = cudaGetDevice(&dev);
@@ -58,6 +61,7 @@ nvfp4_status scratch_on_current_device(float** out) {
 
 extern "C" nvfp4_status weight_qdq_noalloc(const uint16_t* w, int64_t n_tensors, int64_t elems_per_tensor,
                                            uint16_t* w_out, float* s_g_out, int32_t* dev_status, void* stream) {
+  nvfp4::clear_host_error();
   if (!w || !w_out) return nvfp4::record_host_error(NVFP4_ERR_INVALID_ARG, "w / w_out is NULL");
   if (n_tensors <= 0 || elems_per_tensor <= 0 || elems_per_tensor % 16 != 0)
     return nvfp4::record_host_error(NVFP4_ERR_UNSUPPORTED_SHAPE,

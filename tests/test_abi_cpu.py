@@ -90,6 +90,30 @@ def test_host_side_rejections(lib):
     assert lib.nvfp4_selftest_wait_timeout(1000, None, None) == 1
 
 
+def test_noalloc_host_side_rejections(lib):
+    """weight_qdq_noalloc checks its arguments and its scratch limit on the host, before any CUDA
+    call, and a good call after a rejected one leaves no stale error text."""
+    fn = lib.weight_qdq_noalloc
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    fn.argtypes = [vp, i64, i64, vp, vp, vp, vp]
+    fn.restype = ctypes.c_int
+    # NULL input or output
+    assert fn(None, 1, 16, 16, None, None, None) == 1
+    assert fn(16, 1, 16, None, None, None, None) == 1
+    # elements per tensor not a multiple of 16, no tensors
+    assert fn(16, 1, 24, 16, None, None, None) == 2
+    assert fn(16, 0, 16, 16, None, None, None) == 2
+    # misaligned input
+    assert fn(18, 1, 16, 16, None, None, None) == 3
+    # the fixed scratch holds one amax partial per tensor from 512 tensors on: 4097 is too many
+    assert fn(16, 4097, 16, 16, None, None, None) == 2
+    assert b"4096" in lib.nvfp4_last_error_string()
+    # a later call does not keep that text: without a GPU it stops at the device lookup and
+    # reports that instead
+    assert fn(16, 4096, 16, 16, None, None, None) == 5
+    assert b"4096" not in lib.nvfp4_last_error_string()
+
+
 def test_decode_and_layout_rejections(lib):
     from nvfp4_w4a4_moe_02_b200.nvfp4rac import SF_SLAB16, CTensor
 

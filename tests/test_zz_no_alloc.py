@@ -56,12 +56,26 @@ def test_weight_qdq_noalloc_rejects_oversize():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+    from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 
     lib = R.load()
     fn = _noalloc_fn(lib)
     dev = torch.device("cuda:0")
     w = torch.zeros(4097, 16, dtype=torch.bfloat16, device=dev)
     out = torch.empty_like(w)
-    rc = fn(w.data_ptr(), 4097, 16, out.data_ptr(), None, None, torch.cuda.current_stream().cuda_stream)
+    stream = torch.cuda.current_stream().cuda_stream
+    rc = fn(w.data_ptr(), 4097, 16, out.data_ptr(), None, None, stream)
     assert rc == 2
     assert b"4096" in lib.nvfp4_last_error_string()
+    # the largest accepted call (4096 tensors) right after the rejected one: it succeeds, leaves
+    # no stale error text, and matches weight_qdq
+    w = torch.from_numpy(syn.normal_bf16(3, 9, 4096, 16, 0.02).view(np.int16)).to(dev).view(torch.bfloat16)
+    ref, s_ref = R.weight_qdq(w)
+    out = torch.empty_like(w)
+    s_g = torch.empty(4096, dtype=torch.float32, device=dev)
+    st = R.new_status(dev)
+    rc = fn(w.data_ptr(), 4096, 16, out.data_ptr(), s_g.data_ptr(), st.data_ptr(), stream)
+    assert rc == 0 and lib.nvfp4_last_error_string() == b""
+    torch.cuda.synchronize()
+    assert int(st.item()) == 0
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16)) and torch.equal(s_g, s_ref)
