@@ -367,6 +367,57 @@ def test_compensation_never_increases_error_on_calibration_data(orc):
     assert all(b <= a for a, b in zip(errs, errs[1:])), errs  # monotone in r on this batch
 
 
+@pytest.mark.slow
+def test_compensation_never_increases_error_on_moe_prefill_calibration_data(orc):
+    """The MoE prefill block (4096 tokens, hidden 2048, 128 experts, top-8, intermediate 768) on its
+    own calibration data: mean |Y - Y_bf16| over r in {0, 0.25, 0.5, 1} never rises (r = 0 is
+    plain W4A4).  Y is the whole block through the oracle: quantise X (+ residual), gate_up,
+    SwiGLU, quantise h (+ residual), down; Y_bf16 the binary64 product of the bf16 inputs.  The
+    rows are every calibration pair of six experts; the channel lists are calibrated on the whole
+    calibration batch (gate_up on X_cal, down on the pooled h_cal) as the rollout does."""
+    wl = syn.moe_prefill()
+    h_cal = syn.moe_down_calibration_batch(wl)
+    off = syn.moe_down_calibration_offsets(wl)
+    T = wl.x_cal.shape[0]
+    topk = syn.route_topk(wl.seed, T, wl.E, wl.topk_ids.shape[1], stream=syn.STREAM_ROUTER_CAL)
+    pt, pe, _ = syn.sort_pairs(topk, wl.E)
+    experts = [0, 17, 42, 64, 101, 127]
+    f64 = lambda a: syn.bf16_to_f32(a).astype(np.float64)
+    xf = f64(wl.x_cal)
+    s_x = orc.global_scale(orc.amax_bf16(wl.x_cal))
+    rows = {e: pt[off[e]:off[e + 1]] for e in experts}
+    y_ref = {}
+    for e in experts:
+        gu = xf[rows[e]] @ f64(wl.gate_up_expert(e)).T
+        h = gu[:, :wl.I] / (1.0 + np.exp(-gu[:, :wl.I])) * gu[:, wl.I:]
+        y_ref[e] = h @ f64(wl.down_expert(e)).T
+    errs = []
+    for r in (0.0, 0.25, 0.5, 1.0):
+        Kp_gu, Kp_dn = syn.kp_from_ratio(wl.H, r), syn.kp_from_ratio(wl.I, r)
+        sel_gu = orc.calibrate(wl.x_cal, Kp_gu)[0] if Kp_gu else np.zeros(0, np.int32)
+        sel_dn = orc.calibrate(h_cal, Kp_dn)[0] if Kp_dn else np.zeros(0, np.int32)
+        hs = {}
+        for e in experts:
+            ac, aS, rc, rS, _ = orc.act_quant_rac(wl.x_cal[rows[e]], s_x, sel_gu)
+            wgu = wl.gate_up_expert(e)
+            s_w = orc.global_scale(orc.amax_bf16(wgu))
+            gu, _ = orc.gemm_rac(ac, aS, rc, rS, *orc.weight_pack(wgu, s_w, sel_gu), s_x, s_w)
+            hs[e] = orc.swiglu(orc.f64_to_bf16_array(gu))[0]
+        s_h = orc.global_scale(orc.amax_bf16(np.concatenate([hs[e] for e in experts])))
+        tot, n = 0.0, 0
+        for e in experts:
+            hc, hS, hrc, hrS, _ = orc.act_quant_rac(hs[e], s_h, sel_dn)
+            wdn = wl.down_expert(e)
+            s_w = orc.global_scale(orc.amax_bf16(wdn))
+            y, _ = orc.gemm_rac(hc, hS, hrc, hrS, *orc.weight_pack(wdn, s_w, sel_dn), s_h, s_w)
+            tot += float(np.abs(y - y_ref[e]).sum())
+            n += y.size
+        errs.append(tot / n)
+    print('mean |Y - Y_bf16| at r = 0, 0.25, 0.5, 1:', errs)
+    assert all(e <= errs[0] for e in errs[1:]), errs
+    assert all(b <= a for a, b in zip(errs, errs[1:])), errs
+
+
 def test_compensation_shrinks_activation_error(orc):
     """Against X_bf16 @ DQ(Q(W))^T (weight error removed), the residual pass over all channels
     removes most of the activation quantisation error."""
