@@ -96,6 +96,34 @@ def quant_bytes(rows, K, Kp):
     return rows * (2.0 * K + 0.5625 * (K + Kp))
 
 
+def device_layout(R, wl, dev, pad, status, decode=False):
+    """The workload's expert-grouped layout made on the device by moe_dispatch_plan (segments padded
+    to `pad` rows; 16-row slot tables for decode).  Returns a dict of device tensors and, for the
+    error sampling and the configuration record, the host copies it needs."""
+    import torch
+
+    T, k = wl.topk_ids.shape
+    ids = torch.from_numpy(np.ascontiguousarray(wl.topk_ids, dtype=np.int32)).to(dev)
+    cap = R.moe_rows_capacity(T, k, wl.E, pad)
+    n_slots = cap // 16 if decode else None
+    off, rs, se, sc = R.moe_dispatch_plan(ids, wl.E, pad, rows_capacity=cap, n_slots=n_slots, status=status,
+                                          expert_rows=(er := torch.empty(wl.E, dtype=torch.int32, device=dev)))
+    torch.cuda.synchronize()
+    R.check_status(status)
+    rows_scatter = rs.cpu().numpy()
+    # the row of every (expert, token)-sorted pair, for sampling rows of the outputs
+    e_flat = wl.topk_ids.reshape(-1)
+    t_flat = np.repeat(np.arange(T), k)
+    order = np.lexsort((t_flat, e_flat))
+    assert np.array_equal(t_flat[order], wl.pair_token) and np.array_equal(e_flat[order], wl.pair_expert)
+    out = dict(offsets=off, row_scatter=rs, expert_rows=er, cap=cap, rows_used=int(off[-1].item()),
+               pair_rows=rows_scatter.reshape(-1)[order].astype(np.int64))
+    if decode:
+        out.update(slot_expert=se, slot_count=sc, n_slots=n_slots, slots_used=int((sc > 0).sum().item()),
+                   slot_first_row=torch.arange(n_slots, dtype=torch.int32, device=dev) * 16)
+    return out
+
+
 class MoEStep:
     """Device-resident state of one replica and the step itself (C-ABI calls only)."""
 
@@ -125,28 +153,30 @@ class MoEStep:
             self.pgu, self.pgus = R.pack_weights(to(wl.wgu), self.sel_gu, gate_up_interleave=True,
                                                  status=self.status)
             self.pdn, self.pdns = R.pack_weights(to(wl.wdn), self.sel_dn, status=self.status)
-        g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
-        self.pair_rows = pair_rows
-        self.rows_padded = int(off[-1])
-        self.scatter = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0],
-                                                      wl.topk_ids.shape[1])).to(dev)
-        self.offsets = torch.from_numpy(off.astype(np.int32)).to(dev)
-        self.expert_rows = torch.from_numpy(np.asarray(wl.counts, dtype=np.int32)).to(dev)
-        # per-expert lists: each expert-sorted row of h takes its expert's list (routing is fixed
-        # for the step, like the offsets)
-        self.row_group = R.moe_row_groups(self.offsets, wl.E, self.rows_padded) if h_cal_offsets is not None else None
+        # expert-grouped layout of the routed pairs, made on the device (routing is fixed for the
+        # run, so the plan is made once; the *_layer workloads make it every step)
+        lay = device_layout(R, wl, dev, 128, self.status)
+        self.pair_rows = lay["pair_rows"]
+        self.rows_padded = lay["rows_used"]
+        self.scatter, self.offsets, self.expert_rows = lay["row_scatter"], lay["offsets"], lay["expert_rows"]
+        cap = lay["cap"]
+        # per-expert lists: each expert-sorted row of h takes its expert's list
+        self.row_group = R.moe_row_groups(self.offsets, wl.E, cap) if h_cal_offsets is not None else None
         self.x = to(wl.x)
-        # preallocated outputs (the step allocates nothing)
+        # preallocated outputs (the step allocates nothing), sized for the worst-case layout;
+        # padding rows of the expert-grouped activations are never written: zero them once
         P = R.Packed
-        # padding rows of the expert-sorted activations are never written: zero them once
-        self.a = P.empty(self.rows_padded, wl.H, rows_padded=self.rows_padded, device=dev, zero=True)
-        self.ar = P.empty(self.rows_padded, wl.H if masked else wl.Kp_gu, rows_padded=self.rows_padded, device=dev,
-                          zero=True)
-        self.h = torch.empty(self.rows_padded, wl.I, dtype=torch.bfloat16, device=dev)
+        self.a = P.empty(cap, wl.H, rows_padded=cap, device=dev, zero=True)
+        self.ar = P.empty(cap, wl.H if masked else wl.Kp_gu, rows_padded=cap, device=dev, zero=True)
+        self.h = torch.zeros(cap, wl.I, dtype=torch.bfloat16, device=dev)
         self.amax_h = torch.zeros(1, dtype=torch.float32, device=dev)
-        self.hq = P.empty(self.rows_padded, wl.I, device=dev)
-        self.hqr = P.empty(self.rows_padded, wl.I if masked else wl.Kp_dn, rows_padded=self.hq.rows_padded, device=dev)
-        self.y = torch.empty(self.rows_padded, wl.H, dtype=torch.bfloat16, device=dev)
+        self.hq = P.empty(cap, wl.I, rows_padded=cap, device=dev, zero=True)
+        self.hqr = P.empty(cap, wl.I if masked else wl.Kp_dn, rows_padded=cap, device=dev, zero=True)
+        self.y = torch.empty(cap, wl.H, dtype=torch.bfloat16, device=dev)
+        # the variants quantise h with the row quantiser over the used rows (views of the same storage)
+        self.h_used = self.h[:self.rows_padded]
+        self.hq_used, self.hqr_used = self.hq.prefix(self.rows_padded), self.hqr.prefix(self.rows_padded)
+        self.row_group_used = self.row_group[:self.rows_padded] if self.row_group is not None else None
         torch.cuda.synchronize()
         R.check_status(self.status)
         torch.cuda.empty_cache()  # drop the bf16 weight staging buffers
@@ -165,8 +195,13 @@ class MoEStep:
                                amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status,
-                         row_group=self.row_group)
+        if self.masked or self.row_group is not None:
+            R.nvfp4_quantize(self.h_used, self.sel_dn, amax_in=self.amax_h, out=self.hq_used, out_res=self.hqr_used,
+                             status=self.status, masked=self.masked, row_group=self.row_group_used)
+        else:
+            # the token rows of each expert segment only
+            R.nvfp4_quantize_segments(self.h, self.offsets, self.expert_rows, self.sel_dn, amax_in=self.amax_h,
+                                      out=self.hq, out_res=self.hqr, status=self.status)
         if "d0" in ev:
             ev["d0"].record()
         R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.offsets, self.pdn, self.pdns, y=self.y, status=self.status,
@@ -196,19 +231,17 @@ class Mx8MoEStep:
         self.status = R.new_status(dev)
         self.wgu = F.pack_weights(to(wl.wgu), gate_up_interleave=True, status=self.status)
         self.wdn = F.pack_weights(to(wl.wdn), status=self.status)
-        _, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
-        self.pair_rows = pair_rows
-        self.rows_padded = int(off[-1])
-        self.scatter = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0],
-                                                      wl.topk_ids.shape[1])).to(dev)
-        self.offsets = torch.from_numpy(off.astype(np.int32)).to(dev)
-        self.expert_rows = torch.from_numpy(np.asarray(wl.counts, dtype=np.int32)).to(dev)
+        lay = device_layout(R, wl, dev, 128, self.status)
+        self.pair_rows = lay["pair_rows"]
+        self.rows_padded = lay["rows_used"]
+        self.scatter, self.offsets, self.expert_rows = lay["row_scatter"], lay["offsets"], lay["expert_rows"]
         self.x = to(wl.x)
         # padding rows are never written: the activations and h start zeroed and stay so
-        self.a = F.Mx8Packed.empty(self.rows_padded, wl.H, rows_padded=self.rows_padded, device=dev, zero=True)
-        self.h = torch.zeros(self.rows_padded, wl.I, dtype=torch.bfloat16, device=dev)
-        self.hq = F.Mx8Packed.empty(self.rows_padded, wl.I, device=dev)
-        self.y = torch.empty(self.rows_padded, wl.H, dtype=torch.bfloat16, device=dev)
+        rp = self.rows_padded
+        self.a = F.Mx8Packed.empty(rp, wl.H, rows_padded=rp, device=dev, zero=True)
+        self.h = torch.zeros(rp, wl.I, dtype=torch.bfloat16, device=dev)
+        self.hq = F.Mx8Packed.empty(rp, wl.I, device=dev)
+        self.y = torch.empty(rp, wl.H, dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize()
         R.check_status(self.status)
         torch.cuda.empty_cache()
@@ -304,22 +337,25 @@ class DecodeStep:
             R.pack_weights(wl.down_expert_torch(e, dev, out=dbuf), self.sel_dn, out=self.pdn.slab(e),
                            out_sel=self.pdns.slab(e), status=self.status)
         del wbuf, dbuf
-        se, sc, pair_rows = R.decode_slots(wl.counts)
-        self.n_slots = int(se.size)
+        # 16-token expert slabs from the device plan (worst-case slot table; the decode GEMM skips
+        # the unused slots, the h quantiser takes the used rows of each slot only)
+        lay = device_layout(R, wl, dev, 16, self.status, decode=True)
+        self.n_slots = lay["n_slots"]
+        self.slots_used = lay["slots_used"]
         self.rows = 16 * self.n_slots
-        self.slot_expert = torch.from_numpy(se).to(dev)
-        self.slot_count = torch.from_numpy(sc).to(dev)
-        self.scatter = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0],
-                                                      wl.topk_ids.shape[1])).to(dev)
+        self.slot_expert, self.slot_count = lay["slot_expert"], lay["slot_count"]
+        self.slot_first_row = lay["slot_first_row"]
+        self.scatter = lay["row_scatter"]
+        self.pair_rows = lay["pair_rows"]
         self.x = to(wl.x)
         S16 = R.SF_SLAB16
         # rows of a slab past its count are never named by the scatter map: zero them once
         self.a = P.empty(self.rows, wl.H, rows_padded=self.rows, device=dev, zero=True, sf_layout=S16)
         self.ar = P.empty(self.rows, wl.Kp_gu, rows_padded=self.rows, device=dev, zero=True, sf_layout=S16)
-        self.h = torch.empty(self.rows, wl.I, dtype=torch.bfloat16, device=dev)
+        self.h = torch.zeros(self.rows, wl.I, dtype=torch.bfloat16, device=dev)
         self.amax_h = torch.zeros(1, dtype=torch.float32, device=dev)
-        self.hq = P.empty(self.rows, wl.I, rows_padded=self.rows, device=dev, sf_layout=S16)
-        self.hqr = P.empty(self.rows, wl.Kp_dn, rows_padded=self.rows, device=dev, sf_layout=S16)
+        self.hq = P.empty(self.rows, wl.I, rows_padded=self.rows, device=dev, sf_layout=S16, zero=True)
+        self.hqr = P.empty(self.rows, wl.Kp_dn, rows_padded=self.rows, device=dev, sf_layout=S16, zero=True)
         self.y = torch.empty(self.rows, wl.H, dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize()
         R.check_status(self.status)
@@ -338,7 +374,9 @@ class DecodeStep:
                                       swiglu=True, y=self.h, amax_out=self.amax_h, status=self.status)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        # the token rows of each slot only (slot s: rows 16 s .. 16 s + slot_count[s] - 1)
+        R.nvfp4_quantize_segments(self.h, self.slot_first_row, self.slot_count, self.sel_dn, amax_in=self.amax_h,
+                                  out=self.hq, out_res=self.hqr, status=self.status)
         if "d0" in ev:
             ev["d0"].record()
         R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.slot_expert, self.slot_count, self.pdn, self.pdns,
@@ -387,8 +425,9 @@ class MoEBlockStep:
         self.ar = P.empty(self.cap, wl.Kp_gu, rows_padded=self.cap, device=dev, zero=True, sf_layout=lay)
         self.h = torch.zeros(self.cap, wl.I, dtype=torch.bfloat16, device=dev)
         self.amax_h = torch.zeros(1, dtype=torch.float32, device=dev)
-        self.hq = P.empty(self.cap, wl.I, rows_padded=self.cap, device=dev, sf_layout=lay)
-        self.hqr = P.empty(self.cap, wl.Kp_dn, rows_padded=self.cap, device=dev, sf_layout=lay)
+        self.hq = P.empty(self.cap, wl.I, rows_padded=self.cap, device=dev, sf_layout=lay, zero=True)
+        self.hqr = P.empty(self.cap, wl.Kp_dn, rows_padded=self.cap, device=dev, sf_layout=lay, zero=True)
+        self.slot_first_row = torch.arange(self.n_slots, dtype=torch.int32, device=dev) * 16 if decode else None
         self.ye = torch.zeros(self.cap, wl.H, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize()
@@ -417,7 +456,10 @@ class MoEBlockStep:
                                    amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
         if "q1" in ev:
             ev["q1"].record()
-        R.nvfp4_quantize(self.h, self.sel_dn, amax_in=self.amax_h, out=self.hq, out_res=self.hqr, status=self.status)
+        # the token rows only: each expert segment's (prefill) or each slot's (decode)
+        seg_first, seg_rows = (self.slot_first_row, self.sc) if self.decode else (self.off, self.expert_rows)
+        R.nvfp4_quantize_segments(self.h, seg_first, seg_rows, self.sel_dn, amax_in=self.amax_h, out=self.hq,
+                                  out_res=self.hqr, status=self.status)
         if "d0" in ev:
             ev["d0"].record()
         if self.decode:
@@ -526,13 +568,35 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------------------------------ CPU oracle leg
-def oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=0):
-    """The oracle on a bounded sample of the step: n_pairs (token, expert) rows through quantise,
-    gate_up, SwiGLU, quantise, down.  Returns (seconds, flops of the sample)."""
+def oracle_pack(wl, sel_gu, sel_dn, experts):
+    """The oracle's packed weights of the given experts (the rollout's once-per-sync weight pack,
+    kept out of the timed step like the GPU path's)."""
     import oracle as orc
 
+    packed = {}
+    for e in experts:
+        e = int(e)
+        wgu, wdn = wl.gate_up_expert(e), wl.down_expert(e)
+        s_gu = orc.global_scale(orc.amax_bf16(wgu))
+        s_dn = orc.global_scale(orc.amax_bf16(wdn))
+        packed[e] = (s_gu, orc.weight_pack(wgu, s_gu, sel_gu), s_dn, orc.weight_pack(wdn, s_dn, sel_dn))
+    return packed
+
+
+def sample_pairs(wl, n_pairs, seed):
     rng = np.random.default_rng(seed)
-    pairs = np.sort(rng.choice(wl.pair_token.size, n_pairs, replace=False))
+    return np.sort(rng.choice(wl.pair_token.size, n_pairs, replace=False))
+
+
+def oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=0, packed=None):
+    """The oracle on a bounded sample of the step: n_pairs (token, expert) rows through quantise,
+    gate_up, SwiGLU, quantise, down, with the experts' weights packed beforehand (outside the
+    timing, as on the GPU).  Returns (seconds, flops of the sample)."""
+    import oracle as orc
+
+    pairs = sample_pairs(wl, n_pairs, seed)
+    if packed is None:
+        packed = oracle_pack(wl, sel_gu, sel_dn, np.unique(wl.pair_expert[pairs]))
     t0 = time.perf_counter()
     s_x = orc.global_scale(orc.amax_bf16(wl.x))
     h_rows, exps = [], []
@@ -540,9 +604,7 @@ def oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=0):
         idx = pairs[wl.pair_expert[pairs] == e]
         xa = wl.x[wl.pair_token[idx]]
         ac, aS, rc, rS, _ = orc.act_quant_rac(xa, s_x, sel_gu)
-        wgu = wl.gate_up_expert(int(e))
-        s_w = orc.global_scale(orc.amax_bf16(wgu))
-        wc, wS, wsc, wsS = orc.weight_pack(wgu, s_w, sel_gu)
+        s_w, (wc, wS, wsc, wsS), _, _ = packed[int(e)]
         gu, _ = orc.gemm_rac(ac, aS, rc, rS, wc, wS, wsc, wsS, s_x, s_w)
         gu_b = orc.f64_to_bf16_array(gu)
         h, _ = orc.swiglu(gu_b)
@@ -553,9 +615,7 @@ def oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=0):
     start = 0
     for e, n in exps:
         hc, hS, hrc, hrS, _ = orc.act_quant_rac(hh[start:start + n], s_h, sel_dn)
-        wdn = wl.down_expert(int(e))
-        s_w = orc.global_scale(orc.amax_bf16(wdn))
-        dc, dS, dsc, dsS = orc.weight_pack(wdn, s_w, sel_dn)
+        _, _, s_w, (dc, dS, dsc, dsS) = packed[int(e)]
         orc.gemm_rac(hc, hS, hrc, hrS, dc, dS, dsc, dsS, s_h, s_w)
         start += n
     dt = time.perf_counter() - t0
@@ -576,11 +636,15 @@ def run_reference(args):
     sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
     sel_dn, _ = orc.calibrate(h_cal, wl.Kp_dn)
     n_pairs = args.ref_pairs
+    # the weight pack happens once per trainer -> rollout sync, outside the steps (as on the GPU)
+    packed = oracle_pack(wl, sel_gu, sel_dn, np.unique(np.concatenate(
+        [wl.pair_expert[sample_pairs(wl, n, i)] for i, n in [(0, max(8, n_pairs // 8))] +
+         [(i, n_pairs) for i in range(args.steps)]])))
     for _ in range(args.warmup):
-        oracle_sample(wl, sel_gu, sel_dn, max(8, n_pairs // 8))
+        oracle_sample(wl, sel_gu, sel_dn, max(8, n_pairs // 8), packed=packed)
     times, flops = [], 0.0
     for i in range(args.steps):
-        dt, f = oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=i)
+        dt, f = oracle_sample(wl, sel_gu, sel_dn, n_pairs, seed=i, packed=packed)
         times.append(dt)
         flops += f
     total = sum(times)
@@ -592,7 +656,8 @@ def run_reference(args):
             "data": "synthetic (seeded)",
             "config": {"workload": wl.name + f"_r{wl.r}", "sample_pairs_per_step": n_pairs},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": cores, "kind": "oracle",
-                             "sample": f"{n_pairs} of {wl.pair_token.size} (token, expert) rows per step"},
+                             "sample": f"{n_pairs} of {wl.pair_token.size} (token, expert) rows per step, "
+                                       "weights packed before the timed steps"},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -610,12 +675,21 @@ def spec_moe(dev, args, peaks):
         import oracle as orc
 
         orc.build()
-        dt, f = oracle_sample(wl, step.sel_gu.cpu().numpy(), step.sel_dn.cpu().numpy(), args.cpu_pairs)
+        sg, sd = step.sel_gu.cpu().numpy(), step.sel_dn.cpu().numpy()
+        packed = oracle_pack(wl, sg, sd, np.unique(wl.pair_expert[sample_pairs(wl, args.cpu_pairs, 0)]))
+        dt, f = oracle_sample(wl, sg, sd, args.cpu_pairs, packed=packed)
         return {"value": f / dt / 1e12, "unit": "TFLOP/s", "cores": orc.num_threads(), "kind": "oracle",
-                "sample": f"{args.cpu_pairs} of {P} (token, expert) rows of one step, {dt:.1f} s"}
+                "sample": f"{args.cpu_pairs} of {P} (token, expert) rows of one step, weights packed beforehand "
+                          f"(outside the timing), {dt:.1f} s"}
+
+    # end to end: the whole layer through the public API (router top-k of the logits, dispatch
+    # plan, quantise, both GEMMs, weighted combine into [T, H]) with X and the logits copied in
+    # and the [T, H] output copied out every step
+    e2e_step = MoEBlockStep(wl, (step.pgu, step.pgus, step.pdn, step.pdns), step.sel_gu, step.sel_dn, False, dev)
 
     return dict(
         step=step, x_np=wl.x, flops=gu_f + dn_f, events=["q0", "g0", "q1", "d0", "end"],
+        e2e_step=e2e_step, e2e_extra_h2d={"logits": e2e_step.logits_np},
         segments={"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")},
         dominant=("gate_up", gu_f, gu_bytes, "grouped gate_up W4A4+RAC GEMM (SwiGLU epilogue)"),
         # DRAM traffic of the gate_up launch is reported only from a capture of the kernel as it is
@@ -744,7 +818,8 @@ def spec_decode(dev, args, peaks):
         extra_gbs={"gate_up": ("gate_up", gu_bytes), "down": ("down", dn_bytes),
                    "weights_step": (None, gu_w + dn_w)},
         config={"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P, "experts": wl.E,
-                "touched_experts": touched, "slabs": step.n_slots, "hidden": wl.H, "intermediate": wl.I,
+                "touched_experts": touched, "slabs": step.slots_used, "slot_table": step.n_slots, "hidden": wl.H,
+                "intermediate": wl.I,
                 "Kp_gate_up": wl.Kp_gu, "Kp_down": wl.Kp_dn, "weight_bytes_touched": gu_w + dn_w},
         cpu=cpu_leg, kernels_per_step=DecodeStep.KERNELS_PER_STEP)
 
@@ -793,10 +868,10 @@ def spec_block_decode(dev, args, peaks):
     return _spec_block(dev, args, True)
 
 
-def _spec_qdq(dev, args, n_tensors):
+def _spec_qdq(dev, args, n_tensors, elems=1 << 31):
     from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 
-    w = syn.trainer_weights(n_tensors=n_tensors)
+    w = syn.trainer_weights(n_tensors=n_tensors, elems=elems)
     step = QdqStep(w, dev)
     n = w.size
     label = f"weight_qdq_{n_tensors}x{w.shape[1]}"
@@ -823,7 +898,8 @@ def _spec_qdq(dev, args, n_tensors):
 
 
 def spec_qdq(dev, args, peaks):
-    return _spec_qdq(dev, args, 1024)
+    # tensors of 1024 x 2048 elements (1024 of them: 2^31 elements)
+    return _spec_qdq(dev, args, args.qdq_tensors, args.qdq_tensors << 21)
 
 
 def spec_qdq_single(dev, args, peaks):
@@ -962,6 +1038,8 @@ def main():
     ap.add_argument("--cpu-pairs", type=int, default=256)
     ap.add_argument("--cpu-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--qdq-tensors", type=int, default=1024,
+                    help="qdq workload: number of 1024 x 2048 tensors (1024 = 2^31 elements; fewer for profiler captures)")
     ap.add_argument("--experts", type=int, default=None,
                     help="MoE workloads: expert count override (smaller device footprint for profiler captures)")
     args = ap.parse_args()
@@ -1048,12 +1126,15 @@ def main():
     roof["peak_source"] = (f"{peak_kind}: HBM = copy bandwidth, FP4 = bf16 burst x {FP4_OVER_BF16:g} (nominal ratio)"
                            if peak_kind == "measured" else "recipe fallback")
 
-    # end-to-end through the public API with host buffers: H2D of X, D2H of Y every step
+    # end-to-end through the public API with host buffers: H2D of the inputs, D2H of the result
+    # every step (for the MoE block: the whole layer, [T, H] out)
+    e2e_step = sp.get("e2e_step", step)
+    e2e_h2d = sp.get("e2e_extra_h2d", sp.get("extra_h2d", {}))
     x_np = sp["x_np"]
     x_host = torch.from_numpy(x_np.view(np.int16)).pin_memory()
-    y_host = torch.empty(step.y.shape, dtype=torch.bfloat16).pin_memory()
+    y_host = torch.empty(e2e_step.y.shape, dtype=torch.bfloat16).pin_memory()
     x_dev = torch.empty(x_np.shape, dtype=torch.bfloat16, device=dev)
-    extra_host = {k: torch.from_numpy(v).pin_memory() for k, v in sp.get("extra_h2d", {}).items()}
+    extra_host = {k: torch.from_numpy(v).pin_memory() for k, v in e2e_h2d.items()}
     extra_dev = {k: torch.empty_like(v, device=dev) for k, v in extra_host.items()}
     barrier()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -1065,15 +1146,18 @@ def main():
         x_dev.view(torch.int16).copy_(x_host, non_blocking=True)
         for k, v in extra_host.items():
             extra_dev[k].copy_(v, non_blocking=True)
-        y = step.run(x=x_dev, **extra_dev)
+        y = e2e_step.run(x=x_dev, **extra_dev)
         y_host.copy_(y, non_blocking=True)
         e1.record()
         torch.cuda.synchronize()
         e2e_ms += e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms / n_e2e, ws, dev)
+    R.check_status(e2e_step.status)
     e2e = {"value": whole_job_rate(work, ws, e2e_ms, scale), "unit": unit,
-           "h2d_bytes_per_step": int(x_np.nbytes) + sum(int(v.nbytes) for v in sp.get("extra_h2d", {}).values()),
-           "d2h_bytes_per_step": int(y_host.numel() * 2)}
+           "h2d_bytes_per_step": int(x_np.nbytes) + sum(int(v.nbytes) for v in e2e_h2d.values()),
+           "d2h_bytes_per_step": int(y_host.numel() * 2),
+           "call": "whole MoE layer (router, plan, quantise, GEMMs, combine into [T, H])" if "e2e_step" in sp
+           else "the timed step"}
 
     cpu = sp["cpu"]() if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
 

@@ -122,6 +122,13 @@ int32_t nvfp4_kp_from_ratio(int64_t K, double r);
 void nvfp4_set_wait_limit_ns(uint64_t ns);
 /* Tuning: N-tile of the GEMM kernels, 128 or 256 (0 = automatic choice per shape). */
 void nvfp4_set_gemm_tile_n(int32_t n);
+/* Tuning: 1 runs the W4A4 + RAC GEMMs whose N is a multiple of 256 on pairs of SMs (one
+ * 256 x 256 tile per cluster of two CTAs); 0 (default) keeps one SM per 128-row tile. */
+void nvfp4_set_gemm_pairs(int32_t on);
+/* Tuning: rows per tile (1..16) and consumer warps (4, 6, 7 or 8) of the activation quantiser
+ * (0 = automatic choice per shape).  A forced shape that does not fit shared memory makes the
+ * quantise calls fall back to the row quantiser. */
+void nvfp4_set_act_tile(int32_t rows, int32_t warps);
 
 /* ---------------------------------------------------------------------------------------- */
 /* nvfp4_quantize -- online activation quantisation with the RAC residual pass              */
@@ -162,6 +169,27 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
                                     int32_t fanout, const int32_t* sel, int32_t Kp, const float* amax_in,
                                     const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
                                     size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* nvfp4_quantize_segments -- nvfp4_quantize of the token rows of an expert-grouped layout   */
+/* only: the input of the down projection (h), whose expert segments are padded to 128 rows. */
+/*   x              bf16 [M x K] in the padded expert-grouped row order (pitch ldx).          */
+/*   expert_offsets int32 [E] (device): first row of each segment (moe_dispatch_plan's         */
+/*                  offsets); expert_rows int32 [E] (device): token rows of each segment.      */
+/*   Rows [expert_offsets[e], expert_offsets[e] + expert_rows[e]) of x are quantised into the  */
+/*   same rows of q / q_res; every other row of q / q_res is left untouched (a caller zeroes   */
+/*   them once if it wants the padding to stay zero; the grouped GEMM does not store the       */
+/*   output boxes of padding rows when given the same expert_rows).  A segment reaching past  */
+/*   row M is skipped and NVFP4_ERR_INVALID_ARG goes to *dev_status.                          */
+/*   s_g is computed over all M rows unless amax_in is given (the SwiGLU epilogue's amax      */
+/*   covers the token rows).  q.rows_padded >= M; 1 <= E <= 1024.  Other arguments as         */
+/*   nvfp4_quantize (shared list, compact residual).                                          */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status nvfp4_quantize_segments(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                     const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
+                                     const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                                     const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* nvfp4_quantize_grouped_sel -- nvfp4_quantize with one channel list per group of output    */
@@ -270,6 +298,33 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
                                   void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* grouped_w4a4_rac_moe_segments -- grouped_w4a4_rac_moe over arbitrary row segments, each   */
+/* with its own weight slab: what an expert-parallel rank receives (one 128-padded segment per */
+/* source rank and local expert, source-major), run without reordering the rows.             */
+/*   seg_offsets int32 [n_seg + 1] (device): segment i is rows [seg_offsets[i],               */
+/*               seg_offsets[i+1]) (multiples of 128); seg_rows optional int32 [n_seg]: token */
+/*               rows of each segment (as expert_rows); seg_expert int32 [n_seg]: slab of w /  */
+/*               w_sel used by segment i (0 <= seg_expert[i] < w->slabs, else                  */
+/*               NVFP4_ERR_INVALID_ARG in *dev_status and slab 0 is read instead).              */
+/*   Other arguments as grouped_w4a4_rac_moe (E there = n_seg here).                           */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status grouped_w4a4_rac_moe_segments(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
+                                           const int32_t* seg_offsets, const int32_t* seg_rows,
+                                           const int32_t* seg_expert, int32_t n_seg, const nvfp4_tensor* w,
+                                           const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp,
+                                           nvfp4_epilogue ep, nvfp4_dtype out, void* y, int64_t ldy,
+                                           float* amax_out, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* nvfp4_amax -- max |x| over a bf16 [M x K] matrix (pitch ldx) into *amax_out (device float): */
+/* the input of the per-tensor scale s_g = amax / 2688.  An expert-parallel layer reduces it  */
+/* over the ranks (a MAX all-reduce) and passes it to the quantise calls as amax_in, so that  */
+/* every rank quantises with the scale of the whole batch.  workspace as nvfp4_quantize.       */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status nvfp4_amax(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float* amax_out, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
 /* grouped_w4a4_rac_moe_decode -- the grouped GEMM above for decode, where each expert sees   */
 /* only a few tokens.  The expert's weight rows are streamed as the MMA's 128-row operand and  */
 /* the expert's tokens, gathered into 16-row slabs, are the 16-column operand, so one pass     */
@@ -351,6 +406,32 @@ size_t weight_qdq_workspace_size(int64_t n_tensors, int64_t elems_per_tensor);
 nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_tensor, uint16_t* w_out,
                         float* s_g_out, void* workspace, size_t workspace_bytes, int32_t* dev_status,
                         void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* weight_qdq_backward -- gradient of the trainer fake-quant (Two fixes: Asymmetric QAT       */
+/* fake-quantises the weights only) under the straight-through estimator: the rounding of     */
+/* W_fq = bf16(DQ(Q(W))) is treated as the identity, so dL/dW = dL/dW_fq.  (A reading: the    */
+/* pages name QAT on weights without its backward rule; the straight-through estimator is the */
+/* usual one, and with a per-tensor amax scale no element sits in a clipped range.)            */
+/*   grad_fq   bf16 [n]: dL/dW_fq.                                                            */
+/*   grad_w    optional bf16 [n]: receives dL/dW (== grad_fq bitwise; grad_w == grad_fq is    */
+/*             allowed and launches nothing).                                                  */
+/*   grad_acc  optional float32 [n]: the trainer's master gradient, grad_acc += dL/dW (one     */
+/*             binary32 add per element).  At least one of grad_w / grad_acc.                 */
+/*   All buffers 16-byte aligned.                                                              */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status weight_qdq_backward(const uint16_t* grad_fq, int64_t n, uint16_t* grad_w, float* grad_acc,
+                                 void* stream);
+
+/* ---------------------------------------------------------------------------------------- */
+/* nvfp4_unpack_logical -- a packed matrix in logical order (inspection and test helper).     */
+/*   q          packed tensor (either scale layout); slab in [0, q->slabs) picks one matrix.  */
+/*   codes_out  optional uint8 [q->rows x q->cols] (16-byte aligned): one E2M1 code per byte.  */
+/*   sf_out     optional uint8 [q->rows x q->cols/16]: the E4M3 scale of (row, 16-block).      */
+/*   Rows >= q->rows are not read.                                                             */
+/* ---------------------------------------------------------------------------------------- */
+nvfp4_status nvfp4_unpack_logical(const nvfp4_tensor* q, int64_t slab, uint8_t* codes_out, uint8_t* sf_out,
+                                  void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* weight_qdq_noalloc -- weight_qdq for callers that cannot allocate device memory.          */

@@ -19,6 +19,8 @@ namespace {
 thread_local std::string g_last_error;
 std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_tile_n{0};  // 0: automatic
+std::atomic<int> g_act_rows{0}, g_act_warps{0};  // activation quantiser tile: 0 = automatic
+std::atomic<int> g_gemm_pair{0};  // CTA-pair GEMM where the shape allows it
 
 nvfp4_status fail(nvfp4_status s, const char* fmt, ...) {
   char buf[512];
@@ -188,6 +190,13 @@ void nvfp4_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 
 void nvfp4_set_gemm_tile_n(int32_t n) { g_tile_n.store((n == 128 || n == 256) ? n : 0); }
 
+void nvfp4_set_gemm_pairs(int32_t on) { g_gemm_pair.store(on ? 1 : 0); }
+
+void nvfp4_set_act_tile(int32_t rows, int32_t warps) {
+  g_act_rows.store(rows >= 1 && rows <= 16 ? rows : 0);
+  g_act_warps.store((warps == 4 || warps == 6 || warps == 7 || warps == 8) ? warps : 0);
+}
+
 // ------------------------------------------------------------------------------------------ quantize
 size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K) {
   (void)M;
@@ -196,6 +205,45 @@ size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K) {
 }
 
 }  // extern "C"
+
+namespace {
+// The bulk-copy activation quantiser serves the method's compact residual with one shared list
+// (and no residual); the masked and per-group variants keep the row quantiser.
+bool use_act_kernel(int64_t K, int32_t Kp, int fanout, int32_t n_seg, bool masked, int32_t groups) {
+  int R, W, smem;
+  return !masked && groups == 0 &&
+         act_plan_choose(K, Kp, fanout, n_seg, &R, &W, &smem, g_act_rows.load(), g_act_warps.load());
+}
+
+nvfp4::ActArgs act_args(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* sel, int32_t Kp,
+                        const float* partial, int P, const float* amax_in, const nvfp4_tensor* q,
+                        const nvfp4_tensor* q_res, int32_t* dev_status) {
+  nvfp4::ActArgs a;
+  memset(&a, 0, sizeof(a));
+  a.src = x;
+  a.src_rows = M;
+  a.ld = ldx;
+  a.K = (int32_t)K;
+  a.Kp = Kp;
+  a.fanout = 1;
+  a.rows_out = q->rows_padded;
+  a.sel = sel;
+  a.partial = partial;
+  a.P = P;
+  a.amax_in = amax_in;
+  a.s_g_out = q->s_g;
+  a.s_g_out2 = Kp > 0 ? q_res->s_g : nullptr;
+  a.codes = q->codes;
+  a.sf = q->sf;
+  a.rcodes = Kp > 0 ? q_res->codes : nullptr;
+  a.rsf = Kp > 0 ? q_res->sf : nullptr;
+  a.sf_slab16 = q->sf_layout == NVFP4_SF_SLAB16;
+  a.status = dev_status;
+  a.wait_limit_ns = g_wait_limit_ns.load();
+  return a;
+}
+
+}  // namespace
 
 namespace {
 // nvfp4_quantize and its per-group form: groups == 0 -> one shared list sel [Kp]; groups > 0 ->
@@ -238,6 +286,16 @@ nvfp4_status quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
   if (!amax_in) {
     cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  }
+  const bool masked = Kp > 0 && Kp < K && q_res->cols == K;
+  if (q->rows_padded > 0 && use_act_kernel(K, Kp, 1, 0, masked, groups)) {
+    nvfp4::ActArgs b = act_args(x, M, K, ldx, sel, Kp, partial, P, amax_in, q, q_res, dev_status);
+    b.map = row_gather ? kMapGather : kMapRows;
+    b.row_gather = row_gather;
+    b.rows_valid = M_out;
+    cudaError_t e = launch_act(b, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    return NVFP4_OK;
   }
   RowArgs a;
   memset(&a, 0, sizeof(a));
@@ -331,6 +389,16 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
     cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "amax launch");
   }
+  const bool masked = Kp > 0 && Kp < K && q_res->cols == K;
+  if (use_act_kernel(K, Kp, fanout, 0, masked, 0)) {
+    nvfp4::ActArgs b = act_args(x, M, K, ldx, sel, Kp, partial, P, amax_in, q, q_res, dev_status);
+    b.map = kMapScatter;
+    b.row_scatter = row_scatter;
+    b.fanout = fanout;
+    cudaError_t e = launch_act(b, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
+    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+    return NVFP4_OK;
+  }
   RowArgs a;
   memset(&a, 0, sizeof(a));
   a.mode = kModeAct;
@@ -357,6 +425,56 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
   a.rsf = Kp > 0 ? q_res->sf : nullptr;
   a.status = dev_status;
   cudaError_t e = launch_rows(a, num_sms(), s);
+  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
+  return NVFP4_OK;
+}
+
+nvfp4_status nvfp4_quantize_segments(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                     const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
+                                     const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                                     const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
+  if (!expert_offsets || !expert_rows) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets / expert_rows is NULL");
+  if (E < 1 || E > kMaxRouteExperts) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be in [1, %d]", kMaxRouteExperts);
+  if (M < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "negative row count");
+  if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64 <= %lld", (long long)K, (long long)kMaxK);
+  if (ldx < K || ldx % 8 != 0) return fail(NVFP4_ERR_ALIGNMENT, "ldx = %lld must be >= K and a multiple of 8", (long long)ldx);
+  if (x && !aligned16(x)) return fail(NVFP4_ERR_ALIGNMENT, "x must be 16-byte aligned");
+  if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp = %d must be a multiple of 64 in [0, K]", Kp);
+  nvfp4_status st = check_tensor(q, "q", K, M, 1, kAnyLayout);
+  if (st != NVFP4_OK) return st;
+  if (Kp > 0) {
+    if (!sel) return fail(NVFP4_ERR_INVALID_ARG, "sel is NULL with Kp > 0");
+    st = check_tensor(q_res, "q_res", Kp, M, 1, kAnyLayout);
+    if (st != NVFP4_OK) return st;
+    if (q_res->rows_padded != q->rows_padded || q_res->sf_layout != q->sf_layout)
+      return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res must have q's rows_padded and sf_layout");
+  }
+  if (!use_act_kernel(K, Kp, 1, E, false, 0))
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld, Kp = %d too large for the segment quantiser", (long long)K, Kp);
+  const int P = act_partials(M, K);
+  if (!amax_in) {
+    if (!workspace || workspace_bytes < nvfp4_quantize_workspace_size(M, K))
+      return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+    if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
+  }
+  if (M == 0) return NVFP4_OK;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* partial = reinterpret_cast<float*>(workspace);
+  if (!amax_in) {
+    cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "amax launch");
+  }
+  nvfp4::ActArgs b = act_args(x, M, K, ldx, sel, Kp, partial, P, amax_in, q, q_res, dev_status);
+  b.map = kMapSegments;
+  b.seg_off = expert_offsets;
+  b.seg_rows = expert_rows;
+  b.n_seg = E;
+  b.rows_valid = M;
+  b.src_rows = M;
+  cudaError_t e = launch_act(b, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
   if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
   return NVFP4_OK;
 }
@@ -524,7 +642,8 @@ nvfp4_status pack_weights_grouped_sel(const uint16_t* w, int64_t E, int64_t N, i
 static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
                                 const nvfp4_tensor* w_sel, int64_t rows_needed, int64_t N, int64_t K, int32_t Kp,
                                 int64_t E, nvfp4_dtype out, void* y, int64_t ldy, int64_t y_cols, int64_t y_rows,
-                                int bn, CUtensorMap* maps, GemmArgs* g) {
+                                int bn, CUtensorMap* maps, GemmArgs* g, int w_box_rows = 0) {
+  if (w_box_rows == 0) w_box_rows = bn;
   if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
   if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp must be a multiple of 64 in [0, K]");
   if (N <= 0 || N % 128 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "N must be a positive multiple of 128");
@@ -553,12 +672,13 @@ static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res
   }
   st = make_code_map(&maps[0], a->codes, (uint64_t)K / 2, (uint64_t)a->rows_padded, 1, 128, 2, "A");
   if (st != NVFP4_OK) return st;
-  st = make_code_map(&maps[2], w->codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, (uint32_t)bn, 3, "W");
+  st = make_code_map(&maps[2], w->codes, (uint64_t)K / 2, (uint64_t)N, (uint64_t)E, (uint32_t)w_box_rows, 3, "W");
   if (st != NVFP4_OK) return st;
   if (Kp > 0) {
     st = make_code_map(&maps[1], a_res->codes, (uint64_t)Kp / 2, (uint64_t)a_res->rows_padded, 1, 128, 2, "A_res");
     if (st != NVFP4_OK) return st;
-    st = make_code_map(&maps[3], w_sel->codes, (uint64_t)Kp / 2, (uint64_t)N, (uint64_t)E, (uint32_t)bn, 3, "W_sel");
+    st = make_code_map(&maps[3], w_sel->codes, (uint64_t)Kp / 2, (uint64_t)N, (uint64_t)E, (uint32_t)w_box_rows, 3,
+                       "W_sel");
     if (st != NVFP4_OK) return st;
   } else {
     maps[1] = maps[0];
@@ -592,10 +712,11 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, con
                            void* y, int64_t ldy, int32_t* dev_status, void* stream) {
   g_last_error.clear();
   if (M < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M must be >= 0");
-  const int bn = choose_tile_n(N, K, Kp);
+  const bool pairs = g_gemm_pair.load() != 0 && N % 256 == 0 && g_tile_n.load() != 128;
+  const int bn = pairs ? 256 : choose_tile_n(N, K, Kp);
   CUtensorMap maps[5];
   GemmArgs g;
-  nvfp4_status st = gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, M, bn, maps, &g);
+  nvfp4_status st = gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, M, bn, maps, &g, pairs ? 128 : bn);
   if (st != NVFP4_OK) return st;
   if (M == 0) return NVFP4_OK;
   g.offsets = nullptr;
@@ -605,21 +726,30 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, con
   g.epi = 0;
   g.status = dev_status;
   int64_t tiles = (int64_t)g.m_blocks_dense * g.n_blocks;
-  int grid = (int)(tiles < num_sms() ? tiles : num_sms());
-  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, grid,
-                              reinterpret_cast<cudaStream_t>(stream));
+  cudaError_t e;
+  if (pairs) {
+    const int64_t pair_tiles = (int64_t)((g.m_blocks_dense + 1) / 2) * g.n_blocks;
+    const int n_pairs = (int)(pair_tiles < num_sms() / 2 ? pair_tiles : num_sms() / 2);
+    e = launch_gemm_pair(maps[0], maps[1], maps[2], maps[3], maps[4], g, n_pairs, reinterpret_cast<cudaStream_t>(stream));
+  } else {
+    int grid = (int)(tiles < num_sms() ? tiles : num_sms());
+    e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, grid, reinterpret_cast<cudaStream_t>(stream));
+  }
   if (e != cudaSuccess) return cuda_fail(e, "gemm launch");
   return NVFP4_OK;
 }
 
-nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
-                                  const int32_t* expert_rows, int32_t E, const nvfp4_tensor* w,
-                                  const nvfp4_tensor* w_sel, int64_t N, int64_t K,
-                                  int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y, int64_t ldy,
-                                  float* amax_out, int32_t* dev_status, void* stream) {
-  g_last_error.clear();
-  if (!expert_offsets) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets is NULL");
-  if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
+}  // extern "C"
+
+namespace {
+// The grouped GEMM over n_seg row segments; segment i uses weight slab seg_expert[i] (or i).
+nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* offsets,
+                            const int32_t* seg_rows, const int32_t* seg_expert, int32_t n_seg, const nvfp4_tensor* w,
+                            const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp, nvfp4_epilogue ep,
+                            nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
+                            void* stream) {
+  if (!offsets) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets is NULL");
+  if (n_seg <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the segment count must be positive");
   if (ep != NVFP4_EPI_NONE && ep != NVFP4_EPI_SWIGLU_AMAX) return fail(NVFP4_ERR_INVALID_ARG, "bad epilogue");
   if (ep == NVFP4_EPI_SWIGLU_AMAX) {
     if (out != NVFP4_OUT_BF16) return fail(NVFP4_ERR_INVALID_ARG, "the SwiGLU epilogue writes bf16");
@@ -627,16 +757,21 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
   }
   if (ep == NVFP4_EPI_SWIGLU_AMAX && N % 256 != 0)
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the SwiGLU epilogue needs N %% 256 == 0");
-  const int bn = ep == NVFP4_EPI_SWIGLU_AMAX ? 256 : choose_tile_n(N, K, Kp);
+  if (!w) return fail(NVFP4_ERR_INVALID_ARG, "w is NULL");
+  const int64_t E = seg_expert ? w->slabs : n_seg;
+  const bool pairs = g_gemm_pair.load() != 0 && N % 256 == 0 && g_tile_n.load() != 128 && n_seg <= kMaxRouteExperts;
+  const int bn = (pairs || ep == NVFP4_EPI_SWIGLU_AMAX) ? 256 : choose_tile_n(N, K, Kp);
   CUtensorMap maps[5];
   GemmArgs g;
   const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
-  nvfp4_status st =
-      gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, a ? a->rows_padded : 0, bn, maps, &g);
+  nvfp4_status st = gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, a ? a->rows_padded : 0, bn,
+                                maps, &g, pairs ? 128 : bn);
   if (st != NVFP4_OK) return st;
-  g.offsets = expert_offsets;
-  g.expert_rows = expert_rows;
-  g.E = E;
+  g.offsets = offsets;
+  g.expert_rows = seg_rows;
+  g.E = n_seg;
+  g.seg_expert = seg_expert;
+  g.n_weights = (int32_t)E;
   g.M = a->rows_padded;
   g.m_blocks_dense = 0;
   g.epi = ep == NVFP4_EPI_SWIGLU_AMAX ? 1 : 0;
@@ -647,9 +782,57 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
     cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
     if (e != cudaSuccess) return cuda_fail(e, "amax reset");
   }
-  cudaError_t e = launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms(), s);
+  cudaError_t e = pairs ? launch_gemm_pair(maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms() / 2, s)
+                        : launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "grouped gemm launch");
   return NVFP4_OK;
+}
+}  // namespace
+
+extern "C" {
+
+nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
+                                  const int32_t* expert_rows, int32_t E, const nvfp4_tensor* w,
+                                  const nvfp4_tensor* w_sel, int64_t N, int64_t K,
+                                  int32_t Kp, nvfp4_epilogue ep, nvfp4_dtype out, void* y, int64_t ldy,
+                                  float* amax_out, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
+  return grouped_common(a, a_res, expert_offsets, expert_rows, nullptr, E, w, w_sel, N, K, Kp, ep, out, y, ldy,
+                        amax_out, dev_status, stream);
+}
+
+nvfp4_status grouped_w4a4_rac_moe_segments(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
+                                           const int32_t* seg_offsets, const int32_t* seg_rows,
+                                           const int32_t* seg_expert, int32_t n_seg, const nvfp4_tensor* w,
+                                           const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp,
+                                           nvfp4_epilogue ep, nvfp4_dtype out, void* y, int64_t ldy,
+                                           float* amax_out, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!seg_expert) return fail(NVFP4_ERR_INVALID_ARG, "seg_expert is NULL");
+  return grouped_common(a, a_res, seg_offsets, seg_rows, seg_expert, n_seg, w, w_sel, N, K, Kp, ep, out, y, ldy,
+                        amax_out, dev_status, stream);
+}
+
+nvfp4_status nvfp4_amax(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float* amax_out, void* workspace,
+                        size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (!amax_out || (!x && M > 0)) return fail(NVFP4_ERR_INVALID_ARG, "x / amax_out is NULL");
+  if (M < 0 || K <= 0 || K % 8 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M >= 0 and K a positive multiple of 8");
+  if (ldx < K || ldx % 8 != 0) return fail(NVFP4_ERR_ALIGNMENT, "ldx must be >= K and a multiple of 8");
+  if (x && !aligned16(x)) return fail(NVFP4_ERR_ALIGNMENT, "x must be 16-byte aligned");
+  if (!workspace || workspace_bytes < nvfp4_quantize_workspace_size(M, K))
+    return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (M == 0) {
+    cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
+    return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "amax reset");
+  }
+  float* partial = reinterpret_cast<float*>(workspace);
+  const int P = act_partials(M, K);
+  cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
+  if (e == cudaSuccess) e = launch_reduce_amax(partial, P, amax_out, s);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "amax launch");
 }
 
 nvfp4_status grouped_w4a4_rac_moe_decode(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
@@ -829,6 +1012,39 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_
   e = launch_qdq(w, n_tensors, elems_per_tensor, w_out, partial, P, s_g_out, dev_status, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "qdq launch");
   return NVFP4_OK;
+}
+
+nvfp4_status weight_qdq_backward(const uint16_t* grad_fq, int64_t n, uint16_t* grad_w, float* grad_acc,
+                                 void* stream) {
+  g_last_error.clear();
+  if (n < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "n must be >= 0");
+  if (n > 0 && !grad_fq) return fail(NVFP4_ERR_INVALID_ARG, "grad_fq is NULL");
+  if (!grad_w && !grad_acc) return fail(NVFP4_ERR_INVALID_ARG, "grad_w and grad_acc are both NULL");
+  if ((grad_fq && !aligned16(grad_fq)) || (grad_w && !aligned16(grad_w)) || (grad_acc && !aligned16(grad_acc)))
+    return fail(NVFP4_ERR_ALIGNMENT, "gradient buffers must be 16-byte aligned");
+  if (grad_w == grad_fq) grad_w = nullptr;  // in place: the identity needs no copy
+  if (n == 0 || (!grad_w && !grad_acc)) return NVFP4_OK;
+  cudaError_t e = launch_qdq_backward(grad_fq, n, grad_w, grad_acc, num_sms(), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "qdq backward launch");
+}
+
+nvfp4_status nvfp4_unpack_logical(const nvfp4_tensor* q, int64_t slab, uint8_t* codes_out, uint8_t* sf_out,
+                                  void* stream) {
+  g_last_error.clear();
+  if (!q) return fail(NVFP4_ERR_INVALID_ARG, "q is NULL");
+  if (!codes_out && !sf_out) return fail(NVFP4_ERR_INVALID_ARG, "codes_out and sf_out are both NULL");
+  if (q->slabs < 1 || slab < 0 || slab >= q->slabs) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "slab out of range");
+  nvfp4_status st = check_tensor(q, "q", q->cols, q->rows, q->slabs, kAnyLayout);
+  if (st != NVFP4_OK) return st;
+  if (q->cols <= 0 || q->cols % 64 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q.cols must be a positive multiple of 64");
+  if (codes_out && !aligned16(codes_out)) return fail(NVFP4_ERR_ALIGNMENT, "codes_out must be 16-byte aligned");
+  if (q->rows == 0) return NVFP4_OK;
+  const int64_t cb = q->rows_padded * q->cols / 2;
+  const int64_t sb = (int64_t)nvfp4_sf_bytes_layout(q->rows_padded, q->cols, q->sf_layout);
+  cudaError_t e = launch_unpack_logical(q->codes + slab * cb, q->sf + slab * sb, q->rows, q->cols,
+                                        q->sf_layout == NVFP4_SF_SLAB16, codes_out, sf_out, num_sms(),
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "unpack launch");
 }
 
 // ------------------------------------------------------------------------------------------ helpers

@@ -31,6 +31,19 @@ constexpr int BM = 128;
 constexpr int KT_BYTES = 128;  // bytes of one row per k-tile: 256 FP4 elements
 constexpr int NUM_THREADS = 320;  // producer warp, MMA warp, 8 epilogue warps
 
+// Weight slab of grouped segment `seg`: the segment itself, or seg_expert[seg] (segments of
+// several sources that share an expert, as an expert-parallel rank receives them).  An index
+// outside the weight slabs is reported and replaced by slab 0, so no load leaves the weights.
+__device__ __forceinline__ int segment_weight(const GemmArgs& args, int seg) {
+  if (args.seg_expert == nullptr) return seg;
+  const int e = __ldg(args.seg_expert + seg);
+  if (e < 0 || e >= args.n_weights) {
+    report_status(args.status, kErrInvalid);
+    return 0;
+  }
+  return e;
+}
+
 template <int BN>
 struct Cfg {
   static constexpr int STAGES = (BN == 256) ? 3 : 5;
@@ -156,7 +169,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int64_t t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
         const int64_t mb = t / args.n_blocks;
         const int nb = (int)(t - mb * args.n_blocks);
-        const int e = grouped ? find_expert(args.offsets, args.E, mb * BM) : 0;
+        const int e = grouped ? segment_weight(args, find_expert(args.offsets, args.E, mb * BM)) : 0;
         for (int kt = 0; kt < kt_total; ++kt) {
           if (!mbar_wait(bar_empty(stage), phase ^ 1u, limit, abort_flag)) {
             report_status(args.status, kErrTimeout);
@@ -291,7 +304,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t acc_phase = (uint32_t)((tile_idx >> 1) & 1);
       const int64_t mb = t / args.n_blocks;
       const int nb = (int)(t - mb * args.n_blocks);
-      const int e = grouped ? find_expert(args.offsets, args.E, mb * BM) : 0;
+      const int seg = grouped ? find_expert(args.offsets, args.E, mb * BM) : 0;
+      const int e = grouped ? segment_weight(args, seg) : 0;
       // every lane polls (acquire), and all lanes agree on the outcome before the
       // warp-collective tensor-memory loads
       const bool got = __all_sync(0xffffffffu, mbar_wait(bar_accf(acc), acc_phase, limit, abort_flag));
@@ -307,7 +321,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // with per-expert row counts, rows past the expert's tokens are padding: a 32-row output
       // box that holds no token row is not stored
       const int64_t rows_e = (grouped && args.expert_rows != nullptr)
-                                 ? (int64_t)__ldg(args.offsets + e) + __ldg(args.expert_rows + e)
+                                 ? (int64_t)__ldg(args.offsets + seg) + __ldg(args.expert_rows + seg)
                                  : row_limit;
       const bool row_ok = row < row_limit && row < args.rows_capacity && row < rows_e;
       const float alpha = FP8 ? 1.0f : __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));

@@ -47,8 +47,45 @@ struct RowArgs {
   int32_t* status;
 };
 
+// Activation quantiser fed by bulk copies of row tiles (csrc/quant_act.cu): one shared channel
+// list (or none); the masked and per-group residual variants use the row quantiser above.
+enum { kMapRows = 0, kMapGather = 1, kMapScatter = 2, kMapSegments = 3 };
+struct ActArgs {
+  const uint16_t* src;           // bf16 rows, pitch ld elements
+  int64_t src_rows;
+  int64_t ld;
+  int32_t K, Kp;                 // K % 64 == 0, Kp % 64 == 0
+  int32_t map;                   // kMap*
+  const int32_t* row_gather;     // gather: output row -> source row (< 0: zero row)
+  const int32_t* row_scatter;    // scatter: [src_rows x fanout] output rows (< 0: none)
+  int32_t fanout;                // 1 unless scatter
+  const int32_t* seg_off;        // segments: first row of each segment [n_seg]
+  const int32_t* seg_rows;       // segments: token rows of each segment [n_seg]
+  int32_t n_seg;
+  int64_t rows_out;              // rows (rows_padded) of the outputs
+  int64_t rows_valid;            // rows / gather: output rows >= rows_valid are zero rows
+  const int32_t* sel;            // ascending channel list [Kp]
+  const float* partial;          // amax partials [P] (unless amax_in)
+  int32_t P;
+  const float* amax_in;
+  float* s_g_out;
+  float* s_g_out2;
+  uint8_t* codes;
+  uint8_t* sf;
+  uint8_t* rcodes;
+  uint8_t* rsf;
+  int32_t sf_slab16;
+  int32_t* status;
+  uint64_t wait_limit_ns;
+  int32_t R;                     // set by the launcher
+};
+bool act_plan_choose(int64_t K, int32_t Kp, int fanout, int32_t n_seg, int* R, int* W, int* smem, int force_R = 0,
+                     int force_W = 0);
+cudaError_t launch_act(ActArgs a, int num_sms, int force_R, int force_W, cudaStream_t st);
+
 cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64_t cols, int64_t ld, float* partial,
                         int P, int32_t* status, cudaStream_t st);
+cudaError_t launch_reduce_amax(const float* partial, int P, float* out, cudaStream_t st);
 cudaError_t launch_rows(const RowArgs& a, int num_sms, cudaStream_t st);
 size_t rows_smem_bytes(int64_t K, int32_t Kp, int warps, bool masked = false);
 cudaError_t launch_chan_err(const float* resid, int64_t T, int64_t K, const int32_t* off, int32_t groups,
@@ -57,6 +94,9 @@ cudaError_t launch_select(const double* err, int32_t K, int32_t Kp, int32_t grou
                           cudaStream_t st);
 cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint16_t* out, const float* partial, int P,
                        float* s_g_out, int32_t* status, int num_sms, cudaStream_t st);
+cudaError_t launch_unpack_logical(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t cols, int slab16,
+                                  uint8_t* codes_out, uint8_t* sf_out, int num_sms, cudaStream_t st);
+cudaError_t launch_qdq_backward(const uint16_t* g, int64_t n, uint16_t* gw, float* acc, int num_sms, cudaStream_t st);
 cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
 cudaError_t launch_encode_e4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
 
@@ -93,9 +133,11 @@ struct GemmArgs {
   int32_t kt_main, kt_res;   // k-tiles of 256 elements (last may be partial)
   int32_t N;                 // output columns of the MMA (before the SwiGLU halving)
   int32_t n_blocks;          // N / BN
-  const int32_t* offsets;    // grouped: device [E+1]; dense: nullptr
+  const int32_t* offsets;    // grouped: device [E+1] segment starts; dense: nullptr
   const int32_t* expert_rows;  // grouped, optional device [E]: rows holding tokens per segment
-  int32_t E;
+  int32_t E;                 // grouped: segments (one per expert unless seg_expert is given)
+  const int32_t* seg_expert; // grouped, optional device [E]: weight slab of each segment
+  int32_t n_weights;         // grouped: weight slabs (bound of seg_expert)
   int64_t M;                 // dense: valid rows (stores masked beyond)
   int32_t m_blocks_dense;    // dense: ceil(M/128)
   int64_t rows_capacity;     // rows of the A / Y buffers
@@ -116,6 +158,12 @@ cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_a
                         const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
                         cudaStream_t st);
 size_t gemm_smem_bytes(int bn);
+// CTA-pair form (csrc/gemm2.cu): FP4, N % 256 == 0, W tensor maps with 128-row boxes; grid of
+// n_pairs clusters of two CTAs
+cudaError_t launch_gemm_pair(const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
+                             const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int n_pairs,
+                             cudaStream_t st);
+size_t gemm_pair_smem_bytes();
 
 // ---- swap-AB decode GEMM (weights = MMA A, 16-token slabs = MMA B)
 struct DecodeArgs {

@@ -77,6 +77,12 @@ __device__ __forceinline__ float reduce_partials(const float* partial, int P) {
   return warp_max(m);
 }
 
+// amax of one tensor from its partials, written to a device float (one warp)
+__global__ void reduce_amax_kernel(const float* __restrict__ partial, int P, float* out) {
+  const float m = reduce_partials(partial, P);
+  if (threadIdx.x == 0) *out = m;
+}
+
 // ----------------------------------------------------------------------------------------
 // K2 / K7 / calibration: the row quantiser.  One warp per row, 512 elements per warp
 // iteration: lane l owns the 16-element block [it*512 + 16l, +16), so a block's scale is
@@ -556,6 +562,61 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ w
 }
 
 // ----------------------------------------------------------------------------------------
+// logical view of a packed matrix: one code per byte, scales row-major [rows x cols/16]
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) unpack_logical_kernel(const uint8_t* __restrict__ codes,
+                                                             const uint8_t* __restrict__ sf, int64_t rows,
+                                                             int64_t cols, int slab16, uint8_t* __restrict__ codes_out,
+                                                             uint8_t* __restrict__ sf_out) {
+  const int64_t nblk = cols / 16;
+  const int64_t k64 = cols / 64;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * nblk;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t r = i / nblk, kb = i - r * nblk;
+    if (codes_out) {
+      const uint2 c = *reinterpret_cast<const uint2*>(codes + r * (cols / 2) + kb * 8);
+      const uint32_t w[2] = {c.x, c.y};
+      uint32_t o[4];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // bytes of 4 nibble pairs -> 8 bytes: low nibble first
+        const uint32_t lo = w[h] & 0x0F0F0F0Fu, hi = (w[h] >> 4) & 0x0F0F0F0Fu;
+        o[2 * h] = __byte_perm(lo, hi, 0x5140);
+        o[2 * h + 1] = __byte_perm(lo, hi, 0x7362);
+      }
+      *reinterpret_cast<uint4*>(codes_out + r * cols + kb * 16) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+    if (sf_out) sf_out[r * nblk + kb] = sf[sf_offset_any(r, kb, k64, slab16 != 0)];
+  }
+}
+
+// ----------------------------------------------------------------------------------------
+// trainer fake-quant backward (straight-through): grad_w = grad_fq, grad_acc += grad_fq
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) qdq_backward_kernel(const uint16_t* __restrict__ g, int64_t n,
+                                                           uint16_t* __restrict__ gw, float* __restrict__ acc) {
+  const int64_t n8 = n / 8;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(g) + i);
+    if (gw) reinterpret_cast<uint4*>(gw)[i] = v;
+    if (acc) {
+      float x[8];
+      unpack8(v, x);
+      float4* a = reinterpret_cast<float4*>(acc) + 2 * i;
+      const float4 a0 = a[0], a1 = a[1];
+      a[0] = make_float4(__fadd_rn(a0.x, x[0]), __fadd_rn(a0.y, x[1]), __fadd_rn(a0.z, x[2]), __fadd_rn(a0.w, x[3]));
+      a[1] = make_float4(__fadd_rn(a1.x, x[4]), __fadd_rn(a1.y, x[5]), __fadd_rn(a1.z, x[6]), __fadd_rn(a1.w, x[7]));
+    }
+  }
+  // the tail (n % 8 elements), one thread each
+  const int64_t t = n8 * 8 + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (t < n) {
+    if (gw) gw[t] = g[t];
+    if (acc) acc[t] = __fadd_rn(acc[t], bf16_bits_to_f32(g[t]));
+  }
+}
+
+// ----------------------------------------------------------------------------------------
 // codec test kernels
 // ----------------------------------------------------------------------------------------
 __global__ void encode_e2m1_kernel(const float* v, int64_t n, uint8_t* out) {
@@ -582,6 +643,11 @@ cudaError_t launch_amax(const uint16_t* x, int64_t segs, int64_t seg_rows, int64
                         int P, int32_t* status, cudaStream_t st) {
   dim3 grid(P, (unsigned)segs);
   amax_kernel<<<grid, 256, 0, st>>>(x, seg_rows, cols, ld, partial, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_reduce_amax(const float* partial, int P, float* out, cudaStream_t st) {
+  reduce_amax_kernel<<<1, 32, 0, st>>>(partial, P, out);
   return cudaGetLastError();
 }
 
@@ -666,6 +732,24 @@ cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint
   if (grid > cap) grid = cap;
   if (grid < 1) grid = 1;
   qdq_kernel<<<(unsigned)grid, 256, 0, st>>>(w, n_tensors, elems, out, partial, P, s_g_out, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_logical(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t cols, int slab16,
+                                  uint8_t* codes_out, uint8_t* sf_out, int num_sms, cudaStream_t st) {
+  const int64_t work = rows * (cols / 16);
+  int64_t grid = (work + 255) / 256;
+  if (grid > (int64_t)num_sms * 16) grid = (int64_t)num_sms * 16;
+  if (grid < 1) grid = 1;
+  unpack_logical_kernel<<<(unsigned)grid, 256, 0, st>>>(codes, sf, rows, cols, slab16, codes_out, sf_out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qdq_backward(const uint16_t* g, int64_t n, uint16_t* gw, float* acc, int num_sms, cudaStream_t st) {
+  int64_t grid = (n / 8 + 255) / 256;
+  if (grid > (int64_t)num_sms * 8) grid = (int64_t)num_sms * 8;
+  if (grid < 1) grid = 1;
+  qdq_backward_kernel<<<(unsigned)grid, 256, 0, st>>>(g, n, gw, acc);
   return cudaGetLastError();
 }
 

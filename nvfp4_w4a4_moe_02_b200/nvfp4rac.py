@@ -61,9 +61,13 @@ def load() -> ctypes.CDLL:
         "nvfp4_kp_from_ratio": ([i64, ctypes.c_double], i32),
         "nvfp4_set_wait_limit_ns": ([u64], None),
         "nvfp4_set_gemm_tile_n": ([i32], None),
+        "nvfp4_set_act_tile": ([i32, i32], None),
+        "nvfp4_set_gemm_pairs": ([i32], None),
         "nvfp4_quantize_workspace_size": ([i64, i64], sz),
         "nvfp4_quantize": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
         "nvfp4_quantize_scatter": ([vp, i64, i64, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "nvfp4_quantize_segments": ([vp, i64, i64, i64, vp, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp],
+                                    ctypes.c_int),
         "nvfp4_quantize_grouped_sel": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp],
                                        ctypes.c_int),
         "rac_calibrate_workspace_size": ([i64, i64], sz),
@@ -77,6 +81,9 @@ def load() -> ctypes.CDLL:
         "w4a4_rac_gemm": ([tp, tp, tp, tp, i64, i64, i64, i32, ctypes.c_int, vp, i64, vp, vp], ctypes.c_int),
         "grouped_w4a4_rac_moe": ([tp, tp, vp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, i64,
                                   vp, vp, vp], ctypes.c_int),
+        "grouped_w4a4_rac_moe_segments": ([tp, tp, vp, vp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int,
+                                           ctypes.c_int, vp, i64, vp, vp, vp], ctypes.c_int),
+        "nvfp4_amax": ([vp, i64, i64, i64, vp, vp, sz, vp, vp], ctypes.c_int),
         "grouped_w4a4_rac_moe_decode": ([tp, tp, vp, vp, i32, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int,
                                          vp, i64, vp, vp, vp], ctypes.c_int),
         "moe_route_topk": ([vp, i64, i32, i32, vp, vp, vp, vp], ctypes.c_int),
@@ -86,6 +93,8 @@ def load() -> ctypes.CDLL:
         "moe_combine": ([vp, i64, i64, vp, vp, i64, i32, i64, vp, i64, vp, vp], ctypes.c_int),
         "weight_qdq_workspace_size": ([i64, i64], sz),
         "weight_qdq": ([vp, i64, i64, vp, vp, vp, sz, vp, vp], ctypes.c_int),
+        "weight_qdq_backward": ([vp, i64, vp, vp, vp], ctypes.c_int),
+        "nvfp4_unpack_logical": ([tp, i64, vp, vp, vp], ctypes.c_int),
         "nvfp4_encode_e2m1": ([vp, i64, vp, vp], ctypes.c_int),
         "nvfp4_encode_e4m3": ([vp, i64, vp, vp], ctypes.c_int),
         "nvfp4_selftest_wait_timeout": ([u64, vp, vp], ctypes.c_int),
@@ -159,6 +168,14 @@ class Packed:
         return CTensor(self.codes.data_ptr(), self.sf.data_ptr(), self.s_g.data_ptr(), self.slabs, self.rows,
                        self.rows_padded, self.cols, self.sf_layout)
 
+    def prefix(self, rows_padded: int) -> "Packed":
+        """View of the first rows_padded rows (a multiple of the scale layout's row group) of a
+        single-slab tensor, sharing storage."""
+        group = 16 if self.sf_layout == SF_SLAB16 else 128
+        assert self.slabs == 1 and rows_padded % group == 0 and rows_padded <= self.rows_padded
+        return Packed(self.codes[:rows_padded * self.cols // 2], self.sf[:sf_bytes(rows_padded, self.cols, self.sf_layout)],
+                      self.s_g, 1, min(self.rows, rows_padded), rows_padded, self.cols, self.sf_layout)
+
     def slab(self, e: int) -> "Packed":
         """View of slab e alone (slabs = 1), sharing storage (e.g. to pack one expert at a time)."""
         cb = self.rows_padded * self.cols // 2
@@ -211,6 +228,17 @@ def set_wait_limit_ns(ns: int):
 def set_gemm_tile_n(n: int):
     """Force the GEMM N-tile (128 or 256); 0 restores the automatic choice."""
     load().nvfp4_set_gemm_tile_n(n)
+
+
+def set_gemm_pairs(on: bool):
+    """Run the GEMMs with N % 256 == 0 on CTA pairs (default) or on single SMs."""
+    load().nvfp4_set_gemm_pairs(1 if on else 0)
+
+
+def set_act_tile(rows: int, warps: int):
+    """Force the activation quantiser's rows per tile and consumer warps; 0, 0 restores the
+    automatic choice."""
+    load().nvfp4_set_act_tile(rows, warps)
 
 
 # ------------------------------------------------------------------------------------- calls
@@ -283,6 +311,35 @@ def nvfp4_quantize_scatter(x: torch.Tensor, row_scatter: torch.Tensor, rows_padd
     _check(lib.nvfp4_quantize_scatter(x.data_ptr(), M, K, x.stride(0), row_scatter.data_ptr(), fanout, _ptr(sel), Kp,
                                       _ptr(amax_in), ctypes.byref(q), ctypes.byref(qr) if qr is not None else None,
                                       ws.data_ptr(), ws.numel(), st.data_ptr(), _stream(stream)))
+    return out, (out_res if Kp > 0 else None)
+
+
+def nvfp4_quantize_segments(x: torch.Tensor, expert_offsets: torch.Tensor, expert_rows: torch.Tensor,
+                            sel: torch.Tensor | None = None, amax_in: torch.Tensor | None = None,
+                            out: Packed | None = None, out_res: Packed | None = None,
+                            status: torch.Tensor | None = None, stream=None):
+    """Quantise only the token rows of an expert-grouped layout: rows
+    [expert_offsets[e], expert_offsets[e] + expert_rows[e]) of x (device int32 [E] each) into the
+    same rows of the outputs; other output rows are left as they are.  Returns (Packed, Packed | None)."""
+    lib = load()
+    _u16(x)
+    M, K = x.shape
+    assert x.stride(1) == 1
+    assert expert_offsets.dtype == torch.int32 and expert_rows.dtype == torch.int32
+    E = int(expert_rows.numel())
+    Kp = 0 if sel is None else int(sel.numel())
+    if out is None:
+        out = Packed.empty(M, K, device=x.device, zero=True)
+    if Kp > 0 and out_res is None:
+        out_res = Packed.empty(M, Kp, rows_padded=out.rows_padded, device=x.device, zero=True)
+    ws = _workspace(x.device).get(lib.nvfp4_quantize_workspace_size(M, K))
+    st = status if status is not None else new_status(x.device)
+    q = out.c()
+    qr = out_res.c() if Kp > 0 else None
+    _check(lib.nvfp4_quantize_segments(x.data_ptr(), M, K, x.stride(0), expert_offsets.data_ptr(),
+                                       expert_rows.data_ptr(), E, _ptr(sel), Kp, _ptr(amax_in), ctypes.byref(q),
+                                       ctypes.byref(qr) if qr is not None else None, ws.data_ptr(), ws.numel(),
+                                       st.data_ptr(), _stream(stream)))
     return out, (out_res if Kp > 0 else None)
 
 
@@ -408,6 +465,50 @@ def grouped_w4a4_rac_moe(a: Packed, a_res: Packed | None, expert_offsets: torch.
     return (y, amax_out) if swiglu else y
 
 
+def grouped_w4a4_rac_moe_segments(a: Packed, a_res: Packed | None, seg_offsets: torch.Tensor,
+                                  seg_rows: torch.Tensor | None, seg_expert: torch.Tensor, w: Packed,
+                                  w_sel: Packed | None, swiglu: bool = False, out_dtype=torch.bfloat16,
+                                  y: torch.Tensor | None = None, amax_out: torch.Tensor | None = None,
+                                  status: torch.Tensor | None = None, stream=None):
+    """Grouped GEMM over row segments [seg_offsets[i], seg_offsets[i+1]) with weight slab
+    seg_expert[i] (device int32 tensors) -> y [and the amax of the SwiGLU output]."""
+    lib = load()
+    N, K = w.rows, w.cols
+    Kp = 0 if a_res is None else a_res.cols
+    n_seg = int(seg_expert.numel())
+    assert seg_offsets.dtype == torch.int32 and seg_expert.dtype == torch.int32 and seg_offsets.numel() >= n_seg + 1
+    ycols = N // 2 if swiglu else N
+    if y is None:
+        y = torch.empty(a.rows_padded, ycols, dtype=torch.bfloat16 if swiglu else out_dtype, device=a.codes.device)
+    if swiglu and amax_out is None:
+        amax_out = torch.empty(1, dtype=torch.float32, device=a.codes.device)
+    od = OUT_BF16 if y.dtype == torch.bfloat16 else OUT_F32
+    st = status if status is not None else new_status(a.codes.device)
+    ca, cw = a.c(), w.c()
+    car = a_res.c() if Kp > 0 else None
+    cws = w_sel.c() if Kp > 0 else None
+    _check(lib.grouped_w4a4_rac_moe_segments(ctypes.byref(ca), ctypes.byref(car) if car else None,
+                                             seg_offsets.data_ptr(), _ptr(seg_rows), seg_expert.data_ptr(), n_seg,
+                                             ctypes.byref(cw), ctypes.byref(cws) if cws else None, N, K, Kp,
+                                             EPI_SWIGLU_AMAX if swiglu else EPI_NONE, od, y.data_ptr(), y.stride(0),
+                                             _ptr(amax_out), st.data_ptr(), _stream(stream)))
+    return (y, amax_out) if swiglu else y
+
+
+def nvfp4_amax(x: torch.Tensor, out: torch.Tensor | None = None, status: torch.Tensor | None = None, stream=None):
+    """max |x| of a bf16 matrix into a device float32 [1]."""
+    lib = load()
+    _u16(x)
+    M, K = x.shape
+    assert x.stride(1) == 1
+    out = torch.empty(1, dtype=torch.float32, device=x.device) if out is None else out
+    ws = _workspace(x.device).get(lib.nvfp4_quantize_workspace_size(M, K))
+    st = status if status is not None else new_status(x.device)
+    _check(lib.nvfp4_amax(x.data_ptr(), M, K, x.stride(0), out.data_ptr(), ws.data_ptr(), ws.numel(), st.data_ptr(),
+                          _stream(stream)))
+    return out
+
+
 def grouped_w4a4_rac_moe_decode(a: Packed, a_res: Packed | None, slot_expert: torch.Tensor,
                                 slot_count: torch.Tensor, w: Packed, w_sel: Packed | None, swiglu: bool = False,
                                 out_dtype=torch.bfloat16, y: torch.Tensor | None = None,
@@ -516,6 +617,48 @@ def weight_qdq(w: torch.Tensor, out: torch.Tensor | None = None, s_g: torch.Tens
     return out, s_g
 
 
+def weight_qdq_backward(grad_fq: torch.Tensor, grad_w: torch.Tensor | None = None,
+                        grad_acc: torch.Tensor | None = None, stream=None):
+    """Straight-through gradient of the fake-quant: grad_w = grad_fq (bf16) and/or
+    grad_acc += grad_fq (float32 master gradient)."""
+    lib = load()
+    _u16(grad_fq)
+    assert grad_fq.is_contiguous()
+    if grad_w is None and grad_acc is None:
+        grad_w = torch.empty_like(grad_fq)
+    if grad_acc is not None:
+        assert grad_acc.dtype == torch.float32 and grad_acc.is_contiguous() and grad_acc.numel() == grad_fq.numel()
+    _check(lib.weight_qdq_backward(grad_fq.data_ptr(), grad_fq.numel(), _ptr(grad_w), _ptr(grad_acc),
+                                   _stream(stream)))
+    return grad_w if grad_w is not None else grad_acc
+
+
+class FakeQuantSTE(torch.autograd.Function):
+    """W -> bf16(DQ(Q(W))) per tensor in the forward pass (weight_qdq), the straight-through
+    gradient in the backward pass (weight_qdq_backward): the trainer side of the shared
+    quantise-dequantise path."""
+
+    @staticmethod
+    def forward(ctx, w):
+        out, _ = weight_qdq(w.contiguous())
+        return out
+
+    @staticmethod
+    def backward(ctx, g):
+        return weight_qdq_backward(g.contiguous())
+
+
+def unpack_logical(p: Packed, slab: int = 0, stream=None):
+    """Codes (uint8 [rows, cols], one per byte) and block scales (uint8 [rows, cols/16]) of one
+    slab of a packed tensor, in logical order, made by the library's unpack kernel."""
+    lib = load()
+    codes = torch.empty(p.rows, p.cols, dtype=torch.uint8, device=p.codes.device)
+    sf = torch.empty(p.rows, p.cols // 16, dtype=torch.uint8, device=p.codes.device)
+    c = p.c()
+    _check(lib.nvfp4_unpack_logical(ctypes.byref(c), slab, codes.data_ptr(), sf.data_ptr(), _stream(stream)))
+    return codes, sf
+
+
 def encode_e2m1(v: torch.Tensor, stream=None) -> torch.Tensor:
     out = torch.empty(v.numel(), dtype=torch.uint8, device=v.device)
     _check(load().nvfp4_encode_e2m1(v.data_ptr(), v.numel(), out.data_ptr(), _stream(stream)))
@@ -530,66 +673,3 @@ def encode_e4m3(v: torch.Tensor, stream=None) -> torch.Tensor:
 
 def selftest_wait_timeout(limit_ns: int, status: torch.Tensor, stream=None):
     _check(load().nvfp4_selftest_wait_timeout(limit_ns, status.data_ptr(), _stream(stream)))
-
-
-# ------------------------------------------------------------------------------------- MoE host logic
-def expert_layout(counts, pad: int = 128):
-    """Padded expert segments for a token-sorted pair list.
-
-    counts: pairs per expert.  Returns (offsets_padded [E+1] int64, rows_padded_total, pair_rows [P]) where
-    pair_rows maps the i-th (expert, token)-sorted pair to its row in the padded layout.
-    """
-    import numpy as np
-
-    counts = np.asarray(counts, dtype=np.int64)
-    padded = (counts + pad - 1) // pad * pad
-    off = np.zeros(counts.size + 1, dtype=np.int64)
-    off[1:] = np.cumsum(padded)
-    starts = off[:-1]
-    pair_rows = np.concatenate([starts[e] + np.arange(c) for e, c in enumerate(counts)]) if counts.sum() else \
-        np.zeros(0, np.int64)
-    return off, int(off[-1]), pair_rows
-
-
-def gather_map(pair_token, counts, pad: int = 128):
-    """row_gather [rows_padded] (source token of each padded row, -1 for padding) and offsets."""
-    import numpy as np
-
-    off, total, pair_rows = expert_layout(counts, pad)
-    g = np.full(total, -1, dtype=np.int32)
-    g[pair_rows] = np.asarray(pair_token, dtype=np.int32)
-    return g, off, pair_rows
-
-
-def scatter_map(pair_token, pair_rows, T: int, fanout: int):
-    """row_scatter [T, fanout]: the padded rows of each token's (token, expert) pairs, -1 padded."""
-    import numpy as np
-
-    m = np.full((T, fanout), -1, dtype=np.int32)
-    fill = np.zeros(T, dtype=np.int64)
-    for t, r in zip(np.asarray(pair_token), np.asarray(pair_rows)):
-        m[t, fill[t]] = r
-        fill[t] += 1
-    return m
-
-
-def decode_slots(counts, slab: int = 16):
-    """16-token slabs for a decode step's (expert, token)-sorted pair list.
-
-    counts: pairs per expert.  Returns (slot_expert [S] int32, slot_count [S] int32, pair_rows [P] int64)
-    where expert e's pairs fill ceil(counts[e] / 16) consecutive slabs and pair i lands in row
-    16 * slot + j of the slab layout.
-    """
-    import numpy as np
-
-    counts = np.asarray(counts, dtype=np.int64)
-    slot_expert, slot_count, pair_rows = [], [], []
-    for e, c in enumerate(counts):
-        for k in range(0, int(c), slab):
-            n = min(slab, int(c) - k)
-            base = len(slot_expert) * slab
-            slot_expert.append(e)
-            slot_count.append(n)
-            pair_rows.extend(range(base, base + n))
-    return (np.asarray(slot_expert, dtype=np.int32), np.asarray(slot_count, dtype=np.int32),
-            np.asarray(pair_rows, dtype=np.int64))

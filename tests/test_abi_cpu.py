@@ -208,7 +208,7 @@ def test_fp8_path_rejections(lib):
 
 
 def test_decode_slots_host_logic():
-    from nvfp4_w4a4_moe_02_b200.nvfp4rac import decode_slots
+    from nvfp4_layout import decode_slots
 
     counts = [0, 3, 16, 17, 0, 1, 40]
     se, sc, rows = decode_slots(counts)

@@ -8,6 +8,7 @@ import torch
 
 from nvfp4_w4a4_moe_02_b200 import mxfp8 as F
 from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+import nvfp4_layout as L
 from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 from test_gpu_parity import assert_gemm_close, bf16_bits, bf16_ulp, to_dev
 
@@ -112,13 +113,13 @@ def test_fp8_gemm_matches_oracle(dev, orc, M, N, K, bf16):
 def test_fp8_moe_block_matches_oracle(dev, orc):
     """gate_up (SwiGLU epilogue) and down on FP8 operands over ragged expert segments."""
     wl = syn.moe_block(T=96, H=512, E=8, topk=2, I=128, T_cal=64)
-    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    g, off, pair_rows = L.gather_map(wl.pair_token, wl.counts)
     offd = torch.from_numpy(off.astype(np.int32)).to(dev)
     rows = torch.from_numpy(np.asarray(wl.counts, np.int32)).to(dev)
     st = R.new_status(dev)
     wgu = F.pack_weights(to_dev(wl.wgu, dev), gate_up_interleave=True, status=st)
     wdn = F.pack_weights(to_dev(wl.wdn, dev), status=st)
-    sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
+    sm = torch.from_numpy(L.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
     a = F.quantize_scatter(to_dev(wl.x, dev), sm, g.size, status=st)
     # padding-only output boxes are skipped: h starts zeroed so its padding rows stay finite zeros
     h = torch.zeros(g.size, wl.I, dtype=torch.bfloat16, device=dev)

@@ -11,6 +11,7 @@ import pytest
 import torch
 
 from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+import nvfp4_layout as L
 from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 from test_gpu_parity import bf16_bits, bf16_ulp, decode_pipeline, moe_pipeline, pack_host_weights, to_dev
 
@@ -84,7 +85,7 @@ def test_dispatch_plan_matches_oracle(dev, orc, pad):
     assert np.array_equal(rows.cpu().numpy(), rows_ref)
     if pad == 16:
         counts = np.bincount(ids_ref.reshape(-1), minlength=E)
-        se_ref, sc_ref, _ = R.decode_slots(counts)
+        se_ref, sc_ref, _ = L.decode_slots(counts)
         se_g, sc_g = se.cpu().numpy(), sc.cpu().numpy()
         assert np.array_equal(se_g[:se_ref.size], se_ref) and np.array_equal(sc_g[:sc_ref.size], sc_ref)
         assert np.all(se_g[se_ref.size:] == -1) and np.all(sc_g[se_ref.size:] == 0)

@@ -10,6 +10,7 @@ import pytest
 import torch
 
 from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+import nvfp4_layout as L
 from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 from nvfp4_layout import unpack_codes, unpack_sf
 
@@ -103,6 +104,41 @@ def test_codec_e4m3_matches_oracle(dev, orc):
     assert bad.size == 0, [(float(arr[i]), int(got[i]), int(ref[i])) for i in bad[:8]]
 
 
+def _bit_patterns(lo: int, n: int, dev):
+    """float32 values with the bit patterns lo .. lo + n - 1 (as int32), on the device and on the host."""
+    d = torch.arange(lo, lo + n, dtype=torch.int64, device=dev).to(torch.int32).view(torch.float32)
+    h = np.arange(lo, lo + n, dtype=np.int64).astype(np.int32).view(np.float32)
+    return d, h
+
+
+def test_codec_e2m1_exhaustive(dev, orc):
+    """The device E2M1 encoder (the conversion instruction the quantisers use) against the
+    oracle's nearest-with-ties-to-even encoder on every float32 bit pattern except NaNs (the
+    quantisers never convert a NaN: a non-finite input is an error of the call)."""
+    chunk = 1 << 26
+    for lo in range(-(1 << 31), 1 << 31, chunk):
+        vd, vh = _bit_patterns(lo, chunk, dev)
+        got = R.encode_e2m1(vd).cpu().numpy()
+        ref = orc.e2m1_encode_array(vh)
+        bad = np.nonzero((got != ref) & ~np.isnan(vh))[0]
+        assert bad.size == 0, [(hex(int(vh[i:i + 1].view(np.uint32)[0])), int(got[i]), int(ref[i])) for i in bad[:8]]
+
+
+def test_codec_e4m3_exhaustive_scale_range(dev, orc):
+    """The device E4M3 scale encoder against the oracle on every non-negative float32 up to 2^9
+    (bit patterns 0 .. 0x44000000): the scale rule feeds it RN(b / RN(6 s_g)) <= 448 (up to
+    rounding), so this covers every input it can receive, saturation included."""
+    end = 0x44000000 + 1
+    chunk = 1 << 26
+    for lo in range(0, end, chunk):
+        n = min(chunk, end - lo)
+        vd, vh = _bit_patterns(lo, n, dev)
+        got = R.encode_e4m3(vd).cpu().numpy()
+        ref = orc.e4m3_encode_array(vh)
+        bad = np.nonzero(got != ref)[0]
+        assert bad.size == 0, [(float(vh[i]), int(got[i]), int(ref[i])) for i in bad[:8]]
+
+
 # ------------------------------------------------------------------------------------------ quantiser
 def check_act_quant(dev, orc, x: np.ndarray, sel: np.ndarray, rows_padded=None):
     xd = to_dev(x, dev)
@@ -158,7 +194,7 @@ def test_quantize_dense_prefill_full(dev, orc):
 
 def test_quantize_row_gather(dev, orc):
     wl = syn.moe_block(T=300, H=1024, E=16, topk=4, I=256, T_cal=64, materialize_weights=False)
-    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    g, off, pair_rows = L.gather_map(wl.pair_token, wl.counts)
     xd = to_dev(wl.x, dev)
     sel = np.arange(1, 1024, 2, dtype=np.int32)
     gd = torch.from_numpy(g).to(dev)
@@ -179,8 +215,8 @@ def test_quantize_scatter_matches_gather(dev, orc):
     """Scatter mode (each token quantised once, written to its expert rows) gives the same bytes
     as the gather mode and as the oracle; unnamed (padding) rows stay zero."""
     wl = syn.moe_block(T=300, H=1024, E=16, topk=4, I=256, T_cal=64, materialize_weights=False)
-    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
-    sm = R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], 4)
+    g, off, pair_rows = L.gather_map(wl.pair_token, wl.counts)
+    sm = L.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], 4)
     xd = to_dev(wl.x, dev)
     sel = np.arange(3, 1024, 2, dtype=np.int32)[:448]
     seld = torch.from_numpy(sel).to(dev)
@@ -363,15 +399,30 @@ def test_gemm_ragged_shapes(dev, orc, M, N, K, Kp):
     run_dense(dev, orc, x, w, x_cal, Kp, torch.bfloat16)
 
 
+def tile_order_blocks(m_blocks: int, n_blocks: int, grid: int = 148):
+    """128-row m-blocks spread over a persistent GEMM's tile order (grid CTAs; tile
+    t = m_block * n_blocks + n_block runs on CTA t % grid as its (t // grid)-th tile, into
+    accumulator buffer (t // grid) % 2): the first and the last m-block, the middle one, and the
+    m-blocks holding the first tiles of the CTAs' second and third turns."""
+    picks = {0, m_blocks - 1, m_blocks // 2}
+    for turn in (1, 2):
+        picks.add(min(m_blocks - 1, (turn * grid + n_blocks - 1) // n_blocks))
+    return sorted(picks)
+
+
 def test_gemm_dense_prefill_sampled(dev, orc):
+    """The dense prefill projection at full size: every row of whole m-blocks spread over the
+    tile order (both accumulator buffers, first and last tiles of CTAs)."""
     wl = syn.dense_prefill()
-    rows = np.array([0, 1, 127, 128, 1000, 4095, 4096, 6000, 8190, 8191])
+    blocks = tile_order_blocks(wl.M // 128, wl.N // 256)
+    assert len(blocks) >= 4
+    rows = np.concatenate([np.arange(128 * b, 128 * b + 128) for b in blocks])
     run_dense(dev, orc, wl.x, wl.w, wl.x_cal, wl.Kp, torch.bfloat16, rows=rows)
 
 
 # ------------------------------------------------------------------------------------------ MoE
 def moe_pipeline(dev, wl, sel_gu, sel_dn):
-    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    g, off, pair_rows = L.gather_map(wl.pair_token, wl.counts)
     st = R.new_status(dev)
     offd = torch.from_numpy(off.astype(np.int32)).to(dev)
     wgu = to_dev(wl.wgu, dev)
@@ -380,7 +431,7 @@ def moe_pipeline(dev, wl, sel_gu, sel_dn):
     seld_dn = torch.from_numpy(np.ascontiguousarray(sel_dn)).to(dev)  # 2-D: one list per expert
     pgu, pgus = R.pack_weights(wgu, seld_gu, gate_up_interleave=True, status=st)
     pdn, pdns = R.pack_weights(wdn, seld_dn, status=st)
-    sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
+    sm = torch.from_numpy(L.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
     a, ar = R.nvfp4_quantize_scatter(to_dev(wl.x, dev), sm, g.size, seld_gu, status=st)
     h, amax_h = R.grouped_w4a4_rac_moe(a, ar, offd, pgu, pgus, swiglu=True, status=st)
     row_group = R.moe_row_groups(offd, wl.E, g.size) if seld_dn.dim() == 2 else None
@@ -410,7 +461,8 @@ def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs, wgu_of=None, wdn_of=No
     s_h = orc.global_scale(np.float32(out["amax_h"].item()))
     assert out["hq"].s_g.item() == float(s_h)
     gq_c, gq_S = logical(out["hq"], rows=out["hq"].rows_padded)
-    gqr_c, gqr_S = logical(out["hqr"], rows=out["hqr"].rows_padded)
+    if out["hqr"] is not None:
+        gqr_c, gqr_S = logical(out["hqr"], rows=out["hqr"].rows_padded)
     for e in sorted(set(int(wl.pair_expert[i]) for i in sample_pairs)):
         pidx = [i for i in sample_pairs if wl.pair_expert[i] == e]
         rows = out["pair_rows"][pidx]
@@ -439,7 +491,10 @@ def check_moe(orc, wl, sel_gu, sel_dn, out, sample_pairs, wgu_of=None, wdn_of=No
         hrows = h_gpu[rows]
         hc, hS, hrc, hrS, _ = orc.act_quant_rac(hrows, s_h, sel_e)
         assert np.array_equal(gq_c[rows], hc) and np.array_equal(gq_S[rows], hS)
-        assert np.array_equal(gqr_c[rows], hrc) and np.array_equal(gqr_S[rows], hrS)
+        if out["hqr"] is not None:
+            assert np.array_equal(gqr_c[rows], hrc) and np.array_equal(gqr_S[rows], hrS)
+        else:
+            assert len(sel_e) == 0
         wdn = wdn_of(e)
         s_wd = orc.global_scale(orc.amax_bf16(wdn))
         dc, dS, dsc, dsS = orc.weight_pack(wdn, s_wd, sel_e)
@@ -523,7 +578,7 @@ def test_grouped_expert_rows_skips_padding_boxes(dev, orc):
     wl = syn.moe_block(T=300, H=512, E=6, topk=2, I=128, T_cal=64)
     sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
     st = R.new_status(dev)
-    g, off, pair_rows = R.gather_map(wl.pair_token, wl.counts)
+    g, off, pair_rows = L.gather_map(wl.pair_token, wl.counts)
     seld = torch.from_numpy(sel_gu).to(dev)
     a, ar = R.nvfp4_quantize(to_dev(wl.x, dev), seld, row_gather=torch.from_numpy(g).to(dev), M_out=g.size, status=st)
     w, ws = R.pack_weights(to_dev(wl.wgu, dev), seld, gate_up_interleave=True, status=st)
@@ -549,7 +604,17 @@ def test_grouped_expert_rows_skips_padding_boxes(dev, orc):
             assert np.all(yn[lo + n:live_end] == 0.0), e               # padding rows of live boxes
 
 
+def whole_block_pairs(pair_rows: np.ndarray, rows_padded: int, n_blocks: int, grid: int = 148):
+    """The (token, expert) pairs whose rows lie in the m-blocks tile_order_blocks picks for the
+    grouped GEMM: every token row of those blocks."""
+    picks = tile_order_blocks(rows_padded // 128, n_blocks, grid)
+    pairs = np.nonzero(np.isin(pair_rows // 128, picks))[0]
+    return picks, pairs.tolist()
+
+
 def test_moe_prefill_full_sampled(dev, orc):
+    """The MoE prefill block at full size, r = 0.5: every row of whole m-blocks spread over the
+    tile order (both accumulator buffers, first and last tiles) plus random pairs."""
     wl = syn.moe_prefill()
     sel_gu, _ = orc.calibrate(wl.x_cal, wl.Kp_gu)
     h_cal = syn.moe_down_calibration_batch(wl)
@@ -557,8 +622,31 @@ def test_moe_prefill_full_sampled(dev, orc):
     out = moe_pipeline(dev, wl, sel_gu, sel_dn)
     rng = np.random.default_rng(0)
     P = wl.pair_token.size
-    sample = sorted(set(rng.choice(P, 96, replace=False).tolist() + [0, P - 1]))
+    blocks, pairs = whole_block_pairs(out["pair_rows"], out["g"].size, 1536 // 256)
+    assert len(blocks) >= 4 and len(pairs) >= 3 * 100
+    sample = sorted(set(rng.choice(P, 96, replace=False).tolist() + [0, P - 1] + pairs))
     check_moe(orc, wl, sel_gu, sel_dn, out, sample)
+
+
+@pytest.mark.parametrize("r", [0.0, 0.25, 1.0])
+def test_moe_prefill_ratio_sweep_matches_oracle(dev, orc, r):
+    """The RAC ratio sweep on the MoE prefill shapes (r = 0 is plain W4A4, K' = 0 in both GEMMs;
+    r = 0.25 gives K' = 512 / 192, a partial last residual k-tile in the down GEMM; r = 1 the
+    residual over every channel): every row of whole m-blocks spread over the tile order
+    against the oracle, as at r = 0.5."""
+    import dataclasses
+
+    base = syn.moe_prefill()
+    wl = dataclasses.replace(base, r=r, Kp_gu=syn.kp_from_ratio(base.H, r), Kp_dn=syn.kp_from_ratio(base.I, r))
+    empty = np.zeros(0, np.int32)
+    sel_gu = orc.calibrate(wl.x_cal, wl.Kp_gu)[0] if wl.Kp_gu else empty
+    sel_dn = orc.calibrate(syn.moe_down_calibration_batch(wl), wl.Kp_dn)[0] if wl.Kp_dn else empty
+    out = moe_pipeline(dev, wl, sel_gu, sel_dn)
+    if wl.Kp_gu == 0:
+        assert out["ar"] is None and out["hqr"] is None
+    blocks, pairs = whole_block_pairs(out["pair_rows"], out["g"].size, 1536 // 256)
+    assert len(blocks) >= 4
+    check_moe(orc, wl, sel_gu, sel_dn, out, pairs + [0, wl.pair_token.size - 1])
 
 
 # ------------------------------------------------------------------------------------------ MoE decode
@@ -568,13 +656,13 @@ def decode_pipeline(dev, wl, sel_gu, sel_dn, packed, counts=None):
     st = R.new_status(dev)
     pgu, pgus, pdn, pdns = packed
     counts = wl.counts if counts is None else counts
-    se, sc, pair_rows = R.decode_slots(counts)
+    se, sc, pair_rows = L.decode_slots(counts)
     rows = 16 * se.size
     sed = torch.from_numpy(se).to(dev)
     scd = torch.from_numpy(sc).to(dev)
     seld_gu = torch.from_numpy(sel_gu).to(dev) if sel_gu.size else None
     seld_dn = torch.from_numpy(sel_dn).to(dev) if sel_dn.size else None
-    sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
+    sm = torch.from_numpy(L.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], wl.topk_ids.shape[1])).to(dev)
     a, ar = R.nvfp4_quantize_scatter(to_dev(wl.x, dev), sm, rows, seld_gu, status=st, sf_layout=R.SF_SLAB16)
     h, amax_h = R.grouped_w4a4_rac_moe_decode(a, ar, sed, scd, pgu, pgus, swiglu=True, status=st)
     hq = R.Packed.empty(rows, wl.I, rows_padded=rows, device=dev, sf_layout=R.SF_SLAB16)
@@ -636,8 +724,8 @@ def test_decode_plain_epilogue_fp32(dev, orc, r):
     st = R.new_status(dev)
     seld = torch.from_numpy(sel).to(dev) if Kp else None
     w, ws = R.pack_weights(to_dev(wl.wgu, dev), seld, status=st)
-    se, sc, pair_rows = R.decode_slots(wl.counts)
-    sm = torch.from_numpy(R.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], 2)).to(dev)
+    se, sc, pair_rows = L.decode_slots(wl.counts)
+    sm = torch.from_numpy(L.scatter_map(wl.pair_token, pair_rows, wl.x.shape[0], 2)).to(dev)
     a, ar = R.nvfp4_quantize_scatter(to_dev(wl.x, dev), sm, 16 * se.size, seld, status=st, sf_layout=R.SF_SLAB16)
     y = R.grouped_w4a4_rac_moe_decode(a, ar, torch.from_numpy(se).to(dev), torch.from_numpy(sc).to(dev), w, ws,
                                       out_dtype=torch.float32, status=st)

@@ -4,6 +4,7 @@ projection's calibration rows."""
 import numpy as np
 
 from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
+import nvfp4_layout as L
 from nvfp4_w4a4_moe_02_b200 import synthetic as syn
 
 
@@ -14,21 +15,21 @@ def test_gather_and_scatter_maps_describe_the_same_padded_layout():
     ids[ids == 5] = 4  # expert 5 gets nothing
     ids[:, 1] = np.where(ids[:, 1] == ids[:, 0], (ids[:, 0] + 1) % 5, ids[:, 1])
     pt, pe, counts = syn.sort_pairs(ids, E)
-    g, off, pair_rows = R.gather_map(pt, counts)
+    g, off, pair_rows = L.gather_map(pt, counts)
     assert off[0] == 0 and np.all(np.diff(off) % 128 == 0) and counts[5] == 0 and off[6] == off[5]
     for e in range(E):  # each expert's pairs fill the head of its 128-padded segment, in order
         rows = pair_rows[pe == e]
         assert np.array_equal(rows, off[e] + np.arange(counts[e]))
         assert np.all(g[off[e] + counts[e]:off[e + 1]] == -1)
     assert np.array_equal(g[pair_rows], pt)
-    sm = R.scatter_map(pt, pair_rows, T, k)
+    sm = L.scatter_map(pt, pair_rows, T, k)
     for t in range(T):  # a token's scatter rows are exactly the rows whose gather source is t
         assert sorted(sm[t][sm[t] >= 0].tolist()) == sorted(np.nonzero(g == t)[0].tolist())
 
 
 def test_decode_slots_cover_each_expert_in_16_row_slabs():
     counts = np.array([0, 17, 3, 0, 16, 33])
-    se, sc, pr = R.decode_slots(counts)
+    se, sc, pr = L.decode_slots(counts)
     assert se.tolist() == [1, 1, 2, 4, 5, 5, 5] and sc.tolist() == [16, 1, 3, 16, 16, 16, 1]
     assert pr.size == counts.sum() and len(set(pr.tolist())) == pr.size
     assert np.all(pr // 16 < se.size) and np.all(pr % 16 < sc[pr // 16])
