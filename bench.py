@@ -1038,6 +1038,8 @@ def main():
     ap.add_argument("--cpu-pairs", type=int, default=256)
     ap.add_argument("--cpu-rows", type=int, default=16)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--gemm-pairs", type=int, default=None, choices=[0, 1],
+                    help="GEMMs on CTA pairs (1) or single SMs (0); default: the library's choice")
     ap.add_argument("--qdq-tensors", type=int, default=1024,
                     help="qdq workload: number of 1024 x 2048 tensors (1024 = 2^31 elements; fewer for profiler captures)")
     ap.add_argument("--experts", type=int, default=None,
@@ -1066,6 +1068,8 @@ def main():
     from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
 
     R.load()
+    if args.gemm_pairs is not None:
+        R.set_gemm_pairs(bool(args.gemm_pairs))
     peaks, peak_kind = load_peaks()
     sp = SPECS[args.workload](dev, args, peaks)
     step = sp["step"]
@@ -1165,6 +1169,8 @@ def main():
         config = dict(sp["config"])
         config["l2"] = "flushed between timed steps (256 MiB write outside the per-step events)"
         config["parallelism"] = f"replicas x{ws}"
+        if args.gemm_pairs is not None:
+            config["gemm_pairs"] = bool(args.gemm_pairs)
         line = {
             "metric": METRIC, "value": value, "unit": unit, "n_gpus": ws, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": t_step_ms, "higher_is_better": True, "scaling": "weak",

@@ -49,6 +49,7 @@ struct Plan {
   int off_seg;       // n_seg + 1 int32 tile prefix (segments mode)
   int off_bar;       // full[S], empty[S]
   int off_misc;      // s_g, t6, n_tiles, abort
+  int off_tab;       // float2 [128]: (d, 1/d) per E4M3 code
   int smem;
 };
 
@@ -69,7 +70,8 @@ __host__ __device__ inline Plan make_plan(int K, int Kp, int fanout, int n_seg, 
   p.off_seg = p.off_sel + round16(Kp * 2);
   p.off_bar = p.off_seg + round16(n_seg > 0 ? (n_seg + 1) * 4 : 0);
   p.off_misc = p.off_bar + 2 * kStages * 8;
-  p.smem = p.off_misc + 64;
+  p.off_tab = p.off_misc + 64;     // (d, 1/d) of the 128 E4M3 codes
+  p.smem = p.off_tab + 128 * 8;
   return p;
 }
 
@@ -153,10 +155,30 @@ __device__ __forceinline__ uint32_t codes8(const float x[8], const BlockScale& b
   return bs.S == 0 ? 0u : c;
 }
 
+// Eight E2M1 codes (nibble i = element i) -> their exact values, by the f16x2 <- e2m1x2
+// conversion (one byte = two codes, the low nibble to the low half); -0 for a negative zero code.
+__device__ __forceinline__ void e2m1_decode8_cvt(uint32_t c, float e[8]) {
+  uint32_t h[4];
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(c));
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+    e[2 * i] = f.x;
+    e[2 * i + 1] = f.y;
+  }
+}
+
 // r = RN(x - RN(e(c) * d)) for 8 values
 __device__ __forceinline__ void resid8(const float x[8], uint32_t c, float d, float r[8]) {
   float e[8];
-  e2m1_decode8(c, e);
+  e2m1_decode8_cvt(c, e);
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     const float2 dq = __fmul2_rn(make_float2(e[i], e[i + 1]), make_float2(d, d));
@@ -167,6 +189,17 @@ __device__ __forceinline__ void resid8(const float x[8], uint32_t c, float d, fl
 }
 
 // W consumer warps (4..8, chosen per shape so that both passes divide evenly) + 1 producer warp
+// The block scale with (d, 1/d) looked up per E4M3 code: for a fixed tensor scale s_g the 127
+// codes give 127 (d, 1/d) pairs, computed once per CTA with the same operations as block_scale.
+__device__ __forceinline__ BlockScale block_scale_tab(float b, float s_g, float t6, const float2* tab) {
+  BlockScale bs;
+  bs.S = s_g > 0.0f ? e4m3_encode(__fdiv_rn(b, t6)) : 0u;
+  const float2 di = tab[bs.S];
+  bs.d = di.x;
+  bs.inv = di.y;
+  return bs;
+}
+
 template <bool RES, int W>
 __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a) {
   constexpr int kConsumerWarps = W;
@@ -266,6 +299,13 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
   __syncthreads();
   const int n_tiles = misc_i[2];
   const float s_g = misc_f[0], t6 = misc_f[1];
+  float2* dtab = reinterpret_cast<float2*>(smem + p.off_tab);
+  if (threadIdx.x < 128) {
+    const uint32_t S = threadIdx.x;
+    const float d = __fmul_rn(e4m3_decode(S), s_g);
+    dtab[S] = make_float2(d, (S != 0 && S < 0x7F) ? __frcp_rn(d) : 0.0f);
+  }
+  __syncthreads();
   const uint64_t limit = a.wait_limit_ns;
 
   if (warp == kConsumerWarps) {
@@ -388,6 +428,18 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
 
   // ============================================================== consumers
   const int tid = threadIdx.x;  // 0 .. kConsumers-1
+  // when kConsumers is a multiple of QB a thread works on the same residual block q = tid % QB in
+  // every tile: its 16 channel offsets are read once, into registers
+  const bool fixed_q = RES && QB > 0 && kConsumers % QB == 0;
+  uint32_t my_off[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) my_off[i] = 0;
+  if (fixed_q) {
+    const int q = tid % QB;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      my_off[i] = (uint32_t)sel_off[(2 * i) * QB + q] | ((uint32_t)sel_off[(2 * i + 1) * QB + q] << 16);
+  }
   float* rbuf = reinterpret_cast<float*>(smem + p.off_rbuf);
   const int rpitch = KB * kPitch;  // words per row of the residual buffer
   int j = 0;
@@ -422,7 +474,7 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
         u0 = src[0];
         u1 = src[1];
       }
-      const BlockScale bs = block_scale(absmax16(u0, u1), s_g, t6);
+      const BlockScale bs = block_scale_tab(absmax16(u0, u1), s_g, t6, dtab);
       float x[16];
       bf16x8_to_f32(u0, x);
       bf16x8_to_f32(u1, x + 8);
@@ -457,12 +509,20 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
         }
         const float* rrow = rbuf + rs * rpitch;
         float v[16];
+        if (fixed_q) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i) v[i] = rrow[sel_off[i * QB + q]];
+          for (int i = 0; i < 8; ++i) {
+            v[2 * i] = rrow[my_off[i] & 0xFFFFu];
+            v[2 * i + 1] = rrow[my_off[i] >> 16];
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) v[i] = rrow[sel_off[i * QB + q]];
+        }
         float b = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(v[i]));
-        const BlockScale bs = block_scale(b, s_g, t6);
+        const BlockScale bs = block_scale_tab(b, s_g, t6, dtab);
         const uint2 c = make_uint2(codes8(v, bs), codes8(v + 8, bs));
         const int32_t blk = sf_blk_off(q);
         for (int jj = 0; jj < fo; ++jj) {
