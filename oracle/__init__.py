@@ -179,6 +179,37 @@ def act_quant_rac(x: np.ndarray, s_g: float, sel: np.ndarray):
     return codes, S, rcodes, rS, resid
 
 
+def act_quant_rac_own(x: np.ndarray, s_g: float, sel: np.ndarray, s_r: float | None = None):
+    """RAC variant with the residual's own tensor scale: the main pass and R_sel exactly as in
+    act_quant_rac, then R_sel quantised with s_r = RN(amax(R_sel) / 2688) (amax over every row of
+    the tensor) instead of s_g.  s_r may be given (an amax taken over a larger batch).
+    -> (codes, S, rcodes, rS, s_r)."""
+    codes, S, _, _, resid = act_quant_rac(x, s_g, sel)
+    if resid.size == 0:
+        rows = resid.shape[0]
+        return codes, S, np.zeros((rows, 0), np.uint8), np.zeros((rows, 0), np.uint8), np.float32(0.0)
+    if s_r is None:
+        s_r = global_scale(amax_f32(resid))
+    rcodes, rS, _ = quantize_f32(resid, s_r)
+    return codes, S, rcodes, rS, np.float32(s_r)
+
+
+def gemm_rac_own(a, aS, r, rS, w, wS, ws, wsS, s_a: float, s_r: float, s_w: float, rows=None):
+    """The two-accumulator form of the RAC GEMM: y = s_a s_w (Q(X) Q(W)^T) + s_r s_w (Q(R_sel)
+    Q(W_sel)^T), each product exact (gemm_rac with no residual), scaled and summed in binary64.
+    -> (y float64, absdot of both products)."""
+    y1, ad1 = gemm_rac(a, aS, None, None, w, wS, None, None, s_a, s_w, rows=rows)
+    if r is None or r.size == 0:
+        return y1, ad1
+    y2, ad2 = gemm_rac(r, rS, None, None, ws, wsS, None, None, s_r, s_w, rows=rows)
+    return y1 + y2, ad1 + ad2
+
+
+def amax_f32(t: np.ndarray) -> np.float32:
+    t = _c(t, np.float32).reshape(-1)
+    return np.float32(_get().orc_amax_f32(_p(t), t.size))
+
+
 def act_quant_masked(x: np.ndarray, s_g: float, sel: np.ndarray):
     """RAC variant with the residual kept at its channels (zero off sel) and quantised along K:
     bf16 x [rows, K] -> (codes [rows,K], S [rows,K/16], mcodes [rows,K], mS [rows,K/16])."""

@@ -725,6 +725,82 @@ def test_grouped_weight_sel_is_each_experts_raw_columns(orc):
         assert np.array_equal(codes[e], c3) and np.array_equal(S[e], S3)
 
 
+def test_own_scale_residual_largest_block_scale_is_448(orc):
+    """With its own tensor scale s_r = amax(R_sel) / 2688 the block holding the residual's amax gets
+    the largest finite E4M3 scale (448, code 0x7E) and no block scale is larger; with the shared
+    scale of X the residual's scales stay far below it.  A mix-up of the two scales fails here."""
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    _, _, rc_sh, rS_sh, resid = orc.act_quant_rac(wl.x, s_x, sel)
+    codes, S, rc, rS, s_r = orc.act_quant_rac_own(wl.x, s_x, sel)
+    assert s_r == orc.global_scale(np.float32(np.abs(resid).max()))
+    assert rS.max() == 0x7E and S.max() == 0x7E
+    assert rS_sh.max() < 0x70
+    # main codes do not depend on the residual's scale
+    c2, S2, _, _, _ = orc.act_quant_rac(wl.x, s_x, sel)
+    assert np.array_equal(codes, c2) and np.array_equal(S, S2)
+
+
+def test_own_scale_residual_is_scale_equivariant(orc):
+    """x -> 2^k x (exact in bf16) leaves every code and block scale unchanged and multiplies s_x and
+    s_r by 2^k."""
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    x = wl.x
+    x8 = (syn.bf16_to_f32(x) * np.float32(8.0)).astype(np.float32).view(np.uint32) >> 16
+    x8 = x8.astype(np.uint16)
+    s_x = orc.global_scale(orc.amax_bf16(x))
+    s_x8 = orc.global_scale(orc.amax_bf16(x8))
+    assert s_x8 == np.float32(8.0) * s_x
+    a = orc.act_quant_rac_own(x, s_x, sel)
+    b = orc.act_quant_rac_own(x8, s_x8, sel)
+    for u, v in zip(a[:4], b[:4]):
+        assert np.array_equal(u, v)
+    assert b[4] == np.float32(8.0) * a[4]
+
+
+def test_own_scale_gemm_is_the_sum_of_both_scaled_products(orc):
+    """gemm_rac_own equals the float64 product of the dequantised operands, each residual factor
+    taken with its own scale (s_r for R_sel, s_w for W_sel); with s_r = s_x it is the shared-scale
+    GEMM; with no channels it is plain W4A4."""
+    wl = syn.dense_tiny()
+    sel, _ = orc.calibrate(wl.x_cal, wl.Kp)
+    s_x = orc.global_scale(orc.amax_bf16(wl.x))
+    s_w = orc.global_scale(orc.amax_bf16(wl.w))
+    codes, S, rc, rS, s_r = orc.act_quant_rac_own(wl.x, s_x, sel)
+    wc, wS, wsc, wsS = orc.weight_pack(wl.w, s_w, sel)
+    y, _ = orc.gemm_rac_own(codes, S, rc, rS, wc, wS, wsc, wsS, s_x, s_r, s_w)
+    ref = orc.dequant(codes, S, s_x) @ orc.dequant(wc, wS, s_w).T + \
+        orc.dequant(rc, rS, s_r) @ orc.dequant(wsc, wsS, s_w).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-12)
+    _, _, rc2, rS2, _ = orc.act_quant_rac_own(wl.x, s_x, sel, s_r=s_x)
+    _, _, rc3, rS3, _ = orc.act_quant_rac(wl.x, s_x, sel)
+    assert np.array_equal(rc2, rc3) and np.array_equal(rS2, rS3)
+    y_sh, _ = orc.gemm_rac_own(codes, S, rc3, rS3, wc, wS, wsc, wsS, s_x, s_x, s_w)
+    y_ref, ad = orc.gemm_rac(codes, S, rc3, rS3, wc, wS, wsc, wsS, s_x, s_w)
+    assert np.all(np.abs(y_sh - y_ref) <= 1e-13 * ad)  # two binary64 sums instead of one
+    y0, _ = orc.gemm_rac_own(codes, S, None, None, wc, wS, None, None, s_x, s_r, s_w)
+    y0_ref, _ = orc.gemm_rac(codes, S, None, None, wc, wS, None, None, s_x, s_w)
+    assert np.array_equal(y0, y0_ref)
+
+
+def test_own_scale_wins_where_shared_residual_scales_are_subnormal(orc):
+    """A few very large channels raise s_x so far that the other channels' residual block scales
+    under s_x fall into the E4M3 subnormals (or to zero); quantised with its own scale the
+    residual then loses far less (the case the variant is for)."""
+    K = 256
+    x = syn.normal_bf16(5, 1, 64, K, 1.0, np.where(np.arange(K) < 4, 3.0e5, 1.0))
+    sel = np.arange(64, 128, dtype=np.int32)  # ordinary channels only
+    s_x = orc.global_scale(orc.amax_bf16(x))
+    _, _, rc, rS, resid = orc.act_quant_rac(x, s_x, sel)
+    assert np.all(rS < 8)                        # subnormal (or zero) residual block scales under s_x
+    _, _, rco, rSo, s_r = orc.act_quant_rac_own(x, s_x, sel)
+    e_sh = np.linalg.norm(resid - orc.dequant(rc, rS, s_x))
+    e_own = np.linalg.norm(resid - orc.dequant(rco, rSo, s_r))
+    assert e_own < 0.5 * e_sh
+
+
 def test_own_scale_residual_changes_little_on_the_workload_inputs(orc):
     """The variant that quantises R_sel with its own tensor scale (s_r = amax(R_sel) / 2688, two
     accumulators) would change the activation error only where shared-scale residual block scales
