@@ -127,14 +127,16 @@ def device_layout(R, wl, dev, pad, status, decode=False):
 class MoEStep:
     """Device-resident state of one replica and the step itself (C-ABI calls only)."""
 
-    def __init__(self, wl, h_cal, dev, masked=False, h_cal_offsets=None):
+    def __init__(self, wl, h_cal, dev, masked=False, h_cal_offsets=None, own_scale=False):
         """h_cal_offsets (int64 [E + 1], rows of h_cal per expert) selects the per-expert variant:
-        one down-projection channel list per expert, calibrated on that expert's rows."""
+        one down-projection channel list per expert, calibrated on that expert's rows.  own_scale
+        selects the variant with the residual's own tensor scale (two accumulators)."""
         import torch
 
         from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
 
         self.R, self.torch, self.dev, self.wl, self.masked = R, torch, dev, wl, masked
+        self.own = own_scale
         to = lambda a: torch.from_numpy(np.ascontiguousarray(a).view(np.int16)).to(dev).view(torch.bfloat16)
         self.status = R.new_status(dev)
         # offline: channel selection on the calibration batches, weight pack
@@ -188,11 +190,12 @@ class MoEStep:
         if "q0" in ev:
             ev["q0"].record()
         R.nvfp4_quantize_scatter(x, self.scatter, self.rows_padded, self.sel_gu, out=self.a, out_res=self.ar,
-                                 status=self.status)
+                                 status=self.status, own_scale=self.own)
         if "g0" in ev:
             ev["g0"].record()
         R.grouped_w4a4_rac_moe(self.a, self.ar, self.offsets, self.pgu, self.pgus, swiglu=True, y=self.h,
-                               amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows)
+                               amax_out=self.amax_h, status=self.status, expert_rows=self.expert_rows,
+                               own_scale=self.own)
         if "q1" in ev:
             ev["q1"].record()
         if self.masked or self.row_group is not None:
@@ -201,11 +204,11 @@ class MoEStep:
         else:
             # the token rows of each expert segment only
             R.nvfp4_quantize_segments(self.h, self.offsets, self.expert_rows, self.sel_dn, amax_in=self.amax_h,
-                                      out=self.hq, out_res=self.hqr, status=self.status)
+                                      out=self.hq, out_res=self.hqr, status=self.status, own_scale=self.own)
         if "d0" in ev:
             ev["d0"].record()
         R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.offsets, self.pdn, self.pdns, y=self.y, status=self.status,
-                               expert_rows=self.expert_rows)
+                               expert_rows=self.expert_rows, own_scale=self.own)
         if "end" in ev:
             ev["end"].record()
         return self.y
@@ -1000,6 +1003,14 @@ def run_sweep(args):
                       "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12, **e}
     del step
     torch.cuda.empty_cache()
+    # the residual with its own tensor scale (two accumulators) at r = 0.5
+    step = MoEStep(wl, h_cal, dev, own_scale=True)
+    ms, e = measure(step)
+    own_row = {"variant": "own_scale_residual", "r": 0.5, "ms_per_step": ms,
+               "tflops": sum(flops_of(wl, wl.Kp_gu, wl.Kp_dn)) / (ms * 1e-3) / 1e12,
+               "tflops_plain_w4a4_equivalent": plain_f / (ms * 1e-3) / 1e12, **e}
+    del step
+    torch.cuda.empty_cache()
     # the FP8 comparison format on the same block (E4M3, power-of-two scale per 32 elements)
     step = Mx8MoEStep(base, dev)
     ms, e = measure(step)
@@ -1020,8 +1031,9 @@ def run_sweep(args):
                                           "sampled (token, expert) rows",
                        "l2": "flushed between timed steps (256 MiB write outside the per-step events)"},
             "sweep": rows, "masked_variant": masked_row, "per_expert_variant": per_expert_row,
+            "own_scale_variant": own_row,
             "fp8_comparison": fp8_row, "y_error_non_increasing_in_r": mono, "e2e": None,
-            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * (len(rows) + 2) +
+            "gpu_launches": MoEStep.KERNELS_PER_STEP * args.steps * (len(rows) + 3) + 2 * args.steps +
             Mx8MoEStep.KERNELS_PER_STEP * args.steps}
     print(json.dumps(line), flush=True)
     return 0

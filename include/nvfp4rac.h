@@ -157,6 +157,25 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
                             void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
+/* The own-scale residual (a variant the pages leave open).  "Why 4-bit RL rollout collapses  */
+/* ..." (Two fixes, on two different sides) gives the residual pass over the selected channels */
+/* but not the tensor scale of the residual.  The method's reading here shares s_g of X (both  */
+/* products then add in one accumulator).  With NVFP4_RAC_OWN_RES_SCALE in `flags`:            */
+/*   the quantise calls (*_ex) give Q(R_sel) its own tensor scale s_r = amax(R_sel) / 2688,    */
+/*   amax over every row the call quantises (one extra pass over x that only finds max|R_sel|), */
+/*   and write s_r to q_res->s_g (q->s_g keeps s_g of x); the workspace is required.           */
+/*   the GEMM calls (*_ex) keep the main and the residual products in two accumulators and      */
+/*   compute y = s_a s_w (Q(X) Q(W)^T) + s_r s_w (Q(R_sel) Q(W_sel)^T) with s_r = *a_res->s_g  */
+/*   (N-tile 128, the SwiGLU epilogue included).                                               */
+/* Without the flag the *_ex calls are the calls without the suffix.                            */
+/* ---------------------------------------------------------------------------------------- */
+#define NVFP4_RAC_OWN_RES_SCALE 1u
+nvfp4_status nvfp4_quantize_ex(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                               int64_t M_out, const int32_t* sel, int32_t Kp, const float* amax_in,
+                               const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, void* stream, uint32_t flags);
+
+/* ---------------------------------------------------------------------------------------- */
 /* nvfp4_quantize_scatter -- nvfp4_quantize for an MoE dispatch: each source row is quantised */
 /* once and its codes / scales are written to up to `fanout` output rows.                    */
 /*   row_scatter  int32 [M x fanout]: output rows of source row m (entries < 0 are skipped;  */
@@ -169,6 +188,12 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
                                     int32_t fanout, const int32_t* sel, int32_t Kp, const float* amax_in,
                                     const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
                                     size_t workspace_bytes, int32_t* dev_status, void* stream);
+
+nvfp4_status nvfp4_quantize_scatter_ex(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                       const int32_t* row_scatter, int32_t fanout, const int32_t* sel, int32_t Kp,
+                                       const float* amax_in, const nvfp4_tensor* q, const nvfp4_tensor* q_res,
+                                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream,
+                                       uint32_t flags);
 
 /* ---------------------------------------------------------------------------------------- */
 /* nvfp4_quantize_segments -- nvfp4_quantize of the token rows of an expert-grouped layout   */
@@ -190,6 +215,11 @@ nvfp4_status nvfp4_quantize_segments(const uint16_t* x, int64_t M, int64_t K, in
                                      const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
                                      const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes,
                                      int32_t* dev_status, void* stream);
+nvfp4_status nvfp4_quantize_segments_ex(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                        const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
+                                        const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                                        const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes,
+                                        int32_t* dev_status, void* stream, uint32_t flags);
 
 /* ---------------------------------------------------------------------------------------- */
 /* nvfp4_quantize_grouped_sel -- nvfp4_quantize with one channel list per group of output    */
@@ -275,6 +305,10 @@ nvfp4_status pack_weights_grouped_sel(const uint16_t* w, int64_t E, int64_t N, i
 nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
                            const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp,
                            nvfp4_dtype out, void* y, int64_t ldy, int32_t* dev_status, void* stream);
+/* w4a4_rac_gemm with flags (NVFP4_RAC_OWN_RES_SCALE: see the quantise calls above). */
+nvfp4_status w4a4_rac_gemm_ex(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
+                              const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp, nvfp4_dtype out,
+                              void* y, int64_t ldy, int32_t* dev_status, void* stream, uint32_t flags);
 
 /* ---------------------------------------------------------------------------------------- */
 /* grouped_w4a4_rac_moe -- the GEMM above over token-sorted expert segments (MoE rollout).   */
@@ -296,6 +330,12 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
                                   const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp, nvfp4_epilogue ep,
                                   nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
                                   void* stream);
+/* grouped_w4a4_rac_moe with flags (NVFP4_RAC_OWN_RES_SCALE: see the quantise calls above). */
+nvfp4_status grouped_w4a4_rac_moe_ex(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
+                                     const int32_t* expert_rows, int32_t E, const nvfp4_tensor* w,
+                                     const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp, nvfp4_epilogue ep,
+                                     nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
+                                     void* stream, uint32_t flags);
 
 /* ---------------------------------------------------------------------------------------- */
 /* grouped_w4a4_rac_moe_segments -- grouped_w4a4_rac_moe over arbitrary row segments, each   */

@@ -84,16 +84,19 @@ nvfp4_status make_code_map(CUtensorMap* m, const void* base, uint64_t inner_byte
 
 // Output matrix [rows x cols] (bf16 or fp32, row pitch ld elements) stored by the GEMM epilogue
 // in boxes of 32 rows x 128 bytes, 128-byte swizzle.  Rows beyond `rows` are clipped.
-nvfp4_status make_out_map(CUtensorMap* m, void* base, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld) {
+// narrow: boxes of 32 rows x 64 bytes without swizzle (the SwiGLU stores of the own-scale mode)
+nvfp4_status make_out_map(CUtensorMap* m, void* base, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld,
+                          bool narrow = false) {
   auto fn = encode_fn();
   if (!fn) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   const uint64_t esz = bf16 ? 2 : 4;
   cuuint64_t dims[2] = {cols, rows};
   cuuint64_t strides[1] = {ld * esz};
-  cuuint32_t box[2] = {(cuuint32_t)(128 / esz), 32};
+  cuuint32_t box[2] = {(cuuint32_t)((narrow ? 64 : 128) / esz), 32};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  narrow ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(NVFP4_ERR_CUDA, "tensor map for the output failed (error %d, cols %llu, rows %llu)", (int)r,
@@ -201,7 +204,7 @@ void nvfp4_set_act_tile(int32_t rows, int32_t warps) {
 size_t nvfp4_quantize_workspace_size(int64_t M, int64_t K) {
   (void)M;
   (void)K;
-  return 1024 * sizeof(float);
+  return 1024 * sizeof(float) + 256;  // amax partials, then the residual's amax (own-scale variant)
 }
 
 }  // extern "C"
@@ -243,6 +246,28 @@ nvfp4::ActArgs act_args(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, co
   return a;
 }
 
+// One activation quantisation: a single launch, or for the own-scale residual (flag
+// NVFP4_RAC_OWN_RES_SCALE, Kp > 0) a pass that folds max |R_sel| into the workspace float after
+// the amax partials, then the quantisation with the residual's own scale.
+nvfp4_status run_act(nvfp4::ActArgs b, uint32_t flags, void* workspace, cudaStream_t s) {
+  if ((flags & NVFP4_RAC_OWN_RES_SCALE) && b.Kp > 0) {
+    float* res_amax = reinterpret_cast<float*>(reinterpret_cast<char*>(workspace) + 1024 * sizeof(float));
+    cudaError_t e = cudaMemsetAsync(res_amax, 0, sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "residual amax reset");
+    nvfp4::ActArgs pass = b;
+    pass.res_mode = 2;
+    pass.res_amax_out = res_amax;
+    pass.s_g_out = nullptr;
+    pass.s_g_out2 = nullptr;
+    e = launch_act(pass, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
+    if (e != cudaSuccess) return cuda_fail(e, "residual amax launch");
+    b.res_mode = 1;
+    b.res_amax_in = res_amax;
+  }
+  cudaError_t e = launch_act(b, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "quantize launch");
+}
+
 }  // namespace
 
 namespace {
@@ -251,7 +276,7 @@ namespace {
 nvfp4_status quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
                            int64_t M_out, const int32_t* row_group, int32_t groups, const int32_t* sel, int32_t Kp,
                            const float* amax_in, const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
-                           size_t workspace_bytes, int32_t* dev_status, void* stream) {
+                           size_t workspace_bytes, int32_t* dev_status, void* stream, uint32_t flags = 0) {
   if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
   if (M < 0 || M_out < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "negative row count");
   if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld must be a positive multiple of 64 <= %lld", (long long)K, (long long)kMaxK);
@@ -276,26 +301,28 @@ nvfp4_status quantize_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
     if (!aligned16(sel)) return fail(NVFP4_ERR_ALIGNMENT, "sel must be 16-byte aligned");
   }
   const int P = act_partials(M, K);
-  if (!amax_in) {
+  const bool own = (flags & NVFP4_RAC_OWN_RES_SCALE) && Kp > 0;
+  if (!amax_in || own) {
     if (!workspace || workspace_bytes < nvfp4_quantize_workspace_size(M, K))
       return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
     if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   }
+  const bool masked = Kp > 0 && Kp < K && q_res->cols == K;
+  const bool act_kernel = q->rows_padded > 0 && use_act_kernel(K, Kp, 1, 0, masked, groups);
+  if (own && !act_kernel)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the own-scale residual takes the compact residual with one list");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* partial = reinterpret_cast<float*>(workspace);
   if (!amax_in) {
     cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "amax launch");
   }
-  const bool masked = Kp > 0 && Kp < K && q_res->cols == K;
-  if (q->rows_padded > 0 && use_act_kernel(K, Kp, 1, 0, masked, groups)) {
+  if (act_kernel) {
     nvfp4::ActArgs b = act_args(x, M, K, ldx, sel, Kp, partial, P, amax_in, q, q_res, dev_status);
     b.map = row_gather ? kMapGather : kMapRows;
     b.row_gather = row_gather;
     b.rows_valid = M_out;
-    cudaError_t e = launch_act(b, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
-    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
-    return NVFP4_OK;
+    return run_act(b, flags, workspace, s);
   }
   RowArgs a;
   memset(&a, 0, sizeof(a));
@@ -342,6 +369,15 @@ nvfp4_status nvfp4_quantize(const uint16_t* x, int64_t M, int64_t K, int64_t ldx
                        workspace_bytes, dev_status, stream);
 }
 
+nvfp4_status nvfp4_quantize_ex(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_gather,
+                               int64_t M_out, const int32_t* sel, int32_t Kp, const float* amax_in,
+                               const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                               size_t workspace_bytes, int32_t* dev_status, void* stream, uint32_t flags) {
+  g_last_error.clear();
+  return quantize_rows(x, M, K, ldx, row_gather, M_out, nullptr, 0, sel, Kp, amax_in, q, q_res, workspace,
+                       workspace_bytes, dev_status, stream, flags);
+}
+
 nvfp4_status nvfp4_quantize_grouped_sel(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
                                         const int32_t* row_gather, int64_t M_out, const int32_t* row_group,
                                         int32_t groups, const int32_t* sel, int32_t Kp, const float* amax_in,
@@ -354,11 +390,13 @@ nvfp4_status nvfp4_quantize_grouped_sel(const uint16_t* x, int64_t M, int64_t K,
                        workspace_bytes, dev_status, stream);
 }
 
-nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
-                                    int32_t fanout, const int32_t* sel, int32_t Kp, const float* amax_in,
-                                    const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
-                                    size_t workspace_bytes, int32_t* dev_status, void* stream) {
-  g_last_error.clear();
+}  // extern "C"
+
+namespace {
+nvfp4_status scatter_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
+                          int32_t fanout, const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                          const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                          void* stream, uint32_t flags) {
   if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
   if (!row_scatter && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "row_scatter is NULL");
   if (M < 0 || fanout <= 0 || fanout > 64) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M >= 0 and 1 <= fanout <= 64 required");
@@ -377,11 +415,16 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
       return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "q_res must have q's rows_padded and sf_layout");
   }
   const int P = act_partials(M, K);
-  if (!amax_in) {
+  const bool own = (flags & NVFP4_RAC_OWN_RES_SCALE) && Kp > 0;
+  if (!amax_in || own) {
     if (!workspace || workspace_bytes < nvfp4_quantize_workspace_size(M, K))
       return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
     if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
   }
+  const bool masked = Kp > 0 && Kp < K && q_res->cols == K;
+  const bool act_kernel = use_act_kernel(K, Kp, fanout, 0, masked, 0);
+  if (own && !act_kernel)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the own-scale residual takes the compact residual with one list");
   if (M == 0) return NVFP4_OK;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   float* partial = reinterpret_cast<float*>(workspace);
@@ -389,15 +432,12 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
     cudaError_t e = launch_amax(x, 1, M, K, ldx, partial, P, dev_status, s);
     if (e != cudaSuccess) return cuda_fail(e, "amax launch");
   }
-  const bool masked = Kp > 0 && Kp < K && q_res->cols == K;
-  if (use_act_kernel(K, Kp, fanout, 0, masked, 0)) {
+  if (act_kernel) {
     nvfp4::ActArgs b = act_args(x, M, K, ldx, sel, Kp, partial, P, amax_in, q, q_res, dev_status);
     b.map = kMapScatter;
     b.row_scatter = row_scatter;
     b.fanout = fanout;
-    cudaError_t e = launch_act(b, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
-    if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
-    return NVFP4_OK;
+    return run_act(b, flags, workspace, s);
   }
   RowArgs a;
   memset(&a, 0, sizeof(a));
@@ -429,12 +469,10 @@ nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int
   return NVFP4_OK;
 }
 
-nvfp4_status nvfp4_quantize_segments(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
-                                     const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
-                                     const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
-                                     const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes,
-                                     int32_t* dev_status, void* stream) {
-  g_last_error.clear();
+nvfp4_status segments_rows(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* expert_offsets,
+                           const int32_t* expert_rows, int32_t E, const int32_t* sel, int32_t Kp,
+                           const float* amax_in, const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                           size_t workspace_bytes, int32_t* dev_status, void* stream, uint32_t flags) {
   if (!x && M > 0) return fail(NVFP4_ERR_INVALID_ARG, "x is NULL");
   if (!expert_offsets || !expert_rows) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets / expert_rows is NULL");
   if (E < 1 || E > kMaxRouteExperts) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be in [1, %d]", kMaxRouteExperts);
@@ -455,7 +493,7 @@ nvfp4_status nvfp4_quantize_segments(const uint16_t* x, int64_t M, int64_t K, in
   if (!use_act_kernel(K, Kp, 1, E, false, 0))
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K = %lld, Kp = %d too large for the segment quantiser", (long long)K, Kp);
   const int P = act_partials(M, K);
-  if (!amax_in) {
+  if (!amax_in || ((flags & NVFP4_RAC_OWN_RES_SCALE) && Kp > 0)) {
     if (!workspace || workspace_bytes < nvfp4_quantize_workspace_size(M, K))
       return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
     if (!aligned16(workspace)) return fail(NVFP4_ERR_ALIGNMENT, "workspace must be 16-byte aligned");
@@ -474,9 +512,49 @@ nvfp4_status nvfp4_quantize_segments(const uint16_t* x, int64_t M, int64_t K, in
   b.n_seg = E;
   b.rows_valid = M;
   b.src_rows = M;
-  cudaError_t e = launch_act(b, num_sms(), g_act_rows.load(), g_act_warps.load(), s);
-  if (e != cudaSuccess) return cuda_fail(e, "quantize launch");
-  return NVFP4_OK;
+  return run_act(b, flags, workspace, s);
+}
+}  // namespace
+
+extern "C" {
+
+nvfp4_status nvfp4_quantize_scatter(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, const int32_t* row_scatter,
+                                    int32_t fanout, const int32_t* sel, int32_t Kp, const float* amax_in,
+                                    const nvfp4_tensor* q, const nvfp4_tensor* q_res, void* workspace,
+                                    size_t workspace_bytes, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  return scatter_rows(x, M, K, ldx, row_scatter, fanout, sel, Kp, amax_in, q, q_res, workspace, workspace_bytes,
+                      dev_status, stream, 0);
+}
+
+nvfp4_status nvfp4_quantize_scatter_ex(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                       const int32_t* row_scatter, int32_t fanout, const int32_t* sel, int32_t Kp,
+                                       const float* amax_in, const nvfp4_tensor* q, const nvfp4_tensor* q_res,
+                                       void* workspace, size_t workspace_bytes, int32_t* dev_status, void* stream,
+                                       uint32_t flags) {
+  g_last_error.clear();
+  return scatter_rows(x, M, K, ldx, row_scatter, fanout, sel, Kp, amax_in, q, q_res, workspace, workspace_bytes,
+                      dev_status, stream, flags);
+}
+
+nvfp4_status nvfp4_quantize_segments(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                     const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
+                                     const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                                     const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes,
+                                     int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  return segments_rows(x, M, K, ldx, expert_offsets, expert_rows, E, sel, Kp, amax_in, q, q_res, workspace,
+                       workspace_bytes, dev_status, stream, 0);
+}
+
+nvfp4_status nvfp4_quantize_segments_ex(const uint16_t* x, int64_t M, int64_t K, int64_t ldx,
+                                        const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
+                                        const int32_t* sel, int32_t Kp, const float* amax_in, const nvfp4_tensor* q,
+                                        const nvfp4_tensor* q_res, void* workspace, size_t workspace_bytes,
+                                        int32_t* dev_status, void* stream, uint32_t flags) {
+  g_last_error.clear();
+  return segments_rows(x, M, K, ldx, expert_offsets, expert_rows, E, sel, Kp, amax_in, q, q_res, workspace,
+                       workspace_bytes, dev_status, stream, flags);
 }
 
 // ------------------------------------------------------------------------------------------ calibrate
@@ -642,7 +720,8 @@ nvfp4_status pack_weights_grouped_sel(const uint16_t* w, int64_t E, int64_t N, i
 static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
                                 const nvfp4_tensor* w_sel, int64_t rows_needed, int64_t N, int64_t K, int32_t Kp,
                                 int64_t E, nvfp4_dtype out, void* y, int64_t ldy, int64_t y_cols, int64_t y_rows,
-                                int bn, CUtensorMap* maps, GemmArgs* g, int w_box_rows = 0) {
+                                int bn, CUtensorMap* maps, GemmArgs* g, int w_box_rows = 0, bool own = false,
+                                bool swiglu = false) {
   if (w_box_rows == 0) w_box_rows = bn;
   if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
   if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp must be a multiple of 64 in [0, K]");
@@ -667,7 +746,8 @@ static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res
   }
   memset(maps, 0, 5 * sizeof(CUtensorMap));
   if (y_rows > 0) {
-    st = make_out_map(&maps[4], y, out == NVFP4_OUT_BF16, (uint64_t)y_cols, (uint64_t)y_rows, (uint64_t)ldy);
+    st = make_out_map(&maps[4], y, out == NVFP4_OUT_BF16, (uint64_t)y_cols, (uint64_t)y_rows, (uint64_t)ldy,
+                      own && swiglu);
     if (st != NVFP4_OK) return st;
   }
   st = make_code_map(&maps[0], a->codes, (uint64_t)K / 2, (uint64_t)a->rows_padded, 1, 128, 2, "A");
@@ -704,19 +784,22 @@ static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res
   g->ldy = ldy;
   g->out_bf16 = out == NVFP4_OUT_BF16;
   g->wait_limit_ns = g_wait_limit_ns.load();
+  g->own_res_scale = own ? 1 : 0;
+  g->s_a_res = (own && Kp > 0) ? a_res->s_g : a->s_g;
   return NVFP4_OK;
 }
 
-nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
-                           const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp, nvfp4_dtype out,
-                           void* y, int64_t ldy, int32_t* dev_status, void* stream) {
-  g_last_error.clear();
+static nvfp4_status dense_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
+                               const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp, nvfp4_dtype out,
+                               void* y, int64_t ldy, int32_t* dev_status, void* stream, uint32_t flags) {
   if (M < 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "M must be >= 0");
-  const bool pairs = g_gemm_pair.load() != 0 && N % 256 == 0 && g_tile_n.load() != 128;
-  const int bn = pairs ? 256 : choose_tile_n(N, K, Kp);
+  const bool own = (flags & NVFP4_RAC_OWN_RES_SCALE) != 0;
+  const bool pairs = !own && g_gemm_pair.load() != 0 && N % 256 == 0 && g_tile_n.load() != 128;
+  const int bn = own ? 128 : pairs ? 256 : choose_tile_n(N, K, Kp);
   CUtensorMap maps[5];
   GemmArgs g;
-  nvfp4_status st = gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, M, bn, maps, &g, pairs ? 128 : bn);
+  nvfp4_status st =
+      gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, M, bn, maps, &g, pairs ? 128 : bn, own, false);
   if (st != NVFP4_OK) return st;
   if (M == 0) return NVFP4_OK;
   g.offsets = nullptr;
@@ -739,6 +822,20 @@ nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, con
   return NVFP4_OK;
 }
 
+nvfp4_status w4a4_rac_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
+                           const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp, nvfp4_dtype out,
+                           void* y, int64_t ldy, int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  return dense_gemm(a, a_res, w, w_sel, M, N, K, Kp, out, y, ldy, dev_status, stream, 0);
+}
+
+nvfp4_status w4a4_rac_gemm_ex(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const nvfp4_tensor* w,
+                              const nvfp4_tensor* w_sel, int64_t M, int64_t N, int64_t K, int32_t Kp, nvfp4_dtype out,
+                              void* y, int64_t ldy, int32_t* dev_status, void* stream, uint32_t flags) {
+  g_last_error.clear();
+  return dense_gemm(a, a_res, w, w_sel, M, N, K, Kp, out, y, ldy, dev_status, stream, flags);
+}
+
 }  // extern "C"
 
 namespace {
@@ -747,7 +844,7 @@ nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, co
                             const int32_t* seg_rows, const int32_t* seg_expert, int32_t n_seg, const nvfp4_tensor* w,
                             const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp, nvfp4_epilogue ep,
                             nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
-                            void* stream) {
+                            void* stream, uint32_t flags = 0) {
   if (!offsets) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets is NULL");
   if (n_seg <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the segment count must be positive");
   if (ep != NVFP4_EPI_NONE && ep != NVFP4_EPI_SWIGLU_AMAX) return fail(NVFP4_ERR_INVALID_ARG, "bad epilogue");
@@ -759,13 +856,15 @@ nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, co
     return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the SwiGLU epilogue needs N %% 256 == 0");
   if (!w) return fail(NVFP4_ERR_INVALID_ARG, "w is NULL");
   const int64_t E = seg_expert ? w->slabs : n_seg;
-  const bool pairs = g_gemm_pair.load() != 0 && N % 256 == 0 && g_tile_n.load() != 128 && n_seg <= kMaxRouteExperts;
-  const int bn = (pairs || ep == NVFP4_EPI_SWIGLU_AMAX) ? 256 : choose_tile_n(N, K, Kp);
+  const bool own = (flags & NVFP4_RAC_OWN_RES_SCALE) != 0;
+  const bool pairs =
+      !own && g_gemm_pair.load() != 0 && N % 256 == 0 && g_tile_n.load() != 128 && n_seg <= kMaxRouteExperts;
+  const int bn = own ? 128 : (pairs || ep == NVFP4_EPI_SWIGLU_AMAX) ? 256 : choose_tile_n(N, K, Kp);
   CUtensorMap maps[5];
   GemmArgs g;
   const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
   nvfp4_status st = gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, a ? a->rows_padded : 0, bn,
-                                maps, &g, pairs ? 128 : bn);
+                                maps, &g, pairs ? 128 : bn, own, ep == NVFP4_EPI_SWIGLU_AMAX);
   if (st != NVFP4_OK) return st;
   g.offsets = offsets;
   g.expert_rows = seg_rows;
@@ -800,6 +899,17 @@ nvfp4_status grouped_w4a4_rac_moe(const nvfp4_tensor* a, const nvfp4_tensor* a_r
   if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
   return grouped_common(a, a_res, expert_offsets, expert_rows, nullptr, E, w, w_sel, N, K, Kp, ep, out, y, ldy,
                         amax_out, dev_status, stream);
+}
+
+nvfp4_status grouped_w4a4_rac_moe_ex(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* expert_offsets,
+                                     const int32_t* expert_rows, int32_t E, const nvfp4_tensor* w,
+                                     const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp, nvfp4_epilogue ep,
+                                     nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
+                                     void* stream, uint32_t flags) {
+  g_last_error.clear();
+  if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
+  return grouped_common(a, a_res, expert_offsets, expert_rows, nullptr, E, w, w_sel, N, K, Kp, ep, out, y, ldy,
+                        amax_out, dev_status, stream, flags);
 }
 
 nvfp4_status grouped_w4a4_rac_moe_segments(const nvfp4_tensor* a, const nvfp4_tensor* a_res,

@@ -8,6 +8,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -52,24 +53,24 @@ __device__ __forceinline__ uint32_t e2m1_encode8(const float v[8]) {
   return out;
 }
 
-// Eight E2M1 codes (nibble i = element i) -> their values, exact.  The eight magnitudes
-// {0, .5, 1, 1.5, 2, 3, 4, 6} are exact bf16 numbers; their high and low bytes are looked up
-// with byte permutes (index = code & 7), the sign is code bit 3.  (The f16x2 <- e2m1x2
-// conversion instruction is not used: it does not return these values on sm_100.)
+// Eight E2M1 codes (nibble i = element i) -> their values, exact: the f16x2 <- e2m1x2
+// conversion turns one byte (two codes, the low nibble into the low half) into two exact halves,
+// which widen exactly to binary32; a negative zero code gives -0.
 __device__ __forceinline__ void e2m1_decode8(uint32_t codes, float out[8]) {
-  const uint32_t idx = codes & 0x77777777u;
-  const uint32_t hi_a = __byte_perm(0x3F3F3F00u, 0x40404040u, idx & 0xFFFFu);
-  const uint32_t hi_b = __byte_perm(0x3F3F3F00u, 0x40404040u, idx >> 16);
-  const uint32_t lo_a = __byte_perm(0xC0800000u, 0xC0804000u, idx & 0xFFFFu);
-  const uint32_t lo_b = __byte_perm(0xC0800000u, 0xC0804000u, idx >> 16);
+  uint32_t h[4];
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(codes));
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // bytes 2, 3 of the result = low, high byte of element i's bf16 value
-    const uint32_t sel = ((uint32_t)i << 8) | ((uint32_t)(4 + i) << 12);
-    const uint32_t va = __byte_perm(lo_a, hi_a, sel) & 0xFFFF0000u;
-    const uint32_t vb = __byte_perm(lo_b, hi_b, sel) & 0xFFFF0000u;
-    out[i] = __uint_as_float(va | ((codes << (28 - 4 * i)) & 0x80000000u));
-    out[4 + i] = __uint_as_float(vb | ((codes << (12 - 4 * i)) & 0x80000000u));
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
+    out[2 * i] = f.x;
+    out[2 * i + 1] = f.y;
   }
 }
 
@@ -116,12 +117,20 @@ __device__ __forceinline__ uint32_t quant8(const float x[8], const BlockScale& b
   }
   float v[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(x[i], bs.inv);
+  for (int i = 0; i < 8; i += 2) {
+    const float2 p = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(bs.inv, bs.inv));
+    v[i] = p.x;
+    v[i + 1] = p.y;
+  }
   uint32_t c = e2m1_encode8(v);
   float e[8];
   e2m1_decode8(c, e);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) dq[i] = __fmul_rn(e[i], bs.d);
+  for (int i = 0; i < 8; i += 2) {
+    const float2 p = __fmul2_rn(make_float2(e[i], e[i + 1]), make_float2(bs.d, bs.d));
+    dq[i] = p.x;
+    dq[i + 1] = p.y;
+  }
   return c;
 }
 
@@ -129,7 +138,11 @@ __device__ __forceinline__ uint32_t quant8_codes(const float x[8], const BlockSc
   if (bs.S == 0) return 0u;
   float v[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(x[i], bs.inv);
+  for (int i = 0; i < 8; i += 2) {
+    const float2 p = __fmul2_rn(make_float2(x[i], x[i + 1]), make_float2(bs.inv, bs.inv));
+    v[i] = p.x;
+    v[i + 1] = p.y;
+  }
   return e2m1_encode8(v);
 }
 

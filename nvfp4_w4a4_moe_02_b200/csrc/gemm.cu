@@ -44,8 +44,13 @@ __device__ __forceinline__ int segment_weight(const GemmArgs& args, int seg) {
   return e;
 }
 
-template <int BN>
+// OWN: the residual operand carries its own tensor scale (the own-scale RAC variant), so the main
+// and the residual products go to two accumulators (columns [0, BN) and [BN, 2 BN) of a buffer)
+// and the epilogue adds them with their own scales; only BN = 128 (the two halves then take the
+// tensor memory of one BN = 256 accumulator).
+template <int BN, bool OWN = false>
 struct Cfg {
+  static constexpr int ACC_W = OWN ? 2 * BN : BN;  // accumulator columns per tile
   static constexpr int STAGES = (BN == 256) ? 3 : 5;
   // epilogue staging: per epilogue warp, STG boxes of 32 rows x 128 bytes for TMA stores
   static constexpr int STG = (BN == 256) ? 2 : 1;
@@ -56,17 +61,18 @@ struct Cfg {
   static constexpr int SFB_BYTES = (BN / 128) * 4 * 512;
   // Tensor memory: two accumulator buffers and two per-MMA scale slots (A: 4 columns, B: 4
   // per 128 columns of N).  The tensor pipe executes copies and MMAs of one thread in order,
-  // so a scale slot can be rewritten for the next-but-one MMA.  With BN = 256 the buffers
-  // overlap: buffer 1 starts ACC_OVERLAP columns before buffer 0 ends, and the epilogue drains
-  // that strip first and releases it early.
+  // so a scale slot can be rewritten for the next-but-one MMA.  When 2 accumulators and the slots
+  // exceed the 512 columns, the buffers overlap: buffer 1 starts ACC_OVERLAP columns before
+  // buffer 0 ends, and the epilogue drains that strip first and releases it early.
   static constexpr int SF_SLOT = 4 + 4 * (BN / 128);
   static constexpr int SF_COLS = 2 * SF_SLOT;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int ACC_OVERLAP = (2 * BN + SF_COLS > TMEM_COLS) ? (2 * BN + SF_COLS - TMEM_COLS) : 0;
-  static constexpr int ACC1_BASE = BN - ACC_OVERLAP;
-  static constexpr int SF_BASE = ACC1_BASE + BN;
+  static constexpr int ACC_OVERLAP = (2 * ACC_W + SF_COLS > TMEM_COLS) ? (2 * ACC_W + SF_COLS - TMEM_COLS) : 0;
+  static constexpr int ACC1_BASE = ACC_W - ACC_OVERLAP;
+  static constexpr int SF_BASE = ACC1_BASE + ACC_W;
   static_assert(SF_BASE + SF_COLS <= TMEM_COLS, "tensor memory budget");
   static_assert(ACC_OVERLAP <= 32, "the shared strip must lie in one 32-column chunk");
+  static_assert(!OWN || BN == 128, "two accumulators only at BN = 128");
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
@@ -85,12 +91,12 @@ struct Cfg {
 // FP8: the comparison operands (E4M3 codes, one E8M0 scale per 32 elements): a 128-byte k-tile
 // holds 128 elements and one scale atom per 128 rows, copied once per k-tile; its four K = 32
 // MMAs pick their scale byte by id.  No residual loop, no tensor scales (alpha = 1).
-template <int BN, bool FP8>
+template <int BN, bool FP8, bool OWN = false>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_ar,
                          const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_ws,
                          const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
-  using C = Cfg<BN>;
+  using C = Cfg<BN, OWN>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   unsigned char* smem = smem_raw;
@@ -266,14 +272,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           // FP4: each MMA's scale atoms are copied right before it (into alternating slots): the
           // tensor pipe overlaps the copies with the preceding MMA
+          // own-scale variant: the residual k-tiles go to the second accumulator, which starts
+          // fresh at the first of them
+          const uint32_t d_k = d_tmem + ((OWN && res) ? (uint32_t)BN : 0u);
+          const int kt_first = (OWN && res) ? args.kt_main : 0;
           for (int j = 0; j < (FP8 ? 0 : nk64); ++j, ++mma_count) {
             const uint32_t sfa_t = tmem_base + (uint32_t)(C::SF_BASE + (mma_count & 1) * C::SF_SLOT);
             const uint32_t sfb_t = sfa_t + 4;
             tc_copy_sf(sfa_t, desc_sf(sfa_s + j * 512));
 #pragma unroll
             for (int rb = 0; rb < BN / 128; ++rb) tc_copy_sf(sfb_t + 4 * rb, desc_sf(sfb_s + rb * 2048 + j * 512));
-            tc_mma_fp4(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, sfa_t, sfb_t,
-                       (kt | j) != 0 ? 1u : 0u);
+            tc_mma_fp4(d_k, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, sfa_t, sfb_t,
+                       (kt != kt_first || j != 0) ? 1u : 0u);
           }
           tc_commit(bar_empty(stage));
           if (++stage == C::STAGES) {
@@ -294,7 +304,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // Eight warps: two per tensor-memory lane quadrant, each owning half of the tile's
     // columns.  A warp drains its columns into registers, releases the accumulator, and only
     // then converts and stores, so the math overlaps the next tile's MMAs.
-    constexpr int NCH = BN / 64;            // 32-column chunks per warp
+    constexpr int NCH = C::ACC_W / 64;      // 32-column chunks per warp
     const int quad = warp & 3;              // tensor-memory lanes [32*quad, 32*quad + 32)
     const int half = (warp - 2) >> 2;       // which half of the tile's columns
     float amax = 0.0f;
@@ -325,11 +335,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                                  : row_limit;
       const bool row_ok = row < row_limit && row < args.rows_capacity && row < rows_e;
       const float alpha = FP8 ? 1.0f : __fmul_rn(__ldg(args.s_a), __ldg(args.s_w + e));
+      // own-scale variant: the residual product's scale (0 when there is no residual loop, so the
+      // second accumulator, never written, is not read)
+      const bool has_res = OWN && args.kt_res > 0;
+      const float alpha_r = has_res ? __fmul_rn(__ldg(args.s_a_res), __ldg(args.s_w + e)) : 0.0f;
       const uint32_t t_row = tmem_base + (uint32_t)(acc ? C::ACC1_BASE : 0) + ((uint32_t)(quad * 32) << 16);
       // chunk i of this warp: plain -> columns half*BN/2 + 32i; SwiGLU -> output features
       // [half*BN/4, ...): chunks 0..NCH/2-1 gate (column (f/64)*128 + f%64), NCH/2.. the up
-      // columns 64 further (gate/up interleave of the packed weight)
+      // columns 64 further (gate/up interleave of the packed weight).  Own-scale variant: the
+      // same for the main accumulator in chunks 0..NCH/2-1 and the residual one (columns + BN)
+      // in chunks NCH/2..NCH-1.
       auto chunk_col = [&](int i) -> int {
+        if (OWN) {
+          const int base = i >= NCH / 2 ? BN : 0;
+          const int ii = i % (NCH / 2);
+          if (args.epi == 0) return base + half * (BN / 2) + 32 * ii;
+          const int f = half * (BN / 4);
+          return base + (f / 64) * 128 + (f % 64) + (ii == 1 ? 64 : 0);
+        }
         if (args.epi == 0) return half * (BN / 2) + 32 * i;
         const int ii = i % (NCH / 2);
         const int f = half * (BN / 4) + 32 * ii;
@@ -358,6 +381,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_acce(acc));
+      if (OWN) {
+        // y = alpha * main + alpha_r * residual, the sum in binary32; the values of the
+        // SwiGLU / store paths below then come from chunks 0..NCH/2-1 with alpha 1
+#pragma unroll
+        for (int i = 0; i < NCH / 2; ++i)
+#pragma unroll
+          for (int k = 0; k < 32; ++k) {
+            const float m = __fmul_rn(__uint_as_float(v[i][k]), alpha);
+            const float r = has_res ? __fmul_rn(__uint_as_float(v[NCH / 2 + i][k]), alpha_r) : 0.0f;
+            v[i][k] = __float_as_uint(__fadd_rn(m, r));
+          }
+      }
+      const float alpha_out = OWN ? 1.0f : alpha;
       // ---- output through shared memory: each box is 32 rows x 128 bytes in the 128-byte
       // swizzled layout (16-byte chunk c of row r at chunk c ^ (r % 8)), stored by one TMA copy
       const uint32_t stg = sbase + C::OFF_STG + (uint32_t)((warp - 2) * C::STG * C::BOX_BYTES);
@@ -378,31 +414,34 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           bulk_commit_group();
         }
       };
+      // output chunks: all NCH of the plain accumulator; the first NCH / 2 in the own-scale
+      // variant (already combined above)
+      constexpr int NOUT = OWN ? NCH / 2 : NCH;
       if (!box_live) {
         // padding only: nothing to store
       } else if (args.epi == 0 && args.out_bf16) {
         // 64 columns per box
 #pragma unroll
-        for (int b = 0; b < NCH / 2; ++b) {
+        for (int b = 0; b < NOUT / 2; ++b) {
           uint32_t w[32];
 #pragma unroll
           for (int h = 0; h < 2; ++h)
 #pragma unroll
             for (int k = 0; k < 16; ++k)
-              w[16 * h + k] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * b + h][2 * k]), alpha),
-                                          __fmul_rn(__uint_as_float(v[2 * b + h][2 * k + 1]), alpha));
+              w[16 * h + k] = pack_bf16x2(__fmul_rn(__uint_as_float(v[2 * b + h][2 * k]), alpha_out),
+                                          __fmul_rn(__uint_as_float(v[2 * b + h][2 * k + 1]), alpha_out));
           put_box(b % C::STG, w, (int32_t)(nb * BN + half * (BN / 2) + 64 * b));
         }
       } else if (args.epi == 0) {
         // fp32: 32 columns per box
 #pragma unroll
-        for (int b = 0; b < NCH; ++b) {
+        for (int b = 0; b < NOUT; ++b) {
           uint32_t w[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__fmul_rn(__uint_as_float(v[b][k]), alpha));
+          for (int k = 0; k < 32; ++k) w[k] = __float_as_uint(__fmul_rn(__uint_as_float(v[b][k]), alpha_out));
           put_box(b % C::STG, w, (int32_t)(nb * BN + half * (BN / 2) + 32 * b));
         }
-      } else {
+      } else if (!OWN) {
         // SwiGLU (BN = 256): this warp's 64 output features form one box
         uint32_t w[32];
 #pragma unroll
@@ -423,6 +462,36 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             w[16 * i + k] = pack_bf16x2(hv[0], hv[1]);
           }
         put_box(0, w, (int32_t)(nb * (BN / 2) + half * (BN / 4)));
+      } else {
+        // SwiGLU of the own-scale variant (BN = 128): this warp's 32 output features (gate in
+        // chunk 0, up in chunk 1) form one box of 32 rows x 64 bytes, row-major (the output
+        // tensor map of this mode has 64-byte boxes and no swizzle)
+        uint32_t w[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          float hv[2];
+#pragma unroll
+          for (int z = 0; z < 2; ++z) {
+            const int j = 2 * k + z;
+            const float gv = bf16_round(__uint_as_float(v[0][j]));
+            const float uv = bf16_round(__uint_as_float(v[1][j]));
+            const float sg = __fdividef(gv, 1.0f + __expf(-gv));
+            hv[z] = bf16_round(sg * uv);
+            if (row_ok) amax = fmaxf(amax, fabsf(hv[z]));
+          }
+          w[k] = pack_bf16x2(hv[0], hv[1]);
+        }
+        if (lane == 0) bulk_wait_group_read<C::STG - 1>();
+        __syncwarp();
+        const uint32_t rowp = stg + (uint32_t)(lane * 64);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) st_shared_v4(rowp + 16u * c, w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_2d(&tm_y, stg, (int32_t)(nb * (BN / 2) + half * (BN / 4)), y0);
+          bulk_commit_group();
+        }
       }
     }
     if (lane == 0) bulk_wait_group_all();  // this warp's stores complete before exit
@@ -470,21 +539,25 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, int32_t* status) {
 
 size_t gemm_smem_bytes(int bn) { return bn == 256 ? (size_t)tc::Cfg<256>::SMEM : (size_t)tc::Cfg<128>::SMEM; }
 
-template <int BN, bool FP8>
+template <int BN, bool FP8, bool OWN = false>
 static cudaError_t launch_gemm_t(const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
                                  const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
                                  cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<BN, FP8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       tc::Cfg<BN>::SMEM);
+  constexpr int smem = tc::Cfg<BN, OWN>::SMEM;
+  cudaError_t e =
+      cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<BN, FP8, OWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  tc::w4a4_rac_gemm_kernel<BN, FP8><<<grid, tc::NUM_THREADS, tc::Cfg<BN>::SMEM, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y,
-                                                                                     args);
+  tc::w4a4_rac_gemm_kernel<BN, FP8, OWN><<<grid, tc::NUM_THREADS, smem, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(int bn, const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
                         const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
                         cudaStream_t st) {
+  if (args.own_res_scale) {
+    if (bn != 128 || args.fp8) return cudaErrorInvalidValue;
+    return launch_gemm_t<128, false, true>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args, grid, st);
+  }
   if (bn == 256)
     return args.fp8 ? launch_gemm_t<256, true>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args, grid, st)
                     : launch_gemm_t<256, false>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args, grid, st);

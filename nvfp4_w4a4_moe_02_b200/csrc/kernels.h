@@ -78,6 +78,11 @@ struct ActArgs {
   int32_t* status;
   uint64_t wait_limit_ns;
   int32_t R;                     // set by the launcher
+  // residual tensor scale: 0 = the tensor scale of x (the method's reading); 1 = its own scale
+  // from *res_amax_in; 2 = no output, max |R_sel| over the rows folded into *res_amax_out
+  int32_t res_mode;
+  const float* res_amax_in;
+  float* res_amax_out;
 };
 bool act_plan_choose(int64_t K, int32_t Kp, int fanout, int32_t n_seg, int* R, int* W, int* smem, int force_R = 0,
                      int force_W = 0);
@@ -151,6 +156,8 @@ struct GemmArgs {
   int32_t* status;
   uint64_t wait_limit_ns;
   int32_t fp8;               // 1: the FP8 comparison operands (E4M3, E8M0 per 32; kt_main = K/128, no residual)
+  int32_t own_res_scale;     // 1: the residual has its own tensor scale *s_a_res (two accumulators, BN = 128)
+  const float* s_a_res;      // own_res_scale: device scalar
 };
 
 // bn: 128 or 256

@@ -70,8 +70,8 @@ __host__ __device__ inline Plan make_plan(int K, int Kp, int fanout, int n_seg, 
   p.off_seg = p.off_sel + round16(Kp * 2);
   p.off_bar = p.off_seg + round16(n_seg > 0 ? (n_seg + 1) * 4 : 0);
   p.off_misc = p.off_bar + 2 * kStages * 8;
-  p.off_tab = p.off_misc + 64;     // (d, 1/d) of the 128 E4M3 codes
-  p.smem = p.off_tab + 128 * 8;
+  p.off_tab = p.off_misc + 64;     // (d, 1/d) of the 128 E4M3 codes, for s_g and for the residual
+  p.smem = p.off_tab + 2 * 128 * 8;
   return p;
 }
 
@@ -155,30 +155,10 @@ __device__ __forceinline__ uint32_t codes8(const float x[8], const BlockScale& b
   return bs.S == 0 ? 0u : c;
 }
 
-// Eight E2M1 codes (nibble i = element i) -> their exact values, by the f16x2 <- e2m1x2
-// conversion (one byte = two codes, the low nibble to the low half); -0 for a negative zero code.
-__device__ __forceinline__ void e2m1_decode8_cvt(uint32_t c, float e[8]) {
-  uint32_t h[4];
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(c));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-    e[2 * i] = f.x;
-    e[2 * i + 1] = f.y;
-  }
-}
-
 // r = RN(x - RN(e(c) * d)) for 8 values
 __device__ __forceinline__ void resid8(const float x[8], uint32_t c, float d, float r[8]) {
   float e[8];
-  e2m1_decode8_cvt(c, e);
+  e2m1_decode8(c, e);
 #pragma unroll
   for (int i = 0; i < 8; i += 2) {
     const float2 dq = __fmul2_rn(make_float2(e[i], e[i + 1]), make_float2(d, d));
@@ -260,9 +240,9 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
     if (lane == 0) {
       misc_f[0] = s_g;
       misc_f[1] = __fmul_rn(6.0f, s_g);
-      if (blockIdx.x == 0) {
+      if (blockIdx.x == 0 && a.res_mode != 2) {
         if (a.s_g_out) *a.s_g_out = s_g;
-        if (a.s_g_out2) *a.s_g_out2 = s_g;
+        if (a.s_g_out2 && a.res_mode == 0) *a.s_g_out2 = s_g;
       }
     }
   }
@@ -300,12 +280,23 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
   const int n_tiles = misc_i[2];
   const float s_g = misc_f[0], t6 = misc_f[1];
   float2* dtab = reinterpret_cast<float2*>(smem + p.off_tab);
+  // the residual's tensor scale: that of x, or its own (own-scale variant)
+  const float s_r = a.res_mode == 1 ? scale_from_amax(*a.res_amax_in, nullptr) : s_g;
+  const float t6_r = __fmul_rn(6.0f, s_r);
+  float2* dtab_r = a.res_mode == 1 ? dtab + 128 : dtab;
   if (threadIdx.x < 128) {
     const uint32_t S = threadIdx.x;
     const float d = __fmul_rn(e4m3_decode(S), s_g);
     dtab[S] = make_float2(d, (S != 0 && S < 0x7F) ? __frcp_rn(d) : 0.0f);
+    if (a.res_mode == 1) {
+      const float dr = __fmul_rn(e4m3_decode(S), s_r);
+      dtab_r[S] = make_float2(dr, (S != 0 && S < 0x7F) ? __frcp_rn(dr) : 0.0f);
+    }
   }
+  if (a.res_mode == 1 && blockIdx.x == 0 && threadIdx.x == 0 && a.s_g_out2) *a.s_g_out2 = s_r;
   __syncthreads();
+  const bool amax_only = a.res_mode == 2;
+  float res_max = 0.0f;
   const uint64_t limit = a.wait_limit_ns;
 
   if (warp == kConsumerWarps) {
@@ -480,7 +471,7 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
       bf16x8_to_f32(u1, x + 8);
       const uint2 c = make_uint2(codes8(x, bs), codes8(x + 8, bs));
       const int32_t blk = sf_blk_off(kb);
-      for (int jj = 0; jj < fo; ++jj) {
+      for (int jj = 0; jj < (amax_only ? 0 : fo); ++jj) {
         const int e = slot * fo + jj;
         const int64_t co = m.code[e];
         if (co < 0) continue;
@@ -522,7 +513,11 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
         float b = 0.0f;
 #pragma unroll
         for (int i = 0; i < 16; ++i) b = fmaxf(b, fabsf(v[i]));
-        const BlockScale bs = block_scale_tab(b, s_g, t6, dtab);
+        if (amax_only) {
+          res_max = fmaxf(res_max, b);
+          continue;
+        }
+        const BlockScale bs = block_scale_tab(b, s_r, t6_r, dtab_r);
         const uint2 c = make_uint2(codes8(v, bs), codes8(v + 8, bs));
         const int32_t blk = sf_blk_off(q);
         for (int jj = 0; jj < fo; ++jj) {
@@ -537,6 +532,11 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
     // this stage (rows and metadata) is free for the producer
     __syncwarp();
     if (lane == 0) tc::mbar_arrive(bar_empty(s));
+  }
+  if (amax_only) {
+    res_max = warp_max(res_max);
+    if (lane == 0 && res_max > 0.0f)
+      atomicMax(reinterpret_cast<unsigned int*>(a.res_amax_out), __float_as_uint(res_max));
   }
 }
 

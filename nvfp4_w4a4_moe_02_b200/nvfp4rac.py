@@ -23,6 +23,7 @@ OK = 0
 STATUS_NAMES = {0: "OK", 1: "ERR_INVALID_ARG", 2: "ERR_UNSUPPORTED_SHAPE", 3: "ERR_ALIGNMENT", 4: "ERR_RANGE",
                 5: "ERR_CUDA", 6: "ERR_TIMEOUT"}
 OUT_F32, OUT_BF16 = 0, 1
+RAC_OWN_RES_SCALE = 1  # the residual's own tensor scale (quantise and GEMM *_ex calls)
 EPI_NONE, EPI_SWIGLU_AMAX = 0, 1
 
 
@@ -66,6 +67,16 @@ def load() -> ctypes.CDLL:
         "nvfp4_quantize_workspace_size": ([i64, i64], sz),
         "nvfp4_quantize": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
         "nvfp4_quantize_scatter": ([vp, i64, i64, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
+        "nvfp4_quantize_ex": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp, ctypes.c_uint32],
+                              ctypes.c_int),
+        "nvfp4_quantize_scatter_ex": ([vp, i64, i64, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp,
+                                       ctypes.c_uint32], ctypes.c_int),
+        "nvfp4_quantize_segments_ex": ([vp, i64, i64, i64, vp, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp,
+                                        ctypes.c_uint32], ctypes.c_int),
+        "w4a4_rac_gemm_ex": ([tp, tp, tp, tp, i64, i64, i64, i32, ctypes.c_int, vp, i64, vp, vp, ctypes.c_uint32],
+                             ctypes.c_int),
+        "grouped_w4a4_rac_moe_ex": ([tp, tp, vp, vp, i32, tp, tp, i64, i64, i32, ctypes.c_int, ctypes.c_int, vp, i64,
+                                     vp, vp, vp, ctypes.c_uint32], ctypes.c_int),
         "nvfp4_quantize_segments": ([vp, i64, i64, i64, vp, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp],
                                     ctypes.c_int),
         "nvfp4_quantize_grouped_sel": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp],
@@ -245,7 +256,7 @@ def set_act_tile(rows: int, warps: int):
 def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather: torch.Tensor | None = None,
                    M_out: int | None = None, rows_padded: int | None = None, amax_in: torch.Tensor | None = None,
                    out: Packed | None = None, out_res: Packed | None = None, status: torch.Tensor | None = None,
-                   stream=None, masked: bool = False, row_group: torch.Tensor | None = None):
+                   stream=None, masked: bool = False, row_group: torch.Tensor | None = None, own_scale: bool = False):
     """Online activation quantisation with the residual pass on ``sel`` -> (Packed, Packed | None).
 
     masked=True selects the masked full-K residual variant (residual at its channel, zero off
@@ -278,16 +289,17 @@ def nvfp4_quantize(x: torch.Tensor, sel: torch.Tensor | None = None, row_gather:
                                               ctypes.byref(qr), ws.data_ptr(), ws.numel(), st.data_ptr(),
                                               _stream(stream)))
         return out, out_res
-    _check(lib.nvfp4_quantize(x.data_ptr(), M, K, ldx, _ptr(row_gather), M_out, _ptr(sel), Kp, _ptr(amax_in),
-                              ctypes.byref(q), ctypes.byref(qr) if qr is not None else None, ws.data_ptr(),
-                              ws.numel(), st.data_ptr(), _stream(stream)))
+    _check(lib.nvfp4_quantize_ex(x.data_ptr(), M, K, ldx, _ptr(row_gather), M_out, _ptr(sel), Kp, _ptr(amax_in),
+                                 ctypes.byref(q), ctypes.byref(qr) if qr is not None else None, ws.data_ptr(),
+                                 ws.numel(), st.data_ptr(), _stream(stream), RAC_OWN_RES_SCALE if own_scale else 0))
     return out, (out_res if Kp > 0 else None)
 
 
 def nvfp4_quantize_scatter(x: torch.Tensor, row_scatter: torch.Tensor, rows_padded: int,
                            sel: torch.Tensor | None = None, amax_in: torch.Tensor | None = None,
                            out: Packed | None = None, out_res: Packed | None = None,
-                           status: torch.Tensor | None = None, stream=None, sf_layout: int = SF_ATOM128):
+                           status: torch.Tensor | None = None, stream=None, sf_layout: int = SF_ATOM128,
+                           own_scale: bool = False):
     """Quantise each row of x once and write it to the rows row_scatter[m, :] of the outputs.
 
     row_scatter: int32 [M, fanout] (-1 = unused).  Rows no entry names are left untouched, so
@@ -308,16 +320,17 @@ def nvfp4_quantize_scatter(x: torch.Tensor, row_scatter: torch.Tensor, rows_padd
     st = status if status is not None else new_status(x.device)
     q = out.c()
     qr = out_res.c() if Kp > 0 else None
-    _check(lib.nvfp4_quantize_scatter(x.data_ptr(), M, K, x.stride(0), row_scatter.data_ptr(), fanout, _ptr(sel), Kp,
-                                      _ptr(amax_in), ctypes.byref(q), ctypes.byref(qr) if qr is not None else None,
-                                      ws.data_ptr(), ws.numel(), st.data_ptr(), _stream(stream)))
+    _check(lib.nvfp4_quantize_scatter_ex(x.data_ptr(), M, K, x.stride(0), row_scatter.data_ptr(), fanout, _ptr(sel),
+                                         Kp, _ptr(amax_in), ctypes.byref(q),
+                                         ctypes.byref(qr) if qr is not None else None, ws.data_ptr(), ws.numel(),
+                                         st.data_ptr(), _stream(stream), RAC_OWN_RES_SCALE if own_scale else 0))
     return out, (out_res if Kp > 0 else None)
 
 
 def nvfp4_quantize_segments(x: torch.Tensor, expert_offsets: torch.Tensor, expert_rows: torch.Tensor,
                             sel: torch.Tensor | None = None, amax_in: torch.Tensor | None = None,
                             out: Packed | None = None, out_res: Packed | None = None,
-                            status: torch.Tensor | None = None, stream=None):
+                            status: torch.Tensor | None = None, stream=None, own_scale: bool = False):
     """Quantise only the token rows of an expert-grouped layout: rows
     [expert_offsets[e], expert_offsets[e] + expert_rows[e]) of x (device int32 [E] each) into the
     same rows of the outputs; other output rows are left as they are.  Returns (Packed, Packed | None)."""
@@ -336,10 +349,10 @@ def nvfp4_quantize_segments(x: torch.Tensor, expert_offsets: torch.Tensor, exper
     st = status if status is not None else new_status(x.device)
     q = out.c()
     qr = out_res.c() if Kp > 0 else None
-    _check(lib.nvfp4_quantize_segments(x.data_ptr(), M, K, x.stride(0), expert_offsets.data_ptr(),
-                                       expert_rows.data_ptr(), E, _ptr(sel), Kp, _ptr(amax_in), ctypes.byref(q),
-                                       ctypes.byref(qr) if qr is not None else None, ws.data_ptr(), ws.numel(),
-                                       st.data_ptr(), _stream(stream)))
+    _check(lib.nvfp4_quantize_segments_ex(x.data_ptr(), M, K, x.stride(0), expert_offsets.data_ptr(),
+                                          expert_rows.data_ptr(), E, _ptr(sel), Kp, _ptr(amax_in), ctypes.byref(q),
+                                          ctypes.byref(qr) if qr is not None else None, ws.data_ptr(), ws.numel(),
+                                          st.data_ptr(), _stream(stream), RAC_OWN_RES_SCALE if own_scale else 0))
     return out, (out_res if Kp > 0 else None)
 
 
@@ -418,7 +431,7 @@ def pack_weights(w: torch.Tensor, sel: torch.Tensor | None = None, gate_up_inter
 
 def w4a4_rac_gemm(a: Packed, a_res: Packed | None, w: Packed, w_sel: Packed | None, M: int,
                   out_dtype=torch.bfloat16, y: torch.Tensor | None = None, status: torch.Tensor | None = None,
-                  stream=None) -> torch.Tensor:
+                  stream=None, own_scale: bool = False) -> torch.Tensor:
     """Dense Y = s_a s_w (Q(X)Q(W)^T + Q(R_sel)Q(W_sel)^T) -> y [M, N]."""
     lib = load()
     N, K = w.rows, w.cols
@@ -430,16 +443,17 @@ def w4a4_rac_gemm(a: Packed, a_res: Packed | None, w: Packed, w_sel: Packed | No
     ca, cw = a.c(), w.c()
     car = a_res.c() if Kp > 0 else None
     cws = w_sel.c() if Kp > 0 else None
-    _check(lib.w4a4_rac_gemm(ctypes.byref(ca), ctypes.byref(car) if car else None, ctypes.byref(cw),
-                             ctypes.byref(cws) if cws else None, M, N, K, Kp, od, y.data_ptr(), y.stride(0),
-                             st.data_ptr(), _stream(stream)))
+    _check(lib.w4a4_rac_gemm_ex(ctypes.byref(ca), ctypes.byref(car) if car else None, ctypes.byref(cw),
+                                ctypes.byref(cws) if cws else None, M, N, K, Kp, od, y.data_ptr(), y.stride(0),
+                                st.data_ptr(), _stream(stream), RAC_OWN_RES_SCALE if own_scale else 0))
     return y
 
 
 def grouped_w4a4_rac_moe(a: Packed, a_res: Packed | None, expert_offsets: torch.Tensor, w: Packed,
                          w_sel: Packed | None, swiglu: bool = False, out_dtype=torch.bfloat16,
                          y: torch.Tensor | None = None, amax_out: torch.Tensor | None = None,
-                         status: torch.Tensor | None = None, stream=None, expert_rows: torch.Tensor | None = None):
+                         status: torch.Tensor | None = None, stream=None, expert_rows: torch.Tensor | None = None,
+                         own_scale: bool = False):
     """Grouped GEMM over expert segments -> y (rows a.rows_padded) [and amax of the SwiGLU output].
 
     expert_rows (optional device int32 [E]): token rows per segment; 32-row output boxes of padding
@@ -458,10 +472,12 @@ def grouped_w4a4_rac_moe(a: Packed, a_res: Packed | None, expert_offsets: torch.
     ca, cw = a.c(), w.c()
     car = a_res.c() if Kp > 0 else None
     cws = w_sel.c() if Kp > 0 else None
-    _check(lib.grouped_w4a4_rac_moe(ctypes.byref(ca), ctypes.byref(car) if car else None, expert_offsets.data_ptr(),
-                                    _ptr(expert_rows), E, ctypes.byref(cw), ctypes.byref(cws) if cws else None, N, K, Kp,
-                                    EPI_SWIGLU_AMAX if swiglu else EPI_NONE, od, y.data_ptr(), y.stride(0),
-                                    _ptr(amax_out), st.data_ptr(), _stream(stream)))
+    _check(lib.grouped_w4a4_rac_moe_ex(ctypes.byref(ca), ctypes.byref(car) if car else None,
+                                       expert_offsets.data_ptr(), _ptr(expert_rows), E, ctypes.byref(cw),
+                                       ctypes.byref(cws) if cws else None, N, K, Kp,
+                                       EPI_SWIGLU_AMAX if swiglu else EPI_NONE, od, y.data_ptr(), y.stride(0),
+                                       _ptr(amax_out), st.data_ptr(), _stream(stream),
+                                       RAC_OWN_RES_SCALE if own_scale else 0))
     return (y, amax_out) if swiglu else y
 
 
