@@ -53,24 +53,25 @@ __device__ __forceinline__ uint32_t e2m1_encode8(const float v[8]) {
   return out;
 }
 
-// Eight E2M1 codes (nibble i = element i) -> their values, exact: the f16x2 <- e2m1x2
-// conversion turns one byte (two codes, the low nibble into the low half) into two exact halves,
-// which widen exactly to binary32; a negative zero code gives -0.
+// Eight E2M1 codes (nibble i = element i) -> their values, exact.  The eight magnitudes
+// {0, .5, 1, 1.5, 2, 3, 4, 6} are exact bf16 numbers; their high and low bytes are looked up
+// with byte permutes (index = code & 7), the sign is code bit 3.  (The f16x2 <- e2m1x2
+// conversion is exact only when its byte operand arrives zero-extended in a 32-bit register;
+// bytes unpacked from a word by a vector move gave wrong values, so it is not used here.)
 __device__ __forceinline__ void e2m1_decode8(uint32_t codes, float out[8]) {
-  uint32_t h[4];
-  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
-      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, b0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, b1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, b2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, b3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(codes));
+  const uint32_t idx = codes & 0x77777777u;
+  const uint32_t hi_a = __byte_perm(0x3F3F3F00u, 0x40404040u, idx & 0xFFFFu);
+  const uint32_t hi_b = __byte_perm(0x3F3F3F00u, 0x40404040u, idx >> 16);
+  const uint32_t lo_a = __byte_perm(0xC0800000u, 0xC0804000u, idx & 0xFFFFu);
+  const uint32_t lo_b = __byte_perm(0xC0800000u, 0xC0804000u, idx >> 16);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h[i]));
-    out[2 * i] = f.x;
-    out[2 * i + 1] = f.y;
+    // bytes 2, 3 of the result = low, high byte of element i's bf16 value
+    const uint32_t sel = ((uint32_t)i << 8) | ((uint32_t)(4 + i) << 12);
+    const uint32_t va = __byte_perm(lo_a, hi_a, sel) & 0xFFFF0000u;
+    const uint32_t vb = __byte_perm(lo_b, hi_b, sel) & 0xFFFF0000u;
+    out[i] = __uint_as_float(va | ((codes << (28 - 4 * i)) & 0x80000000u));
+    out[4 + i] = __uint_as_float(vb | ((codes << (12 - 4 * i)) & 0x80000000u));
   }
 }
 
