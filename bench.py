@@ -395,7 +395,9 @@ class MoEBlockStep:
     combine into [T, H].  Prefill uses 128-row expert segments and the grouped GEMM; decode uses
     16-token slabs (worst-case slot count, unused slots skipped) and the swap-AB GEMM."""
 
-    KERNELS_PER_STEP = 10  # router, count, offsets, rank, amax, quantise X, gate_up, quantise h, down, combine
+    # router, count, offsets, rank, amax, quantise X, gate_up, quantise h, down, combine; prefill with
+    # the combine in the down GEMM's epilogue: + row pairs, the combine kernel becomes the bf16 finalise
+    KERNELS_PER_STEP = 10
 
     def __init__(self, wl, packed, sel_gu, sel_dn, decode, dev):
         import torch
@@ -431,7 +433,13 @@ class MoEBlockStep:
         self.hq = P.empty(self.cap, wl.I, rows_padded=self.cap, device=dev, sf_layout=lay, zero=True)
         self.hqr = P.empty(self.cap, wl.Kp_dn, rows_padded=self.cap, device=dev, sf_layout=lay, zero=True)
         self.slot_first_row = torch.arange(self.n_slots, dtype=torch.int32, device=dev) * 16 if decode else None
-        self.ye = torch.zeros(self.cap, wl.H, dtype=torch.bfloat16, device=dev)
+        self.fused_combine = not decode
+        self.kernels_per_step = self.KERNELS_PER_STEP + (1 if self.fused_combine else 0)
+        if self.fused_combine:
+            self.row_pair = torch.empty(self.cap, dtype=torch.int32, device=dev)
+            self.y32 = torch.empty(T, wl.H, dtype=torch.float32, device=dev)
+        else:
+            self.ye = torch.zeros(self.cap, wl.H, dtype=torch.bfloat16, device=dev)
         self.y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize()
 
@@ -445,6 +453,8 @@ class MoEBlockStep:
         R.moe_dispatch_plan(self.ids, self.wl.E, self.pad, rows_capacity=self.cap, n_slots=self.n_slots,
                             offsets=self.off, row_scatter=self.rows, slot_expert=self.se, slot_count=self.sc,
                             status=self.status, expert_rows=self.expert_rows)
+        if self.fused_combine:
+            R.moe_row_pairs(self.rows, self.cap, row_pair=self.row_pair, status=self.status)
         if "q0" in ev:
             ev["q0"].record()
         R.nvfp4_quantize_scatter(self.x if x is None else x, self.rows, self.cap, self.sel_gu, out=self.a,
@@ -465,15 +475,19 @@ class MoEBlockStep:
                                   out_res=self.hqr, status=self.status)
         if "d0" in ev:
             ev["d0"].record()
-        if self.decode:
+        if self.fused_combine:
+            # down projection with the weighted combine in its epilogue, then the bf16 rows
+            R.grouped_w4a4_rac_moe_combine(self.hq, self.hqr, self.off, self.pdn, self.pdns, self.row_pair, self.w,
+                                           out=self.y, out32=self.y32, status=self.status,
+                                           expert_rows=self.expert_rows)
+            if "c0" in ev:
+                ev["c0"].record()
+        else:
             R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.se, self.sc, self.pdn, self.pdns, y=self.ye,
                                           status=self.status)
-        else:
-            R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.off, self.pdn, self.pdns, y=self.ye, status=self.status,
-                                   expert_rows=self.expert_rows)
-        if "c0" in ev:
-            ev["c0"].record()
-        R.moe_combine(self.ye, self.rows, self.w, out=self.y, status=self.status)
+            if "c0" in ev:
+                ev["c0"].record()
+            R.moe_combine(self.ye, self.rows, self.w, out=self.y, status=self.status)
         if "end" in ev:
             ev["end"].record()
         return self.y
@@ -481,8 +495,6 @@ class MoEBlockStep:
 
 class QdqStep:
     """Trainer-side fake quantisation of a set of weight tensors: one weight_qdq call."""
-
-    KERNELS_PER_STEP = 2  # amax, qdq
 
     def __init__(self, w_np, dev):
         import torch
@@ -495,6 +507,8 @@ class QdqStep:
         self.x = torch.from_numpy(w_np.view(np.int16)).to(dev).view(torch.bfloat16)
         self.y = torch.empty_like(self.x)
         self.s_g = torch.empty(self.n_tensors, dtype=torch.float32, device=dev)
+        # tensors of up to 4M elements: one kernel (the one-pass form); larger: amax, then qdq
+        self.kernels_per_step = 1 if self.elems <= (4 << 20) else 2
 
     def run(self, x=None, events=None):
         ev = events or {}
@@ -860,7 +874,7 @@ def _spec_block(dev, args, decode):
         quant={}, config={"workload": name, "tokens": T, "experts": wl.E, "hidden": wl.H, "intermediate": wl.I,
                           "plan": "device (router top-k, dispatch plan); combine into [T, H]",
                           "rows_capacity": step.cap},
-        cpu=lambda: None, kernels_per_step=MoEBlockStep.KERNELS_PER_STEP)
+        cpu=lambda: None, kernels_per_step=step.kernels_per_step)
 
 
 def spec_block_prefill(dev, args, peaks):
@@ -892,12 +906,18 @@ def _spec_qdq(dev, args, n_tensors, elems=1 << 31):
         return {"value": 4.0 * rows.size / dt / 1e9, "unit": "GB/s", "cores": orc.num_threads(), "kind": "oracle",
                 "sample": f"{rows.shape[0]} tensors of {rows.shape[1]} elements (amax + QDQ), {dt:.1f} s"}
 
+    # a tensor that fits on chip is read once and written once (4 B per element); one larger than
+    # L2 must be read twice, since its scale depends on every element before any can be quantised
+    fits = step.kernels_per_step == 1
+    d_bytes = (4.0 if fits else 6.0) * n
+    d_label = ("weight_qdq (amax + fake-quant in one pass, 4 B/element algorithmic: one read, one write)" if fits
+               else "weight_qdq (amax pass + fake-quant pass, 6 B/element algorithmic: two reads, one write)")
     return dict(
         step=step, x_np=w, flops=0.0, work=4.0 * n, unit="GB/s", dtype="bf16 -> nvfp4 -> bf16 (f32 arithmetic)",
         events=["q0", "end"], segments={"qdq": ("q0", "end")},
-        dominant=("qdq", 0.0, 4.0 * n, "weight_qdq (amax + fake-quant, 4 B/element algorithmic)"), quant={},
+        dominant=("qdq", 0.0, d_bytes, d_label), quant={},
         config={"workload": label, "tensors": n_tensors, "elements": int(n), "distribution": "N(0, 0.02)"},
-        cpu=cpu_leg, kernels_per_step=QdqStep.KERNELS_PER_STEP)
+        cpu=cpu_leg, kernels_per_step=step.kernels_per_step)
 
 
 def spec_qdq(dev, args, peaks):

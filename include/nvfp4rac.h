@@ -125,6 +125,10 @@ void nvfp4_set_gemm_tile_n(int32_t n);
 /* Tuning: 1 runs the W4A4 + RAC GEMMs whose N is a multiple of 256 on pairs of SMs (one
  * 256 x 256 tile per cluster of two CTAs); 0 (default) keeps one SM per 128-row tile. */
 void nvfp4_set_gemm_pairs(int32_t on);
+/* Tuning: 1 (default) runs weight_qdq on tensors of up to 4M elements in one pass over HBM
+ * (groups of CTAs meet at a per-tensor counter in the workspace, then re-read the tensor from
+ * L2); 0 keeps the two passes (amax, then the fake-quant).  Results are identical. */
+void nvfp4_set_qdq_one_pass(int32_t on);
 /* Tuning: rows per tile (1..16) and consumer warps (4, 6, 7 or 8) of the activation quantiser
  * (0 = automatic choice per shape).  A forced shape that does not fit shared memory makes the
  * quantise calls fall back to the row quantiser. */
@@ -434,6 +438,32 @@ nvfp4_status moe_row_groups(const int32_t* expert_offsets, int32_t E, int64_t ro
 nvfp4_status moe_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* row_scatter,
                          const float* topk_w, int64_t T, int32_t k, int64_t H, uint16_t* out, int64_t ldo,
                          int32_t* dev_status, void* stream);
+
+/* moe_row_pairs -- the inverse of row_scatter: row_pair[r] = t * k + j where                 */
+/*   row_scatter[t, j] = r, -1 on rows that hold no pair (padding).  row_pair int32 [rows]     */
+/*   (device); a row_scatter entry >= rows is NVFP4_ERR_INVALID_ARG in *dev_status.            */
+nvfp4_status moe_row_pairs(const int32_t* row_scatter, int64_t T, int32_t k, int64_t rows, int32_t* row_pair,
+                           int32_t* dev_status, void* stream);
+/* grouped_w4a4_rac_moe_combine -- the down projection of the MoE block with moe_combine in    */
+/*   its epilogue (the expert rows are never written to memory):                               */
+/*   out[t, :] = bf16( sum_j topk_w[t, j] * y_r ),  y_r = bf16(alpha_e * acc_r), r the row of   */
+/*   pair (t, j), acc_r as in grouped_w4a4_rac_moe (NVFP4_EPI_NONE).  Each product            */
+/*   RN(topk_w * y_r) is added into the binary32 row out32[t] by atomic vector adds, so the   */
+/*   k terms of a token are summed in an unspecified order (reading: the same sum as          */
+/*   moe_combine up to binary32 reassociation, |difference| <= k * 2^-23 * sum_j |w_j y_j|    */
+/*   before the final bf16 rounding).                                                          */
+/*   a, a_res, expert_offsets, expert_rows, E, w, w_sel, N, K, Kp  as grouped_w4a4_rac_moe.  */
+/*   row_pair   int32 [a.rows_padded] (device, moe_row_pairs): the pair of each row, -1 none.  */
+/*   topk_w     float32 [T x k] (device, moe_route_topk).                                      */
+/*   out32      float32 [T x N] workspace, pitch N, 16-byte aligned; the call zeroes it.       */
+/*   out        bf16 [T x N], pitch ldo (multiple of 8, 16-byte aligned).                      */
+/*   Single-SM GEMM tiles only (NVFP4_ERR_UNSUPPORTED_SHAPE while CTA pairs are switched on). */
+nvfp4_status grouped_w4a4_rac_moe_combine(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
+                                          const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
+                                          const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N, int64_t K,
+                                          int32_t Kp, const int32_t* row_pair, const float* topk_w, int64_t T,
+                                          int32_t k, float* out32, uint16_t* out, int64_t ldo, int32_t* dev_status,
+                                          void* stream);
 
 /* ---------------------------------------------------------------------------------------- */
 /* weight_qdq -- trainer-side Asymmetric QAT fake quantisation of weights only (Two fixes):  */

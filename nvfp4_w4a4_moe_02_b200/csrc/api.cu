@@ -21,6 +21,7 @@ std::atomic<uint64_t> g_wait_limit_ns{2000000000ull};
 std::atomic<int> g_tile_n{0};  // 0: automatic
 std::atomic<int> g_act_rows{0}, g_act_warps{0};  // activation quantiser tile: 0 = automatic
 std::atomic<int> g_gemm_pair{0};  // CTA-pair GEMM where the shape allows it
+std::atomic<int> g_qdq_fused{1};  // one-pass fake-quant where the tensors fit
 
 nvfp4_status fail(nvfp4_status s, const char* fmt, ...) {
   char buf[512];
@@ -194,6 +195,8 @@ void nvfp4_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns); }
 void nvfp4_set_gemm_tile_n(int32_t n) { g_tile_n.store((n == 128 || n == 256) ? n : 0); }
 
 void nvfp4_set_gemm_pairs(int32_t on) { g_gemm_pair.store(on ? 1 : 0); }
+
+void nvfp4_set_qdq_one_pass(int32_t on) { g_qdq_fused.store(on ? 1 : 0); }
 
 void nvfp4_set_act_tile(int32_t rows, int32_t warps) {
   g_act_rows.store(rows >= 1 && rows <= 16 ? rows : 0);
@@ -839,12 +842,21 @@ nvfp4_status w4a4_rac_gemm_ex(const nvfp4_tensor* a, const nvfp4_tensor* a_res, 
 }  // extern "C"
 
 namespace {
+// The weighted combine of the down projection's epilogue (grouped_w4a4_rac_moe_combine).
+struct CombineSpec {
+  const int32_t* row_pair;
+  const float* topk_w;
+  int64_t T;
+  int32_t k;
+};
+
 // The grouped GEMM over n_seg row segments; segment i uses weight slab seg_expert[i] (or i).
+// With `comb`, y is the binary32 [T x N] combine accumulator (zeroed here) instead of the rows.
 nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, const int32_t* offsets,
                             const int32_t* seg_rows, const int32_t* seg_expert, int32_t n_seg, const nvfp4_tensor* w,
                             const nvfp4_tensor* w_sel, int64_t N, int64_t K, int32_t Kp, nvfp4_epilogue ep,
                             nvfp4_dtype out, void* y, int64_t ldy, float* amax_out, int32_t* dev_status,
-                            void* stream, uint32_t flags = 0) {
+                            void* stream, uint32_t flags = 0, const CombineSpec* comb = nullptr) {
   if (!offsets) return fail(NVFP4_ERR_INVALID_ARG, "expert_offsets is NULL");
   if (n_seg <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the segment count must be positive");
   if (ep != NVFP4_EPI_NONE && ep != NVFP4_EPI_SWIGLU_AMAX) return fail(NVFP4_ERR_INVALID_ARG, "bad epilogue");
@@ -863,8 +875,9 @@ nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, co
   CUtensorMap maps[5];
   GemmArgs g;
   const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
-  nvfp4_status st = gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, a ? a->rows_padded : 0, bn,
-                                maps, &g, pairs ? 128 : bn, own, ep == NVFP4_EPI_SWIGLU_AMAX);
+  const int64_t y_rows = comb ? comb->T : (a ? a->rows_padded : 0);
+  nvfp4_status st = gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, y_rows, bn, maps, &g,
+                                pairs ? 128 : bn, own, ep == NVFP4_EPI_SWIGLU_AMAX);
   if (st != NVFP4_OK) return st;
   g.offsets = offsets;
   g.expert_rows = seg_rows;
@@ -873,7 +886,7 @@ nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, co
   g.n_weights = (int32_t)E;
   g.M = a->rows_padded;
   g.m_blocks_dense = 0;
-  g.epi = ep == NVFP4_EPI_SWIGLU_AMAX ? 1 : 0;
+  g.epi = ep == NVFP4_EPI_SWIGLU_AMAX ? 1 : comb ? 2 : 0;
   g.amax_out = amax_out;
   g.status = dev_status;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -881,8 +894,19 @@ nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, co
     cudaError_t e = cudaMemsetAsync(amax_out, 0, sizeof(float), s);
     if (e != cudaSuccess) return cuda_fail(e, "amax reset");
   }
-  cudaError_t e = pairs ? launch_gemm_pair(maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms() / 2, s)
-                        : launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms(), s);
+  if (comb) {
+    g.row_pair = comb->row_pair;
+    g.topk_w = comb->topk_w;
+    g.k_top = comb->k;
+    g.n_pairs = comb->T * comb->k;
+    g.comb = reinterpret_cast<float*>(y);
+    g.ld_comb = ldy;
+    cudaError_t e = cudaMemsetAsync(y, 0, (size_t)comb->T * (size_t)ldy * sizeof(float), s);
+    if (e != cudaSuccess) return cuda_fail(e, "combine accumulator reset");
+    if (comb->T == 0) return NVFP4_OK;
+  }
+  cudaError_t e = (pairs && !comb) ? launch_gemm_pair(maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms() / 2, s)
+                                   : launch_gemm(bn, maps[0], maps[1], maps[2], maps[3], maps[4], g, num_sms(), s);
   if (e != cudaSuccess) return cuda_fail(e, "grouped gemm launch");
   return NVFP4_OK;
 }
@@ -922,6 +946,41 @@ nvfp4_status grouped_w4a4_rac_moe_segments(const nvfp4_tensor* a, const nvfp4_te
   if (!seg_expert) return fail(NVFP4_ERR_INVALID_ARG, "seg_expert is NULL");
   return grouped_common(a, a_res, seg_offsets, seg_rows, seg_expert, n_seg, w, w_sel, N, K, Kp, ep, out, y, ldy,
                         amax_out, dev_status, stream);
+}
+
+nvfp4_status grouped_w4a4_rac_moe_combine(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
+                                          const int32_t* expert_offsets, const int32_t* expert_rows, int32_t E,
+                                          const nvfp4_tensor* w, const nvfp4_tensor* w_sel, int64_t N, int64_t K,
+                                          int32_t Kp, const int32_t* row_pair, const float* topk_w, int64_t T,
+                                          int32_t k, float* out32, uint16_t* out, int64_t ldo, int32_t* dev_status,
+                                          void* stream) {
+  g_last_error.clear();
+  if (E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "E must be positive");
+  if (T < 0 || k <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T >= 0 and k > 0 required");
+  if (T > 0 && (!row_pair || !topk_w || !out32 || !out)) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  if (ldo < N || ldo % 8 != 0 || (out && !aligned16(out)))
+    return fail(NVFP4_ERR_ALIGNMENT, "out must be 16-byte aligned with a pitch >= N, a multiple of 8");
+  if (T == 0) return NVFP4_OK;
+  if (g_gemm_pair.load() != 0 && N % 256 == 0 && g_tile_n.load() != 128)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "the combine epilogue runs on single-SM tiles (CTA pairs are on)");
+  const CombineSpec comb{row_pair, topk_w, T, k};
+  nvfp4_status st = grouped_common(a, a_res, expert_offsets, expert_rows, nullptr, E, w, w_sel, N, K, Kp,
+                                   NVFP4_EPI_NONE, NVFP4_OUT_F32, out32, N, nullptr, dev_status, stream, 0, &comb);
+  if (st != NVFP4_OK) return st;
+  cudaError_t e = launch_combine_finalize(out32, T, N, out, ldo, num_sms(), reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "combine finalize launch");
+}
+
+nvfp4_status moe_row_pairs(const int32_t* row_scatter, int64_t T, int32_t k, int64_t rows, int32_t* row_pair,
+                           int32_t* dev_status, void* stream) {
+  g_last_error.clear();
+  if (T < 0 || k <= 0 || rows < 0 || rows > INT32_MAX) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T >= 0, k > 0, 0 <= rows <= INT32_MAX");
+  if (T * k > INT32_MAX) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T * k must fit in int32");
+  if (rows == 0) return NVFP4_OK;
+  if (!row_pair || (T > 0 && !row_scatter)) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");
+  cudaError_t e = launch_row_pairs(row_scatter, T * k, rows, row_pair, num_sms(), dev_status,
+                                   reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? NVFP4_OK : cuda_fail(e, "row pairs launch");
 }
 
 nvfp4_status nvfp4_amax(const uint16_t* x, int64_t M, int64_t K, int64_t ldx, float* amax_out, void* workspace,
@@ -1102,7 +1161,10 @@ nvfp4_status moe_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const i
 // ------------------------------------------------------------------------------------------ qdq
 size_t weight_qdq_workspace_size(int64_t n_tensors, int64_t elems_per_tensor) {
   (void)elems_per_tensor;
-  return round_up((size_t)(n_tensors > 0 ? n_tensors : 1) * (size_t)slab_partials(n_tensors) * sizeof(float), 256);
+  const size_t n = (size_t)(n_tensors > 0 ? n_tensors : 1);
+  const size_t partials = n * (size_t)slab_partials(n_tensors) * sizeof(float);
+  const size_t words = n * 2 * sizeof(uint32_t);  // one-pass form: amax and arrival count per tensor
+  return round_up(partials > words ? partials : words, 256);
 }
 
 nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_tensor, uint16_t* w_out,
@@ -1115,6 +1177,17 @@ nvfp4_status weight_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems_per_
   if (!workspace || workspace_bytes < weight_qdq_workspace_size(n_tensors, elems_per_tensor))
     return fail(NVFP4_ERR_INVALID_ARG, "workspace too small");
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // one pass over HBM when two tensors per CTA group fit in L2 next to each other: tensors of up
+  // to 4M elements (8 MB of bf16); larger ones take the two passes (amax, then the fake-quant)
+  if (g_qdq_fused.load() && elems_per_tensor <= (4ll << 20)) {
+    uint32_t* sync_ws = reinterpret_cast<uint32_t*>(workspace);
+    cudaError_t e = cudaMemsetAsync(sync_ws, 0, (size_t)n_tensors * 2 * sizeof(uint32_t), s);
+    if (e == cudaSuccess)
+      e = launch_qdq_fused(w, n_tensors, elems_per_tensor, w_out, sync_ws, 0, s_g_out, dev_status,
+                           g_wait_limit_ns.load(), num_sms(), s);
+    if (e == cudaSuccess) return NVFP4_OK;
+    cudaGetLastError();  // a grid that cannot be co-resident: the two-pass form below
+  }
   float* partial = reinterpret_cast<float*>(workspace);
   const int P = slab_partials(n_tensors);
   cudaError_t e = launch_amax(w, n_tensors, 1, elems_per_tensor, elems_per_tensor, partial, P, dev_status, s);

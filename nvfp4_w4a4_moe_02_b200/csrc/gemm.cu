@@ -349,11 +349,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         if (OWN) {
           const int base = i >= NCH / 2 ? BN : 0;
           const int ii = i % (NCH / 2);
-          if (args.epi == 0) return base + half * (BN / 2) + 32 * ii;
+          if (args.epi != 1) return base + half * (BN / 2) + 32 * ii;
           const int f = half * (BN / 4);
           return base + (f / 64) * 128 + (f % 64) + (ii == 1 ? 64 : 0);
         }
-        if (args.epi == 0) return half * (BN / 2) + 32 * i;
+        if (args.epi != 1) return half * (BN / 2) + 32 * i;
         const int ii = i % (NCH / 2);
         const int f = half * (BN / 4) + 32 * ii;
         return (f / 64) * 128 + (f % 64) + (i >= NCH / 2 ? 64 : 0);
@@ -419,6 +419,25 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       constexpr int NOUT = OWN ? NCH / 2 : NCH;
       if (!box_live) {
         // padding only: nothing to store
+      } else if (args.epi == 2) {
+        // weighted combine: this row's products w * bf16(alpha * acc) go into its token's binary32
+        // row by vector atomic adds (the order of a token's k terms is not fixed)
+        const int32_t pair = row_ok ? __ldg(args.row_pair + row) : -1;
+        if (pair >= 0 && (int64_t)pair >= args.n_pairs) report_status(args.status, kErrInvalid);
+        if (pair >= 0 && (int64_t)pair < args.n_pairs) {
+          const float wt = __ldg(args.topk_w + pair);
+          float* dst = args.comb + (int64_t)(pair / args.k_top) * args.ld_comb + (int64_t)nb * BN;
+#pragma unroll
+          for (int i = 0; i < NOUT; ++i)
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              float o[4];
+#pragma unroll
+              for (int z = 0; z < 4; ++z)
+                o[z] = __fmul_rn(wt, bf16_round(__fmul_rn(__uint_as_float(v[i][4 * q + z]), alpha_out)));
+              red_add_v4(dst + chunk_col(i) + 4 * q, o);
+            }
+        }
       } else if (args.epi == 0 && args.out_bf16) {
         // 64 columns per box
 #pragma unroll

@@ -101,6 +101,9 @@ cudaError_t launch_qdq(const uint16_t* w, int64_t n_tensors, int64_t elems, uint
                        float* s_g_out, int32_t* status, int num_sms, cudaStream_t st);
 cudaError_t launch_unpack_logical(const uint8_t* codes, const uint8_t* sf, int64_t rows, int64_t cols, int slab16,
                                   uint8_t* codes_out, uint8_t* sf_out, int num_sms, cudaStream_t st);
+int qdq_fused_group(int64_t n_tensors, int64_t elems, int grid);
+cudaError_t launch_qdq_fused(const uint16_t* w, int64_t n_tensors, int64_t elems, uint16_t* out, uint32_t* sync_ws,
+                             int GS, float* s_g_out, int32_t* status, uint64_t limit_ns, int num_sms, cudaStream_t st);
 cudaError_t launch_qdq_backward(const uint16_t* g, int64_t n, uint16_t* gw, float* acc, int num_sms, cudaStream_t st);
 cudaError_t launch_encode_e2m1(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
 cudaError_t launch_encode_e4m3(const float* v, int64_t n, uint8_t* out, cudaStream_t st);
@@ -151,13 +154,21 @@ struct GemmArgs {
   void* y;
   int64_t ldy;
   int32_t out_bf16;
-  int32_t epi;               // 0 none, 1 SwiGLU + amax
+  int32_t epi;               // 0 none, 1 SwiGLU + amax, 2 weighted combine (row_pair, topk_w -> comb)
   float* amax_out;
   int32_t* status;
   uint64_t wait_limit_ns;
   int32_t fp8;               // 1: the FP8 comparison operands (E4M3, E8M0 per 32; kt_main = K/128, no residual)
   int32_t own_res_scale;     // 1: the residual has its own tensor scale *s_a_res (two accumulators, BN = 128)
   const float* s_a_res;      // own_res_scale: device scalar
+  // epi == 2: row r's products topk_w[p] * bf16(alpha * acc) are added into comb[p / k_top]
+  // (binary32, pitch ld_comb), p = row_pair[r] (< 0: no pair; >= n_pairs: reported)
+  const int32_t* row_pair;
+  const float* topk_w;
+  int32_t k_top;
+  int64_t n_pairs;
+  float* comb;
+  int64_t ld_comb;
 };
 
 // bn: 128 or 256
@@ -192,7 +203,7 @@ struct DecodeArgs {
   void* y;
   int64_t ldy;
   int32_t out_bf16;
-  int32_t epi;               // 0 none, 1 SwiGLU + amax
+  int32_t epi;               // 0 none, 1 SwiGLU + amax, 2 weighted combine (row_pair, topk_w -> comb)
   float* amax_out;
   int32_t* status;
   uint64_t wait_limit_ns;
@@ -210,6 +221,10 @@ cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, in
                                  int32_t* slot_expert, int32_t* slot_count, int n_slots, int num_sms,
                                  int32_t* status, cudaStream_t st);
 cudaError_t launch_row_groups(const int32_t* off, int E, int64_t rows, int32_t* group, int num_sms, cudaStream_t st);
+cudaError_t launch_row_pairs(const int32_t* row_scatter, int64_t n, int64_t rows, int32_t* row_pair, int num_sms,
+                             int32_t* status, cudaStream_t st);
+cudaError_t launch_combine_finalize(const float* acc, int64_t T, int64_t H, uint16_t* out, int64_t ldo, int num_sms,
+                                    cudaStream_t st);
 cudaError_t launch_combine(const uint16_t* y, int64_t ldy, int64_t y_rows, const int32_t* rows, const float* w,
                            int64_t T, int k, int64_t H, uint16_t* out, int64_t ldo, int num_sms, int32_t* status,
                            cudaStream_t st);

@@ -235,8 +235,67 @@ __global__ void __launch_bounds__(256) row_groups_kernel(const int32_t* __restri
 }
 
 // ----------------------------------------------------------------------------------------
+// inverse of the pair -> row map: row_pair[row_scatter[p]] = p for every routed pair p = t*k + j
+// (the caller's memset leaves -1 on the other rows); a row past `rows` is reported
+// ----------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) row_pairs_kernel(const int32_t* __restrict__ row_scatter, int64_t n,
+                                                        int64_t rows, int32_t* __restrict__ row_pair,
+                                                        int32_t* status) {
+  for (int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; p < n; p += (int64_t)gridDim.x * blockDim.x) {
+    const int32_t r = __ldg(row_scatter + p);
+    if (r < 0) continue;
+    if (r >= rows) {
+      report_status(status, kErrInvalid);
+      continue;
+    }
+    row_pair[r] = (int32_t)p;
+  }
+}
+
+// binary32 combine sums -> bf16 rows (8 features per thread)
+__global__ void __launch_bounds__(256) combine_finalize_kernel(const float* __restrict__ acc, int64_t T, int64_t H,
+                                                               uint16_t* __restrict__ out, int64_t ldo) {
+  const int64_t per_tok = H / 8;
+  const int64_t n = T * per_tok;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / per_tok;
+    const int64_t h = (i - t * per_tok) * 8;
+    const float4 a = __ldg(reinterpret_cast<const float4*>(acc + t * H + h));
+    const float4 b = __ldg(reinterpret_cast<const float4*>(acc + t * H + h + 4));
+    const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    uint4 o;
+    uint32_t* ow = reinterpret_cast<uint32_t*>(&o);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      __nv_bfloat162 p = __floats2bfloat162_rn(v[2 * c], v[2 * c + 1]);
+      ow[c] = *reinterpret_cast<uint32_t*>(&p);
+    }
+    *reinterpret_cast<uint4*>(out + t * ldo + h) = o;
+  }
+}
+
+// ----------------------------------------------------------------------------------------
 // launchers
 // ----------------------------------------------------------------------------------------
+cudaError_t launch_row_pairs(const int32_t* row_scatter, int64_t n, int64_t rows, int32_t* row_pair, int num_sms,
+                             int32_t* status, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(row_pair, 0xFF, sizeof(int32_t) * (size_t)rows, st);  // -1: no pair
+  if (e != cudaSuccess || n == 0) return e;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+  row_pairs_kernel<<<(unsigned)blocks, 256, 0, st>>>(row_scatter, n, rows, row_pair, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine_finalize(const float* acc, int64_t T, int64_t H, uint16_t* out, int64_t ldo, int num_sms,
+                                    cudaStream_t st) {
+  const int64_t n = T * (H / 8);
+  if (n == 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > (int64_t)num_sms * 16) blocks = (int64_t)num_sms * 16;
+  combine_finalize_kernel<<<(unsigned)blocks, 256, 0, st>>>(acc, T, H, out, ldo);
+  return cudaGetLastError();
+}
 cudaError_t launch_row_groups(const int32_t* off, int E, int64_t rows, int32_t* group, int num_sms, cudaStream_t st) {
   int64_t blocks = (rows + 255) / 256;
   if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;

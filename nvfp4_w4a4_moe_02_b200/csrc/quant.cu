@@ -5,6 +5,9 @@
 // block (one shuffle for the block max), packed e2m1 stores that stay contiguous across the
 // warp, and scales written straight into the 512-byte scale atoms the tcgen05 MMA reads.
 #include "common.cuh"
+#include <algorithm>
+#include <climits>
+
 #include "kernels.h"
 
 namespace nvfp4 {
@@ -562,6 +565,149 @@ __global__ void __launch_bounds__(256) qdq_kernel(const uint16_t* __restrict__ w
 }
 
 // ----------------------------------------------------------------------------------------
+// K8 in one pass over HBM: groups of GS co-resident CTAs (a cooperative launch) take tensors
+// group, group + n_groups, ...  A CTA reduces max|w| over its slice of a tensor, folds it into
+// the tensor's word of the workspace and counts itself in; once all GS are in (a bounded wait on
+// the counter) it reads the tensor scale and fake-quantises its slice, reading it a second time,
+// now from L2.  The wait on tensor t comes after the amax pass over the group's next tensor, so
+// the meeting is hidden behind HBM reads; two tensors per group are in flight, which the host
+// keeps well inside L2.  HBM sees each weight read once and written once: 4 bytes per element.
+// ----------------------------------------------------------------------------------------
+__device__ __forceinline__ uint64_t l2_policy_keep() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint64_t l2_policy_stream() {
+  uint64_t p;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+  return p;
+}
+__device__ __forceinline__ uint4 ld_hint(const uint16_t* p, uint64_t pol) {
+  uint4 v;
+  asm volatile("ld.global.nc.L2::cache_hint.v4.u32 {%0, %1, %2, %3}, [%4], %5;"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p), "l"(pol));
+  return v;
+}
+__device__ __forceinline__ void st_hint(uint16_t* p, const uint4 v, uint64_t pol) {
+  asm volatile("st.global.L2::cache_hint.v4.u32 [%0], {%1, %2, %3, %4}, %5;" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w), "l"(pol)
+               : "memory");
+}
+
+// max |w| over elements [v_lo*8, v_hi*8) of one tensor, four 16-byte loads in flight per thread
+__device__ __forceinline__ float slice_amax(const uint16_t* wt, int64_t v_lo, int64_t v_hi, uint64_t pol,
+                                            bool& nonfinite) {
+  float m = 0.0f;
+  const int64_t stride = blockDim.x;
+  for (int64_t i0 = v_lo + threadIdx.x; i0 < v_hi; i0 += 4 * stride) {
+    uint4 q[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      q[u] = (i0 + u * stride < v_hi) ? ld_hint(wt + 8 * (i0 + u * stride), pol) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t wq[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const float a = fabsf(bf16_bits_to_f32(wq[j] & 0xFFFFu)), b = fabsf(bf16_bits_to_f32(wq[j] >> 16));
+        nonfinite |= !(a <= 3.4e38f) || !(b <= 3.4e38f);
+        m = fmaxf(m, fmaxf(a, b));
+      }
+    }
+  }
+  return m;
+}
+
+__global__ void __launch_bounds__(256, 4) qdq_fused_kernel(const uint16_t* __restrict__ w, int64_t n_tensors,
+                                                           int64_t elems, uint16_t* __restrict__ out,
+                                                           uint32_t* __restrict__ sync_ws, int GS, float* s_g_out,
+                                                           int32_t* status, uint64_t limit_ns) {
+  __shared__ float red[8];
+  __shared__ float sg_sh;
+  __shared__ int bad_sh;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
+  const int n_groups = (int)(gridDim.x / GS);
+  const int group = (int)(blockIdx.x / GS), rank = (int)(blockIdx.x % GS);
+  if (group >= n_groups) return;  // a CTA beyond the last whole group has no tensor
+  const int64_t chunks = (elems + 511) / 512;  // 512-element chunks (one warp step of the fake-quant)
+  const int64_t c_lo = chunks * rank / GS, c_hi = chunks * (rank + 1) / GS;
+  const int64_t v_lo = c_lo * 64, v_hi = min(c_hi * 64, elems / 8);
+  const uint64_t keep = l2_policy_keep(), stream = l2_policy_stream();
+  bool nonfinite = false;
+
+  // amax pass over tensor t, then this CTA's arrival at the tensor's counter
+  auto amax_and_arrive = [&](int64_t t) {
+    float m = warp_max(slice_amax(w + t * elems, v_lo, v_hi, keep, nonfinite));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float mm = 0.0f;
+      for (int i = 0; i < nw; ++i) mm = fmaxf(mm, red[i]);
+      atomicMax(sync_ws + 2 * t, __float_as_uint(mm));  // non-negative floats order as their bits
+      __threadfence();
+      atomicAdd(sync_ws + 2 * t + 1, 1u);
+    }
+  };
+
+  int64_t t = group;
+  if (t < n_tensors) amax_and_arrive(t);
+  for (; t < n_tensors; t += n_groups) {
+    if (t + n_groups < n_tensors) amax_and_arrive(t + n_groups);
+    if (threadIdx.x == 0) {
+      const uint32_t* count = sync_ws + 2 * t + 1;
+      bool ok = false;
+      const uint64_t t0 = globaltimer_ns();
+      while (true) {
+        uint32_t c;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(c) : "l"(count) : "memory");
+        if (c >= (uint32_t)GS) {
+          ok = true;
+          break;
+        }
+        if (globaltimer_ns() - t0 > limit_ns) break;
+        __nanosleep(100);
+      }
+      if (!ok) report_status(status, kErrTimeout);
+      uint32_t am;
+      asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(am) : "l"(sync_ws + 2 * t) : "memory");
+      const float s_g = scale_from_amax(__uint_as_float(am), status);
+      if (ok && rank == 0 && s_g_out) s_g_out[t] = s_g;
+      sg_sh = s_g;
+      bad_sh = ok ? 0 : 1;
+    }
+    __syncthreads();
+    if (bad_sh) break;
+    const float s_g = sg_sh, t6 = __fmul_rn(6.0f, s_g);
+    // the fake-quant of this CTA's chunks, one warp per 512-element chunk (lane pairs hold the two
+    // halves of a 16-block), the next chunk's loads issued before this one's arithmetic
+    const uint16_t* wt = w + t * elems;
+    uint16_t* ot = out + t * elems;
+    int64_t ch = c_lo + warp;
+    int64_t e0 = ch * 512 + 8 * lane, e1 = e0 + 256;
+    uint4 n0 = (ch < c_hi && e0 < elems) ? ld_hint(wt + e0, stream) : make_uint4(0, 0, 0, 0);
+    uint4 n1 = (ch < c_hi && e1 < elems) ? ld_hint(wt + e1, stream) : make_uint4(0, 0, 0, 0);
+    for (; ch < c_hi; ch += nw) {
+      const uint4 q0 = n0, q1 = n1;
+      const int64_t f0 = e0, f1 = e1;
+      e0 += 512 * nw;
+      e1 += 512 * nw;
+      if (ch + nw < c_hi) {
+        n0 = e0 < elems ? ld_hint(wt + e0, stream) : make_uint4(0, 0, 0, 0);
+        n1 = e1 < elems ? ld_hint(wt + e1, stream) : make_uint4(0, 0, 0, 0);
+      }
+      uint4 o0, o1;
+      qdq_half(q0, s_g, t6, o0);
+      qdq_half(q1, s_g, t6, o1);
+      if (f0 < elems) st_hint(ot + f0, o0, stream);
+      if (f1 < elems) st_hint(ot + f1, o1, stream);
+    }
+  }
+  if (nonfinite) report_status(status, kErrRange);
+}
+
+// ----------------------------------------------------------------------------------------
 // logical view of a packed matrix: one code per byte, scales row-major [rows x cols/16]
 // ----------------------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) unpack_logical_kernel(const uint8_t* __restrict__ codes,
@@ -742,6 +888,46 @@ cudaError_t launch_unpack_logical(const uint8_t* codes, const uint8_t* sf, int64
   if (grid > (int64_t)num_sms * 16) grid = (int64_t)num_sms * 16;
   if (grid < 1) grid = 1;
   unpack_logical_kernel<<<(unsigned)grid, 256, 0, st>>>(codes, sf, rows, cols, slab16, codes_out, sf_out);
+  return cudaGetLastError();
+}
+
+// CTAs per group for the one-pass fake-quant on `grid` co-resident CTAs: the fewest slice-steps
+// per CTA (rounds of tensors x 512-element chunks per slice) while the two tensors per group in
+// flight stay within 48 MB of L2; ties go to the smaller group (fewer CTAs meet per tensor).
+int qdq_fused_group(int64_t n_tensors, int64_t elems, int grid) {
+  const int64_t chunks = (elems + 511) / 512;
+  const double budget = 48.0 * (1 << 20);
+  int best = 0;
+  int64_t best_cost = INT64_MAX;
+  for (int gs = 1; gs <= grid; ++gs) {
+    const int64_t ng = grid / gs;
+    if ((double)std::min<int64_t>(ng, n_tensors) * 2.0 * (double)elems * 2.0 > budget) continue;
+    const int64_t cost = ((n_tensors + ng - 1) / ng) * ((chunks + gs - 1) / gs);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = gs;
+    }
+  }
+  return best;
+}
+
+// Grid of the fused fake-quant: co-resident CTAs (occupancy x SMs, at most 4 per SM) in whole
+// groups of GS CTAs (GS <= 0: chosen by qdq_fused_group).
+cudaError_t launch_qdq_fused(const uint16_t* w, int64_t n_tensors, int64_t elems, uint16_t* out, uint32_t* sync_ws,
+                             int GS, float* s_g_out, int32_t* status, uint64_t limit_ns, int num_sms,
+                             cudaStream_t st) {
+  int per_sm = 0;
+  cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, qdq_fused_kernel, 256, 0);
+  if (e != cudaSuccess) return e;
+  if (per_sm > 4) per_sm = 4;
+  const int grid_max = num_sms * per_sm;
+  if (GS <= 0) GS = qdq_fused_group(n_tensors, elems, grid_max);
+  if (GS <= 0 || GS > grid_max) return cudaErrorInvalidValue;
+  int grid = grid_max / GS * GS;
+  void* args[] = {(void*)&w, (void*)&n_tensors, (void*)&elems, (void*)&out, (void*)&sync_ws, (void*)&GS,
+                  (void*)&s_g_out, (void*)&status, (void*)&limit_ns};
+  e = cudaLaunchCooperativeKernel((const void*)qdq_fused_kernel, dim3((unsigned)grid), dim3(256), args, 0, st);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -168,6 +168,12 @@ __device__ __forceinline__ int find_expert(const int32_t* off, int E, int64_t ro
   return lo;
 }
 
+// four binary32 atomic adds to 16 consecutive bytes of global memory (one vector reduction)
+__device__ __forceinline__ void red_add_v4(float* p, const float (&v)[4]) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3])
+               : "memory");
+}
+
 __device__ __forceinline__ float bf16_round(float x) { return __bfloat162float(__float2bfloat16_rn(x)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {

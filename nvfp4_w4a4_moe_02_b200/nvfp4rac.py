@@ -64,6 +64,7 @@ def load() -> ctypes.CDLL:
         "nvfp4_set_gemm_tile_n": ([i32], None),
         "nvfp4_set_act_tile": ([i32, i32], None),
         "nvfp4_set_gemm_pairs": ([i32], None),
+        "nvfp4_set_qdq_one_pass": ([i32], None),
         "nvfp4_quantize_workspace_size": ([i64, i64], sz),
         "nvfp4_quantize": ([vp, i64, i64, i64, vp, i64, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
         "nvfp4_quantize_scatter": ([vp, i64, i64, i64, vp, i32, vp, i32, vp, tp, tp, vp, sz, vp, vp], ctypes.c_int),
@@ -102,6 +103,9 @@ def load() -> ctypes.CDLL:
         "moe_dispatch_workspace_size": ([i32], sz),
         "moe_dispatch_plan": ([vp, i64, i32, i32, i32, i64, vp, vp, vp, vp, vp, i32, vp, sz, vp, vp], ctypes.c_int),
         "moe_combine": ([vp, i64, i64, vp, vp, i64, i32, i64, vp, i64, vp, vp], ctypes.c_int),
+        "moe_row_pairs": ([vp, i64, i32, i64, vp, vp, vp], ctypes.c_int),
+        "grouped_w4a4_rac_moe_combine": ([tp, tp, vp, vp, i32, tp, tp, i64, i64, i32, vp, vp, i64, i32, vp, vp, i64,
+                                          vp, vp], ctypes.c_int),
         "weight_qdq_workspace_size": ([i64, i64], sz),
         "weight_qdq": ([vp, i64, i64, vp, vp, vp, sz, vp, vp], ctypes.c_int),
         "weight_qdq_backward": ([vp, i64, vp, vp, vp], ctypes.c_int),
@@ -244,6 +248,11 @@ def set_gemm_tile_n(n: int):
 def set_gemm_pairs(on: bool):
     """Run the GEMMs with N % 256 == 0 on CTA pairs (default) or on single SMs."""
     load().nvfp4_set_gemm_pairs(1 if on else 0)
+
+
+def set_qdq_one_pass(on: bool):
+    """weight_qdq in one pass over HBM (default, tensors of up to 4M elements) or in two."""
+    load().nvfp4_set_qdq_one_pass(1 if on else 0)
 
 
 def set_act_tile(rows: int, warps: int):
@@ -611,6 +620,49 @@ def moe_combine(y: torch.Tensor, row_scatter: torch.Tensor, w: torch.Tensor, out
     st = status if status is not None else new_status(y.device)
     _check(lib.moe_combine(y.data_ptr(), y.stride(0), y.shape[0], row_scatter.data_ptr(), w.data_ptr(), T, k, H,
                            out.data_ptr(), out.stride(0), st.data_ptr(), _stream(stream)))
+    return out
+
+
+def moe_row_pairs(row_scatter: torch.Tensor, rows: int, row_pair: torch.Tensor | None = None,
+                  status: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """row_pair[r] = t * k + j for row_scatter[t, j] = r, -1 elsewhere (device int32 [rows])."""
+    lib = load()
+    T, k = row_scatter.shape
+    assert row_scatter.dtype == torch.int32 and row_scatter.is_contiguous()
+    if row_pair is None:
+        row_pair = torch.empty(rows, dtype=torch.int32, device=row_scatter.device)
+    st = status if status is not None else new_status(row_scatter.device)
+    _check(lib.moe_row_pairs(row_scatter.data_ptr(), T, k, rows, row_pair.data_ptr(), st.data_ptr(),
+                             _stream(stream)))
+    return row_pair
+
+
+def grouped_w4a4_rac_moe_combine(a: Packed, a_res: Packed | None, expert_offsets: torch.Tensor, w: Packed,
+                                 w_sel: Packed | None, row_pair: torch.Tensor, topk_w: torch.Tensor,
+                                 out: torch.Tensor | None = None, out32: torch.Tensor | None = None,
+                                 status: torch.Tensor | None = None, stream=None,
+                                 expert_rows: torch.Tensor | None = None) -> torch.Tensor:
+    """Down projection with the weighted combine in the GEMM epilogue -> bf16 [T, N]."""
+    lib = load()
+    E = w.slabs
+    N, K = w.rows, w.cols
+    Kp = 0 if a_res is None else a_res.cols
+    T, k = topk_w.shape
+    dev = a.codes.device
+    assert topk_w.dtype == torch.float32 and topk_w.is_contiguous() and row_pair.dtype == torch.int32
+    if out is None:
+        out = torch.empty(T, N, dtype=torch.bfloat16, device=dev)
+    if out32 is None:
+        out32 = torch.empty(T, N, dtype=torch.float32, device=dev)
+    st = status if status is not None else new_status(dev)
+    ca, cw = a.c(), w.c()
+    car = a_res.c() if Kp > 0 else None
+    cws = w_sel.c() if Kp > 0 else None
+    _check(lib.grouped_w4a4_rac_moe_combine(ctypes.byref(ca), ctypes.byref(car) if car else None,
+                                            expert_offsets.data_ptr(), _ptr(expert_rows), E, ctypes.byref(cw),
+                                            ctypes.byref(cws) if cws else None, N, K, Kp, row_pair.data_ptr(),
+                                            topk_w.data_ptr(), T, k, out32.data_ptr(), out.data_ptr(), out.stride(0),
+                                            st.data_ptr(), _stream(stream)))
     return out
 
 

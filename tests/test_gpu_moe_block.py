@@ -162,6 +162,57 @@ def test_prefill_pipeline_with_device_plan(dev, orc):
     assert np.all(np.abs(got - ref) <= k * 2.0 ** -23 * absdot + bf16_ulp(ref))
 
 
+@pytest.mark.parametrize("with_rows", [True, False])
+def test_down_projection_with_fused_combine(dev, orc, with_rows):
+    """grouped_w4a4_rac_moe_combine (the weighted combine in the down GEMM's epilogue) against the
+    oracle's combine of the unfused down projection's rows, and moe_row_pairs against the
+    inverse of the plan's row map; both tile widths of the down GEMM (N = 512 and 384)."""
+    for H in (512, 384):
+        wl = syn.moe_block(T=300, H=H, E=8, topk=3, I=256, T_cal=64)
+        sel_dn, _ = orc.calibrate(syn.moe_down_calibration_batch(wl), wl.Kp_dn)
+        st = R.new_status(dev)
+        T, k = wl.topk_ids.shape
+        ids = torch.from_numpy(wl.topk_ids.astype(np.int32)).to(dev)
+        cap = R.moe_rows_capacity(T, k, wl.E, 128)
+        off, rows, _, _ = R.moe_dispatch_plan(ids, wl.E, 128, rows_capacity=cap, status=st)
+        er = torch.empty(wl.E, dtype=torch.int32, device=dev)
+        R.moe_dispatch_plan(ids, wl.E, 128, rows_capacity=cap, offsets=off, row_scatter=rows, expert_rows=er,
+                            status=st)
+        # h: any bf16 rows in the padded expert-grouped order
+        h_np = syn.normal_bf16(7, 3, cap, wl.I, 1.0)
+        seld = torch.from_numpy(sel_dn).to(dev)
+        hq, hqr = R.nvfp4_quantize(to_dev(h_np, dev), seld, status=st)
+        pdn, pdns = R.pack_weights(to_dev(wl.wdn, dev), seld, status=st)
+        _, w_np = orc.route_topk(router_logits(T, wl.E, seed=3), k)
+        wd = torch.from_numpy(w_np).to(dev)
+        pairs = R.moe_row_pairs(rows, cap, status=st)
+        kw = {"expert_rows": er} if with_rows else {}
+        y = R.grouped_w4a4_rac_moe(hq, hqr, off, pdn, pdns, status=st, **kw)
+        out = R.grouped_w4a4_rac_moe_combine(hq, hqr, off, pdn, pdns, pairs, wd, status=st, **kw)
+        torch.cuda.synchronize()
+        R.check_status(st)
+        rows_np, pairs_np = rows.cpu().numpy(), pairs.cpu().numpy()
+        inv = np.full(cap, -1, np.int64)
+        inv[rows_np.reshape(-1)] = np.arange(T * k)
+        assert np.array_equal(pairs_np, inv)
+        yb = bf16_bits(y)
+        ref = orc.combine(yb, rows_np.astype(np.int64), w_np)
+        absdot = orc.combine(syn._f32_to_bf16_bits(np.abs(syn.bf16_to_f32(yb))), rows_np.astype(np.int64), w_np)
+        got = syn.bf16_to_f32(bf16_bits(out)).astype(np.float64)
+        tol = k * 2.0 ** -23 * absdot + bf16_ulp(ref)
+        bad = np.argwhere(np.abs(got - ref) > tol)
+        assert bad.size == 0, (H, bad[:5])
+
+
+def test_row_pairs_rejects_rows_past_the_buffer(dev):
+    rows = torch.tensor([[0, 5], [-1, 9]], dtype=torch.int32, device=dev)
+    st = R.new_status(dev)
+    pairs = R.moe_row_pairs(rows, 8, status=st)
+    torch.cuda.synchronize()
+    assert int(st.item()) == 1
+    assert pairs.cpu().numpy().tolist() == [0, -1, -1, -1, -1, 1, -1, -1]
+
+
 def test_decode_pipeline_with_device_slot_tables(dev, orc):
     """Decode driven by device slot tables (worst-case slot count, unused slots skipped) gives the
     host-slot pipeline's rows bit for bit."""

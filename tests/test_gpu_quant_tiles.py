@@ -207,3 +207,29 @@ def test_weight_qdq_backward_is_straight_through(dev):
     y.backward(up)
     assert torch.equal(w.grad.view(torch.int16), up.view(torch.int16))
     assert w.grad.dtype == torch.bfloat16 and w.grad.shape == w.shape
+
+
+@pytest.mark.parametrize("n,elems", [(1, 16), (5, 512 * 3 + 48), (37, 4096), (600, 1040), (3, 4 << 20)])
+def test_weight_qdq_one_pass_equals_two_pass(dev, orc, n, elems):
+    """The one-pass fake-quant (CTA groups meeting at a per-tensor counter) and the two-pass form
+    give the same bits and scales; sampled tensors also against the oracle."""
+    w = syn.normal_bf16(5, 11, n, elems, 0.02)
+    w[n - 1, : min(16, elems)] = syn.normal_bf16(5, 12, 1, min(16, elems), 2.0)[0]
+    wd = to_dev(w, dev)
+    st = torch.zeros(1, dtype=torch.int32, device=dev)
+    try:
+        R.set_qdq_one_pass(True)
+        o1, s1 = R.weight_qdq(wd, status=st)
+        R.set_qdq_one_pass(False)
+        o2, s2 = R.weight_qdq(wd, status=st)
+    finally:
+        R.set_qdq_one_pass(True)
+    torch.cuda.synchronize()
+    assert st.item() == 0
+    assert torch.equal(s1, s2)
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16))
+    got = o1.view(torch.int16).cpu().numpy().view(np.uint16).reshape(n, elems)
+    for t in sorted({0, n // 2, n - 1}):
+        ref, s_ref = orc.weight_qdq(w[t])
+        assert s1[t].item() == float(s_ref)
+        assert np.array_equal(got[t], ref), (t, np.argwhere(got[t] != ref)[:5])
