@@ -399,7 +399,7 @@ class MoEBlockStep:
     # the combine in the down GEMM's epilogue: + row pairs, the combine kernel becomes the bf16 finalise
     KERNELS_PER_STEP = 10
 
-    def __init__(self, wl, packed, sel_gu, sel_dn, decode, dev):
+    def __init__(self, wl, packed, sel_gu, sel_dn, decode, dev, fused_combine=False):
         import torch
 
         from nvfp4_w4a4_moe_02_b200 import nvfp4rac as R
@@ -433,7 +433,9 @@ class MoEBlockStep:
         self.hq = P.empty(self.cap, wl.I, rows_padded=self.cap, device=dev, sf_layout=lay, zero=True)
         self.hqr = P.empty(self.cap, wl.Kp_dn, rows_padded=self.cap, device=dev, sf_layout=lay, zero=True)
         self.slot_first_row = torch.arange(self.n_slots, dtype=torch.int32, device=dev) * 16 if decode else None
-        self.fused_combine = not decode
+        # the combine in the down GEMM's epilogue (atomic binary32 adds) measured slower than the
+        # bf16 rows + combine kernel on the prefill block; kept as an option
+        self.fused_combine = fused_combine and not decode
         self.kernels_per_step = self.KERNELS_PER_STEP + (1 if self.fused_combine else 0)
         if self.fused_combine:
             self.row_pair = torch.empty(self.cap, dtype=torch.int32, device=dev)
@@ -483,8 +485,12 @@ class MoEBlockStep:
             if "c0" in ev:
                 ev["c0"].record()
         else:
-            R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.se, self.sc, self.pdn, self.pdns, y=self.ye,
-                                          status=self.status)
+            if self.decode:
+                R.grouped_w4a4_rac_moe_decode(self.hq, self.hqr, self.se, self.sc, self.pdn, self.pdns, y=self.ye,
+                                              status=self.status)
+            else:
+                R.grouped_w4a4_rac_moe(self.hq, self.hqr, self.off, self.pdn, self.pdns, y=self.ye,
+                                       status=self.status, expert_rows=self.expert_rows)
             if "c0" in ev:
                 ev["c0"].record()
             R.moe_combine(self.ye, self.rows, self.w, out=self.y, status=self.status)
@@ -851,7 +857,8 @@ def _spec_block(dev, args, decode):
     else:
         wl, h_cal = build_inputs(experts=args.experts)
         inner = MoEStep(wl, h_cal, dev)
-    step = MoEBlockStep(wl, (inner.pgu, inner.pgus, inner.pdn, inner.pdns), inner.sel_gu, inner.sel_dn, decode, dev)
+    step = MoEBlockStep(wl, (inner.pgu, inner.pgus, inner.pdn, inner.pdns), inner.sel_gu, inner.sel_dn, decode, dev,
+                        fused_combine=bool(getattr(args, "fused_combine", False)))
     # the device router must reproduce the workload's routing (same logits, same reading)
     step.run()
     import torch
@@ -873,6 +880,7 @@ def _spec_block(dev, args, decode):
         dominant=("gate_up", gu_f, gu_bytes, "gate_up W4A4+RAC GEMM of the layer (SwiGLU epilogue)"),
         quant={}, config={"workload": name, "tokens": T, "experts": wl.E, "hidden": wl.H, "intermediate": wl.I,
                           "plan": "device (router top-k, dispatch plan); combine into [T, H]",
+                          "combine": "in the down GEMM's epilogue" if step.fused_combine else "combine kernel",
                           "rows_capacity": step.cap},
         cpu=lambda: None, kernels_per_step=step.kernels_per_step)
 
@@ -1074,6 +1082,8 @@ def main():
                     help="GEMMs on CTA pairs (1) or single SMs (0); default: the library's choice")
     ap.add_argument("--qdq-tensors", type=int, default=1024,
                     help="qdq workload: number of 1024 x 2048 tensors (1024 = 2^31 elements; fewer for profiler captures)")
+    ap.add_argument("--fused-combine", action="store_true",
+                    help="layer workloads (prefill): the weighted combine in the down GEMM's epilogue")
     ap.add_argument("--experts", type=int, default=None,
                     help="MoE workloads: expert count override (smaller device footprint for profiler captures)")
     args = ap.parse_args()

@@ -53,25 +53,28 @@ __device__ __forceinline__ uint32_t e2m1_encode8(const float v[8]) {
   return out;
 }
 
-// Eight E2M1 codes (nibble i = element i) -> their values, exact.  The eight magnitudes
-// {0, .5, 1, 1.5, 2, 3, 4, 6} are exact bf16 numbers; their high and low bytes are looked up
-// with byte permutes (index = code & 7), the sign is code bit 3.  (The f16x2 <- e2m1x2
-// conversion is exact only when its byte operand arrives zero-extended in a 32-bit register;
-// bytes unpacked from a word by a vector move gave wrong values, so it is not used here.)
+// Two E2M1 codes (one byte, zero-extended in a 32-bit register) -> two exact halves, the low
+// nibble into the low half; a negative zero code gives -0.  The byte is narrowed inside the asm
+// block, so the conversion sees exactly the byte (fed with bytes unpacked from a word by a
+// vector move it returned wrong values).
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.u8.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(r)
+      : "r"(byte));
+  return r;
+}
+
+// Eight E2M1 codes (nibble i = element i) -> their values, exact (halves widen exactly).
 __device__ __forceinline__ void e2m1_decode8(uint32_t codes, float out[8]) {
-  const uint32_t idx = codes & 0x77777777u;
-  const uint32_t hi_a = __byte_perm(0x3F3F3F00u, 0x40404040u, idx & 0xFFFFu);
-  const uint32_t hi_b = __byte_perm(0x3F3F3F00u, 0x40404040u, idx >> 16);
-  const uint32_t lo_a = __byte_perm(0xC0800000u, 0xC0804000u, idx & 0xFFFFu);
-  const uint32_t lo_b = __byte_perm(0xC0800000u, 0xC0804000u, idx >> 16);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    // bytes 2, 3 of the result = low, high byte of element i's bf16 value
-    const uint32_t sel = ((uint32_t)i << 8) | ((uint32_t)(4 + i) << 12);
-    const uint32_t va = __byte_perm(lo_a, hi_a, sel) & 0xFFFF0000u;
-    const uint32_t vb = __byte_perm(lo_b, hi_b, sel) & 0xFFFF0000u;
-    out[i] = __uint_as_float(va | ((codes << (28 - 4 * i)) & 0x80000000u));
-    out[4 + i] = __uint_as_float(vb | ((codes << (12 - 4 * i)) & 0x80000000u));
+    const uint32_t h = e2m1x2_to_f16x2((codes >> (8 * i)) & 0xFFu);
+    const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&h));
+    out[2 * i] = f.x;
+    out[2 * i + 1] = f.y;
   }
 }
 

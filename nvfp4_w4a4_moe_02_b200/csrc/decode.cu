@@ -13,8 +13,12 @@
 // accumulates into the same tensor-memory accumulator as the main K loop.
 //
 // Roles: warp 0 TMA producer; warp 1 TMEM allocation + MMA issue; warps 2..5 epilogue, one per
-// TMEM lane quadrant (32 weight rows each).  A unit's accumulator is 128 lanes x 16 columns
-// (weight rows x tokens); four accumulator buffers let the epilogue trail the MMAs.
+// TMEM lane quadrant (32 weight rows each); warps 6..9 scale warps, one per quadrant, which store
+// each k-tile's scale atoms (shared -> registers -> tensor memory, tcgen05.st, the four-way
+// replicated layout) into a two-slot ring, so the tensor pipe runs only the MMAs (a scale copy on
+// the tensor pipe costs about as much as an N = 16 MMA, and each MMA needs two).  A unit's
+// accumulator is 128 lanes x 16 columns (weight rows x tokens); four accumulator buffers let the
+// epilogue trail the MMAs.
 #include "common.cuh"
 #include "kernels.h"
 #include "tc_ptx.cuh"
@@ -32,10 +36,11 @@ constexpr int B_BYTES = BT * KT_BYTES;  // 2 KB
 constexpr int SFA_BYTES = 4 * 512;
 constexpr int SFB_BYTES = 4 * 512;
 constexpr int ACC_BUFS = 4;
-constexpr int SF_SLOT = 8;              // A: 4 columns, B: 4 columns
+constexpr int SF_KT = 32;               // a stored k-tile: A scales of its 4 blocks, then B's (4 + 4 columns each)
 constexpr int SF_BASE = ACC_BUFS * BT;  // 64
 constexpr int TMEM_COLS = 128;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_THREADS = 320;
+constexpr int SF_WARP0 = 6;
 constexpr int XCH_BYTES = 64 * BT * 4;  // SwiGLU exchange: 64 up rows x 16 tokens, fp32
 constexpr int OFF_A = 0;
 constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -43,12 +48,12 @@ constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
 constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
 constexpr int OFF_XCH = OFF_SFB + STAGES * SFB_BYTES;  // two exchange buffers
 constexpr int OFF_BAR = OFF_XCH + 2 * XCH_BYTES;
-// full[STAGES] empty[STAGES] accf[ACC_BUFS] acce[ACC_BUFS] drain xfull[2] xempty[2]
-constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1 + 4;
+// full[STAGES] empty[STAGES] accf[ACC_BUFS] acce[ACC_BUFS] drain xfull[2] xempty[2] sf_full[2]
+constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1 + 4 + 2;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM = OFF_MISC + 32;
 static_assert(SMEM <= 232448, "shared memory budget");
-static_assert(SF_BASE + 2 * SF_SLOT <= TMEM_COLS, "tensor memory budget");
+static_assert(SF_BASE + 2 * SF_KT <= TMEM_COLS, "tensor memory budget");
 static_assert(OFF_B % 1024 == 0 && B_BYTES % 1024 == 0, "swizzled tiles need 1024-byte alignment");
 }  // namespace dec
 
@@ -91,6 +96,7 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
   const uint32_t bar_drain = sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS);
   auto bar_xfull = [&](int b) { return sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS + 1 + b); };
   auto bar_xempty = [&](int b) { return sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS + 3 + b); };
+  auto bar_sff = [&](int b) { return sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS + 5 + b); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
   volatile int* prod_issued = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
@@ -109,6 +115,7 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_xfull(b), 2);
       mbar_init(bar_xempty(b), 2);
+      mbar_init(bar_sff(b), 4);
     }
     *abort_flag = 0;
     *prod_issued = 0;
@@ -202,6 +209,7 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
       uint32_t mma_count = 0;
       bool ok = true;
       int64_t uidx = 0;  // units processed by this CTA (skipped slots not counted)
+      uint32_t g = 0;    // k-tiles taken (the scale ring's sequence)
       for (int64_t u = blockIdx.x; u < total_units && !*abort_flag; u += gridDim.x) {
         const int slot = (int)(u / args.m_tiles);
         const int eu = unit_expert(slot);
@@ -216,7 +224,8 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(buf * BT);
         for (int kt = 0; kt < kt_total; ++kt) {
-          if (!mbar_wait(bar_full(stage), phase, limit, abort_flag)) {
+          if (!mbar_wait(bar_full(stage), phase, limit, abort_flag) ||
+              !mbar_wait(bar_sff(g & 1), (g >> 1) & 1u, limit, abort_flag)) {
             ok = false;
             break;
           }
@@ -229,19 +238,13 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
           const int nk64 = min(4, k64 - kk * 4);
           const uint32_t a_s = sbase + OFF_A + stage * A_BYTES;
           const uint32_t b_s = sbase + OFF_B + stage * B_BYTES;
-          const uint32_t sfa_s = sbase + OFF_SFA + stage * SFA_BYTES;
-          const uint32_t sfb_s = sbase + OFF_SFB + stage * SFB_BYTES;
-          for (int j = 0; j < nk64; ++j, ++mma_count) {
-            // alternate between two scale slots so a copy never overwrites scales that the
-            // previous (still running) MMA reads
-            const uint32_t sfa_t = tmem_base + (uint32_t)(SF_BASE + (mma_count & 1) * SF_SLOT);
-            const uint32_t sfb_t = sfa_t + 4;
-            tc_copy_sf(sfa_t, desc_sf(sfa_s + j * 512));
-            tc_copy_sf(sfb_t, desc_sf(sfb_s + j * 512));
-            tc_mma_fp4(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, sfa_t, sfb_t,
-                       (kt | j) != 0 ? 1u : 0u);
-          }
+          // scales of block j: A at +4j, B at +16 + 4j of slot g & 1 (stored by the scale warps)
+          const uint32_t sf_t = tmem_base + (uint32_t)(SF_BASE + (int)(g & 1) * SF_KT);
+          for (int j = 0; j < nk64; ++j, ++mma_count)
+            tc_mma_fp4(d_tmem, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, sf_t + 4 * j,
+                       sf_t + 16 + 4 * j, (kt | j) != 0 ? 1u : 0u);
           tc_commit(bar_empty(stage));
+          ++g;
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -254,6 +257,58 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
       if (!ok) {
         report_status(args.status, kErrTimeout);
         *abort_flag = 1;
+      }
+    }
+  } else if (warp >= SF_WARP0) {
+    // ===================================================================== scale warps
+    // Warp w stores lanes [32 (w % 4), +32): lane j takes the 16 bytes at 16 j of each 512-byte
+    // atom into 4 columns.  Per k-tile g: its stage has landed, slot g & 1 is free (the commit that
+    // empties the stage of k-tile g - 2 has arrived, so its MMAs are complete), then the 4 A and
+    // 4 B atoms -> 32 columns, wait for the stores, arrive on sf_full.
+    const int quad = warp & 3;
+    const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
+    uint32_t g = 0;
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    for (int64_t u = blockIdx.x; u < total_units && ok && !*abort_flag; u += gridDim.x) {
+      const int e = unit_expert((int)(u / args.m_tiles));
+      if (e == kSkip) continue;
+      if (e == kBad) break;
+      for (int kt = 0; kt < kt_total; ++kt) {
+        bool w_ok = mbar_wait(bar_full(stage), phase, limit, abort_flag);
+        if (w_ok && g >= 2) {
+          const uint32_t gp = g - 2;
+          w_ok = mbar_wait(bar_empty((int)(gp % STAGES)), (gp / STAGES) & 1u, limit, abort_flag);
+        }
+        if (!__all_sync(0xffffffffu, w_ok)) {
+          if (lane == 0) {
+            if (!*abort_flag) report_status(args.status, kErrTimeout);
+            *abort_flag = 1;
+          }
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sl = t_lane + (uint32_t)(SF_BASE + (int)(g & 1) * SF_KT);
+        const uint32_t sfa_s = sbase + OFF_SFA + stage * SFA_BYTES + lane * 16;
+        const uint32_t sfb_s = sbase + OFF_SFB + stage * SFB_BYTES + lane * 16;
+        uint32_t r[16];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ld_shared_v4(sfa_s + j * 512, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        tmem_st16(sl, r);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) ld_shared_v4(sfb_s + j * 512, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+        tmem_st16(sl + 16, r);
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_sff((int)(g & 1)));
+        ++g;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
       }
     }
   } else {

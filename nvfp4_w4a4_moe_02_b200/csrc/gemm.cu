@@ -8,14 +8,21 @@
 // columns of the residual and of the gathered weight columns) that accumulates into the
 // same tensor-memory accumulator as the main loop, so one epilogue applies the scale.
 //
-// Structure (one CTA per SM, persistent over output tiles of 128 x BN):
+// Structure (one CTA per SM, persistent over output tiles of 128 x BN; four warpgroups whose
+// register shares are moved with setmaxnreg: 128 x (56 + 72) + 256 x 192 = 65536 registers):
 //   warp 0      TMA producer: A/B code tiles (128-byte swizzle) by tensor-map copies, the
 //               scale atoms (512 B each) by bulk copies, into a STAGES-deep shared ring.
-//   warp 1      tensor-memory allocation and the single MMA-issuing thread: scale atoms
-//               shared -> tensor memory (tcgen05.cp 32x128b.warpx4), then
+//   warp 1      tensor-memory allocation and the single MMA-issuing thread:
 //               tcgen05.mma.kind::mxf4nvf4.block_scale (K = 64 per instruction); commits
 //               free the shared stage and, at the end of a tile, publish the accumulator.
-//   warps 2..9  epilogue: tcgen05.ld of the FP32 accumulator (two warps per lane quadrant,
+//   warps 4..7  scale warps (one per tensor-memory lane quadrant): each k-tile's scale atoms,
+//               shared -> registers -> tensor memory (tcgen05.st, the four-way replicated
+//               layout the MMA reads), into a two-slot ring.  Measured: a 512-byte atom copy
+//               on the tensor pipe (tcgen05.cp 32x128b.warpx4) costs about 55 cycles there,
+//               serialised with the MMAs (three per K = 64 MMA at BN = 256, about as much
+//               time as the MMA itself); stores by warps run beside the MMAs.  The FP8 and
+//               own-scale modes keep the copies on the tensor pipe.
+//   warps 8..15 epilogue: tcgen05.ld of the FP32 accumulator (two warps per lane quadrant,
 //               one column half each) into registers, release, then scale by alpha and
 //               store bf16/FP32 rows (or SwiGLU + amax) while the next tile's MMAs run.
 // Every mbarrier wait is bounded by a wall-clock limit; on expiry the kernel records
@@ -29,7 +36,12 @@ namespace tc {
 
 constexpr int BM = 128;
 constexpr int KT_BYTES = 128;  // bytes of one row per k-tile: 256 FP4 elements
-constexpr int NUM_THREADS = 320;  // producer warp, MMA warp, 8 epilogue warps
+constexpr int NUM_THREADS = 512;  // producer, MMA, 2 idle | 4 scale warps | 8 epilogue warps
+constexpr int EPI_WARP0 = 8;      // first epilogue warp
+constexpr int SF_WARP0 = 4;       // first scale warp
+// per-thread registers after the split (warpgroups 0, 1, 2-3): 128 x (56 + 72) + 256 x 192
+constexpr int REG_CTRL = 56, REG_SF = 72, REG_EPI = 192;
+static_assert(128 * (REG_CTRL + REG_SF) + 256 * REG_EPI <= 65536, "register split over the launch's total");
 
 // Weight slab of grouped segment `seg`: the segment itself, or seg_expert[seg] (segments of
 // several sources that share an expert, as an expert-parallel rank receives them).  An index
@@ -48,7 +60,9 @@ __device__ __forceinline__ int segment_weight(const GemmArgs& args, int seg) {
 // and the residual products go to two accumulators (columns [0, BN) and [BN, 2 BN) of a buffer)
 // and the epilogue adds them with their own scales; only BN = 128 (the two halves then take the
 // tensor memory of one BN = 256 accumulator).
-template <int BN, bool OWN = false>
+// SFST: the scale warps store each k-tile's scale factors into a two-slot ring of tensor memory
+// (FP4 without the own-scale mode); otherwise the MMA thread copies them per MMA (two slots).
+template <int BN, bool OWN = false, bool SFST = false>
 struct Cfg {
   static constexpr int ACC_W = OWN ? 2 * BN : BN;  // accumulator columns per tile
   static constexpr int STAGES = (BN == 256) ? 3 : 5;
@@ -65,13 +79,19 @@ struct Cfg {
   // exceed the 512 columns, the buffers overlap: buffer 1 starts ACC_OVERLAP columns before
   // buffer 0 ends, and the epilogue drains that strip first and releases it early.
   static constexpr int SF_SLOT = 4 + 4 * (BN / 128);
-  static constexpr int SF_COLS = 2 * SF_SLOT;
+  // a stored k-tile: the A scales of its four K = 64 blocks (4 columns each), then their B scales
+  // (4 columns per 128 rows of B each)
+  static constexpr int SF_KT = 4 * 4 + 4 * 4 * (BN / 128);
+  static constexpr int SF_COLS = SFST ? 2 * SF_KT : 2 * SF_SLOT;
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_OVERLAP = (2 * ACC_W + SF_COLS > TMEM_COLS) ? (2 * ACC_W + SF_COLS - TMEM_COLS) : 0;
   static constexpr int ACC1_BASE = ACC_W - ACC_OVERLAP;
   static constexpr int SF_BASE = ACC1_BASE + ACC_W;
   static_assert(SF_BASE + SF_COLS <= TMEM_COLS, "tensor memory budget");
-  static_assert(ACC_OVERLAP <= 32, "the shared strip must lie in one 32-column chunk");
+  static_assert(ACC_OVERLAP % 32 == 0 || ACC_OVERLAP < 32, "the shared strip is whole 32-column chunks");
+  static_assert(ACC_OVERLAP <= 96, "at most three chunks of a half are shared");
+  // chunks of a half (of BN / 2 columns) in the strip shared by the two buffers
+  static constexpr int OVL_CHUNKS = (ACC_OVERLAP + 31) / 32;
   static_assert(!OWN || BN == 128, "two accumulators only at BN = 128");
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
@@ -79,8 +99,8 @@ struct Cfg {
   static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
   static constexpr int OFF_STG = OFF_SFB + STAGES * SFB_BYTES;  // 1024-aligned
   static constexpr int OFF_BAR = OFF_STG + 8 * STG * BOX_BYTES;
-  // full[S], empty[S], accf[2], acce[2], ovf[2], drain
-  static constexpr int NUM_BARS = 2 * STAGES + 7;
+  // full[S], empty[S], accf[2], acce[2], ovf[2], drain, sf_full[2]
+  static constexpr int NUM_BARS = 2 * STAGES + 9;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // the dynamic shared window starts 1024-byte aligned (checked in the kernel)
   static constexpr int SMEM = OFF_MISC + 32;
@@ -96,7 +116,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     w4a4_rac_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_ar,
                          const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_ws,
                          const __grid_constant__ CUtensorMap tm_y, const GemmArgs args) {
-  using C = Cfg<BN, OWN>;
+  constexpr bool SFST = !FP8 && !OWN;  // scale factors stored by the scale warps
+  using C = Cfg<BN, OWN, SFST>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t sbase = smem_u32(smem_raw);
   unsigned char* smem = smem_raw;
@@ -113,6 +134,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto bar_acce = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 2 + a); };  // fully drained
   auto bar_ovf = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 4 + a); };   // shared strip drained
   const uint32_t bar_drain = sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 6);
+  auto bar_sff = [&](int i) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 7 + i); };  // scale slot stored
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* prod_issued = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
@@ -129,6 +151,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       mbar_init(bar_ovf(a), 4);
     }
     mbar_init(bar_drain, 1);
+    mbar_init(bar_sff(0), 4);
+    mbar_init(bar_sff(1), 4);
     *abort_flag = 0;
     *prod_issued = 0;
     *mma_taken = 0;
@@ -166,6 +190,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   const int kt_total = args.kt_main + args.kt_res;
   const uint64_t limit = args.wait_limit_ns;
 
+  // Roles by warpgroup; each first moves its register share (every warp of a warpgroup executes
+  // the same setmaxnreg), so the code of each role is compiled within that share.
+  if (warp < SF_WARP0) {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_CTRL));
   if (warp == 0) {
     // ===================================================================== TMA producer
     if (lane == 0) {
@@ -224,6 +252,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       uint32_t mma_count = 0;
       bool ok = true;
       int64_t tile_idx = 0;
+      uint32_t g = 0;  // k-tiles taken so far (the scale ring's sequence)
       for (int64_t t = blockIdx.x; t < total_tiles && ok && !*abort_flag; t += gridDim.x, ++tile_idx) {
         const int acc = (int)(tile_idx & 1);
         const int64_t use = tile_idx >> 1;  // how many times buffer `acc` was used before
@@ -242,6 +271,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc ? C::ACC1_BASE : 0);
         for (int kt = 0; kt < kt_total; ++kt) {
           if (!mbar_wait(bar_full(stage), phase, limit, abort_flag)) {
+            ok = false;
+            break;
+          }
+          // the scale warps stored this k-tile's scales into slot g & 1
+          if (SFST && !mbar_wait(bar_sff(g & 1), (g >> 1) & 1u, limit, abort_flag)) {
             ok = false;
             break;
           }
@@ -276,7 +310,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // fresh at the first of them
           const uint32_t d_k = d_tmem + ((OWN && res) ? (uint32_t)BN : 0u);
           const int kt_first = (OWN && res) ? args.kt_main : 0;
-          for (int j = 0; j < (FP8 ? 0 : nk64); ++j, ++mma_count) {
+          if constexpr (SFST) {
+            // scales already in tensor memory: A of block j at +4j, B at +16 + 4 (BN / 128) j
+            const uint32_t slot = tmem_base + (uint32_t)(C::SF_BASE + (int)(g & 1) * C::SF_KT);
+            for (int j = 0; j < nk64; ++j)
+              tc_mma_fp4(d_k, desc_sw128(a_s + 32 * j), desc_sw128(b_s + 32 * j), idesc, slot + 4 * j,
+                         slot + 16 + 4 * (BN / 128) * j, (kt != kt_first || j != 0) ? 1u : 0u);
+          }
+          for (int j = 0; j < ((FP8 || SFST) ? 0 : nk64); ++j, ++mma_count) {
             const uint32_t sfa_t = tmem_base + (uint32_t)(C::SF_BASE + (mma_count & 1) * C::SF_SLOT);
             const uint32_t sfb_t = sfa_t + 4;
             tc_copy_sf(sfa_t, desc_sf(sfa_s + j * 512));
@@ -286,6 +327,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
                        (kt != kt_first || j != 0) ? 1u : 0u);
           }
           tc_commit(bar_empty(stage));
+          ++g;
           if (++stage == C::STAGES) {
             stage = 0;
             phase ^= 1u;
@@ -299,14 +341,77 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         *abort_flag = 1;
       }
     }
+  }
+  } else if (warp < EPI_WARP0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(REG_SF));
+    // ===================================================================== scale warps
+    // Warp w stores into lanes [32 (w % 4), +32): lane j takes 16 bytes at 16 j of each 512-byte
+    // atom (the scales of rows j, 32 + j, 64 + j, 96 + j) into 4 columns, as the replicating
+    // copy would.  Per k-tile g: its stage has landed (full), slot g & 1 is free (the MMAs of
+    // k-tile g - 2 are complete: the commit that empties their stage), then 12 atoms -> 48
+    // (BN = 256) or 8 atoms -> 32 columns, wait for the stores, arrive on sf_full.
+    if constexpr (SFST) {
+      const int quad = warp & 3;
+      const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
+      uint32_t g = 0;
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        for (int kt = 0; kt < kt_total; ++kt) {
+          bool w_ok = mbar_wait(bar_full(stage), phase, limit, abort_flag);
+          if (w_ok && g >= 2) {
+            const uint32_t gp = g - 2;
+            w_ok = mbar_wait(bar_empty((int)(gp % C::STAGES)), (gp / C::STAGES) & 1u, limit, abort_flag);
+          }
+          if (!__all_sync(0xffffffffu, w_ok)) {
+            if (lane == 0) {
+              if (!*abort_flag) report_status(args.status, kErrTimeout);
+              *abort_flag = 1;
+            }
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t slot = t_lane + (uint32_t)(C::SF_BASE + (int)(g & 1) * C::SF_KT);
+          const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_BYTES + lane * 16;
+          const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_BYTES + lane * 16;
+          uint32_t r[16];
+          // A scales of the four K = 64 blocks -> columns 0..15
+#pragma unroll
+          for (int j = 0; j < 4; ++j) ld_shared_v4(sfa_s + j * 512, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+          tmem_st16(slot, r);
+          // B scales: block j, 128-row group rb at column 16 + 4 (BN / 128) j + 4 rb
+#pragma unroll
+          for (int h = 0; h < BN / 128; ++h) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int jb = (h * 4 + q) / (BN / 128), rb = (h * 4 + q) % (BN / 128);
+              ld_shared_v4(sfb_s + rb * 2048 + jb * 512, r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
+            }
+            tmem_st16(slot + 16 + 16 * h, r);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar_sff((int)(g & 1)));
+          ++g;
+          if (++stage == C::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(REG_EPI));
     // ===================================================================== epilogue
     // Eight warps: two per tensor-memory lane quadrant, each owning half of the tile's
     // columns.  A warp drains its columns into registers, releases the accumulator, and only
     // then converts and stores, so the math overlaps the next tile's MMAs.
     constexpr int NCH = C::ACC_W / 64;      // 32-column chunks per warp
     const int quad = warp & 3;              // tensor-memory lanes [32*quad, 32*quad + 32)
-    const int half = (warp - 2) >> 2;       // which half of the tile's columns
+    const int half = (warp - EPI_WARP0) >> 2;  // which half of the tile's columns
     float amax = 0.0f;
     int64_t tile_idx = 0;
     for (int64_t t = blockIdx.x; t < total_tiles; t += gridDim.x, ++tile_idx) {
@@ -358,17 +463,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int f = half * (BN / 4) + 32 * ii;
         return (f / 64) * 128 + (f % 64) + (i >= NCH / 2 ? 64 : 0);
       };
-      // the chunk holding the strip shared with the other buffer is drained and released first
-      int ovl_i = -1;
-      if (C::ACC_OVERLAP > 0) {
-        if (acc == 0 && half == 1) ovl_i = NCH - 1;  // buffer 0: its last columns
-        if (acc == 1 && half == 0) ovl_i = 0;        // buffer 1: its first columns
-      }
+      // the chunks holding the strip shared with the other buffer are drained and released first:
+      // buffer 0's last columns (the last OVL_CHUNKS chunks of half 1), buffer 1's first ones
+      // (the first OVL_CHUNKS chunks of half 0)
+      auto in_strip = [&](int i) -> bool {
+        if (C::ACC_OVERLAP == 0) return false;
+        if (acc == 0) return half == 1 && i >= NCH - C::OVL_CHUNKS;
+        return half == 0 && i < C::OVL_CHUNKS;
+      };
+      const bool holds_strip = C::ACC_OVERLAP > 0 && ((acc == 0 && half == 1) || (acc == 1 && half == 0));
       uint32_t v[NCH][32];
-      if (ovl_i >= 0) {
+      if (holds_strip) {
 #pragma unroll
         for (int i = 0; i < NCH; ++i)
-          if (i == ovl_i) tmem_ld32(t_row + chunk_col(i), v[i]);
+          if (in_strip(i)) tmem_ld32(t_row + chunk_col(i), v[i]);
         tmem_wait_ld();
         tc_fence_before();
         __syncwarp();
@@ -376,7 +484,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       }
 #pragma unroll
       for (int i = 0; i < NCH; ++i)
-        if (i != ovl_i) tmem_ld32(t_row + chunk_col(i), v[i]);
+        if (!in_strip(i)) tmem_ld32(t_row + chunk_col(i), v[i]);
       tmem_wait_ld();
       tc_fence_before();
       __syncwarp();
@@ -396,7 +504,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const float alpha_out = OWN ? 1.0f : alpha;
       // ---- output through shared memory: each box is 32 rows x 128 bytes in the 128-byte
       // swizzled layout (16-byte chunk c of row r at chunk c ^ (r % 8)), stored by one TMA copy
-      const uint32_t stg = sbase + C::OFF_STG + (uint32_t)((warp - 2) * C::STG * C::BOX_BYTES);
+      const uint32_t stg = sbase + C::OFF_STG + (uint32_t)((warp - EPI_WARP0) * C::STG * C::BOX_BYTES);
       const int32_t y0 = (int32_t)(mb * BM + quad * 32);
       const bool box_live = (int64_t)y0 < rows_e;
       auto put_box = [&](int slot, const uint32_t (&w)[32], int32_t x) {
@@ -556,16 +664,25 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, int32_t* status) {
 
 }  // namespace tc
 
-size_t gemm_smem_bytes(int bn) { return bn == 256 ? (size_t)tc::Cfg<256>::SMEM : (size_t)tc::Cfg<128>::SMEM; }
+size_t gemm_smem_bytes(int bn) {
+  return bn == 256 ? (size_t)tc::Cfg<256, false, true>::SMEM : (size_t)tc::Cfg<128, false, true>::SMEM;
+}
 
 template <int BN, bool FP8, bool OWN = false>
 static cudaError_t launch_gemm_t(const CUtensorMap& tm_a, const CUtensorMap& tm_ar, const CUtensorMap& tm_w,
                                  const CUtensorMap& tm_ws, const CUtensorMap& tm_y, const GemmArgs& args, int grid,
                                  cudaStream_t st) {
-  constexpr int smem = tc::Cfg<BN, OWN>::SMEM;
+  constexpr int smem = tc::Cfg<BN, OWN, !FP8 && !OWN>::SMEM;
   cudaError_t e =
       cudaFuncSetAttribute(tc::w4a4_rac_gemm_kernel<BN, FP8, OWN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
+  // the warpgroups' setmaxnreg shares are drawn from the registers the CTA is launched with: a
+  // build whose launch count falls short would leave setmaxnreg.inc waiting, so it is refused
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, tc::w4a4_rac_gemm_kernel<BN, FP8, OWN>);
+  if (e != cudaSuccess) return e;
+  if ((int64_t)fa.numRegs * tc::NUM_THREADS < 128ll * (tc::REG_CTRL + tc::REG_SF) + 256ll * tc::REG_EPI)
+    return cudaErrorInvalidConfiguration;
   tc::w4a4_rac_gemm_kernel<BN, FP8, OWN><<<grid, tc::NUM_THREADS, smem, st>>>(tm_a, tm_ar, tm_w, tm_ws, tm_y, args);
   return cudaGetLastError();
 }
