@@ -49,7 +49,8 @@ constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
 constexpr int OFF_XCH = OFF_SFB + STAGES * SFB_BYTES;  // two exchange buffers
 constexpr int OFF_BAR = OFF_XCH + 2 * XCH_BYTES;
 // full[STAGES] empty[STAGES] accf[ACC_BUFS] acce[ACC_BUFS] drain xfull[2] xempty[2] sf_full[2]
-constexpr int NUM_BARS = 2 * STAGES + 2 * ACC_BUFS + 1 + 4 + 2;
+// sf_landed[STAGES]
+constexpr int NUM_BARS = 3 * STAGES + 2 * ACC_BUFS + 1 + 4 + 2;
 constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int SMEM = OFF_MISC + 32;
 static_assert(SMEM <= 232448, "shared memory budget");
@@ -97,6 +98,8 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
   auto bar_xfull = [&](int b) { return sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS + 1 + b); };
   auto bar_xempty = [&](int b) { return sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS + 3 + b); };
   auto bar_sff = [&](int b) { return sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS + 5 + b); };
+  // a stage's scale atoms landed (apart from its operands, so the scale warps can start first)
+  auto bar_sfl = [&](int s) { return sbase + OFF_BAR + 8u * (2 * STAGES + 2 * ACC_BUFS + 7 + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + OFF_MISC + 4);
   volatile int* prod_issued = reinterpret_cast<volatile int*>(smem + OFF_MISC + 8);
@@ -106,6 +109,7 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full(s), 1);
       mbar_init(bar_empty(s), 1);
+      mbar_init(bar_sfl(s), 1);
     }
     for (int a = 0; a < ACC_BUFS; ++a) {
       mbar_init(bar_accf(a), 1);
@@ -172,7 +176,8 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
           const int k64 = res ? args.k64_res : args.k64_main;
           const int nk64 = min(4, k64 - kk * 4);
           const uint32_t sf_bytes = (uint32_t)nk64 * 512u;
-          mbar_expect_tx(bar_full(stage), (uint32_t)(A_BYTES + B_BYTES) + 2u * sf_bytes);
+          mbar_expect_tx(bar_sfl(stage), 2u * sf_bytes);
+          mbar_expect_tx(bar_full(stage), (uint32_t)(A_BYTES + B_BYTES));
           tma_load_3d(sbase + OFF_A + stage * A_BYTES, res ? &tm_ws : &tm_w, kk * KT_BYTES, mt * BM, e,
                       bar_full(stage));
           tma_load_2d(sbase + OFF_B + stage * B_BYTES, res ? &tm_xr : &tm_x, kk * KT_BYTES, slot * BT,
@@ -180,11 +185,11 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
           const uint8_t* sfw = res ? args.sfw_sel + (int64_t)e * args.sfw_sel_slab_bytes
                                    : args.sfw + (int64_t)e * args.sfw_slab_bytes;
           bulk_load(sbase + OFF_SFA + stage * SFA_BYTES, sfw + ((int64_t)mt * k64 + kk * 4) * 512, sf_bytes,
-                    bar_full(stage));
+                    bar_sfl(stage));
           // slab layout: slab `slot` owns one scale atom per 64 columns
           const uint8_t* sfx = res ? args.sfx_res : args.sfx;
           bulk_load(sbase + OFF_SFB + stage * SFB_BYTES, sfx + ((int64_t)slot * k64 + kk * 4) * 512, sf_bytes,
-                    bar_full(stage));
+                    bar_sfl(stage));
           ++issued;
           *prod_issued = issued;
           if (++stage == STAGES) {
@@ -276,7 +281,7 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
       if (e == kSkip) continue;
       if (e == kBad) break;
       for (int kt = 0; kt < kt_total; ++kt) {
-        bool w_ok = mbar_wait(bar_full(stage), phase, limit, abort_flag);
+        bool w_ok = mbar_wait(bar_sfl(stage), phase, limit, abort_flag);
         if (w_ok && g >= 2) {
           const uint32_t gp = g - 2;
           w_ok = mbar_wait(bar_empty((int)(gp % STAGES)), (gp / STAGES) & 1u, limit, abort_flag);
@@ -413,8 +418,10 @@ __global__ void __launch_bounds__(dec::NUM_THREADS, 1)
     }
     if (warp == 0 && lane == 0) {
       // tensor copies still in flight land before the shared memory is released
-      for (int i = *mma_taken; i < *prod_issued; ++i)
+      for (int i = *mma_taken; i < *prod_issued; ++i) {
         mbar_wait(bar_full(i % STAGES), (uint32_t)((i / STAGES) & 1), limit, nullptr);
+        mbar_wait(bar_sfl(i % STAGES), (uint32_t)((i / STAGES) & 1), limit, nullptr);
+      }
     }
     __syncthreads();
   }

@@ -66,8 +66,13 @@ template <int BN, bool OWN = false, bool SFST = false>
 struct Cfg {
   static constexpr int ACC_W = OWN ? 2 * BN : BN;  // accumulator columns per tile
   static constexpr int STAGES = (BN == 256) ? 3 : 5;
-  // epilogue staging: per epilogue warp, STG boxes of 32 rows x 128 bytes for TMA stores
-  static constexpr int STG = (BN == 256) ? 2 : 1;
+  // scale atoms: in scale-warp mode a ring of their own, SFR k-tiles deep (filled by a second
+  // producer thread ahead of the operand ring, so the scale warps finish before the operands
+  // land); otherwise part of each operand stage
+  static constexpr int SFR = SFST ? 6 : STAGES;
+  // epilogue staging: per epilogue warp, STG boxes of 32 rows x 128 bytes for TMA stores (one in
+  // scale-warp mode, whose scale ring takes the shared memory of the second)
+  static constexpr int STG = SFST ? 1 : (BN == 256) ? 2 : 1;
   static constexpr int BOX_BYTES = 32 * 128;
   static constexpr int A_BYTES = BM * KT_BYTES;
   static constexpr int B_BYTES = BN * KT_BYTES;
@@ -96,11 +101,11 @@ struct Cfg {
   static constexpr int OFF_A = 0;
   static constexpr int OFF_B = OFF_A + STAGES * A_BYTES;
   static constexpr int OFF_SFA = OFF_B + STAGES * B_BYTES;
-  static constexpr int OFF_SFB = OFF_SFA + STAGES * SFA_BYTES;
-  static constexpr int OFF_STG = OFF_SFB + STAGES * SFB_BYTES;  // 1024-aligned
+  static constexpr int OFF_SFB = OFF_SFA + SFR * SFA_BYTES;
+  static constexpr int OFF_STG = OFF_SFB + SFR * SFB_BYTES;  // 1024-aligned
   static constexpr int OFF_BAR = OFF_STG + 8 * STG * BOX_BYTES;
-  // full[S], empty[S], accf[2], acce[2], ovf[2], drain, sf_full[2]
-  static constexpr int NUM_BARS = 2 * STAGES + 9;
+  // full[S], empty[S], accf[2], acce[2], ovf[2], drain, sf_full[2], sf_landed[SFR], sf_free[SFR]
+  static constexpr int NUM_BARS = 2 * STAGES + 9 + 2 * SFR;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   // the dynamic shared window starts 1024-byte aligned (checked in the kernel)
   static constexpr int SMEM = OFF_MISC + 32;
@@ -135,10 +140,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto bar_ovf = [&](int a) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 4 + a); };   // shared strip drained
   const uint32_t bar_drain = sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 6);
   auto bar_sff = [&](int i) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 7 + i); };  // scale slot stored
+  // scale-warp mode: a slot of the scale ring landed / was read by the four scale warps
+  auto bar_sfl = [&](int s) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 9 + s); };
+  auto bar_sfe = [&](int s) { return sbase + C::OFF_BAR + 8u * (2 * C::STAGES + 9 + C::SFR + s); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
   volatile int* prod_issued = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 8);
   volatile int* mma_taken = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 12);
+  volatile int* sf_issued = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 16);  // scale ring
+  volatile int* sf_seen = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 20);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::STAGES; ++s) {
@@ -153,9 +163,15 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     mbar_init(bar_drain, 1);
     mbar_init(bar_sff(0), 4);
     mbar_init(bar_sff(1), 4);
+    for (int s = 0; s < C::SFR; ++s) {
+      mbar_init(bar_sfl(s), 1);
+      mbar_init(bar_sfe(s), 4);
+    }
     *abort_flag = 0;
     *prod_issued = 0;
     *mma_taken = 0;
+    *sf_issued = 0;
+    *sf_seen = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   }
@@ -219,24 +235,69 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const int64_t at_row = FP8 ? (int64_t)args.kt_main : (int64_t)k64;
           const int64_t at0 = FP8 ? (int64_t)kk : (int64_t)kk * 4;
           const uint32_t sf_bytes = (uint32_t)n_at * 512u;
-          mbar_expect_tx(bar_full(stage), (uint32_t)(C::A_BYTES + C::B_BYTES) + sf_bytes * (1u + BN / 128));
+          mbar_expect_tx(bar_full(stage),
+                         (uint32_t)(C::A_BYTES + C::B_BYTES) + (SFST ? 0u : sf_bytes * (1u + BN / 128)));
           tma_load_2d(sbase + C::OFF_A + stage * C::A_BYTES, res ? &tm_ar : &tm_a, kk * KT_BYTES, (int32_t)(mb * BM),
                       bar_full(stage));
           tma_load_3d(sbase + C::OFF_B + stage * C::B_BYTES, res ? &tm_ws : &tm_w, kk * KT_BYTES, nb * BN, e,
                       bar_full(stage));
-          const uint8_t* sfa = (res ? args.sfa_res : args.sfa) + (mb * at_row + at0) * 512;
-          bulk_load(sbase + C::OFF_SFA + stage * C::SFA_BYTES, sfa, sf_bytes, bar_full(stage));
-          const uint8_t* sfw = res ? args.sfw_sel + (int64_t)e * args.sfw_sel_slab_bytes
-                                   : args.sfw + (int64_t)e * args.sfw_slab_bytes;
+          if constexpr (!SFST) {
+            const uint8_t* sfa = (res ? args.sfa_res : args.sfa) + (mb * at_row + at0) * 512;
+            bulk_load(sbase + C::OFF_SFA + stage * C::SFA_BYTES, sfa, sf_bytes, bar_full(stage));
+            const uint8_t* sfw = res ? args.sfw_sel + (int64_t)e * args.sfw_sel_slab_bytes
+                                     : args.sfw + (int64_t)e * args.sfw_slab_bytes;
 #pragma unroll
-          for (int rb = 0; rb < BN / 128; ++rb) {
-            const uint8_t* src = sfw + ((int64_t)(nb * (BN / 128) + rb) * at_row + at0) * 512;
-            bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES + rb * 2048, src, sf_bytes, bar_full(stage));
+            for (int rb = 0; rb < BN / 128; ++rb) {
+              const uint8_t* src = sfw + ((int64_t)(nb * (BN / 128) + rb) * at_row + at0) * 512;
+              bulk_load(sbase + C::OFF_SFB + stage * C::SFB_BYTES + rb * 2048, src, sf_bytes, bar_full(stage));
+            }
           }
           ++issued;
           *prod_issued = issued;
           if (++stage == C::STAGES) {
             stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // ===================================================================== scale-ring producer
+    // Scale-warp mode: the scale atoms of k-tile g go to ring slot g % SFR once the four scale
+    // warps have read that slot's previous contents; the ring runs up to SFR k-tiles ahead.
+    if (SFST && lane == 0) {
+      int slot = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      for (int64_t t = blockIdx.x; t < total_tiles && !*abort_flag; t += gridDim.x) {
+        const int64_t mb = t / args.n_blocks;
+        const int nb = (int)(t - mb * args.n_blocks);
+        const int e = grouped ? segment_weight(args, find_expert(args.offsets, args.E, mb * BM)) : 0;
+        for (int kt = 0; kt < kt_total; ++kt) {
+          if (!mbar_wait(bar_sfe(slot), phase ^ 1u, limit, abort_flag)) {
+            report_status(args.status, kErrTimeout);
+            *abort_flag = 1;
+            break;
+          }
+          const bool res = kt >= args.kt_main;
+          const int kk = res ? kt - args.kt_main : kt;
+          const int k64 = res ? args.k64_res : args.k64_main;
+          const int n_at = min(4, k64 - kk * 4);
+          const uint32_t sf_bytes = (uint32_t)n_at * 512u;
+          mbar_expect_tx(bar_sfl(slot), sf_bytes * (1u + BN / 128));
+          const uint8_t* sfa = (res ? args.sfa_res : args.sfa) + (mb * (int64_t)k64 + kk * 4) * 512;
+          bulk_load(sbase + C::OFF_SFA + slot * C::SFA_BYTES, sfa, sf_bytes, bar_sfl(slot));
+          const uint8_t* sfw = res ? args.sfw_sel + (int64_t)e * args.sfw_sel_slab_bytes
+                                   : args.sfw + (int64_t)e * args.sfw_slab_bytes;
+#pragma unroll
+          for (int rb = 0; rb < BN / 128; ++rb) {
+            const uint8_t* src = sfw + ((int64_t)(nb * (BN / 128) + rb) * k64 + kk * 4) * 512;
+            bulk_load(sbase + C::OFF_SFB + slot * C::SFB_BYTES + rb * 2048, src, sf_bytes, bar_sfl(slot));
+          }
+          ++issued;
+          *sf_issued = issued;
+          if (++slot == C::SFR) {
+            slot = 0;
             phase ^= 1u;
           }
         }
@@ -354,12 +415,32 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int quad = warp & 3;
       const uint32_t t_lane = tmem_base + ((uint32_t)(quad * 32) << 16);
       uint32_t g = 0;
-      int stage = 0;
-      uint32_t phase = 0;
+      int rslot = 0;  // scale-ring slot of k-tile g, and its phase
+      uint32_t rphase = 0;
       bool ok = true;
       for (int64_t t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
         for (int kt = 0; kt < kt_total; ++kt) {
-          bool w_ok = mbar_wait(bar_full(stage), phase, limit, abort_flag);
+          // the atoms of k-tile g landed in ring slot rslot: read them into registers and release
+          // the slot before waiting for tensor memory, so only the stores follow that wait
+          bool w_ok = __all_sync(0xffffffffu, mbar_wait(bar_sfl(rslot), rphase, limit, abort_flag));
+          if (w_ok && warp == SF_WARP0 && lane == 0) *sf_seen = (int)g + 1;
+          uint32_t r[16 + 16 * (BN / 128)];
+          if (w_ok) {
+            const uint32_t sfa_s = sbase + C::OFF_SFA + rslot * C::SFA_BYTES + lane * 16;
+            const uint32_t sfb_s = sbase + C::OFF_SFB + rslot * C::SFB_BYTES + lane * 16;
+            // A scales of the four K = 64 blocks -> columns 0..15; B scales: block j, 128-row group
+            // rb -> column 16 + 4 (BN / 128) j + 4 rb
+#pragma unroll
+            for (int j = 0; j < 4; ++j) ld_shared_v4(sfa_s + j * 512, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
+#pragma unroll
+            for (int q = 0; q < 4 * (BN / 128); ++q) {
+              const int jb = q / (BN / 128), rb = q % (BN / 128);
+              ld_shared_v4(sfb_s + rb * 2048 + jb * 512, r[16 + 4 * q], r[17 + 4 * q], r[18 + 4 * q], r[19 + 4 * q]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_sfe(rslot));
+          }
+          // tensor-memory slot g & 1 is free once the MMAs of k-tile g - 2 are complete
           if (w_ok && g >= 2) {
             const uint32_t gp = g - 2;
             w_ok = mbar_wait(bar_empty((int)(gp % C::STAGES)), (gp / C::STAGES) & 1u, limit, abort_flag);
@@ -374,31 +455,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
           tc_fence_after();
           const uint32_t slot = t_lane + (uint32_t)(C::SF_BASE + (int)(g & 1) * C::SF_KT);
-          const uint32_t sfa_s = sbase + C::OFF_SFA + stage * C::SFA_BYTES + lane * 16;
-          const uint32_t sfb_s = sbase + C::OFF_SFB + stage * C::SFB_BYTES + lane * 16;
-          uint32_t r[16];
-          // A scales of the four K = 64 blocks -> columns 0..15
 #pragma unroll
-          for (int j = 0; j < 4; ++j) ld_shared_v4(sfa_s + j * 512, r[4 * j], r[4 * j + 1], r[4 * j + 2], r[4 * j + 3]);
-          tmem_st16(slot, r);
-          // B scales: block j, 128-row group rb at column 16 + 4 (BN / 128) j + 4 rb
+          for (int h = 0; h < 1 + BN / 128; ++h) {
+            uint32_t q16[16];
 #pragma unroll
-          for (int h = 0; h < BN / 128; ++h) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int jb = (h * 4 + q) / (BN / 128), rb = (h * 4 + q) % (BN / 128);
-              ld_shared_v4(sfb_s + rb * 2048 + jb * 512, r[4 * q], r[4 * q + 1], r[4 * q + 2], r[4 * q + 3]);
-            }
-            tmem_st16(slot + 16 + 16 * h, r);
+            for (int i = 0; i < 16; ++i) q16[i] = r[16 * h + i];
+            tmem_st16(slot + 16 * h, q16);
           }
           tmem_wait_st();
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar_sff((int)(g & 1)));
           ++g;
-          if (++stage == C::STAGES) {
-            stage = 0;
-            phase ^= 1u;
+          if (++rslot == C::SFR) {
+            rslot = 0;
+            rphase ^= 1u;
           }
         }
       }
@@ -640,6 +711,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // copies issued but never consumed by the MMA thread
       for (int i = *mma_taken; i < *prod_issued; ++i)
         mbar_wait(bar_full(i % C::STAGES), (uint32_t)((i / C::STAGES) & 1), limit, nullptr);
+    }
+    if (SFST && warp == 2 && lane == 0) {
+      // scale-ring copies issued but never seen landed by the scale warps
+      for (int i = *sf_seen; i < *sf_issued; ++i)
+        mbar_wait(bar_sfl(i % C::SFR), (uint32_t)((i / C::SFR) & 1), limit, nullptr);
     }
     __syncthreads();
   }

@@ -46,7 +46,7 @@ struct Plan {
   int meta_bytes;    // one stage: 4 x mc int64 offsets, R int32 valid flags, the slot count
   int off_rbuf;      // R x (K/16) x 17 floats (residual mode)
   int off_sel;       // Kp uint16 word offsets, transposed [16][Kp/16]
-  int off_seg;       // n_seg + 1 int32 tile prefix (segments mode)
+  int off_seg;       // segments mode: n_seg + 1 int32 tile prefix, then each segment's first row and rows
   int off_bar;       // full[S], empty[S]
   int off_misc;      // s_g, t6, n_tiles, abort
   int off_tab;       // float2 [128]: (d, 1/d) per E4M3 code
@@ -68,7 +68,7 @@ __host__ __device__ inline Plan make_plan(int K, int Kp, int fanout, int n_seg, 
   const int rbuf = Kp > 0 ? R * (K / 16) * kPitch * 4 : 0;
   p.off_sel = p.off_rbuf + round16(rbuf);
   p.off_seg = p.off_sel + round16(Kp * 2);
-  p.off_bar = p.off_seg + round16(n_seg > 0 ? (n_seg + 1) * 4 : 0);
+  p.off_bar = p.off_seg + round16(n_seg > 0 ? (3 * n_seg + 1) * 4 : 0);
   p.off_misc = p.off_bar + 2 * kStages * 8;
   p.off_tab = p.off_misc + 64;     // (d, 1/d) of the 128 E4M3 codes, for s_g and for the residual
   p.smem = p.off_tab + 2 * 128 * 8;
@@ -216,14 +216,26 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
   if (RES) {
     // channel list -> word offsets of the channels in the residual buffer's row, transposed so
     // that position j of residual block q sits at [j][q] (consecutive q for consecutive lanes)
-    for (int j = threadIdx.x; j < Kp; j += blockDim.x) {
-      int c = __ldg(a.sel + j);
-      const bool ok = c >= 0 && c < K && (j == 0 || __ldg(a.sel + j - 1) < c);
-      if (!ok) {
-        report_status(a.status, kErrInvalid);
-        c = 0;
+    // four entries per thread and round, their loads issued before any is used
+    for (int j0 = threadIdx.x; j0 < Kp; j0 += 4 * blockDim.x) {
+      int c[4], prev[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * blockDim.x;
+        c[u] = j < Kp ? __ldg(a.sel + j) : 0;
+        prev[u] = (j < Kp && j > 0) ? __ldg(a.sel + j - 1) : -1;
       }
-      sel_off[(j & 15) * QB + (j >> 4)] = (uint16_t)((c >> 4) * kPitch + (c & 15));
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = j0 + u * blockDim.x;
+        if (j >= Kp) break;
+        int cc = c[u];
+        if (!(cc >= 0 && cc < K && prev[u] < cc)) {
+          report_status(a.status, kErrInvalid);
+          cc = 0;
+        }
+        sel_off[(j & 15) * QB + (j >> 4)] = (uint16_t)((cc >> 4) * kPitch + (cc & 15));
+      }
     }
   }
   if (warp == 0) {
@@ -250,12 +262,21 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
     // number of tiles (segments: prefix over the segments' tiles)
     int64_t n_tiles;
     if (a.map == kMapSegments) {
+      // each segment's first row and row count, kept in shared memory for the producer's tiles
+      // (all of a lane's loads issued before any is used)
+      int32_t* seg_first_s = seg_prefix + a.n_seg + 1;
+      int32_t* seg_rows_s = seg_first_s + a.n_seg;
+      for (int e = lane; e < a.n_seg; e += 32) {
+        seg_first_s[e] = __ldg(a.seg_off + e);
+        seg_rows_s[e] = __ldg(a.seg_rows + e);
+      }
+      __syncwarp();
       int carry = 0;
       for (int base = 0; base < a.n_seg; base += 32) {
         const int e = base + lane;
         int t = 0;
         if (e < a.n_seg) {
-          const int rows = __ldg(a.seg_rows + e);
+          const int rows = seg_rows_s[e];
           t = rows > 0 ? (rows + R - 1) / R : 0;
         }
         int incl = t;
@@ -301,21 +322,13 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
 
   if (warp == kConsumerWarps) {
     // ============================================================ producer
+    // Per tile: its rows and the global reads of its row map are issued first, then the wait for
+    // a free stage (which hides their latency), then the stage's metadata and the row copies.
     int j = 0;
+    const int32_t* seg_first_s = seg_prefix + a.n_seg + 1;
+    const int32_t* seg_rows_s = seg_first_s + a.n_seg;
     for (int t = blockIdx.x; t < n_tiles; t += gridDim.x, ++j) {
       const int s = j % kStages;
-      if (j >= kStages) {
-        bool ok = true;
-        if (lane == 0) ok = tc::mbar_wait(bar_empty(s), (uint32_t)(((j / kStages) - 1) & 1), limit, abort_flag);
-        ok = __shfl_sync(0xffffffffu, ok, 0);
-        if (!ok) {
-          if (lane == 0) {
-            if (!*abort_flag) report_status(a.status, kErrTimeout);
-            *abort_flag = 1;
-          }
-          break;
-        }
-      }
       // rows of this tile
       int64_t r0;      // first source row (rows / segments / scatter) or first output row (gather)
       int n;           // slots in use
@@ -328,8 +341,8 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
           else hi = mid - 1;
         }
         const int c = t - seg_prefix[lo];
-        const int rows = __ldg(a.seg_rows + lo);
-        r0 = (int64_t)__ldg(a.seg_off + lo) + (int64_t)c * R;
+        const int rows = seg_rows_s[lo];
+        r0 = (int64_t)seg_first_s[lo] + (int64_t)c * R;
         n = min(R, rows - c * R);
         out0 = r0;
         if (r0 < 0 || r0 + n > a.src_rows || r0 + n > a.rows_out) {  // a segment outside the rows
@@ -345,8 +358,7 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
         n = (int)min((int64_t)R, a.rows_out - out0);
         r0 = out0;
       }
-      MetaView m(smem + p.off_meta + s * p.meta_bytes, p.mc, R);
-      // per slot: source row (or -1 for a zero row)
+      // per slot: source row (or -1 for a zero row); scatter: up to 4 destinations per lane
       int64_t my_src = -1;
       if (lane < n) {
         if (a.map == kMapGather) {
@@ -361,15 +373,39 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
           my_src = r0 + lane;
         }
       }
+      const int fo = p.fanout;
+      int32_t dpre[kMaxMeta / 32];
+#pragma unroll
+      for (int q = 0; q < kMaxMeta / 32; ++q) {
+        const int e = lane + 32 * q;
+        const int slot = e / fo, jj = e - slot * fo;
+        dpre[q] = (a.map == kMapScatter && e < R * fo && slot < n) ? __ldg(a.row_scatter + (r0 + slot) * fo + jj) : -1;
+      }
+      if (j >= kStages) {
+        bool ok = true;
+        if (lane == 0) ok = tc::mbar_wait(bar_empty(s), (uint32_t)(((j / kStages) - 1) & 1), limit, abort_flag);
+        ok = __shfl_sync(0xffffffffu, ok, 0);
+        if (!ok) {
+          if (lane == 0) {
+            if (!*abort_flag) report_status(a.status, kErrTimeout);
+            *abort_flag = 1;
+          }
+          break;
+        }
+      }
+      MetaView m(smem + p.off_meta + s * p.meta_bytes, p.mc, R);
       if (lane < R) m.valid[lane] = (lane < n && my_src >= 0) ? 1 : 0;
       // per (slot, destination): output row and its byte offsets
-      const int fo = p.fanout;
-      for (int e = lane; e < R * fo; e += 32) {
+#pragma unroll
+      for (int q = 0; q < kMaxMeta / 32; ++q) {
+        const int e = lane + 32 * q;
+        if (e >= R * fo) break;
         const int slot = e / fo, jj = e - slot * fo;
+        (void)jj;
         int64_t drow = -1;
         if (slot < n) {
           if (a.map == kMapScatter) {
-            drow = __ldg(a.row_scatter + (r0 + slot) * fo + jj);
+            drow = dpre[q];
             if (drow >= a.rows_out) {
               report_status(a.status, kErrInvalid);
               drow = -1;
