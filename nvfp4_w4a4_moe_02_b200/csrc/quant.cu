@@ -594,10 +594,19 @@ __device__ __forceinline__ void st_hint(uint16_t* p, const uint4 v, uint64_t pol
                : "memory");
 }
 
-// max |w| over elements [v_lo*8, v_hi*8) of one tensor, four 16-byte loads in flight per thread
+// |w| of two bf16 as their bit patterns (non-negative bf16 values order as their bits), a NaN as
+// 0 (a binary32 max ignores it); flags collects the halves that are infinite or NaN
+__device__ __forceinline__ uint32_t bf16x2_abs_bits(uint32_t w, uint32_t& flags) {
+  const uint32_t v = w & 0x7FFF7FFFu;
+  flags |= __vcmpgeu2(v, 0x7F807F80u);
+  return v & ~__vcmpgtu2(v, 0x7F807F80u);
+}
+
+// max |w| over elements [v_lo*8, v_hi*8) of one tensor, four 16-byte loads in flight per thread;
+// the maximum is taken on the bf16 bit patterns, two per instruction
 __device__ __forceinline__ float slice_amax(const uint16_t* wt, int64_t v_lo, int64_t v_hi, uint64_t pol,
                                             bool& nonfinite) {
-  float m = 0.0f;
+  uint32_t m = 0, flags = 0;
   const int64_t stride = blockDim.x;
   for (int64_t i0 = v_lo + threadIdx.x; i0 < v_hi; i0 += 4 * stride) {
     uint4 q[4];
@@ -606,16 +615,35 @@ __device__ __forceinline__ float slice_amax(const uint16_t* wt, int64_t v_lo, in
       q[u] = (i0 + u * stride < v_hi) ? ld_hint(wt + 8 * (i0 + u * stride), pol) : make_uint4(0, 0, 0, 0);
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const uint32_t wq[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float a = fabsf(bf16_bits_to_f32(wq[j] & 0xFFFFu)), b = fabsf(bf16_bits_to_f32(wq[j] >> 16));
-        nonfinite |= !(a <= 3.4e38f) || !(b <= 3.4e38f);
-        m = fmaxf(m, fmaxf(a, b));
-      }
+      m = __vmaxu2(m, __vmaxu2(bf16x2_abs_bits(q[u].x, flags), bf16x2_abs_bits(q[u].y, flags)));
+      m = __vmaxu2(m, __vmaxu2(bf16x2_abs_bits(q[u].z, flags), bf16x2_abs_bits(q[u].w, flags)));
     }
   }
-  return m;
+  nonfinite |= flags != 0;
+  return __uint_as_float(max(m >> 16, m & 0xFFFFu) << 16);
+}
+
+// qdq_half with (d, 1/d) looked up per scale code in a table made for the tensor's scale
+__device__ __forceinline__ void qdq_half_tab(const uint4 q, float s_g, float t6, const float2* tab, uint4& o) {
+  uint32_t m = __vmaxu2(__vmaxu2(q.x & 0x7FFF7FFFu, q.y & 0x7FFF7FFFu), __vmaxu2(q.z & 0x7FFF7FFFu, q.w & 0x7FFF7FFFu));
+  m = max(m >> 16, m & 0xFFFFu);
+  m = max(m, __shfl_xor_sync(0xffffffffu, m, 1));
+  float x[8];
+  unpack8(q, x);
+  BlockScale b;
+  b.S = s_g > 0.0f ? e4m3_encode(__fdiv_rn(__uint_as_float(m << 16), t6)) : 0u;
+  const float2 di = tab[b.S];
+  b.d = di.x;
+  b.inv = di.y;
+  float dq[8];
+  quant8(x, b, dq);
+  uint32_t r[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    __nv_bfloat162 p = __floats2bfloat162_rn(dq[2 * j], dq[2 * j + 1]);
+    r[j] = *reinterpret_cast<uint32_t*>(&p);
+  }
+  o = make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 __global__ void __launch_bounds__(256, 4) qdq_fused_kernel(const uint16_t* __restrict__ w, int64_t n_tensors,
@@ -625,6 +653,7 @@ __global__ void __launch_bounds__(256, 4) qdq_fused_kernel(const uint16_t* __res
   __shared__ float red[8];
   __shared__ float sg_sh;
   __shared__ int bad_sh;
+  __shared__ float2 tab[128];  // (d, 1/d) of the 128 E4M3 codes for the current tensor's scale
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = (int)(blockDim.x >> 5);
   const int n_groups = (int)(gridDim.x / GS);
   const int group = (int)(blockIdx.x / GS), rank = (int)(blockIdx.x % GS);
@@ -678,6 +707,12 @@ __global__ void __launch_bounds__(256, 4) qdq_fused_kernel(const uint16_t* __res
     __syncthreads();
     if (bad_sh) break;
     const float s_g = sg_sh, t6 = __fmul_rn(6.0f, s_g);
+    if (threadIdx.x < 128) {
+      const uint32_t S = threadIdx.x;
+      const float d = __fmul_rn(e4m3_decode(S), s_g);
+      tab[S] = make_float2(d, (S != 0 && S < 0x7F) ? __frcp_rn(d) : 0.0f);
+    }
+    __syncthreads();
     // the fake-quant of this CTA's chunks, one warp per 512-element chunk (lane pairs hold the two
     // halves of a 16-block), the next chunk's loads issued before this one's arithmetic
     const uint16_t* wt = w + t * elems;
@@ -696,8 +731,8 @@ __global__ void __launch_bounds__(256, 4) qdq_fused_kernel(const uint16_t* __res
         n1 = e1 < elems ? ld_hint(wt + e1, stream) : make_uint4(0, 0, 0, 0);
       }
       uint4 o0, o1;
-      qdq_half(q0, s_g, t6, o0);
-      qdq_half(q1, s_g, t6, o1);
+      qdq_half_tab(q0, s_g, t6, tab, o0);
+      qdq_half_tab(q1, s_g, t6, tab, o1);
       if (f0 < elems) st_hint(ot + f0, o0, stream);
       if (f1 < elems) st_hint(ot + f1, o1, stream);
     }
