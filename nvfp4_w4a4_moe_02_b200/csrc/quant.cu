@@ -24,16 +24,17 @@ __global__ void __launch_bounds__(256) amax_kernel(const uint16_t* __restrict__ 
   bool bad = false;
   const uint16_t* base = x + seg * seg_rows * ld;
   if (ld == cols) {
-    // contiguous segment: flat vector loop, four independent 16-byte loads in flight per thread
+    // contiguous segment: flat vector loop, eight independent 16-byte loads in flight per thread
+    // (a partial covers 16K elements: one round of loads)
     const int64_t nvec = seg_rows * cols / 8;
     const uint4* v = reinterpret_cast<const uint4*>(base);
     const int64_t stride = (int64_t)P * blockDim.x;
-    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < nvec; i0 += 4 * stride) {
-      uint4 q[4];
+    for (int64_t i0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i0 < nvec; i0 += 8 * stride) {
+      uint4 q[8];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) q[u] = (i0 + u * stride < nvec) ? __ldg(v + i0 + u * stride) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < 8; ++u) q[u] = (i0 + u * stride < nvec) ? __ldg(v + i0 + u * stride) : make_uint4(0, 0, 0, 0);
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const uint32_t w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
 #pragma unroll
         for (int j = 0; j < 4; ++j) {

@@ -580,8 +580,9 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
 
 // Launch shape: rows per tile R (stages of at most ~16 KB) and consumer warps W.  Chosen so that
 // the main pass (R * K/16 blocks) and the residual pass (R * Kp/16 blocks) leave the fewest idle
-// thread steps, then for the most bytes in flight per SM (CTAs per SM x the two stages ahead,
-// up to 96 KB), then for more CTAs per SM.  force_R / force_W (> 0) override the choice.
+// thread steps, discounted when fewer than 18 consumer warps fit on an SM, then for the most
+// bytes in flight per SM (CTAs per SM x the two stages ahead, up to 96 KB), then for more CTAs per
+// SM.  force_R / force_W (> 0) override the choice.
 bool act_plan_choose(int64_t K, int32_t Kp, int fanout, int32_t n_seg, int* R_out, int* W_out, int* smem_out,
                      int force_R, int force_W) {
   if (K <= 0 || K % 64 != 0 || fanout < 1 || fanout > act::kMaxMeta) return false;
@@ -604,7 +605,10 @@ bool act_plan_choose(int64_t K, int32_t Kp, int fanout, int32_t n_seg, int* R_ou
       const int T = 32 * warps[wi];
       const int steps = (R * KB + T - 1) / T + (QB > 0 ? (R * QB + T - 1) / T : 0);
       const double eff = (double)R * (KB + QB) / ((double)steps * T);
-      const double score = (double)(int)(eff * 100.0) * 1e9 + min(inflight, 96.0 * 1024) * 100.0 + per_sm;
+      // consumer warps resident per SM: below ~18 the dependent chains of a block are not hidden
+      const int ctas = min(per_sm, 64 / (warps[wi] + 1));
+      const double occ = min(1.0, (double)(ctas * warps[wi]) / 18.0);
+      const double score = (double)(int)(eff * occ * 100.0) * 1e9 + min(inflight, 96.0 * 1024) * 100.0 + per_sm;
       if (score > best) {
         best = score;
         bR = R;
