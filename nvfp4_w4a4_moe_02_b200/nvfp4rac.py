@@ -246,7 +246,7 @@ def set_gemm_tile_n(n: int):
 
 
 def set_gemm_pairs(on: bool):
-    """Run the GEMMs with N % 256 == 0 on CTA pairs (default) or on single SMs."""
+    """Run the GEMMs with N % 256 == 0 on CTA pairs or on single SMs (default)."""
     load().nvfp4_set_gemm_pairs(1 if on else 0)
 
 
