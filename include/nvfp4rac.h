@@ -409,7 +409,7 @@ nvfp4_status moe_route_topk(const float* logits, int64_t T, int32_t E, int32_t k
 int64_t moe_rows_capacity(int64_t T, int32_t k, int32_t E, int32_t pad);
 size_t moe_dispatch_workspace_size(int32_t E);
 /* moe_dispatch_plan -- expert-grouped layout of the (token, expert) pairs of topk_ids [T x k]  */
-/* (a token's experts must be distinct).                                                      */
+/* (a token's experts must be distinct; k <= 128).                                            */
 /*   pad            segment granularity, a multiple of 16: 128 for grouped_w4a4_rac_moe, 16 for */
 /*                  the decode slabs.                                                          */
 /*   expert_offsets int32 [E+1]: padded segment starts; offsets[E] = rows used, or -1 if they   */

@@ -85,9 +85,12 @@ nvfp4_status make_code_map(CUtensorMap* m, const void* base, uint64_t inner_byte
 
 // Output matrix [rows x cols] (bf16 or fp32, row pitch ld elements) stored by the GEMM epilogue
 // in boxes of 32 rows x 128 bytes, 128-byte swizzle.  Rows beyond `rows` are clipped.
-// narrow: boxes of 32 rows x 64 bytes without swizzle (the SwiGLU stores of the own-scale mode)
+// kOutNarrow: boxes of 32 rows x 64 bytes without swizzle (the SwiGLU stores of the own-scale
+// mode); kOutNarrow64: 32 rows x 64 bytes, 64-byte swizzle (the four-stage BN = 256 kernel)
+enum OutBox { kOutWide = 0, kOutNarrow = 1, kOutNarrow64 = 2 };
 nvfp4_status make_out_map(CUtensorMap* m, void* base, bool bf16, uint64_t cols, uint64_t rows, uint64_t ld,
-                          bool narrow = false) {
+                          OutBox mode = kOutWide) {
+  const bool narrow = mode != kOutWide;
   auto fn = encode_fn();
   if (!fn) return fail(NVFP4_ERR_CUDA, "cuTensorMapEncodeTiled entry point unavailable");
   const uint64_t esz = bf16 ? 2 : 4;
@@ -97,7 +100,10 @@ nvfp4_status make_out_map(CUtensorMap* m, void* base, bool bf16, uint64_t cols, 
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
                   box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  narrow ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                  mode == kOutNarrow    ? CU_TENSOR_MAP_SWIZZLE_NONE
+                  : mode == kOutNarrow64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                         : CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_NONE,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS)
     return fail(NVFP4_ERR_CUDA, "tensor map for the output failed (error %d, cols %llu, rows %llu)", (int)r,
@@ -724,7 +730,7 @@ static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res
                                 const nvfp4_tensor* w_sel, int64_t rows_needed, int64_t N, int64_t K, int32_t Kp,
                                 int64_t E, nvfp4_dtype out, void* y, int64_t ldy, int64_t y_cols, int64_t y_rows,
                                 int bn, CUtensorMap* maps, GemmArgs* g, int w_box_rows = 0, bool own = false,
-                                bool swiglu = false) {
+                                bool swiglu = false, bool pair_kernel = false) {
   if (w_box_rows == 0) w_box_rows = bn;
   if (K <= 0 || K % 64 != 0 || K > kMaxK) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "K must be a positive multiple of 64");
   if (Kp < 0 || Kp % 64 != 0 || Kp > K) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "Kp must be a multiple of 64 in [0, K]");
@@ -749,8 +755,9 @@ static nvfp4_status gemm_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res
   }
   memset(maps, 0, 5 * sizeof(CUtensorMap));
   if (y_rows > 0) {
-    st = make_out_map(&maps[4], y, out == NVFP4_OUT_BF16, (uint64_t)y_cols, (uint64_t)y_rows, (uint64_t)ldy,
-                      own && swiglu);
+    // the single-SM FP4 kernel at BN = 256 stages its stores in 64-byte boxes
+    const OutBox box = (own && swiglu) ? kOutNarrow : (!own && !pair_kernel && bn == 256) ? kOutNarrow64 : kOutWide;
+    st = make_out_map(&maps[4], y, out == NVFP4_OUT_BF16, (uint64_t)y_cols, (uint64_t)y_rows, (uint64_t)ldy, box);
     if (st != NVFP4_OK) return st;
   }
   st = make_code_map(&maps[0], a->codes, (uint64_t)K / 2, (uint64_t)a->rows_padded, 1, 128, 2, "A");
@@ -802,7 +809,8 @@ static nvfp4_status dense_gemm(const nvfp4_tensor* a, const nvfp4_tensor* a_res,
   CUtensorMap maps[5];
   GemmArgs g;
   nvfp4_status st =
-      gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, M, bn, maps, &g, pairs ? 128 : bn, own, false);
+      gemm_common(a, a_res, w, w_sel, M, N, K, Kp, 1, out, y, ldy, N, M, bn, maps, &g, pairs ? 128 : bn, own, false,
+                  pairs);
   if (st != NVFP4_OK) return st;
   if (M == 0) return NVFP4_OK;
   g.offsets = nullptr;
@@ -877,7 +885,7 @@ nvfp4_status grouped_common(const nvfp4_tensor* a, const nvfp4_tensor* a_res, co
   const int64_t y_cols = ep == NVFP4_EPI_SWIGLU_AMAX ? N / 2 : N;
   const int64_t y_rows = comb ? comb->T : (a ? a->rows_padded : 0);
   nvfp4_status st = gemm_common(a, a_res, w, w_sel, 0, N, K, Kp, E, out, y, ldy, y_cols, y_rows, bn, maps, &g,
-                                pairs ? 128 : bn, own, ep == NVFP4_EPI_SWIGLU_AMAX);
+                                pairs ? 128 : bn, own, ep == NVFP4_EPI_SWIGLU_AMAX, pairs && !comb);
   if (st != NVFP4_OK) return st;
   g.offsets = offsets;
   g.expert_rows = seg_rows;
@@ -1119,7 +1127,8 @@ nvfp4_status moe_dispatch_plan(const int32_t* topk_ids, int64_t T, int32_t k, in
                                void* workspace,
                                size_t workspace_bytes, int32_t* dev_status, void* stream) {
   g_last_error.clear();
-  if (T < 0 || k <= 0 || E <= 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T >= 0, k > 0 and E > 0 required");
+  if (T < 0 || k <= 0 || k > 128 || E <= 0)
+    return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "T >= 0, 0 < k <= 128 and E > 0 required");
   if (pad <= 0 || pad % 16 != 0) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "pad = %d must be a positive multiple of 16", pad);
   if (rows_capacity < 0 || rows_capacity > INT32_MAX) return fail(NVFP4_ERR_UNSUPPORTED_SHAPE, "rows_capacity out of range");
   if (!expert_offsets || (T > 0 && (!topk_ids || !row_scatter))) return fail(NVFP4_ERR_INVALID_ARG, "NULL buffer");

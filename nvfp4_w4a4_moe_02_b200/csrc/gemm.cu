@@ -65,15 +65,19 @@ __device__ __forceinline__ int segment_weight(const GemmArgs& args, int seg) {
 template <int BN, bool OWN = false, bool SFST = false>
 struct Cfg {
   static constexpr int ACC_W = OWN ? 2 * BN : BN;  // accumulator columns per tile
-  static constexpr int STAGES = (BN == 256) ? 3 : 5;
+  // NARROW (scale-warp mode at BN = 256): 32-row x 64-byte staging boxes (64-byte swizzle), so
+  // that the shared memory holds a fourth operand stage
+  static constexpr bool NARROW = SFST && BN == 256;
+  static constexpr int STAGES = (BN == 256) ? (NARROW ? 4 : 3) : 5;
   // scale atoms: in scale-warp mode a ring of their own, SFR k-tiles deep (filled by a second
   // producer thread ahead of the operand ring, so the scale warps finish before the operands
   // land); otherwise part of each operand stage
-  static constexpr int SFR = SFST ? 6 : STAGES;
+  static constexpr int SFR = SFST ? (NARROW ? 3 : 6) : STAGES;
   // epilogue staging: per epilogue warp, STG boxes of 32 rows x 128 bytes for TMA stores (one in
-  // scale-warp mode, whose scale ring takes the shared memory of the second)
+  // scale-warp mode, whose scale ring takes the shared memory of the second; one of 32 rows x 64
+  // bytes in the NARROW mode)
   static constexpr int STG = SFST ? 1 : (BN == 256) ? 2 : 1;
-  static constexpr int BOX_BYTES = 32 * 128;
+  static constexpr int BOX_BYTES = NARROW ? 32 * 64 : 32 * 128;
   static constexpr int A_BYTES = BM * KT_BYTES;
   static constexpr int B_BYTES = BN * KT_BYTES;
   static constexpr int SFA_BYTES = 4 * 512;
@@ -104,6 +108,7 @@ struct Cfg {
   static constexpr int OFF_SFB = OFF_SFA + SFR * SFA_BYTES;
   static constexpr int OFF_STG = OFF_SFB + SFR * SFB_BYTES;  // 1024-aligned
   static constexpr int OFF_BAR = OFF_STG + 8 * STG * BOX_BYTES;
+  static_assert(OFF_STG % 1024 == 0, "staging boxes start on a swizzle-pattern boundary");
   // full[S], empty[S], accf[2], acce[2], ovf[2], drain, sf_full[2], sf_landed[SFR], sf_free[SFR]
   static constexpr int NUM_BARS = 2 * STAGES + 9 + 2 * SFR;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
@@ -579,6 +584,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const int32_t y0 = (int32_t)(mb * BM + quad * 32);
       const bool box_live = (int64_t)y0 < rows_e;
       auto put_box = [&](int slot, const uint32_t (&w)[32], int32_t x) {
+        if constexpr (C::NARROW) {
+          // the 128-byte row in two boxes of 32 rows x 64 bytes (64-byte swizzle: 16-byte chunk c
+          // of row r at chunk c ^ ((r / 2) % 4)); x advances by 64 bytes of elements
+          const int32_t dx = args.out_bf16 ? 32 : 16;
+#pragma unroll
+          for (int hb = 0; hb < 2; ++hb) {
+            if (lane == 0) bulk_wait_group_read<0>();
+            __syncwarp();
+            const uint32_t rowp = stg + (uint32_t)(lane * 64);
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+              st_shared_v4(rowp + (uint32_t)((c ^ ((lane >> 1) & 3)) * 16), w[16 * hb + 4 * c],
+                           w[16 * hb + 4 * c + 1], w[16 * hb + 4 * c + 2], w[16 * hb + 4 * c + 3]);
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tm_y, stg, x + hb * dx, y0);
+              bulk_commit_group();
+            }
+          }
+          return;
+        }
         // at most STG - 1 earlier stores of this warp may still be reading the staging boxes
         if (lane == 0) bulk_wait_group_read<C::STG - 1>();
         __syncwarp();

@@ -15,13 +15,14 @@ namespace nvfp4 {
 // ordered by (value descending, expert ascending)
 // ----------------------------------------------------------------------------------------
 
+// V = logits per lane (E <= 32 V): the scan loops are compiled for the expert count's bracket.
+template <int V>
 __global__ void __launch_bounds__(256) route_topk_kernel(const float* __restrict__ logits, int64_t T, int E, int k,
                                                          int32_t* __restrict__ ids, float* __restrict__ w,
                                                          int32_t* status) {
   const int lane = threadIdx.x & 31;
   const int64_t t = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
-  constexpr int V = kMaxRouteExperts / 32;
   float v[V];
   bool bad = false;
 #pragma unroll
@@ -94,6 +95,29 @@ __global__ void count_kernel(const int32_t* __restrict__ ids, int64_t n, int E, 
   }
 }
 
+// the same counts through a per-CTA histogram in shared memory (E <= kCountSmemExperts): one
+// global atomic per CTA and expert instead of one per pair
+constexpr int kCountSmemExperts = 8192;
+__global__ void __launch_bounds__(1024) count_smem_kernel(const int32_t* __restrict__ ids, int64_t n, int E,
+                                                          int32_t* __restrict__ counts, int32_t* status) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  bool bad = false;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+    const int e = __ldg(ids + i);
+    if (e < 0 || e >= E) {
+      bad = true;
+      continue;
+    }
+    atomicAdd(hist + e, 1);
+  }
+  if (bad) report_status(status, kErrInvalid);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    if (hist[e] != 0) atomicAdd(counts + e, hist[e]);
+}
+
 // one CTA: padded segment starts (exclusive scan), then the decode slot tables
 __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict__ counts, int E, int pad,
                                                        int64_t rows_capacity, int32_t* __restrict__ offsets,
@@ -141,32 +165,83 @@ __global__ void __launch_bounds__(1024) offsets_kernel(const int32_t* __restrict
   }
 }
 
-// one CTA per expert: the rank of each of its tokens (ascending) -> row of the pair
-__global__ void __launch_bounds__(256) rank_kernel(const int32_t* __restrict__ ids, int64_t T, int k,
-                                                   const int32_t* __restrict__ offsets, int E,
-                                                   int32_t* __restrict__ row_scatter) {
-  __shared__ int warp_sum[8];
+// one CTA per expert: the rank of each of its tokens (ascending) -> row of the pair.  Thread i
+// takes kRankTpt consecutive tokens of a chunk of kRankThreads * kRankTpt; the CTA's exclusive
+// scan of the per-thread hit counts gives each hit its rank within the chunk.
+constexpr int kRankThreads = 1024;
+constexpr int kRankTpt = 4;
+__global__ void __launch_bounds__(kRankThreads) rank_kernel(const int32_t* __restrict__ ids, int64_t T, int k,
+                                                            const int32_t* __restrict__ offsets, int E,
+                                                            int32_t* __restrict__ row_scatter) {
+  __shared__ int warp_sum[kRankThreads / 32];
+  __shared__ int chunk_total;
   const int e = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (offsets[E] < 0) return;  // unusable plan (reported): every pair stays unrouted (-1)
   int64_t run = offsets[e];
-  for (int64_t base = 0; base < T; base += blockDim.x) {
-    const int64_t t = base + threadIdx.x;
-    int hit = -1;
-    if (t < T)
-      for (int j = 0; j < k; ++j)
-        if (__ldg(ids + t * k + j) == e) hit = j;
-    const unsigned m = __ballot_sync(0xffffffffu, hit >= 0);
-    if (lane == 0) warp_sum[warp] = __popc(m);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int i = 0; i < (int)(blockDim.x >> 5); ++i) {
-      before += i < warp ? warp_sum[i] : 0;
-      total += warp_sum[i];
+  const bool vec = (reinterpret_cast<uintptr_t>(ids) & 15u) == 0;
+  static_assert(kRankTpt == 4, "four tokens per thread: 16-byte groups of ids and one byte of `hits` each");
+  for (int64_t base = 0; base < T; base += (int64_t)kRankThreads * kRankTpt) {
+    const int64_t t0 = base + (int64_t)threadIdx.x * kRankTpt;
+    // byte i of `hits`: 0x80 | slot j for token t0 + i when ids[t0 + i][j] == e (a token's experts
+    // are distinct), else 0.  The thread's kRankTpt * k ids are contiguous: with 16-byte aligned
+    // ids they come in k 16-byte loads, eight in flight at a time.
+    uint32_t hits = 0;
+    if (vec && t0 + kRankTpt <= T) {
+      const int4* src = reinterpret_cast<const int4*>(ids + t0 * k);
+      for (int v0 = 0; v0 < k; v0 += 8) {
+        int4 q[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (v0 + u < k) q[u] = __ldg(src + v0 + u);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          if (v0 + u >= k) break;
+          const int w[4] = {q[u].x, q[u].y, q[u].z, q[u].w};
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            if (w[c] == e) {
+              const int idx = 4 * (v0 + u) + c, tok = idx / k;
+              hits |= (uint32_t)(0x80 | (idx - tok * k)) << (8 * tok);
+            }
+        }
+      }
+    } else {
+      for (int i = 0; i < kRankTpt; ++i)
+        if (t0 + i < T)
+          for (int j = 0; j < k; ++j)
+            if (__ldg(ids + (t0 + i) * k + j) == e) hits |= (uint32_t)(0x80 | j) << (8 * i);
     }
-    if (hit >= 0) row_scatter[t * k + hit] = (int32_t)(run + before + __popc(m & ((1u << lane) - 1u)));
-    run += total;
+    const int mine = __popc(hits & 0x80808080u);
+    // exclusive scan of `mine` over the CTA: in the warp by shuffles, then over the warps
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int up = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += up;
+    }
+    if (lane == 31) warp_sum[warp] = incl;
     __syncthreads();
+    if (warp == 0) {
+      const int ws = warp_sum[lane];
+      int wi = ws;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int up = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += up;
+      }
+      warp_sum[lane] = wi - ws;  // exclusive prefix of the warps
+      if (lane == 31) chunk_total = wi;
+    }
+    __syncthreads();
+    int64_t r = run + warp_sum[warp] + (incl - mine);
+#pragma unroll
+    for (int i = 0; i < kRankTpt; ++i) {
+      const uint32_t h = (hits >> (8 * i)) & 0xFFu;
+      if (h & 0x80u) row_scatter[(t0 + i) * k + (int)(h & 0x7Fu)] = (int32_t)(r++);
+    }
+    run += chunk_total;
+    __syncthreads();  // warp_sum and chunk_total are rewritten by the next chunk
   }
 }
 
@@ -306,8 +381,14 @@ cudaError_t launch_row_groups(const int32_t* off, int E, int64_t rows, int32_t* 
 
 cudaError_t launch_route_topk(const float* logits, int64_t T, int E, int k, int32_t* ids, float* w, int32_t* status,
                               cudaStream_t st) {
-  const int64_t blocks = (T + 7) / 8;
-  route_topk_kernel<<<(unsigned)blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
+  const unsigned blocks = (unsigned)((T + 7) / 8);
+  const int v = (E + 31) / 32;
+  if (v <= 1) route_topk_kernel<1><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
+  else if (v <= 2) route_topk_kernel<2><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
+  else if (v <= 4) route_topk_kernel<4><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
+  else if (v <= 8) route_topk_kernel<8><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
+  else if (v <= 16) route_topk_kernel<16><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
+  else route_topk_kernel<kMaxRouteExperts / 32><<<blocks, 256, 0, st>>>(logits, T, E, k, ids, w, status);
   return cudaGetLastError();
 }
 
@@ -320,13 +401,26 @@ cudaError_t launch_dispatch_plan(const int32_t* ids, int64_t T, int k, int E, in
   e = cudaMemsetAsync(row_scatter, 0xFF, sizeof(int32_t) * (size_t)(T * k), st);  // -1: unrouted
   if (e != cudaSuccess) return e;
   const int64_t n = T * k;
-  int64_t blocks = (n + 255) / 256;
-  if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-  if (blocks < 1) blocks = 1;
-  count_kernel<<<(unsigned)blocks, 256, 0, st>>>(ids, n, E, counts, status);
+  if (E <= kCountSmemExperts) {
+    // about 4096 pairs per CTA
+    int64_t blocks = (n + 4095) / 4096;
+    if (blocks > (int64_t)num_sms) blocks = num_sms;
+    if (blocks < 1) blocks = 1;
+    const size_t smem = sizeof(int) * (size_t)E;
+    if (smem > 48 * 1024) {
+      e = cudaFuncSetAttribute(count_smem_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    count_smem_kernel<<<(unsigned)blocks, 1024, smem, st>>>(ids, n, E, counts, status);
+  } else {
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    if (blocks < 1) blocks = 1;
+    count_kernel<<<(unsigned)blocks, 256, 0, st>>>(ids, n, E, counts, status);
+  }
   offsets_kernel<<<1, 1024, 0, st>>>(counts, E, pad, rows_capacity, offsets, expert_rows, slot_expert, slot_count,
                                      n_slots, status);
-  rank_kernel<<<(unsigned)E, 256, 0, st>>>(ids, T, k, offsets, E, row_scatter);
+  rank_kernel<<<(unsigned)E, kRankThreads, 0, st>>>(ids, T, k, offsets, E, row_scatter);
   return cudaGetLastError();
 }
 

@@ -88,6 +88,10 @@ def test_host_side_rejections(lib):
     assert st == 2
     # null status pointer is rejected by the self-test entry
     assert lib.nvfp4_selftest_wait_timeout(1000, None, None) == 1
+    # dispatch plan: k above 128 (the rank kernel keeps a pair's slot in seven bits)
+    ws = lib.moe_dispatch_workspace_size(8)
+    st = lib.moe_dispatch_plan(16, 4, 129, 8, 128, 4096, 16, 16, None, None, None, 0, 16, ws, None, None)
+    assert st == 2 and b"128" in lib.nvfp4_last_error_string()
 
 
 def test_noalloc_host_side_rejections(lib):

@@ -30,7 +30,8 @@ def router_logits(T, E, seed=0):
     return syn.normal_f64(seed, syn.STREAM_ROUTER, T * E).reshape(T, E).astype(np.float32)
 
 
-@pytest.mark.parametrize("T,E,k", [(4096, 128, 8), (64, 256, 8), (37, 1024, 32), (5, 3, 1)])
+@pytest.mark.parametrize("T,E,k", [(4096, 128, 8), (64, 256, 8), (37, 1024, 32), (5, 3, 1), (300, 40, 6),
+                                   (99, 500, 8)])
 def test_route_topk_matches_oracle(dev, orc, T, E, k):
     logits = router_logits(T, E)
     st = R.new_status(dev)
@@ -59,9 +60,10 @@ def test_route_rejects_non_finite_logits(dev):
     assert int(st.item()) == 4
 
 
-@pytest.mark.parametrize("pad", [128, 16])
-def test_dispatch_plan_matches_oracle(dev, orc, pad):
-    T, E, k = 4096, 128, 8
+@pytest.mark.parametrize("T,E,k,pad", [(4096, 128, 8, 128), (4096, 128, 8, 16), (9000, 64, 4, 128), (300, 12, 3, 16)])
+def test_dispatch_plan_matches_oracle(dev, orc, T, E, k, pad):
+    """Offsets, pair rows and slot tables bit for bit; 9000 tokens span more than one chunk of
+    the rank kernel (4096 tokens)."""
     ids_ref, _ = orc.route_topk(router_logits(T, E, seed=3), k)
     # make one expert empty and one very busy
     ids_ref = np.where(ids_ref == 5, 6, ids_ref)
