@@ -31,7 +31,7 @@
 namespace nvfp4 {
 namespace act {
 
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kMaxMeta = 128;              // R * fanout entries of one stage
 constexpr int kPitch = 17;                 // words per 16-block in the residual buffer
 
