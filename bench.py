@@ -715,9 +715,9 @@ def spec_moe(dev, args, peaks):
         e2e_step=e2e_step, e2e_extra_h2d={"logits": e2e_step.logits_np},
         segments={"quant_x": ("q0", "g0"), "gate_up": ("g0", "q1"), "quant_h": ("q1", "d0"), "down": ("d0", "end")},
         dominant=("gate_up", gu_f, gu_bytes, "grouped gate_up W4A4+RAC GEMM (SwiGLU epilogue)"),
-        # DRAM bytes read + written by one gate_up launch at this workload: none captured for the
-        # kernel as it is
-        traffic=None,
+        # DRAM bytes read + written by one gate_up launch at this workload (one-pass ncu capture of
+        # dram__bytes_read.sum + dram__bytes_write.sum of the kernel as it is: 410.4 + 46.6 MB)
+        traffic=456994304.0,
         quant={"x": ("quant_x", int(wl.x.nbytes) + P * 0.5625 * (wl.H + wl.Kp_gu)),  # X read once, 8 copies out
                "h": ("quant_h", quant_bytes(P, wl.I, wl.Kp_dn))},
         config={"workload": wl.name + f"_r{wl.r}", "tokens": int(wl.x.shape[0]), "pairs": P, "experts": wl.E,
