@@ -445,9 +445,13 @@ class MoEBlockStep:
         self.y = torch.empty(T, wl.H, dtype=torch.bfloat16, device=dev)
         torch.cuda.synchronize()
 
-    def run(self, x=None, logits=None, events=None):
+    # run() takes an output buffer: the end-to-end loop pipelines steps over two of them
+    takes_out = True
+
+    def run(self, x=None, logits=None, events=None, out=None):
         R = self.R
         ev = events or {}
+        y_out = self.y if out is None else out
         if "r0" in ev:
             ev["r0"].record()
         R.moe_route_topk(self.logits if logits is None else logits, self.k, ids=self.ids, w=self.w,
@@ -480,7 +484,7 @@ class MoEBlockStep:
         if self.fused_combine:
             # down projection with the weighted combine in its epilogue, then the bf16 rows
             R.grouped_w4a4_rac_moe_combine(self.hq, self.hqr, self.off, self.pdn, self.pdns, self.row_pair, self.w,
-                                           out=self.y, out32=self.y32, status=self.status,
+                                           out=y_out, out32=self.y32, status=self.status,
                                            expert_rows=self.expert_rows)
             if "c0" in ev:
                 ev["c0"].record()
@@ -493,10 +497,10 @@ class MoEBlockStep:
                                        status=self.status, expert_rows=self.expert_rows)
             if "c0" in ev:
                 ev["c0"].record()
-            R.moe_combine(self.ye, self.rows, self.w, out=self.y, status=self.status)
+            R.moe_combine(self.ye, self.rows, self.w, out=y_out, status=self.status)
         if "end" in ev:
             ev["end"].record()
-        return self.y
+        return y_out
 
 
 class QdqStep:
@@ -1083,6 +1087,8 @@ def main():
                     help="qdq workload: number of 1024 x 2048 tensors (1024 = 2^31 elements; fewer for profiler captures)")
     ap.add_argument("--fused-combine", action="store_true",
                     help="layer workloads (prefill): the weighted combine in the down GEMM's epilogue")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time the step's API calls directly instead of replaying them from a CUDA graph")
     ap.add_argument("--experts", type=int, default=None,
                     help="MoE workloads: expert count override (smaller device footprint for profiler captures)")
     args = ap.parse_args()
@@ -1131,6 +1137,31 @@ def main():
     clocks.wait_first_sample()
     R.check_status(step.status)
 
+    # the step's launches captured once into a CUDA graph (same buffers every step), so the
+    # host's per-call work (argument checks, tensor-map encoding) is off the device's timeline
+    graph = None
+    if not args.no_graph:
+        try:
+            side = torch.cuda.Stream()
+            side.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(side):
+                step.run()
+            torch.cuda.current_stream().wait_stream(side)
+            torch.cuda.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step.run()
+            torch.cuda.synchronize()
+            for _ in range(args.warmup):
+                flush.zero_()
+                graph.replay()
+            torch.cuda.synchronize()
+            R.check_status(step.status)
+        except Exception as ex:  # capture not possible for this step: plain launches
+            print(f"# CUDA graph capture failed ({str(ex)[:120]}); timing plain launches", file=sys.stderr)
+            graph = None
+            torch.cuda.synchronize()
+
     # timed region: K steps with events at the step boundaries only (an event between two
     # kernels holds the second until the first has drained: about 8 us per MoE step); L2 flushed
     # between steps (outside the per-step events)
@@ -1140,7 +1171,12 @@ def main():
     t_wall0 = time.time()
     for i in range(args.steps):
         flush.zero_()
-        step.run(events=evs_step[i])
+        if graph is not None:
+            evs_step[i][first].record()
+            graph.replay()
+            evs_step[i][last].record()
+        else:
+            step.run(events=evs_step[i])
     barrier()
     t_wall1 = time.time()
     clk = clocks.stop(t_wall0, t_wall1)
@@ -1195,32 +1231,77 @@ def main():
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     n_e2e = max(3, args.steps // 4)
     e2e_ms = 0.0
-    for _ in range(n_e2e):
-        flush.zero_()
-        e0.record()
-        x_dev.view(torch.int16).copy_(x_host, non_blocking=True)
-        for k, v in extra_host.items():
-            extra_dev[k].copy_(v, non_blocking=True)
-        y = e2e_step.run(x=x_dev, **extra_dev)
-        y_host.copy_(y, non_blocking=True)
-        e1.record()
+    pipelined = getattr(e2e_step, "takes_out", False)
+    if pipelined:
+        # steps pipelined over two buffer sets: step i's inputs go up on a copy stream while step
+        # i - 1 computes and step i - 2's output comes down on a third stream.  Every step still
+        # copies its inputs in and its [T, H] output out; the packed weights (larger than L2)
+        # stream through L2 every step, so no flush runs between these steps.
+        cur = torch.cuda.current_stream()
+        s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+        xs = [x_dev, torch.empty_like(x_dev)]
+        exs = [extra_dev, {k: torch.empty_like(v) for k, v in extra_dev.items()}]
+        ys = [torch.empty_like(e2e_step.y), torch.empty_like(e2e_step.y)]
+        yh = [y_host, torch.empty_like(y_host).pin_memory()]
+        done_in = [torch.cuda.Event() for _ in range(n_e2e)]
+        done_run = [torch.cuda.Event() for _ in range(n_e2e)]
+        done_out = [torch.cuda.Event() for _ in range(n_e2e)]
         torch.cuda.synchronize()
-        e2e_ms += e0.elapsed_time(e1)
-    e2e_ms = max_over_ranks(e2e_ms / n_e2e, ws, dev)
+        e0.record(s_in)
+        for i in range(n_e2e):
+            b = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(done_run[i - 2])  # buffer set b read by step i - 2
+                xs[b].view(torch.int16).copy_(x_host, non_blocking=True)
+                for k, v in extra_host.items():
+                    exs[b][k].copy_(v, non_blocking=True)
+                done_in[i].record(s_in)
+            cur.wait_event(done_in[i])
+            if i >= 2:
+                cur.wait_event(done_out[i - 2])  # output buffer b read back by step i - 2
+            e2e_step.run(x=xs[b], out=ys[b], **exs[b])
+            done_run[i].record(cur)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done_run[i])
+                yh[b].copy_(ys[b], non_blocking=True)
+                done_out[i].record(s_out)
+        e1.record(s_out)
+        torch.cuda.synchronize()
+        e2e_ms = e0.elapsed_time(e1) / n_e2e
+    else:
+        for _ in range(n_e2e):
+            flush.zero_()
+            e0.record()
+            x_dev.view(torch.int16).copy_(x_host, non_blocking=True)
+            for k, v in extra_host.items():
+                extra_dev[k].copy_(v, non_blocking=True)
+            y = e2e_step.run(x=x_dev, **extra_dev)
+            y_host.copy_(y, non_blocking=True)
+            e1.record()
+            torch.cuda.synchronize()
+            e2e_ms += e0.elapsed_time(e1)
+        e2e_ms /= n_e2e
+    e2e_ms = max_over_ranks(e2e_ms, ws, dev)
     R.check_status(e2e_step.status)
     e2e = {"value": whole_job_rate(work, ws, e2e_ms, scale), "unit": unit,
            "h2d_bytes_per_step": int(x_np.nbytes) + sum(int(v.nbytes) for v in e2e_h2d.values()),
            "d2h_bytes_per_step": int(y_host.numel() * 2),
            "call": "whole MoE layer (router, plan, quantise, GEMMs, combine into [T, H])" if "e2e_step" in sp
-           else "the timed step"}
+           else "the timed step",
+           "schedule": ("steps pipelined on three streams (copy in / compute / copy out, two buffer sets); "
+                        "no L2 flush: the packed weights, larger than L2, stream every step") if pipelined
+           else "one step at a time, L2 flushed before each"}
 
     cpu = sp["cpu"]() if (rank == 0 and ws == 1 and not args.no_cpu_baseline) else None
 
     if rank == 0:
         config = dict(sp["config"])
         config["l2"] = "flushed between timed steps (256 MiB write outside the per-step events)"
-        config["timing"] = ("ms_per_step: events at step boundaries only; kernel_ms and the roofline's kernel "
-                            "duration: the same number of steps right after, with events between the kernels")
+        config["timing"] = ("ms_per_step: events at step boundaries only" +
+                            (", the step's launches replayed from one CUDA graph" if graph is not None else "") +
+                            "; kernel_ms and the roofline's kernel duration: the same number of steps right after, "
+                            "launched through the API with events between the kernels")
         config["parallelism"] = f"replicas x{ws}"
         if args.gemm_pairs is not None:
             config["gemm_pairs"] = bool(args.gemm_pairs)
@@ -1244,6 +1325,7 @@ def main():
             "clocks": clk,
         }
         print(json.dumps(line), flush=True)
+    del graph  # released before the process group goes
     if ws > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
