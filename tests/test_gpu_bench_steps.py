@@ -47,6 +47,46 @@ def test_prefill_layer_step_with_and_without_fused_combine(dev):
     assert np.isfinite(a).all() and np.abs(a).max() > 0
 
 
+def test_step_replayed_from_a_cuda_graph_gives_the_same_outputs(dev):
+    """The bench times the step's C-ABI calls replayed from one CUDA graph: the replay computes the
+    same rows as the calls themselves, bit for bit (prefill block and whole layer)."""
+    wl = syn.moe_block(0, 0.5, T=256, H=512, E=8, topk=2, I=256, T_cal=128)
+    step = bench.MoEStep(wl, syn.moe_down_calibration_batch(wl), dev)
+    layer = bench.MoEBlockStep(wl, (step.pgu, step.pgus, step.pdn, step.pdns), step.sel_gu, step.sel_dn, False, dev)
+    pair_rows = torch.from_numpy(step.pair_rows).to(dev)
+    for s in (step, layer):
+        s.run()
+        torch.cuda.synchronize()
+        # rows that hold pairs (padding rows of the expert-sorted buffers are never written)
+        hr = pair_rows if s is step else s.rows.reshape(-1).long()
+        yr = pair_rows if s is step else torch.arange(s.y.shape[0], device=dev)
+        ref = s.y[yr].clone()
+        href = s.h[hr].clone()
+        s.y.zero_()
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(side):
+            s.run()
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            s.run()
+        s.y.zero_()
+        s.h.zero_()
+        g.replay()
+        g.replay()
+        torch.cuda.synchronize()
+        R.check_status(s.status)
+        assert torch.equal(s.y[yr], ref) and torch.equal(s.h[hr], href)
+        del g
+    # the layer's output buffer argument (the pipelined end-to-end loop): same rows elsewhere
+    out = torch.empty_like(layer.y)
+    layer.run(out=out)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+
+
 def test_decode_layer_step_runs(dev):
     wl = syn.moe_block(0, 0.5, T=16, H=512, E=16, topk=4, I=256, T_cal=128, materialize_weights=False)
     inner = bench.DecodeStep(wl, dev)

@@ -60,7 +60,8 @@ def test_route_rejects_non_finite_logits(dev):
     assert int(st.item()) == 4
 
 
-@pytest.mark.parametrize("T,E,k,pad", [(4096, 128, 8, 128), (4096, 128, 8, 16), (9000, 64, 4, 128), (300, 12, 3, 16)])
+@pytest.mark.parametrize("T,E,k,pad", [(4096, 128, 8, 128), (4096, 128, 8, 16), (9000, 64, 4, 128), (300, 12, 3, 16),
+                                       (50, 160, 128, 128)])
 def test_dispatch_plan_matches_oracle(dev, orc, T, E, k, pad):
     """Offsets, pair rows and slot tables bit for bit; 9000 tokens span more than one chunk of
     the rank kernel (4096 tokens)."""
