@@ -1,6 +1,6 @@
 """Static checks of bench.py that need no GPU: every attribute a step class reads through `self`
 is assigned (or defined) in that class, so a workload cannot fail on a missing attribute only
-once it reaches the GPU machine."""
+once it runs on a GPU."""
 import ast
 import os
 
