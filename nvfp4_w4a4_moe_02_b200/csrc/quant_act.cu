@@ -168,6 +168,18 @@ __device__ __forceinline__ void resid8(const float x[8], uint32_t c, float d, fl
   }
 }
 
+// The scale bytes of four neighbouring blocks of one row (lanes 4g .. 4g+3, blocks 4m .. 4m+3)
+// form one 32-bit word of each destination's scale row (byte i = block 4m + i); every lane of the
+// group gets the whole word.  The callers keep the four lanes of a group on the same row and
+// trip count.
+__device__ __forceinline__ uint32_t scale_word4(uint32_t S, int lane) {
+  const uint32_t gm = 0xFu << (lane & ~3);
+  uint32_t w = S << (8u * (uint32_t)(lane & 3));
+  w |= __shfl_xor_sync(gm, w, 1);
+  w |= __shfl_xor_sync(gm, w, 2);
+  return w;
+}
+
 // W consumer warps (4..8, chosen per shape so that both passes divide evenly) + 1 producer warp
 // The block scale with (d, 1/d) looked up per E4M3 code: for a fixed tensor scale s_g the 127
 // codes give 127 (d, 1/d) pairs, computed once per CTA with the same operations as block_scale.
@@ -506,13 +518,25 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
       bf16x8_to_f32(u0, x);
       bf16x8_to_f32(u1, x + 8);
       const uint2 c = make_uint2(codes8(x, bs), codes8(x + 8, bs));
-      const int32_t blk = sf_blk_off(kb);
-      for (int jj = 0; jj < (amax_only ? 0 : fo); ++jj) {
-        const int e = slot * fo + jj;
-        const int64_t co = m.code[e];
-        if (co < 0) continue;
-        *reinterpret_cast<uint2*>(a.codes + co + kb * 8) = c;
-        a.sf[m.sfrow[e] + blk] = (uint8_t)bs.S;
+      if (fo == 1) {
+        const int64_t co = m.code[slot];
+        if (!amax_only && co >= 0) {
+          *reinterpret_cast<uint2*>(a.codes + co + kb * 8) = c;
+          a.sf[m.sfrow[slot] + sf_blk_off(kb)] = (uint8_t)bs.S;
+        }
+      } else if (!amax_only) {
+        // several destinations: lane p of a four-lane group stores the group's scale word of
+        // destinations p, p + 4, ... (one 32-bit store instead of four byte stores per row)
+        const uint32_t sw = scale_word4(bs.S, lane);
+        for (int jj = 0; jj < fo; ++jj) {
+          const int64_t co = m.code[slot * fo + jj];
+          if (co >= 0) *reinterpret_cast<uint2*>(a.codes + co + kb * 8) = c;
+        }
+        const int32_t wblk = sf_blk_off(kb & ~3);
+        for (int jj = lane & 3; jj < fo; jj += 4) {
+          const int e = slot * fo + jj;
+          if (m.code[e] >= 0) *reinterpret_cast<uint32_t*>(a.sf + m.sfrow[e] + wblk) = sw;
+        }
       }
       if (RES) {
         float r[16];
@@ -555,13 +579,23 @@ __global__ void __launch_bounds__(32 * W + 32) act_quant_kernel(const ActArgs a)
         }
         const BlockScale bs = block_scale_tab(b, s_r, t6_r, dtab_r);
         const uint2 c = make_uint2(codes8(v, bs), codes8(v + 8, bs));
-        const int32_t blk = sf_blk_off(q);
-        for (int jj = 0; jj < fo; ++jj) {
-          const int e = rs * fo + jj;
-          const int64_t co = m.rcode[e];
-          if (co < 0) continue;
-          *reinterpret_cast<uint2*>(a.rcodes + co + q * 8) = c;
-          a.rsf[m.rsfrow[e] + blk] = (uint8_t)bs.S;
+        if (fo == 1) {
+          const int64_t co = m.rcode[rs];
+          if (co >= 0) {
+            *reinterpret_cast<uint2*>(a.rcodes + co + q * 8) = c;
+            a.rsf[m.rsfrow[rs] + sf_blk_off(q)] = (uint8_t)bs.S;
+          }
+        } else {
+          const uint32_t sw = scale_word4(bs.S, lane);
+          for (int jj = 0; jj < fo; ++jj) {
+            const int64_t co = m.rcode[rs * fo + jj];
+            if (co >= 0) *reinterpret_cast<uint2*>(a.rcodes + co + q * 8) = c;
+          }
+          const int32_t wblk = sf_blk_off(q & ~3);
+          for (int jj = lane & 3; jj < fo; jj += 4) {
+            const int e = rs * fo + jj;
+            if (m.rcode[e] >= 0) *reinterpret_cast<uint32_t*>(a.rsf + m.rsfrow[e] + wblk) = sw;
+          }
         }
       }
     }
