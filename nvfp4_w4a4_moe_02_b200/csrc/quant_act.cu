@@ -10,7 +10,8 @@
 //     stage's row metadata (destination rows, byte offsets of codes and scales);
 //   * 4 to 8 consumer warps quantise the stage: thread = one 16-element block (its block max,
 //     its E4M3 scale by one IEEE division and one reciprocal, eight E2M1 conversions), stores
-//     of 8 code bytes and 1 scale byte per destination row;
+//     of 8 code bytes per destination row and its scale byte (one destination) or, with several
+//     destinations, the scale word of four neighbouring blocks from one lane of the four;
 //   * in the same pass each thread writes the block's residual r = x - e*d (binary32) into a
 //     shared buffer whose 16-float blocks sit 17 words apart (the consumer warps' stores and
 //     the residual pass's gathers then spread over the banks), and after a barrier the
@@ -170,8 +171,9 @@ __device__ __forceinline__ void resid8(const float x[8], uint32_t c, float d, fl
 
 // The scale bytes of four neighbouring blocks of one row (lanes 4g .. 4g+3, blocks 4m .. 4m+3)
 // form one 32-bit word of each destination's scale row (byte i = block 4m + i); every lane of the
-// group gets the whole word.  The callers keep the four lanes of a group on the same row and
-// trip count.
+// group gets the whole word.  The four lanes of a group are on the same row and trip count in
+// both passes: K and K' are multiples of 64 (blocks per row a multiple of 4) and the consumer count
+// a multiple of 32, so lane l's block index within the tile is l mod 4 plus a multiple of 4.
 __device__ __forceinline__ uint32_t scale_word4(uint32_t S, int lane) {
   const uint32_t gm = 0xFu << (lane & ~3);
   uint32_t w = S << (8u * (uint32_t)(lane & 3));
